@@ -1,0 +1,414 @@
+"""Benchmark of libqmm's hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode_m1|...]
+
+One JSON line on rank 0.  The headline workload is the decode GEMV: x bf16
+[1, 4096] against W [14336, 4096] quantized affine int4, group size 64,
+transpose=true; the metric is weight+scale+bias bytes per second (GB/s).  The
+same line carries the prefill GEMM (x [2048, 4096], int4) in TFLOP/s, both as
+fractions of their rooflines, the end-to-end number through host buffers,
+clocks sampled during the timed region, and the CPU oracle's throughput.
+
+A step is one call of the hot path on one batch.  Weight copies rotate so the
+bytes a step reads are never L2-resident (8 copies x 33 MB > 126 MB L2).  At
+N > 1 (torchrun) every rank runs an independent replica (no data-path
+collective), timing is the max over ranks, and the value is the sum of the
+work all ranks did.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+from pathlib import Path
+
+import torch
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+from quantized_matmul_03_b200 import workloads as wl  # noqa: E402
+
+N_OUT, K_IN, GS = 14336, 4096, 64
+L2_ROTATE = 8
+
+
+def weight_bytes(n, k, bits, gs, elt=2):
+    """Algorithmic bytes of one packed weight: codes + scales + biases."""
+    return n * k * bits // 8 + 2 * n * (k // gs) * elt
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# ---------------------------------------------------------------------------
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, v: float) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return None
+        self.file.flush()
+        rows = [r.split(",") for r in Path(self.file.name).read_text().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# timing helpers
+# ---------------------------------------------------------------------------
+
+def timed_launches(fns, steps, warmup, world):
+    """Run fns[i % len(fns)] for warmup + steps iterations.  Returns (total ms
+    over the timed steps, mean per-launch ms, launches counted).  The timed
+    region is bracketed by a barrier and a synchronize on both sides; a sleep
+    kernel queued ahead of it lets the host enqueue every step before the GPU
+    reaches them, so per-step events see kernel time, not host launch time."""
+    from quantized_matmul_03_b200 import binding as qb
+    for i in range(warmup):
+        fns[i % len(fns)]()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(int(40e6))             # ~20 ms of GPU time to queue behind
+    n0 = qb.qmm_launch_count()
+    t0.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        fns[i % len(fns)]()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    n1 = qb.qmm_launch_count()
+    torch.cuda.synchronize()
+    barrier(world)
+    total = t0.elapsed_time(t1)
+    per = [a.elapsed_time(b) for a, b in ev]
+    return total, sum(per) / len(per), n1 - n0
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "src": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted((ROOT / "quantized_matmul_03_b200" / "csrc").glob("*.cu*")):
+        h.update(f.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """dram bytes per launch from a committed ncu summary, when the kernel
+    sources have not changed since it was taken; else None."""
+    p = ROOT / "profiles" / "traffic.json"
+    if not p.exists():
+        return None
+    d = json.loads(p.read_text())
+    e = d.get(f"{kernel}:{workload}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+
+def make_packed(w_cpu, gs, bits, copies, device):
+    from quantized_matmul_03_b200 import binding as qb
+    w = w_cpu.to(device)
+    wq, s, b = qb.qmm_quantize(w, gs, bits)
+    out = [(wq, s, b)]
+    for _ in range(copies - 1):
+        out.append((wq.clone(), s.clone(), b.clone()))
+    del w
+    torch.cuda.synchronize()
+    return out
+
+
+def bench_decode(m, steps, warmup, world, device, bits=4):
+    from quantized_matmul_03_b200 import binding as qb
+    c = wl.decode_case(m, bits=bits)
+    packs = make_packed(c.w, c.group_size, c.bits, L2_ROTATE, device)
+    x = c.x.to(device)
+    y = torch.empty((m, N_OUT), dtype=torch.bfloat16, device=device)
+    fns = [lambda p=p: qb.qmm_quantized_matmul(x, *p, True, c.group_size, c.bits, out=y)
+           for p in packs]
+    total_ms, per_ms, launches = timed_launches(fns, steps, warmup, world)
+    nbytes = weight_bytes(N_OUT, K_IN, c.bits, c.group_size)
+    return dict(case=c, packs=packs, x=x, y=y, total_ms=total_ms, per_ms=per_ms,
+                launches=launches, bytes=nbytes, flops=2 * m * N_OUT * K_IN)
+
+
+def bench_decode_e2e(d, steps, warmup, world, device):
+    """Same decode step through the public API with host buffers: pinned x is
+    copied in and y copied out inside the timed region."""
+    from quantized_matmul_03_b200 import binding as qb
+    c = d["case"]
+    x_host = c.x.clone().pin_memory()
+    y_host = torch.empty(tuple(d["y"].shape), dtype=torch.bfloat16).pin_memory()
+    x_dev, y_dev = d["x"], d["y"]
+    packs = d["packs"]
+
+    def step(p):
+        x_dev.copy_(x_host, non_blocking=True)
+        qb.qmm_quantized_matmul(x_dev, *p, True, c.group_size, c.bits, out=y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+
+    fns = [lambda p=p: step(p) for p in packs]
+    total_ms, _, _ = timed_launches(fns, steps, warmup, world)
+    total_ms = max_over_ranks(world, total_ms)
+    gbs = world * steps * d["bytes"] / (total_ms * 1e-3) / 1e9
+    return {"value": gbs, "unit": "GB/s",
+            "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+            "d2h_bytes_per_step": y_host.numel() * y_host.element_size()}
+
+
+def bench_prefill(bits, steps, warmup, world, device):
+    from quantized_matmul_03_b200 import binding as qb
+    c = wl.prefill_case(bits)
+    packs = make_packed(c.w, c.group_size, c.bits, 2, device)
+    x = c.x.to(device)
+    y = torch.empty((x.shape[0], N_OUT), dtype=torch.bfloat16, device=device)
+    fns = [lambda p=p: qb.qmm_quantized_matmul(x, *p, True, c.group_size, c.bits, out=y)
+           for p in packs]
+    total_ms, per_ms, launches = timed_launches(fns, steps, warmup, world)
+    flops = 2 * x.shape[0] * N_OUT * K_IN
+    return dict(total_ms=total_ms, per_ms=per_ms, launches=launches, flops=flops)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample of the decode workload)
+# ---------------------------------------------------------------------------
+
+def oracle_decode_sample(budget_s: float, rows: int = N_OUT):
+    """Time the oracle's quantized_matmul on the decode workload (M = 1, the
+    first `rows` weight rows), repeating until `budget_s` of CPU time."""
+    import oracle
+    c = wl.decode_case(1)
+    w = c.w[:rows].contiguous()
+    wq, s, b = oracle.quantize(w, c.group_size, c.bits)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.quantized_matmul(c.x, wq, s, b, True, c.group_size, c.bits)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    nbytes = weight_bytes(rows, K_IN, c.bits, c.group_size)
+    return {"value": reps * nbytes / el / 1e9, "unit": "GB/s",
+            "cores": torch.get_num_threads(), "kind": "oracle",
+            "sample": (f"oracle quantized_matmul, x [1,4096] x W[{rows},4096] int4 gs64, "
+                       f"{reps} passes in {el:.1f} s (dequantize in C on 1 thread, float64 "
+                       f"matmul on {torch.get_num_threads()} threads)")}
+
+
+# ---------------------------------------------------------------------------
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle, timed on this host's cores."""
+    if rank != 0:
+        return 0
+    import oracle
+    rows = 1792        # 1/8 of the decode weight per step keeps a step ~0.1-0.3 s
+    c = wl.decode_case(1)
+    w = c.w[:rows].contiguous()
+    wq, s, b = oracle.quantize(w, c.group_size, c.bits)
+    for _ in range(args.warmup):
+        oracle.quantized_matmul(c.x, wq, s, b, True, c.group_size, c.bits)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.quantized_matmul(c.x, wq, s, b, True, c.group_size, c.bits)
+    el = time.perf_counter() - t0
+    nbytes = weight_bytes(rows, K_IN, c.bits, c.group_size)
+    v = args.steps * nbytes / el / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "decode_m1_int4_gs64 (rows sampled)", "rows_per_step": rows,
+                   "M": 1, "N": N_OUT, "K": K_IN, "bits": 4, "group_size": GS},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": torch.get_num_threads(),
+                         "kind": "oracle",
+                         "sample": f"W rows [0,{rows}) of the decode weight per step"},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+METRIC = "int4 qmm weight GB/s at M=1 and TFLOP/s at M=2048, % of roofline"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    from quantized_matmul_03_b200 import binding as qb
+    qb.lib()  # fails loudly if the library was not built
+    device = torch.device("cuda", local)
+    pk = peaks()
+
+    with ClockSampler(local) as clk:
+        d = bench_decode(1, args.steps, args.warmup, world, device)
+        pre = None
+        if not args.no_prefill:
+            psteps = max(3, min(args.steps, 20))
+            pre = bench_prefill(4, psteps, max(3, args.warmup // 4), world, device)
+    clocks = clk.summary()
+
+    total_ms = max_over_ranks(world, d["total_ms"])
+    per_ms = max_over_ranks(world, d["per_ms"])
+    value = world * args.steps * d["bytes"] / (total_ms * 1e-3) / 1e9
+    achieved = d["bytes"] / (per_ms * 1e-3) / 1e9
+    e2e = bench_decode_e2e(d, args.steps, args.warmup, world, device)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "decode_m1_int4_gs64", "M": 1, "N": N_OUT, "K": K_IN,
+                   "bits": 4, "group_size": GS, "transpose": True,
+                   "l2": f"rotating {L2_ROTATE} weight copies ({L2_ROTATE * d['bytes'] / 1e6:.0f}"
+                         " MB > 126 MB L2)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                     "peak_src": pk["src"], "kernel_us": per_ms * 1e3,
+                     "traffic": profiled_traffic("gemv", "decode_m1_int4_gs64")},
+        "e2e": e2e,
+        "gpu_launches": d["launches"],
+    }
+    if pre is not None:
+        p_ms = max_over_ranks(world, pre["per_ms"])
+        tf = pre["flops"] / (p_ms * 1e-3) / 1e12
+        line["prefill"] = {
+            "workload": "prefill_m2048_int4_gs64", "value": tf, "unit": "TFLOP/s",
+            "kernel_us": p_ms * 1e3, "launches": pre["launches"],
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"],
+                         "peak_src": pk["src"]}}
+        line["gpu_launches"] += pre["launches"]
+    if clocks:
+        line["clocks"] = clocks
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_decode_sample(args.cpu_budget_s)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

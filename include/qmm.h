@@ -1,0 +1,168 @@
+/*
+ * qmm.h -- C ABI of libqmm, group-wise affine quantized matmul for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operations follow the MLX quantization API as four pages describe it:
+ *   EMLX.Quantization (emlx 0.4.2): quantize, dequantize, quantized_matmul,
+ *     gather_quantized_matmul;
+ *   Emily.QuantizedWeight (emily 0.7.2), section Layout: the packed value /
+ *     scales / biases layout;
+ *   Emily.Quantization.Layers (emily 1.0.0), quantized_dense: the two weight
+ *     layouts selected by `transpose`;
+ *   mlx-rs src/mlx_rs/ops/quantization.rs: quantize, quantized_matmul,
+ *     dequantize, gather_qmm and their defaults (mode "affine", group size 64,
+ *     4 bits).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.  Every array argument is a DEVICE pointer owned by the caller,
+ *   row-major and contiguous, and 16-byte aligned (misaligned pointers are
+ *   rejected with QMM_ERR_INVALID_ARG).  The library allocates no device
+ *   memory; gather_qmm takes a caller-provided workspace.
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *   default stream).  Calls only enqueue work and return; results are ready
+ *   when the stream is synchronised.
+ * Errors.  Arguments are validated before anything is launched; on any error
+ *   nothing is enqueued.  Exceptions never cross the ABI.  A thread-local
+ *   message for the last failure is available from qmm_last_error().
+ * Packing.  bits in {2, 4, 8}; 32/bits codes per uint32 word, code j of a row
+ *   at bit (j mod 32/bits)*bits of word j/(32/bits) (least significant first).
+ * Groups.  group_size in {32, 64, 128}; one scale and one bias per group of
+ *   consecutive elements along the LAST STORED axis of the weight (the packed
+ *   axis), for both matmul layouts.
+ * Dtypes.  scales and biases share the dense weight's dtype; outputs take the
+ *   scales dtype (EMLX.Quantization, section quantized_matmul); activations
+ *   must have that dtype too.
+ * Mode.  `mode` NULL means "affine" (the pages' default).  The microscaled
+ *   modes named on the pages ("mxfp4", "mxfp8", "nvfp4") return
+ *   QMM_ERR_UNSUPPORTED; any other string returns QMM_ERR_INVALID_ARG.
+ */
+#ifndef QMM_H
+#define QMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QMM_OK = 0,
+    QMM_ERR_INVALID_ARG = 1, /* bad size, pointer, group size, bits, ... */
+    QMM_ERR_UNSUPPORTED = 2, /* valid on the pages but not built (e.g. mxfp4) */
+    QMM_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    QMM_ERR_TIMEOUT = 4,     /* a kernel's bounded wait ran out (device word) */
+    QMM_ERR_INDEX = 5,       /* an expert / row index was out of range */
+    QMM_ERR_WORKSPACE = 6    /* workspace missing or smaller than required */
+} qmm_status;
+
+typedef enum { QMM_F32 = 0, QMM_BF16 = 1, QMM_F16 = 2 } qmm_dtype;
+
+/*
+ * qmm_quantize -- EMLX.Quantization, section quantize; mlx-rs quantize.
+ * Quantizes w[rows, cols] (dtype `dtype`) group by group along its last axis.
+ *   w       in : [rows, cols] dense weight (leading axes flattened into rows)
+ *   wq      out: [rows, cols*bits/32] uint32 packed codes
+ *   scales  out: [rows, cols/group_size], dtype `dtype`
+ *   biases  out: [rows, cols/group_size], dtype `dtype`
+ * Rule: bias = group min, scale = (max - min)/(2^bits - 1) in fp32, both
+ * rounded to `dtype` (nearest-even); q = clamp(rint((w - bias)/scale), 0,
+ * 2^bits - 1) against the stored scale and bias, 0 when the scale is 0.
+ * cols must be a positive multiple of group_size; rows may be 0 (no-op).
+ */
+qmm_status qmm_quantize(const void *w, qmm_dtype dtype, int64_t rows, int64_t cols,
+                        int group_size, int bits, const char *mode,
+                        uint32_t *wq, void *scales, void *biases, void *stream);
+
+/*
+ * qmm_dequantize -- EMLX.Quantization, section dequantize; mlx-rs dequantize.
+ *   out[r, c] = round_to_dtype(fmaf(scale[r, c/gs], q[r, c], bias[r, c/gs]))
+ *   wq [rows, cols*bits/32], scales/biases [rows, cols/gs], out [rows, cols],
+ *   all in `dtype` except wq.
+ */
+qmm_status qmm_dequantize(const uint32_t *wq, const void *scales, const void *biases,
+                          qmm_dtype dtype, int64_t rows, int64_t cols, int group_size,
+                          int bits, const char *mode, void *out, void *stream);
+
+/*
+ * qmm_quantized_matmul -- mlx-rs quantized_matmul; EMLX.Quantization, section
+ * quantized_matmul; Emily.Quantization.Layers, quantized_dense.
+ *   x [M, K] (dtype), y [M, N] (dtype).
+ *   transpose != 0: W is [N, K] ("[out, in]"), y = x @ W^T;
+ *                   wq [N, K*bits/32], scales/biases [N, K/gs]; K % gs == 0.
+ *   transpose == 0: W is [K, N] ("[in, out]"), y = x @ W;
+ *                   wq [K, N*bits/32], scales/biases [K, N/gs]; N % gs == 0.
+ * The packed weight is streamed and dequantized inside the product; no dense
+ * weight is written to memory.  M == 0 or N == 0 is a no-op.
+ */
+qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K,
+                                const uint32_t *wq, const void *scales, const void *biases,
+                                qmm_dtype dtype, int64_t N, int transpose,
+                                int group_size, int bits, const char *mode,
+                                void *y, void *stream);
+
+/*
+ * qmm_gather_qmm -- EMLX.Quantization, section gather_quantized_matmul;
+ * mlx-rs gather_qmm.  Experts are stacked on the weight's leading axis:
+ *   transpose != 0: wq [n_experts, N, K*bits/32], scales/biases [n_experts, N, K/gs]
+ *   transpose == 0: wq [n_experts, K, N*bits/32], scales/biases [n_experts, K, N/gs]
+ *   x [x_batch, M, K]; y [batch, M, N].
+ * For b in [0, batch):
+ *   y[b] = x[xi] @ W[ei]^T (or x[xi] @ W[ei] when transpose == 0), with
+ *   xi = lhs_indices[b] if lhs_indices else (x_batch == 1 ? 0 : b),
+ *   ei = rhs_indices[b] if rhs_indices else (n_experts == 1 ? 0 : b).
+ * Without lhs_indices, x_batch must be 1 or batch; without rhs_indices,
+ * n_experts must be 1 or batch.  Indices are int32 device arrays of length
+ * `batch`.  No expert weight is copied.  sorted_indices != 0 promises that
+ * rhs_indices is non-decreasing, which lets the library skip its sort.
+ * Out-of-range indices: the affected output rows are written as zeros and a
+ * later qmm_device_status() reports QMM_ERR_INDEX.
+ * workspace: device scratch of at least qmm_gather_qmm_workspace_size(...)
+ * bytes, 256-byte aligned; contents need not be initialised and are not
+ * preserved.  Two calls in flight at once must not share a workspace.
+ */
+size_t qmm_gather_qmm_workspace_size(int64_t batch, int64_t M, int64_t K,
+                                     int64_t n_experts, qmm_dtype dtype);
+
+qmm_status qmm_gather_qmm(const void *x, int64_t x_batch, int64_t M, int64_t K,
+                          const uint32_t *wq, const void *scales, const void *biases,
+                          qmm_dtype dtype, int64_t n_experts, int64_t N,
+                          const int32_t *lhs_indices, const int32_t *rhs_indices,
+                          int64_t batch, int transpose, int group_size, int bits,
+                          const char *mode, int sorted_indices,
+                          void *y, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
+/*
+ * qmm_device_status -- synchronise `stream`, then read (and, if `reset` is
+ * non-zero, clear) the library's device-side error word, set by kernels whose
+ * bounded waits time out (QMM_ERR_TIMEOUT) or that meet an out-of-range index
+ * (QMM_ERR_INDEX).  Returns QMM_OK when the word is clear.
+ */
+qmm_status qmm_device_status(void *stream, int reset);
+
+/*
+ * Kernel-path selection for qmm_quantized_matmul (process-wide; the default
+ * is QMM_PATH_AUTO).  QMM_PATH_GEMV forces the SIMT decode kernels (M <= 16
+ * rows at a time), QMM_PATH_GEMM the tensor-core (tcgen05) kernel.  A forced
+ * path that cannot run a given call returns QMM_ERR_UNSUPPORTED.
+ */
+typedef enum { QMM_PATH_AUTO = 0, QMM_PATH_GEMV = 1, QMM_PATH_GEMM = 2 } qmm_path;
+qmm_status qmm_set_path(qmm_path path);
+
+/*
+ * Number of CUDA kernels this process has launched through libqmm so far
+ * (all devices, all entry points).  For accounting in benchmarks and tests.
+ */
+uint64_t qmm_launch_count(void);
+
+const char *qmm_status_string(qmm_status status);
+const char *qmm_last_error(void);
+int qmm_version(void); /* major*10000 + minor*100 + patch */
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QMM_H */

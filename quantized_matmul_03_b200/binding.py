@@ -1,0 +1,205 @@
+"""Thin ctypes binding over libqmm's C ABI (``include/qmm.h``).
+
+Argument marshalling only: shapes and dtypes are read off torch tensors,
+outputs are allocated with torch on the input's device, and every step of the
+computation runs in libqmm's CUDA kernels on torch's current stream.  There is
+no fallback: if ``libqmm.so`` is missing or the tensors are not on a CUDA
+device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+from typing import Optional
+
+import torch
+
+LIB_PATH = Path(__file__).resolve().parent / "libqmm.so"
+
+QMM_OK = 0
+STATUS_NAMES = {0: "QMM_OK", 1: "QMM_ERR_INVALID_ARG", 2: "QMM_ERR_UNSUPPORTED",
+                3: "QMM_ERR_CUDA", 4: "QMM_ERR_TIMEOUT", 5: "QMM_ERR_INDEX",
+                6: "QMM_ERR_WORKSPACE"}
+PATHS = {"auto": 0, "gemv": 1, "gemm": 2}
+DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+
+_lib = None
+
+
+class QmmError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqmm.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not LIB_PATH.exists():
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with quantized_matmul_03_b200.build.build() "
+                "(or __graft_entry__.build()); there is no CPU fallback")
+        L = ctypes.CDLL(str(LIB_PATH))
+        i64, i32, vp, sz = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+        cp = ctypes.c_char_p
+        sig = {
+            "qmm_quantize": [vp, i32, i64, i64, i32, i32, cp, vp, vp, vp, vp],
+            "qmm_dequantize": [vp, vp, vp, i32, i64, i64, i32, i32, cp, vp, vp],
+            "qmm_quantized_matmul": [vp, i64, i64, vp, vp, vp, i32, i64, i32, i32, i32, cp,
+                                     vp, vp],
+            "qmm_gather_qmm": [vp, i64, i64, i64, vp, vp, vp, i32, i64, i64, vp, vp, i64, i32,
+                               i32, i32, cp, i32, vp, vp, sz, vp],
+            "qmm_device_status": [vp, i32],
+            "qmm_set_path": [i32],
+        }
+        for name, args in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        L.qmm_gather_qmm_workspace_size.argtypes = [i64, i64, i64, i64, i32]
+        L.qmm_gather_qmm_workspace_size.restype = sz
+        L.qmm_status_string.argtypes = [i32]
+        L.qmm_status_string.restype = cp
+        L.qmm_last_error.argtypes = []
+        L.qmm_last_error.restype = cp
+        L.qmm_launch_count.argtypes = []
+        L.qmm_launch_count.restype = ctypes.c_uint64
+        L.qmm_version.argtypes = []
+        L.qmm_version.restype = i32
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != QMM_OK:
+        raise QmmError(status, (lib().qmm_last_error() or b"").decode())
+
+
+def _p(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _mode(mode: Optional[str]):
+    return None if mode is None else mode.encode()
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and (t.device.type != "cuda" or not t.is_contiguous()):
+            raise ValueError("libqmm takes contiguous CUDA tensors")
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype not in DTYPES:
+        raise ValueError(f"unsupported dtype {t.dtype}")
+    return DTYPES[t.dtype]
+
+
+def qmm_quantize(w: torch.Tensor, group_size: int = 64, bits: int = 4, mode: str = "affine"):
+    """Quantize ``w`` (rank >= 2) along its last axis -> (wq, scales, biases).
+
+    ``wq`` is int32 holding the uint32 words; scales/biases take ``w``'s dtype.
+    """
+    _cuda(w)
+    cols = w.shape[-1]
+    rows = w.numel() // cols if cols else 0
+    lead = tuple(w.shape[:-1])
+    wq = torch.empty(lead + (cols * bits // 32,), dtype=torch.int32, device=w.device)
+    scales = torch.empty(lead + (max(cols // group_size, 0),), dtype=w.dtype, device=w.device)
+    biases = torch.empty_like(scales)
+    _check(lib().qmm_quantize(_p(w), _dtype(w), rows, cols, group_size, bits, _mode(mode),
+                              _p(wq), _p(scales), _p(biases), _stream(w.device)))
+    return wq, scales, biases
+
+
+def qmm_dequantize(wq, scales, biases, group_size: int = 64, bits: int = 4,
+                   mode: str = "affine"):
+    """Dense weight ``scale * q + bias`` in the scales dtype."""
+    _cuda(wq, scales, biases)
+    cols = wq.shape[-1] * 32 // bits
+    rows = wq.numel() // wq.shape[-1] if wq.shape[-1] else 0
+    out = torch.empty(tuple(wq.shape[:-1]) + (cols,), dtype=scales.dtype, device=wq.device)
+    _check(lib().qmm_dequantize(_p(wq), _p(scales), _p(biases), _dtype(scales), rows, cols,
+                                group_size, bits, _mode(mode), _p(out), _stream(wq.device)))
+    return out
+
+
+def qmm_quantized_matmul(x, wq, scales, biases, transpose: bool = True, group_size: int = 64,
+                         bits: int = 4, mode: str = "affine", out: Optional[torch.Tensor] = None):
+    """``x @ W.T`` (transpose) or ``x @ W`` with W packed; x is [..., K]."""
+    _cuda(x, wq, scales, biases, out)
+    K = x.shape[-1]
+    M = x.numel() // K if K else 0
+    if transpose:
+        N = wq.shape[-2]
+    else:
+        N = wq.shape[-1] * 32 // bits
+    if out is None:
+        out = torch.empty(tuple(x.shape[:-1]) + (N,), dtype=scales.dtype, device=x.device)
+    _check(lib().qmm_quantized_matmul(_p(x), M, K, _p(wq), _p(scales), _p(biases),
+                                      _dtype(scales), N, int(bool(transpose)), group_size, bits,
+                                      _mode(mode), _p(out), _stream(x.device)))
+    return out
+
+
+def qmm_gather_qmm_workspace_size(batch: int, M: int, K: int, n_experts: int,
+                                  dtype=torch.bfloat16) -> int:
+    return int(lib().qmm_gather_qmm_workspace_size(batch, M, K, n_experts, DTYPES[dtype]))
+
+
+def qmm_gather_qmm(x, wq, scales, biases, lhs_indices=None, rhs_indices=None,
+                   transpose: bool = True, group_size: int = 64, bits: int = 4,
+                   mode: str = "affine", sorted_indices: bool = False,
+                   workspace: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None):
+    """Mixture-of-experts quantized matmul: x [x_batch, M, K], experts stacked
+    on wq's leading axis; returns y [batch, M, N]."""
+    _cuda(x, wq, scales, biases, lhs_indices, rhs_indices, workspace, out)
+    for t in (lhs_indices, rhs_indices):
+        if t is not None and t.dtype != torch.int32:
+            raise ValueError("indices must be int32")
+    x_batch, M, K = x.shape
+    n_experts = wq.shape[0]
+    N = wq.shape[1] if transpose else wq.shape[2] * 32 // bits
+    sizes = [t.numel() for t in (lhs_indices, rhs_indices) if t is not None]
+    if lhs_indices is None:
+        sizes.append(x_batch)
+    if rhs_indices is None:
+        sizes.append(n_experts)
+    batch = max(sizes)
+    if out is None:
+        out = torch.empty((batch, M, N), dtype=scales.dtype, device=x.device)
+    need = qmm_gather_qmm_workspace_size(batch, M, K, n_experts, scales.dtype)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().qmm_gather_qmm(_p(x), x_batch, M, K, _p(wq), _p(scales), _p(biases),
+                                _dtype(scales), n_experts, N, _p(lhs_indices), _p(rhs_indices),
+                                batch, int(bool(transpose)), group_size, bits, _mode(mode),
+                                int(bool(sorted_indices)), _p(out), _p(workspace), ws_bytes,
+                                _stream(x.device)))
+    return out
+
+
+def qmm_device_status(reset: bool = True, device=None):
+    """Synchronise the current stream and raise if a kernel recorded an error."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    _check(lib().qmm_device_status(_stream(dev), int(bool(reset))))
+
+
+def qmm_set_path(path: str = "auto"):
+    _check(lib().qmm_set_path(PATHS[path]))
+
+
+def qmm_launch_count() -> int:
+    """Kernels launched through libqmm by this process so far."""
+    return int(lib().qmm_launch_count())
+
+
+def qmm_version() -> int:
+    return int(lib().qmm_version())

@@ -1,0 +1,76 @@
+"""Build ``libqmm.so`` in-tree from ``csrc/*.cu`` with nvcc for sm_100a.
+
+Each translation unit is compiled separately (in parallel) into ``_build/``
+and linked into one shared library next to this file, so the library travels
+with the source tree.  No GPU is needed to build.
+"""
+from __future__ import annotations
+
+import concurrent.futures as cf
+import os
+import shutil
+import subprocess
+import sys
+from pathlib import Path
+
+PKG = Path(__file__).resolve().parent
+CSRC = PKG / "csrc"
+INCLUDE = PKG.parent / "include"
+BUILD = PKG.parent / "_build"
+LIB = PKG / "libqmm.so"
+
+NVCC = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+# No --use_fast_math: the quantize path relies on IEEE division and rounding.
+NVCC_FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-O3", "-lineinfo", "-std=c++17",
+    "-Xcompiler", "-fPIC,-O2,-Wall",
+    "--expt-relaxed-constexpr",
+    "-I", str(INCLUDE),
+]
+
+
+def _sources():
+    return sorted(CSRC.glob("*.cu"))
+
+
+def _headers():
+    return sorted(CSRC.glob("*.cuh")) + sorted(INCLUDE.glob("*.h"))
+
+
+def _stale(target: Path, deps) -> bool:
+    if not target.exists():
+        return True
+    t = target.stat().st_mtime
+    return any(d.stat().st_mtime > t for d in deps)
+
+
+def _compile(src: Path, extra) -> Path:
+    obj = BUILD / (src.stem + ".o")
+    if _stale(obj, [src, *_headers()]) or extra:
+        cmd = [NVCC, *NVCC_FLAGS, *extra, "-dc" if False else "-c", str(src), "-o", str(obj)]
+        subprocess.run(cmd, check=True)
+    return obj
+
+
+def build(force: bool = False, verbose_ptxas: bool = False) -> Path:
+    """Compile every CUDA source and link libqmm.so; return its path."""
+    BUILD.mkdir(exist_ok=True)
+    extra = ["-Xptxas", "-v"] if verbose_ptxas else []
+    if force:
+        for o in BUILD.glob("*.o"):
+            o.unlink()
+    srcs = _sources()
+    with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        objs = list(ex.map(lambda s: _compile(s, extra), srcs))
+    if _stale(LIB, objs) or force:
+        tmp = LIB.with_suffix(f".so.tmp{os.getpid()}")
+        cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
+               "-Xcompiler", "-fPIC", *map(str, objs), "-o", str(tmp)]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose_ptxas="--ptxas-v" in sys.argv))

@@ -1,0 +1,262 @@
+// api.cu -- the extern "C" boundary of libqmm (declared in include/qmm.h).
+//
+// Every entry point validates its arguments completely before enqueueing
+// anything, reports failures as qmm_status values (the Rust binding on the
+// mlx-rs page returns Result / Exception, Emily raises "with a clear error
+// before touching MLX"), and never lets a C++ exception cross the ABI.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "qmm_internal.cuh"
+
+namespace qmm {
+
+__device__ int g_qmm_device_error = 0;
+
+namespace {
+
+thread_local std::string t_last_error;
+qmm_path g_path = QMM_PATH_AUTO;
+
+qmm_status fail(qmm_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+qmm_status fail(qmm_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return st;
+}
+
+qmm_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(QMM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Mode strings of the pages: "affine" (default), and the microscaled modes
+// that carry fixed group sizes and no biases (Emily.QuantizedWeight, section
+// Microscaled modes).
+qmm_status check_mode(const char *mode) {
+    if (mode == nullptr || std::strcmp(mode, "affine") == 0) return QMM_OK;
+    if (!std::strcmp(mode, "mxfp4") || !std::strcmp(mode, "mxfp8") || !std::strcmp(mode, "nvfp4"))
+        return fail(QMM_ERR_UNSUPPORTED, "mode \"%s\" is not built (affine only)", mode);
+    return fail(QMM_ERR_INVALID_ARG, "unknown quantization mode \"%s\"", mode);
+}
+
+qmm_status check_common(qmm_dtype dt, int group_size, int bits, const char *mode) {
+    qmm_status st = check_mode(mode);
+    if (st != QMM_OK) return st;
+    if (dt != QMM_F32 && dt != QMM_BF16 && dt != QMM_F16)
+        return fail(QMM_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    if (bits == 3 || bits == 6)
+        return fail(QMM_ERR_UNSUPPORTED, "bits=%d is not built (2, 4, 8 only)", bits);
+    if (bits != 2 && bits != 4 && bits != 8)
+        return fail(QMM_ERR_INVALID_ARG, "bits must be 2, 4 or 8 (got %d)", bits);
+    if (group_size != 32 && group_size != 64 && group_size != 128)
+        return fail(QMM_ERR_INVALID_ARG, "group_size must be 32, 64 or 128 (got %d)", group_size);
+    return QMM_OK;
+}
+
+#define QMM_CHECK_PTR(p, name)                                                        \
+    do {                                                                              \
+        if ((p) == nullptr) return fail(QMM_ERR_INVALID_ARG, "%s is NULL", name);     \
+        if (!aligned16(p)) return fail(QMM_ERR_INVALID_ARG, "%s is not 16-byte aligned", name); \
+    } while (0)
+
+qmm_status check_matmul(const void *x, int64_t M, int64_t K, const uint32_t *wq,
+                        const void *scales, const void *biases, int64_t N, int transpose,
+                        int group_size, void *y) {
+    if (M < 0 || N < 0 || K <= 0)
+        return fail(QMM_ERR_INVALID_ARG, "sizes must satisfy M >= 0, N >= 0, K > 0");
+    const int64_t packed_axis = transpose ? K : N;
+    if (packed_axis % group_size != 0)
+        return fail(QMM_ERR_INVALID_ARG,
+                    "the packed axis (%s = %lld) must be a multiple of group_size %d",
+                    transpose ? "K" : "N", (long long)packed_axis, group_size);
+    if (M == 0 || N == 0) return QMM_OK;
+    QMM_CHECK_PTR(x, "x");
+    QMM_CHECK_PTR(wq, "wq");
+    QMM_CHECK_PTR(scales, "scales");
+    if (biases == nullptr)
+        return fail(QMM_ERR_INVALID_ARG, "biases is NULL (required for mode \"affine\")");
+    QMM_CHECK_PTR(biases, "biases");
+    QMM_CHECK_PTR(y, "y");
+    return QMM_OK;
+}
+
+qmm_status finish_launch(cudaError_t e, const char *what) {
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return QMM_OK;
+}
+
+}  // namespace
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+int *device_error_word() {
+    static int *cached[64] = {nullptr};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return nullptr;
+    if (cached[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_qmm_device_error) != cudaSuccess) return nullptr;
+        cached[dev] = static_cast<int *>(p);
+    }
+    return cached[dev];
+}
+
+int num_sms() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+}  // namespace qmm
+
+using namespace qmm;
+
+extern "C" {
+
+qmm_status qmm_quantize(const void *w, qmm_dtype dtype, int64_t rows, int64_t cols,
+                        int group_size, int bits, const char *mode, uint32_t *wq, void *scales,
+                        void *biases, void *stream) {
+    try {
+        qmm_status st = check_common(dtype, group_size, bits, mode);
+        if (st != QMM_OK) return st;
+        if (rows < 0 || cols <= 0 || cols % group_size != 0)
+            return fail(QMM_ERR_INVALID_ARG,
+                        "need rows >= 0 and cols a positive multiple of group_size");
+        if (rows == 0) return QMM_OK;
+        QMM_CHECK_PTR(w, "w");
+        QMM_CHECK_PTR(wq, "wq");
+        QMM_CHECK_PTR(scales, "scales");
+        QMM_CHECK_PTR(biases, "biases");
+        QuantArgs a{w, rows, cols, group_size, bits, wq, scales, biases};
+        return finish_launch(launch_quantize(dtype, a, (cudaStream_t)stream), "quantize launch");
+    } catch (...) {
+        return fail(QMM_ERR_CUDA, "unexpected exception in qmm_quantize");
+    }
+}
+
+qmm_status qmm_dequantize(const uint32_t *wq, const void *scales, const void *biases,
+                          qmm_dtype dtype, int64_t rows, int64_t cols, int group_size, int bits,
+                          const char *mode, void *out, void *stream) {
+    try {
+        qmm_status st = check_common(dtype, group_size, bits, mode);
+        if (st != QMM_OK) return st;
+        if (rows < 0 || cols <= 0 || cols % group_size != 0)
+            return fail(QMM_ERR_INVALID_ARG,
+                        "need rows >= 0 and cols a positive multiple of group_size");
+        if (rows == 0) return QMM_OK;
+        QMM_CHECK_PTR(wq, "wq");
+        QMM_CHECK_PTR(scales, "scales");
+        if (biases == nullptr)
+            return fail(QMM_ERR_INVALID_ARG, "biases is NULL (required for mode \"affine\")");
+        QMM_CHECK_PTR(biases, "biases");
+        QMM_CHECK_PTR(out, "out");
+        DequantArgs a{wq, scales, biases, rows, cols, group_size, bits, out};
+        return finish_launch(launch_dequantize(dtype, a, (cudaStream_t)stream),
+                             "dequantize launch");
+    } catch (...) {
+        return fail(QMM_ERR_CUDA, "unexpected exception in qmm_dequantize");
+    }
+}
+
+qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K, const uint32_t *wq,
+                                const void *scales, const void *biases, qmm_dtype dtype,
+                                int64_t N, int transpose, int group_size, int bits,
+                                const char *mode, void *y, void *stream) {
+    try {
+        qmm_status st = check_common(dtype, group_size, bits, mode);
+        if (st != QMM_OK) return st;
+        st = check_matmul(x, M, K, wq, scales, biases, N, transpose, group_size, y);
+        if (st != QMM_OK) return st;
+        if (M == 0 || N == 0) return QMM_OK;
+        QmmArgs a{x, wq, scales, biases, y, M, N, K, group_size, bits, transpose != 0};
+        if (g_path == QMM_PATH_GEMM)
+            return fail(QMM_ERR_UNSUPPORTED, "the tensor-core path is not available");
+        return finish_launch(launch_gemv(dtype, a, (cudaStream_t)stream), "gemv launch");
+    } catch (...) {
+        return fail(QMM_ERR_CUDA, "unexpected exception in qmm_quantized_matmul");
+    }
+}
+
+size_t qmm_gather_qmm_workspace_size(int64_t batch, int64_t M, int64_t K, int64_t n_experts,
+                                     qmm_dtype dtype) {
+    (void)batch; (void)M; (void)K; (void)n_experts; (void)dtype;
+    return 0;
+}
+
+qmm_status qmm_gather_qmm(const void *x, int64_t x_batch, int64_t M, int64_t K,
+                          const uint32_t *wq, const void *scales, const void *biases,
+                          qmm_dtype dtype, int64_t n_experts, int64_t N,
+                          const int32_t *lhs_indices, const int32_t *rhs_indices, int64_t batch,
+                          int transpose, int group_size, int bits, const char *mode,
+                          int sorted_indices, void *y, void *workspace, size_t workspace_bytes,
+                          void *stream) {
+    (void)x; (void)x_batch; (void)M; (void)K; (void)wq; (void)scales; (void)biases;
+    (void)dtype; (void)n_experts; (void)N; (void)lhs_indices; (void)rhs_indices; (void)batch;
+    (void)transpose; (void)group_size; (void)bits; (void)mode; (void)sorted_indices; (void)y;
+    (void)workspace; (void)workspace_bytes; (void)stream;
+    return fail(QMM_ERR_UNSUPPORTED, "gather_qmm is not built yet");
+}
+
+qmm_status qmm_device_status(void *stream, int reset) {
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    int word = 0;
+    e = cudaMemcpyFromSymbol(&word, g_qmm_device_error, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+    if (reset && word != 0) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_qmm_device_error, &zero, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+    }
+    if (word == QMM_ERR_TIMEOUT) return fail(QMM_ERR_TIMEOUT, "a kernel's bounded wait timed out");
+    if (word == QMM_ERR_INDEX) return fail(QMM_ERR_INDEX, "an index was out of range");
+    if (word != 0) return fail((qmm_status)word, "device error word %d", word);
+    return QMM_OK;
+}
+
+qmm_status qmm_set_path(qmm_path path) {
+    if (path != QMM_PATH_AUTO && path != QMM_PATH_GEMV && path != QMM_PATH_GEMM)
+        return fail(QMM_ERR_INVALID_ARG, "unknown path %d", (int)path);
+    g_path = path;
+    return QMM_OK;
+}
+
+const char *qmm_status_string(qmm_status s) {
+    switch (s) {
+    case QMM_OK: return "QMM_OK";
+    case QMM_ERR_INVALID_ARG: return "QMM_ERR_INVALID_ARG";
+    case QMM_ERR_UNSUPPORTED: return "QMM_ERR_UNSUPPORTED";
+    case QMM_ERR_CUDA: return "QMM_ERR_CUDA";
+    case QMM_ERR_TIMEOUT: return "QMM_ERR_TIMEOUT";
+    case QMM_ERR_INDEX: return "QMM_ERR_INDEX";
+    case QMM_ERR_WORKSPACE: return "QMM_ERR_WORKSPACE";
+    }
+    return "QMM_ERR_UNKNOWN";
+}
+
+uint64_t qmm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *qmm_last_error(void) { return t_last_error.c_str(); }
+
+int qmm_version(void) { return 100; }
+
+}  // extern "C"

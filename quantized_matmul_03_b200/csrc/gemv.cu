@@ -1,0 +1,271 @@
+// gemv.cu -- SIMT quantized matmul for few activation rows (decode shapes).
+//
+// y = x @ W^T (transpose, W stored [N, K]) or y = x @ W (W stored [K, N]),
+// W = scale * q + bias group-wise along W's last stored axis (mlx-rs
+// ops/quantization.rs, quantized_matmul; Emily.Quantization.Layers,
+// quantized_dense for the two layouts).  The packed weight is streamed once;
+// nothing dense is written back.
+//
+// gemv_t (transpose):  a warp owns RW weight rows; its lanes stride the row's
+//   packed words (128-byte coalesced warp loads) against activations staged in
+//   shared memory chunk by chunk along K, accumulate in fp32 registers and
+//   finish with a warp-shuffle reduction.
+// gemv_n (no transpose): a lane owns one packed word column (32/bits output
+//   features); the K range is split across the CTA's warps and across the
+//   CTAs of a thread-block cluster, and the partial sums are reduced through
+//   shared memory and then distributed shared memory.
+#include <algorithm>
+
+#include <cooperative_groups.h>
+
+#include "qmm_internal.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace qmm {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+// ---------------------------------------------------------------------------
+// transpose = true
+// ---------------------------------------------------------------------------
+template <typename T, int BITS, int MT, int RW>
+__global__ void __launch_bounds__(kThreads)
+gemv_t_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
+              const T *__restrict__ scales, const T *__restrict__ biases,
+              T *__restrict__ y, int M, int64_t N, int64_t K, int group_size, int kc) {
+    constexpr int EPW = 32 / BITS;
+    constexpr uint32_t MASK = (1u << BITS) - 1u;
+    extern __shared__ float xs[];  // [MT][kc]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row0 = (int64_t)blockIdx.x * (kWarps * RW) + (int64_t)warp * RW;
+    const int64_t wpr = K / EPW;          // packed words per weight row
+    const int64_t gpr = K / group_size;   // groups per weight row
+
+    float acc[RW][MT];
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
+
+    for (int64_t k0 = 0; k0 < K; k0 += kc) {
+        const int klen = (int)min((int64_t)kc, K - k0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < MT * klen; i += kThreads) {
+            const int m = i / klen, kk = i - m * klen;
+            xs[m * kc + kk] = (m < M) ? Dt<T>::to_f(x[(int64_t)m * K + k0 + kk]) : 0.f;
+        }
+        __syncthreads();
+        const int wlen = klen / EPW;
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+            const int64_t row = row0 + r;
+            if (row >= N) break;  // warp-uniform
+            const uint32_t *wr = wq + row * wpr + k0 / EPW;
+            for (int j = lane; j < wlen; j += 32) {
+                const uint32_t pk = __ldg(wr + j);
+                const int64_t g = (k0 + (int64_t)j * EPW) / group_size;
+                const float s = Dt<T>::to_f(scales[row * gpr + g]);
+                const float b = Dt<T>::to_f(biases[row * gpr + g]);
+#pragma unroll
+                for (int e = 0; e < EPW; ++e) {
+                    const float wv = __fmaf_rn(s, (float)((pk >> (e * BITS)) & MASK), b);
+#pragma unroll
+                    for (int m = 0; m < MT; ++m)
+                        acc[r][m] = __fmaf_rn(xs[m * kc + j * EPW + e], wv, acc[r][m]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < RW; ++r) {
+        const int64_t row = row0 + r;
+        if (row >= N) break;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const float v = warp_sum(acc[r][m]);
+            if (lane == 0 && m < M) y[(int64_t)m * N + row] = Dt<T>::from_f(v);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// transpose = false: W stored [K, N], groups run along N.
+// ---------------------------------------------------------------------------
+template <typename T, int BITS, int MT>
+__global__ void __launch_bounds__(kThreads)
+gemv_n_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
+              const T *__restrict__ scales, const T *__restrict__ biases,
+              T *__restrict__ y, int M, int64_t N, int64_t K, int group_size, int64_t k_split) {
+    constexpr int EPW = 32 / BITS;
+    constexpr uint32_t MASK = (1u << BITS) - 1u;
+    constexpr int NE = EPW * MT;           // partial sums per lane
+    __shared__ float red[kWarps][NE][32];  // per-warp partials
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t wpr = N / EPW;            // packed words per weight row
+    const int64_t gpr = N / group_size;
+    const int64_t col = (int64_t)blockIdx.x * 32 + lane;  // packed word column
+    const bool col_ok = col < wpr;
+    const int64_t kbeg = (int64_t)blockIdx.y * k_split;
+    const int64_t kend = min(K, kbeg + k_split);
+
+    float acc[NE];
+#pragma unroll
+    for (int i = 0; i < NE; ++i) acc[i] = 0.f;
+
+    if (col_ok) {
+        const int64_t g = col * EPW / group_size;
+        for (int64_t k = kbeg + warp; k < kend; k += kWarps) {
+            const uint32_t pk = __ldg(wq + k * wpr + col);
+            const float s = Dt<T>::to_f(scales[k * gpr + g]);
+            const float b = Dt<T>::to_f(biases[k * gpr + g]);
+            float xv[MT];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) xv[m] = (m < M) ? Dt<T>::to_f(x[(int64_t)m * K + k]) : 0.f;
+#pragma unroll
+            for (int e = 0; e < EPW; ++e) {
+                const float wv = __fmaf_rn(s, (float)((pk >> (e * BITS)) & MASK), b);
+#pragma unroll
+                for (int m = 0; m < MT; ++m) acc[e * MT + m] = __fmaf_rn(xv[m], wv, acc[e * MT + m]);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NE; ++i) red[warp][i][lane] = acc[i];
+    __syncthreads();
+    // Sum the warps' partials into warp 0's slot.
+    for (int i = threadIdx.x; i < NE * 32; i += kThreads) {
+        const int e = i >> 5, l = i & 31;
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) v += red[w][e][l];
+        red[0][e][l] = v;
+    }
+    // Sum across the cluster's CTAs (the K splits) via distributed shared memory.
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int nrank = (int)cluster.num_blocks();
+    const int rank = (int)cluster.block_rank();
+    for (int i = rank * kThreads + threadIdx.x; i < NE * 32; i += nrank * kThreads) {
+        const int e = i >> 5, l = i & 31;
+        float v = 0.f;
+        for (int q = 0; q < nrank; ++q) v += cluster.map_shared_rank(&red[0][0][0], q)[e * 32 + l];
+        const int64_t c = (int64_t)blockIdx.x * 32 + l;
+        const int ei = e / MT, m = e - ei * MT;
+        if (c < wpr && m < M) y[(int64_t)m * N + c * EPW + ei] = Dt<T>::from_f(v);
+    }
+    cluster.sync();
+}
+
+template <typename T, int BITS, int MT>
+cudaError_t run_gemv_t(const QmmArgs &a, int M, const T *x, T *y, cudaStream_t s) {
+    constexpr int RW = 2;
+    const int64_t rows_per_cta = kWarps * RW;
+    const int64_t grid = (a.N + rows_per_cta - 1) / rows_per_cta;
+    // Activation chunk: at most 48 KB of fp32, a multiple of 128 elements.
+    int kc = (int)std::min<int64_t>(a.K, (48 * 1024 / 4) / MT);
+    kc = (kc / 128) * 128;
+    if (kc <= 0) kc = 128;
+    if (kc > a.K) kc = (int)a.K;
+    const size_t smem = (size_t)MT * kc * sizeof(float);
+    gemv_t_kernel<T, BITS, MT, RW><<<grid, kThreads, smem, s>>>(
+        x, a.wq, static_cast<const T *>(a.scales), static_cast<const T *>(a.biases), y, M,
+        a.N, a.K, a.group_size, kc);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+template <typename T, int BITS, int MT>
+cudaError_t run_gemv_n(const QmmArgs &a, int M, const T *x, T *y, cudaStream_t s) {
+    constexpr int EPW = 32 / BITS;
+    const int64_t wpr = a.N / EPW;
+    const int gx = (int)((wpr + 31) / 32);
+    // Split K over a cluster of up to 8 CTAs so that small-N problems still
+    // fill the GPU; each split is at least 64 rows of W.
+    int ks = 8;
+    while (ks > 1 && (int64_t)gx * ks > 4LL * num_sms()) ks >>= 1;
+    while (ks > 1 && a.K / ks < 64) ks >>= 1;
+    const int64_t k_split = (a.K + ks - 1) / ks;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(gx, ks, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = ks;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    count_launches(1);
+    return cudaLaunchKernelEx(&cfg, gemv_n_kernel<T, BITS, MT>, x, a.wq,
+                              static_cast<const T *>(a.scales), static_cast<const T *>(a.biases),
+                              y, M, a.N, a.K, a.group_size, k_split);
+}
+
+// Largest activation tile per launch: gemv_t keeps RW*MT accumulators per
+// lane; gemv_n keeps (32/bits)*MT, capped at 32 (so MT <= bits).
+template <typename T, int BITS>
+cudaError_t gemv_bits(const QmmArgs &a, cudaStream_t s) {
+    const T *x = static_cast<const T *>(a.x);
+    T *y = static_cast<T *>(a.y);
+    const int tile = a.transpose ? 16 : BITS;
+    for (int64_t m0 = 0; m0 < a.M; m0 += tile) {
+        const int mt = (int)std::min<int64_t>(tile, a.M - m0);
+        const T *xm = x + m0 * a.K;
+        T *ym = y + m0 * a.N;
+        cudaError_t e;
+        if (a.transpose) {
+            if (mt == 1) e = run_gemv_t<T, BITS, 1>(a, mt, xm, ym, s);
+            else if (mt == 2) e = run_gemv_t<T, BITS, 2>(a, mt, xm, ym, s);
+            else if (mt <= 4) e = run_gemv_t<T, BITS, 4>(a, mt, xm, ym, s);
+            else if (mt <= 8) e = run_gemv_t<T, BITS, 8>(a, mt, xm, ym, s);
+            else e = run_gemv_t<T, BITS, 16>(a, mt, xm, ym, s);
+        } else {
+            if (mt == 1) e = run_gemv_n<T, BITS, 1>(a, mt, xm, ym, s);
+            else if (mt == 2) e = run_gemv_n<T, BITS, 2>(a, mt, xm, ym, s);
+            else if constexpr (BITS >= 4) {
+                if (mt <= 4) e = run_gemv_n<T, BITS, 4>(a, mt, xm, ym, s);
+                else if constexpr (BITS >= 8) e = run_gemv_n<T, BITS, 8>(a, mt, xm, ym, s);
+                else e = cudaErrorInvalidValue;
+            } else {
+                e = cudaErrorInvalidValue;
+            }
+        }
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+template <typename T>
+cudaError_t gemv_t_dtype(const QmmArgs &a, cudaStream_t s) {
+    switch (a.bits) {
+    case 2: return gemv_bits<T, 2>(a, s);
+    case 4: return gemv_bits<T, 4>(a, s);
+    default: return gemv_bits<T, 8>(a, s);
+    }
+}
+
+}  // namespace
+
+bool gemv_supported(qmm_dtype, const QmmArgs &) { return true; }
+
+cudaError_t launch_gemv(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
+    if (a.M == 0 || a.N == 0) return cudaSuccess;
+    switch (dt) {
+    case QMM_F32: return gemv_t_dtype<float>(a, s);
+    case QMM_BF16: return gemv_t_dtype<__nv_bfloat16>(a, s);
+    default: return gemv_t_dtype<__half>(a, s);
+    }
+}
+
+}  // namespace qmm

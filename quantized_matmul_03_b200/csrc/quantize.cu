@@ -1,0 +1,184 @@
+// quantize.cu -- group-wise affine quantize and dequantize (sm_100a).
+//
+// Quantization runs along the last axis, one scale and one bias per
+// `group_size` consecutive elements, `bits`-bit codes packed 32/bits per
+// uint32 least-significant first (EMLX.Quantization, section quantize;
+// Emily.QuantizedWeight, section Layout; mlx-rs ops/quantization.rs,
+// quantize / dequantize).
+//
+// Both kernels are HBM-bound streams: one thread per packed word, 16-byte
+// vector loads and stores, and the group min/max reduced across the
+// group_size/(32/bits) lanes that share a group with warp shuffles.  Every
+// floating-point step uses an explicitly rounded intrinsic so the result is
+// bit-identical to a sequential IEEE fp32 evaluation of the same rule.
+#include "qmm_internal.cuh"
+
+namespace qmm {
+
+namespace {
+
+template <typename T, int N>
+__device__ __forceinline__ void load_elems(const T *__restrict__ p, float (&v)[N]) {
+    constexpr int BYTES = N * (int)sizeof(T);
+    if constexpr (BYTES % 16 == 0) {
+        constexpr int NV = BYTES / 16;
+        uint4 raw[NV];
+#pragma unroll
+        for (int i = 0; i < NV; ++i) raw[i] = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+        const T *t = reinterpret_cast<const T *>(raw);
+#pragma unroll
+        for (int i = 0; i < N; ++i) v[i] = Dt<T>::to_f(t[i]);
+    } else {
+        static_assert(BYTES == 8, "unexpected vector width");
+        uint2 raw = __ldg(reinterpret_cast<const uint2 *>(p));
+        const T *t = reinterpret_cast<const T *>(&raw);
+#pragma unroll
+        for (int i = 0; i < N; ++i) v[i] = Dt<T>::to_f(t[i]);
+    }
+}
+
+template <typename T, int N>
+__device__ __forceinline__ void store_elems(T *__restrict__ p, const T (&t)[N]) {
+    constexpr int BYTES = N * (int)sizeof(T);
+    if constexpr (BYTES % 16 == 0) {
+        constexpr int NV = BYTES / 16;
+#pragma unroll
+        for (int i = 0; i < NV; ++i)
+            reinterpret_cast<uint4 *>(p)[i] = reinterpret_cast<const uint4 *>(t)[i];
+    } else {
+        static_assert(BYTES == 8, "unexpected vector width");
+        *reinterpret_cast<uint2 *>(p) = *reinterpret_cast<const uint2 *>(t);
+    }
+}
+
+// One thread per packed word; `tpg` = words per group (a power of two <= 32),
+// so the lanes of one group are contiguous and aligned within the warp.
+template <typename T, int BITS>
+__global__ void __launch_bounds__(256)
+quantize_kernel(const T *__restrict__ w, int64_t n_words, int tpg,
+                uint32_t *__restrict__ wq, T *__restrict__ scales, T *__restrict__ biases) {
+    constexpr int EPW = 32 / BITS;
+    constexpr int QMAX = (1 << BITS) - 1;
+    const int64_t word = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool valid = word < n_words;
+
+    float v[EPW];
+    if (valid) {
+        load_elems<T, EPW>(w + word * EPW, v);
+    } else {
+#pragma unroll
+        for (int j = 0; j < EPW; ++j) v[j] = 0.f;
+    }
+    float lo = v[0], hi = v[0];
+#pragma unroll
+    for (int j = 1; j < EPW; ++j) {
+        lo = fminf(lo, v[j]);
+        hi = fmaxf(hi, v[j]);
+    }
+    // Invalid lanes form whole groups (n_words is a multiple of tpg), and the
+    // xor partners of a lane stay inside its own group.
+    for (int off = tpg >> 1; off > 0; off >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (!valid) return;
+
+    const float scale32 = __fdiv_rn(__fsub_rn(hi, lo), (float)QMAX);
+    const T s_t = Dt<T>::from_f(scale32);
+    const T b_t = Dt<T>::from_f(lo);
+    const float s = Dt<T>::to_f(s_t);
+    const float b = Dt<T>::to_f(b_t);
+
+    uint32_t packed = 0;
+    if (s != 0.f) {
+#pragma unroll
+        for (int j = 0; j < EPW; ++j) {
+            int q = __float2int_rn(__fdiv_rn(__fsub_rn(v[j], b), s));
+            q = min(max(q, 0), QMAX);
+            packed |= (uint32_t)q << (j * BITS);
+        }
+    }
+    wq[word] = packed;
+    if ((threadIdx.x & (tpg - 1)) == 0) {
+        const int64_t g = word / tpg;
+        scales[g] = s_t;
+        biases[g] = b_t;
+    }
+}
+
+template <typename T, int BITS>
+__global__ void __launch_bounds__(256)
+dequantize_kernel(const uint32_t *__restrict__ wq, const T *__restrict__ scales,
+                  const T *__restrict__ biases, int64_t n_words, int tpg, T *__restrict__ out) {
+    constexpr int EPW = 32 / BITS;
+    constexpr uint32_t MASK = (1u << BITS) - 1u;
+    const int64_t word = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (word >= n_words) return;
+    const int64_t g = word / tpg;
+    const float s = Dt<T>::to_f(scales[g]);
+    const float b = Dt<T>::to_f(biases[g]);
+    const uint32_t packed = __ldg(wq + word);
+    T o[EPW];
+#pragma unroll
+    for (int j = 0; j < EPW; ++j)
+        o[j] = Dt<T>::from_f(__fmaf_rn(s, (float)((packed >> (j * BITS)) & MASK), b));
+    store_elems<T, EPW>(out + word * EPW, o);
+}
+
+template <typename T>
+cudaError_t quantize_t(const QuantArgs &a, cudaStream_t s) {
+    const int epw = 32 / a.bits;
+    const int64_t n_words = a.rows * (a.cols / epw);
+    const int tpg = a.group_size / epw;
+    const int64_t blocks = (n_words + 255) / 256;
+    auto w = static_cast<const T *>(a.w);
+    auto sc = static_cast<T *>(a.scales);
+    auto bi = static_cast<T *>(a.biases);
+    switch (a.bits) {
+    case 2: quantize_kernel<T, 2><<<blocks, 256, 0, s>>>(w, n_words, tpg, a.wq, sc, bi); break;
+    case 4: quantize_kernel<T, 4><<<blocks, 256, 0, s>>>(w, n_words, tpg, a.wq, sc, bi); break;
+    default: quantize_kernel<T, 8><<<blocks, 256, 0, s>>>(w, n_words, tpg, a.wq, sc, bi); break;
+    }
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t dequantize_t(const DequantArgs &a, cudaStream_t s) {
+    const int epw = 32 / a.bits;
+    const int64_t n_words = a.rows * (a.cols / epw);
+    const int tpg = a.group_size / epw;
+    const int64_t blocks = (n_words + 255) / 256;
+    auto sc = static_cast<const T *>(a.scales);
+    auto bi = static_cast<const T *>(a.biases);
+    auto out = static_cast<T *>(a.out);
+    switch (a.bits) {
+    case 2: dequantize_kernel<T, 2><<<blocks, 256, 0, s>>>(a.wq, sc, bi, n_words, tpg, out); break;
+    case 4: dequantize_kernel<T, 4><<<blocks, 256, 0, s>>>(a.wq, sc, bi, n_words, tpg, out); break;
+    default: dequantize_kernel<T, 8><<<blocks, 256, 0, s>>>(a.wq, sc, bi, n_words, tpg, out); break;
+    }
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(qmm_dtype dt, const QuantArgs &a, cudaStream_t s) {
+    if (a.rows == 0) return cudaSuccess;
+    switch (dt) {
+    case QMM_F32: return quantize_t<float>(a, s);
+    case QMM_BF16: return quantize_t<__nv_bfloat16>(a, s);
+    default: return quantize_t<__half>(a, s);
+    }
+}
+
+cudaError_t launch_dequantize(qmm_dtype dt, const DequantArgs &a, cudaStream_t s) {
+    if (a.rows == 0) return cudaSuccess;
+    switch (dt) {
+    case QMM_F32: return dequantize_t<float>(a, s);
+    case QMM_BF16: return dequantize_t<__nv_bfloat16>(a, s);
+    default: return dequantize_t<__half>(a, s);
+    }
+}
+
+}  // namespace qmm

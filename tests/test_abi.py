@@ -1,0 +1,98 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+declared in include/qmm.h, and rejects invalid arguments before launching."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+from quantized_matmul_03_b200 import binding
+
+HEADER = Path(__file__).resolve().parents[1] / "include" / "qmm.h"
+
+
+@pytest.fixture(scope="module")
+def L():
+    from quantized_matmul_03_b200 import build
+    build.build()
+    return binding.lib()
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qmm_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("qmm_quantize", "qmm_dequantize", "qmm_quantized_matmul", "qmm_gather_qmm",
+              "qmm_gather_qmm_workspace_size", "qmm_status_string", "qmm_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_function(L):
+    missing = [n for n in declared_functions() if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_status_strings(L):
+    for code, name in binding.STATUS_NAMES.items():
+        assert L.qmm_status_string(code).decode() == name
+    assert L.qmm_version() >= 100
+
+
+FAKE = ctypes.c_void_p(0x10000)        # aligned, never dereferenced: calls fail first
+MISALIGNED = ctypes.c_void_p(0x10004)
+NULL = ctypes.c_void_p(0)
+
+
+def q(L, **kw):
+    a = dict(w=FAKE, dtype=1, rows=4, cols=128, gs=64, bits=4, mode=b"affine",
+             wq=FAKE, s=FAKE, b=FAKE)
+    a.update(kw)
+    return L.qmm_quantize(a["w"], a["dtype"], a["rows"], a["cols"], a["gs"], a["bits"],
+                          a["mode"], a["wq"], a["s"], a["b"], NULL)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(bits=3), 2), (dict(bits=6), 2), (dict(bits=5), 1), (dict(bits=16), 1),
+    (dict(gs=48), 1), (dict(gs=16), 1), (dict(cols=96), 1), (dict(cols=0), 1),
+    (dict(rows=-1), 1), (dict(mode=b"nvfp4"), 2), (dict(mode=b"mxfp4"), 2),
+    (dict(mode=b"mxfp8"), 2), (dict(mode=b"bogus"), 1), (dict(dtype=7), 1),
+    (dict(w=NULL), 1), (dict(wq=MISALIGNED), 1), (dict(b=NULL), 1),
+])
+def test_quantize_rejects_before_launch(L, kw, status):
+    assert q(L, **kw) == status
+    assert L.qmm_last_error()
+
+
+def test_quantize_zero_rows_is_a_noop(L):
+    assert q(L, rows=0, w=NULL, wq=NULL, s=NULL, b=NULL) == 0
+
+
+def mm(L, **kw):
+    a = dict(x=FAKE, M=2, K=128, wq=FAKE, s=FAKE, b=FAKE, dtype=1, N=64, tr=1, gs=64,
+             bits=4, mode=None, y=FAKE)
+    a.update(kw)
+    return L.qmm_quantized_matmul(a["x"], a["M"], a["K"], a["wq"], a["s"], a["b"], a["dtype"],
+                                  a["N"], a["tr"], a["gs"], a["bits"], a["mode"], a["y"], NULL)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(K=96), 1), (dict(tr=0, N=96), 1), (dict(K=0), 1), (dict(M=-1), 1),
+    (dict(b=NULL), 1), (dict(x=MISALIGNED), 1), (dict(y=NULL), 1),
+    (dict(mode=b"nvfp4"), 2), (dict(bits=3), 2), (dict(gs=256), 1),
+])
+def test_matmul_rejects_before_launch(L, kw, status):
+    assert mm(L, **kw) == status
+
+
+def test_matmul_empty_is_a_noop(L):
+    assert mm(L, M=0, x=NULL, y=NULL) == 0
+    assert mm(L, N=0, x=NULL, y=NULL) == 0
+
+
+def test_set_path(L):
+    assert L.qmm_set_path(7) == 1
+    assert L.qmm_set_path(0) == 0

@@ -1,0 +1,86 @@
+"""GPU parity: quantized_matmul against the oracle's dequantize-then-float64
+product, on every kernel path that can run the case."""
+import pytest
+import torch
+
+import oracle
+from parity import REL_TOL, row_rel_err
+from quantized_matmul_03_b200 import binding as qb
+from quantized_matmul_03_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _reset_path():
+    yield
+    qb.qmm_set_path("auto")
+
+
+def run_case(x, w, gs, bits, transpose, path="auto"):
+    """Quantize w with the oracle (so both sides share packed inputs), run the
+    GPU product on `path` and compare with the oracle's product."""
+    wq, s, b = oracle.quantize(w, gs, bits)
+    ref = oracle.quantized_matmul(x, wq, s, b, transpose, gs, bits)
+    qb.qmm_set_path(path)
+    y = qb.qmm_quantized_matmul(x.cuda(), wq.cuda(), s.cuda(), b.cuda(), transpose, gs, bits)
+    torch.cuda.synchronize()
+    assert y.shape == ref.shape and y.dtype == s.dtype
+    err = row_rel_err(y, ref)
+    assert err <= REL_TOL[s.dtype], f"rel err {err}"
+    return err
+
+
+def test_tiny_f32_case():
+    c = wl.tiny_case()
+    run_case(c.x, c.w, c.group_size, c.bits, c.transpose, "gemv")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32])
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("gs", [32, 64, 128])
+@pytest.mark.parametrize("transpose", [True, False])
+@pytest.mark.parametrize("m", [1, 3, 16])
+def test_gemv_small(dtype, bits, gs, transpose, m):
+    # W stored [rows, cols]; groups along cols.  Ragged rows (not a multiple of
+    # any tile) and a K that spans several chunks.
+    rows, cols = (200, 1024) if transpose else (384, 640)
+    w = wl.with_outliers((rows, cols), seed=bits * 7 + gs, dtype=dtype)
+    k = cols if transpose else rows
+    x = wl.normal((m, k), seed=m + 5, dtype=dtype)
+    run_case(x, w, gs, bits, transpose, "gemv")
+
+
+@pytest.mark.parametrize("transpose", [True, False])
+def test_gemv_m_larger_than_tile(transpose):
+    w = wl.normal((96, 256), 3, 0.02, torch.bfloat16)
+    x = wl.normal((37, 256 if transpose else 96), 4, 1.0, torch.bfloat16)
+    run_case(x, w, 64, 4, transpose, "gemv")
+
+
+def test_mlx_rs_quantized_matmul_restated():
+    """mlx-rs unit test test_quantized_matmul: m=32, n=k=128, gs 64, 4 bits,
+    x and w ~ N(0,1)/sqrt(k), w stored [k, n], transpose=False; |y - x@w_hat| < 1e-3."""
+    m, n, k = 32, 128, 128
+    x = wl.normal((m, k), 0).float() / k ** 0.5
+    w = wl.normal((k, n), 1).float() / k ** 0.5
+    wq, s, b = oracle.quantize(w, 64, 4)
+    w_hat = oracle.dequantize(wq, s, b, 64, 4)
+    y = qb.qmm_quantized_matmul(x.cuda(), wq.cuda(), s.cuda(), b.cuda(), False, 64, 4)
+    torch.cuda.synchronize()
+    assert (y.cpu() - x @ w_hat).abs().max().item() < 1e-3
+
+
+def test_empty_problems_are_noops():
+    wq, s, b = oracle.quantize(wl.normal((64, 128), 1, 1.0, torch.bfloat16), 64, 4)
+    x = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    y = qb.qmm_quantized_matmul(x, wq.cuda(), s.cuda(), b.cuda(), True, 64, 4)
+    assert y.shape == (0, 64)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("m", [1, 4, 8, 16])
+def test_decode_full_size(m):
+    """x bf16 [m, 4096] against W [14336, 4096] int4 gs64 (the decode workload)."""
+    c = wl.decode_case(m)
+    run_case(c.x, c.w, c.group_size, c.bits, c.transpose)

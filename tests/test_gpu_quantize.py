@@ -1,0 +1,72 @@
+"""GPU parity: quantize and dequantize are bit-exact against the oracle."""
+import pytest
+import torch
+
+import oracle
+from parity import words
+from quantized_matmul_03_b200 import binding as qb
+from quantized_matmul_03_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+DTYPES = [torch.float32, torch.bfloat16, torch.float16]
+
+
+def check_quantize(w_cpu, gs, bits):
+    wq, s, b = qb.qmm_quantize(w_cpu.cuda(), gs, bits)
+    torch.cuda.synchronize()
+    rq, rs, rb = oracle.quantize(w_cpu, gs, bits)
+    assert torch.equal(words(wq), words(rq))
+    assert torch.equal(s.cpu(), rs)
+    assert torch.equal(b.cpu(), rb)
+    d = qb.qmm_dequantize(wq, s, b, gs, bits)
+    torch.cuda.synchronize()
+    assert torch.equal(d.cpu(), oracle.dequantize(rq, rs, rb, gs, bits))
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("gs", [32, 64, 128])
+def test_quantize_dequantize_bit_exact(dtype, bits, gs):
+    # 37 rows x 640 cols: several thread blocks and a ragged last block.
+    w = wl.with_outliers((37, 640), seed=100 + bits + gs, dtype=dtype)
+    check_quantize(w, gs, bits)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_quantize_rank3_and_minimal_row(bits):
+    check_quantize(wl.normal((3, 5, 128), 7, 1.0, torch.bfloat16), 64, bits)
+    check_quantize(wl.normal((1, 32), 8, 1.0, torch.float32), 32, bits)
+
+
+def test_quantize_degenerate_and_iota():
+    w = torch.zeros((4, 128), dtype=torch.bfloat16)
+    w[1] = 3.5
+    w[2, 5] = -1.0
+    check_quantize(w, 64, 4)
+    check_quantize(wl.iota((4, 64)), 64, 4)
+    check_quantize(wl.iota((4, 128)), 64, 4)
+
+
+def test_quantize_empty_rows():
+    w = torch.empty((0, 128), dtype=torch.bfloat16, device="cuda")
+    wq, s, b = qb.qmm_quantize(w, 64, 4)
+    assert wq.shape == (0, 16) and s.shape == (0, 2)
+
+
+@pytest.mark.slow
+def test_quantize_full_decode_weight():
+    """The 14336 x 4096 bf16 weight of the decode/prefill workloads, int4 and int8."""
+    w = wl.normal((14336, 4096), 1, 0.02, torch.bfloat16)
+    for bits in (4, 8):
+        check_quantize(w, 64, bits)
+
+
+def test_invalid_args_raise():
+    w = torch.zeros((4, 96), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(qb.QmmError) as e:
+        qb.qmm_quantize(w, 64, 4)
+    assert e.value.status == 1
+    with pytest.raises(qb.QmmError) as e:
+        qb.qmm_quantize(w, 32, 4, mode="nvfp4")
+    assert e.value.status == 2
