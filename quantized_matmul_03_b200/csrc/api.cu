@@ -190,6 +190,8 @@ qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K, const uint3
         QmmArgs a{x, wq, scales, biases, y, M, N, K, group_size, bits, transpose != 0};
         if (g_path == QMM_PATH_GEMM)
             return fail(QMM_ERR_UNSUPPORTED, "the tensor-core path is not available");
+        if (gemv_fast_supported(dtype, a))
+            return finish_launch(launch_gemv_fast(dtype, a, (cudaStream_t)stream), "gemv launch");
         return finish_launch(launch_gemv(dtype, a, (cudaStream_t)stream), "gemv launch");
     } catch (...) {
         return fail(QMM_ERR_CUDA, "unexpected exception in qmm_quantized_matmul");

@@ -73,6 +73,8 @@ struct QmmArgs {
 };
 cudaError_t launch_gemv(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 bool gemv_supported(qmm_dtype dt, const QmmArgs &a);
+cudaError_t launch_gemv_fast(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
+bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a);
 
 int num_sms();
 void count_launches(int n);  // bump the process-wide launch counter
