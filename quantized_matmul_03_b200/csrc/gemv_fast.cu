@@ -136,8 +136,11 @@ qgemv_t_fast_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     __shared__ float red[kWarps][RB];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // The block holds whole teams only (blockDim.x = teams * TW * 32); a warp
+    // outside every team would wait at a team barrier nobody else reaches.
+    const int teams_per_cta = (int)(blockDim.x >> 5) / TW;
+    if (warp >= teams_per_cta * TW) return;
     const int team = warp / TW, wt = warp - team * TW;
-    const int teams_per_cta = kWarps / TW;
     const int gteam = blockIdx.x * teams_per_cta + team;
     const int row0 = gteam * rows_per_team;
     const int nrows = max(0, min(rows_per_team, N - row0));
@@ -284,16 +287,17 @@ cudaError_t launch_fast(const QmmArgs &a, cudaStream_t s) {
     const int spr = (int)(a.K / PK::EPU);
     const int TW = (spr + 32 * UPL - 1) / (32 * UPL);
     auto kern = qgemv_t_fast_kernel<T, BITS, UPL, P, RB, VAR>;
+    const int teams_per_cta = kWarps / TW;          // TW <= kWarps (checked by the caller)
+    const int threads = teams_per_cta * TW * 32;    // whole teams only
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
     if (e != cudaSuccess) return e;
     per_sm = std::max(per_sm, 1);
-    const int teams_per_cta = kWarps / TW;
     const int64_t teams = (int64_t)num_sms() * per_sm * teams_per_cta;
     const int rows_per_team = (int)((a.N + teams - 1) / teams);
     const int64_t need_teams = (a.N + rows_per_team - 1) / rows_per_team;
     const int grid = (int)((need_teams + teams_per_cta - 1) / teams_per_cta);
-    kern<<<grid, kThreads, 0, s>>>(static_cast<const T *>(a.x), a.wq, static_cast<const T *>(a.scales),
+    kern<<<grid, threads, 0, s>>>(static_cast<const T *>(a.x), a.wq, static_cast<const T *>(a.scales),
                                     static_cast<const T *>(a.biases), static_cast<T *>(a.y),
                                     (int)a.N, (int)a.K, a.group_size, TW, rows_per_team);
     count_launches(1);
@@ -304,7 +308,7 @@ template <typename T, int BITS>
 cudaError_t fast_bits(const QmmArgs &a, cudaStream_t s) {
     using PK = Pack<BITS>;
     const int spr = (int)(a.K / PK::EPU);
-    const bool two = g_upl == 2 || (g_upl == 0 && spr > 32 * 8);  // keep TW <= 8
+    const bool two = g_upl == 2 || spr > 32 * 8;  // keep TW <= 8
     if constexpr (BITS == 4 && std::is_same<T, __nv_bfloat16>::value) {
         if (g_var == 1) return two ? launch_fast<T, BITS, 2, 1>(a, s) : launch_fast<T, BITS, 1, 1>(a, s);
     }
