@@ -1,115 +1,81 @@
-// gemv_fast.cu -- HBM-streaming quantized GEMV for one activation row
-// (decode), transpose layout: y[n] = sum_k x[k] * (s[n,g] * q[n,k] + b[n,g]),
-// W stored [N, K] (mlx-rs ops/quantization.rs, quantized_matmul;
+// gemv_fast.cu -- HBM-streaming quantized GEMV for 1..4 activation rows
+// (decode), transpose layout:  y[m, n] = sum_k x[m, k] * (s[n,g] q[n,k] + b[n,g])
+// with W stored [N, K] (mlx-rs ops/quantization.rs, quantized_matmul;
 // Emily.Quantization.Layers, quantized_dense with transpose: true).
 //
-// The weight is read exactly once, in 16-byte slices.  A "team" of TW warps
-// covers one weight row: lane l of team-warp w owns the same UPL consecutive
-// slices of every row it visits, so the activation values it multiplies are
-// loaded once into registers and never re-read.  Per group the product is
-// factored as  s * sum(x*q) + b * sum(x):  codes become bf16/f16 values with
-// one LOP3 per pair (magic-exponent trick: OR-ing a code into the mantissa of
-// 128.0 (bf16) / 1024.0 (f16) gives OFF + q exactly), multiplied into fp32
-// accumulators, and the OFF * sum(x) term is folded into the bias.  Each lane
-// keeps one partial per row for a batch of RB rows and the warp reduces them
-// all at once with a butterfly reduce-scatter; the team's warps then combine
-// through shared memory.  Rows are split evenly over a persistent grid of
-// teams and loads run P rows ahead of the arithmetic.
+// Memory side.  Each CTA owns a contiguous block of weight rows, which is one
+// contiguous byte range of the packed weight (and of the scales and biases).
+// A producer warp streams it through a ring of shared-memory stages with 1-D
+// bulk copies (cp.async.bulk) completing on mbarriers, so ~100 KB per SM are in
+// flight regardless of register pressure.  The weight is read exactly once.
+//
+// Arithmetic side.  A team of TW consumer warps covers one weight row; lane l
+// owns the same 16-byte slice(s) of every row, so its activations live in
+// registers for the whole kernel.  Per group the product is factored as
+//   s * sum(x q) + b * sum(x).
+// For sum(x q) a code is masked, in place, into the mantissa of an fp16 word
+// whose exponent bits are zero: the word IS the subnormal number q * 2^-24 *
+// 2^p (p = the code's bit offset inside its 16-bit half), exactly.  One AND
+// therefore yields two codes as an fp16x2 operand, and one HFMA2 multiplies
+// them by activations pre-scaled by 2^(sh - p) (sh per lane and row, chosen
+// so the largest |x| maps into [2^14, 2^15)).  Products are exact to 2^-12;
+// a slice's 16 products per half are summed in fp16, then converted and
+// scaled back to fp32.  Lane partials for a stage's rows are combined by a
+// butterfly reduce-scatter and shared-memory atomics; results leave as one
+// coalesced store per CTA.
 #include <algorithm>
 #include <cstdlib>
 #include <type_traits>
 
+#include <cuda_fp16.h>
+
+#include "ptx_sm100.cuh"
 #include "qmm_internal.cuh"
 
 namespace qmm {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+constexpr int kCW = 8;                    // consumer warps
+constexpr int kThreads = 32 * (kCW + 1);  // plus one producer warp
 
-__device__ __forceinline__ uint4 ldg_stream(const void *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
+// Codes of step E of a packed word, masked in place (see the header comment).
+// Step E yields element E (low half) and element E + 16/BITS (high half).
+template <int BITS, int E>
+__device__ __forceinline__ uint32_t sub_codes(uint32_t w) {
+    if constexpr (BITS == 4) {
+        constexpr uint32_t m = (E & 1) ? 0x00F000F0u : 0x000F000Fu;
+        return ((E < 2) ? w : (w >> 8)) & m;
+    } else if constexpr (BITS == 2) {
+        constexpr int p = (E < 5) ? E : E - 5;
+        constexpr uint32_t m = 0x00030003u << (2 * p);
+        return ((E < 5) ? w : (w >> 10)) & m;
+    } else {
+        return ((E == 0) ? w : (w >> 8)) & 0x00FF00FFu;
+    }
+}
+// log2 of the place value of step e's codes inside their 16-bit half.
+template <int BITS>
+__host__ __device__ constexpr int sub_pw(int e) {
+    return BITS == 4 ? (e & 1) * 4 : (BITS == 2 ? 2 * (e < 5 ? e : e - 5) : 0);
 }
 
-__device__ __forceinline__ uint16_t ldg_u16(const void *p) {
-    uint16_t v;
-    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
-    return v;
+template <int BITS, int E = 0>
+__device__ __forceinline__ void dot_word(uint32_t w, const __half2 *xp, __half2 &acc) {
+    constexpr int STEPS = 16 / BITS;
+    if constexpr (E < STEPS) {
+        const uint32_t t = sub_codes<BITS, E>(w);
+        acc = __hfma2(xp[E], *reinterpret_cast<const __half2 *>(&t), acc);
+        dot_word<BITS, E + 1>(w, xp, acc);
+    }
 }
 
-// 16-bit storage type traits for the fast path.
-template <typename T> struct Half16;
-template <> struct Half16<__nv_bfloat16> {
-    static constexpr uint32_t MAGIC = 0x43004300u;  // bf16 128.0 | 128.0
-    static constexpr float OFF = 128.f;
-    static __device__ __forceinline__ float to_f(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
-    // acc_lo += lo(x) * lo(t); acc_hi += hi(x) * hi(t), products exact in fp32.
-    static __device__ __forceinline__ void fma2(float &lo, float &hi, uint32_t xp, uint32_t t) {
-        asm("{.reg .b16 xl, xh, tl, th;\n\t"
-            "mov.b32 {xl, xh}, %2;\n\t"
-            "mov.b32 {tl, th}, %3;\n\t"
-            "fma.rn.f32.bf16 %0, xl, tl, %0;\n\t"
-            "fma.rn.f32.bf16 %1, xh, th, %1;\n\t}"
-            : "+f"(lo), "+f"(hi)
-            : "r"(xp), "r"(t));
-    }
-};
-template <> struct Half16<__half> {
-    static constexpr uint32_t MAGIC = 0x64006400u;  // f16 1024.0 | 1024.0
-    static constexpr float OFF = 1024.f;
-    static __device__ __forceinline__ float to_f(uint16_t h) {
-        return __half2float(__ushort_as_half(h));
-    }
-    static __device__ __forceinline__ void fma2(float &lo, float &hi, uint32_t xp, uint32_t t) {
-        asm("{.reg .b16 xl, xh, tl, th;\n\t"
-            "mov.b32 {xl, xh}, %2;\n\t"
-            "mov.b32 {tl, th}, %3;\n\t"
-            "fma.rn.f32.f16 %0, xl, tl, %0;\n\t"
-            "fma.rn.f32.f16 %1, xh, th, %1;\n\t}"
-            : "+f"(lo), "+f"(hi)
-            : "r"(xp), "r"(t));
-    }
-};
-
-// Alternative inner step: unpack both halves to fp32 and use the packed
-// fp32x2 FMA.  Selected by VAR == 1.
-template <typename T>
-__device__ __forceinline__ void fma2_f32x2(float &lo, float &hi, float2 xf, uint32_t t);
-template <>
-__device__ __forceinline__ void fma2_f32x2<__nv_bfloat16>(float &lo, float &hi, float2 xf, uint32_t t) {
-    float2 q = make_float2(__uint_as_float(t << 16), __uint_as_float(t & 0xffff0000u));
-    float2 a = __ffma2_rn(xf, q, make_float2(lo, hi));
-    lo = a.x;
-    hi = a.y;
-}
-
-// Codes per 16-byte slice, and the pairing of codes produced by one LOP3:
-//   bits 4: word w, step e (0..3) -> codes (8w+e, 8w+e+4)
-//   bits 2: word w, step e (0..7) -> codes (16w+e, 16w+e+8)
-//   bits 8: word w, step e (0..1) -> codes (4w+e, 4w+e+2)   (f16 only)
-template <int BITS> struct Pack {
-    static constexpr int EPW = 32 / BITS;           // codes per word
-    static constexpr int EPU = 4 * EPW;             // codes per slice
-    static constexpr int STEPS = EPW / 2;           // LOP3 steps per word
-    static constexpr uint32_t MASK = BITS == 8 ? 0x00FF00FFu : (BITS == 4 ? 0x000F000Fu : 0x00030003u);
-};
-
-// Reduce v[0..RB) across the warp; afterwards lane l (l < RB) holds the warp
-// sum of everyone's v[l] in v[0].  Butterfly reduce-scatter: log2(32) rounds,
-// each halving the live slots.
-template <int RB>
-__device__ __forceinline__ float reduce_scatter(float (&v)[RB], int lane) {
-    static_assert(RB == 32 || RB == 16, "batch of 16 or 32 rows");
-    if constexpr (RB == 16) {
+// Sum v[0..V) over the 32 lanes; afterwards lane l holds the total of index
+// (l mod V).  Butterfly halving over lane bits below V, then xor-reduction
+// over the remaining lane bits.
+template <int V>
+__device__ __forceinline__ float reduce_scatter(float (&v)[V], int lane) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] += __shfl_xor_sync(0xffffffffu, v[j], 16);
-    }
-#pragma unroll
-    for (int s = RB / 2; s >= 1; s >>= 1) {
+    for (int s = V / 2; s >= 1; s >>= 1) {
         const bool upper = (lane & s) != 0;
 #pragma unroll
         for (int j = 0; j < s; ++j) {
@@ -118,230 +84,290 @@ __device__ __forceinline__ float reduce_scatter(float (&v)[RB], int lane) {
             v[j] = keep + __shfl_xor_sync(0xffffffffu, send, s);
         }
     }
-    return v[0];
+    float r = v[0];
+#pragma unroll
+    for (int s = V; s < 32; s <<= 1) r += __shfl_xor_sync(0xffffffffu, r, s);
+    return r;
 }
 
-template <typename T, int BITS, int UPL, int P, int RB, int VAR>
-__global__ void __launch_bounds__(kThreads, 2)
-qgemv_t_fast_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
+__device__ __forceinline__ float h16_to_f(uint16_t h, bool is_bf16) {
+    return is_bf16 ? __uint_as_float((uint32_t)h << 16) : __half2float(__ushort_as_half(h));
+}
+
+template <typename T, int BITS, int MR, int UPL, int RPT>
+__global__ void __launch_bounds__(kThreads, 1)
+qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     const T *__restrict__ scales, const T *__restrict__ biases,
-                    T *__restrict__ y, int N, int K, int group_size, int TW, int rows_per_team) {
-    using H = Half16<T>;
-    using PK = Pack<BITS>;
-    constexpr int EPU = PK::EPU;
-    constexpr int NX = 4 * PK::STEPS;  // packed x pairs per slice (= EPU / 2)
-    static_assert(BITS != 8 || VAR == 0, "8-bit codes use the f16 magic only");
-    static_assert(P == 1 || P == 2 || P == 4, "prefetch depth must divide the row batch");
+                    T *__restrict__ y, int M, int N, int K, int group_size, int rpc, int S,
+                    int TW, int *err) {
+    constexpr int EPW = 32 / BITS;       // codes per word
+    constexpr int EPU = 4 * EPW;         // codes per 16-byte slice
+    constexpr int STEPS = EPW / 2;       // code pairs per word
+    constexpr int V = MR * RPT;          // partials per lane per stage
+    constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+    static_assert((V & (V - 1)) == 0 && V <= 32, "V must be a power of two <= 32");
 
-    __shared__ float red[kWarps][RB];
-
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int NT = kCW / TW;                 // teams; warps past NT*TW only pace the ring
+    const int SR = NT * RPT;                 // rows per stage
+    const int row_bytes = K / 8 * BITS;
+    const int gpr = K / group_size;
+    const int sb_bytes = gpr * 2;
+    const int stage_bytes = SR * (row_bytes + 2 * sb_bytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)S * stage_bytes);
+    float *ysm = reinterpret_cast<float *>(bars + 2 * S);
+    const int r0 = blockIdx.x * rpc;
+    const int nrows = max(0, min(rpc, N - r0));
+    const int nst = (nrows + SR - 1) / SR;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // The block holds whole teams only (blockDim.x = teams * TW * 32); a warp
-    // outside every team would wait at a team barrier nobody else reaches.
-    const int teams_per_cta = (int)(blockDim.x >> 5) / TW;
-    if (warp >= teams_per_cta * TW) return;
-    const int team = warp / TW, wt = warp - team * TW;
-    const int gteam = blockIdx.x * teams_per_cta + team;
-    const int row0 = gteam * rows_per_team;
-    const int nrows = max(0, min(rows_per_team, N - row0));
-    const int spr = K / EPU;                 // slices per row
-    const int gpr = K / group_size;          // groups per row
-    const int64_t row_words = (int64_t)K / PK::EPW;
+    const uint32_t full0 = ptx::smem_addr(bars), empty0 = ptx::smem_addr(bars + S);
 
-    // ---- this lane's slices and their activations ------------------------
-    int sl[UPL];
-    bool sv[UPL];
-    uint32_t xp[UPL][NX];     // x pairs matching the LOP3 code pairing
-    float2 xf[UPL][VAR == 1 ? NX : 1];
-    float xs[UPL];            // sum of x over the slice
-    int gi[UPL];              // group of the slice
-#pragma unroll
-    for (int u = 0; u < UPL; ++u) {
-        sl[u] = (wt * 32 + lane) * UPL + u;
-        sv[u] = sl[u] < spr;
-        gi[u] = sv[u] ? (sl[u] * EPU) / group_size : 0;
-        xs[u] = 0.f;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            // EPW x values of word w: EPW*2 bytes = (EPW/8) uint4
-            uint32_t raw[PK::EPW / 2];
-            const T *xw = x + (int64_t)sl[u] * EPU + w * PK::EPW;
-            if constexpr (PK::EPW == 4) {
-                uint2 v = sv[u] ? *reinterpret_cast<const uint2 *>(xw) : make_uint2(0, 0);
-                raw[0] = v.x; raw[1] = v.y;
-            } else {
-#pragma unroll
-                for (int c = 0; c < PK::EPW / 8; ++c) {
-                    uint4 v = sv[u] ? *reinterpret_cast<const uint4 *>(xw + c * 8) : make_uint4(0, 0, 0, 0);
-                    raw[4 * c + 0] = v.x; raw[4 * c + 1] = v.y; raw[4 * c + 2] = v.z; raw[4 * c + 3] = v.w;
-                }
-            }
-            // pair e: codes (e, e + EPW/2) of this word
-#pragma unroll
-            for (int e = 0; e < PK::STEPS; ++e) {
-                const int a = e, b = e + PK::EPW / 2;  // element indices within the word
-                const uint32_t ra = raw[a >> 1], rb = raw[b >> 1];
-                const uint32_t lo = (a & 1) ? (ra >> 16) : (ra & 0xffffu);
-                const uint32_t hi = (b & 1) ? (rb & 0xffff0000u) : (rb << 16);
-                xp[u][w * PK::STEPS + e] = lo | hi;
-                const float fa = H::to_f((uint16_t)lo), fb = H::to_f((uint16_t)(hi >> 16));
-                if constexpr (VAR == 1) xf[u][w * PK::STEPS + e] = make_float2(fa, fb);
-                xs[u] += fa + fb;
+    for (int i = threadIdx.x; i < MR * rpc; i += kThreads) ysm[i] = 0.f;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(full0 + 8 * s, 1);
+            ptx::mbar_init(empty0 + 8 * s, kCW);
+        }
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(wq) + (int64_t)r0 * row_bytes;
+            const uint8_t *ssrc = reinterpret_cast<const uint8_t *>(scales) + (int64_t)r0 * sb_bytes;
+            const uint8_t *bsrc = reinterpret_cast<const uint8_t *>(biases) + (int64_t)r0 * sb_bytes;
+            for (int i = 0; i < nst; ++i) {
+                const int s = i % S;
+                if (i >= S) ptx::mbar_wait(empty0 + 8 * s, ((i / S) + 1) & 1, err);
+                const int nr = min(SR, nrows - i * SR);
+                const uint32_t wb = (uint32_t)(nr * row_bytes), sb = (uint32_t)(nr * sb_bytes);
+                const uint32_t st = ptx::smem_addr(smem + (size_t)s * stage_bytes);
+                const uint32_t bar = full0 + 8 * s;
+                ptx::mbar_arrive_expect_tx(bar, wb + 2 * sb);
+                const int64_t roff = (int64_t)i * SR;
+                ptx::bulk_g2s(st, wsrc + roff * row_bytes, wb, bar);
+                ptx::bulk_g2s(st + SR * row_bytes, ssrc + roff * sb_bytes, sb, bar);
+                ptx::bulk_g2s(st + SR * row_bytes + SR * sb_bytes, bsrc + roff * sb_bytes, sb, bar);
             }
         }
-    }
+    } else {
+        // ---------------- consumers ----------------
+        const int cw = warp - 1;
+        const int team = cw / TW, wt = cw - team * TW;
+        const bool active = team < NT;
+        const int spr = K / EPU;
 
-    // ---- software pipeline over this team's rows ------------------------
-    uint4 wb[P][UPL];
-    uint16_t sb[P][UPL], bb[P][UPL];
-    auto load_row = [&](int p, int r) {
-        const int64_t row = row0 + r;
-        const uint32_t *wr = wq + row * row_words;
+        int sl[UPL];
+        bool sv[UPL];
+        int gi[UPL];
 #pragma unroll
         for (int u = 0; u < UPL; ++u) {
-            if (sv[u]) {
-                wb[p][u] = ldg_stream(wr + (int64_t)sl[u] * 4);
-                sb[p][u] = ldg_u16(scales + row * gpr + gi[u]);
-                bb[p][u] = ldg_u16(biases + row * gpr + gi[u]);
-            } else {
-                wb[p][u] = make_uint4(0, 0, 0, 0);
-                sb[p][u] = 0;
-                bb[p][u] = 0;
+            sl[u] = (wt * 32 + lane) * UPL + u;
+            sv[u] = active && sl[u] < spr;
+            gi[u] = sv[u] ? (sl[u] * EPU) / group_size : 0;
+        }
+
+        // Activations: scaled fp16 pairs, per-slice sums, per-row scale-back.
+        __half2 xp[MR][UPL][4 * STEPS];
+        float xsum[MR][UPL];
+        float inv[MR];
+#pragma unroll
+        for (int m = 0; m < MR; ++m) {
+            float xv[UPL][EPU];
+            float amax = 0.f;
+#pragma unroll
+            for (int u = 0; u < UPL; ++u) {
+                const bool ok = sv[u] && m < M;
+#pragma unroll
+                for (int c = 0; c < EPU / 8; ++c) {
+                    uint4 raw = ok ? *reinterpret_cast<const uint4 *>(
+                                         x + (int64_t)m * K + (int64_t)sl[u] * EPU + 8 * c)
+                                   : make_uint4(0, 0, 0, 0);
+                    const uint16_t *h = reinterpret_cast<const uint16_t *>(&raw);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        xv[u][8 * c + q] = h16_to_f(h[q], kBF16);
+                        amax = fmaxf(amax, fabsf(xv[u][8 * c + q]));
+                    }
+                }
+            }
+            int ex = 0;
+            frexpf(amax, &ex);                       // amax in [2^(ex-1), 2^ex)
+            const int sh = amax > 0.f ? min(100, max(-100, 15 - ex)) : 0;
+            inv[m] = ldexpf(1.f, 24 - sh);
+#pragma unroll
+            for (int u = 0; u < UPL; ++u) {
+                float sum = 0.f;
+#pragma unroll
+                for (int wd = 0; wd < 4; ++wd) {
+#pragma unroll
+                    for (int e = 0; e < STEPS; ++e) {
+                        const float a = xv[u][wd * EPW + e];
+                        const float b = xv[u][wd * EPW + e + EPW / 2];
+                        const int pw = sh - sub_pw<BITS>(e);
+                        xp[m][u][wd * STEPS + e] =
+                            __floats2half2_rn(ldexpf(a, pw), ldexpf(b, pw));
+                        sum += a + b;
+                    }
+                }
+                xsum[m][u] = sum;
             }
         }
-    };
-#pragma unroll
-    for (int p = 0; p < P; ++p)
-        if (p < nrows) load_row(p, p);
 
-    const int nbatch = (nrows + RB - 1) / RB;
-    for (int bt = 0; bt < nbatch; ++bt) {
-        float part[RB];
+        for (int i = 0; i < nst; ++i) {
+            const int s = i % S;
+            ptx::mbar_wait(full0 + 8 * s, (i / S) & 1, err);
+            const uint8_t *st = smem + (size_t)s * stage_bytes;
+            float part[V];
 #pragma unroll
-        for (int j = 0; j < RB; ++j) {
-            const int r = bt * RB + j;
-            float acc = 0.f;
-            if (r < nrows) {
-                const int p = j % P;
+            for (int q = 0; q < V; ++q) part[q] = 0.f;
+#pragma unroll
+            for (int j = 0; j < RPT; ++j) {
+                const int jr = team + j * NT;               // row within the stage
+                if (!active || i * SR + jr >= nrows) continue;
 #pragma unroll
                 for (int u = 0; u < UPL; ++u) {
-                    float lo = 0.f, hi = 0.f;
-                    const uint32_t wv[4] = {wb[p][u].x, wb[p][u].y, wb[p][u].z, wb[p][u].w};
+                    if (!sv[u]) continue;
+                    const uint4 wv = *reinterpret_cast<const uint4 *>(st + jr * row_bytes + sl[u] * 16);
+                    const uint16_t sr = *reinterpret_cast<const uint16_t *>(
+                        st + SR * row_bytes + jr * sb_bytes + gi[u] * 2);
+                    const uint16_t br = *reinterpret_cast<const uint16_t *>(
+                        st + SR * row_bytes + SR * sb_bytes + jr * sb_bytes + gi[u] * 2);
+                    const float sc = h16_to_f(sr, kBF16), bi = h16_to_f(br, kBF16);
 #pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-#pragma unroll
-                        for (int e = 0; e < PK::STEPS; ++e) {
-                            const uint32_t t = ((wv[w] >> (BITS * e)) & PK::MASK) | H::MAGIC;
-                            if constexpr (VAR == 1)
-                                fma2_f32x2<T>(lo, hi, xf[u][w * PK::STEPS + e], t);
-                            else
-                                H::fma2(lo, hi, xp[u][w * PK::STEPS + e], t);
-                        }
+                    for (int m = 0; m < MR; ++m) {
+                        __half2 acc = __float2half2_rn(0.f);
+                        dot_word<BITS>(wv.x, &xp[m][u][0 * STEPS], acc);
+                        dot_word<BITS>(wv.y, &xp[m][u][1 * STEPS], acc);
+                        dot_word<BITS>(wv.z, &xp[m][u][2 * STEPS], acc);
+                        dot_word<BITS>(wv.w, &xp[m][u][3 * STEPS], acc);
+                        const float2 a = __half22float2(acc);
+                        part[m * RPT + j] = __fmaf_rn(sc * inv[m], a.x + a.y,
+                                                      __fmaf_rn(bi, xsum[m][u], part[m * RPT + j]));
                     }
-                    const float s = H::to_f(sb[p][u]);
-                    const float b = H::to_f(bb[p][u]);
-                    // s * sum(x*(OFF+q)) + (b - OFF*s) * sum(x)
-                    acc = __fmaf_rn(s, lo + hi, acc);
-                    acc = __fmaf_rn(__fmaf_rn(-H::OFF, s, b), xs[u], acc);
                 }
-                if (r + P < nrows) load_row(p, r + P);
             }
-            part[j] = acc;
-        }
-        const float v = reduce_scatter<RB>(part, lane);
-        // Combine the team's warps: lane l holds this warp's sum for row bt*RB + l.
-        if (lane < RB) red[warp][lane] = v;
-        if (TW > 1) {
-            asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(TW * 32) : "memory");
-        } else {
             __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(empty0 + 8 * s);
+            const float v = reduce_scatter<V>(part, lane);
+            if (active && lane < V) {
+                const int m = lane / RPT, j = lane - m * RPT;
+                const int r = i * SR + team + j * NT;
+                if (m < M && r < nrows) atomicAdd(&ysm[m * rpc + r], v);
+            }
         }
-        if (wt == 0 && lane < RB) {
-            float tot = 0.f;
-            for (int q = 0; q < TW; ++q) tot += red[team * TW + q][lane];
-            const int r = bt * RB + lane;
-            if (r < nrows) y[row0 + r] = Dt<T>::from_f(tot);
-        }
-        if (TW > 1) {
-            asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(TW * 32) : "memory");
-        } else {
-            __syncwarp();
-        }
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < M * nrows; idx += kThreads) {
+        const int m = idx / nrows, r = idx - m * nrows;
+        y[(int64_t)m * N + r0 + r] = Dt<T>::from_f(ysm[m * rpc + r]);
     }
 }
 
-// Inner-loop variant and slices per lane.  Defaults are the measured best;
-// QMM_GEMV_VAR / QMM_GEMV_UPL override them for experiments.
-int env_int(const char *name, int dflt) {
-    const char *v = getenv(name);
-    return v ? atoi(v) : dflt;
-}
-int g_var = env_int("QMM_GEMV_VAR", 0);
-int g_upl = env_int("QMM_GEMV_UPL", 0);  // 0 = auto
+struct StreamPlan {
+    int upl, tw, rpt, sr, stages, rpc, grid;
+    size_t smem;
+};
 
-template <typename T, int BITS, int UPL, int VAR>
-cudaError_t launch_fast(const QmmArgs &a, cudaStream_t s) {
-    using PK = Pack<BITS>;
-    constexpr int P = 4;
-    constexpr int RB = 32;
-    const int spr = (int)(a.K / PK::EPU);
-    const int TW = (spr + 32 * UPL - 1) / (32 * UPL);
-    auto kern = qgemv_t_fast_kernel<T, BITS, UPL, P, RB, VAR>;
-    const int teams_per_cta = kWarps / TW;          // TW <= kWarps (checked by the caller)
-    const int threads = teams_per_cta * TW * 32;    // whole teams only
-    int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
+constexpr size_t kSmemBudget = 200 * 1024;
+
+int rows_per_team_stage(int mr) { return mr == 4 ? 2 : 4; }
+
+bool plan_stream(const QmmArgs &a, int mr, StreamPlan &p) {
+    const int bits = a.bits;
+    const int epu = 128 / bits;
+    const int64_t spr = a.K / epu;
+    p.upl = spr > 32 * kCW ? 2 : 1;
+    p.tw = (int)((spr + 32 * p.upl - 1) / (32 * p.upl));
+    if (p.tw > kCW) return false;
+    const int nt = kCW / p.tw;
+    p.rpt = rows_per_team_stage(mr);
+    p.sr = nt * p.rpt;
+    const int64_t row_bytes = a.K / 8 * bits;
+    const int64_t sb_bytes = a.K / a.group_size * 2;
+    const int64_t stage = (int64_t)p.sr * (row_bytes + 2 * sb_bytes);
+    const int sms = num_sms();
+    int64_t rpc = (a.N + sms - 1) / sms;
+    rpc = std::min<int64_t>(rpc, 4096 / mr);
+    rpc = std::max<int64_t>(rpc, 1);
+    p.rpc = (int)rpc;
+    p.grid = (int)((a.N + rpc - 1) / rpc);
+    const size_t fixed = 16 * 8 + (size_t)mr * p.rpc * 4 + 128;
+    if ((size_t)stage * 2 + fixed > kSmemBudget) return false;
+    p.stages = (int)std::min<int64_t>(8, (int64_t)((kSmemBudget - fixed) / stage));
+    p.smem = (size_t)p.stages * stage + (size_t)2 * p.stages * 8 + (size_t)mr * p.rpc * 4;
+    return p.stages >= 2;
+}
+
+template <typename T, int BITS, int MR, int UPL>
+cudaError_t launch_stream(const QmmArgs &a, const StreamPlan &p, cudaStream_t s) {
+    constexpr int RPT = MR == 4 ? 2 : 4;
+    auto kern = qgemv_stream_kernel<T, BITS, MR, UPL, RPT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)p.smem);
     if (e != cudaSuccess) return e;
-    per_sm = std::max(per_sm, 1);
-    const int64_t teams = (int64_t)num_sms() * per_sm * teams_per_cta;
-    const int rows_per_team = (int)((a.N + teams - 1) / teams);
-    const int64_t need_teams = (a.N + rows_per_team - 1) / rows_per_team;
-    const int grid = (int)((need_teams + teams_per_cta - 1) / teams_per_cta);
-    kern<<<grid, threads, 0, s>>>(static_cast<const T *>(a.x), a.wq, static_cast<const T *>(a.scales),
-                                    static_cast<const T *>(a.biases), static_cast<T *>(a.y),
-                                    (int)a.N, (int)a.K, a.group_size, TW, rows_per_team);
+    kern<<<p.grid, kThreads, p.smem, s>>>(
+        static_cast<const T *>(a.x), a.wq, static_cast<const T *>(a.scales),
+        static_cast<const T *>(a.biases), static_cast<T *>(a.y), (int)a.M, (int)a.N, (int)a.K,
+        a.group_size, p.rpc, p.stages, p.tw, device_error_word());
     count_launches(1);
     return cudaGetLastError();
 }
 
 template <typename T, int BITS>
-cudaError_t fast_bits(const QmmArgs &a, cudaStream_t s) {
-    using PK = Pack<BITS>;
-    const int spr = (int)(a.K / PK::EPU);
-    const bool two = g_upl == 2 || spr > 32 * 8;  // keep TW <= 8
-    if constexpr (BITS == 4 && std::is_same<T, __nv_bfloat16>::value) {
-        if (g_var == 1) return two ? launch_fast<T, BITS, 2, 1>(a, s) : launch_fast<T, BITS, 1, 1>(a, s);
+cudaError_t stream_bits(const QmmArgs &a, cudaStream_t s) {
+    const int mr = a.M == 1 ? 1 : (a.M == 2 ? 2 : 4);
+    StreamPlan p;
+    if (!plan_stream(a, mr, p)) return cudaErrorInvalidValue;
+    // Register-heavy combinations (2-bit codes with several rows, or four
+    // rows with two slices per lane) are not instantiated: they would spill,
+    // and gemv_fast_supported() sends them to the general kernel.
+    if (mr == 1) return p.upl == 1 ? launch_stream<T, BITS, 1, 1>(a, p, s)
+                                   : launch_stream<T, BITS, 1, 2>(a, p, s);
+    if constexpr (BITS != 2) {
+        if (mr == 2) return p.upl == 1 ? launch_stream<T, BITS, 2, 1>(a, p, s)
+                                       : launch_stream<T, BITS, 2, 2>(a, p, s);
+        if (p.upl == 1) return launch_stream<T, BITS, 4, 1>(a, p, s);
     }
-    return two ? launch_fast<T, BITS, 2, 0>(a, s) : launch_fast<T, BITS, 1, 0>(a, s);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-// The fast path takes one activation row of a bf16/f16 problem in the
-// transpose layout, whole 16-byte slices per row, one group per slice at
-// least (group_size >= codes per slice), and a team of at most 8 warps.
+// Fast path: bf16/f16, transpose layout, 1..4 rows, whole 16-byte slices per
+// row, scales/biases rows of whole 16-byte units, no group boundary inside a
+// slice (group_size >= codes per slice), rows at most 8 warps wide.
 bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a) {
-    if (!a.transpose || a.M != 1) return false;
-    if (dt == QMM_F32) return false;
-    if (dt == QMM_BF16 && a.bits == 8) return false;  // no exact bf16 magic for 8-bit codes
+    if (!a.transpose || a.M < 1 || a.M > 4) return false;
+    if (dt != QMM_BF16 && dt != QMM_F16) return false;
     const int epu = 128 / a.bits;
     if (a.K % epu != 0 || a.group_size < epu) return false;
-    if (a.K > (int64_t)epu * 32 * 2 * kWarps) return false;
-    if (a.N > INT32_MAX || a.K > INT32_MAX) return false;
-    return true;
+    if ((a.K / a.group_size) % 8 != 0) return false;
+    if (a.N > (1 << 30) || a.K > (1 << 24)) return false;
+    if ((reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases) |
+         reinterpret_cast<uintptr_t>(a.wq)) & 15)
+        return false;
+    const int mr = a.M == 1 ? 1 : (a.M == 2 ? 2 : 4);
+    if (a.bits == 2 && mr > 1) return false;
+    StreamPlan p;
+    if (!plan_stream(a, mr, p)) return false;
+    return !(mr == 4 && p.upl == 2);
 }
 
 cudaError_t launch_gemv_fast(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
     if (dt == QMM_BF16) {
         switch (a.bits) {
-        case 2: return fast_bits<__nv_bfloat16, 2>(a, s);
-        default: return fast_bits<__nv_bfloat16, 4>(a, s);
+        case 2: return stream_bits<__nv_bfloat16, 2>(a, s);
+        case 4: return stream_bits<__nv_bfloat16, 4>(a, s);
+        default: return stream_bits<__nv_bfloat16, 8>(a, s);
         }
     }
     switch (a.bits) {
-    case 2: return fast_bits<__half, 2>(a, s);
-    case 4: return fast_bits<__half, 4>(a, s);
-    default: return fast_bits<__half, 8>(a, s);
+    case 2: return stream_bits<__half, 2>(a, s);
+    case 4: return stream_bits<__half, 4>(a, s);
+    default: return stream_bits<__half, 8>(a, s);
     }
 }
 

@@ -89,14 +89,18 @@ def test_decode_full_size(m):
 @pytest.mark.parametrize("dtype,bits,gs", [
     (torch.bfloat16, 4, 32), (torch.bfloat16, 4, 64), (torch.bfloat16, 4, 128),
     (torch.bfloat16, 2, 64), (torch.bfloat16, 2, 128),
+    (torch.bfloat16, 8, 32), (torch.bfloat16, 8, 128),
     (torch.float16, 4, 64), (torch.float16, 8, 32), (torch.float16, 8, 128), (torch.float16, 2, 64),
 ])
-@pytest.mark.parametrize("n,k", [(1, 4096), (301, 4096), (77, 14336), (1000, 640), (4099, 1024)])
-def test_gemv_one_row(dtype, bits, gs, n, k):
-    """One activation row (the decode-shaped fast kernel): ragged N, K from one
-    slice per lane to teams of seven warps."""
+@pytest.mark.parametrize("n,k", [(1, 4096), (301, 4096), (77, 14336), (1000, 1024),
+                                 (4099, 1024), (150, 2048)])
+@pytest.mark.parametrize("m", [1, 2, 3, 4])
+def test_gemv_few_rows(dtype, bits, gs, n, k, m):
+    """1..4 activation rows (the decode-shaped streaming kernel where it
+    applies, the general kernel elsewhere): ragged N, K from one slice per
+    lane to teams of seven warps."""
     if k % gs:
         pytest.skip("K must be a multiple of the group size")
     w = wl.with_outliers((n, k), seed=n + k + bits, dtype=dtype)
-    x = wl.normal((1, k), seed=k, dtype=dtype)
+    x = wl.normal((m, k), seed=k + m, dtype=dtype)
     run_case(x, w, gs, bits, True)
