@@ -13,21 +13,20 @@
 // owns the same 16-byte slice(s) of every row, so its activations live in
 // registers for the whole kernel.  Per group the product is factored as
 //   s * sum(x q) + b * sum(x).
-// For sum(x q) a code is masked, in place, into the mantissa of an fp16 word
-// whose exponent bits are zero: the word IS the subnormal number q * 2^-24 *
-// 2^p (p = the code's bit offset inside its 16-bit half), exactly.  One AND
-// therefore yields two codes as an fp16x2 operand, and one HFMA2 multiplies
-// them by activations pre-scaled by 2^(sh - p) (sh per lane and row, chosen
-// so the largest |x| maps into [2^14, 2^15)).  Products are exact to 2^-12;
-// a slice's 16 products per half are summed in fp16, then converted and
-// scaled back to fp32.  Lane partials for a stage's rows are combined by a
-// butterfly reduce-scatter and shared-memory atomics; results leave as one
-// coalesced store per CTA.
+// For sum(x q) a code is masked, in place, into the low 23 bits of a 32-bit
+// word: with its exponent bits zero the word IS the fp32 subnormal
+// q * 2^p * 2^-149 exactly (p = the code's bit offset in the word; codes that
+// would touch bit 23 are taken from the word shifted right first).  So one AND
+// turns a code into an fp32 operand, and one packed FFMA2 multiplies two of
+// them by activations pre-scaled by 2^(sh - p) (sh per lane and row, chosen so
+// the largest |x| maps just below 2^127).  Products are exact normal fp32
+// numbers (8-bit x mantissa times a <= 8-bit code), accumulation is fp32, and
+// a slice's sum is scaled back by 2^(149 - sh).  Lane partials for a stage's
+// rows are combined by a butterfly reduce-scatter and shared-memory atomics;
+// results leave as one coalesced store per CTA.
 #include <algorithm>
 #include <cstdlib>
 #include <type_traits>
-
-#include <cuda_fp16.h>
 
 #include "ptx_sm100.cuh"
 #include "qmm_internal.cuh"
@@ -38,34 +37,33 @@ namespace {
 constexpr int kCW = 8;                    // consumer warps
 constexpr int kThreads = 32 * (kCW + 1);  // plus one producer warp
 
-// Codes of step E of a packed word, masked in place (see the header comment).
-// Step E yields element E (low half) and element E + 16/BITS (high half).
-template <int BITS, int E>
-__device__ __forceinline__ uint32_t sub_codes(uint32_t w) {
-    if constexpr (BITS == 4) {
-        constexpr uint32_t m = (E & 1) ? 0x00F000F0u : 0x000F000Fu;
-        return ((E < 2) ? w : (w >> 8)) & m;
-    } else if constexpr (BITS == 2) {
-        constexpr int p = (E < 5) ? E : E - 5;
-        constexpr uint32_t m = 0x00030003u << (2 * p);
-        return ((E < 5) ? w : (w >> 10)) & m;
-    } else {
-        return ((E == 0) ? w : (w >> 8)) & 0x00FF00FFu;
-    }
-}
-// log2 of the place value of step e's codes inside their 16-bit half.
+// Element I of a packed word as an fp32 subnormal bit pattern (see above).
+// Codes whose bits reach bit 23 or above are read from the word shifted right
+// by SHIFT and keep place value sub_pw<BITS>(I).
+template <int BITS> struct Sub {
+    static constexpr int EPW = 32 / BITS;
+    static constexpr int SHIFT = BITS == 4 ? 12 : (BITS == 2 ? 10 : 16);
+    // first element taken from the shifted word
+    static constexpr int SPLIT = BITS == 4 ? 5 : (BITS == 2 ? 11 : 2);
+};
 template <int BITS>
-__host__ __device__ constexpr int sub_pw(int e) {
-    return BITS == 4 ? (e & 1) * 4 : (BITS == 2 ? 2 * (e < 5 ? e : e - 5) : 0);
+__host__ __device__ constexpr int sub_pw(int i) {
+    return i < Sub<BITS>::SPLIT ? BITS * i : BITS * i - Sub<BITS>::SHIFT;
+}
+template <int BITS, int I>
+__device__ __forceinline__ float sub_code(uint32_t w, uint32_t ws) {
+    constexpr uint32_t mask = ((1u << BITS) - 1u) << sub_pw<BITS>(I);
+    return __uint_as_float((I < Sub<BITS>::SPLIT ? w : ws) & mask);
 }
 
-template <int BITS, int E = 0>
-__device__ __forceinline__ void dot_word(uint32_t w, const __half2 *xp, __half2 &acc) {
-    constexpr int STEPS = 16 / BITS;
-    if constexpr (E < STEPS) {
-        const uint32_t t = sub_codes<BITS, E>(w);
-        acc = __hfma2(xp[E], *reinterpret_cast<const __half2 *>(&t), acc);
-        dot_word<BITS, E + 1>(w, xp, acc);
+// acc += x'[2j] * code[2j] , x'[2j+1] * code[2j+1] for every pair of a word.
+template <int BITS, int J = 0>
+__device__ __forceinline__ void dot_word(uint32_t w, uint32_t ws, const float2 *xq, float2 &acc) {
+    constexpr int PAIRS = Sub<BITS>::EPW / 2;
+    if constexpr (J < PAIRS) {
+        const float2 t = make_float2(sub_code<BITS, 2 * J>(w, ws), sub_code<BITS, 2 * J + 1>(w, ws));
+        acc = __ffma2_rn(xq[J], t, acc);
+        dot_word<BITS, J + 1>(w, ws, xq, acc);
     }
 }
 
@@ -169,8 +167,8 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
             gi[u] = sv[u] ? (sl[u] * EPU) / group_size : 0;
         }
 
-        // Activations: scaled fp16 pairs, per-slice sums, per-row scale-back.
-        __half2 xp[MR][UPL][4 * STEPS];
+        // Activations: scaled fp32 pairs, per-slice sums, per-row scale-back.
+        float2 xq[MR][UPL][4 * STEPS];
         float xsum[MR][UPL];
         float inv[MR];
 #pragma unroll
@@ -193,22 +191,23 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     }
                 }
             }
+            // amax in [2^(ex-1), 2^ex): x * 2^sh stays below 2^127.  sh >= 22
+            // keeps the scale-back 2^(149 - sh) finite (|x| < 2^105).
             int ex = 0;
-            frexpf(amax, &ex);                       // amax in [2^(ex-1), 2^ex)
-            const int sh = amax > 0.f ? min(100, max(-100, 15 - ex)) : 0;
-            inv[m] = ldexpf(1.f, 24 - sh);
+            frexpf(amax, &ex);
+            const int sh = amax > 0.f ? max(22, 127 - ex) : 127;
+            inv[m] = ldexpf(1.f, 149 - sh);
 #pragma unroll
             for (int u = 0; u < UPL; ++u) {
                 float sum = 0.f;
 #pragma unroll
                 for (int wd = 0; wd < 4; ++wd) {
 #pragma unroll
-                    for (int e = 0; e < STEPS; ++e) {
-                        const float a = xv[u][wd * EPW + e];
-                        const float b = xv[u][wd * EPW + e + EPW / 2];
-                        const int pw = sh - sub_pw<BITS>(e);
-                        xp[m][u][wd * STEPS + e] =
-                            __floats2half2_rn(ldexpf(a, pw), ldexpf(b, pw));
+                    for (int j = 0; j < STEPS; ++j) {
+                        const float a = xv[u][wd * EPW + 2 * j];
+                        const float b = xv[u][wd * EPW + 2 * j + 1];
+                        xq[m][u][wd * STEPS + j] = make_float2(ldexpf(a, sh - sub_pw<BITS>(2 * j)),
+                                                               ldexpf(b, sh - sub_pw<BITS>(2 * j + 1)));
                         sum += a + b;
                     }
                 }
@@ -238,12 +237,12 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     const float sc = h16_to_f(sr, kBF16), bi = h16_to_f(br, kBF16);
 #pragma unroll
                     for (int m = 0; m < MR; ++m) {
-                        __half2 acc = __float2half2_rn(0.f);
-                        dot_word<BITS>(wv.x, &xp[m][u][0 * STEPS], acc);
-                        dot_word<BITS>(wv.y, &xp[m][u][1 * STEPS], acc);
-                        dot_word<BITS>(wv.z, &xp[m][u][2 * STEPS], acc);
-                        dot_word<BITS>(wv.w, &xp[m][u][3 * STEPS], acc);
-                        const float2 a = __half22float2(acc);
+                        float2 a = make_float2(0.f, 0.f);
+                        constexpr int SH = Sub<BITS>::SHIFT;
+                        dot_word<BITS>(wv.x, wv.x >> SH, &xq[m][u][0 * STEPS], a);
+                        dot_word<BITS>(wv.y, wv.y >> SH, &xq[m][u][1 * STEPS], a);
+                        dot_word<BITS>(wv.z, wv.z >> SH, &xq[m][u][2 * STEPS], a);
+                        dot_word<BITS>(wv.w, wv.w >> SH, &xq[m][u][3 * STEPS], a);
                         part[m * RPT + j] = __fmaf_rn(sc * inv[m], a.x + a.y,
                                                       __fmaf_rn(bi, xsum[m][u], part[m * RPT + j]));
                     }
@@ -301,6 +300,16 @@ bool plan_stream(const QmmArgs &a, int mr, StreamPlan &p) {
     return p.stages >= 2;
 }
 
+// Variants whose activations and partials fit the register file without
+// spilling (checked with ptxas -v): rows x slices per lane is bounded by the
+// codes per slice (32 for 4-bit, 16 for 8-bit, 64 for 2-bit).
+bool stream_variant_fits(int bits, int mr, int upl) {
+    if (mr == 1) return bits != 2 || upl == 1;
+    if (bits == 4) return mr == 2 && upl == 1;
+    if (bits == 8) return mr == 2 || upl == 1;
+    return false;
+}
+
 template <typename T, int BITS, int MR, int UPL>
 cudaError_t launch_stream(const QmmArgs &a, const StreamPlan &p, cudaStream_t s) {
     constexpr int RPT = MR == 4 ? 2 : 4;
@@ -321,15 +330,18 @@ cudaError_t stream_bits(const QmmArgs &a, cudaStream_t s) {
     const int mr = a.M == 1 ? 1 : (a.M == 2 ? 2 : 4);
     StreamPlan p;
     if (!plan_stream(a, mr, p)) return cudaErrorInvalidValue;
-    // Register-heavy combinations (2-bit codes with several rows, or four
-    // rows with two slices per lane) are not instantiated: they would spill,
-    // and gemv_fast_supported() sends them to the general kernel.
-    if (mr == 1) return p.upl == 1 ? launch_stream<T, BITS, 1, 1>(a, p, s)
-                                   : launch_stream<T, BITS, 1, 2>(a, p, s);
+    // Only the variants that fit in registers are instantiated; the others are
+    // refused by stream_variant_fits() and go to the general kernel.
+    if (mr == 1) {
+        if (p.upl == 1) return launch_stream<T, BITS, 1, 1>(a, p, s);
+        if constexpr (BITS != 2) return launch_stream<T, BITS, 1, 2>(a, p, s);
+    }
     if constexpr (BITS != 2) {
-        if (mr == 2) return p.upl == 1 ? launch_stream<T, BITS, 2, 1>(a, p, s)
-                                       : launch_stream<T, BITS, 2, 2>(a, p, s);
-        if (p.upl == 1) return launch_stream<T, BITS, 4, 1>(a, p, s);
+        if (mr == 2 && p.upl == 1) return launch_stream<T, BITS, 2, 1>(a, p, s);
+    }
+    if constexpr (BITS == 8) {
+        if (mr == 2) return launch_stream<T, BITS, 2, 2>(a, p, s);
+        if (mr == 4 && p.upl == 1) return launch_stream<T, BITS, 4, 1>(a, p, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -350,10 +362,9 @@ bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a) {
          reinterpret_cast<uintptr_t>(a.wq)) & 15)
         return false;
     const int mr = a.M == 1 ? 1 : (a.M == 2 ? 2 : 4);
-    if (a.bits == 2 && mr > 1) return false;
     StreamPlan p;
     if (!plan_stream(a, mr, p)) return false;
-    return !(mr == 4 && p.upl == 2);
+    return stream_variant_fits(a.bits, mr, p.upl);
 }
 
 cudaError_t launch_gemv_fast(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
