@@ -191,12 +191,16 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     }
                 }
             }
-            // amax in [2^(ex-1), 2^ex): x * 2^sh stays below 2^127.  sh >= 22
-            // keeps the scale-back 2^(149 - sh) finite (|x| < 2^105).
-            int ex = 0;
-            frexpf(amax, &ex);
-            const int sh = amax > 0.f ? max(22, 127 - ex) : 127;
-            inv[m] = ldexpf(1.f, 149 - sh);
+            // amax in [2^(ex-1), 2^ex) with ex = biased exponent - 126, so
+            // x * 2^sh stays below 2^127.  sh in [22, 191] keeps every power of
+            // two used here a normal float: x' = (x * 2^(sh-64)) * 2^(64-p)
+            // (the first product is below 2^63, the second below 2^127),
+            // scale-back 2^(149-sh).  (|x| < 2^105 is required; slices whose
+            // |x| are all below 2^-64 lose precision, negligibly.)
+            const int ex = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
+            const int sh = amax > 0.f ? min(191, max(22, 127 - ex)) : 127;
+            const float up = __uint_as_float((uint32_t)(sh + 63) << 23);   // 2^(sh-64)
+            inv[m] = __uint_as_float((uint32_t)(276 - sh) << 23);           // 2^(149-sh)
 #pragma unroll
             for (int u = 0; u < UPL; ++u) {
                 float sum = 0.f;
@@ -206,8 +210,10 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     for (int j = 0; j < STEPS; ++j) {
                         const float a = xv[u][wd * EPW + 2 * j];
                         const float b = xv[u][wd * EPW + 2 * j + 1];
-                        xq[m][u][wd * STEPS + j] = make_float2(ldexpf(a, sh - sub_pw<BITS>(2 * j)),
-                                                               ldexpf(b, sh - sub_pw<BITS>(2 * j + 1)));
+                        // 2^(64 - p) for the two codes' place values p
+                        const float ca = __uint_as_float((uint32_t)(191 - sub_pw<BITS>(2 * j)) << 23);
+                        const float cb = __uint_as_float((uint32_t)(191 - sub_pw<BITS>(2 * j + 1)) << 23);
+                        xq[m][u][wd * STEPS + j] = make_float2((a * up) * ca, (b * up) * cb);
                         sum += a + b;
                     }
                 }
@@ -270,11 +276,13 @@ struct StreamPlan {
     size_t smem;
 };
 
-constexpr size_t kSmemBudget = 200 * 1024;
+// Shared memory per CTA: the whole SM's worth (one CTA per SM) or half of it
+// (two CTAs per SM, which doubles the warps available to hide latency).
+constexpr size_t kSmemPerSm = 200 * 1024;
 
 int rows_per_team_stage(int mr) { return mr == 4 ? 2 : 4; }
 
-bool plan_stream(const QmmArgs &a, int mr, StreamPlan &p) {
+bool plan_stream(const QmmArgs &a, int mr, int ctas_per_sm, StreamPlan &p) {
     const int bits = a.bits;
     const int epu = 128 / bits;
     const int64_t spr = a.K / epu;
@@ -287,15 +295,16 @@ bool plan_stream(const QmmArgs &a, int mr, StreamPlan &p) {
     const int64_t row_bytes = a.K / 8 * bits;
     const int64_t sb_bytes = a.K / a.group_size * 2;
     const int64_t stage = (int64_t)p.sr * (row_bytes + 2 * sb_bytes);
-    const int sms = num_sms();
-    int64_t rpc = (a.N + sms - 1) / sms;
-    rpc = std::min<int64_t>(rpc, 4096 / mr);
+    const int64_t ctas = (int64_t)num_sms() * ctas_per_sm;
+    int64_t rpc = (a.N + ctas - 1) / ctas;
+    rpc = std::min<int64_t>(rpc, 2048 / mr);
     rpc = std::max<int64_t>(rpc, 1);
     p.rpc = (int)rpc;
     p.grid = (int)((a.N + rpc - 1) / rpc);
+    const size_t budget = kSmemPerSm / ctas_per_sm;
     const size_t fixed = 16 * 8 + (size_t)mr * p.rpc * 4 + 128;
-    if ((size_t)stage * 2 + fixed > kSmemBudget) return false;
-    p.stages = (int)std::min<int64_t>(8, (int64_t)((kSmemBudget - fixed) / stage));
+    if ((size_t)stage * 2 + fixed > budget) return false;
+    p.stages = (int)std::min<int64_t>(8, (int64_t)((budget - fixed) / stage));
     p.smem = (size_t)p.stages * stage + (size_t)2 * p.stages * 8 + (size_t)mr * p.rpc * 4;
     return p.stages >= 2;
 }
@@ -311,12 +320,22 @@ bool stream_variant_fits(int bits, int mr, int upl) {
 }
 
 template <typename T, int BITS, int MR, int UPL>
-cudaError_t launch_stream(const QmmArgs &a, const StreamPlan &p, cudaStream_t s) {
+cudaError_t launch_stream(const QmmArgs &a, cudaStream_t s) {
     constexpr int RPT = MR == 4 ? 2 : 4;
     auto kern = qgemv_stream_kernel<T, BITS, MR, UPL, RPT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)p.smem);
-    if (e != cudaSuccess) return e;
+    // Two CTAs per SM when the registers and the halved ring allow it.
+    StreamPlan p;
+    cudaError_t e = cudaSuccess;
+    for (int per_sm = 2; per_sm >= 1; --per_sm) {
+        if (!plan_stream(a, MR, per_sm, p)) continue;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+        if (e != cudaSuccess) return e;
+        int got = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&got, kern, kThreads, p.smem);
+        if (e != cudaSuccess) return e;
+        if (got >= per_sm) break;
+        if (per_sm == 1) return cudaErrorInvalidConfiguration;
+    }
     kern<<<p.grid, kThreads, p.smem, s>>>(
         static_cast<const T *>(a.x), a.wq, static_cast<const T *>(a.scales),
         static_cast<const T *>(a.biases), static_cast<T *>(a.y), (int)a.M, (int)a.N, (int)a.K,
@@ -329,19 +348,19 @@ template <typename T, int BITS>
 cudaError_t stream_bits(const QmmArgs &a, cudaStream_t s) {
     const int mr = a.M == 1 ? 1 : (a.M == 2 ? 2 : 4);
     StreamPlan p;
-    if (!plan_stream(a, mr, p)) return cudaErrorInvalidValue;
+    if (!plan_stream(a, mr, 1, p)) return cudaErrorInvalidValue;
     // Only the variants that fit in registers are instantiated; the others are
     // refused by stream_variant_fits() and go to the general kernel.
     if (mr == 1) {
-        if (p.upl == 1) return launch_stream<T, BITS, 1, 1>(a, p, s);
-        if constexpr (BITS != 2) return launch_stream<T, BITS, 1, 2>(a, p, s);
+        if (p.upl == 1) return launch_stream<T, BITS, 1, 1>(a, s);
+        if constexpr (BITS != 2) return launch_stream<T, BITS, 1, 2>(a, s);
     }
     if constexpr (BITS != 2) {
-        if (mr == 2 && p.upl == 1) return launch_stream<T, BITS, 2, 1>(a, p, s);
+        if (mr == 2 && p.upl == 1) return launch_stream<T, BITS, 2, 1>(a, s);
     }
     if constexpr (BITS == 8) {
-        if (mr == 2) return launch_stream<T, BITS, 2, 2>(a, p, s);
-        if (mr == 4 && p.upl == 1) return launch_stream<T, BITS, 4, 1>(a, p, s);
+        if (mr == 2) return launch_stream<T, BITS, 2, 2>(a, s);
+        if (mr == 4 && p.upl == 1) return launch_stream<T, BITS, 4, 1>(a, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -363,7 +382,7 @@ bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a) {
         return false;
     const int mr = a.M == 1 ? 1 : (a.M == 2 ? 2 : 4);
     StreamPlan p;
-    if (!plan_stream(a, mr, p)) return false;
+    if (!plan_stream(a, mr, 1, p)) return false;
     return stream_variant_fits(a.bits, mr, p.upl);
 }
 
