@@ -159,12 +159,13 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
 
         int sl[UPL];
         bool sv[UPL];
-        int gi[UPL];
+        int gi[UPL], soff[UPL];   // group index and byte offset of the slice (0 if unused)
 #pragma unroll
         for (int u = 0; u < UPL; ++u) {
             sl[u] = (wt * 32 + lane) * UPL + u;
             sv[u] = active && sl[u] < spr;
             gi[u] = sv[u] ? (sl[u] * EPU) / group_size : 0;
+            soff[u] = sv[u] ? sl[u] * 16 : 0;
         }
 
         // Activations: scaled fp32 pairs, per-slice sums, per-row scale-back.
@@ -228,29 +229,35 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
             float part[V];
 #pragma unroll
             for (int q = 0; q < V; ++q) part[q] = 0.f;
+            if (active) {
+                // All RPT rows are computed without branches so their FMA
+                // chains interleave; rows past the block's end read stale (but
+                // in-bounds) stage bytes and are dropped by the selects.
 #pragma unroll
-            for (int j = 0; j < RPT; ++j) {
-                const int jr = team + j * NT;               // row within the stage
-                if (!active || i * SR + jr >= nrows) continue;
+                for (int j = 0; j < RPT; ++j) {
+                    const int jr = team + j * NT;           // row within the stage (< SR)
+                    const bool rv = i * SR + jr < nrows;
+                    const uint8_t *wrow = st + jr * row_bytes;
+                    const uint8_t *srow = st + SR * row_bytes + jr * sb_bytes;
 #pragma unroll
-                for (int u = 0; u < UPL; ++u) {
-                    if (!sv[u]) continue;
-                    const uint4 wv = *reinterpret_cast<const uint4 *>(st + jr * row_bytes + sl[u] * 16);
-                    const uint16_t sr = *reinterpret_cast<const uint16_t *>(
-                        st + SR * row_bytes + jr * sb_bytes + gi[u] * 2);
-                    const uint16_t br = *reinterpret_cast<const uint16_t *>(
-                        st + SR * row_bytes + SR * sb_bytes + jr * sb_bytes + gi[u] * 2);
-                    const float sc = h16_to_f(sr, kBF16), bi = h16_to_f(br, kBF16);
+                    for (int u = 0; u < UPL; ++u) {
+                        const uint4 wv = *reinterpret_cast<const uint4 *>(wrow + soff[u]);
+                        const float sc = h16_to_f(*reinterpret_cast<const uint16_t *>(srow + gi[u] * 2), kBF16);
+                        const float bi = h16_to_f(
+                            *reinterpret_cast<const uint16_t *>(srow + SR * sb_bytes + gi[u] * 2), kBF16);
+                        const bool use = rv && sv[u];
 #pragma unroll
-                    for (int m = 0; m < MR; ++m) {
-                        float2 a = make_float2(0.f, 0.f);
-                        constexpr int SH = Sub<BITS>::SHIFT;
-                        dot_word<BITS>(wv.x, wv.x >> SH, &xq[m][u][0 * STEPS], a);
-                        dot_word<BITS>(wv.y, wv.y >> SH, &xq[m][u][1 * STEPS], a);
-                        dot_word<BITS>(wv.z, wv.z >> SH, &xq[m][u][2 * STEPS], a);
-                        dot_word<BITS>(wv.w, wv.w >> SH, &xq[m][u][3 * STEPS], a);
-                        part[m * RPT + j] = __fmaf_rn(sc * inv[m], a.x + a.y,
-                                                      __fmaf_rn(bi, xsum[m][u], part[m * RPT + j]));
+                        for (int m = 0; m < MR; ++m) {
+                            float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+                            constexpr int SH = Sub<BITS>::SHIFT;
+                            dot_word<BITS>(wv.x, wv.x >> SH, &xq[m][u][0 * STEPS], a0);
+                            dot_word<BITS>(wv.y, wv.y >> SH, &xq[m][u][1 * STEPS], a1);
+                            dot_word<BITS>(wv.z, wv.z >> SH, &xq[m][u][2 * STEPS], a0);
+                            dot_word<BITS>(wv.w, wv.w >> SH, &xq[m][u][3 * STEPS], a1);
+                            const float t = (a0.x + a0.y) + (a1.x + a1.y);
+                            const float c = __fmaf_rn(sc * inv[m], t, bi * xsum[m][u]);
+                            part[m * RPT + j] += use ? c : 0.f;
+                        }
                     }
                 }
             }
