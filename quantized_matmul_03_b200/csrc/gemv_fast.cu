@@ -13,17 +13,20 @@
 // owns the same 16-byte slice(s) of every row, so its activations live in
 // registers for the whole kernel.  Per group the product is factored as
 //   s * sum(x q) + b * sum(x).
-// For sum(x q) a code is masked, in place, into the low 23 bits of a 32-bit
-// word: with its exponent bits zero the word IS the fp32 subnormal
-// q * 2^p * 2^-149 exactly (p = the code's bit offset in the word; codes that
-// would touch bit 23 are taken from the word shifted right first).  So one AND
-// turns a code into an fp32 operand, and one packed FFMA2 multiplies two of
-// them by activations pre-scaled by 2^(sh - p) (sh per lane and row, chosen so
-// the largest |x| maps just below 2^127).  Products are exact normal fp32
-// numbers (8-bit x mantissa times a <= 8-bit code), accumulation is fp32, and
-// a slice's sum is scaled back by 2^(149 - sh).  Lane partials for a stage's
-// rows are combined by a butterfly reduce-scatter and shared-memory atomics;
-// results leave as one coalesced store per CTA.
+// For sum(x q) the codes stay integers: one AND spreads a word's codes into
+// byte lanes ("planes": for 4-bit codes, bytes of w & 0x0F0F0F0F are codes
+// 0,2,4,6 and bytes of (w >> 4) & 0x0F0F0F0F are codes 1,3,5,7), and DP2A
+// multiplies two bytes by two signed 16-bit activations and accumulates in
+// int32.  The activations of each 16-byte slice are held in 16-bit block
+// fixed point, x_int = rint(x * 2^sh) with sh chosen from the slice's largest
+// |x| so that |x_int| < 2^14: the representation error is at most 2^-15 of
+// the slice maximum, and every product and sum after it is exact.  A slice's
+// integer sum is scaled back by 2^-sh in fp32; sum(x) uses the exact x.
+// Per word of 4-bit codes this is 3 ALU + 4 DP2A instructions (8-bit codes:
+// 2 DP2A, no ALU), which keeps the ALU pipe, the limiter of an fp32
+// formulation, below the memory time.  Lane partials for a stage's rows are
+// combined by a butterfly reduce-scatter and shared-memory atomics; results
+// leave as one coalesced store per CTA.
 #include <algorithm>
 #include <cstdlib>
 #include <type_traits>
@@ -37,33 +40,40 @@ namespace {
 constexpr int kCW = 8;                    // consumer warps
 constexpr int kThreads = 32 * (kCW + 1);  // plus one producer warp
 
-// Element I of a packed word as an fp32 subnormal bit pattern (see above).
-// Codes whose bits reach bit 23 or above are read from the word shifted right
-// by SHIFT and keep place value sub_pw<BITS>(I).
-template <int BITS> struct Sub {
-    static constexpr int EPW = 32 / BITS;
-    static constexpr int SHIFT = BITS == 4 ? 12 : (BITS == 2 ? 10 : 16);
-    // first element taken from the shifted word
-    static constexpr int SPLIT = BITS == 4 ? 5 : (BITS == 2 ? 11 : 2);
+// Code planes of a packed word: plane p = (w >> p*BITS) & byte-mask, whose
+// byte j is code j*NP + p (NP = 8/BITS planes).  DP2A.lo takes bytes 0,1 and
+// DP2A.hi bytes 2,3, so the activation pairs of plane p are
+//   lo: (x[p], x[NP + p])     hi: (x[2NP + p], x[3NP + p]).
+template <int BITS> struct Planes {
+    static constexpr int EPW = 32 / BITS;      // codes per word
+    static constexpr int NP = 8 / BITS;        // planes per word
+    static constexpr uint32_t BYTE_MASK = ((1u << BITS) - 1u) * 0x01010101u;
+    // element (within the word) of half h (0/1) of pair k (k = 2p + {0: lo, 1: hi})
+    static __host__ __device__ constexpr int elem(int k, int h) {
+        return (k & 1) * 2 * NP + h * NP + (k >> 1);
+    }
 };
-template <int BITS>
-__host__ __device__ constexpr int sub_pw(int i) {
-    return i < Sub<BITS>::SPLIT ? BITS * i : BITS * i - Sub<BITS>::SHIFT;
+
+__device__ __forceinline__ int dp2a_lo(int xa, uint32_t b, int c) {
+    int d;
+    asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(xa), "r"(b), "r"(c));
+    return d;
 }
-template <int BITS, int I>
-__device__ __forceinline__ float sub_code(uint32_t w, uint32_t ws) {
-    constexpr uint32_t mask = ((1u << BITS) - 1u) << sub_pw<BITS>(I);
-    return __uint_as_float((I < Sub<BITS>::SPLIT ? w : ws) & mask);
+__device__ __forceinline__ int dp2a_hi(int xa, uint32_t b, int c) {
+    int d;
+    asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(xa), "r"(b), "r"(c));
+    return d;
 }
 
-// acc += x'[2j] * code[2j] , x'[2j+1] * code[2j+1] for every pair of a word.
-template <int BITS, int J = 0>
-__device__ __forceinline__ void dot_word(uint32_t w, uint32_t ws, const float2 *xq, float2 &acc) {
-    constexpr int PAIRS = Sub<BITS>::EPW / 2;
-    if constexpr (J < PAIRS) {
-        const float2 t = make_float2(sub_code<BITS, 2 * J>(w, ws), sub_code<BITS, 2 * J + 1>(w, ws));
-        acc = __ffma2_rn(xq[J], t, acc);
-        dot_word<BITS, J + 1>(w, ws, xq, acc);
+// acc0/acc1 += sum over the word's codes of x_int * q.
+template <int BITS, int P = 0>
+__device__ __forceinline__ void dot_word(uint32_t w, const int *xp, int &acc0, int &acc1) {
+    using PL = Planes<BITS>;
+    if constexpr (P < PL::NP) {
+        const uint32_t plane = (P == 0 ? w : (w >> (P * BITS))) & PL::BYTE_MASK;
+        acc0 = dp2a_lo(xp[2 * P], plane, acc0);
+        acc1 = dp2a_hi(xp[2 * P + 1], plane, acc1);
+        dot_word<BITS, P + 1>(w, xp, acc0, acc1);
     }
 }
 
@@ -168,17 +178,19 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
             soff[u] = sv[u] ? sl[u] * 16 : 0;
         }
 
-        // Activations: scaled fp32 pairs, per-slice sums, per-row scale-back.
-        float2 xq[MR][UPL][4 * STEPS];
+        // Activations in 16-bit block fixed point per slice (see the header):
+        // packed (lo, hi) int16 pairs in DP2A order, the slice's scale-back
+        // 2^-sh, and the exact slice sum of x for the bias term.
+        int xp[MR][UPL][4 * STEPS];
+        float fsc[MR][UPL];
         float xsum[MR][UPL];
-        float inv[MR];
 #pragma unroll
         for (int m = 0; m < MR; ++m) {
-            float xv[UPL][EPU];
-            float amax = 0.f;
 #pragma unroll
             for (int u = 0; u < UPL; ++u) {
                 const bool ok = sv[u] && m < M;
+                float xv[EPU];
+                float amax = 0.f, sum = 0.f;
 #pragma unroll
                 for (int c = 0; c < EPU / 8; ++c) {
                     uint4 raw = ok ? *reinterpret_cast<const uint4 *>(
@@ -187,38 +199,27 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     const uint16_t *h = reinterpret_cast<const uint16_t *>(&raw);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        xv[u][8 * c + q] = h16_to_f(h[q], kBF16);
-                        amax = fmaxf(amax, fabsf(xv[u][8 * c + q]));
+                        xv[8 * c + q] = h16_to_f(h[q], kBF16);
+                        amax = fmaxf(amax, fabsf(xv[8 * c + q]));
+                        sum += xv[8 * c + q];
                     }
                 }
-            }
-            // amax in [2^(ex-1), 2^ex) with ex = biased exponent - 126, so
-            // x * 2^sh stays below 2^127.  sh in [22, 191] keeps every power of
-            // two used here a normal float: x' = (x * 2^(sh-64)) * 2^(64-p)
-            // (the first product is below 2^63, the second below 2^127),
-            // scale-back 2^(149-sh).  (|x| < 2^105 is required; slices whose
-            // |x| are all below 2^-64 lose precision, negligibly.)
-            const int ex = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
-            const int sh = amax > 0.f ? min(191, max(22, 127 - ex)) : 127;
-            const float up = __uint_as_float((uint32_t)(sh + 63) << 23);   // 2^(sh-64)
-            inv[m] = __uint_as_float((uint32_t)(276 - sh) << 23);           // 2^(149-sh)
-#pragma unroll
-            for (int u = 0; u < UPL; ++u) {
-                float sum = 0.f;
+                // amax < 2^ex (ex = biased exponent - 126); x * 2^sh < 2^14 with
+                // sh = 14 - ex, clamped so that 2^sh and 2^-sh are normal floats.
+                const int ex = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
+                const int sh = min(126, max(-100, 14 - ex));
+                const float up = __uint_as_float((uint32_t)(127 + sh) << 23);
+                fsc[m][u] = __uint_as_float((uint32_t)(127 - sh) << 23);
+                xsum[m][u] = sum;
 #pragma unroll
                 for (int wd = 0; wd < 4; ++wd) {
 #pragma unroll
-                    for (int j = 0; j < STEPS; ++j) {
-                        const float a = xv[u][wd * EPW + 2 * j];
-                        const float b = xv[u][wd * EPW + 2 * j + 1];
-                        // 2^(64 - p) for the two codes' place values p
-                        const float ca = __uint_as_float((uint32_t)(191 - sub_pw<BITS>(2 * j)) << 23);
-                        const float cb = __uint_as_float((uint32_t)(191 - sub_pw<BITS>(2 * j + 1)) << 23);
-                        xq[m][u][wd * STEPS + j] = make_float2((a * up) * ca, (b * up) * cb);
-                        sum += a + b;
+                    for (int k = 0; k < STEPS; ++k) {
+                        const int lo = __float2int_rn(xv[wd * EPW + Planes<BITS>::elem(k, 0)] * up);
+                        const int hi = __float2int_rn(xv[wd * EPW + Planes<BITS>::elem(k, 1)] * up);
+                        xp[m][u][wd * STEPS + k] = (lo & 0xffff) | (hi << 16);
                     }
                 }
-                xsum[m][u] = sum;
             }
         }
 
@@ -230,7 +231,7 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
 #pragma unroll
             for (int q = 0; q < V; ++q) part[q] = 0.f;
             if (active) {
-                // All RPT rows are computed without branches so their FMA
+                // All RPT rows are computed without branches so their DP2A
                 // chains interleave; rows past the block's end read stale (but
                 // in-bounds) stage bytes and are dropped by the selects.
 #pragma unroll
@@ -248,14 +249,13 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                         const bool use = rv && sv[u];
 #pragma unroll
                         for (int m = 0; m < MR; ++m) {
-                            float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
-                            constexpr int SH = Sub<BITS>::SHIFT;
-                            dot_word<BITS>(wv.x, wv.x >> SH, &xq[m][u][0 * STEPS], a0);
-                            dot_word<BITS>(wv.y, wv.y >> SH, &xq[m][u][1 * STEPS], a1);
-                            dot_word<BITS>(wv.z, wv.z >> SH, &xq[m][u][2 * STEPS], a0);
-                            dot_word<BITS>(wv.w, wv.w >> SH, &xq[m][u][3 * STEPS], a1);
-                            const float t = (a0.x + a0.y) + (a1.x + a1.y);
-                            const float c = __fmaf_rn(sc * inv[m], t, bi * xsum[m][u]);
+                            int a0 = 0, a1 = 0;
+                            dot_word<BITS>(wv.x, &xp[m][u][0 * STEPS], a0, a1);
+                            dot_word<BITS>(wv.y, &xp[m][u][1 * STEPS], a0, a1);
+                            dot_word<BITS>(wv.z, &xp[m][u][2 * STEPS], a0, a1);
+                            dot_word<BITS>(wv.w, &xp[m][u][3 * STEPS], a0, a1);
+                            const float t = (float)(a0 + a1) * fsc[m][u];
+                            const float c = __fmaf_rn(sc, t, bi * xsum[m][u]);
                             part[m * RPT + j] += use ? c : 0.f;
                         }
                     }
