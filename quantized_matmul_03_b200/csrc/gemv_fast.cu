@@ -139,6 +139,11 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
         ptx::fence_mbar_init();
     }
     __syncthreads();
+    // Let the next launch in the stream begin its own prologue (barrier set-up
+    // and weight streaming) as this grid's CTAs retire.  Everything this grid
+    // reads before grid_dependency_wait() is the packed weight, its scales and
+    // biases, which no kernel of this library writes while it may overlap.
+    ptx::grid_launch_dependents();
 
     if (warp == 0) {
         // ---------------- producer ----------------
@@ -178,6 +183,9 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
             soff[u] = sv[u] ? sl[u] * 16 : 0;
         }
 
+        // The activations may be the output of the preceding kernel in the
+        // stream: wait for it (and for every earlier grid) to complete.
+        ptx::grid_dependency_wait();
         // Activations in 16-bit block fixed point per slice (see the header):
         // packed (lo, hi) int16 pairs in DP2A order, the slice's scale-back
         // 2^-sh, and the exact slice sum of x for the bias term.
@@ -343,10 +351,23 @@ cudaError_t launch_stream(const QmmArgs &a, cudaStream_t s) {
         if (got >= per_sm) break;
         if (per_sm == 1) return cudaErrorInvalidConfiguration;
     }
-    kern<<<p.grid, kThreads, p.smem, s>>>(
-        static_cast<const T *>(a.x), a.wq, static_cast<const T *>(a.scales),
-        static_cast<const T *>(a.biases), static_cast<T *>(a.y), (int)a.M, (int)a.N, (int)a.K,
-        a.group_size, p.rpc, p.stages, p.tw, device_error_word());
+    // Programmatic stream serialization: this grid may start while the
+    // preceding kernel of the stream finishes (see grid_dependency_wait()).
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, static_cast<const T *>(a.x), a.wq,
+                           static_cast<const T *>(a.scales), static_cast<const T *>(a.biases),
+                           static_cast<T *>(a.y), (int)a.M, (int)a.N, (int)a.K, a.group_size,
+                           p.rpc, p.stages, p.tw, device_error_word());
+    if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();
 }
