@@ -37,8 +37,9 @@
 namespace qmm {
 namespace {
 
-constexpr int kCW = 8;                    // consumer warps
-constexpr int kThreads = 32 * (kCW + 1);  // plus one producer warp
+constexpr int kCW = 8;               // warps per CTA, all consuming; thread 0 also refills
+constexpr int kThreads = 32 * kCW;   // (a CTA's register allocation rounds warps up to
+                                     // groups of four, so a ninth warp would cost three more)
 
 // Code planes of a packed word: plane p = (w >> p*BITS) & byte-mask, whose
 // byte j is code j*NP + p (NP = 8/BITS planes).  DP2A.lo takes bytes 0,1 and
@@ -201,8 +202,9 @@ struct LaneBlock {
     }
 };
 
+// Single-row variants are held to 128 registers so that two CTAs share an SM.
 template <typename T, int BITS, int MR, int UPL, int NG, int RPT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, MR == 1 ? 2 : 1)
 qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     const T *__restrict__ scales, const T *__restrict__ biases,
                     T *__restrict__ y, int M, int N, int K, int group_size, int rpc, int S,
@@ -242,29 +244,31 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     // biases, which no kernel of this library writes while it may overlap.
     ptx::grid_launch_dependents();
 
-    if (warp == 0) {
-        // ---------------- producer ----------------
-        if (lane == 0) {
-            const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(wq) + (int64_t)r0 * row_bytes;
-            const uint8_t *ssrc = reinterpret_cast<const uint8_t *>(scales) + (int64_t)r0 * sb_bytes;
-            const uint8_t *bsrc = reinterpret_cast<const uint8_t *>(biases) + (int64_t)r0 * sb_bytes;
-            for (int i = 0; i < nst; ++i) {
-                const int s = i % S;
-                if (i >= S) ptx::mbar_wait(empty0 + 8 * s, ((i / S) + 1) & 1, err);
-                const int nr = min(SR, nrows - i * SR);
-                const uint32_t wb = (uint32_t)(nr * row_bytes), sb = (uint32_t)(nr * sb_bytes);
-                const uint32_t st = ptx::smem_addr(smem + (size_t)s * stage_bytes);
-                const uint32_t bar = full0 + 8 * s;
-                ptx::mbar_arrive_expect_tx(bar, wb + 2 * sb);
-                const int64_t roff = (int64_t)i * SR;
-                ptx::bulk_g2s(st, wsrc + roff * row_bytes, wb, bar);
-                ptx::bulk_g2s(st + SR * row_bytes, ssrc + roff * sb_bytes, sb, bar);
-                ptx::bulk_g2s(st + SR * row_bytes + SR * sb_bytes, bsrc + roff * sb_bytes, sb, bar);
-            }
-        }
-    } else {
+    // ---- stage copies: thread 0 fills the ring now and refills stage i-1
+    // after its warp has consumed stage i (every warp has almost surely
+    // released stage i-1 by then, and stage i+1 is already in flight, so the
+    // wait on its "empty" barrier can neither deadlock nor stall for long).
+    const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(wq) + (int64_t)r0 * row_bytes;
+    const uint8_t *ssrc = reinterpret_cast<const uint8_t *>(scales) + (int64_t)r0 * sb_bytes;
+    const uint8_t *bsrc = reinterpret_cast<const uint8_t *>(biases) + (int64_t)r0 * sb_bytes;
+    auto issue_stage = [&](int i) {
+        const int s = i % S;
+        const int nr = min(SR, nrows - i * SR);
+        const uint32_t wb = (uint32_t)(nr * row_bytes), sb = (uint32_t)(nr * sb_bytes);
+        const uint32_t st = ptx::smem_addr(smem + (size_t)s * stage_bytes);
+        const uint32_t bar = full0 + 8 * s;
+        ptx::mbar_arrive_expect_tx(bar, wb + 2 * sb);
+        const int64_t roff = (int64_t)i * SR;
+        ptx::bulk_g2s(st, wsrc + roff * row_bytes, wb, bar);
+        ptx::bulk_g2s(st + SR * row_bytes, ssrc + roff * sb_bytes, sb, bar);
+        ptx::bulk_g2s(st + SR * row_bytes + SR * sb_bytes, bsrc + roff * sb_bytes, sb, bar);
+    };
+    if (threadIdx.x == 0)
+        for (int i = 0; i < min(S, nst); ++i) issue_stage(i);
+
+    {
         // ---------------- consumers ----------------
-        const int cw = warp - 1;
+        const int cw = warp;
         const int team = cw / TW, wt = cw - team * TW;
         const bool active = team < NT;
         const int spr = K / EPU;
@@ -319,6 +323,11 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(empty0 + 8 * s);
+            if (threadIdx.x == 0 && i >= 1 && i - 1 + S < nst) {
+                const int j = i - 1;
+                ptx::mbar_wait(empty0 + 8 * (j % S), (j / S) & 1, err);
+                issue_stage(j + S);
+            }
             const float v = reduce_scatter<V>(part, lane);
             if (active && lane < V) {
                 const int m = lane / RPT, j = lane - m * RPT;
@@ -347,7 +356,7 @@ constexpr size_t kSmemPerSm = 200 * 1024; // shared memory shared by the CTAs of
 void lane_block(const QmmArgs &a, int &upl, int &ng) {
     const int epu = 128 / a.bits;
     const int64_t spr = a.K / epu;
-    upl = spr >= 64 ? 2 : 1;
+    upl = (spr >= 64 && a.bits != 2) ? 2 : 1;  // 2-bit lane blocks of two slices would spill
     ng = (upl == 2 && a.group_size < 2 * epu) ? 2 : 1;
 }
 
