@@ -37,9 +37,8 @@
 namespace qmm {
 namespace {
 
-constexpr int kCW = 8;               // warps per CTA, all consuming; thread 0 also refills
-constexpr int kThreads = 32 * kCW;   // (a CTA's register allocation rounds warps up to
-                                     // groups of four, so a ninth warp would cost three more)
+constexpr int kCW = 8;                    // consumer warps
+constexpr int kThreads = 32 * (kCW + 1);  // plus one producer warp
 
 // Code planes of a packed word: plane p = (w >> p*BITS) & byte-mask, whose
 // byte j is code j*NP + p (NP = 8/BITS planes).  DP2A.lo takes bytes 0,1 and
@@ -103,115 +102,17 @@ __device__ __forceinline__ float h16_to_f(uint16_t h, bool is_bf16) {
     return is_bf16 ? __uint_as_float((uint32_t)h << 16) : __half2float(__ushort_as_half(h));
 }
 
-// One lane's share of a weight row: UPL consecutive 16-byte slices forming NG
-// groups (NG = 1 when the slices share one scale/bias, else NG = UPL).
-template <typename T, int BITS, int MR, int UPL, int NG>
-struct LaneBlock {
-    static constexpr int EPW = 32 / BITS;
-    static constexpr int EPU = 4 * EPW;          // codes per slice
-    static constexpr int STEPS = EPW / 2;        // DP2A operand pairs per word
-    static constexpr int SPG = UPL / NG;         // slices per group
-    static constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
-    int xp[MR][UPL][4 * STEPS];  // int16 activation pairs in DP2A order
-    float fsc[MR][NG];           // 2^-sh of each group's fixed point
-    float xsum[MR][NG];          // exact sum of x over each group
-
-    // Load and convert this lane's activations (all of the group's slices
-    // share one block exponent).
-    __device__ __forceinline__ void load_x(const T *__restrict__ x, int M, int K, const int *sl,
-                                           const bool *sv) {
-#pragma unroll
-        for (int m = 0; m < MR; ++m) {
-#pragma unroll
-            for (int g = 0; g < NG; ++g) {
-                float xv[SPG][EPU];
-                float amax = 0.f, sum = 0.f;
-#pragma unroll
-                for (int v = 0; v < SPG; ++v) {
-                    const int u = g * SPG + v;
-                    const bool ok = sv[u] && m < M;
-#pragma unroll
-                    for (int c = 0; c < EPU / 8; ++c) {
-                        uint4 raw = ok ? *reinterpret_cast<const uint4 *>(
-                                             x + (int64_t)m * K + (int64_t)sl[u] * EPU + 8 * c)
-                                       : make_uint4(0, 0, 0, 0);
-                        const uint16_t *h = reinterpret_cast<const uint16_t *>(&raw);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const float f = h16_to_f(h[q], kBF16);
-                            xv[v][8 * c + q] = f;
-                            amax = fmaxf(amax, fabsf(f));
-                            sum += f;
-                        }
-                    }
-                }
-                // amax < 2^ex (ex = biased exponent - 126); x * 2^sh < 2^14 with
-                // sh = 14 - ex, clamped so that 2^sh and 2^-sh are normal floats.
-                const int ex = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
-                const int sh = min(126, max(-100, 14 - ex));
-                const float up = __uint_as_float((uint32_t)(127 + sh) << 23);
-                fsc[m][g] = __uint_as_float((uint32_t)(127 - sh) << 23);
-                xsum[m][g] = sum;
-#pragma unroll
-                for (int v = 0; v < SPG; ++v) {
-#pragma unroll
-                    for (int wd = 0; wd < 4; ++wd) {
-#pragma unroll
-                        for (int k = 0; k < STEPS; ++k) {
-                            const int lo = __float2int_rn(xv[v][wd * EPW + Planes<BITS>::elem(k, 0)] * up);
-                            const int hi = __float2int_rn(xv[v][wd * EPW + Planes<BITS>::elem(k, 1)] * up);
-                            xp[m][g * SPG + v][wd * STEPS + k] = (lo & 0xffff) | (hi << 16);
-                        }
-                    }
-                }
-            }
-        }
-    }
-
-    // Add this lane's contribution to one weight row into part[m * RPT + j].
-    // wrow: the row's packed bytes in shared memory; srow/brow: its scales and
-    // biases; soff/gi: byte offset and group of each slice (0 when unused).
-    template <int RPT>
-    __device__ __forceinline__ void row(const uint8_t *wrow, const uint8_t *srow,
-                                        const uint8_t *brow, const int *soff, const int *gi,
-                                        const bool *gv, float *part, int j) const {
-        uint4 wv[UPL];
-#pragma unroll
-        for (int u = 0; u < UPL; ++u) wv[u] = *reinterpret_cast<const uint4 *>(wrow + soff[u]);
-#pragma unroll
-        for (int g = 0; g < NG; ++g) {
-            const int gu = g * SPG;
-            const float sc = h16_to_f(*reinterpret_cast<const uint16_t *>(srow + gi[gu] * 2), kBF16);
-            const float bi = h16_to_f(*reinterpret_cast<const uint16_t *>(brow + gi[gu] * 2), kBF16);
-#pragma unroll
-            for (int m = 0; m < MR; ++m) {
-                int a0 = 0, a1 = 0;
-#pragma unroll
-                for (int v = 0; v < SPG; ++v) {
-                    const int u = gu + v;
-                    dot_word<BITS>(wv[u].x, &xp[m][u][0 * STEPS], a0, a1);
-                    dot_word<BITS>(wv[u].y, &xp[m][u][1 * STEPS], a0, a1);
-                    dot_word<BITS>(wv[u].z, &xp[m][u][2 * STEPS], a0, a1);
-                    dot_word<BITS>(wv[u].w, &xp[m][u][3 * STEPS], a0, a1);
-                }
-                const float t = (float)(a0 + a1) * fsc[m][g];
-                const float c = __fmaf_rn(sc, t, bi * xsum[m][g]);
-                part[m * RPT + j] += gv[g] ? c : 0.f;
-            }
-        }
-    }
-};
-
-// Single-row variants are held to 128 registers so that two CTAs share an SM.
-template <typename T, int BITS, int MR, int UPL, int NG, int RPT>
-__global__ void __launch_bounds__(kThreads, MR == 1 ? 2 : 1)
+template <typename T, int BITS, int MR, int UPL, int RPT>
+__global__ void __launch_bounds__(kThreads, 1)
 qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     const T *__restrict__ scales, const T *__restrict__ biases,
                     T *__restrict__ y, int M, int N, int K, int group_size, int rpc, int S,
                     int TW, int *err) {
-    using LB = LaneBlock<T, BITS, MR, UPL, NG>;
-    constexpr int EPU = LB::EPU;
+    constexpr int EPW = 32 / BITS;       // codes per word
+    constexpr int EPU = 4 * EPW;         // codes per 16-byte slice
+    constexpr int STEPS = EPW / 2;       // code pairs per word
     constexpr int V = MR * RPT;          // partials per lane per stage
+    constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
     static_assert((V & (V - 1)) == 0 && V <= 32, "V must be a power of two <= 32");
 
     extern __shared__ __align__(128) uint8_t smem[];
@@ -244,37 +145,36 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     // biases, which no kernel of this library writes while it may overlap.
     ptx::grid_launch_dependents();
 
-    // ---- stage copies: thread 0 fills the ring now and refills stage i-1
-    // after its warp has consumed stage i (every warp has almost surely
-    // released stage i-1 by then, and stage i+1 is already in flight, so the
-    // wait on its "empty" barrier can neither deadlock nor stall for long).
-    const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(wq) + (int64_t)r0 * row_bytes;
-    const uint8_t *ssrc = reinterpret_cast<const uint8_t *>(scales) + (int64_t)r0 * sb_bytes;
-    const uint8_t *bsrc = reinterpret_cast<const uint8_t *>(biases) + (int64_t)r0 * sb_bytes;
-    auto issue_stage = [&](int i) {
-        const int s = i % S;
-        const int nr = min(SR, nrows - i * SR);
-        const uint32_t wb = (uint32_t)(nr * row_bytes), sb = (uint32_t)(nr * sb_bytes);
-        const uint32_t st = ptx::smem_addr(smem + (size_t)s * stage_bytes);
-        const uint32_t bar = full0 + 8 * s;
-        ptx::mbar_arrive_expect_tx(bar, wb + 2 * sb);
-        const int64_t roff = (int64_t)i * SR;
-        ptx::bulk_g2s(st, wsrc + roff * row_bytes, wb, bar);
-        ptx::bulk_g2s(st + SR * row_bytes, ssrc + roff * sb_bytes, sb, bar);
-        ptx::bulk_g2s(st + SR * row_bytes + SR * sb_bytes, bsrc + roff * sb_bytes, sb, bar);
-    };
-    if (threadIdx.x == 0)
-        for (int i = 0; i < min(S, nst); ++i) issue_stage(i);
-
-    {
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(wq) + (int64_t)r0 * row_bytes;
+            const uint8_t *ssrc = reinterpret_cast<const uint8_t *>(scales) + (int64_t)r0 * sb_bytes;
+            const uint8_t *bsrc = reinterpret_cast<const uint8_t *>(biases) + (int64_t)r0 * sb_bytes;
+            for (int i = 0; i < nst; ++i) {
+                const int s = i % S;
+                if (i >= S) ptx::mbar_wait(empty0 + 8 * s, ((i / S) + 1) & 1, err);
+                const int nr = min(SR, nrows - i * SR);
+                const uint32_t wb = (uint32_t)(nr * row_bytes), sb = (uint32_t)(nr * sb_bytes);
+                const uint32_t st = ptx::smem_addr(smem + (size_t)s * stage_bytes);
+                const uint32_t bar = full0 + 8 * s;
+                ptx::mbar_arrive_expect_tx(bar, wb + 2 * sb);
+                const int64_t roff = (int64_t)i * SR;
+                ptx::bulk_g2s(st, wsrc + roff * row_bytes, wb, bar);
+                ptx::bulk_g2s(st + SR * row_bytes, ssrc + roff * sb_bytes, sb, bar);
+                ptx::bulk_g2s(st + SR * row_bytes + SR * sb_bytes, bsrc + roff * sb_bytes, sb, bar);
+            }
+        }
+    } else {
         // ---------------- consumers ----------------
-        const int cw = warp;
+        const int cw = warp - 1;
         const int team = cw / TW, wt = cw - team * TW;
         const bool active = team < NT;
         const int spr = K / EPU;
 
-        int sl[UPL], soff[UPL], gi[UPL];
-        bool sv[UPL], gvalid[NG];
+        int sl[UPL];
+        bool sv[UPL];
+        int gi[UPL], soff[UPL];   // group index and byte offset of the slice (0 if unused)
 #pragma unroll
         for (int u = 0; u < UPL; ++u) {
             sl[u] = (wt * 32 + lane) * UPL + u;
@@ -282,52 +182,95 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
             gi[u] = sv[u] ? (sl[u] * EPU) / group_size : 0;
             soff[u] = sv[u] ? sl[u] * 16 : 0;
         }
-#pragma unroll
-        for (int g = 0; g < NG; ++g) gvalid[g] = sv[g * LB::SPG];
 
         // The activations may be the output of the preceding kernel in the
         // stream: wait for it (and for every earlier grid) to complete.
         ptx::grid_dependency_wait();
-        LB lb;
-        lb.load_x(x, M, K, sl, sv);
+        // Activations in 16-bit block fixed point per slice (see the header):
+        // packed (lo, hi) int16 pairs in DP2A order, the slice's scale-back
+        // 2^-sh, and the exact slice sum of x for the bias term.
+        int xp[MR][UPL][4 * STEPS];
+        float fsc[MR][UPL];
+        float xsum[MR][UPL];
+#pragma unroll
+        for (int m = 0; m < MR; ++m) {
+#pragma unroll
+            for (int u = 0; u < UPL; ++u) {
+                const bool ok = sv[u] && m < M;
+                float xv[EPU];
+                float amax = 0.f, sum = 0.f;
+#pragma unroll
+                for (int c = 0; c < EPU / 8; ++c) {
+                    uint4 raw = ok ? *reinterpret_cast<const uint4 *>(
+                                         x + (int64_t)m * K + (int64_t)sl[u] * EPU + 8 * c)
+                                   : make_uint4(0, 0, 0, 0);
+                    const uint16_t *h = reinterpret_cast<const uint16_t *>(&raw);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        xv[8 * c + q] = h16_to_f(h[q], kBF16);
+                        amax = fmaxf(amax, fabsf(xv[8 * c + q]));
+                        sum += xv[8 * c + q];
+                    }
+                }
+                // amax < 2^ex (ex = biased exponent - 126); x * 2^sh < 2^14 with
+                // sh = 14 - ex, clamped so that 2^sh and 2^-sh are normal floats.
+                const int ex = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
+                const int sh = min(126, max(-100, 14 - ex));
+                const float up = __uint_as_float((uint32_t)(127 + sh) << 23);
+                fsc[m][u] = __uint_as_float((uint32_t)(127 - sh) << 23);
+                xsum[m][u] = sum;
+#pragma unroll
+                for (int wd = 0; wd < 4; ++wd) {
+#pragma unroll
+                    for (int k = 0; k < STEPS; ++k) {
+                        const int lo = __float2int_rn(xv[wd * EPW + Planes<BITS>::elem(k, 0)] * up);
+                        const int hi = __float2int_rn(xv[wd * EPW + Planes<BITS>::elem(k, 1)] * up);
+                        xp[m][u][wd * STEPS + k] = (lo & 0xffff) | (hi << 16);
+                    }
+                }
+            }
+        }
 
         for (int i = 0; i < nst; ++i) {
             const int s = i % S;
             ptx::mbar_wait(full0 + 8 * s, (i / S) & 1, err);
             const uint8_t *st = smem + (size_t)s * stage_bytes;
-            const uint8_t *sst = st + SR * row_bytes;
             float part[V];
 #pragma unroll
             for (int q = 0; q < V; ++q) part[q] = 0.f;
             if (active) {
-                if ((i + 1) * SR <= nrows) {
-                    // Full stage: rows unrolled without branches so that their
-                    // DP2A chains interleave.
+                // All RPT rows are computed without branches so their DP2A
+                // chains interleave; rows past the block's end read stale (but
+                // in-bounds) stage bytes and are dropped by the selects.
 #pragma unroll
-                    for (int j = 0; j < RPT; ++j) {
-                        const int jr = team + j * NT;
-                        lb.template row<RPT>(st + jr * row_bytes, sst + jr * sb_bytes,
-                                             sst + (SR + jr) * sb_bytes, soff, gi, gvalid, part, j);
-                    }
-                } else {
-                    // Last, partial stage: skip rows past the block's end.
+                for (int j = 0; j < RPT; ++j) {
+                    const int jr = team + j * NT;           // row within the stage (< SR)
+                    const bool rv = i * SR + jr < nrows;
+                    const uint8_t *wrow = st + jr * row_bytes;
+                    const uint8_t *srow = st + SR * row_bytes + jr * sb_bytes;
 #pragma unroll
-                    for (int j = 0; j < RPT; ++j) {
-                        const int jr = team + j * NT;
-                        if (i * SR + jr < nrows)
-                            lb.template row<RPT>(st + jr * row_bytes, sst + jr * sb_bytes,
-                                                 sst + (SR + jr) * sb_bytes, soff, gi, gvalid, part,
-                                                 j);
+                    for (int u = 0; u < UPL; ++u) {
+                        const uint4 wv = *reinterpret_cast<const uint4 *>(wrow + soff[u]);
+                        const float sc = h16_to_f(*reinterpret_cast<const uint16_t *>(srow + gi[u] * 2), kBF16);
+                        const float bi = h16_to_f(
+                            *reinterpret_cast<const uint16_t *>(srow + SR * sb_bytes + gi[u] * 2), kBF16);
+                        const bool use = rv && sv[u];
+#pragma unroll
+                        for (int m = 0; m < MR; ++m) {
+                            int a0 = 0, a1 = 0;
+                            dot_word<BITS>(wv.x, &xp[m][u][0 * STEPS], a0, a1);
+                            dot_word<BITS>(wv.y, &xp[m][u][1 * STEPS], a0, a1);
+                            dot_word<BITS>(wv.z, &xp[m][u][2 * STEPS], a0, a1);
+                            dot_word<BITS>(wv.w, &xp[m][u][3 * STEPS], a0, a1);
+                            const float t = (float)(a0 + a1) * fsc[m][u];
+                            const float c = __fmaf_rn(sc, t, bi * xsum[m][u]);
+                            part[m * RPT + j] += use ? c : 0.f;
+                        }
                     }
                 }
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(empty0 + 8 * s);
-            if (threadIdx.x == 0 && i >= 1 && i - 1 + S < nst) {
-                const int j = i - 1;
-                ptx::mbar_wait(empty0 + 8 * (j % S), (j / S) & 1, err);
-                issue_stage(j + S);
-            }
             const float v = reduce_scatter<V>(part, lane);
             if (active && lane < V) {
                 const int m = lane / RPT, j = lane - m * RPT;
@@ -344,31 +287,26 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
 }
 
 struct StreamPlan {
-    int upl, ng, tw, sr, stages, rpc, grid;
+    int upl, tw, rpt, sr, stages, rpc, grid;
     size_t smem;
 };
 
-constexpr int kRPT = 2;                   // rows per team per stage
-constexpr size_t kSmemPerSm = 200 * 1024; // shared memory shared by the CTAs of an SM
+// Shared memory per CTA: the whole SM's worth (one CTA per SM) or half of it
+// (two CTAs per SM, which doubles the warps available to hide latency).
+constexpr size_t kSmemPerSm = 200 * 1024;
 
-// Slices per lane: two (one group of 2x the slice's codes, one scale/bias)
-// once a row is wide enough to keep every lane busy, else one.
-void lane_block(const QmmArgs &a, int &upl, int &ng) {
-    const int epu = 128 / a.bits;
-    const int64_t spr = a.K / epu;
-    upl = (spr >= 64 && a.bits != 2) ? 2 : 1;  // 2-bit lane blocks of two slices would spill
-    ng = (upl == 2 && a.group_size < 2 * epu) ? 2 : 1;
-}
+int rows_per_team_stage(int mr) { return mr == 4 ? 2 : 4; }
 
 bool plan_stream(const QmmArgs &a, int mr, int ctas_per_sm, StreamPlan &p) {
     const int bits = a.bits;
     const int epu = 128 / bits;
     const int64_t spr = a.K / epu;
-    lane_block(a, p.upl, p.ng);
+    p.upl = spr > 32 * kCW ? 2 : 1;
     p.tw = (int)((spr + 32 * p.upl - 1) / (32 * p.upl));
     if (p.tw > kCW) return false;
     const int nt = kCW / p.tw;
-    p.sr = nt * kRPT;
+    p.rpt = rows_per_team_stage(mr);
+    p.sr = nt * p.rpt;
     const int64_t row_bytes = a.K / 8 * bits;
     const int64_t sb_bytes = a.K / a.group_size * 2;
     const int64_t stage = (int64_t)p.sr * (row_bytes + 2 * sb_bytes);
@@ -387,31 +325,32 @@ bool plan_stream(const QmmArgs &a, int mr, int ctas_per_sm, StreamPlan &p) {
 }
 
 // Variants whose activations and partials fit the register file without
-// spilling (checked with ptxas -v).
+// spilling (checked with ptxas -v): rows x slices per lane is bounded by the
+// codes per slice (32 for 4-bit, 16 for 8-bit, 64 for 2-bit).
 bool stream_variant_fits(int bits, int mr, int upl) {
-    if (mr == 1) return true;
-    if (bits == 2) return false;
-    if (mr == 2) return true;
-    return upl == 1;  // four rows
+    if (mr == 1) return bits != 2 || upl == 1;
+    if (bits == 4) return mr == 2 && upl == 1;
+    if (bits == 8) return mr == 2 || upl == 1;
+    return false;
 }
 
-template <typename T, int BITS, int MR, int UPL, int NG>
+template <typename T, int BITS, int MR, int UPL>
 cudaError_t launch_stream(const QmmArgs &a, cudaStream_t s) {
-    auto kern = qgemv_stream_kernel<T, BITS, MR, UPL, NG, kRPT>;
-    // As many CTAs per SM (up to three) as registers and the split ring allow.
+    constexpr int RPT = MR == 4 ? 2 : 4;
+    auto kern = qgemv_stream_kernel<T, BITS, MR, UPL, RPT>;
+    // Two CTAs per SM when the registers and the halved ring allow it.
     StreamPlan p{};
     cudaError_t e = cudaSuccess;
-    bool ok = false;
-    for (int per_sm = 3; per_sm >= 1 && !ok; --per_sm) {
+    for (int per_sm = 2; per_sm >= 1; --per_sm) {
         if (!plan_stream(a, MR, per_sm, p)) continue;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
         if (e != cudaSuccess) return e;
         int got = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&got, kern, kThreads, p.smem);
         if (e != cudaSuccess) return e;
-        ok = got >= per_sm;
+        if (got >= per_sm) break;
+        if (per_sm == 1) return cudaErrorInvalidConfiguration;
     }
-    if (!ok) return cudaErrorInvalidConfiguration;
     // Programmatic stream serialization: this grid may start while the
     // preceding kernel of the stream finishes (see grid_dependency_wait()).
     cudaLaunchConfig_t cfg = {};
@@ -433,24 +372,23 @@ cudaError_t launch_stream(const QmmArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-template <typename T, int BITS, int MR>
-cudaError_t stream_rows(const QmmArgs &a, int upl, int ng, cudaStream_t s) {
-    if (upl == 1) return launch_stream<T, BITS, MR, 1, 1>(a, s);
-    if constexpr (MR <= 2) {
-        if (ng == 1) return launch_stream<T, BITS, MR, 2, 1>(a, s);
-        return launch_stream<T, BITS, MR, 2, 2>(a, s);
-    }
-    return cudaErrorInvalidValue;
-}
-
 template <typename T, int BITS>
 cudaError_t stream_bits(const QmmArgs &a, cudaStream_t s) {
-    int upl = 1, ng = 1;
-    lane_block(a, upl, ng);
-    if (a.M == 1) return stream_rows<T, BITS, 1>(a, upl, ng, s);
+    const int mr = a.M == 1 ? 1 : (a.M == 2 ? 2 : 4);
+    StreamPlan p{};
+    if (!plan_stream(a, mr, 1, p)) return cudaErrorInvalidValue;
+    // Only the variants that fit in registers are instantiated; the others are
+    // refused by stream_variant_fits() and go to the general kernel.
+    if (mr == 1) {
+        if (p.upl == 1) return launch_stream<T, BITS, 1, 1>(a, s);
+        if constexpr (BITS != 2) return launch_stream<T, BITS, 1, 2>(a, s);
+    }
     if constexpr (BITS != 2) {
-        if (a.M == 2) return stream_rows<T, BITS, 2>(a, upl, ng, s);
-        return stream_rows<T, BITS, 4>(a, upl, ng, s);
+        if (mr == 2 && p.upl == 1) return launch_stream<T, BITS, 2, 1>(a, s);
+    }
+    if constexpr (BITS == 8) {
+        if (mr == 2) return launch_stream<T, BITS, 2, 2>(a, s);
+        if (mr == 4 && p.upl == 1) return launch_stream<T, BITS, 4, 1>(a, s);
     }
     return cudaErrorInvalidValue;
 }
