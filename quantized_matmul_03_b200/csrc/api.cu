@@ -19,6 +19,8 @@ __device__ int g_qmm_device_error = 0;
 namespace {
 
 thread_local std::string t_last_error;
+// Activation rows up to which the SIMT decode kernels are used (AUTO path).
+constexpr int64_t kGemvMaxRows = 4;
 qmm_path g_path = QMM_PATH_AUTO;
 
 qmm_status fail(qmm_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
@@ -188,11 +190,23 @@ qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K, const uint3
         if (st != QMM_OK) return st;
         if (M == 0 || N == 0) return QMM_OK;
         QmmArgs a{x, wq, scales, biases, y, M, N, K, group_size, bits, transpose != 0};
-        if (g_path == QMM_PATH_GEMM)
-            return fail(QMM_ERR_UNSUPPORTED, "the tensor-core path is not available");
-        if (gemv_fast_supported(dtype, a))
-            return finish_launch(launch_gemv_fast(dtype, a, (cudaStream_t)stream), "gemv launch");
-        return finish_launch(launch_gemv(dtype, a, (cudaStream_t)stream), "gemv launch");
+        cudaStream_t s = (cudaStream_t)stream;
+        const bool tc_ok = gemm_supported(dtype, a);
+        if (g_path == QMM_PATH_GEMM) {
+            if (!tc_ok)
+                return fail(QMM_ERR_UNSUPPORTED,
+                            "the tensor-core path needs bf16/f16, transpose, K %% 64 == 0");
+            return finish_launch(launch_gemm(dtype, a, s), "tensor-core gemm launch");
+        }
+        // Decode shapes stream the weight through the SIMT kernels; larger
+        // activation counts use the tensor cores.
+        const bool few_rows = a.M <= kGemvMaxRows;
+        if (g_path == QMM_PATH_GEMV || few_rows || !tc_ok) {
+            if (gemv_fast_supported(dtype, a))
+                return finish_launch(launch_gemv_fast(dtype, a, s), "gemv launch");
+            return finish_launch(launch_gemv(dtype, a, s), "gemv launch");
+        }
+        return finish_launch(launch_gemm(dtype, a, s), "tensor-core gemm launch");
     } catch (...) {
         return fail(QMM_ERR_CUDA, "unexpected exception in qmm_quantized_matmul");
     }

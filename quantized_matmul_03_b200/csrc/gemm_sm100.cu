@@ -1,0 +1,537 @@
+// gemm_sm100.cu -- tensor-core quantized matmul for many activation rows
+// (prefill), transpose layout:  y[m, n] = sum_k x[m, k] * (s[n,g] q[n,k] + b[n,g])
+// with W stored [N, K] (mlx-rs ops/quantization.rs, quantized_matmul;
+// Emily.Quantization.Layers, quantized_dense with transpose: true).  The dense
+// weight never exists in global memory: each 128 x 64 tile is dequantized into
+// shared memory right before the tensor cores consume it.
+//
+// Orientation ("swap AB"): the UMMA M dimension (128) runs over weight rows n
+// and the UMMA N dimension (BN = 16..256) over activation rows m, so the
+// dequantized tile is the A operand and the activations are the B operand:
+//     D[n, m] (TMEM, fp32) += W~[n, k] * x[m, k]   for k-blocks of 64.
+// Both operands are K-major bf16/f16 in the canonical 128-byte-swizzle layout
+// (8-row x 128-byte atoms, row r's 16-byte chunk c at chunk c ^ (r mod 8)).
+//
+// Roles (one CTA per SM, persistent over output tiles):
+//   warps 0-7   dequantize: thread t owns weight row t mod 128 and half t / 128
+//               of the k-block; it reads the packed codes the producer staged,
+//               forms s*q + b two codes at a time (bf16x2/f16x2 FMA, one
+//               rounding), and writes the swizzled A tile;
+//   warps 8-11  epilogue: tcgen05.ld of the accumulator quadrant the warp may
+//               address (lanes 32*(warp%4)..), convert, store y;
+//   warp 12     producer: TMA loads of the packed weight tile and the
+//               activation tile for each k-block into a ring of stages;
+//   warp 13     MMA issuer (one thread) and TMEM owner.
+// Every wait is a bounded mbarrier wait (device error word on timeout); no
+// cluster multicast is used.
+#include <cuda.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "ptx_sm100.cuh"
+#include "qmm_internal.cuh"
+
+namespace qmm {
+namespace {
+
+constexpr int kDqWarps = 8;
+constexpr int kEpiWarps = 4;
+constexpr int kWarpTma = kDqWarps + kEpiWarps;  // 12
+constexpr int kWarpMma = kWarpTma + 1;          // 13
+constexpr int kThreads = 32 * (kWarpMma + 1);   // 448
+constexpr int kBM = 128;                        // weight rows per tile (UMMA M)
+constexpr int kBK = 64;                         // k per stage: one 128-byte swizzle row
+
+// ---------------------------------------------------------------------------
+// tcgen05 / TMA wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Arrive on `bar` once every tcgen05.mma this thread issued so far completed.
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+// D[tmem] (+)= A[desc_a] * B[desc_b]^T, shapes and types from idesc.
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t desc_a, uint64_t desc_b,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(desc_a), "l"(desc_b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+          "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+          "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(map), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), LBO unused (16), descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, A/B both bf16 (or
+// both f16), both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t make_idesc(bool f16, int m, int n) {
+    return (1u << 4) | ((f16 ? 0u : 1u) << 7) | ((f16 ? 0u : 1u) << 10) |
+           ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// Dequantization of a half k-block of one weight row (32 codes) into four
+// 16-byte chunks of 16-bit values, two codes per FMA.
+// ---------------------------------------------------------------------------
+template <typename T> struct Pair;
+template <> struct Pair<__nv_bfloat16> {
+    using V2 = __nv_bfloat162;
+    static constexpr uint32_t MAGIC = 0x43004300u;  // 128.0 | 128.0
+    static __device__ __forceinline__ V2 bits(uint32_t u) { return *reinterpret_cast<V2 *>(&u); }
+    static __device__ __forceinline__ uint32_t ubits(V2 v) { return *reinterpret_cast<uint32_t *>(&v); }
+    static __device__ __forceinline__ V2 off() { return __float2bfloat162_rn(128.f); }
+    static __device__ __forceinline__ V2 splat(uint16_t h) {
+        __nv_bfloat16 b = *reinterpret_cast<__nv_bfloat16 *>(&h);
+        return __bfloat162bfloat162(b);
+    }
+};
+template <> struct Pair<__half> {
+    using V2 = __half2;
+    static constexpr uint32_t MAGIC = 0x64006400u;  // 1024.0 | 1024.0
+    static __device__ __forceinline__ V2 bits(uint32_t u) { return *reinterpret_cast<V2 *>(&u); }
+    static __device__ __forceinline__ uint32_t ubits(V2 v) { return *reinterpret_cast<uint32_t *>(&v); }
+    static __device__ __forceinline__ V2 off() { return __float2half2_rn(1024.f); }
+    static __device__ __forceinline__ V2 splat(uint16_t h) {
+        __half b = *reinterpret_cast<__half *>(&h);
+        return __half2half2(b);
+    }
+};
+
+// Magic-number path (4- and 2-bit codes; 8-bit codes with f16): OR a code
+// into the mantissa of OFF (exact), subtract OFF (exact), then s*q + b.
+// Produces 16-bit values in k order, 8 per output uint4.
+template <typename T, int BITS>
+__device__ __forceinline__ void dequant_half(const uint32_t *w, uint16_t s16, uint16_t b16,
+                                             uint4 (&out)[4]) {
+    using P = Pair<T>;
+    using V2 = typename P::V2;
+    constexpr int EPW = 32 / BITS;                 // codes per word
+    constexpr int NW = 32 / EPW;                   // words per 32 codes
+    constexpr uint32_t MASK = BITS == 8 ? 0x00FF00FFu : (BITS == 4 ? 0x000F000Fu : 0x00030003u);
+    const V2 s2 = P::splat(s16), b2 = P::splat(b16), off = P::off();
+    uint32_t vals[16];  // 32 values as 16 pairs (2i, 2i+1)
+#pragma unroll
+    for (int wi = 0; wi < NW; ++wi) {
+        // step e yields codes (e, e + EPW/2) of the word
+        uint32_t pe[EPW / 2];
+#pragma unroll
+        for (int e = 0; e < EPW / 2; ++e) {
+            const uint32_t t = ((w[wi] >> (BITS * e)) & MASK) | P::MAGIC;
+            const V2 q = __hsub2(P::bits(t), off);
+            pe[e] = P::ubits(__hfma2(q, s2, b2));
+        }
+        // re-pair (e, e+H) into consecutive pairs (2i, 2i+1)
+        constexpr int H = EPW / 2;
+#pragma unroll
+        for (int i = 0; i < EPW / 2; ++i) {
+            const int a = 2 * i, b = 2 * i + 1;  // element indices within the word
+            const uint32_t ra = pe[a % H], rb = pe[b % H];
+            const uint32_t sel = (a < H ? 0x0010u : 0x0032u) | (b < H ? 0x5400u : 0x7600u);
+            vals[wi * (EPW / 2) + i] = __byte_perm(ra, rb, sel);
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        out[c] = make_uint4(vals[4 * c], vals[4 * c + 1], vals[4 * c + 2], vals[4 * c + 3]);
+}
+
+// 8-bit codes with bf16 (no exact bf16 magic for 0..255): fp32 magic.
+template <>
+__device__ __forceinline__ void dequant_half<__nv_bfloat16, 8>(const uint32_t *w, uint16_t s16,
+                                                               uint16_t b16, uint4 (&out)[4]) {
+    const float s = __uint_as_float((uint32_t)s16 << 16), b = __uint_as_float((uint32_t)b16 << 16);
+    uint32_t vals[16];
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) {
+        float f[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float q = __uint_as_float(__byte_perm(w[wi], 0x4B000000u, 0x7650u + e)) - 8388608.f;
+            f[e] = __fmaf_rn(s, q, b);
+        }
+        __nv_bfloat162 lo = __floats2bfloat162_rn(f[0], f[1]), hi = __floats2bfloat162_rn(f[2], f[3]);
+        vals[2 * wi] = *reinterpret_cast<uint32_t *>(&lo);
+        vals[2 * wi + 1] = *reinterpret_cast<uint32_t *>(&hi);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        out[c] = make_uint4(vals[4 * c], vals[4 * c + 1], vals[4 * c + 2], vals[4 * c + 3]);
+}
+
+struct GemmParams {
+    const void *scales, *biases;
+    void *y;
+    int M, N, K, group_size;
+    int m_tiles, n_tiles, num_tiles, stages;
+    int *err;
+};
+
+template <typename T, int BITS, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                const GemmParams p) {
+    constexpr bool kF16 = std::is_same<T, __half>::value;
+    constexpr int A_BYTES = kBM * kBK * 2;         // 16 KB dequantized tile
+    constexpr int B_BYTES = BN * kBK * 2;          // activation tile
+    constexpr int P_ROW = kBK * BITS / 8;          // packed bytes per row per k-block
+    constexpr int P_BYTES = kBM * P_ROW;
+    constexpr int W_WORDS = kBK * BITS / 32;       // packed words per row per k-block
+    constexpr uint32_t TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
+    constexpr uint32_t IDESC = make_idesc(kF16, kBM, BN);
+
+    extern __shared__ uint8_t smem_raw[];
+    const int S = p.stages;
+    // 1024-byte aligned carve-up: A[S] | B[S] | P[S] | barriers | tmem slot
+    const uint32_t raw = ptx::smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (base - raw);
+    const uint32_t a0 = base, b0 = a0 + S * A_BYTES, p0 = b0 + S * B_BYTES;
+    const uint32_t bar0 = p0 + S * P_BYTES;
+    const uint32_t full_pb = bar0, full_a = bar0 + 8 * S, empty = bar0 + 16 * S;
+    const uint32_t acc_full = bar0 + 24 * S, acc_empty = acc_full + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + (acc_empty + 16 - base));
+    const uint8_t *pg = gbase + (p0 - base);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(full_pb + 8 * s, 1);
+            ptx::mbar_init(full_a + 8 * s, kDqWarps);
+            ptx::mbar_init(empty + 8 * s, 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            ptx::mbar_init(acc_full + 8 * a, 1);
+            ptx::mbar_init(acc_empty + 8 * a, kEpiWarps);
+        }
+        ptx::fence_mbar_init();
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(ptx::smem_addr(tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int KB = (p.K + kBK - 1) / kBK;
+    const int gpr = p.K / p.group_size;
+
+    if (warp < kDqWarps) {
+        // ------------------------- dequantize -------------------------
+        const int r = threadIdx.x & (kBM - 1), h = threadIdx.x >> 7;  // row, k half
+        const uint16_t *sc = static_cast<const uint16_t *>(p.scales);
+        const uint16_t *bi = static_cast<const uint16_t *>(p.biases);
+        int c = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+            const int n0 = (tile / p.m_tiles) * kBM;
+            const int n = n0 + r;
+            const bool rv = n < p.N;
+            for (int kb = 0; kb < KB; ++kb, ++c) {
+                const int s = c % S;
+                const int k0 = kb * kBK + 32 * h;
+                uint16_t s16 = 0, b16 = 0;
+                if (rv && k0 < p.K) {
+                    const int64_t gi = (int64_t)n * gpr + k0 / p.group_size;
+                    s16 = __ldg(sc + gi);
+                    b16 = __ldg(bi + gi);
+                }
+                ptx::mbar_wait(full_pb + 8 * s, (c / S) & 1, p.err);
+                uint32_t w[BITS];  // 32 codes = BITS words
+                const uint8_t *src = pg + s * P_BYTES + r * P_ROW + h * (P_ROW / 2);
+                if constexpr (BITS == 8) {
+                    const uint4 u0 = *reinterpret_cast<const uint4 *>(src);
+                    const uint4 u1 = *reinterpret_cast<const uint4 *>(src + 16);
+                    w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
+                    w[4] = u1.x; w[5] = u1.y; w[6] = u1.z; w[7] = u1.w;
+                } else if constexpr (BITS == 4) {
+                    const uint4 u0 = *reinterpret_cast<const uint4 *>(src);
+                    w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
+                } else {
+                    const uint2 u0 = *reinterpret_cast<const uint2 *>(src);
+                    w[0] = u0.x; w[1] = u0.y;
+                }
+                uint4 out[4];
+                dequant_half<T, BITS>(w, s16, b16, out);
+                uint8_t *arow = gbase + (a0 - base) + s * A_BYTES + r * 128;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int chunk = 4 * h + j;
+                    *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) = out[j];
+                }
+                ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(full_a + 8 * s);
+            }
+        }
+    } else if (warp < kWarpTma) {
+        // ------------------------- epilogue -------------------------
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        T *y = static_cast<T *>(p.y);
+        int i = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++i) {
+            const int acc = i & 1;
+            const int n0 = (tile / p.m_tiles) * kBM, m0 = (tile % p.m_tiles) * BN;
+            ptx::mbar_wait(acc_full + 8 * acc, (i >> 1) & 1, p.err);
+            tc_fence_after();
+            const int n = n0 + 32 * q + lane;
+            // Columns acc*BN .. acc*BN+BN-1 of this warp's 32 lanes, 32 (or, for
+            // BN = 16, 16) columns per load so no load leaves the allocation.
+            constexpr int CW = BN < 32 ? BN : 32;
+#pragma unroll 1
+            for (int j = 0; j < BN / CW; ++j) {
+                uint32_t v[32];
+                const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + acc * BN + CW * j;
+                if constexpr (CW == 32) tmem_ld32(taddr, v);
+                else tmem_ld16(taddr, v);
+                tmem_ld_wait();
+                if (n < p.N) {
+#pragma unroll
+                    for (int cc = 0; cc < CW; ++cc) {
+                        const int m = m0 + CW * j + cc;
+                        if (m < p.M) y[(int64_t)m * p.N + n] = Dt<T>::from_f(__uint_as_float(v[cc]));
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(acc_empty + 8 * acc);
+        }
+    } else if (warp == kWarpTma) {
+        // ------------------------- producer -------------------------
+        if (lane == 0) {
+            int c = 0;
+            for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+                const int n0 = (tile / p.m_tiles) * kBM, m0 = (tile % p.m_tiles) * BN;
+                for (int kb = 0; kb < KB; ++kb, ++c) {
+                    const int s = c % S;
+                    if (c >= S) ptx::mbar_wait(empty + 8 * s, ((c / S) + 1) & 1, p.err);
+                    ptx::mbar_arrive_expect_tx(full_pb + 8 * s, P_BYTES + B_BYTES);
+                    tma_load_2d(p0 + s * P_BYTES, &tmap_w, kb * W_WORDS, n0, full_pb + 8 * s);
+                    tma_load_2d(b0 + s * B_BYTES, &tmap_x, kb * kBK, m0, full_pb + 8 * s);
+                }
+            }
+            // Drain: wait (bounded) for the last copies to land before exit.
+            for (int d = max(0, c - S); d < c; ++d)
+                ptx::mbar_wait(full_pb + 8 * (d % S), (d / S) & 1, p.err);
+        }
+    } else {
+        // ------------------------- MMA issuer -------------------------
+        if (lane == 0) {
+            int c = 0, i = 0;
+            for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++i) {
+                const int acc = i & 1;
+                if (i >= 2) ptx::mbar_wait(acc_empty + 8 * acc, ((i >> 1) + 1) & 1, p.err);
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * BN;
+                for (int kb = 0; kb < KB; ++kb, ++c) {
+                    const int s = c % S;
+                    ptx::mbar_wait(full_a + 8 * s, (c / S) & 1, p.err);
+                    ptx::mbar_wait(full_pb + 8 * s, (c / S) & 1, p.err);
+                    tc_fence_after();
+                    const uint64_t da = sw128_desc(a0 + s * A_BYTES);
+                    const uint64_t db = sw128_desc(b0 + s * B_BYTES);
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)  // UMMA K = 16: 32 bytes along the row
+                        tc_mma(d, da + 2 * k, db + 2 * k, IDESC, (kb | k) != 0);
+                    tc_commit(empty + 8 * s);
+                }
+                tc_commit(acc_full + 8 * acc);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *ptr, uint64_t inner,
+                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int pick_bn(int64_t M) {
+    if (M <= 16) return 16;
+    if (M <= 32) return 32;
+    if (M <= 64) return 64;
+    if (M <= 128) return 128;
+    return 256;
+}
+
+template <typename T, int BITS, int BN>
+cudaError_t run_gemm(const QmmArgs &a, cudaStream_t s) {
+    constexpr int A_BYTES = kBM * kBK * 2, B_BYTES = BN * kBK * 2, P_BYTES = kBM * kBK * BITS / 8;
+    constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
+    constexpr size_t kSmemMax = 227 * 1024;
+    const size_t fixed = 1024 /*alignment*/ + 64 /*acc bars + slot*/;
+    int stages = (int)std::min<size_t>(8, (kSmemMax - fixed) / (STAGE + 24));
+    if (stages < 2) return cudaErrorInvalidConfiguration;
+    const size_t smem = fixed + (size_t)stages * (STAGE + 24);
+
+    CUtensorMap tx, tw;
+    const CUtensorMapDataType xdt =
+        std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!make_map_2d(&tx, xdt, a.x, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * 2, kBK, BN,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    const uint64_t words = (uint64_t)a.K * BITS / 32;
+    if (!make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.wq, words, (uint64_t)a.N, words * 4,
+                     kBK * BITS / 32, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+
+    GemmParams p{};
+    p.scales = a.scales;
+    p.biases = a.biases;
+    p.y = a.y;
+    p.M = (int)a.M;
+    p.N = (int)a.N;
+    p.K = (int)a.K;
+    p.group_size = a.group_size;
+    p.m_tiles = (int)((a.M + BN - 1) / BN);
+    p.n_tiles = (int)((a.N + kBM - 1) / kBM);
+    p.num_tiles = p.m_tiles * p.n_tiles;
+    p.stages = stages;
+    p.err = device_error_word();
+    auto kern = qgemm_tc_kernel<T, BITS, BN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = std::min(p.num_tiles, num_sms());
+    kern<<<grid, kThreads, smem, s>>>(tx, tw, p);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+template <typename T, int BITS>
+cudaError_t gemm_bits(const QmmArgs &a, cudaStream_t s) {
+    switch (pick_bn(a.M)) {
+    case 16: return run_gemm<T, BITS, 16>(a, s);
+    case 32: return run_gemm<T, BITS, 32>(a, s);
+    case 64: return run_gemm<T, BITS, 64>(a, s);
+    case 128: return run_gemm<T, BITS, 128>(a, s);
+    default: return run_gemm<T, BITS, 256>(a, s);
+    }
+}
+
+}  // namespace
+
+// The tensor-core path: bf16/f16, transpose layout, K a multiple of the
+// 64-wide k-block, whole 16-byte packed rows, sizes in int range.
+bool gemm_supported(qmm_dtype dt, const QmmArgs &a) {
+    if (!a.transpose) return false;
+    if (dt != QMM_BF16 && dt != QMM_F16) return false;
+    if (a.K % kBK != 0) return false;
+    if ((a.K * a.bits / 8) % 16 != 0) return false;
+    if (a.M > INT32_MAX / 2 || a.N > INT32_MAX / 2 || a.K > INT32_MAX / 2) return false;
+    return encode_fn() != nullptr;
+}
+
+cudaError_t launch_gemm(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
+    if (dt == QMM_BF16) {
+        switch (a.bits) {
+        case 2: return gemm_bits<__nv_bfloat16, 2>(a, s);
+        case 4: return gemm_bits<__nv_bfloat16, 4>(a, s);
+        default: return gemm_bits<__nv_bfloat16, 8>(a, s);
+        }
+    }
+    switch (a.bits) {
+    case 2: return gemm_bits<__half, 2>(a, s);
+    case 4: return gemm_bits<__half, 4>(a, s);
+    default: return gemm_bits<__half, 8>(a, s);
+    }
+}
+
+}  // namespace qmm

@@ -75,6 +75,8 @@ cudaError_t launch_gemv(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 bool gemv_supported(qmm_dtype dt, const QmmArgs &a);
 cudaError_t launch_gemv_fast(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a);
+cudaError_t launch_gemm(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
+bool gemm_supported(qmm_dtype dt, const QmmArgs &a);
 
 int num_sms();
 void count_launches(int n);  // bump the process-wide launch counter

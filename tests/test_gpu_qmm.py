@@ -104,3 +104,44 @@ def test_gemv_few_rows(dtype, bits, gs, n, k, m):
     w = wl.with_outliers((n, k), seed=n + k + bits, dtype=dtype)
     x = wl.normal((m, k), seed=k + m, dtype=dtype)
     run_case(x, w, gs, bits, True)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("bits,gs", [(4, 64), (4, 32), (4, 128), (8, 64), (8, 32), (2, 128), (2, 64)])
+@pytest.mark.parametrize("m,n,k", [(1, 128, 64), (16, 200, 1024), (17, 256, 128),
+                                   (100, 1000, 512), (300, 384, 256)])
+def test_gemm_tensor_core(dtype, bits, gs, m, n, k):
+    """The tcgen05 path: ragged activation rows (every tile width from 16 to
+    256), ragged weight rows, several k-blocks."""
+    if k % gs:
+        pytest.skip("K must be a multiple of the group size")
+    w = wl.with_outliers((n, k), seed=m + n + bits, dtype=dtype)
+    x = wl.normal((m, k), seed=k + m, dtype=dtype)
+    run_case(x, w, gs, bits, True, "gemm")
+
+
+def test_gemm_path_refuses_unsupported():
+    w = wl.normal((64, 96), 1, 1.0, torch.bfloat16)
+    wq, s, b = oracle.quantize(w, 32, 4)
+    x = wl.normal((8, 96), 2, 1.0, torch.bfloat16).cuda()
+    qb.qmm_set_path("gemm")
+    with pytest.raises(qb.QmmError) as e:
+        qb.qmm_quantized_matmul(x, wq.cuda(), s.cuda(), b.cuda(), True, 32, 4)
+    assert e.value.status == 2
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("bits", [4, 8])
+def test_prefill_full_size_sampled(bits):
+    """x [2048, 4096] against W [14336, 4096] (the prefill workload), checked
+    on 96 sampled activation rows spread over every 256-row tile."""
+    c = wl.prefill_case(bits)
+    wq, s, b = oracle.quantize(c.w, c.group_size, c.bits)
+    y = qb.qmm_quantized_matmul(c.x.cuda(), wq.cuda(), s.cuda(), b.cuda(), True, c.group_size,
+                                c.bits)
+    torch.cuda.synchronize()
+    rows = torch.cat([torch.arange(0, 2048, 256) + o for o in (0, 1, 37, 100, 128, 200, 254, 255,
+                                                                 17, 64, 190, 222)])
+    ref = oracle.quantized_matmul(c.x[rows], wq, s, b, True, c.group_size, c.bits)
+    err = row_rel_err(y.cpu()[rows], ref)
+    assert err <= REL_TOL[torch.bfloat16], f"rel err {err}"
