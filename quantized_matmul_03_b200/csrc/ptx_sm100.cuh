@@ -59,6 +59,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *err) {
     if (mbar_try_wait(bar, parity)) return true;
+    // Once any wait has given up, do not wait again: finish quickly.
+    if (*reinterpret_cast<volatile int *>(err) != 0) return false;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (globaltimer_ns() - t0 > kWaitNs) {
