@@ -362,6 +362,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time only the prefill GEMM (for profiling); prints its own line")
+    ap.add_argument("--prefill-bits", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
     args = ap.parse_args()
@@ -376,6 +379,16 @@ def main():
     qb.lib()  # fails loudly if the library was not built
     device = torch.device("cuda", local)
     pk = peaks()
+
+    if args.prefill_only:
+        pre = bench_prefill(args.prefill_bits, args.steps, args.warmup, world, device)
+        p_ms = max_over_ranks(world, pre["per_ms"])
+        tf = pre["flops"] / (p_ms * 1e-3) / 1e12
+        if rank == 0:
+            print(json.dumps({"workload": f"prefill_m2048_int{args.prefill_bits}_gs64",
+                              "value": tf, "unit": "TFLOP/s", "kernel_us": p_ms * 1e3,
+                              "frac": tf / pk["bf16_tflops"], "launches": pre["launches"]}))
+        return 0
 
     with ClockSampler(local) as clk:
         d = bench_decode(1, args.steps, args.warmup, world, device)
