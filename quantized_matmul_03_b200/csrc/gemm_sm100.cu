@@ -219,6 +219,12 @@ __device__ __forceinline__ void dequant_half<__nv_bfloat16, 8>(const uint32_t *w
         out[c] = make_uint4(vals[4 * c], vals[4 * c + 1], vals[4 * c + 2], vals[4 * c + 3]);
 }
 
+// v.x / v.y / v.z / v.w by a runtime index without indexing registers.
+__device__ __forceinline__ uint32_t pick_word(const uint4 &v, int i) {
+    const uint32_t lo = (i & 1) ? v.y : v.x, hi = (i & 1) ? v.w : v.z;
+    return (i & 2) ? hi : lo;
+}
+
 struct GemmParams {
     const void *scales, *biases;
     void *y;
@@ -279,22 +285,52 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
 
     if (warp < kDqWarps) {
         // ------------------------- dequantize -------------------------
-        const int r = threadIdx.x & (kBM - 1), h = threadIdx.x >> 7;  // row, k half
+        // Adjacent lanes take the two halves of one row, so a warp's packed
+        // reads are contiguous and its swizzled A writes hit distinct banks.
+        const int h = threadIdx.x & 1, r = threadIdx.x >> 1;  // k half, row
         const uint16_t *sc = static_cast<const uint16_t *>(p.scales);
         const uint16_t *bi = static_cast<const uint16_t *>(p.biases);
+        // Scales/biases are read 8 groups (16 bytes) at a time, one window
+        // ahead of use, when rows are whole 16-byte units; else one by one.
+        const bool vec = (gpr % 8) == 0;
         int c = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
             const int n0 = (tile / p.m_tiles) * kBM;
             const int n = n0 + r;
             const bool rv = n < p.N;
+            const uint16_t *srow = sc + (int64_t)n * gpr, *brow = bi + (int64_t)n * gpr;
+            uint4 s_cur = make_uint4(0, 0, 0, 0), b_cur = s_cur, s_nxt = s_cur, b_nxt = s_cur;
+            int wbase = 0;  // first group of the current window
+            if (vec && rv) {
+                s_cur = __ldg(reinterpret_cast<const uint4 *>(srow));
+                b_cur = __ldg(reinterpret_cast<const uint4 *>(brow));
+                if (gpr > 8) {
+                    s_nxt = __ldg(reinterpret_cast<const uint4 *>(srow + 8));
+                    b_nxt = __ldg(reinterpret_cast<const uint4 *>(brow + 8));
+                }
+            }
             for (int kb = 0; kb < KB; ++kb, ++c) {
                 const int s = c % S;
                 const int k0 = kb * kBK + 32 * h;
+                const int g = k0 / p.group_size;
                 uint16_t s16 = 0, b16 = 0;
-                if (rv && k0 < p.K) {
-                    const int64_t gi = (int64_t)n * gpr + k0 / p.group_size;
-                    s16 = __ldg(sc + gi);
-                    b16 = __ldg(bi + gi);
+                if (vec) {
+                    if (g >= wbase + 8) {  // advance the window, fetch the one after
+                        s_cur = s_nxt;
+                        b_cur = b_nxt;
+                        wbase += 8;
+                        if (rv && wbase + 8 < gpr) {
+                            s_nxt = __ldg(reinterpret_cast<const uint4 *>(srow + wbase + 8));
+                            b_nxt = __ldg(reinterpret_cast<const uint4 *>(brow + wbase + 8));
+                        }
+                    }
+                    const int o = g - wbase;
+                    const uint32_t sw = pick_word(s_cur, o >> 1), bw = pick_word(b_cur, o >> 1);
+                    s16 = (uint16_t)((o & 1) ? (sw >> 16) : (sw & 0xffffu));
+                    b16 = (uint16_t)((o & 1) ? (bw >> 16) : (bw & 0xffffu));
+                } else if (rv) {
+                    s16 = __ldg(srow + g);
+                    b16 = __ldg(brow + g);
                 }
                 ptx::mbar_wait(full_pb + 8 * s, (c / S) & 1, p.err);
                 uint32_t w[BITS];  // 32 codes = BITS words
