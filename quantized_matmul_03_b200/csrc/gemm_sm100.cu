@@ -13,10 +13,11 @@
 // (8-row x 128-byte atoms, row r's 16-byte chunk c at chunk c ^ (r mod 8)).
 //
 // Roles (one CTA per SM, persistent over output tiles):
-//   warps 0-7   dequantize: thread t owns weight row t mod 128 and half t / 128
-//               of the k-block; it reads the packed codes the producer staged,
-//               forms s*q + b two codes at a time (bf16x2/f16x2 FMA, one
-//               rounding), and writes the swizzled A tile;
+//   warps 0-7   dequantize, as two groups of four warps taking alternate
+//               k-blocks; thread r of a group owns weight row r, reads the
+//               packed codes the producer staged, forms s*q + b two codes at a
+//               time (bf16x2/f16x2 FMA, one rounding), and writes the
+//               swizzled A tile;
 //   warps 8-11  epilogue: tcgen05.ld of the accumulator quadrant the warp may
 //               address (lanes 32*(warp%4)..), convert, store y;
 //   warp 12     producer: TMA loads of the packed weight tile and the
@@ -263,7 +264,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             ptx::mbar_init(full_pb + 8 * s, 1);
-            ptx::mbar_init(full_a + 8 * s, kDqWarps);
+            ptx::mbar_init(full_a + 8 * s, kDqWarps / 2);  // one dequant group per k-block
             ptx::mbar_init(empty + 8 * s, 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -285,9 +286,9 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
 
     if (warp < kDqWarps) {
         // ------------------------- dequantize -------------------------
-        // Adjacent lanes take the two halves of one row, so a warp's packed
-        // reads are contiguous and its swizzled A writes hit distinct banks.
-        const int h = threadIdx.x & 1, r = threadIdx.x >> 1;  // k half, row
+        // Two groups of four warps take alternate k-blocks, so two k-blocks
+        // are dequantized at once; thread r of a group owns weight row r.
+        const int grp = warp >> 2, r = threadIdx.x & (kBM - 1);
         const uint16_t *sc = static_cast<const uint16_t *>(p.scales);
         const uint16_t *bi = static_cast<const uint16_t *>(p.biases);
         // Scales/biases are read 8 groups (16 bytes) at a time, one window
@@ -309,13 +310,9 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     b_nxt = __ldg(reinterpret_cast<const uint4 *>(brow + 8));
                 }
             }
-            for (int kb = 0; kb < KB; ++kb, ++c) {
-                const int s = c % S;
-                const int k0 = kb * kBK + 32 * h;
-                const int g = k0 / p.group_size;
-                uint16_t s16 = 0, b16 = 0;
+            auto scale_bias = [&](int g, uint16_t &s16, uint16_t &b16) {
                 if (vec) {
-                    if (g >= wbase + 8) {  // advance the window, fetch the one after
+                    while (g >= wbase + 8) {  // advance the window, fetch the one after
                         s_cur = s_nxt;
                         b_cur = b_nxt;
                         wbase += 8;
@@ -328,32 +325,52 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     const uint32_t sw = pick_word(s_cur, o >> 1), bw = pick_word(b_cur, o >> 1);
                     s16 = (uint16_t)((o & 1) ? (sw >> 16) : (sw & 0xffffu));
                     b16 = (uint16_t)((o & 1) ? (bw >> 16) : (bw & 0xffffu));
-                } else if (rv) {
-                    s16 = __ldg(srow + g);
-                    b16 = __ldg(brow + g);
-                }
-                ptx::mbar_wait(full_pb + 8 * s, (c / S) & 1, p.err);
-                uint32_t w[BITS];  // 32 codes = BITS words
-                const uint8_t *src = pg + s * P_BYTES + r * P_ROW + h * (P_ROW / 2);
-                if constexpr (BITS == 8) {
-                    const uint4 u0 = *reinterpret_cast<const uint4 *>(src);
-                    const uint4 u1 = *reinterpret_cast<const uint4 *>(src + 16);
-                    w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
-                    w[4] = u1.x; w[5] = u1.y; w[6] = u1.z; w[7] = u1.w;
-                } else if constexpr (BITS == 4) {
-                    const uint4 u0 = *reinterpret_cast<const uint4 *>(src);
-                    w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
                 } else {
-                    const uint2 u0 = *reinterpret_cast<const uint2 *>(src);
-                    w[0] = u0.x; w[1] = u0.y;
+                    s16 = rv ? __ldg(srow + g) : (uint16_t)0;
+                    b16 = rv ? __ldg(brow + g) : (uint16_t)0;
                 }
-                uint4 out[4];
-                dequant_half<T, BITS>(w, s16, b16, out);
+            };
+            for (int kb = 0; kb < KB; ++kb, ++c) {
+                if ((c & 1) != grp) continue;
+                const int s = c % S;
+                uint16_t s0, b0v, s1, b1v;
+                scale_bias((kb * kBK) / p.group_size, s0, b0v);
+                scale_bias((kb * kBK + 32) / p.group_size, s1, b1v);
+                ptx::mbar_wait(full_pb + 8 * s, (c / S) & 1, p.err);
+                // The packed tile was staged with the swizzle matching its row
+                // width (none / 32B / 64B): 16-byte chunk q of row r sits at
+                // chunk q ^ ((r >> 2) & 1) (32-byte rows) or q ^ ((r >> 1) & 3)
+                // (64-byte rows).
+                const uint8_t *prow = pg + s * P_BYTES + r * P_ROW;
+                uint32_t w[2 * BITS];  // 64 codes
+                if constexpr (BITS == 2) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(prow);
+                    w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+                } else if constexpr (BITS == 4) {
+                    const int x = (r >> 2) & 1;
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(prow + ((q ^ x) << 4));
+                        w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
+                    }
+                } else {
+                    const int x = (r >> 1) & 3;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(prow + ((q ^ x) << 4));
+                        w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
+                    }
+                }
                 uint8_t *arow = gbase + (a0 - base) + s * A_BYTES + r * 128;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int chunk = 4 * h + j;
-                    *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) = out[j];
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint4 out[4];
+                    dequant_half<T, BITS>(w + hh * BITS, hh ? s1 : s0, hh ? b1v : b0v, out);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int chunk = 4 * hh + j;
+                        *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) = out[j];
+                    }
                 }
                 ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
                 __syncwarp();
@@ -506,7 +523,9 @@ cudaError_t run_gemm(const QmmArgs &a, cudaStream_t s) {
         return cudaErrorInvalidValue;
     const uint64_t words = (uint64_t)a.K * BITS / 32;
     if (!make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.wq, words, (uint64_t)a.N, words * 4,
-                     kBK * BITS / 32, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
+                     kBK * BITS / 32, kBM,
+                     BITS == 2 ? CU_TENSOR_MAP_SWIZZLE_NONE
+                               : (BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B)))
         return cudaErrorInvalidValue;
 
     GemmParams p{};
