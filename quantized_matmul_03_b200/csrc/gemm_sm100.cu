@@ -350,7 +350,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 uint16_t s0, b0v, s1, b1v;
                 scale_bias((kb * kBK) / p.group_size, s0, b0v);
                 scale_bias((kb * kBK + 32) / p.group_size, s1, b1v);
-                ptx::mbar_wait(full_p + 8 * sp, (c / SP) & 1, p.err);
+                ptx::mbar_wait<false>(full_p + 8 * sp, (c / SP) & 1, p.err);
                 // The packed tile was staged with the swizzle matching its row
                 // width (none / 32B / 64B): 16-byte chunk q of row r sits at
                 // chunk q ^ ((r >> 2) & 1) (32-byte rows) or q ^ ((r >> 1) & 3)
@@ -379,7 +379,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 // until the MMA of k-block c - SA has freed the A slot.
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(empty_p + 8 * sp);
-                if (c >= SA) ptx::mbar_wait(empty_a + 8 * sa, ((c / SA) + 1) & 1, p.err);
+                if (c >= SA) ptx::mbar_wait<false>(empty_a + 8 * sa, ((c / SA) + 1) & 1, p.err);
                 uint8_t *arow = gbase + (a0 - base) + sa * A_BYTES + r * 128;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -443,7 +443,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 const int n0 = (tile / p.m_tiles) * kBM, m0 = (tile % p.m_tiles) * BN;
                 for (int kb = 0; kb < KB; ++kb, ++c) {
                     const int s = c % R;
-                    if (c >= R) ptx::mbar_wait(emptyb + 8 * s, ((c / R) + 1) & 1, p.err);
+                    if (c >= R) ptx::mbar_wait<false>(emptyb + 8 * s, ((c / R) + 1) & 1, p.err);
                     if (wp) {
                         ptx::mbar_arrive_expect_tx(fullb + 8 * s, P_BYTES);
                         tma_load_2d(p0 + s * P_BYTES, &tmap_w, kb * W_WORDS, n0, fullb + 8 * s);
@@ -468,8 +468,8 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 const uint32_t d = tmem_base + acc * BN;
                 for (int kb = 0; kb < KB; ++kb, ++c) {
                     const int sa = c % SA, sb = c % SB;
-                    ptx::mbar_wait(full_a + 8 * sa, (c / SA) & 1, p.err);
-                    ptx::mbar_wait(full_b + 8 * sb, (c / SB) & 1, p.err);
+                    ptx::mbar_wait<false>(full_a + 8 * sa, (c / SA) & 1, p.err);
+                    ptx::mbar_wait<false>(full_b + 8 * sb, (c / SB) & 1, p.err);
                     tc_fence_after();
                     const uint64_t da = sw128_desc(a0 + sa * A_BYTES);
                     const uint64_t db = sw128_desc(b0 + sb * B_BYTES);

@@ -37,6 +37,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
 }
+// Test the phase once, without blocking.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 // Test the phase; if it is not complete, the thread may be suspended for up
 // to ~1 ms (or until the phase completes, whichever is first) instead of
 // spinning, so waiting warps leave the issue slots to working ones.
@@ -56,19 +68,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // On timeout the device error word gets QMM_ERR_TIMEOUT and false is
 // returned; callers then carry on without the data (their shared-memory
 // accesses stay in bounds), so every thread still reaches the kernel's end.
+// SLEEP selects suspending waits (long, off the critical path) or spinning
+// ones (short hand-offs where a wake-up delay would cost throughput).
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
+template <bool SLEEP = true>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *err) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test(bar, parity)) return true;
     // Once any wait has given up, do not wait again: finish quickly.
     if (*reinterpret_cast<volatile int *>(err) != 0) return false;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (SLEEP ? mbar_try_wait(bar, parity) : mbar_test(bar, parity)) return true;
         if (globaltimer_ns() - t0 > kWaitNs) {
             record_device_error(err, QMM_ERR_TIMEOUT);
             return false;
         }
     }
-    return true;
 }
 
 // ---- programmatic dependent launch -----------------------------------------
