@@ -13,11 +13,10 @@
 // (8-row x 128-byte atoms, row r's 16-byte chunk c at chunk c ^ (r mod 8)).
 //
 // Roles (one CTA per SM, persistent over output tiles):
-//   warps 0-7   dequantize, as two groups of four warps taking alternate
-//               k-blocks; thread r of a group owns weight row r, reads the
-//               packed codes the producer staged, forms s*q + b two codes at a
-//               time (bf16x2/f16x2 FMA, one rounding), and writes the
-//               swizzled A tile;
+//   warps 0-7   dequantize: lanes 2r and 2r+1 own the two 32-code halves of
+//               weight row r of the k-block; each reads the packed codes the
+//               producer staged, forms s*q + b two codes at a time (bf16x2 or
+//               f16x2 FMA, one rounding), and writes the swizzled A tile;
 //   warps 8-11  epilogue: tcgen05.ld of the accumulator quadrant the warp may
 //               address (lanes 32*(warp%4)..), convert, store y;
 //   warps 12,14 producers: TMA loads of the packed weight tiles (ring P,
@@ -270,7 +269,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < SA; ++s) {
-            ptx::mbar_init(full_a + 8 * s, kDqWarps / 2);  // the dequant group of the k-block
+            ptx::mbar_init(full_a + 8 * s, kDqWarps);      // every dequant warp
             ptx::mbar_init(empty_a + 8 * s, 1);             // MMA commit
         }
         for (int s = 0; s < SB; ++s) {
@@ -279,7 +278,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         }
         for (int s = 0; s < SP; ++s) {
             ptx::mbar_init(full_p + 8 * s, 1);              // producer + TMA bytes
-            ptx::mbar_init(empty_p + 8 * s, kDqWarps / 2);  // the group has read the codes
+            ptx::mbar_init(empty_p + 8 * s, kDqWarps);      // every dequant warp has read its codes
         }
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(acc_full + 8 * a, 1);
@@ -300,9 +299,10 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
 
     if (warp < kDqWarps) {
         // ------------------------- dequantize -------------------------
-        // Two groups of four warps take alternate k-blocks, so two k-blocks
-        // are dequantized at once; thread r of a group owns weight row r.
-        const int grp = warp >> 2, r = threadIdx.x & (kBM - 1);
+        // All eight warps work on each k-block: adjacent lanes take the two
+        // 32-code halves of one weight row, so the per-k-block latency (on the
+        // MMA's critical path) is that of 32 codes per thread.
+        const int h = threadIdx.x & 1, r = threadIdx.x >> 1;  // k half, row
         const uint16_t *sc = static_cast<const uint16_t *>(p.scales);
         const uint16_t *bi = static_cast<const uint16_t *>(p.biases);
         // Scales/biases are read 8 groups (16 bytes) at a time, one window
@@ -345,33 +345,27 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 }
             };
             for (int kb = 0; kb < KB; ++kb, ++c) {
-                if ((c & 1) != grp) continue;
                 const int sp = c % SP, sa = c % SA;
-                uint16_t s0, b0v, s1, b1v;
-                scale_bias((kb * kBK) / p.group_size, s0, b0v);
-                scale_bias((kb * kBK + 32) / p.group_size, s1, b1v);
+                uint16_t s16, b16;
+                scale_bias((kb * kBK + 32 * h) / p.group_size, s16, b16);
                 ptx::mbar_wait<false>(full_p + 8 * sp, (c / SP) & 1, p.err);
                 // The packed tile was staged with the swizzle matching its row
                 // width (none / 32B / 64B): 16-byte chunk q of row r sits at
                 // chunk q ^ ((r >> 2) & 1) (32-byte rows) or q ^ ((r >> 1) & 3)
                 // (64-byte rows).
                 const uint8_t *prow = pg + sp * P_BYTES + r * P_ROW;
-                uint32_t w[2 * BITS];  // 64 codes
+                uint32_t w[BITS];  // this half's 32 codes
                 if constexpr (BITS == 2) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(prow);
-                    w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+                    const uint2 u = *reinterpret_cast<const uint2 *>(prow + 8 * h);
+                    w[0] = u.x; w[1] = u.y;
                 } else if constexpr (BITS == 4) {
-                    const int x = (r >> 2) & 1;
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const uint4 u = *reinterpret_cast<const uint4 *>(prow + ((q ^ x) << 4));
-                        w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
-                    }
+                    const uint4 u = *reinterpret_cast<const uint4 *>(prow + ((h ^ ((r >> 2) & 1)) << 4));
+                    w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
                 } else {
                     const int x = (r >> 1) & 3;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 u = *reinterpret_cast<const uint4 *>(prow + ((q ^ x) << 4));
+                    for (int q = 0; q < 2; ++q) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(prow + (((2 * h + q) ^ x) << 4));
                         w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
                     }
                 }
@@ -379,17 +373,14 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 // until the MMA of k-block c - SA has freed the A slot.
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(empty_p + 8 * sp);
+                uint4 out[4];
+                dequant_half<T, BITS>(w, s16, b16, out);
                 if (c >= SA) ptx::mbar_wait<false>(empty_a + 8 * sa, ((c / SA) + 1) & 1, p.err);
                 uint8_t *arow = gbase + (a0 - base) + sa * A_BYTES + r * 128;
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint4 out[4];
-                    dequant_half<T, BITS>(w + hh * BITS, hh ? s1 : s0, hh ? b1v : b0v, out);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int chunk = 4 * hh + j;
-                        *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) = out[j];
-                    }
+                for (int j = 0; j < 4; ++j) {
+                    const int chunk = 4 * h + j;
+                    *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) = out[j];
                 }
                 ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
                 __syncwarp();
@@ -541,11 +532,16 @@ cudaError_t run_gemm(const QmmArgs &a, cudaStream_t s) {
     constexpr size_t kSmemMax = 227 * 1024;
     const size_t fixed = 1024 /*alignment*/ + 64 /*accumulator barriers + tmem slot*/;
     // Packed tiles are small and freed early: keep a deep ring (up to 8, at
-    // most 32 KB); three dequantized tiles; the activation ring takes the rest.
-    const int sa = 3;
+    // most 32 KB); four dequantized tiles if the activation ring keeps four
+    // stages, else three; the activation ring takes the rest.
     const int sp = std::min(8, std::max(2, (int)(32768 / P_BYTES)));
-    const size_t rest = kSmemMax - fixed - (size_t)sa * (A_BYTES + 16) - (size_t)sp * (P_BYTES + 16);
-    const int sb = (int)std::min<size_t>(8, rest / (B_BYTES + 16));
+    int sa = 4, sb = 0;
+    for (; sa >= 3; --sa) {
+        const size_t rest =
+            kSmemMax - fixed - (size_t)sa * (A_BYTES + 16) - (size_t)sp * (P_BYTES + 16);
+        sb = (int)std::min<size_t>(8, rest / (B_BYTES + 16));
+        if (sb >= 4) break;
+    }
     if (sb < 2) return cudaErrorInvalidConfiguration;
     const size_t smem = fixed + (size_t)sa * (A_BYTES + 16) + (size_t)sb * (B_BYTES + 16) +
                         (size_t)sp * (P_BYTES + 16);
