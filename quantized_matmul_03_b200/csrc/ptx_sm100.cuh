@@ -74,16 +74,18 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
 template <bool SLEEP = true>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *err) {
     if (mbar_test(bar, parity)) return true;
-    // Once any wait has given up, do not wait again: finish quickly.
-    if (*reinterpret_cast<volatile int *>(err) != 0) return false;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         for (int i = 0; i < 64; ++i)
             if (SLEEP ? mbar_try_wait(bar, parity) : mbar_test(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitNs) {
+        const uint64_t dt = globaltimer_ns() - t0;
+        if (dt > kWaitNs) {
             record_device_error(err, QMM_ERR_TIMEOUT);
             return false;
         }
+        // After 1 ms, give up at once if another wait already timed out (the
+        // error word is global memory: never read it on the fast path).
+        if (dt > 1000000ull && *reinterpret_cast<volatile int *>(err) != 0) return false;
     }
 }
 
