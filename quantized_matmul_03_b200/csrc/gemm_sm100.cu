@@ -13,18 +13,16 @@
 // (8-row x 128-byte atoms, row r's 16-byte chunk c at chunk c ^ (r mod 8)).
 //
 // Roles (one CTA per SM, persistent over output tiles):
-//   warps 0-7   dequantize: lanes 2r and 2r+1 own the two 32-code halves of
-//               weight row r of the k-block; each reads the packed codes the
-//               producer staged, forms s*q + b two codes at a time (bf16x2 or
-//               f16x2 FMA, one rounding), and writes the swizzled A tile;
+//   warps 0-7   dequantize, as two groups of four warps taking alternate
+//               k-blocks; thread r of a group owns weight row r, reads the
+//               packed codes the producer staged, forms s*q + b two codes at a
+//               time (bf16x2/f16x2 FMA, one rounding), and writes the
+//               swizzled A tile;
 //   warps 8-11  epilogue: tcgen05.ld of the accumulator quadrant the warp may
 //               address (lanes 32*(warp%4)..), convert, store y;
-//   warps 12,14 producers: TMA loads of the packed weight tiles (ring P,
-//               freed once the dequantizers have read them) and of the
-//               activation tiles (ring B, freed by the MMA);
+//   warp 12     producer: TMA loads of the packed weight tile and the
+//               activation tile for each k-block into a ring of stages;
 //   warp 13     MMA issuer (one thread) and TMEM owner.
-// The dequantized tiles have their own ring (A, freed by the MMA), so the
-// dequantizers wait only for an A slot, never for activation traffic.
 // Every wait is a bounded mbarrier wait (device error word on timeout); no
 // cluster multicast is used.
 #include <cuda.h>
@@ -41,10 +39,9 @@ namespace {
 
 constexpr int kDqWarps = 8;
 constexpr int kEpiWarps = 4;
-constexpr int kWarpTma = kDqWarps + kEpiWarps;  // 12: packed-weight producer
-constexpr int kWarpMma = kWarpTma + 1;          // 13: MMA issuer, TMEM owner
-constexpr int kWarpTmaX = kWarpMma + 1;         // 14: activation producer
-constexpr int kThreads = 32 * (kWarpTmaX + 1);  // 480
+constexpr int kWarpTma = kDqWarps + kEpiWarps;  // 12
+constexpr int kWarpMma = kWarpTma + 1;          // 13
+constexpr int kThreads = 32 * (kWarpMma + 1);   // 448
 constexpr int kBM = 128;                        // weight rows per tile (UMMA M)
 constexpr int kBK = 64;                         // k per stage: one 128-byte swizzle row
 
@@ -233,8 +230,7 @@ struct GemmParams {
     const void *scales, *biases;
     void *y;
     int M, N, K, group_size;
-    int m_tiles, n_tiles, num_tiles;
-    int stages_a, stages_b, stages_p;  // ring depths: dequantized, activation, packed tiles
+    int m_tiles, n_tiles, num_tiles, stages;
     int *err;
 };
 
@@ -252,33 +248,24 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     constexpr uint32_t IDESC = make_idesc(kF16, kBM, BN);
 
     extern __shared__ uint8_t smem_raw[];
-    const int SA = p.stages_a, SB = p.stages_b, SP = p.stages_p;
-    // 1024-byte aligned carve-up: A[SA] | B[SB] | P[SP] | barriers | tmem slot
+    const int S = p.stages;
+    // 1024-byte aligned carve-up: A[S] | B[S] | P[S] | barriers | tmem slot
     const uint32_t raw = ptx::smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
-    const uint32_t a0 = base, b0 = a0 + SA * A_BYTES, p0 = b0 + SB * B_BYTES;
-    const uint32_t bar0 = p0 + SP * P_BYTES;
-    const uint32_t full_a = bar0, empty_a = full_a + 8 * SA;
-    const uint32_t full_b = empty_a + 8 * SA, empty_b = full_b + 8 * SB;
-    const uint32_t full_p = empty_b + 8 * SB, empty_p = full_p + 8 * SP;
-    const uint32_t acc_full = empty_p + 8 * SP, acc_empty = acc_full + 16;
+    const uint32_t a0 = base, b0 = a0 + S * A_BYTES, p0 = b0 + S * B_BYTES;
+    const uint32_t bar0 = p0 + S * P_BYTES;
+    const uint32_t full_pb = bar0, full_a = bar0 + 8 * S, empty = bar0 + 16 * S;
+    const uint32_t acc_full = bar0 + 24 * S, acc_empty = acc_full + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + (acc_empty + 16 - base));
     const uint8_t *pg = gbase + (p0 - base);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < SA; ++s) {
-            ptx::mbar_init(full_a + 8 * s, kDqWarps);      // every dequant warp
-            ptx::mbar_init(empty_a + 8 * s, 1);             // MMA commit
-        }
-        for (int s = 0; s < SB; ++s) {
-            ptx::mbar_init(full_b + 8 * s, 1);              // producer + TMA bytes
-            ptx::mbar_init(empty_b + 8 * s, 1);             // MMA commit
-        }
-        for (int s = 0; s < SP; ++s) {
-            ptx::mbar_init(full_p + 8 * s, 1);              // producer + TMA bytes
-            ptx::mbar_init(empty_p + 8 * s, kDqWarps);      // every dequant warp has read its codes
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(full_pb + 8 * s, 1);
+            ptx::mbar_init(full_a + 8 * s, kDqWarps / 2);  // one dequant group per k-block
+            ptx::mbar_init(empty + 8 * s, 1);
         }
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(acc_full + 8 * a, 1);
@@ -299,10 +286,9 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
 
     if (warp < kDqWarps) {
         // ------------------------- dequantize -------------------------
-        // All eight warps work on each k-block: adjacent lanes take the two
-        // 32-code halves of one weight row, so the per-k-block latency (on the
-        // MMA's critical path) is that of 32 codes per thread.
-        const int h = threadIdx.x & 1, r = threadIdx.x >> 1;  // k half, row
+        // Two groups of four warps take alternate k-blocks, so two k-blocks
+        // are dequantized at once; thread r of a group owns weight row r.
+        const int grp = warp >> 2, r = threadIdx.x & (kBM - 1);
         const uint16_t *sc = static_cast<const uint16_t *>(p.scales);
         const uint16_t *bi = static_cast<const uint16_t *>(p.biases);
         // Scales/biases are read 8 groups (16 bytes) at a time, one window
@@ -345,46 +331,50 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 }
             };
             for (int kb = 0; kb < KB; ++kb, ++c) {
-                const int sp = c % SP, sa = c % SA;
-                uint16_t s16, b16;
-                scale_bias((kb * kBK + 32 * h) / p.group_size, s16, b16);
-                ptx::mbar_wait<false>(full_p + 8 * sp, (c / SP) & 1, p.err);
+                if ((c & 1) != grp) continue;
+                const int s = c % S;
+                uint16_t s0, b0v, s1, b1v;
+                scale_bias((kb * kBK) / p.group_size, s0, b0v);
+                scale_bias((kb * kBK + 32) / p.group_size, s1, b1v);
+                ptx::mbar_wait(full_pb + 8 * s, (c / S) & 1, p.err);
                 // The packed tile was staged with the swizzle matching its row
                 // width (none / 32B / 64B): 16-byte chunk q of row r sits at
                 // chunk q ^ ((r >> 2) & 1) (32-byte rows) or q ^ ((r >> 1) & 3)
                 // (64-byte rows).
-                const uint8_t *prow = pg + sp * P_BYTES + r * P_ROW;
-                uint32_t w[BITS];  // this half's 32 codes
+                const uint8_t *prow = pg + s * P_BYTES + r * P_ROW;
+                uint32_t w[2 * BITS];  // 64 codes
                 if constexpr (BITS == 2) {
-                    const uint2 u = *reinterpret_cast<const uint2 *>(prow + 8 * h);
-                    w[0] = u.x; w[1] = u.y;
-                } else if constexpr (BITS == 4) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(prow + ((h ^ ((r >> 2) & 1)) << 4));
+                    const uint4 u = *reinterpret_cast<const uint4 *>(prow);
                     w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+                } else if constexpr (BITS == 4) {
+                    const int x = (r >> 2) & 1;
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(prow + ((q ^ x) << 4));
+                        w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
+                    }
                 } else {
                     const int x = (r >> 1) & 3;
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const uint4 u = *reinterpret_cast<const uint4 *>(prow + (((2 * h + q) ^ x) << 4));
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(prow + ((q ^ x) << 4));
                         w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
                     }
                 }
-                // Codes are in registers: release the packed slot, then wait
-                // until the MMA of k-block c - SA has freed the A slot.
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(empty_p + 8 * sp);
-                uint4 out[4];
-                dequant_half<T, BITS>(w, s16, b16, out);
-                if (c >= SA) ptx::mbar_wait<false>(empty_a + 8 * sa, ((c / SA) + 1) & 1, p.err);
-                uint8_t *arow = gbase + (a0 - base) + sa * A_BYTES + r * 128;
+                uint8_t *arow = gbase + (a0 - base) + s * A_BYTES + r * 128;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int chunk = 4 * h + j;
-                    *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) = out[j];
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint4 out[4];
+                    dequant_half<T, BITS>(w + hh * BITS, hh ? s1 : s0, hh ? b1v : b0v, out);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int chunk = 4 * hh + j;
+                        *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) = out[j];
+                    }
                 }
                 ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(full_a + 8 * sa);
+                if (lane == 0) ptx::mbar_arrive(full_a + 8 * s);
             }
         }
     } else if (warp < kWarpTma) {
@@ -420,33 +410,23 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(acc_empty + 8 * acc);
         }
-    } else if (warp == kWarpTma || warp == kWarpTmaX) {
-        // ------------------------- producers -------------------------
-        // Warp 12 streams the packed weight tiles, warp 14 the activation
-        // tiles; the two rings free at different times, so neither waits on
-        // the other.
+    } else if (warp == kWarpTma) {
+        // ------------------------- producer -------------------------
         if (lane == 0) {
-            const bool wp = warp == kWarpTma;
-            const int R = wp ? SP : SB;
-            const uint32_t fullb = wp ? full_p : full_b, emptyb = wp ? empty_p : empty_b;
             int c = 0;
             for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
                 const int n0 = (tile / p.m_tiles) * kBM, m0 = (tile % p.m_tiles) * BN;
                 for (int kb = 0; kb < KB; ++kb, ++c) {
-                    const int s = c % R;
-                    if (c >= R) ptx::mbar_wait<false>(emptyb + 8 * s, ((c / R) + 1) & 1, p.err);
-                    if (wp) {
-                        ptx::mbar_arrive_expect_tx(fullb + 8 * s, P_BYTES);
-                        tma_load_2d(p0 + s * P_BYTES, &tmap_w, kb * W_WORDS, n0, fullb + 8 * s);
-                    } else {
-                        ptx::mbar_arrive_expect_tx(fullb + 8 * s, B_BYTES);
-                        tma_load_2d(b0 + s * B_BYTES, &tmap_x, kb * kBK, m0, fullb + 8 * s);
-                    }
+                    const int s = c % S;
+                    if (c >= S) ptx::mbar_wait(empty + 8 * s, ((c / S) + 1) & 1, p.err);
+                    ptx::mbar_arrive_expect_tx(full_pb + 8 * s, P_BYTES + B_BYTES);
+                    tma_load_2d(p0 + s * P_BYTES, &tmap_w, kb * W_WORDS, n0, full_pb + 8 * s);
+                    tma_load_2d(b0 + s * B_BYTES, &tmap_x, kb * kBK, m0, full_pb + 8 * s);
                 }
             }
-            // Drain: wait (bounded) for this lane's last copies to land.
-            for (int d = max(0, c - R); d < c; ++d)
-                ptx::mbar_wait(fullb + 8 * (d % R), (d / R) & 1, p.err);
+            // Drain: wait (bounded) for the last copies to land before exit.
+            for (int d = max(0, c - S); d < c; ++d)
+                ptx::mbar_wait(full_pb + 8 * (d % S), (d / S) & 1, p.err);
         }
     } else {
         // ------------------------- MMA issuer -------------------------
@@ -458,17 +438,16 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 tc_fence_after();
                 const uint32_t d = tmem_base + acc * BN;
                 for (int kb = 0; kb < KB; ++kb, ++c) {
-                    const int sa = c % SA, sb = c % SB;
-                    ptx::mbar_wait<false>(full_a + 8 * sa, (c / SA) & 1, p.err);
-                    ptx::mbar_wait<false>(full_b + 8 * sb, (c / SB) & 1, p.err);
+                    const int s = c % S;
+                    ptx::mbar_wait(full_a + 8 * s, (c / S) & 1, p.err);
+                    ptx::mbar_wait(full_pb + 8 * s, (c / S) & 1, p.err);
                     tc_fence_after();
-                    const uint64_t da = sw128_desc(a0 + sa * A_BYTES);
-                    const uint64_t db = sw128_desc(b0 + sb * B_BYTES);
+                    const uint64_t da = sw128_desc(a0 + s * A_BYTES);
+                    const uint64_t db = sw128_desc(b0 + s * B_BYTES);
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)  // UMMA K = 16: 32 bytes along the row
                         tc_mma(d, da + 2 * k, db + 2 * k, IDESC, (kb | k) != 0);
-                    tc_commit(empty_a + 8 * sa);
-                    tc_commit(empty_b + 8 * sb);
+                    tc_commit(empty + 8 * s);
                 }
                 tc_commit(acc_full + 8 * acc);
             }
@@ -529,22 +508,12 @@ int pick_bn(int64_t M) {
 template <typename T, int BITS, int BN>
 cudaError_t run_gemm(const QmmArgs &a, cudaStream_t s) {
     constexpr int A_BYTES = kBM * kBK * 2, B_BYTES = BN * kBK * 2, P_BYTES = kBM * kBK * BITS / 8;
+    constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
     constexpr size_t kSmemMax = 227 * 1024;
-    const size_t fixed = 1024 /*alignment*/ + 64 /*accumulator barriers + tmem slot*/;
-    // Packed tiles are small and freed early: keep a deep ring (up to 8, at
-    // most 32 KB); four dequantized tiles if the activation ring keeps four
-    // stages, else three; the activation ring takes the rest.
-    const int sp = std::min(8, std::max(2, (int)(32768 / P_BYTES)));
-    int sa = 4, sb = 0;
-    for (; sa >= 3; --sa) {
-        const size_t rest =
-            kSmemMax - fixed - (size_t)sa * (A_BYTES + 16) - (size_t)sp * (P_BYTES + 16);
-        sb = (int)std::min<size_t>(8, rest / (B_BYTES + 16));
-        if (sb >= 4) break;
-    }
-    if (sb < 2) return cudaErrorInvalidConfiguration;
-    const size_t smem = fixed + (size_t)sa * (A_BYTES + 16) + (size_t)sb * (B_BYTES + 16) +
-                        (size_t)sp * (P_BYTES + 16);
+    const size_t fixed = 1024 /*alignment*/ + 64 /*acc bars + slot*/;
+    int stages = (int)std::min<size_t>(8, (kSmemMax - fixed) / (STAGE + 24));
+    if (stages < 2) return cudaErrorInvalidConfiguration;
+    const size_t smem = fixed + (size_t)stages * (STAGE + 24);
 
     CUtensorMap tx, tw;
     const CUtensorMapDataType xdt =
@@ -570,9 +539,7 @@ cudaError_t run_gemm(const QmmArgs &a, cudaStream_t s) {
     p.m_tiles = (int)((a.M + BN - 1) / BN);
     p.n_tiles = (int)((a.N + kBM - 1) / kBM);
     p.num_tiles = p.m_tiles * p.n_tiles;
-    p.stages_a = sa;
-    p.stages_b = sb;
-    p.stages_p = sp;
+    p.stages = stages;
     p.err = device_error_word();
     auto kern = qgemm_tc_kernel<T, BITS, BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
