@@ -204,22 +204,24 @@ def peaks():
             "src": "fallback"}
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files) -> str:
+    """Hash of the CUDA sources a kernel is built from (its .cu and the
+    device headers it includes)."""
     h = hashlib.sha256()
-    for f in sorted((ROOT / "quantized_matmul_03_b200" / "csrc").glob("*.cu*")):
-        h.update(f.read_bytes())
+    for name in sorted(files):
+        h.update((ROOT / "quantized_matmul_03_b200" / "csrc" / name).read_bytes())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(kernel: str, workload: str):
-    """dram bytes per launch from a committed ncu summary, when the kernel
+    """dram bytes per launch from a committed ncu summary, when the kernel's
     sources have not changed since it was taken; else None."""
     p = ROOT / "profiles" / "traffic.json"
     if not p.exists():
         return None
     d = json.loads(p.read_text())
     e = d.get(f"{kernel}:{workload}")
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(e.get("source_files", [])):
         return None
     return e.get("dram_bytes_per_launch")
 
