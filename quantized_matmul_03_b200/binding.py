@@ -171,7 +171,16 @@ def qmm_gather_qmm(x, wq, scales, biases, lhs_indices=None, rhs_indices=None,
         sizes.append(x_batch)
     if rhs_indices is None:
         sizes.append(n_experts)
-    batch = max(sizes)
+    # Broadcast of the batch sizes (a size of 1 stretches to the other).
+    others = {n for n in sizes if n != 1}
+    if len(others) > 1:
+        raise ValueError(f"batch sizes {sizes} do not broadcast")
+    batch = others.pop() if others else 1
+    # The C ABI takes index arrays of length batch: stretch length-1 ones.
+    if lhs_indices is not None:
+        lhs_indices = lhs_indices.reshape(-1).expand(batch).contiguous()
+    if rhs_indices is not None:
+        rhs_indices = rhs_indices.reshape(-1).expand(batch).contiguous()
     if out is None:
         out = torch.empty((batch, M, N), dtype=scales.dtype, device=x.device)
     need = qmm_gather_qmm_workspace_size(batch, M, K, n_experts, scales.dtype)

@@ -214,8 +214,11 @@ qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K, const uint3
 
 size_t qmm_gather_qmm_workspace_size(int64_t batch, int64_t M, int64_t K, int64_t n_experts,
                                      qmm_dtype dtype) {
-    (void)batch; (void)M; (void)K; (void)n_experts; (void)dtype;
-    return 0;
+    // Only the tensor-core path (bf16/f16) uses the workspace.
+    if (dtype != QMM_BF16 && dtype != QMM_F16) return 0;
+    if (batch <= 0 || M <= 0 || K <= 0 || n_experts <= 0) return 0;
+    if (batch > INT32_MAX || M > INT32_MAX || batch * M > INT32_MAX / 2) return 0;
+    return gather_ws_layout(batch, M, K, n_experts, 2).total;
 }
 
 qmm_status qmm_gather_qmm(const void *x, int64_t x_batch, int64_t M, int64_t K,
@@ -225,11 +228,79 @@ qmm_status qmm_gather_qmm(const void *x, int64_t x_batch, int64_t M, int64_t K,
                           int transpose, int group_size, int bits, const char *mode,
                           int sorted_indices, void *y, void *workspace, size_t workspace_bytes,
                           void *stream) {
-    (void)x; (void)x_batch; (void)M; (void)K; (void)wq; (void)scales; (void)biases;
-    (void)dtype; (void)n_experts; (void)N; (void)lhs_indices; (void)rhs_indices; (void)batch;
-    (void)transpose; (void)group_size; (void)bits; (void)mode; (void)sorted_indices; (void)y;
-    (void)workspace; (void)workspace_bytes; (void)stream;
-    return fail(QMM_ERR_UNSUPPORTED, "gather_qmm is not built yet");
+    // sorted_indices is accepted for parity with the pages' signature.  The
+    // preparation kernel checks the order of rhs_indices itself and skips the
+    // reorder whenever it is already sorted, so the hint is neither needed nor
+    // trusted: a wrong hint cannot produce wrong results.
+    (void)sorted_indices;
+    try {
+        qmm_status st = check_common(dtype, group_size, bits, mode);
+        if (st != QMM_OK) return st;
+        if (batch < 0 || x_batch < 1 || n_experts < 1 || M < 0 || N < 0 || K <= 0)
+            return fail(QMM_ERR_INVALID_ARG,
+                        "need batch >= 0, x_batch >= 1, n_experts >= 1, M >= 0, N >= 0, K > 0");
+        // (An empty batch has nothing to index: its index arrays may be NULL.)
+        if (batch > 0 && lhs_indices == nullptr && x_batch != 1 && x_batch != batch)
+            return fail(QMM_ERR_INVALID_ARG,
+                        "without lhs_indices, x_batch (%lld) must be 1 or batch (%lld)",
+                        (long long)x_batch, (long long)batch);
+        if (batch > 0 && rhs_indices == nullptr && n_experts != 1 && n_experts != batch)
+            return fail(QMM_ERR_INVALID_ARG,
+                        "without rhs_indices, n_experts (%lld) must be 1 or batch (%lld)",
+                        (long long)n_experts, (long long)batch);
+        if (batch > INT32_MAX || M > INT32_MAX || batch * M > INT32_MAX / 2)
+            return fail(QMM_ERR_UNSUPPORTED, "batch * M must stay below 2^30 rows");
+        // Sizes always; pointers only when there is work (empty tensors may be NULL).
+        st = check_matmul(x, batch == 0 ? 0 : M, K, wq, scales, biases, N, transpose, group_size, y);
+        if (st != QMM_OK) return st;
+        if (batch == 0 || M == 0 || N == 0) return QMM_OK;
+        if (lhs_indices != nullptr && (reinterpret_cast<uintptr_t>(lhs_indices) & 3u))
+            return fail(QMM_ERR_INVALID_ARG, "lhs_indices is not 4-byte aligned");
+        if (rhs_indices != nullptr && (reinterpret_cast<uintptr_t>(rhs_indices) & 3u))
+            return fail(QMM_ERR_INVALID_ARG, "rhs_indices is not 4-byte aligned");
+        cudaStream_t s = (cudaStream_t)stream;
+        const GatherIndex gi{lhs_indices, rhs_indices, batch, x_batch, n_experts};
+
+        GroupedArgs probe{};
+        probe.transpose = transpose != 0;
+        probe.K = K;
+        probe.N = N;
+        probe.bits = bits;
+        probe.rows = batch * M;
+        probe.x_rows = x_batch * M;
+        probe.n_experts = n_experts;
+        const bool tc_ok = gemm_grouped_supported(dtype, probe) && gather_prep_fits(n_experts);
+        if (g_path == QMM_PATH_GEMM && !tc_ok)
+            return fail(QMM_ERR_UNSUPPORTED,
+                        "the tensor-core gather path needs bf16/f16, transpose, K %% 64 == 0");
+        if (tc_ok && g_path != QMM_PATH_GEMV) {
+            const size_t need = qmm_gather_qmm_workspace_size(batch, M, K, n_experts, dtype);
+            if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+                return fail(QMM_ERR_WORKSPACE, "workspace must be a 256-byte aligned device buffer");
+            if (workspace_bytes < need)
+                return fail(QMM_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu",
+                            workspace_bytes, need);
+            GatherCall c{};
+            c.x = x;
+            c.M = M;
+            c.K = K;
+            c.N = N;
+            c.wq = wq;
+            c.scales = scales;
+            c.biases = biases;
+            c.gi = gi;
+            c.transpose = transpose != 0;
+            c.group_size = group_size;
+            c.bits = bits;
+            c.y = y;
+            c.workspace = workspace;
+            return finish_launch(launch_gather_tc(dtype, c, s), "gather_qmm tensor-core launch");
+        }
+        QmmArgs a{x, wq, scales, biases, y, M, N, K, group_size, bits, transpose != 0};
+        return finish_launch(launch_gemv_gather(dtype, a, gi, s), "gather_qmm launch");
+    } catch (...) {
+        return fail(QMM_ERR_CUDA, "unexpected exception in qmm_gather_qmm");
+    }
 }
 
 qmm_status qmm_device_status(void *stream, int reset) {

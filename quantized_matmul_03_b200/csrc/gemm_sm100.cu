@@ -232,12 +232,54 @@ struct GemmParams {
     int M, N, K, group_size;
     int m_tiles, n_tiles, num_tiles, stages;
     int *err;
+    // Grouped (gather_qmm) mode only: the chunk table and row map the
+    // preparation kernel wrote.  Tile t covers chunk t / n_tiles and weight
+    // rows (t % n_tiles) * 128 of that chunk's expert.
+    const GatherHeader *hdr;
+    const int4 *chunks;     // {expert, first sorted row, rows, 0}
+    const int32_t *dst_rows;  // sorted activation row -> output row
 };
 
-template <typename T, int BITS, int BN>
+// What one CTA needs to know about an output tile.
+struct Tile {
+    int n0;     // first output feature (weight row within the expert)
+    int wrow0;  // first row of the stacked weight (expert * N + n0)
+    int m0;     // first activation row (of x, or of the sorted rows)
+    int rows;   // activation rows in the tile
+};
+
+template <int BN, bool GROUPED>
+__device__ __forceinline__ Tile decode_tile(const GemmParams &p, int tile) {
+    Tile t;
+    if constexpr (GROUPED) {
+        const int4 c = __ldg(p.chunks + tile / p.n_tiles);
+        t.n0 = (tile % p.n_tiles) * kBM;
+        t.wrow0 = c.x * p.N + t.n0;
+        t.m0 = c.y;
+        t.rows = c.z;
+    } else {
+        t.n0 = (tile / p.m_tiles) * kBM;
+        t.wrow0 = t.n0;
+        t.m0 = (tile % p.m_tiles) * BN;
+        t.rows = min(BN, p.M - t.m0);
+    }
+    return t;
+}
+
+template <bool GROUPED>
+__device__ __forceinline__ int tile_count(const GemmParams &p) {
+    if constexpr (GROUPED) return __ldg(&p.hdr->num_chunks) * p.n_tiles;
+    else return p.num_tiles;
+}
+
+// GROUPED: gather_qmm's grouped product.  Activation tiles then arrive as
+// 64-row boxes (only as many as the chunk has rows), from tmap_xs (the sorted
+// copy) or tmap_x (x itself, when the sorted order is x's own); the MMA N is
+// the chunk's row count rounded up to 16; outputs go through the row map.
+template <typename T, int BITS, int BN, bool GROUPED>
 __global__ void __launch_bounds__(kThreads, 1)
-qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                const GemmParams p) {
+qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_xs,
+                const __grid_constant__ CUtensorMap tmap_w, const GemmParams p) {
     constexpr bool kF16 = std::is_same<T, __half>::value;
     constexpr int A_BYTES = kBM * kBK * 2;         // 16 KB dequantized tile
     constexpr int B_BYTES = BN * kBK * 2;          // activation tile
@@ -283,6 +325,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     const uint32_t tmem_base = *tmem_slot;
     const int KB = (p.K + kBK - 1) / kBK;
     const int gpr = p.K / p.group_size;
+    const int num_tiles = tile_count<GROUPED>(p);
 
     if (warp < kDqWarps) {
         // ------------------------- dequantize -------------------------
@@ -295,11 +338,11 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         // ahead of use, when rows are whole 16-byte units; else one by one.
         const bool vec = (gpr % 8) == 0;
         int c = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-            const int n0 = (tile / p.m_tiles) * kBM;
-            const int n = n0 + r;
-            const bool rv = n < p.N;
-            const uint16_t *srow = sc + (int64_t)n * gpr, *brow = bi + (int64_t)n * gpr;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            const Tile t = decode_tile<BN, GROUPED>(p, tile);
+            const bool rv = t.n0 + r < p.N;
+            const int64_t wrow = (int64_t)t.wrow0 + r;
+            const uint16_t *srow = sc + wrow * gpr, *brow = bi + wrow * gpr;
             uint4 s_cur = make_uint4(0, 0, 0, 0), b_cur = s_cur, s_nxt = s_cur, b_nxt = s_cur;
             int wbase = 0;  // first group of the current window
             if (vec && rv) {
@@ -382,28 +425,38 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
         T *y = static_cast<T *>(p.y);
         int i = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++i) {
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
             const int acc = i & 1;
-            const int n0 = (tile / p.m_tiles) * kBM, m0 = (tile % p.m_tiles) * BN;
+            const Tile t = decode_tile<BN, GROUPED>(p, tile);
             ptx::mbar_wait(acc_full + 8 * acc, (i >> 1) & 1, p.err);
             tc_fence_after();
-            const int n = n0 + 32 * q + lane;
+            const int n = t.n0 + 32 * q + lane;
             // Columns acc*BN .. acc*BN+BN-1 of this warp's 32 lanes, 32 (or, for
-            // BN = 16, 16) columns per load so no load leaves the allocation.
+            // BN = 16, 16) columns per load so no load leaves the allocation;
+            // column chunks past the tile's rows are skipped.
             constexpr int CW = BN < 32 ? BN : 32;
+            const int nj = (t.rows + CW - 1) / CW;
 #pragma unroll 1
-            for (int j = 0; j < BN / CW; ++j) {
+            for (int j = 0; j < nj; ++j) {
                 uint32_t v[32];
                 const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + acc * BN + CW * j;
                 if constexpr (CW == 32) tmem_ld32(taddr, v);
                 else tmem_ld16(taddr, v);
                 tmem_ld_wait();
-                if (n < p.N) {
+                // Output row of column CW*j + cc: lane cc holds it, shuffled out.
+                int my_dst = 0;
+                if constexpr (GROUPED) {
+                    const int mm = CW * j + (lane & (CW - 1));
+                    if (mm < t.rows) my_dst = __ldg(p.dst_rows + t.m0 + mm);
+                }
 #pragma unroll
-                    for (int cc = 0; cc < CW; ++cc) {
-                        const int m = m0 + CW * j + cc;
-                        if (m < p.M) y[(int64_t)m * p.N + n] = Dt<T>::from_f(__uint_as_float(v[cc]));
-                    }
+                for (int cc = 0; cc < CW; ++cc) {
+                    const int mm = CW * j + cc;
+                    int64_t dst;
+                    if constexpr (GROUPED) dst = __shfl_sync(0xffffffffu, my_dst, cc);
+                    else dst = t.m0 + mm;
+                    if (n < p.N && mm < t.rows)
+                        y[dst * p.N + n] = Dt<T>::from_f(__uint_as_float(v[cc]));
                 }
             }
             tc_fence_before();
@@ -414,14 +467,23 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         // ------------------------- producer -------------------------
         if (lane == 0) {
             int c = 0;
-            for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-                const int n0 = (tile / p.m_tiles) * kBM, m0 = (tile % p.m_tiles) * BN;
+            const CUtensorMap *xmap = &tmap_x;
+            if constexpr (GROUPED) {
+                if (__ldg(&p.hdr->use_x) == 0) xmap = &tmap_xs;
+            }
+            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+                const Tile t = decode_tile<BN, GROUPED>(p, tile);
+                // Grouped tiles load only the 64-row boxes that hold their rows.
+                const int nbox = GROUPED ? (t.rows + 63) / 64 : 1;
+                const uint32_t bbytes = GROUPED ? (uint32_t)nbox * 64u * kBK * 2u : (uint32_t)B_BYTES;
                 for (int kb = 0; kb < KB; ++kb, ++c) {
                     const int s = c % S;
                     if (c >= S) ptx::mbar_wait(empty + 8 * s, ((c / S) + 1) & 1, p.err);
-                    ptx::mbar_arrive_expect_tx(full_pb + 8 * s, P_BYTES + B_BYTES);
-                    tma_load_2d(p0 + s * P_BYTES, &tmap_w, kb * W_WORDS, n0, full_pb + 8 * s);
-                    tma_load_2d(b0 + s * B_BYTES, &tmap_x, kb * kBK, m0, full_pb + 8 * s);
+                    ptx::mbar_arrive_expect_tx(full_pb + 8 * s, P_BYTES + bbytes);
+                    tma_load_2d(p0 + s * P_BYTES, &tmap_w, kb * W_WORDS, t.wrow0, full_pb + 8 * s);
+                    for (int j = 0; j < nbox; ++j)
+                        tma_load_2d(b0 + s * B_BYTES + j * 64 * kBK * 2, xmap, kb * kBK, t.m0 + 64 * j,
+                                    full_pb + 8 * s);
                 }
             }
             // Drain: wait (bounded) for the last copies to land before exit.
@@ -432,8 +494,13 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         // ------------------------- MMA issuer -------------------------
         if (lane == 0) {
             int c = 0, i = 0;
-            for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++i) {
+            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
                 const int acc = i & 1;
+                uint32_t idesc = IDESC;
+                if constexpr (GROUPED) {
+                    const Tile t = decode_tile<BN, GROUPED>(p, tile);
+                    idesc = make_idesc(kF16, kBM, (t.rows + 15) & ~15);  // N: 16..BN, step 16
+                }
                 if (i >= 2) ptx::mbar_wait(acc_empty + 8 * acc, ((i >> 1) + 1) & 1, p.err);
                 tc_fence_after();
                 const uint32_t d = tmem_base + acc * BN;
@@ -446,7 +513,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     const uint64_t db = sw128_desc(b0 + s * B_BYTES);
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)  // UMMA K = 16: 32 bytes along the row
-                        tc_mma(d, da + 2 * k, db + 2 * k, IDESC, (kb | k) != 0);
+                        tc_mma(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
                     tc_commit(empty + 8 * s);
                 }
                 tc_commit(acc_full + 8 * acc);
@@ -505,28 +572,44 @@ int pick_bn(int64_t M) {
     return 256;
 }
 
-template <typename T, int BITS, int BN>
-cudaError_t run_gemm(const QmmArgs &a, cudaStream_t s) {
+// Shared-memory budget of one CTA: S stages of (A + B + P) plus barriers.
+template <int BITS, int BN>
+bool gemm_smem_plan(int &stages, size_t &smem) {
     constexpr int A_BYTES = kBM * kBK * 2, B_BYTES = BN * kBK * 2, P_BYTES = kBM * kBK * BITS / 8;
     constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
     constexpr size_t kSmemMax = 227 * 1024;
     const size_t fixed = 1024 /*alignment*/ + 64 /*acc bars + slot*/;
-    int stages = (int)std::min<size_t>(8, (kSmemMax - fixed) / (STAGE + 24));
-    if (stages < 2) return cudaErrorInvalidConfiguration;
-    const size_t smem = fixed + (size_t)stages * (STAGE + 24);
+    stages = (int)std::min<size_t>(8, (kSmemMax - fixed) / (STAGE + 24));
+    smem = fixed + (size_t)stages * (STAGE + 24);
+    return stages >= 2;
+}
 
+CUtensorMapDataType act_type(bool f16) {
+    return f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+}
+
+// Packed-weight map over `rows` stacked weight rows: one 128-row tile of one
+// k-block per box, swizzled to match its row width (8 / 32 / 64 bytes).
+template <int BITS>
+bool make_weight_map(CUtensorMap *map, const uint32_t *wq, uint64_t rows, int64_t K) {
+    const uint64_t words = (uint64_t)K * BITS / 32;
+    return make_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, words, rows, words * 4,
+                       kBK * BITS / 32, kBM,
+                       BITS == 2 ? CU_TENSOR_MAP_SWIZZLE_NONE
+                                 : (BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B));
+}
+
+template <typename T, int BITS, int BN>
+cudaError_t run_gemm(const QmmArgs &a, cudaStream_t s) {
+    int stages;
+    size_t smem;
+    if (!gemm_smem_plan<BITS, BN>(stages, smem)) return cudaErrorInvalidConfiguration;
+    constexpr bool kF16 = std::is_same<T, __half>::value;
     CUtensorMap tx, tw;
-    const CUtensorMapDataType xdt =
-        std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    if (!make_map_2d(&tx, xdt, a.x, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * 2, kBK, BN,
+    if (!make_map_2d(&tx, act_type(kF16), a.x, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * 2, kBK, BN,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    const uint64_t words = (uint64_t)a.K * BITS / 32;
-    if (!make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.wq, words, (uint64_t)a.N, words * 4,
-                     kBK * BITS / 32, kBM,
-                     BITS == 2 ? CU_TENSOR_MAP_SWIZZLE_NONE
-                               : (BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B)))
-        return cudaErrorInvalidValue;
+    if (!make_weight_map<BITS>(&tw, a.wq, (uint64_t)a.N, a.K)) return cudaErrorInvalidValue;
 
     GemmParams p{};
     p.scales = a.scales;
@@ -541,11 +624,55 @@ cudaError_t run_gemm(const QmmArgs &a, cudaStream_t s) {
     p.num_tiles = p.m_tiles * p.n_tiles;
     p.stages = stages;
     p.err = device_error_word();
-    auto kern = qgemm_tc_kernel<T, BITS, BN>;
+    auto kern = qgemm_tc_kernel<T, BITS, BN, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = std::min(p.num_tiles, num_sms());
-    kern<<<grid, kThreads, smem, s>>>(tx, tw, p);
+    kern<<<grid, kThreads, smem, s>>>(tx, tx, tw, p);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+template <typename T, int BITS, int BN>
+cudaError_t run_gemm_grouped(const GroupedArgs &g, cudaStream_t s) {
+    int stages;
+    size_t smem;
+    if (!gemm_smem_plan<BITS, BN>(stages, smem)) return cudaErrorInvalidConfiguration;
+    constexpr bool kF16 = std::is_same<T, __half>::value;
+    // Activation maps: 64-row boxes over x viewed as [x_batch * M, K] and over
+    // the sorted copy [rows, K].
+    CUtensorMap tx, txs, tw;
+    if (!make_map_2d(&tx, act_type(kF16), g.x, (uint64_t)g.K, (uint64_t)g.x_rows, (uint64_t)g.K * 2,
+                     kBK, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!make_map_2d(&txs, act_type(kF16), g.x_sorted, (uint64_t)g.K, (uint64_t)g.rows,
+                     (uint64_t)g.K * 2, kBK, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!make_weight_map<BITS>(&tw, g.wq, (uint64_t)g.n_experts * (uint64_t)g.N, g.K))
+        return cudaErrorInvalidValue;
+
+    GemmParams p{};
+    p.scales = g.scales;
+    p.biases = g.biases;
+    p.y = g.y;
+    p.M = (int)g.rows;
+    p.N = (int)g.N;
+    p.K = (int)g.K;
+    p.group_size = g.group_size;
+    p.n_tiles = (int)((g.N + kBM - 1) / kBM);
+    p.m_tiles = 0;
+    p.num_tiles = 0;  // read from the header on the device
+    p.stages = stages;
+    p.err = device_error_word();
+    p.hdr = g.hdr;
+    p.chunks = g.chunks;
+    p.dst_rows = g.dst_rows;
+    auto kern = qgemm_tc_kernel<T, BITS, BN, true>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t max_tiles = g.max_chunks * (int64_t)p.n_tiles;
+    const int grid = (int)std::min<int64_t>(max_tiles, num_sms());
+    kern<<<grid, kThreads, smem, s>>>(tx, txs, tw, p);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -558,6 +685,15 @@ cudaError_t gemm_bits(const QmmArgs &a, cudaStream_t s) {
     case 64: return run_gemm<T, BITS, 64>(a, s);
     case 128: return run_gemm<T, BITS, 128>(a, s);
     default: return run_gemm<T, BITS, 256>(a, s);
+    }
+}
+
+template <typename T, int BITS>
+cudaError_t grouped_bits(const GroupedArgs &g, cudaStream_t s) {
+    switch (g.chunk_rows) {
+    case 64: return run_gemm_grouped<T, BITS, 64>(g, s);
+    case 128: return run_gemm_grouped<T, BITS, 128>(g, s);
+    default: return run_gemm_grouped<T, BITS, 256>(g, s);
     }
 }
 
@@ -586,6 +722,32 @@ cudaError_t launch_gemm(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
     case 2: return gemm_bits<__half, 2>(a, s);
     case 4: return gemm_bits<__half, 4>(a, s);
     default: return gemm_bits<__half, 8>(a, s);
+    }
+}
+
+bool gemm_grouped_supported(qmm_dtype dt, const GroupedArgs &g) {
+    if (!g.transpose) return false;
+    if (dt != QMM_BF16 && dt != QMM_F16) return false;
+    if (g.K % kBK != 0) return false;
+    if ((g.K * g.bits / 8) % 16 != 0) return false;
+    if (g.N > INT32_MAX / 2 || g.K > INT32_MAX / 2) return false;
+    if (g.rows > INT32_MAX / 2 || g.x_rows > INT32_MAX / 2) return false;
+    if (g.n_experts * g.N > INT32_MAX / 2) return false;  // TMA row coordinates
+    return encode_fn() != nullptr;
+}
+
+cudaError_t launch_gemm_grouped(qmm_dtype dt, const GroupedArgs &g, cudaStream_t s) {
+    if (dt == QMM_BF16) {
+        switch (g.bits) {
+        case 2: return grouped_bits<__nv_bfloat16, 2>(g, s);
+        case 4: return grouped_bits<__nv_bfloat16, 4>(g, s);
+        default: return grouped_bits<__nv_bfloat16, 8>(g, s);
+        }
+    }
+    switch (g.bits) {
+    case 2: return grouped_bits<__half, 2>(g, s);
+    case 4: return grouped_bits<__half, 4>(g, s);
+    default: return grouped_bits<__half, 8>(g, s);
     }
 }
 

@@ -28,6 +28,37 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
+// Which product a CTA computes: blockIdx.z + b0 is the batch entry; a plain
+// matmul is the one-entry batch with zero strides.  gather_qmm entries
+// resolve their activation and expert through GatherIndex; an entry with an
+// out-of-range index computes nothing and writes zeros.
+struct BatchView {
+    GatherIndex gi;
+    int64_t b0;
+    int64_t x_stride, w_stride, sb_stride, y_stride;  // elements / words per entry
+    int *err;
+};
+
+// Offsets (in elements / words) of this CTA's entry; false for an invalid one.
+struct EntryOffsets {
+    int64_t x, w, sb, y;
+};
+__device__ __forceinline__ bool select_entry(const BatchView &bv, EntryOffsets &o) {
+    const int64_t b = bv.b0 + blockIdx.z;
+    int64_t xi, ei;
+    const bool valid = gather_entry(bv.gi, b, xi, ei);
+    if (!valid) {
+        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0)
+            record_device_error(bv.err, QMM_ERR_INDEX);
+        xi = ei = 0;
+    }
+    o.x = xi * bv.x_stride;
+    o.w = ei * bv.w_stride;
+    o.sb = ei * bv.sb_stride;
+    o.y = b * bv.y_stride;
+    return valid;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
@@ -41,7 +72,8 @@ template <typename T, int BITS, int MT, int RW>
 __global__ void __launch_bounds__(kThreads)
 gemv_t_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
               const T *__restrict__ scales, const T *__restrict__ biases,
-              T *__restrict__ y, int M, int64_t N, int64_t K, int group_size, int kc) {
+              T *__restrict__ y, int M, int64_t N, int64_t K, int group_size, int kc,
+              const BatchView bv) {
     constexpr int EPW = 32 / BITS;
     constexpr uint32_t MASK = (1u << BITS) - 1u;
     extern __shared__ float xs[];  // [MT][kc]
@@ -50,13 +82,21 @@ gemv_t_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     const int64_t wpr = K / EPW;          // packed words per weight row
     const int64_t gpr = K / group_size;   // groups per weight row
 
+    EntryOffsets eo;
+    const bool valid = select_entry(bv, eo);
+    x += eo.x;
+    wq += eo.w;
+    scales += eo.sb;
+    biases += eo.sb;
+    y += eo.y;
+
     float acc[RW][MT];
 #pragma unroll
     for (int r = 0; r < RW; ++r)
 #pragma unroll
         for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
 
-    for (int64_t k0 = 0; k0 < K; k0 += kc) {
+    for (int64_t k0 = 0; valid && k0 < K; k0 += kc) {  // (CTA-uniform condition)
         const int klen = (int)min((int64_t)kc, K - k0);
         __syncthreads();
         for (int i = threadIdx.x; i < MT * klen; i += kThreads) {
@@ -104,12 +144,20 @@ template <typename T, int BITS, int MT>
 __global__ void __launch_bounds__(kThreads)
 gemv_n_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
               const T *__restrict__ scales, const T *__restrict__ biases,
-              T *__restrict__ y, int M, int64_t N, int64_t K, int group_size, int64_t k_split) {
+              T *__restrict__ y, int M, int64_t N, int64_t K, int group_size, int64_t k_split,
+              const BatchView bv) {
     constexpr int EPW = 32 / BITS;
     constexpr uint32_t MASK = (1u << BITS) - 1u;
     constexpr int NE = EPW * MT;           // partial sums per lane
     __shared__ float red[kWarps][NE][32];  // per-warp partials
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    EntryOffsets eo;
+    const bool valid = select_entry(bv, eo);
+    x += eo.x;
+    wq += eo.w;
+    scales += eo.sb;
+    biases += eo.sb;
+    y += eo.y;
     const int64_t wpr = N / EPW;            // packed words per weight row
     const int64_t gpr = N / group_size;
     const int64_t col = (int64_t)blockIdx.x * 32 + lane;  // packed word column
@@ -121,7 +169,7 @@ gemv_n_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
 #pragma unroll
     for (int i = 0; i < NE; ++i) acc[i] = 0.f;
 
-    if (col_ok) {
+    if (col_ok && valid) {
         const int64_t g = col * EPW / group_size;
         for (int64_t k = kbeg + warp; k < kend; k += kWarps) {
             const uint32_t pk = __ldg(wq + k * wpr + col);
@@ -166,36 +214,38 @@ gemv_n_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
 }
 
 template <typename T, int BITS, int MT>
-cudaError_t run_gemv_t(const QmmArgs &a, int M, const T *x, T *y, cudaStream_t s) {
+cudaError_t run_gemv_t(const QmmArgs &a, int M, const T *x, T *y, const BatchView &bv, int nb,
+                       cudaStream_t s) {
     constexpr int RW = 2;
     const int64_t rows_per_cta = kWarps * RW;
-    const int64_t grid = (a.N + rows_per_cta - 1) / rows_per_cta;
+    const int64_t gx = (a.N + rows_per_cta - 1) / rows_per_cta;
     // Activation chunk: at most 48 KB of fp32, a multiple of 128 elements.
     int kc = (int)std::min<int64_t>(a.K, (48 * 1024 / 4) / MT);
     kc = (kc / 128) * 128;
     if (kc <= 0) kc = 128;
     if (kc > a.K) kc = (int)a.K;
     const size_t smem = (size_t)MT * kc * sizeof(float);
-    gemv_t_kernel<T, BITS, MT, RW><<<grid, kThreads, smem, s>>>(
+    gemv_t_kernel<T, BITS, MT, RW><<<dim3((unsigned)gx, 1, nb), kThreads, smem, s>>>(
         x, a.wq, static_cast<const T *>(a.scales), static_cast<const T *>(a.biases), y, M,
-        a.N, a.K, a.group_size, kc);
+        a.N, a.K, a.group_size, kc, bv);
     count_launches(1);
     return cudaGetLastError();
 }
 
 template <typename T, int BITS, int MT>
-cudaError_t run_gemv_n(const QmmArgs &a, int M, const T *x, T *y, cudaStream_t s) {
+cudaError_t run_gemv_n(const QmmArgs &a, int M, const T *x, T *y, const BatchView &bv, int nb,
+                       cudaStream_t s) {
     constexpr int EPW = 32 / BITS;
     const int64_t wpr = a.N / EPW;
     const int gx = (int)((wpr + 31) / 32);
     // Split K over a cluster of up to 8 CTAs so that small-N problems still
     // fill the GPU; each split is at least 64 rows of W.
     int ks = 8;
-    while (ks > 1 && (int64_t)gx * ks > 4LL * num_sms()) ks >>= 1;
+    while (ks > 1 && (int64_t)gx * ks * nb > 4LL * num_sms()) ks >>= 1;
     while (ks > 1 && a.K / ks < 64) ks >>= 1;
     const int64_t k_split = (a.K + ks - 1) / ks;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(gx, ks, 1);
+    cfg.gridDim = dim3(gx, ks, nb);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
@@ -209,49 +259,64 @@ cudaError_t run_gemv_n(const QmmArgs &a, int M, const T *x, T *y, cudaStream_t s
     count_launches(1);
     return cudaLaunchKernelEx(&cfg, gemv_n_kernel<T, BITS, MT>, x, a.wq,
                               static_cast<const T *>(a.scales), static_cast<const T *>(a.biases),
-                              y, M, a.N, a.K, a.group_size, k_split);
+                              y, M, a.N, a.K, a.group_size, k_split, bv);
 }
 
 // Largest activation tile per launch: gemv_t keeps RW*MT accumulators per
-// lane; gemv_n keeps (32/bits)*MT, capped at 32 (so MT <= bits).
+// lane; gemv_n keeps (32/bits)*MT, capped at 32 (so MT <= bits).  Entries of
+// a batch go to gridDim.z, at most 65535 per launch.
 template <typename T, int BITS>
-cudaError_t gemv_bits(const QmmArgs &a, cudaStream_t s) {
+cudaError_t gemv_bits(const QmmArgs &a, const BatchView &bv0, int64_t batch, cudaStream_t s) {
     const T *x = static_cast<const T *>(a.x);
     T *y = static_cast<T *>(a.y);
     const int tile = a.transpose ? 16 : BITS;
-    for (int64_t m0 = 0; m0 < a.M; m0 += tile) {
-        const int mt = (int)std::min<int64_t>(tile, a.M - m0);
-        const T *xm = x + m0 * a.K;
-        T *ym = y + m0 * a.N;
-        cudaError_t e;
-        if (a.transpose) {
-            if (mt == 1) e = run_gemv_t<T, BITS, 1>(a, mt, xm, ym, s);
-            else if (mt == 2) e = run_gemv_t<T, BITS, 2>(a, mt, xm, ym, s);
-            else if (mt <= 4) e = run_gemv_t<T, BITS, 4>(a, mt, xm, ym, s);
-            else if (mt <= 8) e = run_gemv_t<T, BITS, 8>(a, mt, xm, ym, s);
-            else e = run_gemv_t<T, BITS, 16>(a, mt, xm, ym, s);
-        } else {
-            if (mt == 1) e = run_gemv_n<T, BITS, 1>(a, mt, xm, ym, s);
-            else if (mt == 2) e = run_gemv_n<T, BITS, 2>(a, mt, xm, ym, s);
-            else if constexpr (BITS >= 4) {
-                if (mt <= 4) e = run_gemv_n<T, BITS, 4>(a, mt, xm, ym, s);
-                else if constexpr (BITS >= 8) e = run_gemv_n<T, BITS, 8>(a, mt, xm, ym, s);
-                else e = cudaErrorInvalidValue;
+    for (int64_t b0 = 0; b0 < batch; b0 += 65535) {
+        const int nb = (int)std::min<int64_t>(65535, batch - b0);
+        BatchView bv = bv0;
+        bv.b0 = b0;
+        for (int64_t m0 = 0; m0 < a.M; m0 += tile) {
+            const int mt = (int)std::min<int64_t>(tile, a.M - m0);
+            const T *xm = x + m0 * a.K;
+            T *ym = y + m0 * a.N;
+            cudaError_t e;
+            if (a.transpose) {
+                if (mt == 1) e = run_gemv_t<T, BITS, 1>(a, mt, xm, ym, bv, nb, s);
+                else if (mt == 2) e = run_gemv_t<T, BITS, 2>(a, mt, xm, ym, bv, nb, s);
+                else if (mt <= 4) e = run_gemv_t<T, BITS, 4>(a, mt, xm, ym, bv, nb, s);
+                else if (mt <= 8) e = run_gemv_t<T, BITS, 8>(a, mt, xm, ym, bv, nb, s);
+                else e = run_gemv_t<T, BITS, 16>(a, mt, xm, ym, bv, nb, s);
             } else {
-                e = cudaErrorInvalidValue;
+                if (mt == 1) e = run_gemv_n<T, BITS, 1>(a, mt, xm, ym, bv, nb, s);
+                else if (mt == 2) e = run_gemv_n<T, BITS, 2>(a, mt, xm, ym, bv, nb, s);
+                else if constexpr (BITS >= 4) {
+                    if (mt <= 4) e = run_gemv_n<T, BITS, 4>(a, mt, xm, ym, bv, nb, s);
+                    else if constexpr (BITS >= 8) e = run_gemv_n<T, BITS, 8>(a, mt, xm, ym, bv, nb, s);
+                    else e = cudaErrorInvalidValue;
+                } else {
+                    e = cudaErrorInvalidValue;
+                }
             }
+            if (e != cudaSuccess) return e;
         }
-        if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
 }
 
 template <typename T>
-cudaError_t gemv_t_dtype(const QmmArgs &a, cudaStream_t s) {
+cudaError_t gemv_t_dtype(const QmmArgs &a, const BatchView &bv, int64_t batch, cudaStream_t s) {
     switch (a.bits) {
-    case 2: return gemv_bits<T, 2>(a, s);
-    case 4: return gemv_bits<T, 4>(a, s);
-    default: return gemv_bits<T, 8>(a, s);
+    case 2: return gemv_bits<T, 2>(a, bv, batch, s);
+    case 4: return gemv_bits<T, 4>(a, bv, batch, s);
+    default: return gemv_bits<T, 8>(a, bv, batch, s);
+    }
+}
+
+cudaError_t gemv_dispatch(qmm_dtype dt, const QmmArgs &a, const BatchView &bv, int64_t batch,
+                          cudaStream_t s) {
+    switch (dt) {
+    case QMM_F32: return gemv_t_dtype<float>(a, bv, batch, s);
+    case QMM_BF16: return gemv_t_dtype<__nv_bfloat16>(a, bv, batch, s);
+    default: return gemv_t_dtype<__half>(a, bv, batch, s);
     }
 }
 
@@ -261,11 +326,26 @@ bool gemv_supported(qmm_dtype, const QmmArgs &) { return true; }
 
 cudaError_t launch_gemv(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
     if (a.M == 0 || a.N == 0) return cudaSuccess;
-    switch (dt) {
-    case QMM_F32: return gemv_t_dtype<float>(a, s);
-    case QMM_BF16: return gemv_t_dtype<__nv_bfloat16>(a, s);
-    default: return gemv_t_dtype<__half>(a, s);
-    }
+    BatchView bv{};
+    bv.gi = GatherIndex{nullptr, nullptr, 1, 1, 1};
+    bv.err = device_error_word();
+    return gemv_dispatch(dt, a, bv, 1, s);
+}
+
+// a describes one entry: x points at x[0] ([M, K]), wq/scales/biases at
+// expert 0, y at y[0] ([M, N]).
+cudaError_t launch_gemv_gather(qmm_dtype dt, const QmmArgs &a, const GatherIndex &gi, cudaStream_t s) {
+    if (a.M == 0 || a.N == 0 || gi.batch == 0) return cudaSuccess;
+    const int bits = a.bits, epw = 32 / bits;
+    const int64_t wrows = a.transpose ? a.N : a.K, wcols = a.transpose ? a.K : a.N;
+    BatchView bv{};
+    bv.gi = gi;
+    bv.x_stride = a.M * a.K;
+    bv.w_stride = wrows * (wcols / epw);
+    bv.sb_stride = wrows * (wcols / a.group_size);
+    bv.y_stride = a.M * a.N;
+    bv.err = device_error_word();
+    return gemv_dispatch(dt, a, bv, gi.batch, s);
 }
 
 }  // namespace qmm

@@ -58,10 +58,7 @@ struct DequantArgs {
 };
 cudaError_t launch_dequantize(qmm_dtype dt, const DequantArgs &a, cudaStream_t s);
 
-// One (possibly batched) quantized product.  Rows of x and y are addressed
-// through optional row maps so that gather_qmm can reuse the same kernels:
-//   activation row i of problem p reads  x + x_row(p, i) * K
-//   and writes                           y + y_row(p, i) * N
+// One quantized product y[M, N] = x[M, K] (*) W.
 struct QmmArgs {
     const void *x;       // [*, K]
     const uint32_t *wq;  // packed weight of this problem
@@ -77,6 +74,78 @@ cudaError_t launch_gemv_fast(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a);
 cudaError_t launch_gemm(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 bool gemm_supported(qmm_dtype dt, const QmmArgs &a);
+
+// ---------------------------------------------------------------------------
+// gather_qmm
+// ---------------------------------------------------------------------------
+// Batch entry b uses activations x[xi(b)] and expert ei(b):
+//   xi = lhs ? lhs[b] : (x_batch == 1 ? 0 : b),  ei = rhs ? rhs[b] : (n_experts == 1 ? 0 : b).
+// An entry whose xi or ei is out of range is "invalid": its output rows are
+// zero and the device error word gets QMM_ERR_INDEX.
+struct GatherIndex {
+    const int32_t *lhs, *rhs;  // nullable
+    int64_t batch, x_batch, n_experts;
+};
+
+__device__ __forceinline__ bool gather_entry(const GatherIndex &gi, int64_t b, int64_t &xi,
+                                             int64_t &ei) {
+    xi = gi.lhs ? (int64_t)__ldg(gi.lhs + b) : (gi.x_batch == 1 ? 0 : b);
+    ei = gi.rhs ? (int64_t)__ldg(gi.rhs + b) : (gi.n_experts == 1 ? 0 : b);
+    return xi >= 0 && xi < gi.x_batch && ei >= 0 && ei < gi.n_experts;
+}
+
+// Header the preparation kernel writes at the start of the workspace.
+struct GatherHeader {
+    int num_chunks;     // entries of the chunk table
+    int use_x;          // 1: the sorted row order is x's own, read x directly
+    int valid_entries;  // batch entries with in-range indices (sorted first)
+    int pad;
+};
+
+// SIMT batched path (any dtype, either layout): one product per entry.
+cudaError_t launch_gemv_gather(qmm_dtype dt, const QmmArgs &a, const GatherIndex &gi, cudaStream_t s);
+
+// Grouped tensor-core product over rows sorted by expert.
+struct GroupedArgs {
+    const void *x;           // [x_rows = x_batch * M, K]
+    const void *x_sorted;    // [rows, K] (workspace)
+    const uint32_t *wq;      // [n_experts * N, K * bits / 32]
+    const void *scales, *biases;
+    void *y;                 // [batch * M, N]
+    int64_t x_rows, rows, N, K, n_experts, max_chunks;
+    int group_size, bits;
+    bool transpose;
+    int chunk_rows;          // 64, 128 or 256: rows per chunk at most
+    const GatherHeader *hdr;
+    const int4 *chunks;
+    const int32_t *dst_rows;
+};
+bool gemm_grouped_supported(qmm_dtype dt, const GroupedArgs &g);
+cudaError_t launch_gemm_grouped(qmm_dtype dt, const GroupedArgs &g, cudaStream_t s);
+
+// Byte offsets of the tensor-core path's pieces in the caller's workspace
+// (each 256-byte aligned), and the total size.
+struct GatherWorkspace {
+    size_t hdr, chunks, perm, dst_rows, x_sorted, total;
+    int64_t max_chunks;
+};
+GatherWorkspace gather_ws_layout(int64_t batch, int64_t M, int64_t K, int64_t n_experts,
+                                 int elt_bytes);
+int gather_chunk_rows(int64_t rows);       // tile width (64/128/256) for `rows` sorted rows
+bool gather_prep_fits(int64_t n_experts);  // the sort's histograms fit shared memory
+
+struct GatherCall {
+    const void *x;  // [x_batch, M, K]
+    int64_t M, K, N;
+    const uint32_t *wq;
+    const void *scales, *biases;
+    GatherIndex gi;
+    bool transpose;
+    int group_size, bits;
+    void *y;  // [batch, M, N]
+    void *workspace;
+};
+cudaError_t launch_gather_tc(qmm_dtype dt, const GatherCall &c, cudaStream_t s);
 
 int num_sms();
 void count_launches(int n);  // bump the process-wide launch counter
