@@ -2,7 +2,7 @@
  * qmm.h -- C ABI of libqmm, group-wise affine quantized matmul for NVIDIA
  * B200 (sm_100a).
  *
- * The operations follow the MLX quantization API as four pages describe it:
+ * The operations follow the MLX quantization API as these documents describe it:
  *   EMLX.Quantization (emlx 0.4.2): quantize, dequantize, quantized_matmul,
  *     gather_quantized_matmul;
  *   Emily.QuantizedWeight (emily 0.7.2), section Layout: the packed value /
@@ -33,8 +33,8 @@
  * Dtypes.  scales and biases share the dense weight's dtype; outputs take the
  *   scales dtype (EMLX.Quantization, section quantized_matmul); activations
  *   must have that dtype too.
- * Mode.  `mode` NULL means "affine" (the pages' default).  The microscaled
- *   modes named on the pages ("mxfp4", "mxfp8", "nvfp4") return
+ * Mode.  `mode` NULL means "affine" (the default in every document above).
+ *   The microscaled modes of Emily.QuantizedWeight ("mxfp4", "mxfp8", "nvfp4") return
  *   QMM_ERR_UNSUPPORTED; any other string returns QMM_ERR_INVALID_ARG.
  */
 #ifndef QMM_H
@@ -50,7 +50,7 @@ extern "C" {
 typedef enum {
     QMM_OK = 0,
     QMM_ERR_INVALID_ARG = 1, /* bad size, pointer, group size, bits, ... */
-    QMM_ERR_UNSUPPORTED = 2, /* valid on the pages but not built (e.g. mxfp4) */
+    QMM_ERR_UNSUPPORTED = 2, /* documented upstream but not built (e.g. mxfp4) */
     QMM_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
     QMM_ERR_TIMEOUT = 4,     /* a kernel's bounded wait ran out (device word) */
     QMM_ERR_INDEX = 5,       /* an expert / row index was out of range */
@@ -114,13 +114,27 @@ qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K,
  *   ei = rhs_indices[b] if rhs_indices else (n_experts == 1 ? 0 : b).
  * Without lhs_indices, x_batch must be 1 or batch; without rhs_indices,
  * n_experts must be 1 or batch.  Indices are int32 device arrays of length
- * `batch`.  No expert weight is copied.  sorted_indices != 0 promises that
- * rhs_indices is non-decreasing, which lets the library skip its sort.
+ * `batch` (4-byte aligned); with batch == 0 the call does nothing and the
+ * index pointers may be NULL.  No expert weight is copied.
+ * sorted_indices: the caller's promise (EMLX.Quantization, section
+ *   gather_quantized_matmul) that rhs_indices is non-decreasing.  The
+ *   library checks the order itself on the device and skips its reorder
+ *   whenever the keys are already sorted, so the hint is accepted but never
+ *   trusted: a wrong hint cannot give wrong results.
+ * Paths: bf16/f16 with transpose != 0 and K % 64 == 0 sort the rows by expert
+ *   and run the grouped tensor-core product (three kernels: prepare, gather
+ *   rows, product).  Other cases (f32, transpose == 0) run the SIMT kernels
+ *   with one grid slice per batch entry.  qmm_set_path() forces either.
  * Out-of-range indices: the affected output rows are written as zeros and a
- * later qmm_device_status() reports QMM_ERR_INDEX.
+ *   later qmm_device_status() reports QMM_ERR_INDEX; nothing is read or
+ *   written out of bounds.
  * workspace: device scratch of at least qmm_gather_qmm_workspace_size(...)
- * bytes, 256-byte aligned; contents need not be initialised and are not
- * preserved.  Two calls in flight at once must not share a workspace.
+ *   bytes, 256-byte aligned, used by the tensor-core path only (the size is 0
+ *   for f32); its contents need not be initialised and are not preserved.
+ *   Two calls in flight at once must not share a workspace.  Too small or
+ *   misaligned: QMM_ERR_WORKSPACE.
+ * Errors: QMM_ERR_INVALID_ARG for sizes that do not broadcast or misaligned
+ *   pointers, QMM_ERR_UNSUPPORTED for batch * M >= 2^30 rows.
  */
 size_t qmm_gather_qmm_workspace_size(int64_t batch, int64_t M, int64_t K,
                                      int64_t n_experts, qmm_dtype dtype);

@@ -18,7 +18,7 @@
  *  - Scales and biases have the source weight's dtype and shape
  *    (..., last_dim / group_size) (Emily.QuantizedWeight, section Layout).
  *
- * The pages do not print the scale/bias rule or the bit order.  The reading
+ * None of the documents above prints the scale/bias rule or the bit order.  The reading
  * used here (stated once, applied everywhere):
  *    bias  = min of the group,
  *    scale = (max - min) / (2^bits - 1)          (fp32, correctly rounded),

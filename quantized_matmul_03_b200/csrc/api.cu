@@ -40,7 +40,7 @@ qmm_status cuda_fail(cudaError_t e, const char *what) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Mode strings of the pages: "affine" (default), and the microscaled modes
+// Mode strings: "affine" (default), and the microscaled modes
 // that carry fixed group sizes and no biases (Emily.QuantizedWeight, section
 // Microscaled modes).
 qmm_status check_mode(const char *mode) {
@@ -228,7 +228,7 @@ qmm_status qmm_gather_qmm(const void *x, int64_t x_batch, int64_t M, int64_t K,
                           int transpose, int group_size, int bits, const char *mode,
                           int sorted_indices, void *y, void *workspace, size_t workspace_bytes,
                           void *stream) {
-    // sorted_indices is accepted for parity with the pages' signature.  The
+    // sorted_indices is accepted for parity with the upstream signature.  The
     // preparation kernel checks the order of rhs_indices itself and skips the
     // reorder whenever it is already sorted, so the hint is neither needed nor
     // trusted: a wrong hint cannot produce wrong results.

@@ -1,7 +1,7 @@
-"""Pins for the CPU oracle: checks against what the pages and the mathematics
+"""Pins for the CPU oracle: checks against what the cited documents and the mathematics
 fix, never against the oracle's own formulas retyped.
 
-Each test names the page passage (or the mathematical fact) it rests on and the
+Each test names the documented passage (or the mathematical fact) it rests on and the
 plausible oracle mistake it would catch.
 """
 import json
@@ -25,7 +25,7 @@ def u32(t: torch.Tensor):
 
 
 # --------------------------------------------------------------------------
-# Shapes printed on the pages (doctests) -- catch a wrong packing ratio, a
+# Shapes printed in the documents (doctests) -- catch a wrong packing ratio, a
 # wrong group axis, a transposed product.
 # --------------------------------------------------------------------------
 
