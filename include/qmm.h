@@ -149,6 +149,37 @@ qmm_status qmm_gather_qmm(const void *x, int64_t x_batch, int64_t M, int64_t K,
                           void *stream);
 
 /*
+ * qmm_gather_qmm_static -- gather_qmm without a caller workspace.  Nothing in
+ * the documents this library follows has a counterpart: it is a convenience
+ * of this library for callers that cannot hand over device memory, such as a
+ * plain C host that links no device allocator, or a step that must not
+ * allocate (cudaMalloc can synchronise the device).  It allocates nothing:
+ * the tensor-core path uses a fixed scratch array of
+ * QMM_GATHER_STATIC_SCRATCH_BYTES built into the library (one per device).
+ *
+ * Arguments, layouts, results and errors are those of qmm_gather_qmm.  In
+ * addition, a bf16/f16 call with transpose != 0 whose
+ * qmm_gather_qmm_workspace_size(batch, M, K, n_experts, dtype) exceeds
+ * QMM_GATHER_STATIC_SCRATCH_BYTES returns QMM_ERR_WORKSPACE before launching
+ * anything (use qmm_gather_qmm with a workspace for such sizes).  Example:
+ * x [512, 1, 4096] bf16 needs about 4.2 MB.
+ *
+ * The scratch needs no initialisation (nothing in it must start at zero).
+ * The first call on a device looks up the scratch's address, so make it
+ * before any stream capture.  All calls on one device share the one scratch:
+ * two calls whose work overlaps in time (on different streams, or from
+ * different host threads) race on it and may return wrong results.  Calls
+ * queued one after another on the same stream are safe.
+ */
+#define QMM_GATHER_STATIC_SCRATCH_BYTES (8u << 20)
+qmm_status qmm_gather_qmm_static(const void *x, int64_t x_batch, int64_t M, int64_t K,
+                                 const uint32_t *wq, const void *scales, const void *biases,
+                                 qmm_dtype dtype, int64_t n_experts, int64_t N,
+                                 const int32_t *lhs_indices, const int32_t *rhs_indices,
+                                 int64_t batch, int transpose, int group_size, int bits,
+                                 const char *mode, int sorted_indices, void *y, void *stream);
+
+/*
  * qmm_device_status -- synchronise `stream`, then read (and, if `reset` is
  * non-zero, clear) the library's device-side error word, set by kernels whose
  * bounded waits time out (QMM_ERR_TIMEOUT) or that meet an out-of-range index

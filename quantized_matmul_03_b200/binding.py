@@ -50,6 +50,8 @@ def lib() -> ctypes.CDLL:
                                      vp, vp],
             "qmm_gather_qmm": [vp, i64, i64, i64, vp, vp, vp, i32, i64, i64, vp, vp, i64, i32,
                                i32, i32, cp, i32, vp, vp, sz, vp],
+            "qmm_gather_qmm_static": [vp, i64, i64, i64, vp, vp, vp, i32, i64, i64, vp, vp, i64,
+                                      i32, i32, i32, cp, i32, vp, vp],
             "qmm_device_status": [vp, i32],
             "qmm_set_path": [i32],
         }
@@ -152,14 +154,9 @@ def qmm_gather_qmm_workspace_size(batch: int, M: int, K: int, n_experts: int,
     return int(lib().qmm_gather_qmm_workspace_size(batch, M, K, n_experts, DTYPES[dtype]))
 
 
-def qmm_gather_qmm(x, wq, scales, biases, lhs_indices=None, rhs_indices=None,
-                   transpose: bool = True, group_size: int = 64, bits: int = 4,
-                   mode: str = "affine", sorted_indices: bool = False,
-                   workspace: Optional[torch.Tensor] = None,
-                   out: Optional[torch.Tensor] = None):
-    """Mixture-of-experts quantized matmul: x [x_batch, M, K], experts stacked
-    on wq's leading axis; returns y [batch, M, N]."""
-    _cuda(x, wq, scales, biases, lhs_indices, rhs_indices, workspace, out)
+def _gather_shapes(x, wq, lhs_indices, rhs_indices, transpose, bits):
+    """Sizes of a gather_qmm call, and the index arrays stretched to the
+    broadcast batch (the C ABI takes arrays of length batch)."""
     for t in (lhs_indices, rhs_indices):
         if t is not None and t.dtype != torch.int32:
             raise ValueError("indices must be int32")
@@ -176,11 +173,23 @@ def qmm_gather_qmm(x, wq, scales, biases, lhs_indices=None, rhs_indices=None,
     if len(others) > 1:
         raise ValueError(f"batch sizes {sizes} do not broadcast")
     batch = others.pop() if others else 1
-    # The C ABI takes index arrays of length batch: stretch length-1 ones.
     if lhs_indices is not None:
         lhs_indices = lhs_indices.reshape(-1).expand(batch).contiguous()
     if rhs_indices is not None:
         rhs_indices = rhs_indices.reshape(-1).expand(batch).contiguous()
+    return x_batch, M, K, n_experts, N, batch, lhs_indices, rhs_indices
+
+
+def qmm_gather_qmm(x, wq, scales, biases, lhs_indices=None, rhs_indices=None,
+                   transpose: bool = True, group_size: int = 64, bits: int = 4,
+                   mode: str = "affine", sorted_indices: bool = False,
+                   workspace: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None):
+    """Mixture-of-experts quantized matmul: x [x_batch, M, K], experts stacked
+    on wq's leading axis; returns y [batch, M, N]."""
+    _cuda(x, wq, scales, biases, lhs_indices, rhs_indices, workspace, out)
+    x_batch, M, K, n_experts, N, batch, lhs_indices, rhs_indices = _gather_shapes(
+        x, wq, lhs_indices, rhs_indices, transpose, bits)
     if out is None:
         out = torch.empty((batch, M, N), dtype=scales.dtype, device=x.device)
     need = qmm_gather_qmm_workspace_size(batch, M, K, n_experts, scales.dtype)
@@ -192,6 +201,25 @@ def qmm_gather_qmm(x, wq, scales, biases, lhs_indices=None, rhs_indices=None,
                                 batch, int(bool(transpose)), group_size, bits, _mode(mode),
                                 int(bool(sorted_indices)), _p(out), _p(workspace), ws_bytes,
                                 _stream(x.device)))
+    return out
+
+
+def qmm_gather_qmm_static(x, wq, scales, biases, lhs_indices=None, rhs_indices=None,
+                          transpose: bool = True, group_size: int = 64, bits: int = 4,
+                          mode: str = "affine", sorted_indices: bool = False,
+                          out: Optional[torch.Tensor] = None):
+    """gather_qmm on the library's built-in scratch (no workspace argument).
+    Calls whose work overlaps in time on one device race on that scratch."""
+    _cuda(x, wq, scales, biases, lhs_indices, rhs_indices, out)
+    x_batch, M, K, n_experts, N, batch, lhs_indices, rhs_indices = _gather_shapes(
+        x, wq, lhs_indices, rhs_indices, transpose, bits)
+    if out is None:
+        out = torch.empty((batch, M, N), dtype=scales.dtype, device=x.device)
+    _check(lib().qmm_gather_qmm_static(_p(x), x_batch, M, K, _p(wq), _p(scales), _p(biases),
+                                       _dtype(scales), n_experts, N, _p(lhs_indices),
+                                       _p(rhs_indices), batch, int(bool(transpose)), group_size,
+                                       bits, _mode(mode), int(bool(sorted_indices)), _p(out),
+                                       _stream(x.device)))
     return out
 
 

@@ -303,6 +303,32 @@ qmm_status qmm_gather_qmm(const void *x, int64_t x_batch, int64_t M, int64_t K,
     }
 }
 
+qmm_status qmm_gather_qmm_static(const void *x, int64_t x_batch, int64_t M, int64_t K,
+                                 const uint32_t *wq, const void *scales, const void *biases,
+                                 qmm_dtype dtype, int64_t n_experts, int64_t N,
+                                 const int32_t *lhs_indices, const int32_t *rhs_indices,
+                                 int64_t batch, int transpose, int group_size, int bits,
+                                 const char *mode, int sorted_indices, void *y, void *stream) {
+    try {
+        if (transpose != 0) {
+            const size_t need = qmm_gather_qmm_workspace_size(batch, M, K, n_experts, dtype);
+            if (need > QMM_GATHER_STATIC_SCRATCH_BYTES)
+                return fail(QMM_ERR_WORKSPACE,
+                            "this call needs %zu bytes of scratch; the built-in scratch holds %u "
+                            "(call qmm_gather_qmm with a workspace instead)",
+                            need, (unsigned)QMM_GATHER_STATIC_SCRATCH_BYTES);
+        }
+        void *scratch = nullptr;
+        const cudaError_t e = gather_static_scratch(&scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "look up the built-in gather scratch");
+        return qmm_gather_qmm(x, x_batch, M, K, wq, scales, biases, dtype, n_experts, N,
+                              lhs_indices, rhs_indices, batch, transpose, group_size, bits, mode,
+                              sorted_indices, y, scratch, QMM_GATHER_STATIC_SCRATCH_BYTES, stream);
+    } catch (...) {
+        return fail(QMM_ERR_CUDA, "unexpected exception in qmm_gather_qmm_static");
+    }
+}
+
 qmm_status qmm_device_status(void *stream, int reset) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");

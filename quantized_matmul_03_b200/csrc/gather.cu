@@ -19,6 +19,7 @@
 // Everything the kernels need is in the caller's workspace; nothing is
 // allocated.  The layout of that workspace is gather_ws_layout below.
 #include <algorithm>
+#include <mutex>
 
 #include "qmm_internal.cuh"
 
@@ -322,6 +323,33 @@ cudaError_t launch_gather_tc(qmm_dtype dt, const GatherCall &c, cudaStream_t s) 
     g.chunks = chunks;
     g.dst_rows = dst_rows;
     return launch_gemm_grouped(dt, g, s);
+}
+
+// ---------------------------------------------------------------------------
+// Built-in scratch for qmm_gather_qmm_static: a fixed device array in this
+// module, so that callers without a device allocator get the tensor-core path
+// without passing a workspace.  Its address is looked up once per device.
+// Nothing in it needs to start at zero: the preparation kernel writes every
+// byte the later kernels read.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_gather_scratch[QMM_GATHER_STATIC_SCRATCH_BYTES];
+
+cudaError_t gather_static_scratch(void **ptr) {
+    static void *cached[64] = {nullptr};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_gather_scratch);
+        if (e != cudaSuccess) return e;
+        cached[dev] = p;
+    }
+    *ptr = cached[dev];
+    return cudaSuccess;
 }
 
 }  // namespace qmm

@@ -146,6 +146,9 @@ struct GatherCall {
     void *workspace;
 };
 cudaError_t launch_gather_tc(qmm_dtype dt, const GatherCall &c, cudaStream_t s);
+// Device address of the built-in scratch (QMM_GATHER_STATIC_SCRATCH_BYTES) on
+// the current device; looked up on the first call per device.
+cudaError_t gather_static_scratch(void **ptr);
 
 int num_sms();
 void count_launches(int n);  // bump the process-wide launch counter
