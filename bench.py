@@ -293,6 +293,79 @@ def bench_prefill(bits, steps, warmup, world, device):
     return dict(total_ms=total_ms, per_ms=per_ms, launches=launches, flops=flops)
 
 
+def roofline_frac(t_ms, nbytes, flops, pk):
+    """Fraction of max(bytes / HBM bandwidth, flops / bf16 peak) achieved."""
+    t_roof = max(nbytes / (pk["hbm_gbs"] * 1e9), flops / (pk["bf16_tflops"] * 1e12))
+    return t_roof / (t_ms * 1e-3), ("hbm" if nbytes / (pk["hbm_gbs"] * 1e9) >=
+                                     flops / (pk["bf16_tflops"] * 1e12) else "tensor")
+
+
+def bench_moe(steps, warmup, world, device):
+    """gather_qmm on the MoE workload: 8 experts W [14336, 4096] int4 gs 64,
+    x [512, 1, 4096], rhs Zipf(1.2).  The stacked experts (264 MB) exceed L2,
+    so one copy suffices.  A step is the whole call (prepare, gather, product)."""
+    from quantized_matmul_03_b200 import binding as qb
+    c = wl.moe_case()
+    wq, s, b = make_packed(c.w, c.group_size, c.bits, 1, device)[0]
+    del c.w
+    x = c.x.to(device)
+    rhs = c.rhs_indices.to(device)
+    batch, k = x.shape[0], x.shape[2]
+    ws = torch.empty(qb.qmm_gather_qmm_workspace_size(batch, 1, k, wq.shape[0]),
+                     dtype=torch.uint8, device=device)
+    y = torch.empty((batch, 1, N_OUT), dtype=torch.bfloat16, device=device)
+    fns = [lambda: qb.qmm_gather_qmm(x, wq, s, b, None, rhs, True, c.group_size, c.bits,
+                                     workspace=ws, out=y)]
+    total_ms, per_ms, launches = timed_launches(fns, steps, warmup, world)
+    nbytes = wq.shape[0] * weight_bytes(N_OUT, K_IN, c.bits, c.group_size)
+    return dict(per_ms=per_ms, launches=launches, bytes=nbytes,
+                flops=2 * batch * N_OUT * K_IN)
+
+
+def run_suite(args, world, device, pk):
+    """Every measured configuration, one entry each (not the headline line)."""
+    from quantized_matmul_03_b200 import binding as qb
+    out = []
+    for m in (1, 4, 8, 16):
+        d = bench_decode(m, args.steps, args.warmup, world, device)
+        nb = d["bytes"] + 2 * m * (K_IN + N_OUT)
+        f, bound = roofline_frac(d["per_ms"], nb, d["flops"], pk)
+        out.append({"workload": f"decode_m{m}_int4_gs64", "us": d["per_ms"] * 1e3,
+                    "GB/s": d["bytes"] / (d["per_ms"] * 1e-3) / 1e9, "frac": f, "bound": bound})
+        del d
+    for bits in (4, 8):
+        pre = bench_prefill(bits, max(3, min(args.steps, 20)), args.warmup, world, device)
+        tf = pre["flops"] / (pre["per_ms"] * 1e-3) / 1e12
+        out.append({"workload": f"prefill_m2048_int{bits}_gs64", "us": pre["per_ms"] * 1e3,
+                    "TFLOP/s": tf, "frac": tf / pk["bf16_tflops"], "bound": "tensor"})
+    w = wl.sweep_weight()
+    for bits in (2, 4, 8):
+        for gs in (32, 64, 128):
+            for transpose in (True, False):
+                wb = weight_bytes(4096, 4096, bits, gs)
+                copies = max(2, -(-256_000_000 // wb))  # > 2x L2 per rotation
+                packs = make_packed(w, gs, bits, copies, device)
+                for m in (1, 16, 256):
+                    x = wl.sweep_x(m).to(device)
+                    y = torch.empty((m, 4096), dtype=torch.bfloat16, device=device)
+                    fns = [lambda p=p: qb.qmm_quantized_matmul(x, *p, transpose, gs, bits, out=y)
+                           for p in packs]
+                    _, per_ms, _ = timed_launches(fns, args.steps, args.warmup, world)
+                    flops = 2 * m * 4096 * 4096
+                    f, bound = roofline_frac(per_ms, wb + 4 * m * 4096, flops, pk)
+                    out.append({"workload": f"sweep_b{bits}_gs{gs}_{'t' if transpose else 'n'}_m{m}",
+                                "us": per_ms * 1e3, "frac": f, "bound": bound})
+                del packs
+                torch.cuda.empty_cache()
+    moe = bench_moe(max(3, min(args.steps, 50)), args.warmup, world, device)
+    f, bound = roofline_frac(moe["per_ms"], moe["bytes"], moe["flops"], pk)
+    out.append({"workload": "moe_e8_t512_int4_gs64", "us": moe["per_ms"] * 1e3,
+                "GB/s": moe["bytes"] / (moe["per_ms"] * 1e-3) / 1e9,
+                "TFLOP/s": moe["flops"] / (moe["per_ms"] * 1e-3) / 1e12, "frac": f,
+                "bound": bound, "launches_per_step": moe["launches"] / max(3, min(args.steps, 50))})
+    return out
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample of the decode workload)
 # ---------------------------------------------------------------------------
@@ -367,6 +440,9 @@ def main():
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the prefill GEMM (for profiling); prints its own line")
     ap.add_argument("--prefill-bits", type=int, default=4)
+    ap.add_argument("--suite", action="store_true",
+                    help="time every configuration (decode M 1/4/8/16, prefill int4/int8, "
+                         "the 54-point sweep, MoE) and print one JSON line of results")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
     args = ap.parse_args()
@@ -381,6 +457,13 @@ def main():
     qb.lib()  # fails loudly if the library was not built
     device = torch.device("cuda", local)
     pk = peaks()
+
+    if args.suite:
+        with ClockSampler(local) as clk:
+            suite = run_suite(args, world, device, pk)
+        if rank == 0:
+            print(json.dumps({"suite": suite, "peaks": pk, "clocks": clk.summary()}), flush=True)
+        return 0
 
     if args.prefill_only:
         pre = bench_prefill(args.prefill_bits, args.steps, args.warmup, world, device)

@@ -7,13 +7,13 @@
  *
  * What it computes, and where that comes from:
  *
- *  - Group-wise quantization "runs along the last axis" of a rank>=2 tensor
- *    (EMLX.Quantization, section `quantize`); "every group_size elements in a
- *    row of w are quantized together" and there is "one floating point scale
- *    and bias per group_size of elements" (mlx-rs ops/quantization.rs, doc
- *    comments of `quantize` and `quantized_matmul`).
- *  - Each element takes `bits` bits packed into unsigned 32-bit words; for
- *    bits=4 "8 nibbles per uint32", so the last axis shrinks by 32/bits
+ *  - Quantization works along the last axis of a tensor of rank 2 or more
+ *    (EMLX.Quantization, section `quantize`): each run of group_size
+ *    consecutive elements of a row forms a group with its own floating-point
+ *    scale and bias (mlx-rs ops/quantization.rs, doc comments of `quantize`
+ *    and `quantized_matmul`).
+ *  - Each element takes `bits` bits packed into unsigned 32-bit words;
+ *    with bits=4 a word holds eight codes, so the last axis shrinks by 32/bits
  *    (Emily.QuantizedWeight, section Layout).
  *  - Scales and biases have the source weight's dtype and shape
  *    (..., last_dim / group_size) (Emily.QuantizedWeight, section Layout).

@@ -3,8 +3,8 @@
 Tensors are CPU ``torch`` tensors; packed words are stored as ``torch.int32``
 holding the uint32 bit patterns.  Quantize and dequantize run in the C half
 (``qmm_oracle.c``); the products are a float64 matmul (library primitive) on
-the dequantized weight, exactly "dequantize, then a dense matmul", which is
-how the mlx-rs tests ``test_quantized_matmul`` and ``test_gather_qmm`` define
+the dequantized weight (dequantize first, then an ordinary dense product),
+which is how the mlx-rs tests ``test_quantized_matmul`` and ``test_gather_qmm`` define
 the expected result of ``quantized_matmul`` and ``gather_qmm``.
 """
 from __future__ import annotations

@@ -1,9 +1,10 @@
 // api.cu -- the extern "C" boundary of libqmm (declared in include/qmm.h).
 //
 // Every entry point validates its arguments completely before enqueueing
-// anything, reports failures as qmm_status values (the Rust binding on the
-// mlx-rs page returns Result / Exception, Emily raises "with a clear error
-// before touching MLX"), and never lets a C++ exception cross the ABI.
+// anything, reports failures as qmm_status values (mlx-rs
+// ops/quantization.rs returns Result with an Exception; Emily checks its
+// arguments and raises before any MLX call), and never lets a C++ exception
+// cross the ABI.
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>

@@ -45,7 +45,6 @@ constexpr int kThreads = 32 * (kCW + 1);  // plus one producer warp
 // DP2A.hi bytes 2,3, so the activation pairs of plane p are
 //   lo: (x[p], x[NP + p])     hi: (x[2NP + p], x[3NP + p]).
 template <int BITS> struct Planes {
-    static constexpr int EPW = 32 / BITS;      // codes per word
     static constexpr int NP = 8 / BITS;        // planes per word
     static constexpr uint32_t BYTE_MASK = ((1u << BITS) - 1u) * 0x01010101u;
     // element (within the word) of half h (0/1) of pair k (k = 2p + {0: lo, 1: hi})
@@ -372,13 +371,11 @@ cudaError_t launch_stream(const QmmArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// One launch for rows [0, mr) of a (mr in {1, 2, 4}, a variant that fits).
 template <typename T, int BITS>
-cudaError_t stream_bits(const QmmArgs &a, cudaStream_t s) {
-    const int mr = a.M == 1 ? 1 : (a.M == 2 ? 2 : 4);
+cudaError_t stream_rows(const QmmArgs &a, int mr, cudaStream_t s) {
     StreamPlan p{};
     if (!plan_stream(a, mr, 1, p)) return cudaErrorInvalidValue;
-    // Only the variants that fit in registers are instantiated; the others are
-    // refused by stream_variant_fits() and go to the general kernel.
     if (mr == 1) {
         if (p.upl == 1) return launch_stream<T, BITS, 1, 1>(a, s);
         if constexpr (BITS != 2) return launch_stream<T, BITS, 1, 2>(a, s);
@@ -391,6 +388,37 @@ cudaError_t stream_bits(const QmmArgs &a, cudaStream_t s) {
         if (mr == 4 && p.upl == 1) return launch_stream<T, BITS, 4, 1>(a, s);
     }
     return cudaErrorInvalidValue;
+}
+
+// Widest variant (4, 2 or 1 rows) that fits the registers for `rows`
+// remaining activation rows; 0 if none does.
+int pick_rows(const QmmArgs &a, int64_t rows) {
+    for (int mr : {4, 2, 1}) {
+        if (mr > rows) continue;
+        QmmArgs t = a;
+        t.M = mr;
+        StreamPlan p{};
+        if (plan_stream(t, mr, 1, p) && stream_variant_fits(a.bits, mr, p.upl)) return mr;
+    }
+    return 0;
+}
+
+// Rows go through the widest variant that fits, a launch per row block (for
+// example 4-bit codes: 3 rows = 2 + 1, 4 rows = 2 + 2).
+template <typename T, int BITS>
+cudaError_t stream_bits(const QmmArgs &a, cudaStream_t s) {
+    for (int64_t m0 = 0; m0 < a.M;) {
+        const int mr = pick_rows(a, a.M - m0);
+        if (mr == 0) return cudaErrorInvalidValue;
+        QmmArgs t = a;
+        t.M = mr;
+        t.x = static_cast<const T *>(a.x) + m0 * a.K;
+        t.y = static_cast<T *>(a.y) + m0 * a.N;
+        const cudaError_t e = stream_rows<T, BITS>(t, mr, s);
+        if (e != cudaSuccess) return e;
+        m0 += mr;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -408,10 +436,9 @@ bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a) {
     if ((reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases) |
          reinterpret_cast<uintptr_t>(a.wq)) & 15)
         return false;
-    const int mr = a.M == 1 ? 1 : (a.M == 2 ? 2 : 4);
-    StreamPlan p{};
-    if (!plan_stream(a, mr, 1, p)) return false;
-    return stream_variant_fits(a.bits, mr, p.upl);
+    // Every row block must find a variant; one-row launches always can when
+    // the single-row plan fits.
+    return pick_rows(a, 1) == 1;
 }
 
 cudaError_t launch_gemv_fast(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
