@@ -57,12 +57,27 @@ def dist_setup():
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:  # host-only runs (the reference arm, CPU tests of the rank logic)
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
+
+
+def dist_teardown(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def whole_job_rate(world, steps, units_per_step, slowest_total_ms):
+    """Units per second of the whole job: every rank does `steps` steps of
+    `units_per_step`, and the job takes as long as its slowest rank."""
+    return world * steps * units_per_step / (slowest_total_ms * 1e-3)
 
 
 def barrier(world):
@@ -75,7 +90,8 @@ def max_over_ranks(world, v: float) -> float:
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -451,7 +467,10 @@ def main():
 
     world, rank, local = dist_setup()
     if args.impl == "reference":
-        return run_reference(args, world, rank)
+        rc = run_reference(args, world, rank)
+        barrier(world)
+        dist_teardown(world)
+        return rc
 
     from quantized_matmul_03_b200 import binding as qb
     qb.lib()  # fails loudly if the library was not built
@@ -485,7 +504,7 @@ def main():
 
     total_ms = max_over_ranks(world, d["total_ms"])
     per_ms = max_over_ranks(world, d["per_ms"])
-    value = world * args.steps * d["bytes"] / (total_ms * 1e-3) / 1e9
+    value = whole_job_rate(world, args.steps, d["bytes"], total_ms) / 1e9
     achieved = d["bytes"] / (per_ms * 1e-3) / 1e9
     e2e = bench_decode_e2e(d, args.steps, args.warmup, world, device)
 
@@ -522,9 +541,7 @@ def main():
         line["cpu_baseline"] = oracle_decode_sample(args.cpu_budget_s)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    dist_teardown(world)
     return 0
 
 
