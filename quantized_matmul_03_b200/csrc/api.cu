@@ -196,12 +196,14 @@ qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K, const uint3
         if (g_path == QMM_PATH_GEMM) {
             if (!tc_ok)
                 return fail(QMM_ERR_UNSUPPORTED,
-                            "the tensor-core path needs bf16/f16, transpose, K %% 64 == 0");
+                            "the tensor-core path needs bf16/f16, K %% 64 == 0 and whole 16-byte "
+                            "packed rows");
             return finish_launch(launch_gemm(dtype, a, s), "tensor-core gemm launch");
         }
-        // Decode shapes stream the weight through the SIMT kernels; larger
-        // activation counts use the tensor cores.
-        const bool few_rows = a.M <= kGemvMaxRows;
+        // Decode shapes of the [N, K] layout stream the weight through the
+        // SIMT decode kernel; larger activation counts, and the [K, N] layout
+        // at any count, use the tensor cores.
+        const bool few_rows = a.M <= kGemvMaxRows && a.transpose;
         if (g_path == QMM_PATH_GEMV || few_rows || !tc_ok) {
             if (gemv_fast_supported(dtype, a))
                 return finish_launch(launch_gemv_fast(dtype, a, s), "gemv launch");

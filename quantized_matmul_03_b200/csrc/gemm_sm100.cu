@@ -105,6 +105,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[32]) {
         : "r"(taddr)
         : "memory");
 }
+// True on one lane of the (converged) warp.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -124,10 +134,17 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+// MN-major, 128-byte swizzle: atoms of 64 MN-elements (128 bytes) x 8 K-rows
+// (1 KB); atoms along MN LBO bytes apart, groups of 8 K-rows SBO bytes apart.
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
 // Instruction descriptor of kind::f16: fp32 accumulator, A/B both bf16 (or
-// both f16), both K-major, shape M x N.
-__host__ __device__ constexpr uint32_t make_idesc(bool f16, int m, int n) {
-    return (1u << 4) | ((f16 ? 0u : 1u) << 7) | ((f16 ? 0u : 1u) << 10) |
+// both f16), B K-major, A K-major (or MN-major with a_mn), shape M x N.
+__host__ __device__ constexpr uint32_t make_idesc(bool f16, int m, int n, bool a_mn = false) {
+    return (1u << 4) | ((f16 ? 0u : 1u) << 7) | ((f16 ? 0u : 1u) << 10) | ((a_mn ? 1u : 0u) << 15) |
            ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
@@ -276,10 +293,18 @@ __device__ __forceinline__ int tile_count(const GemmParams &p) {
 // 64-row boxes (only as many as the chunk has rows), from tmap_xs (the sorted
 // copy) or tmap_x (x itself, when the sorted order is x's own); the MMA N is
 // the chunk's row count rounded up to 16; outputs go through the row map.
-template <typename T, int BITS, int BN, bool GROUPED>
+//
+// KMAJOR = false: the weight is stored [K, N] (transpose = false), packed and
+// grouped along N.  Each 64 x 128 packed tile (64 k-rows of 128 features)
+// arrives by TMA; dequantize thread (k, h) expands the 64 features of half h
+// of row k and writes them as 16-byte chunks of an MN-major, 128-byte-swizzled
+// A tile (atoms of 64 features x 8 k-rows), which the MMA reads with the
+// A-major bit set.  Everything else is shared with the K-major path.
+template <typename T, int BITS, int BN, bool GROUPED, bool KMAJOR = true>
 __global__ void __launch_bounds__(kThreads, 1)
 qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_xs,
                 const __grid_constant__ CUtensorMap tmap_w, const GemmParams p) {
+    static_assert(KMAJOR || !GROUPED, "the grouped product is built for the [N, K] layout");
     constexpr bool kF16 = std::is_same<T, __half>::value;
     constexpr int A_BYTES = kBM * kBK * 2;         // 16 KB dequantized tile
     constexpr int B_BYTES = BN * kBK * 2;          // activation tile
@@ -287,7 +312,9 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     constexpr int P_BYTES = kBM * P_ROW;
     constexpr int W_WORDS = kBK * BITS / 32;       // packed words per row per k-block
     constexpr uint32_t TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
-    constexpr uint32_t IDESC = make_idesc(kF16, kBM, BN);
+    constexpr uint32_t IDESC = make_idesc(kF16, kBM, BN, !KMAJOR);
+    // MN-major A tile: feature atoms (64 features) 1 KB apart, 8-k-row groups 2 KB apart.
+    constexpr uint32_t MN_LBO = 1024, MN_SBO = 2048;
 
     extern __shared__ uint8_t smem_raw[];
     const int S = p.stages;
@@ -327,7 +354,57 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     const int gpr = p.K / p.group_size;
     const int num_tiles = tile_count<GROUPED>(p);
 
-    if (warp < kDqWarps) {
+    if (!KMAJOR && warp < kDqWarps) {
+        // --------------- dequantize, weight stored [K, N] ---------------
+        // Thread t of a group: k-row kl = (t mod 8) + 8 (t div 16), feature
+        // half h = (t div 8) mod 2, so the 8 threads of a store phase cover 8
+        // different k-rows of one half (conflict-free 16-byte stores).
+        const int grp = warp >> 2, t = threadIdx.x & (kBM - 1);
+        const int kl = (t & 7) + 8 * (t >> 4), h = (t >> 3) & 1;
+        const uint16_t *sc = static_cast<const uint16_t *>(p.scales);
+        const uint16_t *bi = static_cast<const uint16_t *>(p.biases);
+        const int gpn = p.N / p.group_size;  // groups per stored row
+        int c = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            const Tile tl = decode_tile<BN, GROUPED>(p, tile);
+            const int f0 = tl.n0 + 64 * h;  // first feature of this thread's half
+            const bool v0 = f0 < p.N, v1 = f0 + 32 < p.N;
+            const int g0 = f0 / p.group_size, g1 = (f0 + 32) / p.group_size;
+            for (int kb = 0; kb < KB; ++kb, ++c) {
+                if ((c & 1) != grp) continue;
+                const int s = c % S;
+                const int64_t srow = (int64_t)(kb * kBK + kl) * gpn;
+                const uint16_t s0 = v0 ? __ldg(sc + srow + g0) : (uint16_t)0;
+                const uint16_t b0v = v0 ? __ldg(bi + srow + g0) : (uint16_t)0;
+                const uint16_t s1 = v1 ? __ldg(sc + srow + g1) : (uint16_t)0;
+                const uint16_t b1v = v1 ? __ldg(bi + srow + g1) : (uint16_t)0;
+                ptx::mbar_wait(full_pb + 8 * s, (c / S) & 1, p.err);
+                // Packed row kl (16*BITS bytes, unswizzled), half h.
+                const uint8_t *prow = pg + s * P_BYTES + kl * (16 * BITS) + h * (8 * BITS);
+                uint32_t w[2 * BITS];
+#pragma unroll
+                for (int q = 0; q < BITS / 2; ++q) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(prow + 16 * q);
+                    w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
+                }
+                uint8_t *arow = gbase + (a0 - base) + s * A_BYTES + (kl >> 3) * MN_SBO + h * MN_LBO +
+                                (kl & 7) * 128;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint4 out[4];
+                    dequant_half<T, BITS>(w + hh * BITS, hh ? s1 : s0, hh ? b1v : b0v, out);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int chunk = 4 * hh + j;
+                        *reinterpret_cast<uint4 *>(arow + ((chunk ^ (kl & 7)) << 4)) = out[j];
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(full_a + 8 * s);
+            }
+        }
+    } else if (warp < kDqWarps) {
         // ------------------------- dequantize -------------------------
         // Two groups of four warps take alternate k-blocks, so two k-blocks
         // are dequantized at once; thread r of a group owns weight row r.
@@ -480,7 +557,10 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     const int s = c % S;
                     if (c >= S) ptx::mbar_wait(empty + 8 * s, ((c / S) + 1) & 1, p.err);
                     ptx::mbar_arrive_expect_tx(full_pb + 8 * s, P_BYTES + bbytes);
-                    tma_load_2d(p0 + s * P_BYTES, &tmap_w, kb * W_WORDS, t.wrow0, full_pb + 8 * s);
+                    if constexpr (KMAJOR)
+                        tma_load_2d(p0 + s * P_BYTES, &tmap_w, kb * W_WORDS, t.wrow0, full_pb + 8 * s);
+                    else  // 64 k-rows x 128 features of the [K, N] packed weight
+                        tma_load_2d(p0 + s * P_BYTES, &tmap_w, t.n0 * BITS / 32, kb * kBK, full_pb + 8 * s);
                     for (int j = 0; j < nbox; ++j)
                         tma_load_2d(b0 + s * B_BYTES + j * 64 * kBK * 2, xmap, kb * kBK, t.m0 + 64 * j,
                                     full_pb + 8 * s);
@@ -492,32 +572,44 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         }
     } else {
         // ------------------------- MMA issuer -------------------------
-        if (lane == 0) {
-            int c = 0, i = 0;
-            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
-                const int acc = i & 1;
-                uint32_t idesc = IDESC;
-                if constexpr (GROUPED) {
-                    const Tile t = decode_tile<BN, GROUPED>(p, tile);
-                    idesc = make_idesc(kF16, kBM, (t.rows + 15) & ~15);  // N: 16..BN, step 16
-                }
-                if (i >= 2) ptx::mbar_wait(acc_empty + 8 * acc, ((i >> 1) + 1) & 1, p.err);
-                tc_fence_after();
-                const uint32_t d = tmem_base + acc * BN;
-                for (int kb = 0; kb < KB; ++kb, ++c) {
-                    const int s = c % S;
-                    ptx::mbar_wait(full_a + 8 * s, (c / S) & 1, p.err);
-                    ptx::mbar_wait(full_pb + 8 * s, (c / S) & 1, p.err);
+        // The warp walks the loop converged; one elected lane waits and
+        // issues, one wait and one commit per k-block: a complete full_a
+        // implies a complete full_pb, since the dequantize warps waited for
+        // the stage before writing its A tile.
+        const bool leader = elect_one();
+        int c = 0, i = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
+            const int acc = i & 1;
+            uint32_t idesc = IDESC;
+            {
+                const Tile t = decode_tile<BN, GROUPED>(p, tile);
+                if (GROUPED || t.rows < BN) idesc = make_idesc(kF16, kBM, (t.rows + 15) & ~15, !KMAJOR);
+            }
+            if (leader && i >= 2) ptx::mbar_wait(acc_empty + 8 * acc, ((i >> 1) + 1) & 1, p.err);
+            __syncwarp();
+            tc_fence_after();
+            const uint32_t d = tmem_base + acc * BN;
+            for (int kb = 0; kb < KB; ++kb, ++c) {
+                const int s = c % S;
+                if (leader) {
+                    ptx::mbar_wait<false>(full_a + 8 * s, (c / S) & 1, p.err);
                     tc_fence_after();
-                    const uint64_t da = sw128_desc(a0 + s * A_BYTES);
                     const uint64_t db = sw128_desc(b0 + s * B_BYTES);
-#pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k)  // UMMA K = 16: 32 bytes along the row
-                        tc_mma(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
+                    // UMMA K = 16: 32 bytes along a K-major 128-byte row, or two
+                    // 8-k-row groups (2 * SBO bytes) of the MN-major tile.
+                    const uint64_t da = KMAJOR ? sw128_desc(a0 + s * A_BYTES)
+                                               : sw128_mn_desc(a0 + s * A_BYTES, MN_LBO, MN_SBO);
+                    constexpr uint64_t DA = KMAJOR ? 2 : (2 * MN_SBO) >> 4;
+                    tc_mma(d, da, db, idesc, kb != 0);
+                    tc_mma(d, da + DA, db + 2, idesc, 1);
+                    tc_mma(d, da + 2 * DA, db + 4, idesc, 1);
+                    tc_mma(d, da + 3 * DA, db + 6, idesc, 1);
                     tc_commit(empty + 8 * s);
                 }
-                tc_commit(acc_full + 8 * acc);
+                __syncwarp();
             }
+            if (leader) tc_commit(acc_full + 8 * acc);
+            __syncwarp();
         }
     }
     tc_fence_before();
@@ -599,8 +691,17 @@ bool make_weight_map(CUtensorMap *map, const uint32_t *wq, uint64_t rows, int64_
                                  : (BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B));
 }
 
-template <typename T, int BITS, int BN>
-cudaError_t run_gemm(const QmmArgs &a, cudaStream_t s) {
+// Packed weight stored [K, N]: one 64 k-row x 128-feature tile per box
+// (128*BITS/32 words per row, unswizzled).
+template <int BITS>
+bool make_weight_map_kn(CUtensorMap *map, const uint32_t *wq, int64_t K, int64_t N) {
+    const uint64_t words = (uint64_t)N * BITS / 32;
+    return make_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, words, (uint64_t)K, words * 4,
+                       kBM * BITS / 32, kBK, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+template <typename T, int BITS, int BN, bool KMAJOR>
+cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
     int stages;
     size_t smem;
     if (!gemm_smem_plan<BITS, BN>(stages, smem)) return cudaErrorInvalidConfiguration;
@@ -609,7 +710,9 @@ cudaError_t run_gemm(const QmmArgs &a, cudaStream_t s) {
     if (!make_map_2d(&tx, act_type(kF16), a.x, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * 2, kBK, BN,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    if (!make_weight_map<BITS>(&tw, a.wq, (uint64_t)a.N, a.K)) return cudaErrorInvalidValue;
+    if (KMAJOR ? !make_weight_map<BITS>(&tw, a.wq, (uint64_t)a.N, a.K)
+               : !make_weight_map_kn<BITS>(&tw, a.wq, a.K, a.N))
+        return cudaErrorInvalidValue;
 
     GemmParams p{};
     p.scales = a.scales;
@@ -624,13 +727,18 @@ cudaError_t run_gemm(const QmmArgs &a, cudaStream_t s) {
     p.num_tiles = p.m_tiles * p.n_tiles;
     p.stages = stages;
     p.err = device_error_word();
-    auto kern = qgemm_tc_kernel<T, BITS, BN, false>;
+    auto kern = qgemm_tc_kernel<T, BITS, BN, false, KMAJOR>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = std::min(p.num_tiles, num_sms());
     kern<<<grid, kThreads, smem, s>>>(tx, tx, tw, p);
     count_launches(1);
     return cudaGetLastError();
+}
+
+template <typename T, int BITS, int BN>
+cudaError_t run_gemm(const QmmArgs &a, cudaStream_t s) {
+    return a.transpose ? run_gemm_layout<T, BITS, BN, true>(a, s) : run_gemm_layout<T, BITS, BN, false>(a, s);
 }
 
 template <typename T, int BITS, int BN>
@@ -699,13 +807,13 @@ cudaError_t grouped_bits(const GroupedArgs &g, cudaStream_t s) {
 
 }  // namespace
 
-// The tensor-core path: bf16/f16, transpose layout, K a multiple of the
-// 64-wide k-block, whole 16-byte packed rows, sizes in int range.
+// The tensor-core path: bf16/f16, K a multiple of the 64-wide k-block, packed
+// rows of whole 16-byte units (K*bits/8 for [N, K] storage, N*bits/8 for
+// [K, N] storage), sizes in int range.
 bool gemm_supported(qmm_dtype dt, const QmmArgs &a) {
-    if (!a.transpose) return false;
     if (dt != QMM_BF16 && dt != QMM_F16) return false;
     if (a.K % kBK != 0) return false;
-    if ((a.K * a.bits / 8) % 16 != 0) return false;
+    if (((a.transpose ? a.K : a.N) * a.bits / 8) % 16 != 0) return false;
     if (a.M > INT32_MAX / 2 || a.N > INT32_MAX / 2 || a.K > INT32_MAX / 2) return false;
     return encode_fn() != nullptr;
 }

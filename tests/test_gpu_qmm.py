@@ -120,6 +120,27 @@ def test_gemm_tensor_core(dtype, bits, gs, m, n, k):
     run_case(x, w, gs, bits, True, "gemm")
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("bits,gs", [(4, 64), (4, 32), (4, 128), (8, 64), (8, 32), (2, 128), (2, 64)])
+@pytest.mark.parametrize("m,k,n", [(1, 64, 128), (16, 1024, 640), (17, 128, 384),
+                                   (100, 512, 1152), (300, 256, 256)])
+def test_gemm_tensor_core_kn_layout(dtype, bits, gs, m, k, n):
+    """The tcgen05 path with the weight stored [K, N] (transpose = false),
+    groups along N: MN-major dequantized tiles, ragged feature tiles."""
+    if n % gs:
+        pytest.skip("N must be a multiple of the group size")
+    w = wl.with_outliers((k, n), seed=m + n + bits, dtype=dtype)
+    x = wl.normal((m, k), seed=k + m + 1, dtype=dtype)
+    run_case(x, w, gs, bits, False, "gemm")
+
+
+def test_gemm_kn_ragged_features():
+    # 160 features: the second 128-feature tile is 32 wide (TMA zero fill).
+    w = wl.with_outliers((128, 160), seed=3, dtype=torch.bfloat16)
+    x = wl.normal((40, 128), seed=4, dtype=torch.bfloat16)
+    run_case(x, w, 32, 4, False, "gemm")
+
+
 def test_gemm_path_refuses_unsupported():
     w = wl.normal((64, 96), 1, 1.0, torch.bfloat16)
     wq, s, b = oracle.quantize(w, 32, 4)
