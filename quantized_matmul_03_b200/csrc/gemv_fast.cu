@@ -37,7 +37,7 @@
 namespace qmm {
 namespace {
 
-constexpr int kCW = 8;                    // consumer warps
+constexpr int kCW = 12;                   // consumer warps
 constexpr int kThreads = 32 * (kCW + 1);  // plus one producer warp
 
 // Code planes of a packed word: plane p = (w >> p*BITS) & byte-mask, whose
@@ -290,9 +290,10 @@ struct StreamPlan {
     size_t smem;
 };
 
-// Shared memory per CTA: the whole SM's worth (one CTA per SM) or half of it
-// (two CTAs per SM, which doubles the warps available to hide latency).
-constexpr size_t kSmemPerSm = 200 * 1024;
+// Shared memory per CTA: one CTA per SM with a ring of at most 110 KB, so that
+// the next call's CTA (launched early by programmatic dependent launch) fits
+// beside it and fills its own ring while this one finishes.
+constexpr size_t kSmemPerSm = 110 * 1024;
 
 int rows_per_team_stage(int mr) { return mr == 4 ? 2 : 4; }
 
@@ -337,19 +338,15 @@ template <typename T, int BITS, int MR, int UPL>
 cudaError_t launch_stream(const QmmArgs &a, cudaStream_t s) {
     constexpr int RPT = MR == 4 ? 2 : 4;
     auto kern = qgemv_stream_kernel<T, BITS, MR, UPL, RPT>;
-    // Two CTAs per SM when the registers and the halved ring allow it.
+    // One CTA per SM (the next call's CTAs take the other half of the SM).
     StreamPlan p{};
-    cudaError_t e = cudaSuccess;
-    for (int per_sm = 2; per_sm >= 1; --per_sm) {
-        if (!plan_stream(a, MR, per_sm, p)) continue;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
-        if (e != cudaSuccess) return e;
-        int got = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&got, kern, kThreads, p.smem);
-        if (e != cudaSuccess) return e;
-        if (got >= per_sm) break;
-        if (per_sm == 1) return cudaErrorInvalidConfiguration;
-    }
+    if (!plan_stream(a, MR, 1, p)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+    if (e != cudaSuccess) return e;
+    int got = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&got, kern, kThreads, p.smem);
+    if (e != cudaSuccess) return e;
+    if (got < 1) return cudaErrorInvalidConfiguration;
     // Programmatic stream serialization: this grid may start while the
     // preceding kernel of the stream finishes (see grid_dependency_wait()).
     cudaLaunchConfig_t cfg = {};
