@@ -248,6 +248,7 @@ struct GemmParams {
     void *y;
     int M, N, K, group_size;
     int m_tiles, n_tiles, num_tiles, stages;
+    int sb_tma;  // [N, K] layout: scale/bias windows arrive by TMA with each stage
     int *err;
     // Grouped (gather_qmm) mode only: the chunk table and row map the
     // preparation kernel wrote.  Tile t covers chunk t / n_tiles and weight
@@ -303,7 +304,8 @@ __device__ __forceinline__ int tile_count(const GemmParams &p) {
 template <typename T, int BITS, int BN, bool GROUPED, bool KMAJOR = true>
 __global__ void __launch_bounds__(kThreads, 1)
 qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_xs,
-                const __grid_constant__ CUtensorMap tmap_w, const GemmParams p) {
+                const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s,
+                const __grid_constant__ CUtensorMap tmap_b, const GemmParams p) {
     static_assert(KMAJOR || !GROUPED, "the grouped product is built for the [N, K] layout");
     constexpr bool kF16 = std::is_same<T, __half>::value;
     constexpr int A_BYTES = kBM * kBK * 2;         // 16 KB dequantized tile
@@ -323,7 +325,11 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
     const uint32_t a0 = base, b0 = a0 + S * A_BYTES, p0 = b0 + S * B_BYTES;
-    const uint32_t bar0 = p0 + S * P_BYTES;
+    // Scale/bias windows ([N, K] layout with sb_tma): per stage 8 groups x 128
+    // rows of scales (2 KB) then of biases (2 KB), row r at byte 16 r.
+    constexpr int SB_BYTES = 2 * kBM * 16;
+    const uint32_t sb0 = p0 + S * P_BYTES;
+    const uint32_t bar0 = sb0 + (p.sb_tma ? S * SB_BYTES : 0);
     const uint32_t full_pb = bar0, full_a = bar0 + 8 * S, empty = bar0 + 16 * S;
     const uint32_t acc_full = bar0 + 24 * S, acc_empty = acc_full + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + (acc_empty + 16 - base));
@@ -422,7 +428,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
             const uint16_t *srow = sc + wrow * gpr, *brow = bi + wrow * gpr;
             uint4 s_cur = make_uint4(0, 0, 0, 0), b_cur = s_cur, s_nxt = s_cur, b_nxt = s_cur;
             int wbase = 0;  // first group of the current window
-            if (vec && rv) {
+            if (vec && rv && !p.sb_tma) {
                 s_cur = __ldg(reinterpret_cast<const uint4 *>(srow));
                 b_cur = __ldg(reinterpret_cast<const uint4 *>(brow));
                 if (gpr > 8) {
@@ -454,9 +460,21 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 if ((c & 1) != grp) continue;
                 const int s = c % S;
                 uint16_t s0, b0v, s1, b1v;
-                scale_bias((kb * kBK) / p.group_size, s0, b0v);
-                scale_bias((kb * kBK + 32) / p.group_size, s1, b1v);
+                const int g0 = (kb * kBK) / p.group_size, g1 = (kb * kBK + 32) / p.group_size;
+                if (!p.sb_tma) {
+                    scale_bias(g0, s0, b0v);
+                    scale_bias(g1, s1, b1v);
+                }
                 ptx::mbar_wait(full_pb + 8 * s, (c / S) & 1, p.err);
+                if (p.sb_tma) {
+                    // Row r's window of 8 groups starts at group (g0 & ~7).
+                    const uint8_t *sw = gbase + (sb0 - base) + s * SB_BYTES + r * 16;
+                    const int o0 = (g0 & 7) * 2, o1 = (g1 - (g0 & ~7)) * 2;
+                    s0 = *reinterpret_cast<const uint16_t *>(sw + o0);
+                    b0v = *reinterpret_cast<const uint16_t *>(sw + SB_BYTES / 2 + o0);
+                    s1 = *reinterpret_cast<const uint16_t *>(sw + o1);
+                    b1v = *reinterpret_cast<const uint16_t *>(sw + SB_BYTES / 2 + o1);
+                }
                 // The packed tile was staged with the swizzle matching its row
                 // width (none / 32B / 64B): 16-byte chunk q of row r sits at
                 // chunk q ^ ((r >> 2) & 1) (32-byte rows) or q ^ ((r >> 1) & 3)
@@ -556,7 +574,14 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 for (int kb = 0; kb < KB; ++kb, ++c) {
                     const int s = c % S;
                     if (c >= S) ptx::mbar_wait(empty + 8 * s, ((c / S) + 1) & 1, p.err);
-                    ptx::mbar_arrive_expect_tx(full_pb + 8 * s, P_BYTES + bbytes);
+                    ptx::mbar_arrive_expect_tx(full_pb + 8 * s,
+                                               P_BYTES + bbytes + (p.sb_tma ? SB_BYTES : 0));
+                    if (KMAJOR && p.sb_tma) {
+                        // the window of 8 groups holding this k-block's groups
+                        const int wx = ((kb * kBK) / p.group_size) & ~7;
+                        tma_load_2d(sb0 + s * SB_BYTES, &tmap_s, wx, t.wrow0, full_pb + 8 * s);
+                        tma_load_2d(sb0 + s * SB_BYTES + SB_BYTES / 2, &tmap_b, wx, t.wrow0, full_pb + 8 * s);
+                    }
                     if constexpr (KMAJOR)
                         tma_load_2d(p0 + s * P_BYTES, &tmap_w, kb * W_WORDS, t.wrow0, full_pb + 8 * s);
                     else  // 64 k-rows x 128 features of the [K, N] packed weight
@@ -664,16 +689,37 @@ int pick_bn(int64_t M) {
     return 256;
 }
 
-// Shared-memory budget of one CTA: S stages of (A + B + P) plus barriers.
+// Shared-memory budget of one CTA: S stages of (A + B + P [+ scale/bias
+// windows]) plus barriers.
 template <int BITS, int BN>
-bool gemm_smem_plan(int &stages, size_t &smem) {
+bool gemm_smem_plan(bool sb_tma, int &stages, size_t &smem) {
     constexpr int A_BYTES = kBM * kBK * 2, B_BYTES = BN * kBK * 2, P_BYTES = kBM * kBK * BITS / 8;
-    constexpr int STAGE = A_BYTES + B_BYTES + P_BYTES;
+    const int STAGE = A_BYTES + B_BYTES + P_BYTES + (sb_tma ? 2 * kBM * 16 : 0);
     constexpr size_t kSmemMax = 227 * 1024;
     const size_t fixed = 1024 /*alignment*/ + 64 /*acc bars + slot*/;
     stages = (int)std::min<size_t>(8, (kSmemMax - fixed) / (STAGE + 24));
     smem = fixed + (size_t)stages * (STAGE + 24);
     return stages >= 2;
+}
+
+// Staging the scale/bias windows costs 4 KB per stage; use it only when the
+// ring keeps its depth (it was measured faster at equal depth, slower with one
+// stage fewer).
+template <int BITS, int BN>
+bool sb_windows_fit() {
+    int s0, s1;
+    size_t m0, m1;
+    gemm_smem_plan<BITS, BN>(false, s0, m0);
+    gemm_smem_plan<BITS, BN>(true, s1, m1);
+    return s1 >= s0;
+}
+
+// Scale or bias window map over [rows, gpr] 16-bit values: 8 groups (16
+// bytes) x 128 rows per box, unswizzled.  Needs gpr % 8 == 0 (rows of whole
+// 16-byte units).
+bool make_sb_map(CUtensorMap *map, const void *ptr, uint64_t rows, int64_t gpr) {
+    return make_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, ptr, (uint64_t)gpr, rows, (uint64_t)gpr * 2, 8,
+                       kBM, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 CUtensorMapDataType act_type(bool f16) {
@@ -702,19 +748,29 @@ bool make_weight_map_kn(CUtensorMap *map, const uint32_t *wq, int64_t K, int64_t
 
 template <typename T, int BITS, int BN, bool KMAJOR>
 cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
+    const int64_t gpr = a.K / a.group_size;
+    const bool sb_tma = KMAJOR && gpr % 8 == 0 && sb_windows_fit<BITS, BN>();
     int stages;
     size_t smem;
-    if (!gemm_smem_plan<BITS, BN>(stages, smem)) return cudaErrorInvalidConfiguration;
+    if (!gemm_smem_plan<BITS, BN>(sb_tma, stages, smem)) return cudaErrorInvalidConfiguration;
     constexpr bool kF16 = std::is_same<T, __half>::value;
-    CUtensorMap tx, tw;
+    CUtensorMap tx, tw, ts, tb;
     if (!make_map_2d(&tx, act_type(kF16), a.x, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * 2, kBK, BN,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     if (KMAJOR ? !make_weight_map<BITS>(&tw, a.wq, (uint64_t)a.N, a.K)
                : !make_weight_map_kn<BITS>(&tw, a.wq, a.K, a.N))
         return cudaErrorInvalidValue;
+    if (sb_tma) {
+        if (!make_sb_map(&ts, a.scales, (uint64_t)a.N, gpr) || !make_sb_map(&tb, a.biases, (uint64_t)a.N, gpr))
+            return cudaErrorInvalidValue;
+    } else {
+        ts = tx;  // unused
+        tb = tx;
+    }
 
     GemmParams p{};
+    p.sb_tma = sb_tma ? 1 : 0;
     p.scales = a.scales;
     p.biases = a.biases;
     p.y = a.y;
@@ -731,7 +787,7 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = std::min(p.num_tiles, num_sms());
-    kern<<<grid, kThreads, smem, s>>>(tx, tx, tw, p);
+    kern<<<grid, kThreads, smem, s>>>(tx, tx, tw, ts, tb, p);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -743,13 +799,15 @@ cudaError_t run_gemm(const QmmArgs &a, cudaStream_t s) {
 
 template <typename T, int BITS, int BN>
 cudaError_t run_gemm_grouped(const GroupedArgs &g, cudaStream_t s) {
+    const int64_t gpr = g.K / g.group_size;
+    const bool sb_tma = gpr % 8 == 0 && sb_windows_fit<BITS, BN>();
     int stages;
     size_t smem;
-    if (!gemm_smem_plan<BITS, BN>(stages, smem)) return cudaErrorInvalidConfiguration;
+    if (!gemm_smem_plan<BITS, BN>(sb_tma, stages, smem)) return cudaErrorInvalidConfiguration;
     constexpr bool kF16 = std::is_same<T, __half>::value;
     // Activation maps: 64-row boxes over x viewed as [x_batch * M, K] and over
     // the sorted copy [rows, K].
-    CUtensorMap tx, txs, tw;
+    CUtensorMap tx, txs, tw, ts, tb;
     if (!make_map_2d(&tx, act_type(kF16), g.x, (uint64_t)g.K, (uint64_t)g.x_rows, (uint64_t)g.K * 2,
                      kBK, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
@@ -758,6 +816,14 @@ cudaError_t run_gemm_grouped(const GroupedArgs &g, cudaStream_t s) {
         return cudaErrorInvalidValue;
     if (!make_weight_map<BITS>(&tw, g.wq, (uint64_t)g.n_experts * (uint64_t)g.N, g.K))
         return cudaErrorInvalidValue;
+    const uint64_t wrows = (uint64_t)g.n_experts * (uint64_t)g.N;
+    if (sb_tma) {
+        if (!make_sb_map(&ts, g.scales, wrows, gpr) || !make_sb_map(&tb, g.biases, wrows, gpr))
+            return cudaErrorInvalidValue;
+    } else {
+        ts = tx;  // unused
+        tb = tx;
+    }
 
     GemmParams p{};
     p.scales = g.scales;
@@ -775,12 +841,13 @@ cudaError_t run_gemm_grouped(const GroupedArgs &g, cudaStream_t s) {
     p.hdr = g.hdr;
     p.chunks = g.chunks;
     p.dst_rows = g.dst_rows;
+    p.sb_tma = sb_tma ? 1 : 0;
     auto kern = qgemm_tc_kernel<T, BITS, BN, true>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t max_tiles = g.max_chunks * (int64_t)p.n_tiles;
     const int grid = (int)std::min<int64_t>(max_tiles, num_sms());
-    kern<<<grid, kThreads, smem, s>>>(tx, txs, tw, p);
+    kern<<<grid, kThreads, smem, s>>>(tx, txs, tw, ts, tb, p);
     count_launches(1);
     return cudaGetLastError();
 }

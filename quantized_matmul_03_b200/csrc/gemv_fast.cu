@@ -343,6 +343,11 @@ cudaError_t launch_stream(const QmmArgs &a, cudaStream_t s) {
     if (!plan_stream(a, MR, 1, p)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
     if (e != cudaSuccess) return e;
+    // All of the SM's unified L1/shared storage as shared memory, so that a
+    // second CTA (of the next call) fits beside this one.
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     int got = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&got, kern, kThreads, p.smem);
     if (e != cudaSuccess) return e;
