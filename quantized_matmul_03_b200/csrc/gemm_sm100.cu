@@ -39,9 +39,11 @@ namespace {
 
 constexpr int kDqWarps = 8;
 constexpr int kEpiWarps = 4;
-constexpr int kWarpTma = kDqWarps + kEpiWarps;  // 12
+constexpr int kWarpTma = kDqWarps + kEpiWarps;  // 12: packed-tile loads
 constexpr int kWarpMma = kWarpTma + 1;          // 13
-constexpr int kThreads = 32 * (kWarpMma + 1);   // 448
+constexpr int kWarpTmaB = kWarpMma + 1;         // 14: activation loads
+constexpr int kWarpTmaS = kWarpMma + 2;         // 15: scale/bias window loads
+constexpr int kThreads = 32 * (kWarpTmaS + 1);  // 512
 constexpr int kBM = 128;                        // weight rows per tile (UMMA M)
 constexpr int kBK = 64;                         // k per stage: one 128-byte swizzle row
 
@@ -338,7 +340,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            ptx::mbar_init(full_pb + 8 * s, 1);
+            ptx::mbar_init(full_pb + 8 * s, p.sb_tma ? 3 : 2);  // one arrival per producer warp
             ptx::mbar_init(full_a + 8 * s, kDqWarps / 2);  // one dequant group per k-block
             ptx::mbar_init(empty + 8 * s, 1);
         }
@@ -558,9 +560,15 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(acc_empty + 8 * acc);
         }
-    } else if (warp == kWarpTma) {
-        // ------------------------- producer -------------------------
-        if (lane == 0) {
+    } else if (warp == kWarpTma || warp == kWarpTmaB || warp == kWarpTmaS) {
+        // ------------------------- producers -------------------------
+        // Issuing a TMA load takes one thread several hundred cycles, so the
+        // stage's loads come from three warps in parallel: the packed tile
+        // (warp 12), the activation boxes (warp 14), the scale and bias
+        // windows (warp 15).  Each arrives on full_pb with its own byte count;
+        // the barrier expects one arrival per producer.
+        const int role = warp == kWarpTma ? 0 : (warp == kWarpTmaB ? 1 : 2);
+        if (lane == 0 && (role < 2 || (KMAJOR && p.sb_tma))) {
             int c = 0;
             const CUtensorMap *xmap = &tmap_x;
             if constexpr (GROUPED) {
@@ -574,28 +582,32 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 for (int kb = 0; kb < KB; ++kb, ++c) {
                     const int s = c % S;
                     if (c >= S) ptx::mbar_wait(empty + 8 * s, ((c / S) + 1) & 1, p.err);
-                    ptx::mbar_arrive_expect_tx(full_pb + 8 * s,
-                                               P_BYTES + bbytes + (p.sb_tma ? SB_BYTES : 0));
-                    if (KMAJOR && p.sb_tma) {
+                    const uint32_t fb = full_pb + 8 * s;
+                    if (role == 0) {
+                        ptx::mbar_arrive_expect_tx(fb, P_BYTES);
+                        if constexpr (KMAJOR)
+                            tma_load_2d(p0 + s * P_BYTES, &tmap_w, kb * W_WORDS, t.wrow0, fb);
+                        else  // 64 k-rows x 128 features of the [K, N] packed weight
+                            tma_load_2d(p0 + s * P_BYTES, &tmap_w, t.n0 * BITS / 32, kb * kBK, fb);
+                    } else if (role == 1) {
+                        ptx::mbar_arrive_expect_tx(fb, bbytes);
+                        for (int j = 0; j < nbox; ++j)
+                            tma_load_2d(b0 + s * B_BYTES + j * 64 * kBK * 2, xmap, kb * kBK, t.m0 + 64 * j, fb);
+                    } else {
                         // the window of 8 groups holding this k-block's groups
+                        ptx::mbar_arrive_expect_tx(fb, SB_BYTES);
                         const int wx = ((kb * kBK) / p.group_size) & ~7;
-                        tma_load_2d(sb0 + s * SB_BYTES, &tmap_s, wx, t.wrow0, full_pb + 8 * s);
-                        tma_load_2d(sb0 + s * SB_BYTES + SB_BYTES / 2, &tmap_b, wx, t.wrow0, full_pb + 8 * s);
+                        tma_load_2d(sb0 + s * SB_BYTES, &tmap_s, wx, t.wrow0, fb);
+                        tma_load_2d(sb0 + s * SB_BYTES + SB_BYTES / 2, &tmap_b, wx, t.wrow0, fb);
                     }
-                    if constexpr (KMAJOR)
-                        tma_load_2d(p0 + s * P_BYTES, &tmap_w, kb * W_WORDS, t.wrow0, full_pb + 8 * s);
-                    else  // 64 k-rows x 128 features of the [K, N] packed weight
-                        tma_load_2d(p0 + s * P_BYTES, &tmap_w, t.n0 * BITS / 32, kb * kBK, full_pb + 8 * s);
-                    for (int j = 0; j < nbox; ++j)
-                        tma_load_2d(b0 + s * B_BYTES + j * 64 * kBK * 2, xmap, kb * kBK, t.m0 + 64 * j,
-                                    full_pb + 8 * s);
                 }
             }
             // Drain: wait (bounded) for the last copies to land before exit.
-            for (int d = max(0, c - S); d < c; ++d)
-                ptx::mbar_wait(full_pb + 8 * (d % S), (d / S) & 1, p.err);
+            if (role == 1)
+                for (int d = max(0, c - S); d < c; ++d)
+                    ptx::mbar_wait(full_pb + 8 * (d % S), (d / S) & 1, p.err);
         }
-    } else {
+    } else if (warp == kWarpMma) {
         // ------------------------- MMA issuer -------------------------
         // The warp walks the loop converged; one elected lane waits and
         // issues, one wait and one commit per k-block: a complete full_a
