@@ -239,6 +239,21 @@ __device__ __forceinline__ void dequant_half<__nv_bfloat16, 8>(const uint32_t *w
         out[c] = make_uint4(vals[4 * c], vals[4 * c + 1], vals[4 * c + 2], vals[4 * c + 3]);
 }
 
+// Position of k-block c in a ring of n stages -- slot c mod n, phase parity
+// (c div n) mod 2, and whether c >= n -- advanced one k-block at a time
+// without integer division.
+struct RingPos {
+    int slot = 0, phase = 0;
+    bool wrapped = false;
+    __device__ __forceinline__ void next(int n) {
+        if (++slot == n) {
+            slot = 0;
+            phase ^= 1;
+            wrapped = true;
+        }
+    }
+};
+
 // v.x / v.y / v.z / v.w by a runtime index without indexing registers.
 __device__ __forceinline__ uint32_t pick_word(const uint4 &v, int i) {
     const uint32_t lo = (i & 1) ? v.y : v.x, hi = (i & 1) ? v.w : v.z;
@@ -371,22 +386,24 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         const int kl = (t & 7) + 8 * (t >> 4), h = (t >> 3) & 1;
         const uint16_t *sc = static_cast<const uint16_t *>(p.scales);
         const uint16_t *bi = static_cast<const uint16_t *>(p.biases);
-        const int gpn = p.N / p.group_size;  // groups per stored row
+        const int gs_log = __ffs(p.group_size) - 1;  // group_size is a power of two
+        const int gpn = p.N >> gs_log;                 // groups per stored row
         int c = 0;
+        RingPos rp;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
             const Tile tl = decode_tile<BN, GROUPED>(p, tile);
             const int f0 = tl.n0 + 64 * h;  // first feature of this thread's half
             const bool v0 = f0 < p.N, v1 = f0 + 32 < p.N;
-            const int g0 = f0 / p.group_size, g1 = (f0 + 32) / p.group_size;
-            for (int kb = 0; kb < KB; ++kb, ++c) {
+            const int g0 = f0 >> gs_log, g1 = (f0 + 32) >> gs_log;
+            for (int kb = 0; kb < KB; ++kb, ++c, rp.next(S)) {
                 if ((c & 1) != grp) continue;
-                const int s = c % S;
+                const int s = rp.slot;
                 const int64_t srow = (int64_t)(kb * kBK + kl) * gpn;
                 const uint16_t s0 = v0 ? __ldg(sc + srow + g0) : (uint16_t)0;
                 const uint16_t b0v = v0 ? __ldg(bi + srow + g0) : (uint16_t)0;
                 const uint16_t s1 = v1 ? __ldg(sc + srow + g1) : (uint16_t)0;
                 const uint16_t b1v = v1 ? __ldg(bi + srow + g1) : (uint16_t)0;
-                ptx::mbar_wait(full_pb + 8 * s, (c / S) & 1, p.err);
+                ptx::mbar_wait(full_pb + 8 * s, rp.phase, p.err);
                 // Packed row kl (16*BITS bytes, unswizzled), half h.
                 const uint8_t *prow = pg + s * P_BYTES + kl * (16 * BITS) + h * (8 * BITS);
                 uint32_t w[2 * BITS];
@@ -422,7 +439,9 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         // Scales/biases are read 8 groups (16 bytes) at a time, one window
         // ahead of use, when rows are whole 16-byte units; else one by one.
         const bool vec = (gpr % 8) == 0;
+        const int gs_log = __ffs(p.group_size) - 1;  // group_size is a power of two
         int c = 0;
+        RingPos rp;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
             const Tile t = decode_tile<BN, GROUPED>(p, tile);
             const bool rv = t.n0 + r < p.N;
@@ -458,16 +477,16 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     b16 = rv ? __ldg(brow + g) : (uint16_t)0;
                 }
             };
-            for (int kb = 0; kb < KB; ++kb, ++c) {
+            for (int kb = 0; kb < KB; ++kb, ++c, rp.next(S)) {
                 if ((c & 1) != grp) continue;
-                const int s = c % S;
+                const int s = rp.slot;
                 uint16_t s0, b0v, s1, b1v;
-                const int g0 = (kb * kBK) / p.group_size, g1 = (kb * kBK + 32) / p.group_size;
+                const int g0 = (kb * kBK) >> gs_log, g1 = (kb * kBK + 32) >> gs_log;
                 if (!p.sb_tma) {
                     scale_bias(g0, s0, b0v);
                     scale_bias(g1, s1, b1v);
                 }
-                ptx::mbar_wait(full_pb + 8 * s, (c / S) & 1, p.err);
+                ptx::mbar_wait(full_pb + 8 * s, rp.phase, p.err);
                 if (p.sb_tma) {
                     // Row r's window of 8 groups starts at group (g0 & ~7).
                     const uint8_t *sw = gbase + (sb0 - base) + s * SB_BYTES + r * 16;
@@ -569,7 +588,9 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         // the barrier expects one arrival per producer.
         const int role = warp == kWarpTma ? 0 : (warp == kWarpTmaB ? 1 : 2);
         if (lane == 0 && (role < 2 || (KMAJOR && p.sb_tma))) {
+            const int gs_log = __ffs(p.group_size) - 1;
             int c = 0;
+            RingPos rp;
             const CUtensorMap *xmap = &tmap_x;
             if constexpr (GROUPED) {
                 if (__ldg(&p.hdr->use_x) == 0) xmap = &tmap_xs;
@@ -579,9 +600,9 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 // Grouped tiles load only the 64-row boxes that hold their rows.
                 const int nbox = GROUPED ? (t.rows + 63) / 64 : 1;
                 const uint32_t bbytes = GROUPED ? (uint32_t)nbox * 64u * kBK * 2u : (uint32_t)B_BYTES;
-                for (int kb = 0; kb < KB; ++kb, ++c) {
-                    const int s = c % S;
-                    if (c >= S) ptx::mbar_wait(empty + 8 * s, ((c / S) + 1) & 1, p.err);
+                for (int kb = 0; kb < KB; ++kb, ++c, rp.next(S)) {
+                    const int s = rp.slot;
+                    if (rp.wrapped) ptx::mbar_wait(empty + 8 * s, rp.phase ^ 1, p.err);
                     const uint32_t fb = full_pb + 8 * s;
                     if (role == 0) {
                         ptx::mbar_arrive_expect_tx(fb, P_BYTES);
@@ -596,7 +617,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     } else {
                         // the window of 8 groups holding this k-block's groups
                         ptx::mbar_arrive_expect_tx(fb, SB_BYTES);
-                        const int wx = ((kb * kBK) / p.group_size) & ~7;
+                        const int wx = ((kb * kBK) >> gs_log) & ~7;
                         tma_load_2d(sb0 + s * SB_BYTES, &tmap_s, wx, t.wrow0, fb);
                         tma_load_2d(sb0 + s * SB_BYTES + SB_BYTES / 2, &tmap_b, wx, t.wrow0, fb);
                     }
@@ -615,6 +636,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         // the stage before writing its A tile.
         const bool leader = elect_one();
         int c = 0, i = 0;
+        RingPos rp;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
             const int acc = i & 1;
             uint32_t idesc = IDESC;
@@ -626,10 +648,10 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
             __syncwarp();
             tc_fence_after();
             const uint32_t d = tmem_base + acc * BN;
-            for (int kb = 0; kb < KB; ++kb, ++c) {
-                const int s = c % S;
+            for (int kb = 0; kb < KB; ++kb, ++c, rp.next(S)) {
+                const int s = rp.slot;
                 if (leader) {
-                    ptx::mbar_wait<false>(full_a + 8 * s, (c / S) & 1, p.err);
+                    ptx::mbar_wait<false>(full_a + 8 * s, rp.phase, p.err);
                     tc_fence_after();
                     const uint64_t db = sw128_desc(b0 + s * B_BYTES);
                     // UMMA K = 16: 32 bytes along a K-major 128-byte row, or two
