@@ -150,9 +150,9 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
             const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(wq) + (int64_t)r0 * row_bytes;
             const uint8_t *ssrc = reinterpret_cast<const uint8_t *>(scales) + (int64_t)r0 * sb_bytes;
             const uint8_t *bsrc = reinterpret_cast<const uint8_t *>(biases) + (int64_t)r0 * sb_bytes;
-            for (int i = 0; i < nst; ++i) {
-                const int s = i % S;
-                if (i >= S) ptx::mbar_wait(empty0 + 8 * s, ((i / S) + 1) & 1, err);
+            // Ring slot and phase advance without integer division.
+            for (int i = 0, s = 0, ph = 0; i < nst; ++i) {
+                if (i >= S) ptx::mbar_wait(empty0 + 8 * s, ph ^ 1, err);
                 const int nr = min(SR, nrows - i * SR);
                 const uint32_t wb = (uint32_t)(nr * row_bytes), sb = (uint32_t)(nr * sb_bytes);
                 const uint32_t st = ptx::smem_addr(smem + (size_t)s * stage_bytes);
@@ -162,6 +162,10 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                 ptx::bulk_g2s(st, wsrc + roff * row_bytes, wb, bar);
                 ptx::bulk_g2s(st + SR * row_bytes, ssrc + roff * sb_bytes, sb, bar);
                 ptx::bulk_g2s(st + SR * row_bytes + SR * sb_bytes, bsrc + roff * sb_bytes, sb, bar);
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1;
+                }
             }
         }
     } else {
@@ -230,9 +234,8 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
             }
         }
 
-        for (int i = 0; i < nst; ++i) {
-            const int s = i % S;
-            ptx::mbar_wait(full0 + 8 * s, (i / S) & 1, err);
+        for (int i = 0, s = 0, ph = 0; i < nst; ++i) {
+            ptx::mbar_wait(full0 + 8 * s, ph, err);
             const uint8_t *st = smem + (size_t)s * stage_bytes;
             float part[V];
 #pragma unroll
@@ -275,6 +278,10 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                 const int m = lane / RPT, j = lane - m * RPT;
                 const int r = i * SR + team + j * NT;
                 if (m < M && r < nrows) atomicAdd(&ysm[m * rpc + r], v);
+            }
+            if (++s == S) {
+                s = 0;
+                ph ^= 1;
             }
         }
     }
