@@ -1,27 +1,40 @@
 // gemm_sm100.cu -- tensor-core quantized matmul for many activation rows
-// (prefill), transpose layout:  y[m, n] = sum_k x[m, k] * (s[n,g] q[n,k] + b[n,g])
-// with W stored [N, K] (mlx-rs ops/quantization.rs, quantized_matmul;
-// Emily.Quantization.Layers, quantized_dense with transpose: true).  The dense
-// weight never exists in global memory: each 128 x 64 tile is dequantized into
-// shared memory right before the tensor cores consume it.
+// (prefill):  y[m, n] = sum_k x[m, k] * (s[n,g] q[n,k] + b[n,g])  with W stored
+// [N, K] (mlx-rs ops/quantization.rs, quantized_matmul; Emily
+// Quantization.Layers, quantized_dense with transpose: true), and x @ W with W
+// stored [K, N].  The dense weight never exists in global memory: each 128 x 64
+// tile is dequantized on chip right before the tensor cores consume it.
 //
 // Orientation ("swap AB"): the UMMA M dimension (128) runs over weight rows n
 // and the UMMA N dimension (BN = 16..256) over activation rows m, so the
 // dequantized tile is the A operand and the activations are the B operand:
 //     D[n, m] (TMEM, fp32) += W~[n, k] * x[m, k]   for k-blocks of 64.
-// Both operands are K-major bf16/f16 in the canonical 128-byte-swizzle layout
-// (8-row x 128-byte atoms, row r's 16-byte chunk c at chunk c ^ (r mod 8)).
+// The activations are K-major bf16/f16 in the canonical 128-byte-swizzle
+// layout (8-row x 128-byte atoms, row r's 16-byte chunk c at chunk c ^ (r mod 8)).
+//
+// Where the dequantized tile lives:
+//   [N, K] layout  tensor memory (tcgen05.st by the dequantize threads, MMA in
+//                  its TMEM-A form).  Shared memory then carries only the
+//                  activation, packed-code and scale/bias tiles, which keeps
+//                  the per-SM shared-memory traffic (TMA writes + tensor-core
+//                  reads + the dequantize threads' reads) below its ceiling
+//                  and frees room for ring stages and an output staging slab;
+//   [K, N] layout  and the grouped (gather) product: a swizzled shared-memory
+//                  tile (MN-major for [K, N], K-major for grouped).
 //
 // Roles (one CTA per SM, persistent over output tiles):
 //   warps 0-7   dequantize, as two groups of four warps taking alternate
 //               k-blocks; thread r of a group owns weight row r, reads the
-//               packed codes the producer staged, forms s*q + b two codes at a
-//               time (bf16x2/f16x2 FMA, one rounding), and writes the
-//               swizzled A tile;
+//               packed codes and scale/bias windows the producers staged,
+//               forms s*q + b two codes at a time (bf16x2/f16x2 FMA, one
+//               rounding) and writes its row of the A tile;
 //   warps 8-11  epilogue: tcgen05.ld of the accumulator quadrant the warp may
-//               address (lanes 32*(warp%4)..), convert, store y;
-//   warp 12     producer: TMA loads of the packed weight tile and the
-//               activation tile for each k-block into a ring of stages;
+//               address (lanes 32*(warp%4)..), convert, then either stage the
+//               values in shared memory for one tensor store per slab or
+//               store y directly (grouped rows, unaligned y);
+//   warps 12,14,15  producers: TMA loads of the packed weight tile, the
+//               activation tile and the scale/bias windows of each k-block
+//               into a ring of stages;
 //   warp 13     MMA issuer (one thread) and TMEM owner.
 // Every wait is a bounded mbarrier wait (device error word on timeout); no
 // cluster multicast is used.
@@ -84,6 +97,34 @@ __device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t desc_a, uint64_
         "l"(desc_a), "l"(desc_b), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D[tmem] (+)= A[tmem_a] * B[desc_b]^T with operand A in tensor memory (lane
+// i = row i, 16-bit K values two per 32-bit column).
+__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t desc_b,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(desc_b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Thread i of the warp writes v[0..31] to columns taddr.col .. +31 of TMEM
+// lane taddr.lane + i.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+        "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -127,6 +168,28 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
         "l"(map), "r"(x), "r"(y), "r"(bar)
         : "memory");
+}
+
+// Tensor store of a shared-memory box to global (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed store has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until every committed store has completed.
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void sts16(uint32_t a, uint16_t v) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(v) : "memory");
+}
+template <typename T>
+__device__ __forceinline__ uint16_t out_bits(float f) {
+    const T h = Dt<T>::from_f(f);
+    return *reinterpret_cast<const uint16_t *>(&h);
 }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
@@ -266,6 +329,7 @@ struct GemmParams {
     int M, N, K, group_size;
     int m_tiles, n_tiles, num_tiles, stages;
     int sb_tma;  // [N, K] layout: scale/bias windows arrive by TMA with each stage
+    int stg_rows;  // output rows staged per tensor store (0: direct stores)
     int *err;
     // Grouped (gather_qmm) mode only: the chunk table and row map the
     // preparation kernel wrote.  Tile t covers chunk t / n_tiles and weight
@@ -322,7 +386,8 @@ template <typename T, int BITS, int BN, bool GROUPED, bool KMAJOR = true>
 __global__ void __launch_bounds__(kThreads, 1)
 qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_xs,
                 const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s,
-                const __grid_constant__ CUtensorMap tmap_b, const GemmParams p) {
+                const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_y,
+                const GemmParams p) {
     static_assert(KMAJOR || !GROUPED, "the grouped product is built for the [N, K] layout");
     constexpr bool kF16 = std::is_same<T, __half>::value;
     constexpr int A_BYTES = kBM * kBK * 2;         // 16 KB dequantized tile
@@ -330,23 +395,32 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     constexpr int P_ROW = kBK * BITS / 8;          // packed bytes per row per k-block
     constexpr int P_BYTES = kBM * P_ROW;
     constexpr int W_WORDS = kBK * BITS / 32;       // packed words per row per k-block
-    constexpr uint32_t TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;
+    // [N, K] layout: the dequantized tile goes to tensor memory (A operand of
+    // the MMA) instead of shared memory.  512 columns: accumulators (two
+    // buffers, or one of 256 columns) then a ring of 32-column A slots.
+    constexpr bool TS = KMAJOR && !GROUPED;
+    constexpr int NACC = (TS && 2 * BN > 256) ? 1 : 2;
+    constexpr uint32_t A_COL0 = NACC * BN < 32 ? 32 : NACC * BN;
+    constexpr uint32_t TMEM_COLS = TS ? 512 : (2 * BN < 32 ? 32 : 2 * BN);
     constexpr uint32_t IDESC = make_idesc(kF16, kBM, BN, !KMAJOR);
     // MN-major A tile: feature atoms (64 features) 1 KB apart, 8-k-row groups 2 KB apart.
     constexpr uint32_t MN_LBO = 1024, MN_SBO = 2048;
 
     extern __shared__ uint8_t smem_raw[];
     const int S = p.stages;
-    // 1024-byte aligned carve-up: A[S] | B[S] | P[S] | barriers | tmem slot
+    // 1024-byte aligned carve-up: A[S] (shared-memory A only) | B[S] | P[S] |
+    // scale/bias windows[S] | output slabs | barriers | tmem slot
     const uint32_t raw = ptx::smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
-    const uint32_t a0 = base, b0 = a0 + S * A_BYTES, p0 = b0 + S * B_BYTES;
+    const uint32_t a0 = base, b0 = a0 + (TS ? 0 : S * A_BYTES), p0 = b0 + S * B_BYTES;
     // Scale/bias windows ([N, K] layout with sb_tma): per stage 8 groups x 128
     // rows of scales (2 KB) then of biases (2 KB), row r at byte 16 r.
     constexpr int SB_BYTES = 2 * kBM * 16;
     const uint32_t sb0 = p0 + S * P_BYTES;
-    const uint32_t bar0 = sb0 + (p.sb_tma ? S * SB_BYTES : 0);
+    // Output staging: one slab of stg_rows x 32 values per epilogue warp.
+    const uint32_t out0 = sb0 + (p.sb_tma ? S * SB_BYTES : 0);
+    const uint32_t bar0 = out0 + (uint32_t)kEpiWarps * 64u * (uint32_t)p.stg_rows;
     const uint32_t full_pb = bar0, full_a = bar0 + 8 * S, empty = bar0 + 16 * S;
     const uint32_t acc_full = bar0 + 24 * S, acc_empty = acc_full + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + (acc_empty + 16 - base));
@@ -520,18 +594,40 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                         w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
                     }
                 }
-                uint8_t *arow = gbase + (a0 - base) + s * A_BYTES + r * 128;
+                if constexpr (TS) {
+                    uint32_t v[32];  // row r's 64 values of the k-block, two per column
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint4 out[4];
-                    dequant_half<T, BITS>(w + hh * BITS, hh ? s1 : s0, hh ? b1v : b0v, out);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint4 out[4];
+                        dequant_half<T, BITS>(w + hh * BITS, hh ? s1 : s0, hh ? b1v : b0v, out);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int chunk = 4 * hh + j;
-                        *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) = out[j];
+                        for (int j = 0; j < 4; ++j) {
+                            v[16 * hh + 4 * j] = out[j].x;
+                            v[16 * hh + 4 * j + 1] = out[j].y;
+                            v[16 * hh + 4 * j + 2] = out[j].z;
+                            v[16 * hh + 4 * j + 3] = out[j].w;
+                        }
                     }
+                    // A slot s was last read by the MMAs of k-block c - S, which
+                    // completed before stage s was refilled (full_pb above).
+                    tc_fence_after();
+                    tmem_st32(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + A_COL0 + 32u * s, v);
+                    tmem_st_wait();
+                    tc_fence_before();
+                } else {
+                    uint8_t *arow = gbase + (a0 - base) + s * A_BYTES + r * 128;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint4 out[4];
+                        dequant_half<T, BITS>(w + hh * BITS, hh ? s1 : s0, hh ? b1v : b0v, out);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int chunk = 4 * hh + j;
+                            *reinterpret_cast<uint4 *>(arow + ((chunk ^ (r & 7)) << 4)) = out[j];
+                        }
+                    }
+                    ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
                 }
-                ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(full_a + 8 * s);
             }
@@ -542,10 +638,47 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         T *y = static_cast<T *>(p.y);
         int i = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
-            const int acc = i & 1;
+            const int acc = NACC == 2 ? (i & 1) : 0, use = NACC == 2 ? (i >> 1) : i;
             const Tile t = decode_tile<BN, GROUPED>(p, tile);
-            ptx::mbar_wait(acc_full + 8 * acc, (i >> 1) & 1, p.err);
+            ptx::mbar_wait(acc_full + 8 * acc, use & 1, p.err);
             tc_fence_after();
+            if (!GROUPED && p.stg_rows > 0) {
+                // Staged: TMEM -> registers -> this warp's slab ([m][32 n],
+                // n contiguous) -> one tensor store per slab; rows past M and
+                // columns past N are clipped by the store.  The accumulator is
+                // handed back as soon as its last columns are in registers.
+                constexpr int CW = BN < 32 ? BN : 32;
+                const int nj = (t.rows + CW - 1) / CW, cpp = p.stg_rows / CW;
+                const uint32_t stg = out0 + (uint32_t)q * 64u * (uint32_t)p.stg_rows;
+                int j = 0;
+                for (int m_off = 0; m_off < t.rows; m_off += p.stg_rows) {
+                    if (lane == 0) bulk_wait_read0();  // the slab's last store has read it
+                    __syncwarp();
+#pragma unroll 1
+                    for (int jj = 0; jj < cpp && j < nj; ++jj, ++j) {
+                        uint32_t v[32];
+                        const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + acc * BN + CW * j;
+                        if constexpr (CW == 32) tmem_ld32(taddr, v);
+                        else tmem_ld16(taddr, v);
+                        tmem_ld_wait();
+                        if (j == nj - 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) ptx::mbar_arrive(acc_empty + 8 * acc);
+                        }
+                        const uint32_t row0 = stg + (uint32_t)(jj * CW) * 64u + 2u * lane;
+#pragma unroll
+                        for (int cc = 0; cc < CW; ++cc) sts16(row0 + 64u * cc, out_bits<T>(__uint_as_float(v[cc])));
+                    }
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmap_y, stg, t.n0 + 32 * q, t.m0 + m_off);
+                        bulk_commit();
+                    }
+                }
+                continue;
+            }
             const int n = t.n0 + 32 * q + lane;
             // Columns acc*BN .. acc*BN+BN-1 of this warp's 32 lanes, 32 (or, for
             // BN = 16, 16) columns per load so no load leaves the allocation;
@@ -579,6 +712,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(acc_empty + 8 * acc);
         }
+        if (lane == 0) bulk_wait0();
     } else if (warp == kWarpTma || warp == kWarpTmaB || warp == kWarpTmaS) {
         // ------------------------- producers -------------------------
         // Issuing a TMA load takes one thread several hundred cycles, so the
@@ -638,13 +772,13 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         int c = 0, i = 0;
         RingPos rp;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
-            const int acc = i & 1;
+            const int acc = NACC == 2 ? (i & 1) : 0, use = NACC == 2 ? (i >> 1) : i;
             uint32_t idesc = IDESC;
             {
                 const Tile t = decode_tile<BN, GROUPED>(p, tile);
                 if (GROUPED || t.rows < BN) idesc = make_idesc(kF16, kBM, (t.rows + 15) & ~15, !KMAJOR);
             }
-            if (leader && i >= 2) ptx::mbar_wait(acc_empty + 8 * acc, ((i >> 1) + 1) & 1, p.err);
+            if (leader && i >= NACC) ptx::mbar_wait(acc_empty + 8 * acc, (use + 1) & 1, p.err);
             __syncwarp();
             tc_fence_after();
             const uint32_t d = tmem_base + acc * BN;
@@ -654,15 +788,24 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     ptx::mbar_wait<false>(full_a + 8 * s, rp.phase, p.err);
                     tc_fence_after();
                     const uint64_t db = sw128_desc(b0 + s * B_BYTES);
-                    // UMMA K = 16: 32 bytes along a K-major 128-byte row, or two
-                    // 8-k-row groups (2 * SBO bytes) of the MN-major tile.
-                    const uint64_t da = KMAJOR ? sw128_desc(a0 + s * A_BYTES)
-                                               : sw128_mn_desc(a0 + s * A_BYTES, MN_LBO, MN_SBO);
-                    constexpr uint64_t DA = KMAJOR ? 2 : (2 * MN_SBO) >> 4;
-                    tc_mma(d, da, db, idesc, kb != 0);
-                    tc_mma(d, da + DA, db + 2, idesc, 1);
-                    tc_mma(d, da + 2 * DA, db + 4, idesc, 1);
-                    tc_mma(d, da + 3 * DA, db + 6, idesc, 1);
+                    if constexpr (TS) {
+                        // UMMA K = 16: 8 columns of the A slot, 32 bytes of B rows.
+                        const uint32_t ta = tmem_base + A_COL0 + 32u * s;
+                        tc_mma_ts(d, ta, db, idesc, kb != 0);
+                        tc_mma_ts(d, ta + 8, db + 2, idesc, 1);
+                        tc_mma_ts(d, ta + 16, db + 4, idesc, 1);
+                        tc_mma_ts(d, ta + 24, db + 6, idesc, 1);
+                    } else {
+                        // UMMA K = 16: 32 bytes along a K-major 128-byte row, or two
+                        // 8-k-row groups (2 * SBO bytes) of the MN-major tile.
+                        const uint64_t da = KMAJOR ? sw128_desc(a0 + s * A_BYTES)
+                                                   : sw128_mn_desc(a0 + s * A_BYTES, MN_LBO, MN_SBO);
+                        constexpr uint64_t DA = KMAJOR ? 2 : (2 * MN_SBO) >> 4;
+                        tc_mma(d, da, db, idesc, kb != 0);
+                        tc_mma(d, da + DA, db + 2, idesc, 1);
+                        tc_mma(d, da + 2 * DA, db + 4, idesc, 1);
+                        tc_mma(d, da + 3 * DA, db + 6, idesc, 1);
+                    }
                     tc_commit(empty + 8 * s);
                 }
                 __syncwarp();
@@ -726,11 +869,11 @@ int pick_bn(int64_t M) {
 // Shared-memory budget of one CTA: S stages of (A + B + P [+ scale/bias
 // windows]) plus barriers.
 template <int BITS, int BN>
-bool gemm_smem_plan(bool sb_tma, int &stages, size_t &smem) {
+bool gemm_smem_plan(bool sb_tma, int &stages, size_t &smem, bool a_smem, size_t extra = 0) {
     constexpr int A_BYTES = kBM * kBK * 2, B_BYTES = BN * kBK * 2, P_BYTES = kBM * kBK * BITS / 8;
-    const int STAGE = A_BYTES + B_BYTES + P_BYTES + (sb_tma ? 2 * kBM * 16 : 0);
+    const int STAGE = (a_smem ? A_BYTES : 0) + B_BYTES + P_BYTES + (sb_tma ? 2 * kBM * 16 : 0);
     constexpr size_t kSmemMax = 227 * 1024;
-    const size_t fixed = 1024 /*alignment*/ + 64 /*acc bars + slot*/;
+    const size_t fixed = 1024 /*alignment*/ + 64 /*acc bars + slot*/ + extra;
     stages = (int)std::min<size_t>(8, (kSmemMax - fixed) / (STAGE + 24));
     smem = fixed + (size_t)stages * (STAGE + 24);
     return stages >= 2;
@@ -743,8 +886,8 @@ template <int BITS, int BN>
 bool sb_windows_fit() {
     int s0, s1;
     size_t m0, m1;
-    gemm_smem_plan<BITS, BN>(false, s0, m0);
-    gemm_smem_plan<BITS, BN>(true, s1, m1);
+    gemm_smem_plan<BITS, BN>(false, s0, m0, true);
+    gemm_smem_plan<BITS, BN>(true, s1, m1, true);
     return s1 >= s0;
 }
 
@@ -783,12 +926,23 @@ bool make_weight_map_kn(CUtensorMap *map, const uint32_t *wq, int64_t K, int64_t
 template <typename T, int BITS, int BN, bool KMAJOR>
 cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
     const int64_t gpr = a.K / a.group_size;
-    const bool sb_tma = KMAJOR && gpr % 8 == 0 && sb_windows_fit<BITS, BN>();
-    int stages;
-    size_t smem;
-    if (!gemm_smem_plan<BITS, BN>(sb_tma, stages, smem)) return cudaErrorInvalidConfiguration;
+    // [N, K] layout: A lives in tensor memory, scale/bias windows come by
+    // TMA, and the output is staged for tensor stores when the ring keeps at
+    // least 4 stages (whole tile, else half of it per store).
+    const bool sb_tma = KMAJOR && gpr % 8 == 0;
+    int stages = 0, stg_rows = 0;
+    size_t smem = 0;
+    const bool y_ok = KMAJOR && (a.N * 2) % 16 == 0 && (reinterpret_cast<uintptr_t>(a.y) & 15) == 0;
+    if (y_ok) {
+        for (int rows = BN; rows >= 16 && stg_rows == 0; rows /= 2)
+            if (gemm_smem_plan<BITS, BN>(sb_tma, stages, smem, false, (size_t)kEpiWarps * 64 * rows) &&
+                stages >= 4)
+                stg_rows = rows;
+    }
+    if (stg_rows == 0 && !gemm_smem_plan<BITS, BN>(sb_tma, stages, smem, !KMAJOR))
+        return cudaErrorInvalidConfiguration;
     constexpr bool kF16 = std::is_same<T, __half>::value;
-    CUtensorMap tx, tw, ts, tb;
+    CUtensorMap tx, tw, ts, tb, ty;
     if (!make_map_2d(&tx, act_type(kF16), a.x, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * 2, kBK, BN,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
@@ -802,9 +956,17 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
         ts = tx;  // unused
         tb = tx;
     }
+    if (stg_rows > 0) {
+        if (!make_map_2d(&ty, act_type(kF16), a.y, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.N * 2, 32,
+                         (uint32_t)stg_rows, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    } else {
+        ty = tx;  // unused
+    }
 
     GemmParams p{};
     p.sb_tma = sb_tma ? 1 : 0;
+    p.stg_rows = stg_rows;
     p.scales = a.scales;
     p.biases = a.biases;
     p.y = a.y;
@@ -821,7 +983,7 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = std::min(p.num_tiles, num_sms());
-    kern<<<grid, kThreads, smem, s>>>(tx, tx, tw, ts, tb, p);
+    kern<<<grid, kThreads, smem, s>>>(tx, tx, tw, ts, tb, ty, p);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -837,7 +999,7 @@ cudaError_t run_gemm_grouped(const GroupedArgs &g, cudaStream_t s) {
     const bool sb_tma = gpr % 8 == 0 && sb_windows_fit<BITS, BN>();
     int stages;
     size_t smem;
-    if (!gemm_smem_plan<BITS, BN>(sb_tma, stages, smem)) return cudaErrorInvalidConfiguration;
+    if (!gemm_smem_plan<BITS, BN>(sb_tma, stages, smem, true)) return cudaErrorInvalidConfiguration;
     constexpr bool kF16 = std::is_same<T, __half>::value;
     // Activation maps: 64-row boxes over x viewed as [x_batch * M, K] and over
     // the sorted copy [rows, K].
@@ -881,7 +1043,7 @@ cudaError_t run_gemm_grouped(const GroupedArgs &g, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const int64_t max_tiles = g.max_chunks * (int64_t)p.n_tiles;
     const int grid = (int)std::min<int64_t>(max_tiles, num_sms());
-    kern<<<grid, kThreads, smem, s>>>(tx, txs, tw, ts, tb, p);
+    kern<<<grid, kThreads, smem, s>>>(tx, txs, tw, ts, tb, tx, p);
     count_launches(1);
     return cudaGetLastError();
 }
