@@ -421,17 +421,25 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     // Output staging: one slab of stg_rows x 32 values per epilogue warp.
     const uint32_t out0 = sb0 + (p.sb_tma ? S * SB_BYTES : 0);
     const uint32_t bar0 = out0 + (uint32_t)kEpiWarps * 64u * (uint32_t)p.stg_rows;
-    const uint32_t full_pb = bar0, full_a = bar0 + 8 * S, empty = bar0 + 16 * S;
-    const uint32_t acc_full = bar0 + 24 * S, acc_empty = acc_full + 16;
+    // Per stage: full_p (packed tile + scale/bias windows landed), full_b
+    // (activation tile landed), full_a (A tile written), p_empty (the
+    // dequantize group has read the packed tile and windows: they can be
+    // refilled before the MMA runs), b_empty (the MMAs of the stage are done:
+    // activation tile and A slot free).
+    const uint32_t full_p = bar0, full_b = bar0 + 8 * S, full_a = bar0 + 16 * S;
+    const uint32_t p_empty = bar0 + 24 * S, b_empty = bar0 + 32 * S;
+    const uint32_t acc_full = bar0 + 40 * S, acc_empty = acc_full + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + (acc_empty + 16 - base));
     const uint8_t *pg = gbase + (p0 - base);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            ptx::mbar_init(full_pb + 8 * s, p.sb_tma ? 3 : 2);  // one arrival per producer warp
+            ptx::mbar_init(full_p + 8 * s, p.sb_tma ? 2 : 1);  // packed [+ windows] producer
+            ptx::mbar_init(full_b + 8 * s, 1);
             ptx::mbar_init(full_a + 8 * s, kDqWarps / 2);  // one dequant group per k-block
-            ptx::mbar_init(empty + 8 * s, 1);
+            ptx::mbar_init(p_empty + 8 * s, kDqWarps / 2);
+            ptx::mbar_init(b_empty + 8 * s, 1);
         }
         for (int a = 0; a < 2; ++a) {
             ptx::mbar_init(acc_full + 8 * a, 1);
@@ -477,7 +485,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 const uint16_t b0v = v0 ? __ldg(bi + srow + g0) : (uint16_t)0;
                 const uint16_t s1 = v1 ? __ldg(sc + srow + g1) : (uint16_t)0;
                 const uint16_t b1v = v1 ? __ldg(bi + srow + g1) : (uint16_t)0;
-                ptx::mbar_wait(full_pb + 8 * s, rp.phase, p.err);
+                ptx::mbar_wait(full_p + 8 * s, rp.phase, p.err);
                 // Packed row kl (16*BITS bytes, unswizzled), half h.
                 const uint8_t *prow = pg + s * P_BYTES + kl * (16 * BITS) + h * (8 * BITS);
                 uint32_t w[2 * BITS];
@@ -486,6 +494,8 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     const uint4 u = *reinterpret_cast<const uint4 *>(prow + 16 * q);
                     w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
                 }
+                // A stage s was last read by the MMAs of k-block c - S.
+                if (rp.wrapped) ptx::mbar_wait(b_empty + 8 * s, rp.phase ^ 1, p.err);
                 uint8_t *arow = gbase + (a0 - base) + s * A_BYTES + (kl >> 3) * MN_SBO + h * MN_LBO +
                                 (kl & 7) * 128;
 #pragma unroll
@@ -500,7 +510,10 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 }
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(full_a + 8 * s);
+                if (lane == 0) {
+                    ptx::mbar_arrive(p_empty + 8 * s);
+                    ptx::mbar_arrive(full_a + 8 * s);
+                }
             }
         }
     } else if (warp < kDqWarps) {
@@ -560,7 +573,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     scale_bias(g0, s0, b0v);
                     scale_bias(g1, s1, b1v);
                 }
-                ptx::mbar_wait(full_pb + 8 * s, rp.phase, p.err);
+                ptx::mbar_wait(full_p + 8 * s, rp.phase, p.err);
                 if (p.sb_tma) {
                     // Row r's window of 8 groups starts at group (g0 & ~7).
                     const uint8_t *sw = gbase + (sb0 - base) + s * SB_BYTES + r * 16;
@@ -608,13 +621,18 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                             v[16 * hh + 4 * j + 3] = out[j].w;
                         }
                     }
-                    // A slot s was last read by the MMAs of k-block c - S, which
-                    // completed before stage s was refilled (full_pb above).
+                    // The codes and windows have been consumed: stage s's packed
+                    // tile can be refilled.  A slot s was last read by the MMAs
+                    // of k-block c - S.
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(p_empty + 8 * s);
+                    if (rp.wrapped) ptx::mbar_wait(b_empty + 8 * s, rp.phase ^ 1, p.err);
                     tc_fence_after();
                     tmem_st32(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + A_COL0 + 32u * s, v);
                     tmem_st_wait();
                     tc_fence_before();
                 } else {
+                    if (rp.wrapped) ptx::mbar_wait(b_empty + 8 * s, rp.phase ^ 1, p.err);
                     uint8_t *arow = gbase + (a0 - base) + s * A_BYTES + r * 128;
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
@@ -627,6 +645,8 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                         }
                     }
                     ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(p_empty + 8 * s);
                 }
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(full_a + 8 * s);
@@ -718,8 +738,9 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         // Issuing a TMA load takes one thread several hundred cycles, so the
         // stage's loads come from three warps in parallel: the packed tile
         // (warp 12), the activation boxes (warp 14), the scale and bias
-        // windows (warp 15).  Each arrives on full_pb with its own byte count;
-        // the barrier expects one arrival per producer.
+        // windows (warp 15).  The packed tile and windows arrive on full_p
+        // (one arrival per producer, each with its own byte count), the
+        // activation tile on full_b.
         const int role = warp == kWarpTma ? 0 : (warp == kWarpTmaB ? 1 : 2);
         if (lane == 0 && (role < 2 || (KMAJOR && p.sb_tma))) {
             const int gs_log = __ffs(p.group_size) - 1;
@@ -736,8 +757,10 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 const uint32_t bbytes = GROUPED ? (uint32_t)nbox * 64u * kBK * 2u : (uint32_t)B_BYTES;
                 for (int kb = 0; kb < KB; ++kb, ++c, rp.next(S)) {
                     const int s = rp.slot;
-                    if (rp.wrapped) ptx::mbar_wait(empty + 8 * s, rp.phase ^ 1, p.err);
-                    const uint32_t fb = full_pb + 8 * s;
+                    // The packed tile and windows are free once the dequantize
+                    // group has read them; the activation tile once the MMAs ran.
+                    if (rp.wrapped) ptx::mbar_wait((role == 1 ? b_empty : p_empty) + 8 * s, rp.phase ^ 1, p.err);
+                    const uint32_t fb = (role == 1 ? full_b : full_p) + 8 * s;
                     if (role == 0) {
                         ptx::mbar_arrive_expect_tx(fb, P_BYTES);
                         if constexpr (KMAJOR)
@@ -758,16 +781,15 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 }
             }
             // Drain: wait (bounded) for the last copies to land before exit.
-            if (role == 1)
-                for (int d = max(0, c - S); d < c; ++d)
-                    ptx::mbar_wait(full_pb + 8 * (d % S), (d / S) & 1, p.err);
+            for (int d = max(0, c - S); d < c; ++d)
+                ptx::mbar_wait((role == 1 ? full_b : full_p) + 8 * (d % S), (d / S) & 1, p.err);
         }
     } else if (warp == kWarpMma) {
         // ------------------------- MMA issuer -------------------------
-        // The warp walks the loop converged; one elected lane waits and
-        // issues, one wait and one commit per k-block: a complete full_a
-        // implies a complete full_pb, since the dequantize warps waited for
-        // the stage before writing its A tile.
+        // The warp walks the loop converged; one elected lane waits for the
+        // stage's A tile and activation tile, issues the four MMAs and
+        // commits them to b_empty, which frees both the activation tile and
+        // the A slot.
         const bool leader = elect_one();
         int c = 0, i = 0;
         RingPos rp;
@@ -786,6 +808,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 const int s = rp.slot;
                 if (leader) {
                     ptx::mbar_wait<false>(full_a + 8 * s, rp.phase, p.err);
+                    ptx::mbar_wait<false>(full_b + 8 * s, rp.phase, p.err);
                     tc_fence_after();
                     const uint64_t db = sw128_desc(b0 + s * B_BYTES);
                     if constexpr (TS) {
@@ -806,7 +829,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                         tc_mma(d, da + 2 * DA, db + 4, idesc, 1);
                         tc_mma(d, da + 3 * DA, db + 6, idesc, 1);
                     }
-                    tc_commit(empty + 8 * s);
+                    tc_commit(b_empty + 8 * s);
                 }
                 __syncwarp();
             }
@@ -874,8 +897,8 @@ bool gemm_smem_plan(bool sb_tma, int &stages, size_t &smem, bool a_smem, size_t 
     const int STAGE = (a_smem ? A_BYTES : 0) + B_BYTES + P_BYTES + (sb_tma ? 2 * kBM * 16 : 0);
     constexpr size_t kSmemMax = 227 * 1024;
     const size_t fixed = 1024 /*alignment*/ + 64 /*acc bars + slot*/ + extra;
-    stages = (int)std::min<size_t>(8, (kSmemMax - fixed) / (STAGE + 24));
-    smem = fixed + (size_t)stages * (STAGE + 24);
+    stages = (int)std::min<size_t>(8, (kSmemMax - fixed) / (STAGE + 40));
+    smem = fixed + (size_t)stages * (STAGE + 40);
     return stages >= 2;
 }
 
