@@ -402,6 +402,10 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     constexpr int NACC = (TS && 2 * BN > 256) ? 1 : 2;
     constexpr uint32_t A_COL0 = NACC * BN < 32 ? 32 : NACC * BN;
     constexpr uint32_t TMEM_COLS = TS ? 512 : (2 * BN < 32 ? 32 : 2 * BN);
+    // Split stage barriers (below) for the wide TMEM-A tiles, where the TMA
+    // latency of the packed tile is on the critical chain; elsewhere one
+    // barrier per stage (measured faster for narrow tiles and [K, N]).
+    constexpr bool SPLIT = TS && BN >= 128;
     constexpr uint32_t IDESC = make_idesc(kF16, kBM, BN, !KMAJOR);
     // MN-major A tile: feature atoms (64 features) 1 KB apart, 8-k-row groups 2 KB apart.
     constexpr uint32_t MN_LBO = 1024, MN_SBO = 2048;
@@ -421,11 +425,12 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     // Output staging: one slab of stg_rows x 32 values per epilogue warp.
     const uint32_t out0 = sb0 + (p.sb_tma ? S * SB_BYTES : 0);
     const uint32_t bar0 = out0 + (uint32_t)kEpiWarps * 64u * (uint32_t)p.stg_rows;
-    // Per stage: full_p (packed tile + scale/bias windows landed), full_b
-    // (activation tile landed), full_a (A tile written), p_empty (the
-    // dequantize group has read the packed tile and windows: they can be
-    // refilled before the MMA runs), b_empty (the MMAs of the stage are done:
-    // activation tile and A slot free).
+    // Per stage: full_p (packed tile + scale/bias windows landed; without
+    // SPLIT also the activation tile), full_b (activation tile landed, SPLIT
+    // only), full_a (A tile written), p_empty (SPLIT only: the dequantize
+    // group has read the packed tile and windows, which can be refilled
+    // before the MMA runs), b_empty (the MMAs of the stage are done:
+    // activation tile and A slot free; without SPLIT the whole stage).
     const uint32_t full_p = bar0, full_b = bar0 + 8 * S, full_a = bar0 + 16 * S;
     const uint32_t p_empty = bar0 + 24 * S, b_empty = bar0 + 32 * S;
     const uint32_t acc_full = bar0 + 40 * S, acc_empty = acc_full + 16;
@@ -435,7 +440,8 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            ptx::mbar_init(full_p + 8 * s, p.sb_tma ? 2 : 1);  // packed [+ windows] producer
+            // one arrival per producer warp that signals the barrier
+            ptx::mbar_init(full_p + 8 * s, (p.sb_tma ? 2 : 1) + (SPLIT ? 0 : 1));
             ptx::mbar_init(full_b + 8 * s, 1);
             ptx::mbar_init(full_a + 8 * s, kDqWarps / 2);  // one dequant group per k-block
             ptx::mbar_init(p_empty + 8 * s, kDqWarps / 2);
@@ -494,8 +500,8 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     const uint4 u = *reinterpret_cast<const uint4 *>(prow + 16 * q);
                     w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
                 }
-                // A stage s was last read by the MMAs of k-block c - S.
-                if (rp.wrapped) ptx::mbar_wait(b_empty + 8 * s, rp.phase ^ 1, p.err);
+                // A stage s is free: its refill (full_p above) waited for the
+                // MMAs of k-block c - S.
                 uint8_t *arow = gbase + (a0 - base) + s * A_BYTES + (kl >> 3) * MN_SBO + h * MN_LBO +
                                 (kl & 7) * 128;
 #pragma unroll
@@ -510,10 +516,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 }
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) {
-                    ptx::mbar_arrive(p_empty + 8 * s);
-                    ptx::mbar_arrive(full_a + 8 * s);
-                }
+                if (lane == 0) ptx::mbar_arrive(full_a + 8 * s);
             }
         }
     } else if (warp < kDqWarps) {
@@ -621,18 +624,20 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                             v[16 * hh + 4 * j + 3] = out[j].w;
                         }
                     }
-                    // The codes and windows have been consumed: stage s's packed
-                    // tile can be refilled.  A slot s was last read by the MMAs
-                    // of k-block c - S.
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(p_empty + 8 * s);
-                    if (rp.wrapped) ptx::mbar_wait(b_empty + 8 * s, rp.phase ^ 1, p.err);
+                    // SPLIT: the codes and windows have been consumed, so stage
+                    // s's packed tile can be refilled; A slot s was last read by
+                    // the MMAs of k-block c - S.  Otherwise the refill of stage
+                    // s (full_p above) already waited for those MMAs.
+                    if constexpr (SPLIT) {
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(p_empty + 8 * s);
+                        if (rp.wrapped) ptx::mbar_wait(b_empty + 8 * s, rp.phase ^ 1, p.err);
+                    }
                     tc_fence_after();
                     tmem_st32(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + A_COL0 + 32u * s, v);
                     tmem_st_wait();
                     tc_fence_before();
                 } else {
-                    if (rp.wrapped) ptx::mbar_wait(b_empty + 8 * s, rp.phase ^ 1, p.err);
                     uint8_t *arow = gbase + (a0 - base) + s * A_BYTES + r * 128;
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
@@ -645,8 +650,6 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                         }
                     }
                     ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(p_empty + 8 * s);
                 }
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(full_a + 8 * s);
@@ -738,9 +741,8 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         // Issuing a TMA load takes one thread several hundred cycles, so the
         // stage's loads come from three warps in parallel: the packed tile
         // (warp 12), the activation boxes (warp 14), the scale and bias
-        // windows (warp 15).  The packed tile and windows arrive on full_p
-        // (one arrival per producer, each with its own byte count), the
-        // activation tile on full_b.
+        // windows (warp 15).  Each arrives with its own byte count on full_p
+        // (SPLIT: the activation tile on full_b).
         const int role = warp == kWarpTma ? 0 : (warp == kWarpTmaB ? 1 : 2);
         if (lane == 0 && (role < 2 || (KMAJOR && p.sb_tma))) {
             const int gs_log = __ffs(p.group_size) - 1;
@@ -757,10 +759,12 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 const uint32_t bbytes = GROUPED ? (uint32_t)nbox * 64u * kBK * 2u : (uint32_t)B_BYTES;
                 for (int kb = 0; kb < KB; ++kb, ++c, rp.next(S)) {
                     const int s = rp.slot;
-                    // The packed tile and windows are free once the dequantize
-                    // group has read them; the activation tile once the MMAs ran.
-                    if (rp.wrapped) ptx::mbar_wait((role == 1 ? b_empty : p_empty) + 8 * s, rp.phase ^ 1, p.err);
-                    const uint32_t fb = (role == 1 ? full_b : full_p) + 8 * s;
+                    // SPLIT: the packed tile and windows are free once the
+                    // dequantize group has read them, the activation tile once
+                    // the MMAs ran; otherwise the whole stage once the MMAs ran.
+                    const bool own = SPLIT && role != 1;
+                    if (rp.wrapped) ptx::mbar_wait((own ? p_empty : b_empty) + 8 * s, rp.phase ^ 1, p.err);
+                    const uint32_t fb = ((SPLIT && role == 1) ? full_b : full_p) + 8 * s;
                     if (role == 0) {
                         ptx::mbar_arrive_expect_tx(fb, P_BYTES);
                         if constexpr (KMAJOR)
@@ -782,14 +786,14 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
             }
             // Drain: wait (bounded) for the last copies to land before exit.
             for (int d = max(0, c - S); d < c; ++d)
-                ptx::mbar_wait((role == 1 ? full_b : full_p) + 8 * (d % S), (d / S) & 1, p.err);
+                ptx::mbar_wait(((SPLIT && role == 1) ? full_b : full_p) + 8 * (d % S), (d / S) & 1, p.err);
         }
     } else if (warp == kWarpMma) {
         // ------------------------- MMA issuer -------------------------
         // The warp walks the loop converged; one elected lane waits for the
-        // stage's A tile and activation tile, issues the four MMAs and
-        // commits them to b_empty, which frees both the activation tile and
-        // the A slot.
+        // stage's A tile (and, SPLIT, its activation tile: otherwise a complete
+        // full_a implies a complete full_p), issues the four MMAs and commits
+        // them to b_empty, which frees the activation tile and the A slot.
         const bool leader = elect_one();
         int c = 0, i = 0;
         RingPos rp;
@@ -808,7 +812,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 const int s = rp.slot;
                 if (leader) {
                     ptx::mbar_wait<false>(full_a + 8 * s, rp.phase, p.err);
-                    ptx::mbar_wait<false>(full_b + 8 * s, rp.phase, p.err);
+                    if constexpr (SPLIT) ptx::mbar_wait<false>(full_b + 8 * s, rp.phase, p.err);
                     tc_fence_after();
                     const uint64_t db = sw128_desc(b0 + s * B_BYTES);
                     if constexpr (TS) {
