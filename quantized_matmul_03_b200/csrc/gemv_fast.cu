@@ -40,6 +40,19 @@ namespace {
 constexpr int kCW = 12;                   // consumer warps
 constexpr int kThreads = 32 * (kCW + 1);  // plus one producer warp
 
+// Per-SM hand-off between consecutive CTAs of this kernel.  Under
+// programmatic dependent launch the next call's CTA sits beside the current
+// one on the SM from the current call's start; if it streams its first stages
+// at once, those copies compete with the current call's own stage copies,
+// which are on the critical path.  So a CTA takes a ticket per SM and issues
+// its first copy only once the CTA before it on the same SM has issued all of
+// its own (or after a short bound).  This orders memory traffic only: results
+// do not depend on it.
+constexpr int kMaxSm = 1024;
+constexpr uint64_t kHandoffWaitNs = 20000;
+__device__ unsigned long long g_sm_ticket[kMaxSm];  // CTAs that entered, per SM
+__device__ unsigned long long g_sm_issued[kMaxSm];  // highest ticket + 1 done issuing
+
 // Code planes of a packed word: plane p = (w >> p*BITS) & byte-mask, whose
 // byte j is code j*NP + p (NP = 8/BITS planes).  DP2A.lo takes bytes 0,1 and
 // DP2A.hi bytes 2,3, so the activation pairs of plane p are
@@ -150,6 +163,20 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
             const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(wq) + (int64_t)r0 * row_bytes;
             const uint8_t *ssrc = reinterpret_cast<const uint8_t *>(scales) + (int64_t)r0 * sb_bytes;
             const uint8_t *bsrc = reinterpret_cast<const uint8_t *>(biases) + (int64_t)r0 * sb_bytes;
+            uint32_t smid;
+            asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+            const bool handoff = smid < (uint32_t)kMaxSm;
+            unsigned long long ticket = 0;
+            if (handoff) {
+                ticket = atomicAdd(&g_sm_ticket[smid], 1ull);
+                const uint64_t t0 = ptx::globaltimer_ns();
+                for (;;) {
+                    unsigned long long done;
+                    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(done) : "l"(&g_sm_issued[smid]));
+                    if (done >= ticket || ptx::globaltimer_ns() - t0 > kHandoffWaitNs) break;
+                    __nanosleep(128);
+                }
+            }
             // Ring slot and phase advance without integer division.
             for (int i = 0, s = 0, ph = 0; i < nst; ++i) {
                 if (i >= S) ptx::mbar_wait(empty0 + 8 * s, ph ^ 1, err);
@@ -167,6 +194,7 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     ph ^= 1;
                 }
             }
+            if (handoff) atomicMax(&g_sm_issued[smid], ticket + 1);
         }
     } else {
         // ---------------- consumers ----------------
