@@ -42,7 +42,9 @@
 
 #include <algorithm>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "ptx_sm100.cuh"
 #include "qmm_internal.cuh"
@@ -330,6 +332,13 @@ struct GemmParams {
     int m_tiles, n_tiles, num_tiles, stages;
     int sb_tma;  // [N, K] layout: scale/bias windows arrive by TMA with each stage
     int stg_rows;  // output rows staged per tensor store (0: direct stores)
+    // Stream-K ([N, K] layout, staged epilogue): tiles below sk_tile0 go
+    // whole to CTAs (blockIdx.x, + gridDim.x, ...); for the rest CTA b works
+    // through k-blocks [b*sk_len, (b+1)*sk_len) of their (tile, k-block)
+    // space.  sk_len = 0: whole tiles only.
+    int sk_len, sk_tile0;
+    float *sk_ws;    // per CTA: one fp32 partial tile, [quadrant][chunk][lane][CW]
+    int *sk_flags;   // per CTA and quadrant: 1 while its partial awaits the tile's owner
     int *err;
     // Grouped (gather_qmm) mode only: the chunk table and row map the
     // preparation kernel wrote.  Tile t covers chunk t / n_tiles and weight
@@ -370,6 +379,48 @@ __device__ __forceinline__ int tile_count(const GemmParams &p) {
     if constexpr (GROUPED) return __ldg(&p.hdr->num_chunks) * p.n_tiles;
     else return p.num_tiles;
 }
+
+// One unit of a CTA's work: k-blocks [kb0, kb1) of output tile `tile`.
+struct Unit {
+    int tile, kb0, kb1;
+};
+
+// The units of one CTA, identical for every role.  Whole tiles blockIdx.x,
+// + gridDim.x, ... below the stream-K region; then the CTA's run of the
+// region's (tile, k-block) space walked from its end, so a tile split
+// between CTAs b and b+1 is finished last by b+1 (which combines the parts)
+// after b wrote its part first -- a waiting CTA only ever waits for
+// lower-numbered ones, which finished the same number of whole tiles.
+struct Work {
+    int next, stride, count, KB;  // whole tiles
+    int cur, begin;               // stream-K
+    __device__ Work(const GemmParams &p, int num_tiles, int KB_) {
+        KB = KB_;
+        next = blockIdx.x;
+        stride = gridDim.x;
+        const bool sk = p.sk_len > 0;
+        count = sk ? p.sk_tile0 : num_tiles;
+        begin = sk ? p.sk_tile0 * KB + (int)blockIdx.x * p.sk_len : 0;
+        cur = sk ? min(num_tiles * KB, begin + p.sk_len) : 0;
+    }
+    __device__ bool get(Unit &u) {
+        if (next < count) {
+            u.tile = next;
+            u.kb0 = 0;
+            u.kb1 = KB;
+            next += stride;
+            return true;
+        }
+        if (cur <= begin) return false;
+        const int tile = (cur - 1) / KB;  // once per unit, not per k-block
+        const int ts = tile * KB;
+        u.tile = tile;
+        u.kb0 = max(ts, begin) - ts;
+        u.kb1 = cur - ts;
+        cur = ts + u.kb0;
+        return true;
+    }
+};
 
 // GROUPED: gather_qmm's grouped product.  Activation tiles then arrive as
 // 64-row boxes (only as many as the chunk has rows), from tmap_xs (the sorted
@@ -478,12 +529,13 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         const int gpn = p.N >> gs_log;                 // groups per stored row
         int c = 0;
         RingPos rp;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            const Tile tl = decode_tile<BN, GROUPED>(p, tile);
+        Work wk(p, num_tiles, KB);
+        for (Unit u; wk.get(u);) {
+            const Tile tl = decode_tile<BN, GROUPED>(p, u.tile);
             const int f0 = tl.n0 + 64 * h;  // first feature of this thread's half
             const bool v0 = f0 < p.N, v1 = f0 + 32 < p.N;
             const int g0 = f0 >> gs_log, g1 = (f0 + 32) >> gs_log;
-            for (int kb = 0; kb < KB; ++kb, ++c, rp.next(S)) {
+            for (int kb = u.kb0; kb < u.kb1; ++kb, ++c, rp.next(S)) {
                 if ((c & 1) != grp) continue;
                 const int s = rp.slot;
                 const int64_t srow = (int64_t)(kb * kBK + kl) * gpn;
@@ -532,8 +584,9 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         const int gs_log = __ffs(p.group_size) - 1;  // group_size is a power of two
         int c = 0;
         RingPos rp;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            const Tile t = decode_tile<BN, GROUPED>(p, tile);
+        Work wk(p, num_tiles, KB);
+        for (Unit u; wk.get(u);) {
+            const Tile t = decode_tile<BN, GROUPED>(p, u.tile);
             const bool rv = t.n0 + r < p.N;
             const int64_t wrow = (int64_t)t.wrow0 + r;
             const uint16_t *srow = sc + wrow * gpr, *brow = bi + wrow * gpr;
@@ -567,7 +620,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     b16 = rv ? __ldg(brow + g) : (uint16_t)0;
                 }
             };
-            for (int kb = 0; kb < KB; ++kb, ++c, rp.next(S)) {
+            for (int kb = u.kb0; kb < u.kb1; ++kb, ++c, rp.next(S)) {
                 if ((c & 1) != grp) continue;
                 const int s = rp.slot;
                 uint16_t s0, b0v, s1, b1v;
@@ -660,9 +713,10 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
         T *y = static_cast<T *>(p.y);
         int i = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
+        Work wk(p, num_tiles, KB);
+        for (Unit u; wk.get(u); ++i) {
             const int acc = NACC == 2 ? (i & 1) : 0, use = NACC == 2 ? (i >> 1) : i;
-            const Tile t = decode_tile<BN, GROUPED>(p, tile);
+            const Tile t = decode_tile<BN, GROUPED>(p, u.tile);
             ptx::mbar_wait(acc_full + 8 * acc, use & 1, p.err);
             tc_fence_after();
             if (!GROUPED && p.stg_rows > 0) {
@@ -673,6 +727,59 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 constexpr int CW = BN < 32 ? BN : 32;
                 const int nj = (t.rows + CW - 1) / CW, cpp = p.stg_rows / CW;
                 const uint32_t stg = out0 + (uint32_t)q * 64u * (uint32_t)p.stg_rows;
+                // Stream-K: a unit that ends before the tile's last k-block
+                // leaves its fp32 part in this CTA's workspace slot; the unit
+                // holding the last k-block (the tile's owner) adds the parts of
+                // the lower-numbered CTAs that hold its first k-blocks, in CTA
+                // order after its own, so the sum is the same on every run.
+                const size_t slot = (size_t)kBM * BN;  // floats per CTA
+                const size_t qoff = (size_t)q * 32 * BN + (size_t)lane * CW;
+                if (p.sk_len > 0 && u.kb1 < KB) {
+                    float *dst = p.sk_ws + blockIdx.x * slot + qoff;
+#pragma unroll 1
+                    for (int jw = 0; jw < nj; ++jw) {
+                        uint32_t v[32];
+                        const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + acc * BN + CW * jw;
+                        if constexpr (CW == 32) tmem_ld32(taddr, v);
+                        else tmem_ld16(taddr, v);
+                        tmem_ld_wait();
+                        if (jw == nj - 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) ptx::mbar_arrive(acc_empty + 8 * acc);
+                        }
+                        uint4 *d4 = reinterpret_cast<uint4 *>(dst + (size_t)jw * 32 * CW);
+#pragma unroll
+                        for (int c4 = 0; c4 < CW / 4; ++c4)
+                            d4[c4] = make_uint4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
+                    }
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) atomicExch(p.sk_flags + 4 * blockIdx.x + q, 1);
+                    continue;
+                }
+                int src0 = 0, nsrc = 0;
+                if (p.sk_len > 0 && u.kb0 > 0) {
+                    src0 = (u.tile * KB - p.sk_tile0 * KB) / p.sk_len;
+                    nsrc = (int)blockIdx.x - src0;
+                    if (lane == 0) {
+                        for (int sI = 0; sI < nsrc; ++sI) {
+                            int *f = p.sk_flags + 4 * (src0 + sI) + q;
+                            const uint64_t t0 = ptx::globaltimer_ns();
+                            for (;;) {
+                                int fv;
+                                asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(fv) : "l"(f));
+                                if (fv != 0) break;
+                                if (ptx::globaltimer_ns() - t0 > ptx::kWaitNs) {
+                                    record_device_error(p.err, QMM_ERR_TIMEOUT);
+                                    break;
+                                }
+                                __nanosleep(64);
+                            }
+                        }
+                    }
+                    __syncwarp();
+                }
                 int j = 0;
                 for (int m_off = 0; m_off < t.rows; m_off += p.stg_rows) {
                     if (lane == 0) bulk_wait_read0();  // the slab's last store has read it
@@ -689,6 +796,19 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                             __syncwarp();
                             if (lane == 0) ptx::mbar_arrive(acc_empty + 8 * acc);
                         }
+#pragma unroll 1
+                        for (int sI = 0; sI < nsrc; ++sI) {
+                            const float4 *src = reinterpret_cast<const float4 *>(
+                                p.sk_ws + (size_t)(src0 + sI) * slot + qoff + (size_t)j * 32 * CW);
+#pragma unroll
+                            for (int c4 = 0; c4 < CW / 4; ++c4) {
+                                const float4 f = __ldcg(src + c4);
+                                v[4 * c4] = __float_as_uint(__uint_as_float(v[4 * c4]) + f.x);
+                                v[4 * c4 + 1] = __float_as_uint(__uint_as_float(v[4 * c4 + 1]) + f.y);
+                                v[4 * c4 + 2] = __float_as_uint(__uint_as_float(v[4 * c4 + 2]) + f.z);
+                                v[4 * c4 + 3] = __float_as_uint(__uint_as_float(v[4 * c4 + 3]) + f.w);
+                            }
+                        }
                         const uint32_t row0 = stg + (uint32_t)(jj * CW) * 64u + 2u * lane;
 #pragma unroll
                         for (int cc = 0; cc < CW; ++cc) sts16(row0 + 64u * cc, out_bits<T>(__uint_as_float(v[cc])));
@@ -700,6 +820,9 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                         bulk_commit();
                     }
                 }
+                // The parts are consumed: clear their flags for the next call.
+                if (lane == 0)
+                    for (int sI = 0; sI < nsrc; ++sI) atomicExch(p.sk_flags + 4 * (src0 + sI) + q, 0);
                 continue;
             }
             const int n = t.n0 + 32 * q + lane;
@@ -752,12 +875,13 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
             if constexpr (GROUPED) {
                 if (__ldg(&p.hdr->use_x) == 0) xmap = &tmap_xs;
             }
-            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-                const Tile t = decode_tile<BN, GROUPED>(p, tile);
+            Work wk(p, num_tiles, KB);
+            for (Unit u; wk.get(u);) {
+                const Tile t = decode_tile<BN, GROUPED>(p, u.tile);
                 // Grouped tiles load only the 64-row boxes that hold their rows.
                 const int nbox = GROUPED ? (t.rows + 63) / 64 : 1;
                 const uint32_t bbytes = GROUPED ? (uint32_t)nbox * 64u * kBK * 2u : (uint32_t)B_BYTES;
-                for (int kb = 0; kb < KB; ++kb, ++c, rp.next(S)) {
+                for (int kb = u.kb0; kb < u.kb1; ++kb, ++c, rp.next(S)) {
                     const int s = rp.slot;
                     // SPLIT: the packed tile and windows are free once the
                     // dequantize group has read them, the activation tile once
@@ -797,18 +921,19 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
         const bool leader = elect_one();
         int c = 0, i = 0;
         RingPos rp;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
+        Work wk(p, num_tiles, KB);
+        for (Unit u; wk.get(u); ++i) {
             const int acc = NACC == 2 ? (i & 1) : 0, use = NACC == 2 ? (i >> 1) : i;
             uint32_t idesc = IDESC;
             {
-                const Tile t = decode_tile<BN, GROUPED>(p, tile);
+                const Tile t = decode_tile<BN, GROUPED>(p, u.tile);
                 if (GROUPED || t.rows < BN) idesc = make_idesc(kF16, kBM, (t.rows + 15) & ~15, !KMAJOR);
             }
             if (leader && i >= NACC) ptx::mbar_wait(acc_empty + 8 * acc, (use + 1) & 1, p.err);
             __syncwarp();
             tc_fence_after();
             const uint32_t d = tmem_base + acc * BN;
-            for (int kb = 0; kb < KB; ++kb, ++c, rp.next(S)) {
+            for (int kb = u.kb0; kb < u.kb1; ++kb, ++c, rp.next(S)) {
                 const int s = rp.slot;
                 if (leader) {
                     ptx::mbar_wait<false>(full_a + 8 * s, rp.phase, p.err);
@@ -818,7 +943,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     if constexpr (TS) {
                         // UMMA K = 16: 8 columns of the A slot, 32 bytes of B rows.
                         const uint32_t ta = tmem_base + A_COL0 + 32u * s;
-                        tc_mma_ts(d, ta, db, idesc, kb != 0);
+                        tc_mma_ts(d, ta, db, idesc, kb != u.kb0);
                         tc_mma_ts(d, ta + 8, db + 2, idesc, 1);
                         tc_mma_ts(d, ta + 16, db + 4, idesc, 1);
                         tc_mma_ts(d, ta + 24, db + 6, idesc, 1);
@@ -828,7 +953,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                         const uint64_t da = KMAJOR ? sw128_desc(a0 + s * A_BYTES)
                                                    : sw128_mn_desc(a0 + s * A_BYTES, MN_LBO, MN_SBO);
                         constexpr uint64_t DA = KMAJOR ? 2 : (2 * MN_SBO) >> 4;
-                        tc_mma(d, da, db, idesc, kb != 0);
+                        tc_mma(d, da, db, idesc, kb != u.kb0);
                         tc_mma(d, da + DA, db + 2, idesc, 1);
                         tc_mma(d, da + 2 * DA, db + 4, idesc, 1);
                         tc_mma(d, da + 3 * DA, db + 6, idesc, 1);
@@ -950,6 +1075,52 @@ bool make_weight_map_kn(CUtensorMap *map, const uint32_t *wq, int64_t K, int64_t
                        kBM * BITS / 32, kBK, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// Stream-K scratch of one stream: a partial-tile slot per SM (128 x 256 fp32,
+// the widest tile) and four flags per slot.  Allocated on the first stream-K
+// call on (device, stream) that is not being captured into a graph, flags
+// zeroed, then kept for the process; calls on one stream are ordered, so they
+// never share a slot at the same time.
+struct SkScratch {
+    float *ws = nullptr;
+    int *flags = nullptr;
+};
+bool stream_k_scratch(cudaStream_t s, SkScratch &out) {
+    static std::mutex mu;
+    static std::map<std::pair<int, uintptr_t>, SkScratch> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const auto key = std::make_pair(dev, reinterpret_cast<uintptr_t>(s));
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+        out = it->second;
+        return true;
+    }
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    const size_t slots = (size_t)num_sms();
+    const size_t ws_bytes = slots * kBM * 256 * sizeof(float), flag_bytes = slots * 4 * sizeof(int);
+    void *mem = nullptr;
+    if (cudaMalloc(&mem, ws_bytes + flag_bytes) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    if (cudaMemset(static_cast<char *>(mem) + ws_bytes, 0, flag_bytes) != cudaSuccess) {
+        (void)cudaGetLastError();
+        cudaFree(mem);
+        return false;
+    }
+    SkScratch sc;
+    sc.ws = static_cast<float *>(mem);
+    sc.flags = reinterpret_cast<int *>(static_cast<char *>(mem) + ws_bytes);
+    cache[key] = sc;
+    out = sc;
+    return true;
+}
+
 template <typename T, int BITS, int BN, bool KMAJOR>
 cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
     const int64_t gpr = a.K / a.group_size;
@@ -1006,10 +1177,33 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
     p.num_tiles = p.m_tiles * p.n_tiles;
     p.stages = stages;
     p.err = device_error_word();
+    int grid = std::min(p.num_tiles, num_sms());
+    // Stream-K when there are fewer tiles than SMs and tiles are narrow
+    // (decode batches, small weights): every SM takes an equal run of at
+    // least 8 k-blocks if that shortens the busiest CTA's run by 10 % or more
+    // (M=16, 4096 x 4096: 24.6 -> 13.3 us; M=64: 24.8 -> 19.7 us).  The
+    // owner of a split tile reads the other parts' fp32 partials one round
+    // trip per 32 columns, which for tiles of 128 or more activation rows
+    // costs more than the split gains (M=128, 14336 x 4096: 28.1 -> 36.2 us),
+    // and with one or more full waves the last, partial wave runs on lightly
+    // loaded SMs (prefill M=2048 with its tail split: unchanged), so both keep
+    // whole tiles.
+    if (KMAJOR && BN <= 64 && stg_rows > 0 && p.num_tiles < num_sms()) {
+        const int64_t KB = a.K / kBK, sms = num_sms();
+        const int64_t total = (int64_t)p.num_tiles * KB;
+        const int64_t len = std::max<int64_t>(8, (total + sms - 1) / sms);
+        SkScratch sc;
+        if (total < (1LL << 30) && len * 10 <= KB * 9 && stream_k_scratch(s, sc)) {
+            p.sk_len = (int)len;
+            p.sk_tile0 = 0;
+            p.sk_ws = sc.ws;
+            p.sk_flags = sc.flags;
+            grid = (int)((total + len - 1) / len);
+        }
+    }
     auto kern = qgemm_tc_kernel<T, BITS, BN, false, KMAJOR>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int grid = std::min(p.num_tiles, num_sms());
     kern<<<grid, kThreads, smem, s>>>(tx, tx, tw, ts, tb, ty, p);
     count_launches(1);
     return cudaGetLastError();

@@ -166,3 +166,27 @@ def test_prefill_full_size_sampled(bits):
     ref = oracle.quantized_matmul(c.x[rows], wq, s, b, True, c.group_size, c.bits)
     err = row_rel_err(y.cpu()[rows], ref)
     assert err <= REL_TOL[torch.bfloat16], f"rel err {err}"
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("m,k,n", [(16, 4096, 1024), (40, 2048, 640), (64, 1536, 384), (9, 4096, 128)])
+def test_gemm_stream_k(bits, m, k, n):
+    """Fewer 128-row tiles than SMs with narrow activation tiles: the k-blocks
+    of each tile are split over several CTAs (up to eight parts per tile for
+    16 x 4096 x 1024) and the parts combined by the tile's owner."""
+    w = wl.with_outliers((n, k), seed=n + k + bits, dtype=torch.bfloat16)
+    x = wl.normal((m, k), seed=m + k, dtype=torch.bfloat16)
+    run_case(x, w, 64, bits, True, "gemm")
+
+
+def test_gemm_stream_k_deterministic():
+    """The owner adds the parts in a fixed order, so repeated calls agree bit
+    for bit."""
+    w = wl.with_outliers((1024, 4096), seed=5, dtype=torch.bfloat16).cuda()
+    x = wl.normal((16, 4096), seed=6, dtype=torch.bfloat16).cuda()
+    wq, s, b = qb.qmm_quantize(w, 64, 4)
+    qb.qmm_set_path("gemm")
+    y0 = qb.qmm_quantized_matmul(x, wq, s, b, True, 64, 4)
+    for _ in range(5):
+        y1 = qb.qmm_quantized_matmul(x, wq, s, b, True, 64, 4)
+        assert torch.equal(y0, y1)
