@@ -45,13 +45,14 @@ constexpr int kThreads = 32 * (kCW + 1);  // plus one producer warp
 // one on the SM from the current call's start; if it streams its first stages
 // at once, those copies compete with the current call's own stage copies,
 // which are on the critical path.  So a CTA takes a ticket per SM and issues
-// its first copy only once the CTA before it on the same SM has issued all of
-// its own (or after a short bound).  This orders memory traffic only: results
-// do not depend on it.
+// its first copy only once the CTA before it on the same SM has at most one
+// stage left to issue (or after a short bound; waiting for all of them, or
+// for two or three stages left, was measured slower).  This orders memory
+// traffic only: results do not depend on it.
 constexpr int kMaxSm = 1024;
 constexpr uint64_t kHandoffWaitNs = 20000;
 __device__ unsigned long long g_sm_ticket[kMaxSm];  // CTAs that entered, per SM
-__device__ unsigned long long g_sm_issued[kMaxSm];  // highest ticket + 1 done issuing
+__device__ unsigned long long g_sm_issued[kMaxSm];  // highest ticket + 1 with <= 1 stage to issue
 
 // Code planes of a packed word: plane p = (w >> p*BITS) & byte-mask, whose
 // byte j is code j*NP + p (NP = 8/BITS planes).  DP2A.lo takes bytes 0,1 and
@@ -189,6 +190,7 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                 ptx::bulk_g2s(st, wsrc + roff * row_bytes, wb, bar);
                 ptx::bulk_g2s(st + SR * row_bytes, ssrc + roff * sb_bytes, sb, bar);
                 ptx::bulk_g2s(st + SR * row_bytes + SR * sb_bytes, bsrc + roff * sb_bytes, sb, bar);
+                if (handoff && i == max(0, nst - 2)) atomicMax(&g_sm_issued[smid], ticket + 1);
                 if (++s == S) {
                     s = 0;
                     ph ^= 1;
