@@ -115,6 +115,12 @@ int *device_error_word() {
     return cached[dev];
 }
 
+int current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
 int num_sms() {
     static int cached[64] = {0};
     int dev = 0;

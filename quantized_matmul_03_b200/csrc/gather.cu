@@ -281,8 +281,10 @@ cudaError_t launch_gather_tc(qmm_dtype dt, const GatherCall &c, cudaStream_t s) 
     p.dst_rows = dst_rows;
     p.err = device_error_word();
     const size_t smem = (size_t)(p.W * E1 + 2 * (E1 + 1)) * sizeof(int);
-    cudaError_t e = cudaFuncSetAttribute(gather_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    struct Tag;
+    cudaError_t e = configure_once<Tag>(smem, [&]() {
+        return cudaFuncSetAttribute(gather_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
     if (e != cudaSuccess) return e;
     gather_prep_kernel<<<1, kPrepThreads, smem, s>>>(p);
     count_launches(1);

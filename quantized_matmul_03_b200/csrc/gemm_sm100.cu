@@ -1202,7 +1202,10 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
         }
     }
     auto kern = qgemm_tc_kernel<T, BITS, BN, false, KMAJOR>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    struct Tag;
+    cudaError_t e = configure_once<Tag>(smem, [&]() {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreads, smem, s>>>(tx, tx, tw, ts, tb, ty, p);
     count_launches(1);
@@ -1260,7 +1263,10 @@ cudaError_t run_gemm_grouped(const GroupedArgs &g, cudaStream_t s) {
     p.dst_rows = g.dst_rows;
     p.sb_tma = sb_tma ? 1 : 0;
     auto kern = qgemm_tc_kernel<T, BITS, BN, true>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    struct Tag;
+    cudaError_t e = configure_once<Tag>(smem, [&]() {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
     if (e != cudaSuccess) return e;
     const int64_t max_tiles = g.max_chunks * (int64_t)p.n_tiles;
     const int grid = (int)std::min<int64_t>(max_tiles, num_sms());

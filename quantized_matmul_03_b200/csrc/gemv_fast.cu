@@ -378,17 +378,21 @@ cudaError_t launch_stream(const QmmArgs &a, cudaStream_t s) {
     // One CTA per SM (the next call's CTAs take the other half of the SM).
     StreamPlan p{};
     if (!plan_stream(a, MR, 1, p)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+    struct Tag;
+    cudaError_t e = configure_once<Tag>(p.smem, [&]() {
+        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+        if (r != cudaSuccess) return r;
+        // All of the SM's unified L1/shared storage as shared memory, so that a
+        // second CTA (of the next call) fits beside this one.
+        r = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (r != cudaSuccess) return r;
+        int got = 0;
+        r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&got, kern, kThreads, p.smem);
+        if (r != cudaSuccess) return r;
+        return got < 1 ? cudaErrorInvalidConfiguration : cudaSuccess;
+    });
     if (e != cudaSuccess) return e;
-    // All of the SM's unified L1/shared storage as shared memory, so that a
-    // second CTA (of the next call) fits beside this one.
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    int got = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&got, kern, kThreads, p.smem);
-    if (e != cudaSuccess) return e;
-    if (got < 1) return cudaErrorInvalidConfiguration;
     // Programmatic stream serialization: this grid may start while the
     // preceding kernel of the stream finishes (see grid_dependency_wait()).
     cudaLaunchConfig_t cfg = {};

@@ -5,6 +5,9 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
 #include <stdint.h>
 
 #include "../../include/qmm.h"
@@ -35,6 +38,26 @@ __device__ __forceinline__ void record_device_error(int *word, int code) {
     atomicCAS(word, 0, code);
 }
 int *device_error_word();  // host: device address of the word (current device)
+
+// Host: the current device (-1 if the runtime cannot say).
+int current_device();
+
+// Host: apply a kernel's launch attributes once per device and per requested
+// dynamic shared-memory size, instead of on every call.  `apply` performs the
+// cudaFuncSetAttribute calls (and any check) for `smem` bytes; its result is
+// remembered only on success.
+template <typename Tag, typename Fn>
+cudaError_t configure_once(size_t smem, Fn &&apply) {
+    static std::mutex mu;
+    static size_t done[64] = {0};
+    const int dev = current_device();
+    if (dev < 0 || dev >= 64) return apply();
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[dev] >= smem && done[dev] != 0) return cudaSuccess;
+    const cudaError_t e = apply();
+    if (e == cudaSuccess) done[dev] = std::max(done[dev], smem);
+    return e;
+}
 
 // ---------------------------------------------------------------------------
 // Launchers (host).  Each returns cudaSuccess or the launch error.  Arguments
