@@ -18,7 +18,8 @@
  * Memory.  Every array argument is a DEVICE pointer owned by the caller,
  *   row-major and contiguous, and 16-byte aligned (misaligned pointers are
  *   rejected with QMM_ERR_INVALID_ARG).  The library allocates no device
- *   memory; gather_qmm takes a caller-provided workspace.
+ *   memory; gather_qmm and qmm_quantized_matmul_ws take caller-provided
+ *   workspaces.
  * Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *   default stream).  Calls only enqueue work and return; results are ready
  *   when the stream is synchronised.
@@ -101,6 +102,35 @@ qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K,
                                 qmm_dtype dtype, int64_t N, int transpose,
                                 int group_size, int bits, const char *mode,
                                 void *y, void *stream);
+
+/*
+ * qmm_quantized_matmul_ws -- qmm_quantized_matmul with a caller workspace.
+ * Nothing in the documents this library follows has a counterpart: the
+ * workspace only lets the tensor-core path split the k-blocks of each output
+ * tile over several CTAs ("stream-K") when a problem has fewer 128-row weight
+ * tiles than the GPU has SMs and at most 64 activation rows per tile (decode
+ * batches of 5..64 rows, small weights), so that every SM works.
+ *   workspace: NULL (whole tiles, exactly qmm_quantized_matmul), or device
+ *     memory of at least qmm_quantized_matmul_workspace_size(...) bytes,
+ *     256-byte aligned, ZEROED before its first use; every call that returns
+ *     QMM_OK leaves it zeroed again (after a QMM_ERR_TIMEOUT from
+ *     qmm_device_status, zero it again).  Calls in flight at once must not
+ *     share a workspace.  A workspace smaller than needed for a call's split
+ *     is not used (whole tiles).  Misaligned: QMM_ERR_WORKSPACE.
+ * Results: the parts of a split tile are added in a fixed order, so repeated
+ *   calls return identical bits; they can differ from the whole-tile result
+ *   in fp32 rounding.
+ * qmm_quantized_matmul_workspace_size returns the bytes a call of these sizes
+ * can use (0 when it would not split).
+ */
+size_t qmm_quantized_matmul_workspace_size(int64_t M, int64_t K, int64_t N, int transpose,
+                                           int bits, qmm_dtype dtype);
+qmm_status qmm_quantized_matmul_ws(const void *x, int64_t M, int64_t K,
+                                   const uint32_t *wq, const void *scales, const void *biases,
+                                   qmm_dtype dtype, int64_t N, int transpose,
+                                   int group_size, int bits, const char *mode,
+                                   void *y, void *workspace, size_t workspace_bytes,
+                                   void *stream);
 
 /*
  * qmm_gather_qmm -- EMLX.Quantization, section gather_quantized_matmul;

@@ -48,6 +48,8 @@ def lib() -> ctypes.CDLL:
             "qmm_dequantize": [vp, vp, vp, i32, i64, i64, i32, i32, cp, vp, vp],
             "qmm_quantized_matmul": [vp, i64, i64, vp, vp, vp, i32, i64, i32, i32, i32, cp,
                                      vp, vp],
+            "qmm_quantized_matmul_ws": [vp, i64, i64, vp, vp, vp, i32, i64, i32, i32, i32, cp,
+                                        vp, vp, sz, vp],
             "qmm_gather_qmm": [vp, i64, i64, i64, vp, vp, vp, i32, i64, i64, vp, vp, i64, i32,
                                i32, i32, cp, i32, vp, vp, sz, vp],
             "qmm_gather_qmm_static": [vp, i64, i64, i64, vp, vp, vp, i32, i64, i64, vp, vp, i64,
@@ -61,6 +63,8 @@ def lib() -> ctypes.CDLL:
             f.restype = ctypes.c_int
         L.qmm_gather_qmm_workspace_size.argtypes = [i64, i64, i64, i64, i32]
         L.qmm_gather_qmm_workspace_size.restype = sz
+        L.qmm_quantized_matmul_workspace_size.argtypes = [i64, i64, i64, i32, i32, i32]
+        L.qmm_quantized_matmul_workspace_size.restype = sz
         L.qmm_status_string.argtypes = [i32]
         L.qmm_status_string.restype = cp
         L.qmm_last_error.argtypes = []
@@ -131,9 +135,34 @@ def qmm_dequantize(wq, scales, biases, group_size: int = 64, bits: int = 4,
     return out
 
 
+# Zeroed stream-K workspaces, one per (device, stream), owned by this module
+# (torch memory) and reused across calls; the library leaves them zeroed.
+_mm_ws = {}
+
+
+def qmm_quantized_matmul_workspace_size(M: int, K: int, N: int, transpose: bool = True,
+                                        bits: int = 4, dtype=torch.bfloat16) -> int:
+    return int(lib().qmm_quantized_matmul_workspace_size(M, K, N, int(bool(transpose)), bits,
+                                                          DTYPES[dtype]))
+
+
+def _matmul_workspace(device: torch.device, nbytes: int) -> torch.Tensor:
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    ws = _mm_ws.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        _mm_ws[key] = ws
+    return ws
+
+
 def qmm_quantized_matmul(x, wq, scales, biases, transpose: bool = True, group_size: int = 64,
-                         bits: int = 4, mode: str = "affine", out: Optional[torch.Tensor] = None):
-    """``x @ W.T`` (transpose) or ``x @ W`` with W packed; x is [..., K]."""
+                         bits: int = 4, mode: str = "affine", out: Optional[torch.Tensor] = None,
+                         workspace="auto"):
+    """``x @ W.T`` (transpose) or ``x @ W`` with W packed; x is [..., K].
+
+    workspace: "auto" (a zeroed workspace kept per device and stream, when the
+    call can use one), None (whole tiles only) or a zeroed uint8 CUDA tensor
+    of at least qmm_quantized_matmul_workspace_size(...) bytes."""
     _cuda(x, wq, scales, biases, out)
     K = x.shape[-1]
     M = x.numel() // K if K else 0
@@ -143,9 +172,22 @@ def qmm_quantized_matmul(x, wq, scales, biases, transpose: bool = True, group_si
         N = wq.shape[-1] * 32 // bits
     if out is None:
         out = torch.empty(tuple(x.shape[:-1]) + (N,), dtype=scales.dtype, device=x.device)
-    _check(lib().qmm_quantized_matmul(_p(x), M, K, _p(wq), _p(scales), _p(biases),
-                                      _dtype(scales), N, int(bool(transpose)), group_size, bits,
-                                      _mode(mode), _p(out), _stream(x.device)))
+    ws = None
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError("workspace must be 'auto', None or a tensor")
+        if scales.dtype in DTYPES:
+            need = qmm_quantized_matmul_workspace_size(M, K, N, transpose, bits, scales.dtype)
+            if need > 0:
+                ws = _matmul_workspace(x.device, need)
+    elif workspace is not None:
+        _cuda(workspace)
+        ws = workspace
+    _check(lib().qmm_quantized_matmul_ws(_p(x), M, K, _p(wq), _p(scales), _p(biases),
+                                         _dtype(scales), N, int(bool(transpose)), group_size, bits,
+                                         _mode(mode), _p(out), _p(ws),
+                                         ws.numel() * ws.element_size() if ws is not None else 0,
+                                         _stream(x.device)))
     return out
 
 

@@ -186,17 +186,22 @@ qmm_status qmm_dequantize(const uint32_t *wq, const void *scales, const void *bi
     }
 }
 
-qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K, const uint32_t *wq,
-                                const void *scales, const void *biases, qmm_dtype dtype,
-                                int64_t N, int transpose, int group_size, int bits,
-                                const char *mode, void *y, void *stream) {
+qmm_status qmm_quantized_matmul_ws(const void *x, int64_t M, int64_t K, const uint32_t *wq,
+                                   const void *scales, const void *biases, qmm_dtype dtype,
+                                   int64_t N, int transpose, int group_size, int bits,
+                                   const char *mode, void *y, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
     try {
         qmm_status st = check_common(dtype, group_size, bits, mode);
         if (st != QMM_OK) return st;
         st = check_matmul(x, M, K, wq, scales, biases, N, transpose, group_size, y);
         if (st != QMM_OK) return st;
+        if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255) != 0)
+            return fail(QMM_ERR_WORKSPACE, "workspace must be 256-byte aligned");
         if (M == 0 || N == 0) return QMM_OK;
         QmmArgs a{x, wq, scales, biases, y, M, N, K, group_size, bits, transpose != 0};
+        a.ws = workspace;
+        a.ws_bytes = workspace ? workspace_bytes : 0;
         cudaStream_t s = (cudaStream_t)stream;
         const bool tc_ok = gemm_supported(dtype, a);
         if (g_path == QMM_PATH_GEMM) {
@@ -218,6 +223,25 @@ qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K, const uint3
         return finish_launch(launch_gemm(dtype, a, s), "tensor-core gemm launch");
     } catch (...) {
         return fail(QMM_ERR_CUDA, "unexpected exception in qmm_quantized_matmul");
+    }
+}
+
+qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K, const uint32_t *wq,
+                                const void *scales, const void *biases, qmm_dtype dtype,
+                                int64_t N, int transpose, int group_size, int bits,
+                                const char *mode, void *y, void *stream) {
+    return qmm_quantized_matmul_ws(x, M, K, wq, scales, biases, dtype, N, transpose, group_size,
+                                   bits, mode, y, nullptr, 0, stream);
+}
+
+size_t qmm_quantized_matmul_workspace_size(int64_t M, int64_t K, int64_t N, int transpose,
+                                           int bits, qmm_dtype dtype) {
+    try {
+        // Decode shapes go to the SIMT kernel under the automatic path.
+        if (g_path != QMM_PATH_GEMM && M <= kGemvMaxRows && transpose) return 0;
+        return gemm_workspace_size(dtype, M, K, N, transpose != 0, bits);
+    } catch (...) {
+        return 0;
     }
 }
 

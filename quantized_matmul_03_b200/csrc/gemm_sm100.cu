@@ -1075,51 +1075,13 @@ bool make_weight_map_kn(CUtensorMap *map, const uint32_t *wq, int64_t K, int64_t
                        kBM * BITS / 32, kBK, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-// Stream-K scratch of one stream: a partial-tile slot per SM (128 x 256 fp32,
-// the widest tile) and four flags per slot.  Allocated on the first stream-K
-// call on (device, stream) that is not being captured into a graph, flags
-// zeroed, then kept for the process; calls on one stream are ordered, so they
-// never share a slot at the same time.
-struct SkScratch {
-    float *ws = nullptr;
-    int *flags = nullptr;
-};
-bool stream_k_scratch(cudaStream_t s, SkScratch &out) {
-    static std::mutex mu;
-    static std::map<std::pair<int, uintptr_t>, SkScratch> cache;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return false;
-    const auto key = std::make_pair(dev, reinterpret_cast<uintptr_t>(s));
-    std::lock_guard<std::mutex> lock(mu);
-    auto it = cache.find(key);
-    if (it != cache.end()) {
-        out = it->second;
-        return true;
-    }
-    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
-        (void)cudaGetLastError();
-        return false;
-    }
-    const size_t slots = (size_t)num_sms();
-    const size_t ws_bytes = slots * kBM * 256 * sizeof(float), flag_bytes = slots * 4 * sizeof(int);
-    void *mem = nullptr;
-    if (cudaMalloc(&mem, ws_bytes + flag_bytes) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return false;
-    }
-    if (cudaMemset(static_cast<char *>(mem) + ws_bytes, 0, flag_bytes) != cudaSuccess) {
-        (void)cudaGetLastError();
-        cudaFree(mem);
-        return false;
-    }
-    SkScratch sc;
-    sc.ws = static_cast<float *>(mem);
-    sc.flags = reinterpret_cast<int *>(static_cast<char *>(mem) + ws_bytes);
-    cache[key] = sc;
-    out = sc;
-    return true;
-}
+// Stream-K workspace layout (caller-owned, zeroed before first use): the
+// flags first, 4 per SM (a fixed place, so that calls of any shape find them
+// zero), then one fp32 partial tile slot per SM of 128 x 64 values (stream-K
+// runs only tiles of at most 64 activation rows).
+constexpr size_t kSkFlagBytes = 4096;
+constexpr int kSkMaxBN = 64;
+size_t sk_workspace_bytes() { return kSkFlagBytes + (size_t)num_sms() * kBM * kSkMaxBN * sizeof(float); }
 
 template <typename T, int BITS, int BN, bool KMAJOR>
 cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
@@ -1188,16 +1150,16 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
     // and with one or more full waves the last, partial wave runs on lightly
     // loaded SMs (prefill M=2048 with its tail split: unchanged), so both keep
     // whole tiles.
-    if (KMAJOR && BN <= 64 && stg_rows > 0 && p.num_tiles < num_sms()) {
+    if (KMAJOR && BN <= kSkMaxBN && stg_rows > 0 && p.num_tiles < num_sms() && a.ws != nullptr &&
+        a.ws_bytes >= sk_workspace_bytes() && (size_t)num_sms() * 4 * sizeof(int) <= kSkFlagBytes) {
         const int64_t KB = a.K / kBK, sms = num_sms();
         const int64_t total = (int64_t)p.num_tiles * KB;
         const int64_t len = std::max<int64_t>(8, (total + sms - 1) / sms);
-        SkScratch sc;
-        if (total < (1LL << 30) && len * 10 <= KB * 9 && stream_k_scratch(s, sc)) {
+        if (total < (1LL << 30) && len * 10 <= KB * 9) {
             p.sk_len = (int)len;
             p.sk_tile0 = 0;
-            p.sk_ws = sc.ws;
-            p.sk_flags = sc.flags;
+            p.sk_flags = static_cast<int *>(a.ws);
+            p.sk_ws = reinterpret_cast<float *>(static_cast<char *>(a.ws) + kSkFlagBytes);
             grid = (int)((total + len - 1) / len);
         }
     }
@@ -1306,6 +1268,15 @@ bool gemm_supported(qmm_dtype dt, const QmmArgs &a) {
     if (((a.transpose ? a.K : a.N) * a.bits / 8) % 16 != 0) return false;
     if (a.M > INT32_MAX / 2 || a.N > INT32_MAX / 2 || a.K > INT32_MAX / 2) return false;
     return encode_fn() != nullptr;
+}
+
+size_t gemm_workspace_size(qmm_dtype dt, int64_t M, int64_t K, int64_t N, bool transpose, int bits) {
+    if ((dt != QMM_BF16 && dt != QMM_F16) || !transpose || M <= 0 || N <= 0 || K % kBK != 0) return 0;
+    if (pick_bn(M) > kSkMaxBN) return 0;
+    const int64_t tiles = ((M + pick_bn(M) - 1) / pick_bn(M)) * ((N + kBM - 1) / kBM);
+    if (tiles >= num_sms()) return 0;
+    (void)bits;
+    return sk_workspace_bytes();
 }
 
 cudaError_t launch_gemm(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {

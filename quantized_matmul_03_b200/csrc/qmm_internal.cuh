@@ -90,12 +90,17 @@ struct QmmArgs {
     int64_t M, N, K;
     int group_size, bits;
     bool transpose;
+    void *ws = nullptr;  // stream-K workspace (zeroed flags first), or null
+    size_t ws_bytes = 0;
 };
 cudaError_t launch_gemv(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 bool gemv_supported(qmm_dtype dt, const QmmArgs &a);
 cudaError_t launch_gemv_fast(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a);
 cudaError_t launch_gemm(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
+// Bytes of stream-K workspace the tensor-core path can use for these sizes
+// (0 when it would keep whole tiles).
+size_t gemm_workspace_size(qmm_dtype dt, int64_t M, int64_t K, int64_t N, bool transpose, int bits);
 bool gemm_supported(qmm_dtype dt, const QmmArgs &a);
 
 // ---------------------------------------------------------------------------

@@ -190,3 +190,22 @@ def test_gemm_stream_k_deterministic():
     for _ in range(5):
         y1 = qb.qmm_quantized_matmul(x, wq, s, b, True, 64, 4)
         assert torch.equal(y0, y1)
+
+
+def test_gemm_stream_k_workspace_options():
+    """Without a workspace (or with one too small) the call keeps whole tiles;
+    both agree with the oracle, and a used workspace is left zeroed."""
+    w = wl.with_outliers((1024, 4096), seed=7, dtype=torch.bfloat16)
+    x = wl.normal((16, 4096), seed=8, dtype=torch.bfloat16)
+    wq, s, b = oracle.quantize(w, 64, 4)
+    ref = oracle.quantized_matmul(x, wq, s, b, True, 64, 4)
+    need = qb.qmm_quantized_matmul_workspace_size(16, 4096, 1024, True, 4, torch.bfloat16)
+    assert need > 0
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    small = torch.zeros(need // 2, dtype=torch.uint8, device="cuda")
+    args = (x.cuda(), wq.cuda(), s.cuda(), b.cuda(), True, 64, 4)
+    for workspace in (None, small, ws):
+        y = qb.qmm_quantized_matmul(*args, workspace=workspace)
+        torch.cuda.synchronize()
+        assert row_rel_err(y, ref) <= REL_TOL[s.dtype]
+    assert int(ws[:4096].count_nonzero()) == 0  # the flags are cleared again
