@@ -270,13 +270,21 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
             float part[V];
 #pragma unroll
             for (int q = 0; q < V; ++q) part[q] = 0.f;
-            if (active) {
-                // All RPT rows are computed without branches so their DP2A
-                // chains interleave; rows past the block's end read stale (but
-                // in-bounds) stage bytes and are dropped by the selects.
+            // Rows of this stage: SR, except in the block's last stage.
+            const int rows_here = nrows - i * SR;
+            // A full stage computes all RPT rows without branches so their DP2A
+            // chains interleave (rows past the block's end read stale but
+            // in-bounds stage bytes and are dropped by the selects); the
+            // block's last, partial stage skips a team's rows past its end,
+            // which shortens the tail that every call waits for.
+            auto rows = [&](auto full) {
+                constexpr bool FULL = decltype(full)::value;
 #pragma unroll
                 for (int j = 0; j < RPT; ++j) {
                     const int jr = team + j * NT;           // row within the stage (< SR)
+                    if constexpr (!FULL) {
+                        if (jr >= rows_here) continue;
+                    }
                     const bool rv = i * SR + jr < nrows;
                     const uint8_t *wrow = st + jr * row_bytes;
                     const uint8_t *srow = st + SR * row_bytes + jr * sb_bytes;
@@ -300,6 +308,10 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                         }
                     }
                 }
+            };
+            if (active) {
+                if (rows_here >= SR) rows(std::true_type{});
+                else rows(std::false_type{});
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(empty0 + 8 * s);
