@@ -61,6 +61,7 @@ constexpr int kWarpTmaS = kWarpMma + 2;         // 15: scale/bias window loads
 constexpr int kThreads = 32 * (kWarpTmaS + 1);  // 512
 constexpr int kBM = 128;                        // weight rows per tile (UMMA M)
 constexpr int kBK = 64;                         // k per stage: one 128-byte swizzle row
+constexpr int kSkMaxBN = 64;                    // widest tile that stream-K splits
 
 // ---------------------------------------------------------------------------
 // tcgen05 / TMA wrappers
@@ -734,7 +735,8 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 // order after its own, so the sum is the same on every run.
                 const size_t slot = (size_t)kBM * BN;  // floats per CTA
                 const size_t qoff = (size_t)q * 32 * BN + (size_t)lane * CW;
-                if (p.sk_len > 0 && u.kb1 < KB) {
+                constexpr bool kSk = BN <= kSkMaxBN && !GROUPED;  // compiled only where used
+                if (kSk && p.sk_len > 0 && u.kb1 < KB) {
                     float *dst = p.sk_ws + blockIdx.x * slot + qoff;
 #pragma unroll 1
                     for (int jw = 0; jw < nj; ++jw) {
@@ -759,7 +761,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     continue;
                 }
                 int src0 = 0, nsrc = 0;
-                if (p.sk_len > 0 && u.kb0 > 0) {
+                if (kSk && p.sk_len > 0 && u.kb0 > 0) {
                     src0 = (u.tile * KB - p.sk_tile0 * KB) / p.sk_len;
                     nsrc = (int)blockIdx.x - src0;
                     if (lane == 0) {
@@ -1080,7 +1082,6 @@ bool make_weight_map_kn(CUtensorMap *map, const uint32_t *wq, int64_t K, int64_t
 // zero), then one fp32 partial tile slot per SM of 128 x 64 values (stream-K
 // runs only tiles of at most 64 activation rows).
 constexpr size_t kSkFlagBytes = 4096;
-constexpr int kSkMaxBN = 64;
 size_t sk_workspace_bytes() { return kSkFlagBytes + (size_t)num_sms() * kBM * kSkMaxBN * sizeof(float); }
 
 template <typename T, int BITS, int BN, bool KMAJOR>
