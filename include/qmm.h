@@ -107,9 +107,10 @@ qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K,
  * qmm_quantized_matmul_ws -- qmm_quantized_matmul with a caller workspace.
  * Nothing in the documents this library follows has a counterpart: the
  * workspace only lets the tensor-core path split the k-blocks of each output
- * tile over several CTAs ("stream-K") when a problem has fewer 128-row weight
- * tiles than the GPU has SMs and at most 64 activation rows per tile (decode
- * batches of 5..64 rows, small weights), so that every SM works.
+ * tile over several CTAs ("stream-K") when a problem has fewer 128-feature
+ * weight tiles than the GPU has SMs and at most 64 activation rows per tile
+ * (decode batches of 5..64 rows with W [N, K], 1..64 rows with W [K, N], small
+ * weights), so that every SM works.
  *   workspace: NULL (whole tiles, exactly qmm_quantized_matmul), or device
  *     memory of at least qmm_quantized_matmul_workspace_size(...) bytes,
  *     256-byte aligned, ZEROED before its first use; every call that returns

@@ -1093,10 +1093,13 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
     const bool sb_tma = KMAJOR && gpr % 8 == 0;
     int stages = 0, stg_rows = 0;
     size_t smem = 0;
-    const bool y_ok = KMAJOR && (a.N * 2) % 16 == 0 && (reinterpret_cast<uintptr_t>(a.y) & 15) == 0;
+    // (The [K, N] layout stages only narrow tiles, which stream-K may split;
+    // its wide tiles keep direct stores and the deeper ring.)
+    const bool y_ok = (KMAJOR || BN <= kSkMaxBN) && (a.N * 2) % 16 == 0 &&
+                      (reinterpret_cast<uintptr_t>(a.y) & 15) == 0;
     if (y_ok) {
         for (int rows = BN; rows >= 16 && stg_rows == 0; rows /= 2)
-            if (gemm_smem_plan<BITS, BN>(sb_tma, stages, smem, false, (size_t)kEpiWarps * 64 * rows) &&
+            if (gemm_smem_plan<BITS, BN>(sb_tma, stages, smem, !KMAJOR, (size_t)kEpiWarps * 64 * rows) &&
                 stages >= 4)
                 stg_rows = rows;
     }
@@ -1151,7 +1154,7 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
     // and with one or more full waves the last, partial wave runs on lightly
     // loaded SMs (prefill M=2048 with its tail split: unchanged), so both keep
     // whole tiles.
-    if (KMAJOR && BN <= kSkMaxBN && stg_rows > 0 && p.num_tiles < num_sms() && a.ws != nullptr &&
+    if (BN <= kSkMaxBN && stg_rows > 0 && p.num_tiles < num_sms() && a.ws != nullptr &&
         a.ws_bytes >= sk_workspace_bytes() && (size_t)num_sms() * 4 * sizeof(int) <= kSkFlagBytes) {
         const int64_t KB = a.K / kBK, sms = num_sms();
         const int64_t total = (int64_t)p.num_tiles * KB;
@@ -1272,7 +1275,7 @@ bool gemm_supported(qmm_dtype dt, const QmmArgs &a) {
 }
 
 size_t gemm_workspace_size(qmm_dtype dt, int64_t M, int64_t K, int64_t N, bool transpose, int bits) {
-    if ((dt != QMM_BF16 && dt != QMM_F16) || !transpose || M <= 0 || N <= 0 || K % kBK != 0) return 0;
+    if ((dt != QMM_BF16 && dt != QMM_F16) || M <= 0 || N <= 0 || K % kBK != 0) return 0;
     if (pick_bn(M) > kSkMaxBN) return 0;
     const int64_t tiles = ((M + pick_bn(M) - 1) / pick_bn(M)) * ((N + kBM - 1) / kBM);
     if (tiles >= num_sms()) return 0;
