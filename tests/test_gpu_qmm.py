@@ -209,3 +209,13 @@ def test_gemm_stream_k_workspace_options():
         torch.cuda.synchronize()
         assert row_rel_err(y, ref) <= REL_TOL[s.dtype]
     assert int(ws[:4096].count_nonzero()) == 0  # the flags are cleared again
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("m,k,n", [(1, 4096, 1024), (16, 2048, 640), (40, 1024, 384)])
+def test_gemm_stream_k_kn_layout(bits, m, k, n):
+    """Stream-K with the weight stored [K, N] (groups along N): several parts
+    per tile (eight for 4096 x 1024) combined by the owner."""
+    w = wl.with_outliers((k, n), seed=n + k + bits + 1, dtype=torch.bfloat16)
+    x = wl.normal((m, k), seed=m + k + 2, dtype=torch.bfloat16)
+    run_case(x, w, 64, bits, False, "gemm")
