@@ -31,7 +31,10 @@
 //   warps 8-11  epilogue: tcgen05.ld of the accumulator quadrant the warp may
 //               address (lanes 32*(warp%4)..), convert, then either stage the
 //               values in shared memory for one tensor store per slab or
-//               store y directly (grouped rows, unaligned y);
+//               store y directly (grouped rows, wide [K, N] tiles, unaligned
+//               y); under stream-K a CTA that stops inside a tile leaves an
+//               fp32 partial in the caller's workspace, and the CTA holding
+//               the tile's last k-block adds it before storing;
 //   warps 12,14,15  producers: TMA loads of the packed weight tile, the
 //               activation tile and the scale/bias windows of each k-block
 //               into a ring of stages;
@@ -333,7 +336,7 @@ struct GemmParams {
     int m_tiles, n_tiles, num_tiles, stages;
     int sb_tma;  // [N, K] layout: scale/bias windows arrive by TMA with each stage
     int stg_rows;  // output rows staged per tensor store (0: direct stores)
-    // Stream-K ([N, K] layout, staged epilogue): tiles below sk_tile0 go
+    // Stream-K (narrow tiles with the staged epilogue): tiles below sk_tile0 go
     // whole to CTAs (blockIdx.x, + gridDim.x, ...); for the rest CTA b works
     // through k-blocks [b*sk_len, (b+1)*sk_len) of their (tile, k-block)
     // space.  sk_len = 0: whole tiles only.
