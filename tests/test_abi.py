@@ -96,3 +96,40 @@ def test_matmul_empty_is_a_noop(L):
 def test_set_path(L):
     assert L.qmm_set_path(7) == 1
     assert L.qmm_set_path(0) == 0
+
+
+def mmws(L, ws=NULL, ws_bytes=0, **kw):
+    a = dict(x=FAKE, M=2, K=128, wq=FAKE, s=FAKE, b=FAKE, dtype=1, N=64, tr=1, gs=64,
+             bits=4, mode=None, y=FAKE)
+    a.update(kw)
+    return L.qmm_quantized_matmul_ws(a["x"], a["M"], a["K"], a["wq"], a["s"], a["b"], a["dtype"],
+                                     a["N"], a["tr"], a["gs"], a["bits"], a["mode"], a["y"],
+                                     ws, ws_bytes, NULL)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(K=96), 1), (dict(tr=0, N=96), 1), (dict(b=NULL), 1), (dict(x=MISALIGNED), 1),
+    (dict(mode=b"nvfp4"), 2), (dict(bits=3), 2),
+])
+def test_matmul_ws_rejects_like_the_plain_call(L, kw, status):
+    assert mmws(L, **kw) == status
+
+
+def test_matmul_ws_checks_workspace_alignment(L):
+    assert mmws(L, ws=ctypes.c_void_p(0x10080), ws_bytes=1 << 20) == 6  # QMM_ERR_WORKSPACE
+    assert mmws(L, M=0, x=NULL, y=NULL) == 0
+
+
+def test_matmul_workspace_size(L):
+    """Stream-K (and so a workspace) only for narrow tiles (at most 64
+    activation rows) when the problem has fewer 128-feature tiles than SMs."""
+    ws = lambda M, K, N, tr=1, bits=4, dt=1: int(L.qmm_quantized_matmul_workspace_size(
+        M, K, N, tr, bits, dt))
+    need = ws(16, 4096, 4096)
+    assert need > 4096                          # flags, then one partial slot per SM
+    assert ws(64, 4096, 4096) == need and ws(1, 4096, 4096, tr=0) == need
+    assert ws(4, 4096, 4096) == 0               # decode rows go to the SIMT kernel
+    assert ws(128, 4096, 4096) == 0             # wide tiles keep whole tiles
+    assert ws(64, 4096, 14336 * 4) == 0         # at least one full wave of tiles
+    assert ws(16, 4096, 4096, dt=0) == 0        # f32 has no tensor-core path
+    assert ws(16, 4000, 4096) == 0              # K not a multiple of the k-block
