@@ -45,9 +45,7 @@
 
 #include <algorithm>
 #include <cstring>
-#include <map>
 #include <mutex>
-#include <utility>
 
 #include "ptx_sm100.cuh"
 #include "qmm_internal.cuh"
@@ -336,11 +334,10 @@ struct GemmParams {
     int m_tiles, n_tiles, num_tiles, stages;
     int sb_tma;  // [N, K] layout: scale/bias windows arrive by TMA with each stage
     int stg_rows;  // output rows staged per tensor store (0: direct stores)
-    // Stream-K (narrow tiles with the staged epilogue): tiles below sk_tile0 go
-    // whole to CTAs (blockIdx.x, + gridDim.x, ...); for the rest CTA b works
-    // through k-blocks [b*sk_len, (b+1)*sk_len) of their (tile, k-block)
-    // space.  sk_len = 0: whole tiles only.
-    int sk_len, sk_tile0;
+    // Stream-K (narrow tiles with the staged epilogue): CTA b works through
+    // k-blocks [b*sk_len, (b+1)*sk_len) of the (tile, k-block) space.
+    // sk_len = 0: whole tiles blockIdx.x, + gridDim.x, ...
+    int sk_len;
     float *sk_ws;    // per CTA: one fp32 partial tile, [quadrant][chunk][lane][CW]
     int *sk_flags;   // per CTA and quadrant: 1 while its partial awaits the tile's owner
     int *err;
@@ -389,12 +386,11 @@ struct Unit {
     int tile, kb0, kb1;
 };
 
-// The units of one CTA, identical for every role.  Whole tiles blockIdx.x,
-// + gridDim.x, ... below the stream-K region; then the CTA's run of the
-// region's (tile, k-block) space walked from its end, so a tile split
-// between CTAs b and b+1 is finished last by b+1 (which combines the parts)
-// after b wrote its part first -- a waiting CTA only ever waits for
-// lower-numbered ones, which finished the same number of whole tiles.
+// The units of one CTA, identical for every role: whole tiles blockIdx.x,
+// + gridDim.x, ...; or, under stream-K, the CTA's run of the (tile, k-block)
+// space walked from its end, so a tile split between CTAs b and b+1 is
+// finished last by b+1 (which combines the parts) after b wrote its part
+// first -- a waiting CTA only ever waits for lower-numbered ones.
 struct Work {
     int next, stride, count, KB;  // whole tiles
     int cur, begin;               // stream-K
@@ -403,8 +399,8 @@ struct Work {
         next = blockIdx.x;
         stride = gridDim.x;
         const bool sk = p.sk_len > 0;
-        count = sk ? p.sk_tile0 : num_tiles;
-        begin = sk ? p.sk_tile0 * KB + (int)blockIdx.x * p.sk_len : 0;
+        count = sk ? 0 : num_tiles;
+        begin = sk ? (int)blockIdx.x * p.sk_len : 0;
         cur = sk ? min(num_tiles * KB, begin + p.sk_len) : 0;
     }
     __device__ bool get(Unit &u) {
@@ -765,7 +761,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 }
                 int src0 = 0, nsrc = 0;
                 if (kSk && p.sk_len > 0 && u.kb0 > 0) {
-                    src0 = (u.tile * KB - p.sk_tile0 * KB) / p.sk_len;
+                    src0 = (u.tile * KB) / p.sk_len;
                     nsrc = (int)blockIdx.x - src0;
                     if (lane == 0) {
                         for (int sI = 0; sI < nsrc; ++sI) {
@@ -1164,7 +1160,6 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
         const int64_t len = std::max<int64_t>(8, (total + sms - 1) / sms);
         if (total < (1LL << 30) && len * 10 <= KB * 9) {
             p.sk_len = (int)len;
-            p.sk_tile0 = 0;
             p.sk_flags = static_cast<int *>(a.ws);
             p.sk_ws = reinterpret_cast<float *>(static_cast<char *>(a.ws) + kSkFlagBytes);
             grid = (int)((total + len - 1) / len);
