@@ -96,6 +96,15 @@ qmm_status qmm_dequantize(const uint32_t *wq, const void *scales, const void *bi
  *                   wq [K, N*bits/32], scales/biases [K, N/gs]; N % gs == 0.
  * The packed weight is streamed and dequantized inside the product; no dense
  * weight is written to memory.  M == 0 or N == 0 is a no-op.
+ * Early start: the decode kernel (bf16/f16, transpose, M <= 4) is launched
+ *   with programmatic dependent launch.  If the kernel queued just before it
+ *   on the stream allows dependents to start early (PTX
+ *   griddepcontrol.launch_dependents), the decode kernel may begin reading
+ *   wq, scales and biases -- never x -- before that kernel has finished.  So
+ *   wq, scales and biases must not be written by such a kernel right before
+ *   the call.  Kernels that do not allow an early start (the usual case, and
+ *   every kernel of this library that writes a packed weight, such as
+ *   qmm_quantize) complete before the call reads anything.
  */
 qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K,
                                 const uint32_t *wq, const void *scales, const void *biases,
@@ -189,11 +198,13 @@ qmm_status qmm_gather_qmm(const void *x, int64_t x_batch, int64_t M, int64_t K,
  * QMM_GATHER_STATIC_SCRATCH_BYTES built into the library (one per device).
  *
  * Arguments, layouts, results and errors are those of qmm_gather_qmm.  In
- * addition, a bf16/f16 call with transpose != 0 whose
+ * addition, a call that takes the tensor-core path (bf16/f16, transpose != 0,
+ * K % 64 == 0, not forced onto the SIMT path by qmm_set_path) and whose
  * qmm_gather_qmm_workspace_size(batch, M, K, n_experts, dtype) exceeds
  * QMM_GATHER_STATIC_SCRATCH_BYTES returns QMM_ERR_WORKSPACE before launching
- * anything (use qmm_gather_qmm with a workspace for such sizes).  Example:
- * x [512, 1, 4096] bf16 needs about 4.2 MB.
+ * anything (use qmm_gather_qmm with a workspace for such sizes); calls on the
+ * SIMT path use no scratch and have no such limit.  Example: x [512, 1, 4096]
+ * bf16 needs about 4.2 MB.
  *
  * The scratch needs no initialisation (nothing in it must start at zero).
  * The first call on a device looks up the scratch's address, so make it
@@ -217,6 +228,33 @@ qmm_status qmm_gather_qmm_static(const void *x, int64_t x_batch, int64_t M, int6
  * (QMM_ERR_INDEX).  Returns QMM_OK when the word is clear.
  */
 qmm_status qmm_device_status(void *stream, int reset);
+
+/*
+ * qmm_set_wait_limit_ns -- limit of the bounded waits with which kernels
+ * wait on another party (a tile part another CTA leaves, a ring stage another
+ * warp fills), on the CURRENT device.  0 restores the default of 2 s.  When a
+ * wait runs out, the kernel records QMM_ERR_TIMEOUT in the device error word,
+ * carries on without the data (its results are then wrong but every access
+ * stays in bounds), and still waits, with the fixed 2 s limit, for its own
+ * copies and tensor-core work in flight before it exits.  For tests of the
+ * failure path; synchronous with the host.
+ */
+qmm_status qmm_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * qmm_inject_fault -- host-side fault injection for tests of the failure
+ * path (process-wide; read when a kernel launch is prepared).
+ *   QMM_FAULT_NONE                 no injection (the default);
+ *   QMM_FAULT_STREAMK_NO_PUBLISH   in the stream-K split of the tensor-core
+ *     product (qmm_quantized_matmul_ws with a workspace), the CTAs that leave
+ *     a tile part write it but never raise its ready flag, so the tile's
+ *     owner waits on a flag that nothing sets until the wait limit runs out
+ *     (QMM_ERR_TIMEOUT).  Such a call leaves the workspace flags as they were
+ *     and its output is wrong; zero the workspace before the next call.
+ * Nothing is injected on the device: no kernel faults, traps or hangs.
+ */
+typedef enum { QMM_FAULT_NONE = 0, QMM_FAULT_STREAMK_NO_PUBLISH = 1 } qmm_fault;
+qmm_status qmm_inject_fault(qmm_fault fault);
 
 /*
  * Kernel-path selection for qmm_quantized_matmul (process-wide; the default

@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
                                       i32, i32, i32, cp, i32, vp, vp],
             "qmm_device_status": [vp, i32],
             "qmm_set_path": [i32],
+            "qmm_set_wait_limit_ns": [ctypes.c_uint64],
+            "qmm_inject_fault": [i32],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -83,11 +85,12 @@ def _check(status: int):
 
 
 def _p(t: Optional[torch.Tensor]):
-    return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+    # A plain int (or None for NULL): ctypes converts it for c_void_p arguments.
+    return t.data_ptr() if t is not None else None
 
 
 def _stream(device: torch.device):
-    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    return torch.cuda.current_stream(device).cuda_stream
 
 
 def _mode(mode: Optional[str]):
@@ -96,7 +99,7 @@ def _mode(mode: Optional[str]):
 
 def _cuda(*ts):
     for t in ts:
-        if t is not None and (t.device.type != "cuda" or not t.is_contiguous()):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("libqmm takes contiguous CUDA tensors")
 
 
@@ -106,18 +109,24 @@ def _dtype(t: torch.Tensor) -> int:
     return DTYPES[t.dtype]
 
 
-def qmm_quantize(w: torch.Tensor, group_size: int = 64, bits: int = 4, mode: str = "affine"):
+def qmm_quantize(w: torch.Tensor, group_size: int = 64, bits: int = 4, mode: str = "affine",
+                 out=None):
     """Quantize ``w`` (rank >= 2) along its last axis -> (wq, scales, biases).
 
     ``wq`` is int32 holding the uint32 words; scales/biases take ``w``'s dtype.
+    ``out``: optional ``(wq, scales, biases)`` tensors to write into.
     """
     _cuda(w)
     cols = w.shape[-1]
     rows = w.numel() // cols if cols else 0
     lead = tuple(w.shape[:-1])
-    wq = torch.empty(lead + (cols * bits // 32,), dtype=torch.int32, device=w.device)
-    scales = torch.empty(lead + (max(cols // group_size, 0),), dtype=w.dtype, device=w.device)
-    biases = torch.empty_like(scales)
+    if out is not None:
+        wq, scales, biases = out
+        _cuda(wq, scales, biases)
+    else:
+        wq = torch.empty(lead + (cols * bits // 32,), dtype=torch.int32, device=w.device)
+        scales = torch.empty(lead + (max(cols // group_size, 0),), dtype=w.dtype, device=w.device)
+        biases = torch.empty_like(scales)
     _check(lib().qmm_quantize(_p(w), _dtype(w), rows, cols, group_size, bits, _mode(mode),
                               _p(wq), _p(scales), _p(biases), _stream(w.device)))
     return wq, scales, biases
@@ -138,12 +147,20 @@ def qmm_dequantize(wq, scales, biases, group_size: int = 64, bits: int = 4,
 # Zeroed stream-K workspaces, one per (device, stream), owned by this module
 # (torch memory) and reused across calls; the library leaves them zeroed.
 _mm_ws = {}
+# Workspace sizes by call shape (they depend on the forced path too, so
+# qmm_set_path clears this).
+_mm_ws_size = {}
 
 
 def qmm_quantized_matmul_workspace_size(M: int, K: int, N: int, transpose: bool = True,
                                         bits: int = 4, dtype=torch.bfloat16) -> int:
-    return int(lib().qmm_quantized_matmul_workspace_size(M, K, N, int(bool(transpose)), bits,
-                                                          DTYPES[dtype]))
+    key = (M, K, N, bool(transpose), bits, dtype)
+    n = _mm_ws_size.get(key)
+    if n is None:
+        n = int(lib().qmm_quantized_matmul_workspace_size(M, K, N, int(bool(transpose)), bits,
+                                                           DTYPES[dtype]))
+        _mm_ws_size[key] = n
+    return n
 
 
 def _matmul_workspace(device: torch.device, nbytes: int) -> torch.Tensor:
@@ -273,6 +290,21 @@ def qmm_device_status(reset: bool = True, device=None):
 
 def qmm_set_path(path: str = "auto"):
     _check(lib().qmm_set_path(PATHS[path]))
+    _mm_ws_size.clear()
+
+
+def qmm_set_wait_limit_ns(ns: int = 0):
+    """Limit of the kernels' bounded waits on the current device (0: the 2 s
+    default).  For tests of the failure path."""
+    _check(lib().qmm_set_wait_limit_ns(int(ns)))
+
+
+FAULTS = {"none": 0, "streamk_no_publish": 1}
+
+
+def qmm_inject_fault(fault: str = "none"):
+    """Host-side fault injection for tests (see include/qmm.h)."""
+    _check(lib().qmm_inject_fault(FAULTS[fault]))
 
 
 def qmm_launch_count() -> int:

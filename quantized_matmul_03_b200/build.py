@@ -48,7 +48,7 @@ def _stale(target: Path, deps) -> bool:
 def _compile(src: Path, extra) -> Path:
     obj = BUILD / (src.stem + ".o")
     if _stale(obj, [src, *_headers()]) or extra:
-        cmd = [NVCC, *NVCC_FLAGS, *extra, "-dc" if False else "-c", str(src), "-o", str(obj)]
+        cmd = [NVCC, *NVCC_FLAGS, *extra, "-c", str(src), "-o", str(obj)]
         subprocess.run(cmd, check=True)
     return obj
 

@@ -15,7 +15,7 @@
 
 namespace qmm {
 
-__device__ int g_qmm_device_error = 0;
+__device__ DeviceState g_qmm_state = {0, 0, kDefaultWaitNs};
 
 namespace {
 
@@ -23,6 +23,7 @@ thread_local std::string t_last_error;
 // Activation rows up to which the SIMT decode kernels are used (AUTO path).
 constexpr int64_t kGemvMaxRows = 4;
 qmm_path g_path = QMM_PATH_AUTO;
+std::atomic<int> g_fault{QMM_FAULT_NONE};
 
 qmm_status fail(qmm_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
 qmm_status fail(qmm_status st, const char *fmt, ...) {
@@ -92,6 +93,21 @@ qmm_status check_matmul(const void *x, int64_t M, int64_t K, const uint32_t *wq,
     return QMM_OK;
 }
 
+// Whether gather_qmm can take the grouped tensor-core path (which needs the
+// workspace) for these sizes.
+bool gather_tc_supported(qmm_dtype dtype, int64_t x_batch, int64_t M, int64_t K, int64_t N,
+                         int64_t n_experts, int64_t batch, int bits, int transpose) {
+    GroupedArgs probe{};
+    probe.transpose = transpose != 0;
+    probe.K = K;
+    probe.N = N;
+    probe.bits = bits;
+    probe.rows = batch * M;
+    probe.x_rows = x_batch * M;
+    probe.n_experts = n_experts;
+    return gemm_grouped_supported(dtype, probe) && gather_prep_fits(n_experts);
+}
+
 qmm_status finish_launch(cudaError_t e, const char *what) {
     if (e != cudaSuccess) return cuda_fail(e, what);
     return QMM_OK;
@@ -109,11 +125,13 @@ int *device_error_word() {
     if (dev < 0 || dev >= 64) return nullptr;
     if (cached[dev] == nullptr) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_qmm_device_error) != cudaSuccess) return nullptr;
-        cached[dev] = static_cast<int *>(p);
+        if (cudaGetSymbolAddress(&p, g_qmm_state) != cudaSuccess) return nullptr;
+        cached[dev] = &static_cast<DeviceState *>(p)->error;
     }
     return cached[dev];
 }
+
+int injected_fault() { return g_fault.load(std::memory_order_relaxed); }
 
 int current_device() {
     int dev = -1;
@@ -294,15 +312,8 @@ qmm_status qmm_gather_qmm(const void *x, int64_t x_batch, int64_t M, int64_t K,
         cudaStream_t s = (cudaStream_t)stream;
         const GatherIndex gi{lhs_indices, rhs_indices, batch, x_batch, n_experts};
 
-        GroupedArgs probe{};
-        probe.transpose = transpose != 0;
-        probe.K = K;
-        probe.N = N;
-        probe.bits = bits;
-        probe.rows = batch * M;
-        probe.x_rows = x_batch * M;
-        probe.n_experts = n_experts;
-        const bool tc_ok = gemm_grouped_supported(dtype, probe) && gather_prep_fits(n_experts);
+        const bool tc_ok = gather_tc_supported(dtype, x_batch, M, K, N, n_experts, batch, bits,
+                                               transpose);
         if (g_path == QMM_PATH_GEMM && !tc_ok)
             return fail(QMM_ERR_UNSUPPORTED,
                         "the tensor-core gather path needs bf16/f16, transpose, K %% 64 == 0");
@@ -343,7 +354,13 @@ qmm_status qmm_gather_qmm_static(const void *x, int64_t x_batch, int64_t M, int6
                                  int64_t batch, int transpose, int group_size, int bits,
                                  const char *mode, int sorted_indices, void *y, void *stream) {
     try {
-        if (transpose != 0) {
+        // Only the tensor-core path uses the scratch; the size limit applies
+        // to calls that take it.  (Invalid sizes are left to qmm_gather_qmm.)
+        const bool sizes_ok = batch >= 0 && x_batch >= 1 && n_experts >= 1 && M >= 0 && N >= 0 &&
+                              K > 0 && batch <= INT32_MAX && M <= INT32_MAX &&
+                              batch * M <= INT32_MAX / 2;
+        if (sizes_ok && g_path != QMM_PATH_GEMV &&
+            gather_tc_supported(dtype, x_batch, M, K, N, n_experts, batch, bits, transpose)) {
             const size_t need = qmm_gather_qmm_workspace_size(batch, M, K, n_experts, dtype);
             if (need > QMM_GATHER_STATIC_SCRATCH_BYTES)
                 return fail(QMM_ERR_WORKSPACE,
@@ -366,16 +383,31 @@ qmm_status qmm_device_status(void *stream, int reset) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
     int word = 0;
-    e = cudaMemcpyFromSymbol(&word, g_qmm_device_error, sizeof(int));
+    e = cudaMemcpyFromSymbol(&word, g_qmm_state, sizeof(int), offsetof(DeviceState, error));
     if (e != cudaSuccess) return cuda_fail(e, "read device error word");
     if (reset && word != 0) {
         const int zero = 0;
-        e = cudaMemcpyToSymbol(g_qmm_device_error, &zero, sizeof(int));
+        e = cudaMemcpyToSymbol(g_qmm_state, &zero, sizeof(int), offsetof(DeviceState, error));
         if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
     }
     if (word == QMM_ERR_TIMEOUT) return fail(QMM_ERR_TIMEOUT, "a kernel's bounded wait timed out");
     if (word == QMM_ERR_INDEX) return fail(QMM_ERR_INDEX, "an index was out of range");
     if (word != 0) return fail((qmm_status)word, "device error word %d", word);
+    return QMM_OK;
+}
+
+qmm_status qmm_set_wait_limit_ns(uint64_t ns) {
+    if (ns == 0) ns = kDefaultWaitNs;
+    const unsigned long long v = ns;
+    const cudaError_t e = cudaMemcpyToSymbol(g_qmm_state, &v, sizeof(v), offsetof(DeviceState, wait_ns));
+    if (e != cudaSuccess) return cuda_fail(e, "set the wait limit");
+    return QMM_OK;
+}
+
+qmm_status qmm_inject_fault(qmm_fault fault) {
+    if (fault != QMM_FAULT_NONE && fault != QMM_FAULT_STREAMK_NO_PUBLISH)
+        return fail(QMM_ERR_INVALID_ARG, "unknown fault %d", (int)fault);
+    g_fault.store((int)fault, std::memory_order_relaxed);
     return QMM_OK;
 }
 

@@ -340,6 +340,7 @@ struct GemmParams {
     int sk_len;
     float *sk_ws;    // per CTA: one fp32 partial tile, [quadrant][chunk][lane][CW]
     int *sk_flags;   // per CTA and quadrant: 1 while its partial awaits the tile's owner
+    int sk_no_publish;  // test injection: parts are written but their flags never raised
     int *err;
     // Grouped (gather_qmm) mode only: the chunk table and row map the
     // preparation kernel wrote.  Tile t covers chunk t / n_tiles and weight
@@ -484,8 +485,10 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
     // activation tile and A slot free; without SPLIT the whole stage).
     const uint32_t full_p = bar0, full_b = bar0 + 8 * S, full_a = bar0 + 16 * S;
     const uint32_t p_empty = bar0 + 24 * S, b_empty = bar0 + 32 * S;
-    const uint32_t acc_full = bar0 + 40 * S, acc_empty = acc_full + 16;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + (acc_empty + 16 - base));
+    // done: the MMA issuer's last tcgen05.mma has completed (tensor memory
+    // may be freed).
+    const uint32_t acc_full = bar0 + 40 * S, acc_empty = acc_full + 16, done = acc_empty + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + (done + 8 - base));
     const uint8_t *pg = gbase + (p0 - base);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -502,6 +505,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
             ptx::mbar_init(acc_full + 8 * a, 1);
             ptx::mbar_init(acc_empty + 8 * a, kEpiWarps);
         }
+        ptx::mbar_init(done, 1);
         ptx::fence_mbar_init();
     }
     if (warp == kWarpMma) {
@@ -756,7 +760,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     }
                     __threadfence();
                     __syncwarp();
-                    if (lane == 0) atomicExch(p.sk_flags + 4 * blockIdx.x + q, 1);
+                    if (lane == 0 && !p.sk_no_publish) atomicExch(p.sk_flags + 4 * blockIdx.x + q, 1);
                     continue;
                 }
                 int src0 = 0, nsrc = 0;
@@ -764,6 +768,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     src0 = (u.tile * KB) / p.sk_len;
                     nsrc = (int)blockIdx.x - src0;
                     if (lane == 0) {
+                        const uint64_t limit = wait_limit_ns(p.err);
                         for (int sI = 0; sI < nsrc; ++sI) {
                             int *f = p.sk_flags + 4 * (src0 + sI) + q;
                             const uint64_t t0 = ptx::globaltimer_ns();
@@ -771,7 +776,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                                 int fv;
                                 asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(fv) : "l"(f));
                                 if (fv != 0) break;
-                                if (ptx::globaltimer_ns() - t0 > ptx::kWaitNs) {
+                                if (ptx::globaltimer_ns() - t0 > limit) {
                                     record_device_error(p.err, QMM_ERR_TIMEOUT);
                                     break;
                                 }
@@ -909,9 +914,10 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     }
                 }
             }
-            // Drain: wait (bounded) for the last copies to land before exit.
+            // Drain: wait (bounded by the fixed limit) for the last copies to
+            // land before exit.
             for (int d = max(0, c - S); d < c; ++d)
-                ptx::mbar_wait(((SPLIT && role == 1) ? full_b : full_p) + 8 * (d % S), (d / S) & 1, p.err);
+                ptx::mbar_drain(((SPLIT && role == 1) ? full_b : full_p) + 8 * (d % S), (d / S) & 1, p.err);
         }
     } else if (warp == kWarpMma) {
         // ------------------------- MMA issuer -------------------------
@@ -966,6 +972,13 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
             if (leader) tc_commit(acc_full + 8 * acc);
             __syncwarp();
         }
+        // Every MMA issued must have completed before tensor memory is freed,
+        // also when a wait above gave up early.
+        if (leader) {
+            tc_commit(done);
+            ptx::mbar_drain(done, 0, p.err);
+        }
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
@@ -1160,6 +1173,7 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
         const int64_t len = std::max<int64_t>(8, (total + sms - 1) / sms);
         if (total < (1LL << 30) && len * 10 <= KB * 9) {
             p.sk_len = (int)len;
+            p.sk_no_publish = injected_fault() == QMM_FAULT_STREAMK_NO_PUBLISH;
             p.sk_flags = static_cast<int *>(a.ws);
             p.sk_ws = reinterpret_cast<float *>(static_cast<char *>(a.ws) + kSkFlagBytes);
             grid = (int)((total + len - 1) / len);

@@ -155,7 +155,11 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     // Let the next launch in the stream begin its own prologue (barrier set-up
     // and weight streaming) as this grid's CTAs retire.  Everything this grid
     // reads before grid_dependency_wait() is the packed weight, its scales and
-    // biases, which no kernel of this library writes while it may overlap.
+    // biases.  Only a preceding kernel that itself allows an early start
+    // (griddepcontrol.launch_dependents) can still be running then: in this
+    // library that is this kernel, which writes none of them; qmm_quantize,
+    // which does write them, never allows it, so a call after it starts only
+    // once it has completed.  The header states the rule for other writers.
     ptx::grid_launch_dependents();
 
     if (warp == 0) {
@@ -197,6 +201,10 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                 }
             }
             if (handoff) atomicMax(&g_sm_issued[smid], ticket + 1);
+            // The CTA must not exit while a copy into its ring can still land
+            // (the consumers may have given up on a stage after a timeout).
+            for (int i = max(0, nst - S); i < nst; ++i)
+                ptx::mbar_drain(full0 + 8 * (i % S), (i / S) & 1, err);
         }
     } else {
         // ---------------- consumers ----------------
@@ -246,9 +254,11 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     }
                 }
                 // amax < 2^ex (ex = biased exponent - 126); x * 2^sh < 2^14 with
-                // sh = 14 - ex, clamped so that 2^sh and 2^-sh are normal floats.
+                // sh = 14 - ex, clamped so that 2^sh and 2^-sh are normal floats
+                // (the lower clamp is reached by no finite 16-bit value: bf16
+                // stays below 2^128, so sh >= -114).
                 const int ex = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
-                const int sh = min(126, max(-100, 14 - ex));
+                const int sh = min(126, max(-126, 14 - ex));
                 const float up = __uint_as_float((uint32_t)(127 + sh) << 23);
                 fsc[m][u] = __uint_as_float((uint32_t)(127 - sh) << 23);
                 xsum[m][u] = sum;

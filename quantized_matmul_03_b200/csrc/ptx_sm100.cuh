@@ -64,28 +64,46 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for the phase of parity `parity` to complete, for at most ~kWaitNs.
-// On timeout the device error word gets QMM_ERR_TIMEOUT and false is
-// returned; callers then carry on without the data (their shared-memory
-// accesses stay in bounds), so every thread still reaches the kernel's end.
-// SLEEP selects suspending waits (long, off the critical path) or spinning
-// ones (short hand-offs where a wake-up delay would cost throughput).
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
+// Wait for the phase of parity `parity` to complete, for at most the
+// library's wait limit (2 s unless qmm_set_wait_limit_ns changed it).  On
+// timeout the device error word gets QMM_ERR_TIMEOUT and false is returned;
+// callers then carry on without the data (their shared-memory accesses stay
+// in bounds), so every thread still reaches the kernel's end.  SLEEP selects
+// suspending waits (long, off the critical path) or spinning ones (short
+// hand-offs where a wake-up delay would cost throughput).
 template <bool SLEEP = true>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *err) {
     if (mbar_test(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
+    const uint64_t limit = wait_limit_ns(err);
     for (;;) {
         for (int i = 0; i < 64; ++i)
             if (SLEEP ? mbar_try_wait(bar, parity) : mbar_test(bar, parity)) return true;
         const uint64_t dt = globaltimer_ns() - t0;
-        if (dt > kWaitNs) {
+        if (dt > limit) {
             record_device_error(err, QMM_ERR_TIMEOUT);
             return false;
         }
         // After 1 ms, give up at once if another wait already timed out (the
         // error word is global memory: never read it on the fast path).
         if (dt > 1000000ull && *reinterpret_cast<volatile int *>(err) != 0) return false;
+    }
+}
+
+// Wait for this CTA's own asynchronous operations (copies into its shared
+// memory, its tensor-core work) before it exits or frees tensor memory.  The
+// limit is the fixed default, never the settable one: a CTA must not leave
+// while its copies can still land.
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, int *err) {
+    if (mbar_test(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > kDefaultWaitNs) {
+            record_device_error(err, QMM_ERR_TIMEOUT);
+            return false;
+        }
     }
 }
 

@@ -8,6 +8,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "../../include/qmm.h"
@@ -31,13 +32,29 @@ template <> struct Dt<__half> {
     static __device__ __forceinline__ __half from_f(float v) { return __float2half_rn(v); }
 };
 
-// Device-side error word (QMM_OK when clear), defined in api.cu.  Kernels
-// that can fail receive its device address (device_error_word()) and set it
-// with atomicCAS so that the first error recorded wins.
+// Device-side state of the library, one per device, defined in api.cu:
+// the error word (QMM_OK when clear) and the limit of the bounded waits.
+// Kernels that can fail receive the address of the error word
+// (device_error_word()), set it with atomicCAS so that the first error
+// recorded wins, and find the wait limit beside it.
+struct DeviceState {
+    int error;
+    int pad;
+    unsigned long long wait_ns;  // limit of a bounded wait on another party
+};
 __device__ __forceinline__ void record_device_error(int *word, int code) {
     atomicCAS(word, 0, code);
 }
-int *device_error_word();  // host: device address of the word (current device)
+// Limit of a bounded wait, read only once a wait has not completed at once.
+__device__ __forceinline__ unsigned long long wait_limit_ns(const int *word) {
+    return *reinterpret_cast<const volatile unsigned long long *>(
+        reinterpret_cast<const char *>(word) + offsetof(DeviceState, wait_ns));
+}
+int *device_error_word();  // host: device address of the error word (current device)
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s
+
+// Host-side test injection (qmm_inject_fault); read when a launch is built.
+int injected_fault();
 
 // Host: the current device (-1 if the runtime cannot say).
 int current_device();

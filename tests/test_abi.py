@@ -133,3 +133,8 @@ def test_matmul_workspace_size(L):
     assert ws(64, 4096, 14336 * 4) == 0         # at least one full wave of tiles
     assert ws(16, 4096, 4096, dt=0) == 0        # f32 has no tensor-core path
     assert ws(16, 4000, 4096) == 0              # K not a multiple of the k-block
+
+
+def test_fault_injection_rejects_unknown_values(L):
+    assert L.qmm_inject_fault(99) == 1
+    assert L.qmm_inject_fault(0) == 0
