@@ -15,15 +15,21 @@ Parity status per function (what pins it is in ``tests/test_oracle_pins.py``):
                       weight is exactly on the grid (both layouts), one-hot
                       rows, the doctest shapes, the mlx-rs
                       ``test_quantized_matmul`` bound.
+  quantized_dense     pinned: a zero bias gives quantized_matmul exactly; a
+                      one-hot row gives a column of the dequantized weight plus
+                      the bias; a constant-bias tensor equals the number form.
   gather_qmm          pinned: the two cases of mlx-rs ``test_gather_qmm``
                       against an independent indexed dense product.
 """
 from .ref import (  # noqa: F401
     DTYPE_TAG,
     dequantize,
+    MX_MODES,
     dequantize_f32,
+    encode_elements,
     gather_qmm,
     quantize,
+    quantized_dense,
     quantized_matmul,
     round_to_dtype,
     unpack_codes,

@@ -108,6 +108,16 @@ static int check_args(int dtype, int64_t rows, int64_t cols, int group_size, int
     return ORC_OK;
 }
 
+/* Store code q of element (r, c): element c of a row sits at bit
+ * (c mod 32/bits) * bits of the row's word c / (32/bits), least significant
+ * code first (words zeroed beforehand). */
+static void put_code(uint32_t *wq, int64_t words_per_row, int bits, int64_t r, int64_t c,
+                     uint32_t q)
+{
+    const int64_t per_word = 32 / bits;
+    wq[r * words_per_row + c / per_word] |= q << ((c % per_word) * bits);
+}
+
 /*
  * Quantize w[rows, cols] (row-major, dtype `dtype`) group by group along the
  * last axis.  Outputs: wq[rows, cols*bits/32] (uint32), scales and biases
@@ -157,7 +167,7 @@ int oracle_quantize(const void *w, int dtype, int64_t rows, int64_t cols,
                     q = (uint32_t)t;
                 }
                 const int64_t c = g * group_size + j; /* column within the row */
-                wq[r * words_per_row + c / per_word] |= q << ((c % per_word) * bits);
+                put_code(wq, words_per_row, bits, r, c, q);
             }
         }
     }
@@ -224,5 +234,193 @@ int oracle_round_to_dtype(const float *in, int dtype, int64_t n, void *out)
         return ORC_BAD_ARG;
     for (int64_t i = 0; i < n; ++i)
         store_elem(out, dtype, i, in[i]);
+    return ORC_OK;
+}
+
+/* ======================================================================
+ * Microscaled modes (Emily.QuantizedWeight, section Microscaled modes):
+ *   mxfp4  group 32, 4-bit E2M1 elements, E8M0 scale byte
+ *   mxfp8  group 32, 8-bit E4M3 elements, E8M0 scale byte
+ *   nvfp4  group 16, 4-bit E2M1 elements, E4M3 scale byte
+ * no biases.  The pages name the formats (a fused e8m0/e4m3 scale stored as
+ * u8) but give no rule; the rule here follows the published definitions:
+ *   - element and scale encodings: OCP Microscaling Formats (MX) v1.0
+ *     (E2M1: bias 1, magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6;  E4M3: bias 7,
+ *     largest finite 448, S.1111.111 is NaN;  E8M0: 2^(E - 127));
+ *   - mx scale: X = 2^(floor(log2(max |v|)) - emax_elem), emax_elem = 2 for
+ *     E2M1 and 8 for E4M3, clamped to the E8M0 range; elements are v / X
+ *     rounded to nearest-even and saturated to the largest finite value
+ *     (OCP MX v1.0, conversion of a vector to MX);
+ *   - nvfp4 scale: the block maximum is mapped to E2M1's 6:  s = max|v| / 6
+ *     rounded (nearest-even, saturating) to E4M3; elements are v / s in E2M1
+ *     (NVIDIA's NVFP4 block format, without the optional per-tensor scale,
+ *     which the pages' calls do not pass).
+ * An all-zero block gets scale byte 0 and zero elements.
+ * ====================================================================== */
+
+#define ORC_MXFP4 1
+#define ORC_MXFP8 2
+#define ORC_NVFP4 3
+
+static const float e2m1_mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+static float e2m1_value(uint32_t code)
+{
+    float m = e2m1_mag[code & 7u];
+    return (code & 8u) ? -m : m;
+}
+
+/* Nearest E2M1 value, ties to the even code (last mantissa bit 0), values
+ * beyond 6 saturated to 6; the sign is kept (so -0.1 gives negative zero). */
+static uint32_t e2m1_encode(float v)
+{
+    const uint32_t sign = signbit(v) ? 8u : 0u;
+    const float a = fabsf(v);
+    uint32_t c;
+    if (a <= 0.25f) c = 0;        /* 0.25: tie between 0 and 0.5 -> 0 (even) */
+    else if (a < 0.75f) c = 1;    /* 0.5 */
+    else if (a <= 1.25f) c = 2;   /* 1.0 (0.75 and 1.25 are ties that go to it) */
+    else if (a < 1.75f) c = 3;    /* 1.5 */
+    else if (a <= 2.5f) c = 4;    /* 2.0 (1.75 and 2.5 go to it) */
+    else if (a < 3.5f) c = 5;     /* 3.0 */
+    else if (a <= 5.0f) c = 6;    /* 4.0 (3.5 and 5.0 go to it) */
+    else c = 7;                   /* 6.0, and everything above */
+    return sign | c;
+}
+
+static float e4m3_value(uint32_t code)
+{
+    const uint32_t e = (code >> 3) & 15u, m = code & 7u;
+    float a;
+    if (e == 15u && m == 7u) a = NAN;
+    else if (e == 0u) a = ldexpf((float)m, -9);                 /* m/8 * 2^-6 */
+    else a = ldexpf(1.0f + (float)m / 8.0f, (int)e - 7);
+    return (code & 0x80u) ? -a : a;
+}
+
+/* Nearest E4M3 value, ties to even, saturated to +-448 (no infinities). */
+static uint32_t e4m3_encode(float v)
+{
+    const uint32_t sign = signbit(v) ? 0x80u : 0u;
+    const float a = fabsf(v);
+    if (a >= 0x1.0p-6f) {
+        int e2;
+        frexpf(a, &e2);              /* a = f * 2^e2, f in [0.5, 1) */
+        int e = e2 - 1;              /* a in [2^e, 2^(e+1)) */
+        float mi = rintf(ldexpf(a, 3 - e) - 8.0f);   /* mantissa in eighths, RNE */
+        if (mi == 8.0f) {
+            mi = 0.0f;
+            ++e;
+        }
+        if (e > 8 || (e == 8 && mi == 7.0f)) return sign | 0x7Eu;  /* 448 */
+        return sign | ((uint32_t)(e + 7) << 3) | (uint32_t)mi;
+    }
+    /* subnormal range: multiples of 2^-9 (m = 8 is the smallest normal, code 8) */
+    const float m = rintf(ldexpf(a, 9));
+    return sign | (uint32_t)m;
+}
+
+static int mx_params(int mode, int *gs, int *bits)
+{
+    switch (mode) {
+    case ORC_MXFP4: *gs = 32; *bits = 4; return ORC_OK;
+    case ORC_MXFP8: *gs = 32; *bits = 8; return ORC_OK;
+    case ORC_NVFP4: *gs = 16; *bits = 4; return ORC_OK;
+    default: return ORC_BAD_ARG;
+    }
+}
+
+/* Element codes of `n` values for a mode's element format (for pins). */
+int oracle_encode_elements(int mode, const float *in, int64_t n, uint8_t *out)
+{
+    int gs, bits;
+    if (mx_params(mode, &gs, &bits) != ORC_OK) return ORC_BAD_ARG;
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = (uint8_t)(bits == 8 ? e4m3_encode(in[i]) : e2m1_encode(in[i]));
+    return ORC_OK;
+}
+
+/* Value of a scale byte (E8M0 for mx modes, E4M3 for nvfp4). */
+static float mx_scale_value(int mode, uint32_t s)
+{
+    return mode == ORC_NVFP4 ? e4m3_value(s) : ldexpf(1.0f, (int)s - 127);
+}
+
+int oracle_quantize_mx(const void *w, int dtype, int64_t rows, int64_t cols, int mode,
+                       uint32_t *wq, uint8_t *scales)
+{
+    int gs, bits;
+    if (mx_params(mode, &gs, &bits) != ORC_OK) return ORC_BAD_ARG;
+    if (dtype != ORC_F32 && dtype != ORC_BF16 && dtype != ORC_F16) return ORC_BAD_ARG;
+    if (rows < 0 || cols <= 0 || cols % gs != 0) return ORC_BAD_ARG;
+    const int64_t per_word = 32 / bits;
+    const int64_t words_per_row = cols / per_word;
+    const int64_t groups_per_row = cols / gs;
+    const int emax = bits == 8 ? 8 : 2;
+    memset(wq, 0, (size_t)(rows * words_per_row) * sizeof(uint32_t));
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t g = 0; g < groups_per_row; ++g) {
+            const int64_t first = r * cols + g * gs;
+            float amax = 0.0f;
+            for (int j = 0; j < gs; ++j) {
+                float a = fabsf(load_elem(w, dtype, first + j));
+                if (a > amax) amax = a;
+            }
+            uint32_t scode;
+            float div = 0.0f;   /* nvfp4: the stored scale the elements are divided by */
+            int shared = -127;  /* mx: scale exponent */
+            if (mode == ORC_NVFP4) {
+                scode = e4m3_encode(amax / 6.0f);
+                div = e4m3_value(scode);
+            } else if (amax == 0.0f) {
+                scode = 0;
+            } else {
+                int e2;
+                frexpf(amax, &e2);
+                shared = (e2 - 1) - emax;          /* floor(log2 amax) - emax_elem */
+                if (shared < -127) shared = -127;
+                if (shared > 127) shared = 127;
+                scode = (uint32_t)(shared + 127);
+            }
+            scales[r * groups_per_row + g] = (uint8_t)scode;
+            for (int j = 0; j < gs; ++j) {
+                const float v = load_elem(w, dtype, first + j);
+                uint32_t q;
+                if (mode == ORC_NVFP4) {
+                    q = div == 0.0f ? 0u : e2m1_encode(v / div);
+                } else if (amax == 0.0f) {
+                    q = 0u;
+                } else {
+                    const float t = ldexpf(v, -shared);   /* v / X */
+                    q = bits == 8 ? e4m3_encode(t) : e2m1_encode(t);
+                }
+                put_code(wq, words_per_row, bits, r, g * gs + j, q);
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/* w = X * element, X the value of the group's scale byte; fp32 (exact) in
+ * out_f32 (may be NULL) and rounded to `dtype` in out (may be NULL). */
+int oracle_dequantize_mx(const uint32_t *wq, const uint8_t *scales, int dtype, int64_t rows,
+                         int64_t cols, int mode, void *out, float *out_f32)
+{
+    int gs, bits;
+    if (mx_params(mode, &gs, &bits) != ORC_OK) return ORC_BAD_ARG;
+    if (dtype != ORC_F32 && dtype != ORC_BF16 && dtype != ORC_F16) return ORC_BAD_ARG;
+    if (rows < 0 || cols <= 0 || cols % gs != 0) return ORC_BAD_ARG;
+    const int64_t words_per_row = cols * bits / 32;
+    const int64_t groups_per_row = cols / gs;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t c = 0; c < cols; ++c) {
+            const float x = mx_scale_value(mode, scales[r * groups_per_row + c / gs]);
+            const uint32_t q = code_at(wq, words_per_row, bits, r, c);
+            const float e = bits == 8 ? e4m3_value(q) : e2m1_value(q);
+            const float v = x * e;
+            if (out_f32) out_f32[r * cols + c] = v;
+            if (out) store_elem(out, dtype, r * cols + c, v);
+        }
+    }
     return ORC_OK;
 }

@@ -30,8 +30,12 @@ def _load():
         lib.oracle_dequantize.argtypes = [vp, vp, vp, i32, i64, i64, i32, i32, vp, vp]
         lib.oracle_unpack_codes.argtypes = [vp, i64, i64, i32, vp]
         lib.oracle_round_to_dtype.argtypes = [vp, i32, i64, vp]
+        lib.oracle_quantize_mx.argtypes = [vp, i32, i64, i64, i32, vp, vp]
+        lib.oracle_dequantize_mx.argtypes = [vp, vp, i32, i64, i64, i32, vp, vp]
+        lib.oracle_encode_elements.argtypes = [i32, vp, i64, vp]
         for f in (lib.oracle_quantize, lib.oracle_dequantize, lib.oracle_unpack_codes,
-                  lib.oracle_round_to_dtype):
+                  lib.oracle_round_to_dtype, lib.oracle_quantize_mx, lib.oracle_dequantize_mx,
+                  lib.oracle_encode_elements):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -46,7 +50,78 @@ def _cpu(t: torch.Tensor) -> torch.Tensor:
     return t.contiguous()
 
 
-def quantize(w: torch.Tensor, group_size: int = 64, bits: int = 4):
+# Microscaled modes (Emily.QuantizedWeight, section Microscaled modes): their
+# fixed (group_size, bits), and the oracle's own tags for them.
+MX_MODES = {"mxfp4": (32, 4, 1), "mxfp8": (32, 8, 2), "nvfp4": (16, 4, 3)}
+
+
+def _mx_mode(mode, group_size, bits):
+    if mode not in MX_MODES:
+        raise ValueError(f"unknown mode {mode!r}")
+    gs, b, tag = MX_MODES[mode]
+    if group_size != gs or bits != b:
+        raise ValueError(f"mode {mode} needs group_size={gs} and bits={b}")
+    return tag
+
+
+def quantize(w: torch.Tensor, group_size: int = 64, bits: int = 4, mode: str = "affine"):
+    """Group-wise quantization along the last axis of a rank>=2 tensor.
+
+    ``mode`` "affine" (below), or a microscaled mode ("mxfp4", "mxfp8",
+    "nvfp4"), which returns ``(wq, scales, None)`` with one scale byte per group
+    (Emily.QuantizedWeight, section Microscaled modes; the rule is in
+    ``qmm_oracle.c``).
+    """
+    if mode != "affine":
+        return _quantize_mx(w, group_size, bits, mode)
+    return _quantize_affine(w, group_size, bits)
+
+
+def _quantize_mx(w, group_size, bits, mode):
+    tag = _mx_mode(mode, group_size, bits)
+    w = _cpu(w)
+    if w.dim() < 2 or w.dtype not in DTYPE_TAG:
+        raise ValueError("quantize needs a float tensor of rank 2 or higher")
+    cols = w.shape[-1]
+    if cols % group_size:
+        raise ValueError("the last axis must be a multiple of the group size")
+    rows = w.numel() // cols
+    lead = tuple(w.shape[:-1])
+    wq = torch.empty(lead + (cols * bits // 32,), dtype=torch.int32)
+    scales = torch.empty(lead + (cols // group_size,), dtype=torch.uint8)
+    if _load().oracle_quantize_mx(_ptr(w), DTYPE_TAG[w.dtype], rows, cols, tag, _ptr(wq),
+                                  _ptr(scales)):
+        raise ValueError("oracle_quantize_mx rejected its arguments")
+    return wq, scales, None
+
+
+def _deq_mx(wq, scales, group_size, bits, mode, dtype, want_f32):
+    tag = _mx_mode(mode, group_size, bits)
+    wq, scales = _cpu(wq), _cpu(scales)
+    cols = wq.shape[-1] * 32 // bits
+    rows = wq.numel() // wq.shape[-1]
+    lead = tuple(wq.shape[:-1])
+    if scales.dtype != torch.uint8 or scales.shape != lead + (cols // group_size,):
+        raise ValueError("microscaled scales are uint8 [..., cols / group_size]")
+    out = torch.empty(lead + (cols,), dtype=torch.float32 if want_f32 else dtype)
+    args = (ctypes.c_void_p(0), _ptr(out)) if want_f32 else (_ptr(out), ctypes.c_void_p(0))
+    if _load().oracle_dequantize_mx(_ptr(wq), _ptr(scales), DTYPE_TAG[dtype], rows, cols, tag,
+                                    *args):
+        raise ValueError("oracle_dequantize_mx rejected its arguments")
+    return out
+
+
+def encode_elements(values: torch.Tensor, mode: str) -> torch.Tensor:
+    """Element codes (uint8) of fp32 values in a microscaled mode's element
+    format: E2M1 for mxfp4/nvfp4, E4M3 for mxfp8 (nearest-even, saturating)."""
+    gs, bits, tag = MX_MODES[mode]
+    v = _cpu(values.to(torch.float32)).reshape(-1)
+    out = torch.empty(v.numel(), dtype=torch.uint8)
+    _load().oracle_encode_elements(tag, _ptr(v), v.numel(), _ptr(out))
+    return out.reshape(values.shape)
+
+
+def _quantize_affine(w: torch.Tensor, group_size: int = 64, bits: int = 4):
     """Group-wise affine quantization along the last axis of a rank>=2 tensor.
 
     EMLX.Quantization, section ``quantize`` (rank 2 or higher, last axis);
@@ -96,18 +171,26 @@ def _deq(wq, scales, biases, group_size, bits, want_f32: bool):
     return out
 
 
-def dequantize(wq, scales, biases, group_size: int = 64, bits: int = 4):
+def dequantize(wq, scales, biases, group_size: int = 64, bits: int = 4, mode: str = "affine",
+               dtype=torch.bfloat16):
     """``w = scale * q + bias`` per element, rounded to the scales dtype.
+
+    Microscaled modes: ``w = X * element`` (no bias), rounded to ``dtype``.
 
     mlx-rs ops/quantization.rs, ``dequantize``; EMLX.Quantization, section
     ``dequantize`` (same logical shape as the dense tensor); output dtype is the
     scales dtype (EMLX.Quantization, section ``quantized_matmul``).
     """
+    if mode != "affine":
+        return _deq_mx(wq, scales, group_size, bits, mode, dtype, want_f32=False)
     return _deq(wq, scales, biases, group_size, bits, want_f32=False)
 
 
-def dequantize_f32(wq, scales, biases, group_size: int = 64, bits: int = 4):
-    """The fp32 value ``fmaf(scale, q, bias)`` before rounding to the dtype."""
+def dequantize_f32(wq, scales, biases, group_size: int = 64, bits: int = 4, mode: str = "affine"):
+    """The fp32 value ``fmaf(scale, q, bias)`` (microscaled: ``X * element``,
+    exact) before rounding to the dtype."""
+    if mode != "affine":
+        return _deq_mx(wq, scales, group_size, bits, mode, torch.float32, want_f32=True)
     return _deq(wq, scales, biases, group_size, bits, want_f32=True)
 
 
@@ -133,17 +216,36 @@ def round_to_dtype(t: torch.Tensor, dtype) -> torch.Tensor:
 
 
 def quantized_matmul(x, wq, scales, biases, transpose: bool = True,
-                     group_size: int = 64, bits: int = 4) -> torch.Tensor:
+                     group_size: int = 64, bits: int = 4, mode: str = "affine") -> torch.Tensor:
     """float64 ``x @ W.T`` (transpose=True, W stored [out, in]) or ``x @ W``
     (transpose=False, W stored [in, out]) with W the dequantized weight.
 
     mlx-rs ops/quantization.rs, ``quantized_matmul``; Emily.Quantization.Layers,
     ``quantized_dense`` (the two layouts).  The weight enters as the fp32 value
-    ``fmaf(scale, q, bias)``; products and sums are float64.
+    ``fmaf(scale, q, bias)`` (microscaled modes: ``X * element``); products and
+    sums are float64.
     """
-    w = dequantize_f32(wq, scales, biases, group_size, bits).double()
+    w = dequantize_f32(wq, scales, biases, group_size, bits, mode).double()
     w = w.transpose(-1, -2) if transpose else w
     return _cpu(x).double() @ w
+
+
+def quantized_dense(x, wq, scales, biases, bias=0, transpose: bool = True,
+                    group_size: int = 64, bits: int = 4) -> torch.Tensor:
+    """float64 ``x @ W (+ bias)``: the dense layer on a quantized weight.
+
+    Emily.Quantization.Layers, ``quantized_dense``: the layer computes the
+    quantized product in the weight's layout and adds a bias that is either a
+    tensor or a number (0 when absent).  Read here as: a tensor holds one value
+    per output feature and is broadcast over the rows of ``x``; a number is
+    added to every output.  The sum is taken in float64, before any rounding to
+    the output dtype (the bias is part of the fused product, not a second
+    rounded step).
+    """
+    y = quantized_matmul(x, wq, scales, biases, transpose, group_size, bits)
+    if isinstance(bias, torch.Tensor):
+        return y + _cpu(bias).double().reshape(-1)
+    return y + float(bias)
 
 
 def gather_qmm(x, wq, scales, biases, lhs_indices=None, rhs_indices=None,

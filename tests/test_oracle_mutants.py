@@ -14,6 +14,7 @@ import oracle
 import oracle.ref as ref
 from oracle import build as obuild
 
+import test_oracle_mx_pins as mx_pins
 import test_oracle_pins as pins
 
 SRC = Path(obuild.SRC).read_text()
@@ -33,6 +34,14 @@ MUTANTS = {
     "truncating_bf16": ("u += 0x7fffu + keep_lsb;", "u += 0u;"),
     "wrong_word_stride": ("uint32_t word = wq[r * words_per_row + c / per_word];",
                           "uint32_t word = wq[r + c / per_word];"),
+    # microscaled modes
+    "mx_emax_e2m1": ("const int emax = bits == 8 ? 8 : 2;", "const int emax = bits == 8 ? 8 : 3;"),
+    "e8m0_bias": ("scode = (uint32_t)(shared + 127);", "scode = (uint32_t)(shared + 126);"),
+    "e2m1_tie_up": ("if (a <= 0.25f) c = 0;", "if (a < 0.25f) c = 0;"),
+    "nvfp4_divisor": ("scode = e4m3_encode(amax / 6.0f);", "scode = e4m3_encode(amax / 4.0f);"),
+    "e4m3_no_saturation": ("if (e > 8 || (e == 8 && mi == 7.0f)) return sign | 0x7Eu;",
+                           "if (e > 8) return sign | 0x7Eu;"),
+    "e4m3_subnormal_step": ("const float m = rintf(ldexpf(a, 9));", "const float m = rintf(ldexpf(a, 8));"),
 }
 
 
@@ -60,6 +69,13 @@ def _pin_calls():
             calls.append(lambda bits=bits, dt=dt: pins.test_on_grid_round_trip_is_exact(dt, bits, 64))
     for dt in (torch.bfloat16, torch.float16):
         calls.append(lambda dt=dt: pins.test_dtype_rounding_matches_library(dt))
+    calls += [mx_pins.test_e2m1_value_table, mx_pins.test_e2m1_rounding_ties_to_even_and_saturates,
+              mx_pins.test_e4m3_named_points_and_saturation, mx_pins.test_e4m3_rounding_matches_torch_float8,
+              mx_pins.test_e4m3_value_table_matches_torch_float8, mx_pins.test_e8m0_scale_values]
+    for i in range(len(mx_pins.GOLD["blocks"]["cases"])):
+        calls.append(lambda i=i: mx_pins.test_worked_blocks(i))
+    for mode in ("mxfp4", "mxfp8", "nvfp4"):
+        calls.append(lambda mode=mode: mx_pins.test_on_grid_blocks_round_trip_exactly(mode))
     return calls
 
 
@@ -92,4 +108,56 @@ def test_pins_catch_mutant(name, tmp_path):
 
 def test_unmutated_oracle_passes_all_pin_calls():
     for call in _pin_calls():
+        call()
+
+
+# quantized_dense adds the layer bias in Python (oracle/ref.py): mutants of
+# that step, swapped in for oracle.quantized_dense while the dense pins run.
+def _dense_mutants():
+    import torch
+    mm = ref.quantized_matmul
+
+    def drops_bias(x, wq, s, b, bias=0, transpose=True, gs=64, bits=4):
+        return mm(x, wq, s, b, transpose, gs, bits)
+
+    def bias_twice(x, wq, s, b, bias=0, transpose=True, gs=64, bits=4):
+        y = mm(x, wq, s, b, transpose, gs, bits)
+        bb = bias.double().reshape(-1) if isinstance(bias, torch.Tensor) else float(bias)
+        return y + 2 * bb
+
+    def bias_along_rows(x, wq, s, b, bias=0, transpose=True, gs=64, bits=4):
+        y = mm(x, wq, s, b, transpose, gs, bits)
+        if isinstance(bias, torch.Tensor):
+            return y + bias.double().reshape(-1)[: y.shape[0]].reshape(-1, 1)
+        return y + float(bias)
+
+    def ignores_number(x, wq, s, b, bias=0, transpose=True, gs=64, bits=4):
+        y = mm(x, wq, s, b, transpose, gs, bits)
+        return y + bias.double().reshape(-1) if isinstance(bias, torch.Tensor) else y
+
+    return {"drops_bias": drops_bias, "bias_twice": bias_twice,
+            "bias_along_rows": bias_along_rows, "ignores_number": ignores_number}
+
+
+def _dense_pin_calls():
+    return [lambda: pins.test_dense_one_hot_rows_give_weight_column_plus_bias(True),
+            lambda: pins.test_dense_one_hot_rows_give_weight_column_plus_bias(False),
+            pins.test_dense_on_grid_reduces_to_library_product_plus_bias,
+            pins.test_dense_number_bias_equals_constant_tensor]
+
+
+@pytest.mark.parametrize("name", sorted(_dense_mutants()))
+def test_dense_pins_catch_mutant(name, monkeypatch):
+    monkeypatch.setattr(oracle, "quantized_dense", _dense_mutants()[name])
+    caught = 0
+    for call in _dense_pin_calls():
+        try:
+            call()
+        except (AssertionError, ValueError, RuntimeError, IndexError):
+            caught += 1
+    assert caught, f"no pin caught dense mutant {name}"
+
+
+def test_unmutated_dense_passes_its_pins():
+    for call in _dense_pin_calls():
         call()

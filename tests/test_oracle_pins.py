@@ -55,6 +55,9 @@ def test_quantized_dense_doctest_shape():
     wq, s, b = oracle.quantize(w, d["group_size"], d["bits"])
     y = oracle.quantized_matmul(x, wq, s, b, d["transpose"], d["group_size"], d["bits"])
     assert list(y.shape) == g["expect"]["y_shape"]
+    # The doctest calls quantized_dense with its default bias (0): the same product.
+    yd = oracle.quantized_dense(x, wq, s, b, 0, d["transpose"], d["group_size"], d["bits"])
+    assert list(yd.shape) == g["expect"]["y_shape"] and torch.equal(yd, y)
 
 
 @pytest.mark.parametrize("bits", [2, 4, 8])
@@ -312,3 +315,58 @@ def test_gather_defaults_broadcast():
     y = oracle.gather_qmm(x2, wq, s, b, None, None, True, 64, 4)
     for i in range(2):
         assert torch.allclose(y[i], x2[i].double() @ deq[i].T, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# quantized_dense (Emily.Quantization.Layers): x @ W (+ bias), the bias a tensor
+# over the output features or a number.  Catches a dropped bias, a bias
+# broadcast along the rows instead of the features, a bias scaled or added
+# twice, the number form ignored.
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("transpose", [True, False])
+def test_dense_one_hot_rows_give_weight_column_plus_bias(transpose):
+    # transpose=True: W stored [out=16, in=64]; False: W stored [in=64, out=32]
+    # (quantized along out, one group of 32).
+    if transpose:
+        w = wl.normal((16, 64), 93, 1.0, torch.float32)
+        wq, s, b = oracle.quantize(w, 64, 4)
+        col = lambda j: oracle.dequantize(wq, s, b, 64, 4)[:, j]
+    else:
+        w = wl.normal((64, 32), 93, 1.0, torch.float32)       # out = 32, one group of 32
+        wq, s, b = oracle.quantize(w, 32, 4)
+        col = lambda j: oracle.dequantize(wq, s, b, 32, 4)[j, :]
+    n = 16 if transpose else 32
+    gs = 64 if transpose else 32
+    bias = torch.arange(n, dtype=torch.float32) * 0.25 - 1.0
+    x = torch.zeros((3, 64))
+    x[0, 0] = 1.0
+    x[1, 63] = 1.0
+    x[2, 17] = -2.0
+    y = oracle.quantized_dense(x, wq, s, b, bias, transpose, gs, 4)
+    assert y.shape == (3, n)
+    assert torch.equal(y[0], col(0).double() + bias.double())
+    assert torch.equal(y[1], col(63).double() + bias.double())
+    assert torch.equal(y[2], -2.0 * col(17).double() + bias.double())
+
+
+def test_dense_on_grid_reduces_to_library_product_plus_bias():
+    w, _, _, _ = _on_grid(48, 128, 32, 4, torch.float32, seed=95)   # [out=48, in=128]
+    wq, s, b = oracle.quantize(w, 32, 4)
+    x = wl.normal((5, 128), 96, 1.0, torch.float32)
+    bias = wl.normal((48,), 97, 1.0, torch.float32)
+    y = oracle.quantized_dense(x, wq, s, b, bias, True, 32, 4)
+    ref = torch.nn.functional.linear(x.double(), w.double(), bias.double())
+    assert torch.allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_dense_number_bias_equals_constant_tensor():
+    w = wl.normal((24, 64), 98, 1.0, torch.float32)
+    wq, s, b = oracle.quantize(w, 64, 4)
+    x = wl.normal((4, 64), 99, 1.0, torch.float32)
+    y_num = oracle.quantized_dense(x, wq, s, b, 0.75, True, 64, 4)
+    y_vec = oracle.quantized_dense(x, wq, s, b, torch.full((24,), 0.75), True, 64, 4)
+    y0 = oracle.quantized_dense(x, wq, s, b, 0, True, 64, 4)
+    assert torch.equal(y_num, y_vec)
+    assert torch.allclose(y_num - y0, torch.full((4, 24), 0.75, dtype=torch.float64),
+                          rtol=0, atol=1e-12)
