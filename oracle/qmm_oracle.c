@@ -24,8 +24,11 @@
  *    scale = (max - min) / (2^bits - 1)          (fp32, correctly rounded),
  *    s, b  = scale, bias rounded to the storage dtype (round-to-nearest-even),
  *    q     = s == 0 ? 0 : clamp(rint((w - b) / s), 0, 2^bits - 1)   (fp32),
- *    element j of a row sits at bit (j mod (32/bits)) * bits of word
- *    j / (32/bits)  (least-significant code first),
+ *    element j of a row occupies bits [j*bits, (j+1)*bits) of the row's
+ *    bit stream, bit i of the stream being bit (i mod 32) of word i / 32
+ *    (least-significant code first; for bits 2, 4, 8 that is bit
+ *    (j mod 32/bits) * bits of word j / (32/bits); 3- and 6-bit codes may
+ *    straddle two words),
  *    dequantized w = fmaf(s, q, b), then rounded to the storage dtype.
  *
  * Every floating-point step is a single IEEE operation in fp32 (build with
@@ -99,7 +102,7 @@ static int check_args(int dtype, int64_t rows, int64_t cols, int group_size, int
 {
     if (dtype != ORC_F32 && dtype != ORC_BF16 && dtype != ORC_F16)
         return ORC_BAD_ARG;
-    if (bits != 2 && bits != 4 && bits != 8)
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 6 && bits != 8)
         return ORC_BAD_ARG;
     if (group_size != 32 && group_size != 64 && group_size != 128)
         return ORC_BAD_ARG;
@@ -108,14 +111,18 @@ static int check_args(int dtype, int64_t rows, int64_t cols, int group_size, int
     return ORC_OK;
 }
 
-/* Store code q of element (r, c): element c of a row sits at bit
- * (c mod 32/bits) * bits of the row's word c / (32/bits), least significant
- * code first (words zeroed beforehand). */
+/* Store code q of element (r, c): bits [c*bits, (c+1)*bits) of row r's bit
+ * stream (words zeroed beforehand); the part past bit 31 of a word goes to
+ * the low bits of the next word. */
 static void put_code(uint32_t *wq, int64_t words_per_row, int bits, int64_t r, int64_t c,
                      uint32_t q)
 {
-    const int64_t per_word = 32 / bits;
-    wq[r * words_per_row + c / per_word] |= q << ((c % per_word) * bits);
+    const int64_t bit = c * bits;
+    const int off = (int)(bit % 32);
+    uint32_t *row = wq + r * words_per_row;
+    row[bit / 32] |= q << off;
+    if (off + bits > 32)
+        row[bit / 32 + 1] |= q >> (32 - off);
 }
 
 /*
@@ -130,8 +137,7 @@ int oracle_quantize(const void *w, int dtype, int64_t rows, int64_t cols,
     int rc = check_args(dtype, rows, cols, group_size, bits);
     if (rc != ORC_OK)
         return rc;
-    const int64_t per_word = 32 / bits;
-    const int64_t words_per_row = cols / per_word;
+    const int64_t words_per_row = cols * bits / 32;
     const int64_t groups_per_row = cols / group_size;
     const float qmax = (float)((1u << bits) - 1u);
 
@@ -174,13 +180,17 @@ int oracle_quantize(const void *w, int dtype, int64_t rows, int64_t cols,
     return ORC_OK;
 }
 
-/* The code of element (r, c) read back from the packed words. */
+/* The code of element (r, c) read back from the row's bit stream. */
 static uint32_t code_at(const uint32_t *wq, int64_t words_per_row, int bits,
                         int64_t r, int64_t c)
 {
-    const int64_t per_word = 32 / bits;
-    uint32_t word = wq[r * words_per_row + c / per_word];
-    return (word >> ((c % per_word) * bits)) & ((1u << bits) - 1u);
+    const int64_t bit = c * bits;
+    const int off = (int)(bit % 32);
+    const uint32_t *row = wq + r * words_per_row;
+    uint32_t v = row[bit / 32] >> off;
+    if (off + bits > 32)
+        v |= row[bit / 32 + 1] << (32 - off);
+    return v & ((1u << bits) - 1u);
 }
 
 /*
@@ -218,7 +228,7 @@ int oracle_dequantize(const uint32_t *wq, const void *scales, const void *biases
 int oracle_unpack_codes(const uint32_t *wq, int64_t rows, int64_t cols, int bits,
                         uint8_t *q)
 {
-    if (bits != 2 && bits != 4 && bits != 8)
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 6 && bits != 8)
         return ORC_BAD_ARG;
     const int64_t words_per_row = cols * bits / 32;
     for (int64_t r = 0; r < rows; ++r)
@@ -343,7 +353,8 @@ int oracle_encode_elements(int mode, const float *in, int64_t n, uint8_t *out)
 /* Value of a scale byte (E8M0 for mx modes, E4M3 for nvfp4). */
 static float mx_scale_value(int mode, uint32_t s)
 {
-    return mode == ORC_NVFP4 ? e4m3_value(s) : ldexpf(1.0f, (int)s - 127);
+    if (mode == ORC_NVFP4) return e4m3_value(s);
+    return s == 255u ? NAN : ldexpf(1.0f, (int)s - 127);   /* E8M0 0xFF is NaN */
 }
 
 int oracle_quantize_mx(const void *w, int dtype, int64_t rows, int64_t cols, int mode,

@@ -138,8 +138,8 @@ def _quantize_affine(w: torch.Tensor, group_size: int = 64, bits: int = 4):
     cols = w.shape[-1]
     rows = w.numel() // cols if cols else 0
     lead = tuple(w.shape[:-1])
-    if bits not in (2, 4, 8) or group_size not in (32, 64, 128) or cols % group_size:
-        raise ValueError("bits must be 2/4/8, group_size 32/64/128 dividing the last axis")
+    if bits not in (2, 3, 4, 6, 8) or group_size not in (32, 64, 128) or cols % group_size:
+        raise ValueError("bits must be 2/3/4/6/8, group_size 32/64/128 dividing the last axis")
     wq = torch.empty(lead + (cols * bits // 32,), dtype=torch.int32)
     scales = torch.empty(lead + (cols // group_size,), dtype=w.dtype)
     biases = torch.empty_like(scales)

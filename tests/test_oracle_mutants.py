@@ -20,8 +20,8 @@ import test_oracle_pins as pins
 SRC = Path(obuild.SRC).read_text()
 
 MUTANTS = {
-    "msb_first_packing": ("wq[r * words_per_row + c / per_word] |= q << ((c % per_word) * bits);",
-                          "wq[r * words_per_row + c / per_word] |= q << ((per_word - 1 - c % per_word) * bits);"),
+    "msb_first_packing": ("row[bit / 32] |= q << off;", "row[bit / 32] |= q << (32 - bits - off);"),
+    "straddle_dropped": ("row[bit / 32 + 1] |= q >> (32 - off);", "(void)0;"),
     "divisor_2_pow_bits": ("float scale32 = (hi - lo) / qmax;",
                            "float scale32 = (hi - lo) / (qmax + 1.0f);"),
     "floor_not_round": ("float t = rintf((v - b) / s);", "float t = floorf((v - b) / s);"),
@@ -32,8 +32,8 @@ MUTANTS = {
     "dequant_wrong_group": ("const int64_t sb = r * groups_per_row + c / group_size;",
                             "const int64_t sb = r * groups_per_row + (c / group_size) % 1;"),
     "truncating_bf16": ("u += 0x7fffu + keep_lsb;", "u += 0u;"),
-    "wrong_word_stride": ("uint32_t word = wq[r * words_per_row + c / per_word];",
-                          "uint32_t word = wq[r + c / per_word];"),
+    "wrong_word_stride": ("const uint32_t *row = wq + r * words_per_row;\n    uint32_t v",
+                          "const uint32_t *row = wq + r;\n    uint32_t v"),
     # microscaled modes
     "mx_emax_e2m1": ("const int emax = bits == 8 ? 8 : 2;", "const int emax = bits == 8 ? 8 : 3;"),
     "e8m0_bias": ("scode = (uint32_t)(shared + 127);", "scode = (uint32_t)(shared + 126);"),
@@ -58,10 +58,12 @@ def _pin_calls():
         pins.test_hand_packed_int8,
         pins.test_one_hot_rows_pick_weight_columns,
     ]
-    for bits in (2, 4, 8):
+    for bits in (2, 3, 4, 6, 8):
         calls.append(lambda bits=bits: pins.test_mlx_rs_quantize_dequantize_bound(bits))
         calls.append(lambda bits=bits: pins.test_code_is_nearest_grid_point(bits))
         calls.append(lambda bits=bits: pins.test_unpack_inverts_pack(bits))
+        if bits in (3, 6):
+            calls.append(lambda bits=bits: pins.test_hand_packed_straddling_codes(bits))
         for tr in (True, False):
             calls.append(lambda bits=bits, tr=tr: pins.test_matmul_reduces_to_dense_on_grid(bits, tr))
         for dt in pins.DTYPES:

@@ -16,7 +16,8 @@ from quantized_matmul_03_b200 import workloads as wl
 
 GOLDEN = json.loads((Path(__file__).parent / "golden" / "page_examples.json").read_text())
 DTYPES = [torch.float32, torch.bfloat16, torch.float16]
-QMAX = {2: 3, 4: 15, 8: 255}
+QMAX = {2: 3, 3: 7, 4: 15, 6: 63, 8: 255}
+ALL_BITS = [2, 3, 4, 6, 8]   # Emily.QuantizedWeight, from_dense: :bits one of [2, 3, 4, 6, 8]
 
 
 def u32(t: torch.Tensor):
@@ -60,7 +61,7 @@ def test_quantized_dense_doctest_shape():
     assert list(yd.shape) == g["expect"]["y_shape"] and torch.equal(yd, y)
 
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", ALL_BITS)
 @pytest.mark.parametrize("gs", [32, 64, 128])
 def test_packed_axis_shrinks_by_32_over_bits(bits, gs):
     w = wl.normal((3, 5, 256), 7, 1.0, torch.float32)
@@ -73,12 +74,12 @@ def test_packed_axis_shrinks_by_32_over_bits(bits, gs):
 # mlx-rs unit tests restated (bounds printed on the page).
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", ALL_BITS)
 def test_mlx_rs_quantize_dequantize_bound(bits):
     g = GOLDEN["mlx_rs_test_quantize_dequantize"]
     x = torch.arange(0, 512, dtype=torch.float32).expand(g["rows"], 512).contiguous()
     wq, s, b = oracle.quantize(x, g["group_size"], bits)
-    assert list(wq.shape) == [128, 512 // (32 // bits)]
+    assert list(wq.shape) == [128, 512 * bits // 32]   # = 512 / (32 / bits) for 2, 4, 8
     assert list(s.shape) == g["expect"]["scales_shape"]
     assert list(b.shape) == g["expect"]["biases_shape"]
     x_hat = oracle.dequantize(wq, s, b, g["group_size"], bits)
@@ -130,6 +131,33 @@ def test_hand_packed_int4():
     assert u32(wq) == [0x87654321, 0xEDCBA9F0, 0, 0, 0, 0, 0, 0]
 
 
+def _stream_words(codes, bits):
+    """Pack codes into uint32 words the long way: one Python integer holding
+    the whole row's bit stream (code j at bit j*bits), cut into 32-bit words
+    least significant first."""
+    v = 0
+    for j, c in enumerate(codes):
+        v |= int(c) << (j * bits)
+    n = len(codes) * bits // 32
+    return [(v >> (32 * i)) & 0xFFFFFFFF for i in range(n)]
+
+
+@pytest.mark.parametrize("bits", [3, 6])
+def test_hand_packed_straddling_codes(bits):
+    """3- and 6-bit codes (from_dense allows them) sit back to back in the
+    row's bit stream, so some straddle two words: 3-bit code 10 occupies bits
+    30..32, 6-bit code 5 bits 30..35."""
+    qmax = QMAX[bits]
+    codes = [(7 * j + 3) % (qmax + 1) for j in range(64)]
+    codes[0], codes[1] = 0, qmax          # the group's min and max are on the grid
+    codes[32], codes[33] = 0, qmax
+    w = torch.tensor([codes], dtype=torch.float32)   # scale 1, bias 0 per group
+    wq, s, b = oracle.quantize(w, 32, bits)
+    assert torch.equal(s, torch.ones((1, 2))) and torch.equal(b, torch.zeros((1, 2)))
+    assert u32(wq) == _stream_words(codes, bits)
+    assert oracle.unpack_codes(wq, bits).reshape(-1).tolist() == codes
+
+
 def test_hand_packed_int2():
     row = [1, 2, 3, 0, 3, 3, 0, 1, 2, 2, 2, 2, 0, 0, 0, 0] + [0] * 16
     w = torch.tensor([row], dtype=torch.float32)
@@ -146,17 +174,16 @@ def test_hand_packed_int8():
     assert u32(wq) == [0x44332211, 0x800700FF] + [0] * 6
 
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", ALL_BITS)
 def test_unpack_inverts_pack(bits):
     w = wl.normal((4, 128), 5, 1.0, torch.float32)
     wq, s, b = oracle.quantize(w, 32, bits)
     q = oracle.unpack_codes(wq, bits)
-    # Re-pack by plain integer arithmetic and compare the words.
-    per = 32 // bits
-    qi = q.to(torch.int64).reshape(4, 128 // per, per)
-    shifts = torch.arange(per, dtype=torch.int64) * bits
-    words = (qi << shifts).sum(-1)
-    assert u32(wq) == [int(v) & 0xFFFFFFFF for v in words.reshape(-1).tolist()]
+    # Re-pack each row as one bit stream (Python integers) and compare the words.
+    want = []
+    for r in range(4):
+        want += _stream_words(q[r].tolist(), bits)
+    assert u32(wq) == want
 
 
 # --------------------------------------------------------------------------
@@ -185,7 +212,7 @@ def _on_grid(rows, cols, gs, bits, dtype, seed):
 
 
 @pytest.mark.parametrize("dtype", DTYPES)
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", ALL_BITS)
 @pytest.mark.parametrize("gs", [32, 64, 128])
 def test_on_grid_round_trip_is_exact(dtype, bits, gs):
     w, q, s, b = _on_grid(6, 256, gs, bits, dtype, seed=bits * 1000 + gs)
@@ -202,7 +229,7 @@ def test_on_grid_round_trip_is_exact(dtype, bits, gs):
 # clamp, a sign error in (w - b).
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", ALL_BITS)
 def test_code_is_nearest_grid_point(bits):
     w = wl.normal((16, 64), 21 + bits, 3.0, torch.float32)
     wq, s, b = oracle.quantize(w, 32, bits)
@@ -230,7 +257,7 @@ def _ulp(t: torch.Tensor) -> torch.Tensor:
 
 
 @pytest.mark.parametrize("dtype", DTYPES)
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", ALL_BITS)
 def test_error_within_half_scale(dtype, bits):
     w = wl.with_outliers((32, 512), 31 + bits, 0.02, 0.01, 20.0, dtype)
     for gs in (32, 64, 128):
@@ -275,7 +302,7 @@ def test_dtype_rounding_matches_library(dtype):
 # wrong axis for transpose=False, a dropped bias term.
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("bits", ALL_BITS)
 @pytest.mark.parametrize("transpose", [True, False])
 def test_matmul_reduces_to_dense_on_grid(bits, transpose):
     w, _, _, _ = _on_grid(48, 128, 32, bits, torch.float32, seed=77 + bits)
