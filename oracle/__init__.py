@@ -18,6 +18,9 @@ Parity status per function (what pins it is in ``tests/test_oracle_pins.py``):
   quantized_dense     pinned: a zero bias gives quantized_matmul exactly; a
                       one-hot row gives a column of the dequantized weight plus
                       the bias; a constant-bias tensor equals the number form.
+  qqmm                pinned: the dequantized operands' library matmul on
+                      values already on both grids, exact in float64; a
+                      weight given dense equals the weight quantized first.
   gather_qmm          pinned: the two cases of mlx-rs ``test_gather_qmm``
                       against an independent indexed dense product.
 """
@@ -28,6 +31,7 @@ from .ref import (  # noqa: F401
     dequantize_f32,
     encode_elements,
     gather_qmm,
+    qqmm,
     quantize,
     quantized_dense,
     quantized_matmul,

@@ -248,6 +248,31 @@ def quantized_dense(x, wq, scales, biases, bias=0, transpose: bool = True,
     return y + float(bias)
 
 
+def qqmm(x, w, w_scales=None, group_size: int = 16, bits: int = 4, mode: str = "nvfp4"):
+    """float64 product with both operands quantized: ``Q(x) @ Q(W).T``.
+
+    mlx-rs ops/quantization.rs, ``qqmm``: ``x`` is quantized on the fly and
+    ``w`` is already quantized (``w`` packed, ``w_scales`` given) or is dense
+    (``w_scales`` None: quantized here); modes "nvfp4" (16, 4) and "mxfp8"
+    (32, 8).  Read as: W is stored [N, K] (the call has no transpose
+    argument), x is quantized along its last axis by the same rule as a
+    weight, no per-tensor global scales (the mlx-rs call passes empty ones),
+    and the product of the dequantized operands is taken in float64.
+    """
+    if mode not in ("nvfp4", "mxfp8"):
+        raise ValueError("qqmm supports modes nvfp4 and mxfp8")
+    _mx_mode(mode, group_size, bits)
+    x = _cpu(x)
+    if w_scales is None:
+        wq, ws, _ = quantize(w, group_size, bits, mode)
+    else:
+        wq, ws = w, w_scales
+    xq, xs, _ = quantize(x, group_size, bits, mode)
+    xd = dequantize_f32(xq, xs, None, group_size, bits, mode).double()
+    wd = dequantize_f32(wq, ws, None, group_size, bits, mode).double()
+    return xd @ wd.transpose(-1, -2)
+
+
 def gather_qmm(x, wq, scales, biases, lhs_indices=None, rhs_indices=None,
                transpose: bool = True, group_size: int = 64, bits: int = 4):
     """Mixture-of-experts quantized matmul, one batch entry at a time.

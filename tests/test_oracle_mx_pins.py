@@ -183,3 +183,62 @@ def test_matmul_uses_the_microscaled_weight():
         deq = oracle.dequantize(wq, s, None, gs, bits, mode, torch.float32).double()
         y = oracle.quantized_matmul(x, wq, s, None, True, gs, bits, mode)
         assert torch.allclose(y, x.double() @ deq.T, rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# qqmm (mlx-rs ops/quantization.rs): both operands quantized, nvfp4 / mxfp8.
+# --------------------------------------------------------------------------
+
+def _on_grid_rows(rows, cols, mode, seed):
+    """Rows whose every group is scale x element values with the group's
+    largest element at the format's top, so quantizing them is exact."""
+    gs, bits, _ = oracle.MX_MODES[mode]
+    g = torch.Generator().manual_seed(seed)
+    if bits == 4:
+        elems = torch.tensor(GOLD["e2m1_values"]["by_code"])
+        top = 6.0
+    else:
+        elems = torch.arange(256, dtype=torch.uint8)
+        elems = elems[(elems & 0x7F) != 0x7F].view(torch.float8_e4m3fn).float()
+        top = 448.0
+    pick = elems[torch.randint(0, elems.numel(), (rows, cols // gs, gs), generator=g)]
+    pick[:, :, 0] = top
+    lo, hi = (-6, 3) if mode == "nvfp4" else (-12, 4)
+    scale = torch.pow(2.0, torch.randint(lo, hi, (rows, cols // gs, 1), generator=g).float())
+    return (pick * scale).reshape(rows, cols)
+
+
+@pytest.mark.parametrize("mode", ["nvfp4", "mxfp8"])
+def test_qqmm_on_grid_is_the_exact_product(mode):
+    """Operands already on their grids quantize exactly, so qqmm is the plain
+    float64 product of the inputs (a library matmul)."""
+    x = _on_grid_rows(5, 128, mode, 11)
+    w = _on_grid_rows(24, 128, mode, 12)
+    gs, bits, _ = oracle.MX_MODES[mode]
+    y = oracle.qqmm(x, w, None, gs, bits, mode)
+    assert torch.equal(y, x.double() @ w.double().T)
+
+
+@pytest.mark.parametrize("mode", ["nvfp4", "mxfp8"])
+def test_qqmm_dense_weight_equals_prequantized(mode):
+    gs, bits, _ = oracle.MX_MODES[mode]
+    x = wl.normal((3, 256), 13, 1.0, torch.bfloat16)
+    w = wl.normal((40, 256), 14, 0.1, torch.bfloat16)
+    wq, ws, _ = oracle.quantize(w, gs, bits, mode)
+    assert torch.equal(oracle.qqmm(x, w, None, gs, bits, mode), oracle.qqmm(x, wq, ws, gs, bits, mode))
+
+
+def test_qqmm_quantizes_the_activations():
+    """Off-grid activations are rounded: the result differs from the product
+    with x kept exact, by no more than the activations' quantization error."""
+    gs, bits, _ = oracle.MX_MODES["mxfp8"]
+    x = wl.normal((4, 256), 15, 1.0, torch.float32)
+    w = _on_grid_rows(16, 256, "mxfp8", 16)
+    y = oracle.qqmm(x, w, None, gs, bits, "mxfp8")
+    exact = x.double() @ w.double().T
+    xq, xs, _ = oracle.quantize(x, gs, bits, "mxfp8")
+    xd = oracle.dequantize(xq, xs, None, gs, bits, "mxfp8", torch.float32).double()
+    assert not torch.equal(y, exact)
+    assert torch.allclose(y, xd @ w.double().T, rtol=1e-12, atol=1e-12)
+    bound = (xd - x.double()).abs() @ w.double().abs().T
+    assert ((y - exact).abs() <= bound + 1e-9).all()
