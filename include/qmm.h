@@ -26,17 +26,36 @@
  * Errors.  Arguments are validated before anything is launched; on any error
  *   nothing is enqueued.  Exceptions never cross the ABI.  A thread-local
  *   message for the last failure is available from qmm_last_error().
- * Packing.  bits in {2, 4, 8}; 32/bits codes per uint32 word, code j of a row
- *   at bit (j mod 32/bits)*bits of word j/(32/bits) (least significant first).
+ * Packing.  bits in {2, 3, 4, 6, 8} (Emily.QuantizedWeight, from_dense); a
+ *   row of cols codes takes cols*bits/32 uint32 words; code j of a row
+ *   occupies bits [j*bits, (j+1)*bits) of the row's bit stream, bit i of the
+ *   stream being bit (i mod 32) of word i/32 (least significant first).  For
+ *   2, 4 and 8 bits that is bit (j mod 32/bits)*bits of word j/(32/bits);
+ *   3- and 6-bit codes may straddle two words.
  * Groups.  group_size in {32, 64, 128}; one scale and one bias per group of
  *   consecutive elements along the LAST STORED axis of the weight (the packed
  *   axis), for both matmul layouts.
- * Dtypes.  scales and biases share the dense weight's dtype; outputs take the
- *   scales dtype (EMLX.Quantization, section quantized_matmul); activations
- *   must have that dtype too.
+ * Dtypes.  "affine": scales and biases share the dense weight's dtype;
+ *   outputs take the scales dtype (EMLX.Quantization, section
+ *   quantized_matmul); activations must have that dtype too.
  * Mode.  `mode` NULL means "affine" (the default in every document above).
- *   The microscaled modes of Emily.QuantizedWeight ("mxfp4", "mxfp8", "nvfp4") return
- *   QMM_ERR_UNSUPPORTED; any other string returns QMM_ERR_INVALID_ARG.
+ *   The microscaled modes of Emily.QuantizedWeight, section Microscaled modes,
+ *   fix group_size and bits and have no biases (pass NULL):
+ *     "mxfp4"  group_size 32, bits 4: E2M1 elements, one E8M0 scale byte per group
+ *     "mxfp8"  group_size 32, bits 8: E4M3 elements, one E8M0 scale byte per group
+ *     "nvfp4"  group_size 16, bits 4: E2M1 elements, one E4M3 scale byte per group
+ *   scales is then a uint8 array [rows, cols/group_size]; the `dtype`
+ *   argument names the dense weight's dtype for qmm_quantize, the output's
+ *   for qmm_dequantize, and the activations' (= output's) for the matmuls
+ *   (EMLX.Quantization, section gather_quantized_matmul: with u8 scales the
+ *   output follows the activations).  Quantize rule: mx modes X =
+ *   2^(floor(log2 max|v|) - emax), emax 2 (E2M1) or 8 (E4M3), clamped to
+ *   E8M0's range (OCP Microscaling Formats v1.0); nvfp4 X = max|v|/6 rounded
+ *   to E4M3; elements v/X rounded to nearest-even and saturated; an
+ *   all-zero group stores zeros; dequantized w = X * element.  A group size or
+ *   bits other than the mode's, or non-NULL biases, is QMM_ERR_INVALID_ARG.
+ *   gather_qmm takes "affine" weights only (QMM_ERR_UNSUPPORTED otherwise).
+ *   Any other mode string returns QMM_ERR_INVALID_ARG.
  */
 #ifndef QMM_H
 #define QMM_H
@@ -51,7 +70,7 @@ extern "C" {
 typedef enum {
     QMM_OK = 0,
     QMM_ERR_INVALID_ARG = 1, /* bad size, pointer, group size, bits, ... */
-    QMM_ERR_UNSUPPORTED = 2, /* documented upstream but not built (e.g. mxfp4) */
+    QMM_ERR_UNSUPPORTED = 2, /* valid, but not for this entry or forced path */
     QMM_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
     QMM_ERR_TIMEOUT = 4,     /* a kernel's bounded wait ran out (device word) */
     QMM_ERR_INDEX = 5,       /* an expert / row index was out of range */
@@ -67,20 +86,24 @@ typedef enum { QMM_F32 = 0, QMM_BF16 = 1, QMM_F16 = 2 } qmm_dtype;
  *   wq      out: [rows, cols*bits/32] uint32 packed codes
  *   scales  out: [rows, cols/group_size], dtype `dtype`
  *   biases  out: [rows, cols/group_size], dtype `dtype`
- * Rule: bias = group min, scale = (max - min)/(2^bits - 1) in fp32, both
- * rounded to `dtype` (nearest-even); q = clamp(rint((w - bias)/scale), 0,
- * 2^bits - 1) against the stored scale and bias, 0 when the scale is 0.
- * cols must be a positive multiple of group_size; rows may be 0 (no-op).
+ * Rule ("affine"): bias = group min, scale = (max - min)/(2^bits - 1) in
+ * fp32, both rounded to `dtype` (nearest-even); q = clamp(rint((w - bias) /
+ * scale), 0, 2^bits - 1) against the stored scale and bias, 0 when the scale
+ * is 0.  Microscaled modes: see the header's Mode paragraph (scales uint8,
+ * biases NULL).  cols must be a positive multiple of group_size; rows may be
+ * 0 (no-op).
  */
 qmm_status qmm_quantize(const void *w, qmm_dtype dtype, int64_t rows, int64_t cols,
                         int group_size, int bits, const char *mode,
                         uint32_t *wq, void *scales, void *biases, void *stream);
 
 /*
- * qmm_dequantize -- EMLX.Quantization, section dequantize; mlx-rs dequantize.
- *   out[r, c] = round_to_dtype(fmaf(scale[r, c/gs], q[r, c], bias[r, c/gs]))
+ * qmm_dequantize -- EMLX.Quantization, section dequantize (every mode);
+ * mlx-rs dequantize.
+ *   "affine": out[r, c] = round_to_dtype(fmaf(scale[r, c/gs], q[r, c], bias[r, c/gs]))
  *   wq [rows, cols*bits/32], scales/biases [rows, cols/gs], out [rows, cols],
- *   all in `dtype` except wq.
+ *   all in `dtype` except wq.  Microscaled modes: out = round_to_dtype(X *
+ *   element), scales uint8, biases NULL, `dtype` the output's.
  */
 qmm_status qmm_dequantize(const uint32_t *wq, const void *scales, const void *biases,
                           qmm_dtype dtype, int64_t rows, int64_t cols, int group_size,
@@ -141,6 +164,54 @@ qmm_status qmm_quantized_matmul_ws(const void *x, int64_t M, int64_t K,
                                    int group_size, int bits, const char *mode,
                                    void *y, void *workspace, size_t workspace_bytes,
                                    void *stream);
+
+/*
+ * qmm_quantized_dense -- Emily.Quantization.Layers, quantized_dense: the
+ * dense-layer form x @ W (+ bias) on a quantized weight, in either layout.
+ * The page lets the bias be a tensor or a number; here both are taken and
+ * added together:
+ *   y[m, n] = round_to_dtype( sum_k x[m, k] W~[k, n] + bias[n] + bias_value )
+ * with the product exactly as qmm_quantized_matmul computes it (same paths,
+ * layouts, sizes and errors) and the bias added in fp32 in the product's
+ * epilogue, before the single rounding of the output (no second pass over y).
+ *   bias        NULL, or a device array of N values in `dtype` (one per output
+ *               feature, broadcast over the rows of x), aligned to its element
+ *               size;
+ *   bias_value  a number added to every output (0 for none); must be finite.
+ *   workspace, workspace_bytes  as for qmm_quantized_matmul_ws (may be NULL/0).
+ * With bias == NULL and bias_value == 0 the result is qmm_quantized_matmul's.
+ */
+qmm_status qmm_quantized_dense(const void *x, int64_t M, int64_t K,
+                               const uint32_t *wq, const void *scales, const void *biases,
+                               qmm_dtype dtype, int64_t N, int transpose,
+                               int group_size, int bits, const char *mode,
+                               const void *bias, double bias_value,
+                               void *y, void *workspace, size_t workspace_bytes,
+                               void *stream);
+
+/*
+ * qmm_qqmm -- mlx-rs ops/quantization.rs, qqmm: the product with BOTH operands
+ * quantized, y = Q(x) @ Q(W)^T, in mode "nvfp4" (group_size 16, bits 4) or
+ * "mxfp8" (32, 8).  The activations are quantized on the fly along K by the
+ * same rule as a weight (see Mode above); the weight is already quantized:
+ *   x [M, K] in `dtype`; wq [N, K*bits/32], w_scales [N, K/gs] uint8 (as
+ *   qmm_quantize writes them in that mode); y [M, N] in `dtype`.
+ * The call has no transpose argument: W is stored [N, K].  No per-tensor
+ * global scales (the mlx-rs call passes none).  The product of the two
+ * dequantized operands is formed in fp32 (every element value and scale is
+ * exact in 16 bits, so the operands are exact).
+ *   workspace: device memory of qmm_qqmm_workspace_size(M, K, group_size,
+ *     bits, dtype) bytes, 256-byte aligned, for the quantized activations (its
+ *     contents need not be initialised); two calls in flight must not share
+ *     one.  Too small or misaligned: QMM_ERR_WORKSPACE.
+ * Other modes: QMM_ERR_UNSUPPORTED.  Three kernels per call (quantize x,
+ * dequantize x, product).
+ */
+size_t qmm_qqmm_workspace_size(int64_t M, int64_t K, int group_size, int bits, qmm_dtype dtype);
+qmm_status qmm_qqmm(const void *x, int64_t M, int64_t K, qmm_dtype dtype,
+                    const uint32_t *wq, const void *w_scales, int64_t N,
+                    int group_size, int bits, const char *mode,
+                    void *y, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * qmm_gather_qmm -- EMLX.Quantization, section gather_quantized_matmul;
@@ -259,10 +330,18 @@ qmm_status qmm_inject_fault(qmm_fault fault);
 /*
  * Kernel-path selection for qmm_quantized_matmul (process-wide; the default
  * is QMM_PATH_AUTO).  QMM_PATH_GEMV forces the SIMT decode kernels (M <= 16
- * rows at a time), QMM_PATH_GEMM the tensor-core (tcgen05) kernel.  A forced
- * path that cannot run a given call returns QMM_ERR_UNSUPPORTED.
+ * rows at a time), QMM_PATH_GEMM the tensor-core (tcgen05) GEMM, and
+ * QMM_PATH_DECODE_TC the decode tensor-core kernel (bf16/f16, transpose,
+ * 1..16 rows, 2- or 4-bit codes, K % 512 == 0, (K / group_size) % 8 == 0;
+ * only when forced: AUTO keeps the faster SIMT decode kernel and GEMM).  A
+ * forced path that cannot run a given call returns QMM_ERR_UNSUPPORTED.
  */
-typedef enum { QMM_PATH_AUTO = 0, QMM_PATH_GEMV = 1, QMM_PATH_GEMM = 2 } qmm_path;
+typedef enum {
+    QMM_PATH_AUTO = 0,
+    QMM_PATH_GEMV = 1,
+    QMM_PATH_GEMM = 2,
+    QMM_PATH_DECODE_TC = 3
+} qmm_path;
 qmm_status qmm_set_path(qmm_path path);
 
 /*

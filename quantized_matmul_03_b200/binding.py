@@ -20,7 +20,7 @@ QMM_OK = 0
 STATUS_NAMES = {0: "QMM_OK", 1: "QMM_ERR_INVALID_ARG", 2: "QMM_ERR_UNSUPPORTED",
                 3: "QMM_ERR_CUDA", 4: "QMM_ERR_TIMEOUT", 5: "QMM_ERR_INDEX",
                 6: "QMM_ERR_WORKSPACE"}
-PATHS = {"auto": 0, "gemv": 1, "gemm": 2}
+PATHS = {"auto": 0, "gemv": 1, "gemm": 2, "decode_tc": 3}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 
 _lib = None
@@ -50,6 +50,9 @@ def lib() -> ctypes.CDLL:
                                      vp, vp],
             "qmm_quantized_matmul_ws": [vp, i64, i64, vp, vp, vp, i32, i64, i32, i32, i32, cp,
                                         vp, vp, sz, vp],
+            "qmm_quantized_dense": [vp, i64, i64, vp, vp, vp, i32, i64, i32, i32, i32, cp,
+                                    vp, ctypes.c_double, vp, vp, sz, vp],
+            "qmm_qqmm": [vp, i64, i64, i32, vp, vp, i64, i32, i32, cp, vp, vp, sz, vp],
             "qmm_gather_qmm": [vp, i64, i64, i64, vp, vp, vp, i32, i64, i64, vp, vp, i64, i32,
                                i32, i32, cp, i32, vp, vp, sz, vp],
             "qmm_gather_qmm_static": [vp, i64, i64, i64, vp, vp, vp, i32, i64, i64, vp, vp, i64,
@@ -63,6 +66,8 @@ def lib() -> ctypes.CDLL:
             f = getattr(L, name)
             f.argtypes = args
             f.restype = ctypes.c_int
+        L.qmm_qqmm_workspace_size.argtypes = [i64, i64, i32, i32, i32]
+        L.qmm_qqmm_workspace_size.restype = sz
         L.qmm_gather_qmm_workspace_size.argtypes = [i64, i64, i64, i64, i32]
         L.qmm_gather_qmm_workspace_size.restype = sz
         L.qmm_quantized_matmul_workspace_size.argtypes = [i64, i64, i64, i32, i32, i32]
@@ -109,37 +114,47 @@ def _dtype(t: torch.Tensor) -> int:
     return DTYPES[t.dtype]
 
 
+# The microscaled modes (Emily.QuantizedWeight, section Microscaled modes):
+# fixed (group_size, bits), one scale byte per group, no biases.
+MX_MODES = {"mxfp4": (32, 4), "mxfp8": (32, 8), "nvfp4": (16, 4)}
+
+
 def qmm_quantize(w: torch.Tensor, group_size: int = 64, bits: int = 4, mode: str = "affine",
                  out=None):
     """Quantize ``w`` (rank >= 2) along its last axis -> (wq, scales, biases).
 
-    ``wq`` is int32 holding the uint32 words; scales/biases take ``w``'s dtype.
+    ``wq`` is int32 holding the uint32 words; scales/biases take ``w``'s dtype
+    ("affine"); in a microscaled mode scales are uint8 and biases is None.
     ``out``: optional ``(wq, scales, biases)`` tensors to write into.
     """
     _cuda(w)
     cols = w.shape[-1]
     rows = w.numel() // cols if cols else 0
     lead = tuple(w.shape[:-1])
+    micro = mode in MX_MODES
     if out is not None:
         wq, scales, biases = out
         _cuda(wq, scales, biases)
     else:
         wq = torch.empty(lead + (cols * bits // 32,), dtype=torch.int32, device=w.device)
-        scales = torch.empty(lead + (max(cols // group_size, 0),), dtype=w.dtype, device=w.device)
-        biases = torch.empty_like(scales)
+        scales = torch.empty(lead + (max(cols // group_size, 0),),
+                             dtype=torch.uint8 if micro else w.dtype, device=w.device)
+        biases = None if micro else torch.empty_like(scales)
     _check(lib().qmm_quantize(_p(w), _dtype(w), rows, cols, group_size, bits, _mode(mode),
                               _p(wq), _p(scales), _p(biases), _stream(w.device)))
     return wq, scales, biases
 
 
 def qmm_dequantize(wq, scales, biases, group_size: int = 64, bits: int = 4,
-                   mode: str = "affine"):
-    """Dense weight ``scale * q + bias`` in the scales dtype."""
+                   mode: str = "affine", dtype=torch.bfloat16):
+    """Dense weight ``scale * q + bias`` in the scales dtype; in a microscaled
+    mode ``X * element`` in ``dtype``."""
     _cuda(wq, scales, biases)
     cols = wq.shape[-1] * 32 // bits
     rows = wq.numel() // wq.shape[-1] if wq.shape[-1] else 0
-    out = torch.empty(tuple(wq.shape[:-1]) + (cols,), dtype=scales.dtype, device=wq.device)
-    _check(lib().qmm_dequantize(_p(wq), _p(scales), _p(biases), _dtype(scales), rows, cols,
+    odt = dtype if mode in MX_MODES else scales.dtype
+    out = torch.empty(tuple(wq.shape[:-1]) + (cols,), dtype=odt, device=wq.device)
+    _check(lib().qmm_dequantize(_p(wq), _p(scales), _p(biases), _dtype(out), rows, cols,
                                 group_size, bits, _mode(mode), _p(out), _stream(wq.device)))
     return out
 
@@ -187,24 +202,99 @@ def qmm_quantized_matmul(x, wq, scales, biases, transpose: bool = True, group_si
         N = wq.shape[-2]
     else:
         N = wq.shape[-1] * 32 // bits
+    # (affine: the output takes the scales dtype; microscaled: the activations')
+    odt = x.dtype if mode in MX_MODES else scales.dtype
     if out is None:
-        out = torch.empty(tuple(x.shape[:-1]) + (N,), dtype=scales.dtype, device=x.device)
+        out = torch.empty(tuple(x.shape[:-1]) + (N,), dtype=odt, device=x.device)
     ws = None
     if isinstance(workspace, str):
         if workspace != "auto":
             raise ValueError("workspace must be 'auto', None or a tensor")
-        if scales.dtype in DTYPES:
-            need = qmm_quantized_matmul_workspace_size(M, K, N, transpose, bits, scales.dtype)
+        if odt in DTYPES and mode not in MX_MODES:
+            need = qmm_quantized_matmul_workspace_size(M, K, N, transpose, bits, odt)
             if need > 0:
                 ws = _matmul_workspace(x.device, need)
     elif workspace is not None:
         _cuda(workspace)
         ws = workspace
     _check(lib().qmm_quantized_matmul_ws(_p(x), M, K, _p(wq), _p(scales), _p(biases),
-                                         _dtype(scales), N, int(bool(transpose)), group_size, bits,
+                                         _dtype(out), N, int(bool(transpose)), group_size, bits,
                                          _mode(mode), _p(out), _p(ws),
                                          ws.numel() * ws.element_size() if ws is not None else 0,
                                          _stream(x.device)))
+    return out
+
+
+def qmm_quantized_dense(x, wq, scales, biases, bias=0, transpose: bool = True,
+                        group_size: int = 64, bits: int = 4, mode: str = "affine",
+                        out: Optional[torch.Tensor] = None, workspace="auto"):
+    """Dense layer ``x @ W (+ bias)`` on a quantized weight (Emily.Quantization.Layers,
+    ``quantized_dense``): ``bias`` is a number, or a tensor of the output
+    features' length in the scales dtype, or a tensor of one element (taken as
+    a number).  The bias is added inside the product before rounding."""
+    _cuda(x, wq, scales, biases, out)
+    K = x.shape[-1]
+    M = x.numel() // K if K else 0
+    N = wq.shape[-2] if transpose else wq.shape[-1] * 32 // bits
+    odt = x.dtype if mode in MX_MODES else scales.dtype
+    bias_t, bias_v = None, 0.0
+    if isinstance(bias, torch.Tensor):
+        if bias.numel() == 1:
+            bias_v = float(bias.reshape(()).item())
+        else:
+            if bias.numel() != N or bias.dtype != odt:
+                raise ValueError(f"bias must hold {N} values of dtype {odt}")
+            bias_t = bias.reshape(-1)
+            _cuda(bias_t)
+    else:
+        bias_v = float(bias)
+    if out is None:
+        out = torch.empty(tuple(x.shape[:-1]) + (N,), dtype=odt, device=x.device)
+    ws = None
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError("workspace must be 'auto', None or a tensor")
+        need = 0 if mode in MX_MODES else qmm_quantized_matmul_workspace_size(
+            M, K, N, transpose, bits, odt)
+        if need > 0:
+            ws = _matmul_workspace(x.device, need)
+    elif workspace is not None:
+        _cuda(workspace)
+        ws = workspace
+    _check(lib().qmm_quantized_dense(_p(x), M, K, _p(wq), _p(scales), _p(biases),
+                                     _dtype(out), N, int(bool(transpose)), group_size, bits,
+                                     _mode(mode), _p(bias_t), bias_v, _p(out), _p(ws),
+                                     ws.numel() * ws.element_size() if ws is not None else 0,
+                                     _stream(x.device)))
+    return out
+
+
+def qmm_qqmm(x, w, w_scales=None, group_size: Optional[int] = None, bits: Optional[int] = None,
+             mode: str = "nvfp4", out: Optional[torch.Tensor] = None,
+             workspace: Optional[torch.Tensor] = None):
+    """mlx-rs ``qqmm``: ``Q(x) @ Q(W).T`` with x quantized on the fly; ``w`` is
+    the packed weight with ``w_scales``, or a dense weight (quantized first
+    when ``w_scales`` is None).  Modes "nvfp4" (default) and "mxfp8"; group
+    size and bits default to the mode's."""
+    if mode not in ("nvfp4", "mxfp8"):
+        raise ValueError("qqmm supports modes nvfp4 and mxfp8")
+    gs_d, bits_d = MX_MODES[mode]
+    group_size = gs_d if group_size is None else group_size
+    bits = bits_d if bits is None else bits
+    if w_scales is None:
+        w, w_scales, _ = qmm_quantize(w, group_size, bits, mode)
+    _cuda(x, w, w_scales, out, workspace)
+    K = x.shape[-1]
+    M = x.numel() // K if K else 0
+    N = w.shape[-2]
+    if out is None:
+        out = torch.empty(tuple(x.shape[:-1]) + (N,), dtype=x.dtype, device=x.device)
+    need = int(lib().qmm_qqmm_workspace_size(M, K, group_size, bits, _dtype(x)))
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().qmm_qqmm(_p(x), M, K, _dtype(x), _p(w), _p(w_scales), N, group_size, bits,
+                          _mode(mode), _p(out), _p(workspace), ws_bytes, _stream(x.device)))
     return out
 
 

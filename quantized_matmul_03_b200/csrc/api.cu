@@ -6,6 +6,7 @@
 // arguments and raises before any MLX call), and never lets a C++ exception
 // cross the ABI.
 #include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -42,25 +43,36 @@ qmm_status cuda_fail(cudaError_t e, const char *what) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Mode strings: "affine" (default), and the microscaled modes
-// that carry fixed group sizes and no biases (Emily.QuantizedWeight, section
+// Mode strings: "affine" (default), and the microscaled modes, which carry a
+// fixed group size and bits and no biases (Emily.QuantizedWeight, section
 // Microscaled modes).
-qmm_status check_mode(const char *mode) {
+qmm_status parse_mode(const char *mode, int *out) {
+    *out = QMM_MODE_AFFINE;
     if (mode == nullptr || std::strcmp(mode, "affine") == 0) return QMM_OK;
-    if (!std::strcmp(mode, "mxfp4") || !std::strcmp(mode, "mxfp8") || !std::strcmp(mode, "nvfp4"))
-        return fail(QMM_ERR_UNSUPPORTED, "mode \"%s\" is not built (affine only)", mode);
-    return fail(QMM_ERR_INVALID_ARG, "unknown quantization mode \"%s\"", mode);
+    if (!std::strcmp(mode, "mxfp4")) *out = QMM_MODE_MXFP4;
+    else if (!std::strcmp(mode, "mxfp8")) *out = QMM_MODE_MXFP8;
+    else if (!std::strcmp(mode, "nvfp4")) *out = QMM_MODE_NVFP4;
+    else return fail(QMM_ERR_INVALID_ARG, "unknown quantization mode \"%s\"", mode);
+    return QMM_OK;
 }
 
-qmm_status check_common(qmm_dtype dt, int group_size, int bits, const char *mode) {
-    qmm_status st = check_mode(mode);
+qmm_status check_common(qmm_dtype dt, int group_size, int bits, const char *mode,
+                        int *mode_out = nullptr) {
+    int m = QMM_MODE_AFFINE;
+    qmm_status st = parse_mode(mode, &m);
     if (st != QMM_OK) return st;
+    if (mode_out) *mode_out = m;
     if (dt != QMM_F32 && dt != QMM_BF16 && dt != QMM_F16)
         return fail(QMM_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
-    if (bits == 3 || bits == 6)
-        return fail(QMM_ERR_UNSUPPORTED, "bits=%d is not built (2, 4, 8 only)", bits);
-    if (bits != 2 && bits != 4 && bits != 8)
-        return fail(QMM_ERR_INVALID_ARG, "bits must be 2, 4 or 8 (got %d)", bits);
+    if (m != QMM_MODE_AFFINE) {
+        const int gs = m == QMM_MODE_NVFP4 ? 16 : 32, b = m == QMM_MODE_MXFP8 ? 8 : 4;
+        if (group_size != gs || bits != b)
+            return fail(QMM_ERR_INVALID_ARG, "mode \"%s\" needs group_size=%d and bits=%d (got %d, %d)",
+                        mode, gs, b, group_size, bits);
+        return QMM_OK;
+    }
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 6 && bits != 8)
+        return fail(QMM_ERR_INVALID_ARG, "bits must be 2, 3, 4, 6 or 8 (got %d)", bits);
     if (group_size != 32 && group_size != 64 && group_size != 128)
         return fail(QMM_ERR_INVALID_ARG, "group_size must be 32, 64 or 128 (got %d)", group_size);
     return QMM_OK;
@@ -74,7 +86,7 @@ qmm_status check_common(qmm_dtype dt, int group_size, int bits, const char *mode
 
 qmm_status check_matmul(const void *x, int64_t M, int64_t K, const uint32_t *wq,
                         const void *scales, const void *biases, int64_t N, int transpose,
-                        int group_size, void *y) {
+                        int group_size, void *y, int mode = QMM_MODE_AFFINE) {
     if (M < 0 || N < 0 || K <= 0)
         return fail(QMM_ERR_INVALID_ARG, "sizes must satisfy M >= 0, N >= 0, K > 0");
     const int64_t packed_axis = transpose ? K : N;
@@ -86,9 +98,14 @@ qmm_status check_matmul(const void *x, int64_t M, int64_t K, const uint32_t *wq,
     QMM_CHECK_PTR(x, "x");
     QMM_CHECK_PTR(wq, "wq");
     QMM_CHECK_PTR(scales, "scales");
-    if (biases == nullptr)
-        return fail(QMM_ERR_INVALID_ARG, "biases is NULL (required for mode \"affine\")");
-    QMM_CHECK_PTR(biases, "biases");
+    if (mode != QMM_MODE_AFFINE) {
+        if (biases != nullptr)
+            return fail(QMM_ERR_INVALID_ARG, "biases must be NULL in a microscaled mode");
+    } else {
+        if (biases == nullptr)
+            return fail(QMM_ERR_INVALID_ARG, "biases is NULL (required for mode \"affine\")");
+        QMM_CHECK_PTR(biases, "biases");
+    }
     QMM_CHECK_PTR(y, "y");
     return QMM_OK;
 }
@@ -114,6 +131,12 @@ qmm_status finish_launch(cudaError_t e, const char *what) {
 }
 
 }  // namespace
+
+// Products with microscaled weights: the SIMT kernels (any shape, either
+// layout; the gather entry takes affine weights only).
+cudaError_t launch_mx_matmul(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
+    return launch_gemv(dt, a, s);
+}
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
@@ -163,7 +186,8 @@ qmm_status qmm_quantize(const void *w, qmm_dtype dtype, int64_t rows, int64_t co
                         int group_size, int bits, const char *mode, uint32_t *wq, void *scales,
                         void *biases, void *stream) {
     try {
-        qmm_status st = check_common(dtype, group_size, bits, mode);
+        int md = QMM_MODE_AFFINE;
+        qmm_status st = check_common(dtype, group_size, bits, mode, &md);
         if (st != QMM_OK) return st;
         if (rows < 0 || cols <= 0 || cols % group_size != 0)
             return fail(QMM_ERR_INVALID_ARG,
@@ -172,6 +196,12 @@ qmm_status qmm_quantize(const void *w, qmm_dtype dtype, int64_t rows, int64_t co
         QMM_CHECK_PTR(w, "w");
         QMM_CHECK_PTR(wq, "wq");
         QMM_CHECK_PTR(scales, "scales");
+        if (md != QMM_MODE_AFFINE) {
+            if (biases != nullptr)
+                return fail(QMM_ERR_INVALID_ARG, "biases must be NULL in a microscaled mode");
+            QuantArgs a{w, rows, cols, group_size, bits, wq, scales, nullptr, md};
+            return finish_launch(launch_quantize_mx(dtype, a, (cudaStream_t)stream), "quantize launch");
+        }
         QMM_CHECK_PTR(biases, "biases");
         QuantArgs a{w, rows, cols, group_size, bits, wq, scales, biases};
         return finish_launch(launch_quantize(dtype, a, (cudaStream_t)stream), "quantize launch");
@@ -184,7 +214,8 @@ qmm_status qmm_dequantize(const uint32_t *wq, const void *scales, const void *bi
                           qmm_dtype dtype, int64_t rows, int64_t cols, int group_size, int bits,
                           const char *mode, void *out, void *stream) {
     try {
-        qmm_status st = check_common(dtype, group_size, bits, mode);
+        int md = QMM_MODE_AFFINE;
+        qmm_status st = check_common(dtype, group_size, bits, mode, &md);
         if (st != QMM_OK) return st;
         if (rows < 0 || cols <= 0 || cols % group_size != 0)
             return fail(QMM_ERR_INVALID_ARG,
@@ -192,6 +223,14 @@ qmm_status qmm_dequantize(const uint32_t *wq, const void *scales, const void *bi
         if (rows == 0) return QMM_OK;
         QMM_CHECK_PTR(wq, "wq");
         QMM_CHECK_PTR(scales, "scales");
+        if (md != QMM_MODE_AFFINE) {
+            if (biases != nullptr)
+                return fail(QMM_ERR_INVALID_ARG, "biases must be NULL in a microscaled mode");
+            QMM_CHECK_PTR(out, "out");
+            DequantArgs a{wq, scales, nullptr, rows, cols, group_size, bits, out, md};
+            return finish_launch(launch_dequantize_mx(dtype, a, (cudaStream_t)stream),
+                                 "dequantize launch");
+        }
         if (biases == nullptr)
             return fail(QMM_ERR_INVALID_ARG, "biases is NULL (required for mode \"affine\")");
         QMM_CHECK_PTR(biases, "biases");
@@ -204,23 +243,41 @@ qmm_status qmm_dequantize(const uint32_t *wq, const void *scales, const void *bi
     }
 }
 
-qmm_status qmm_quantized_matmul_ws(const void *x, int64_t M, int64_t K, const uint32_t *wq,
-                                   const void *scales, const void *biases, qmm_dtype dtype,
-                                   int64_t N, int transpose, int group_size, int bits,
-                                   const char *mode, void *y, void *workspace,
-                                   size_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// quantized_matmul with an optional layer bias (quantized_dense) and an
+// optional stream-K workspace: the implementation of the three entry points.
+qmm_status matmul_impl(const void *x, int64_t M, int64_t K, const uint32_t *wq, const void *scales,
+                       const void *biases, qmm_dtype dtype, int64_t N, int transpose, int group_size,
+                       int bits, const char *mode, const void *bias, double bias_value, void *y,
+                       void *workspace, size_t workspace_bytes, void *stream) {
     try {
-        qmm_status st = check_common(dtype, group_size, bits, mode);
+        int md = QMM_MODE_AFFINE;
+        qmm_status st = check_common(dtype, group_size, bits, mode, &md);
         if (st != QMM_OK) return st;
-        st = check_matmul(x, M, K, wq, scales, biases, N, transpose, group_size, y);
+        st = check_matmul(x, M, K, wq, scales, biases, N, transpose, group_size, y, md);
         if (st != QMM_OK) return st;
         if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255) != 0)
             return fail(QMM_ERR_WORKSPACE, "workspace must be 256-byte aligned");
         if (M == 0 || N == 0) return QMM_OK;
+        if (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) & (dtype == QMM_F32 ? 3u : 1u)))
+            return fail(QMM_ERR_INVALID_ARG, "bias is not aligned to its element size");
+        if (!std::isfinite(bias_value))
+            return fail(QMM_ERR_INVALID_ARG, "bias_value must be finite");
         QmmArgs a{x, wq, scales, biases, y, M, N, K, group_size, bits, transpose != 0};
+        a.mode = md;
+        a.bias = bias;
+        a.bias_value = (float)bias_value;
         a.ws = workspace;
         a.ws_bytes = workspace ? workspace_bytes : 0;
         cudaStream_t s = (cudaStream_t)stream;
+        if (md != QMM_MODE_AFFINE) {
+            if (g_path == QMM_PATH_GEMM || g_path == QMM_PATH_DECODE_TC)
+                return fail(QMM_ERR_UNSUPPORTED, "the forced path does not take microscaled weights");
+            return finish_launch(launch_mx_matmul(dtype, a, s), "microscaled matmul launch");
+        }
         const bool tc_ok = gemm_supported(dtype, a);
         if (g_path == QMM_PATH_GEMM) {
             if (!tc_ok)
@@ -229,9 +286,18 @@ qmm_status qmm_quantized_matmul_ws(const void *x, int64_t M, int64_t K, const ui
                             "packed rows");
             return finish_launch(launch_gemm(dtype, a, s), "tensor-core gemm launch");
         }
-        // Decode shapes of the [N, K] layout stream the weight through the
-        // SIMT decode kernel; larger activation counts, and the [K, N] layout
-        // at any count, use the tensor cores.
+        // Decode shapes of the [N, K] layout (1..4 rows) stream the weight
+        // through the SIMT decode kernel; larger activation counts, and the
+        // [K, N] layout at any count, use the tensor-core GEMM.  The decode
+        // tensor-core kernel runs only when forced (measured slower: its
+        // per-k-block tensor-memory stores set its pace).
+        if (g_path == QMM_PATH_DECODE_TC) {
+            if (!gemv_tc_supported(dtype, a))
+                return fail(QMM_ERR_UNSUPPORTED,
+                            "the decode tensor-core path needs bf16/f16, transpose, 1..16 rows, 2- or "
+                            "4-bit codes, K %% 512 == 0 and (K / group_size) %% 8 == 0");
+            return finish_launch(launch_gemv_tc(dtype, a, s), "decode tensor-core launch");
+        }
         const bool few_rows = a.M <= kGemvMaxRows && a.transpose;
         if (g_path == QMM_PATH_GEMV || few_rows || !tc_ok) {
             if (gemv_fast_supported(dtype, a))
@@ -242,6 +308,28 @@ qmm_status qmm_quantized_matmul_ws(const void *x, int64_t M, int64_t K, const ui
     } catch (...) {
         return fail(QMM_ERR_CUDA, "unexpected exception in qmm_quantized_matmul");
     }
+}
+
+}  // namespace
+
+extern "C" {
+
+qmm_status qmm_quantized_matmul_ws(const void *x, int64_t M, int64_t K, const uint32_t *wq,
+                                   const void *scales, const void *biases, qmm_dtype dtype,
+                                   int64_t N, int transpose, int group_size, int bits,
+                                   const char *mode, void *y, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    return matmul_impl(x, M, K, wq, scales, biases, dtype, N, transpose, group_size, bits, mode,
+                       nullptr, 0.0, y, workspace, workspace_bytes, stream);
+}
+
+qmm_status qmm_quantized_dense(const void *x, int64_t M, int64_t K, const uint32_t *wq,
+                               const void *scales, const void *biases, qmm_dtype dtype, int64_t N,
+                               int transpose, int group_size, int bits, const char *mode,
+                               const void *bias, double bias_value, void *y, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    return matmul_impl(x, M, K, wq, scales, biases, dtype, N, transpose, group_size, bits, mode,
+                       bias, bias_value, y, workspace, workspace_bytes, stream);
 }
 
 qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K, const uint32_t *wq,
@@ -255,8 +343,10 @@ qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K, const uint3
 size_t qmm_quantized_matmul_workspace_size(int64_t M, int64_t K, int64_t N, int transpose,
                                            int bits, qmm_dtype dtype) {
     try {
-        // Decode shapes go to the SIMT kernel under the automatic path.
+        // Decode shapes go to the SIMT decode kernel under the automatic path,
+        // and the forced decode tensor-core kernel takes no workspace.
         if (g_path != QMM_PATH_GEMM && M <= kGemvMaxRows && transpose) return 0;
+        if (g_path == QMM_PATH_DECODE_TC) return 0;
         return gemm_workspace_size(dtype, M, K, N, transpose != 0, bits);
     } catch (...) {
         return 0;
@@ -285,8 +375,12 @@ qmm_status qmm_gather_qmm(const void *x, int64_t x_batch, int64_t M, int64_t K,
     // trusted: a wrong hint cannot produce wrong results.
     (void)sorted_indices;
     try {
-        qmm_status st = check_common(dtype, group_size, bits, mode);
+        int md = QMM_MODE_AFFINE;
+        qmm_status st = check_common(dtype, group_size, bits, mode, &md);
         if (st != QMM_OK) return st;
+        if (md != QMM_MODE_AFFINE)
+            return fail(QMM_ERR_UNSUPPORTED,
+                        "gather_qmm takes affine weights (its callers pass mode \"affine\")");
         if (batch < 0 || x_batch < 1 || n_experts < 1 || M < 0 || N < 0 || K <= 0)
             return fail(QMM_ERR_INVALID_ARG,
                         "need batch >= 0, x_batch >= 1, n_experts >= 1, M >= 0, N >= 0, K > 0");
@@ -344,6 +438,65 @@ qmm_status qmm_gather_qmm(const void *x, int64_t x_batch, int64_t M, int64_t K,
         return finish_launch(launch_gemv_gather(dtype, a, gi, s), "gather_qmm launch");
     } catch (...) {
         return fail(QMM_ERR_CUDA, "unexpected exception in qmm_gather_qmm");
+    }
+}
+
+// qqmm workspace: the quantized activations (codes, scale bytes) and their
+// exact dequantized copy, each piece 256-byte aligned.
+struct QqmmWorkspace {
+    size_t xq, xs, xd, total;
+};
+static QqmmWorkspace qqmm_layout(int64_t M, int64_t K, int group_size, int bits, qmm_dtype dt) {
+    auto up = [](size_t v) { return (v + 255) & ~(size_t)255; };
+    QqmmWorkspace w{};
+    w.xq = 0;
+    w.xs = up((size_t)M * (size_t)(K * bits / 32) * 4);
+    w.xd = w.xs + up((size_t)M * (size_t)(K / group_size));
+    w.total = w.xd + up((size_t)M * (size_t)K * (dt == QMM_F32 ? 4 : 2));
+    return w;
+}
+
+size_t qmm_qqmm_workspace_size(int64_t M, int64_t K, int group_size, int bits, qmm_dtype dtype) {
+    if (M <= 0 || K <= 0 || (group_size != 16 && group_size != 32) || K % group_size) return 0;
+    if (dtype != QMM_F32 && dtype != QMM_BF16 && dtype != QMM_F16) return 0;
+    return qqmm_layout(M, K, group_size, bits, dtype).total;
+}
+
+qmm_status qmm_qqmm(const void *x, int64_t M, int64_t K, qmm_dtype dtype, const uint32_t *wq,
+                    const void *w_scales, int64_t N, int group_size, int bits, const char *mode,
+                    void *y, void *workspace, size_t workspace_bytes, void *stream) {
+    try {
+        int md = QMM_MODE_AFFINE;
+        qmm_status st = check_common(dtype, group_size, bits, mode, &md);
+        if (st != QMM_OK) return st;
+        if (md != QMM_MODE_NVFP4 && md != QMM_MODE_MXFP8)
+            return fail(QMM_ERR_UNSUPPORTED, "qqmm supports modes \"nvfp4\" and \"mxfp8\"");
+        st = check_matmul(x, M, K, wq, w_scales, nullptr, N, 1, group_size, y, md);
+        if (st != QMM_OK) return st;
+        if (M == 0 || N == 0) return QMM_OK;
+        const QqmmWorkspace L = qqmm_layout(M, K, group_size, bits, dtype);
+        if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+            return fail(QMM_ERR_WORKSPACE, "workspace must be a 256-byte aligned device buffer");
+        if (workspace_bytes < L.total)
+            return fail(QMM_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, L.total);
+        cudaStream_t s = (cudaStream_t)stream;
+        char *ws = static_cast<char *>(workspace);
+        uint32_t *xq = reinterpret_cast<uint32_t *>(ws + L.xq);
+        void *xs = ws + L.xs, *xd = ws + L.xd;
+        // 1. the activations quantized in the weight's mode (rows of x, groups
+        //    along K), 2. their exact dequantized values, 3. the product with
+        //    the quantized weight.
+        QuantArgs qa{x, M, K, group_size, bits, xq, xs, nullptr, md};
+        cudaError_t e = launch_quantize_mx(dtype, qa, s);
+        if (e != cudaSuccess) return cuda_fail(e, "qqmm: quantize the activations");
+        DequantArgs da{xq, xs, nullptr, M, K, group_size, bits, xd, md};
+        e = launch_dequantize_mx(dtype, da, s);
+        if (e != cudaSuccess) return cuda_fail(e, "qqmm: dequantize the activations");
+        QmmArgs a{xd, wq, w_scales, nullptr, y, M, N, K, group_size, bits, true};
+        a.mode = md;
+        return finish_launch(launch_mx_matmul(dtype, a, s), "qqmm product launch");
+    } catch (...) {
+        return fail(QMM_ERR_CUDA, "unexpected exception in qmm_qqmm");
     }
 }
 
@@ -412,7 +565,8 @@ qmm_status qmm_inject_fault(qmm_fault fault) {
 }
 
 qmm_status qmm_set_path(qmm_path path) {
-    if (path != QMM_PATH_AUTO && path != QMM_PATH_GEMV && path != QMM_PATH_GEMM)
+    if (path != QMM_PATH_AUTO && path != QMM_PATH_GEMV && path != QMM_PATH_GEMM &&
+        path != QMM_PATH_DECODE_TC)
         return fail(QMM_ERR_INVALID_ARG, "unknown path %d", (int)path);
     g_path = path;
     return QMM_OK;

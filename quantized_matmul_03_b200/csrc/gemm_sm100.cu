@@ -49,6 +49,7 @@
 
 #include "ptx_sm100.cuh"
 #include "qmm_internal.cuh"
+#include "tcgen05.cuh"
 
 namespace qmm {
 namespace {
@@ -63,159 +64,6 @@ constexpr int kThreads = 32 * (kWarpTmaS + 1);  // 512
 constexpr int kBM = 128;                        // weight rows per tile (UMMA M)
 constexpr int kBK = 64;                         // k per stage: one 128-byte swizzle row
 constexpr int kSkMaxBN = 64;                    // widest tile that stream-K splits
-
-// ---------------------------------------------------------------------------
-// tcgen05 / TMA wrappers
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
-                 "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-// Arrive on `bar` once every tcgen05.mma this thread issued so far completed.
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     bar)
-                 : "memory");
-}
-// D[tmem] (+)= A[desc_a] * B[desc_b]^T, shapes and types from idesc.
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t desc_a, uint64_t desc_b,
-                                       uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(desc_a), "l"(desc_b), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// D[tmem] (+)= A[tmem_a] * B[desc_b]^T with operand A in tensor memory (lane
-// i = row i, 16-bit K values two per 32-bit column).
-__device__ __forceinline__ void tc_mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t desc_b,
-                                          uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "r"(tmem_a), "l"(desc_b), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// Thread i of the warp writes v[0..31] to columns taddr.col .. +31 of TMEM
-// lane taddr.lane + i.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
-        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
-        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
-        "r"(v[29]), "r"(v[30]), "r"(v[31])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() {
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-          "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
-          "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
-          "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr)
-        : "memory");
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-          "=r"(v[14]), "=r"(v[15])
-        : "r"(taddr)
-        : "memory");
-}
-// True on one lane of the (converged) warp.
-__device__ __forceinline__ bool elect_one() {
-    uint32_t pred;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "elect.sync _|p, 0xffffffff;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(pred));
-    return pred != 0;
-}
-__device__ __forceinline__ void tmem_ld_wait() {
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                            uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(map), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-
-// Tensor store of a shared-memory box to global (bulk-group completion).
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map),
-                 "r"(x), "r"(y), "r"(src)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Wait until every committed store has finished reading shared memory.
-__device__ __forceinline__ void bulk_wait_read0() {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-// Wait until every committed store has completed.
-__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void sts16(uint32_t a, uint16_t v) {
-    asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(v) : "memory");
-}
-template <typename T>
-__device__ __forceinline__ uint16_t out_bits(float f) {
-    const T h = Dt<T>::from_f(f);
-    return *reinterpret_cast<const uint16_t *>(&h);
-}
-
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
-// 1024 bytes apart (SBO), LBO unused (16), descriptor version 1.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-// MN-major, 128-byte swizzle: atoms of 64 MN-elements (128 bytes) x 8 K-rows
-// (1 KB); atoms along MN LBO bytes apart, groups of 8 K-rows SBO bytes apart.
-__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-// Instruction descriptor of kind::f16: fp32 accumulator, A/B both bf16 (or
-// both f16), B K-major, A K-major (or MN-major with a_mn), shape M x N.
-__host__ __device__ constexpr uint32_t make_idesc(bool f16, int m, int n, bool a_mn = false) {
-    return (1u << 4) | ((f16 ? 0u : 1u) << 7) | ((f16 ? 0u : 1u) << 10) | ((a_mn ? 1u : 0u) << 15) |
-           ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
-}
 
 // ---------------------------------------------------------------------------
 // Dequantization of a half k-block of one weight row (32 codes) into four
@@ -321,11 +169,6 @@ struct RingPos {
     }
 };
 
-// v.x / v.y / v.z / v.w by a runtime index without indexing registers.
-__device__ __forceinline__ uint32_t pick_word(const uint4 &v, int i) {
-    const uint32_t lo = (i & 1) ? v.y : v.x, hi = (i & 1) ? v.w : v.z;
-    return (i & 2) ? hi : lo;
-}
 
 struct GemmParams {
     const void *scales, *biases;
@@ -341,6 +184,8 @@ struct GemmParams {
     float *sk_ws;    // per CTA: one fp32 partial tile, [quadrant][chunk][lane][CW]
     int *sk_flags;   // per CTA and quadrant: 1 while its partial awaits the tile's owner
     int sk_no_publish;  // test injection: parts are written but their flags never raised
+    const void *bias;   // layer bias [N] or null, plus bias_value (not in grouped mode)
+    float bias_value;
     int *err;
     // Grouped (gather_qmm) mode only: the chunk table and row map the
     // preparation kernel wrote.  Tile t covers chunk t / n_tiles and weight
@@ -786,6 +631,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     }
                     __syncwarp();
                 }
+                const float lb = layer_bias<T>(p.bias, p.bias_value, min(t.n0 + 32 * q + lane, p.N - 1));
                 int j = 0;
                 for (int m_off = 0; m_off < t.rows; m_off += p.stg_rows) {
                     if (lane == 0) bulk_wait_read0();  // the slab's last store has read it
@@ -817,7 +663,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                         }
                         const uint32_t row0 = stg + (uint32_t)(jj * CW) * 64u + 2u * lane;
 #pragma unroll
-                        for (int cc = 0; cc < CW; ++cc) sts16(row0 + 64u * cc, out_bits<T>(__uint_as_float(v[cc])));
+                        for (int cc = 0; cc < CW; ++cc) sts16(row0 + 64u * cc, out_bits<T>(__uint_as_float(v[cc]) + lb));
                     }
                     ptx::fence_proxy_async_smem();
                     __syncwarp();
@@ -832,6 +678,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 continue;
             }
             const int n = t.n0 + 32 * q + lane;
+            const float lb = GROUPED ? 0.f : layer_bias<T>(p.bias, p.bias_value, min(n, p.N - 1));
             // Columns acc*BN .. acc*BN+BN-1 of this warp's 32 lanes, 32 (or, for
             // BN = 16, 16) columns per load so no load leaves the allocation;
             // column chunks past the tile's rows are skipped.
@@ -857,7 +704,7 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     if constexpr (GROUPED) dst = __shfl_sync(0xffffffffu, my_dst, cc);
                     else dst = t.m0 + mm;
                     if (n < p.N && mm < t.rows)
-                        y[dst * p.N + n] = Dt<T>::from_f(__uint_as_float(v[cc]));
+                        y[dst * p.N + n] = Dt<T>::from_f(__uint_as_float(v[cc]) + lb);
                 }
             }
             tc_fence_before();
@@ -991,39 +838,6 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *ptr, uint64_t inner,
-                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-                 CUtensorMapSwizzle swz) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int pick_bn(int64_t M) {
     if (M <= 16) return 16;
     if (M <= 32) return 32;
@@ -1154,6 +968,8 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
     p.n_tiles = (int)((a.N + kBM - 1) / kBM);
     p.num_tiles = p.m_tiles * p.n_tiles;
     p.stages = stages;
+    p.bias = a.bias;
+    p.bias_value = a.bias_value;
     p.err = device_error_word();
     int grid = std::min(p.num_tiles, num_sms());
     // Stream-K when there are fewer tiles than SMs and tiles are narrow
@@ -1280,6 +1096,7 @@ cudaError_t grouped_bits(const GroupedArgs &g, cudaStream_t s) {
 // [K, N] storage), sizes in int range.
 bool gemm_supported(qmm_dtype dt, const QmmArgs &a) {
     if (dt != QMM_BF16 && dt != QMM_F16) return false;
+    if (a.mode != QMM_MODE_AFFINE || (a.bits != 2 && a.bits != 4 && a.bits != 8)) return false;
     if (a.K % kBK != 0) return false;
     if (((a.transpose ? a.K : a.N) * a.bits / 8) % 16 != 0) return false;
     if (a.M > INT32_MAX / 2 || a.N > INT32_MAX / 2 || a.K > INT32_MAX / 2) return false;
@@ -1312,6 +1129,7 @@ cudaError_t launch_gemm(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
 
 bool gemm_grouped_supported(qmm_dtype dt, const GroupedArgs &g) {
     if (!g.transpose) return false;
+    if (g.bits != 2 && g.bits != 4 && g.bits != 8) return false;
     if (dt != QMM_BF16 && dt != QMM_F16) return false;
     if (g.K % kBK != 0) return false;
     if ((g.K * g.bits / 8) % 16 != 0) return false;

@@ -18,6 +18,7 @@
 
 #include <cooperative_groups.h>
 
+#include "mx.cuh"
 #include "qmm_internal.cuh"
 
 namespace cg = cooperative_groups;
@@ -36,6 +37,8 @@ struct BatchView {
     GatherIndex gi;
     int64_t b0;
     int64_t x_stride, w_stride, sb_stride, y_stride;  // elements / words per entry
+    const void *bias;  // layer bias (plain matmul only), added before rounding
+    float bias_value;
     int *err;
 };
 
@@ -59,6 +62,41 @@ __device__ __forceinline__ bool select_entry(const BatchView &bv, EntryOffsets &
     return valid;
 }
 
+// The kernels walk packed rows in chunks: one word (32/bits codes) for 2-,
+// 4- and 8-bit codes; for 3- and 6-bit codes, which run back to back in the
+// row's bit stream, the `bits` words that hold 32 codes exactly.  A chunk
+// never leaves its group (group_size >= 32).
+template <int BITS> struct Chunk {
+    static constexpr int W = (BITS == 3 || BITS == 6) ? BITS : 1;  // words per chunk
+    static constexpr int E = W * 32 / BITS;                        // codes per chunk
+};
+
+// The E weights of one chunk: affine s*q + b (fmaf, as dequantize), or, in a
+// microscaled mode, X * element (exact).  `sb` indexes the chunk's group in
+// scales (and biases).
+template <typename T, int BITS, int MODE>
+__device__ __forceinline__ void chunk_weights(const uint32_t *pk, const void *scales,
+                                              const void *biases, int64_t sb, float *wv) {
+    constexpr int E = Chunk<BITS>::E;
+    if constexpr (MODE == QMM_MODE_AFFINE) {
+        constexpr uint32_t MASK = (1u << BITS) - 1u;
+        const float s = Dt<T>::to_f(static_cast<const T *>(scales)[sb]);
+        const float b = Dt<T>::to_f(static_cast<const T *>(biases)[sb]);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int bit = e * BITS, wi = bit >> 5, off = bit & 31;
+            uint32_t q = pk[wi] >> off;
+            if (off + BITS > 32) q |= pk[wi + 1] << (32 - off);
+            wv[e] = __fmaf_rn(s, (float)(q & MASK), b);
+        }
+    } else {
+        const float x = mxf::scale_value<MODE>(static_cast<const uint8_t *>(scales)[sb]);
+        mxf::elements<MODE>(pk[0], wv);
+#pragma unroll
+        for (int e = 0; e < E; ++e) wv[e] = __fmul_rn(x, wv[e]);
+    }
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
@@ -68,26 +106,24 @@ __device__ __forceinline__ float warp_sum(float v) {
 // ---------------------------------------------------------------------------
 // transpose = true
 // ---------------------------------------------------------------------------
-template <typename T, int BITS, int MT, int RW>
+template <typename T, int BITS, int MT, int RW, int MODE>
 __global__ void __launch_bounds__(kThreads)
 gemv_t_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
-              const T *__restrict__ scales, const T *__restrict__ biases,
+              const void *__restrict__ scales, const void *__restrict__ biases,
               T *__restrict__ y, int M, int64_t N, int64_t K, int group_size, int kc,
               const BatchView bv) {
-    constexpr int EPW = 32 / BITS;
-    constexpr uint32_t MASK = (1u << BITS) - 1u;
+    constexpr int CW = Chunk<BITS>::W, CE = Chunk<BITS>::E;
     extern __shared__ float xs[];  // [MT][kc]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row0 = (int64_t)blockIdx.x * (kWarps * RW) + (int64_t)warp * RW;
-    const int64_t wpr = K / EPW;          // packed words per weight row
+    const int64_t wpr = K * BITS / 32;    // packed words per weight row
     const int64_t gpr = K / group_size;   // groups per weight row
 
     EntryOffsets eo;
     const bool valid = select_entry(bv, eo);
     x += eo.x;
     wq += eo.w;
-    scales += eo.sb;
-    biases += eo.sb;
+    const int64_t sb0 = eo.sb;
     y += eo.y;
 
     float acc[RW][MT];
@@ -104,23 +140,24 @@ gemv_t_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
             xs[m * kc + kk] = (m < M) ? Dt<T>::to_f(x[(int64_t)m * K + k0 + kk]) : 0.f;
         }
         __syncthreads();
-        const int wlen = klen / EPW;
+        const int clen = klen / CE;   // chunks of this activation chunk (kc % 128 == 0)
 #pragma unroll
         for (int r = 0; r < RW; ++r) {
             const int64_t row = row0 + r;
             if (row >= N) break;  // warp-uniform
-            const uint32_t *wr = wq + row * wpr + k0 / EPW;
-            for (int j = lane; j < wlen; j += 32) {
-                const uint32_t pk = __ldg(wr + j);
-                const int64_t g = (k0 + (int64_t)j * EPW) / group_size;
-                const float s = Dt<T>::to_f(scales[row * gpr + g]);
-                const float b = Dt<T>::to_f(biases[row * gpr + g]);
+            const uint32_t *wr = wq + row * wpr + k0 * BITS / 32;
+            for (int j = lane; j < clen; j += 32) {
+                uint32_t pk[CW];
 #pragma unroll
-                for (int e = 0; e < EPW; ++e) {
-                    const float wv = __fmaf_rn(s, (float)((pk >> (e * BITS)) & MASK), b);
+                for (int i = 0; i < CW; ++i) pk[i] = __ldg(wr + j * CW + i);
+                const int64_t g = (k0 + (int64_t)j * CE) / group_size;
+                float wv[CE];
+                chunk_weights<T, BITS, MODE>(pk, scales, biases, sb0 + row * gpr + g, wv);
+#pragma unroll
+                for (int e = 0; e < CE; ++e) {
 #pragma unroll
                     for (int m = 0; m < MT; ++m)
-                        acc[r][m] = __fmaf_rn(xs[m * kc + j * EPW + e], wv, acc[r][m]);
+                        acc[r][m] = __fmaf_rn(xs[m * kc + j * CE + e], wv[e], acc[r][m]);
                 }
             }
         }
@@ -132,7 +169,8 @@ gemv_t_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
             const float v = warp_sum(acc[r][m]);
-            if (lane == 0 && m < M) y[(int64_t)m * N + row] = Dt<T>::from_f(v);
+            if (lane == 0 && m < M)
+                y[(int64_t)m * N + row] = Dt<T>::from_f(v + layer_bias<T>(bv.bias, bv.bias_value, row));
         }
     }
 }
@@ -140,14 +178,13 @@ gemv_t_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
 // ---------------------------------------------------------------------------
 // transpose = false: W stored [K, N], groups run along N.
 // ---------------------------------------------------------------------------
-template <typename T, int BITS, int MT>
+template <typename T, int BITS, int MT, int MODE>
 __global__ void __launch_bounds__(kThreads)
 gemv_n_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
-              const T *__restrict__ scales, const T *__restrict__ biases,
+              const void *__restrict__ scales, const void *__restrict__ biases,
               T *__restrict__ y, int M, int64_t N, int64_t K, int group_size, int64_t k_split,
               const BatchView bv) {
-    constexpr int EPW = 32 / BITS;
-    constexpr uint32_t MASK = (1u << BITS) - 1u;
+    constexpr int CW = Chunk<BITS>::W, EPW = Chunk<BITS>::E;  // (EPW: codes per chunk)
     constexpr int NE = EPW * MT;           // partial sums per lane
     __shared__ float red[kWarps][NE][32];  // per-warp partials
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -155,13 +192,13 @@ gemv_n_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     const bool valid = select_entry(bv, eo);
     x += eo.x;
     wq += eo.w;
-    scales += eo.sb;
-    biases += eo.sb;
+    const int64_t sb0 = eo.sb;
     y += eo.y;
-    const int64_t wpr = N / EPW;            // packed words per weight row
+    const int64_t wpr = N * BITS / 32;      // packed words per weight row
+    const int64_t cpr = N / EPW;            // chunks per weight row
     const int64_t gpr = N / group_size;
-    const int64_t col = (int64_t)blockIdx.x * 32 + lane;  // packed word column
-    const bool col_ok = col < wpr;
+    const int64_t col = (int64_t)blockIdx.x * 32 + lane;  // chunk column
+    const bool col_ok = col < cpr;
     const int64_t kbeg = (int64_t)blockIdx.y * k_split;
     const int64_t kend = min(K, kbeg + k_split);
 
@@ -172,17 +209,18 @@ gemv_n_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     if (col_ok && valid) {
         const int64_t g = col * EPW / group_size;
         for (int64_t k = kbeg + warp; k < kend; k += kWarps) {
-            const uint32_t pk = __ldg(wq + k * wpr + col);
-            const float s = Dt<T>::to_f(scales[k * gpr + g]);
-            const float b = Dt<T>::to_f(biases[k * gpr + g]);
+            uint32_t pk[CW];
+#pragma unroll
+            for (int i = 0; i < CW; ++i) pk[i] = __ldg(wq + k * wpr + col * CW + i);
+            float wv[EPW];
+            chunk_weights<T, BITS, MODE>(pk, scales, biases, sb0 + k * gpr + g, wv);
             float xv[MT];
 #pragma unroll
             for (int m = 0; m < MT; ++m) xv[m] = (m < M) ? Dt<T>::to_f(x[(int64_t)m * K + k]) : 0.f;
 #pragma unroll
             for (int e = 0; e < EPW; ++e) {
-                const float wv = __fmaf_rn(s, (float)((pk >> (e * BITS)) & MASK), b);
 #pragma unroll
-                for (int m = 0; m < MT; ++m) acc[e * MT + m] = __fmaf_rn(xv[m], wv, acc[e * MT + m]);
+                for (int m = 0; m < MT; ++m) acc[e * MT + m] = __fmaf_rn(xv[m], wv[e], acc[e * MT + m]);
             }
         }
     }
@@ -208,12 +246,14 @@ gemv_n_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
         for (int q = 0; q < nrank; ++q) v += cluster.map_shared_rank(&red[0][0][0], q)[e * 32 + l];
         const int64_t c = (int64_t)blockIdx.x * 32 + l;
         const int ei = e / MT, m = e - ei * MT;
-        if (c < wpr && m < M) y[(int64_t)m * N + c * EPW + ei] = Dt<T>::from_f(v);
+        if (c < cpr && m < M)
+            y[(int64_t)m * N + c * EPW + ei] =
+                Dt<T>::from_f(v + layer_bias<T>(bv.bias, bv.bias_value, c * EPW + ei));
     }
     cluster.sync();
 }
 
-template <typename T, int BITS, int MT>
+template <typename T, int BITS, int MT, int MODE>
 cudaError_t run_gemv_t(const QmmArgs &a, int M, const T *x, T *y, const BatchView &bv, int nb,
                        cudaStream_t s) {
     constexpr int RW = 2;
@@ -225,19 +265,17 @@ cudaError_t run_gemv_t(const QmmArgs &a, int M, const T *x, T *y, const BatchVie
     if (kc <= 0) kc = 128;
     if (kc > a.K) kc = (int)a.K;
     const size_t smem = (size_t)MT * kc * sizeof(float);
-    gemv_t_kernel<T, BITS, MT, RW><<<dim3((unsigned)gx, 1, nb), kThreads, smem, s>>>(
-        x, a.wq, static_cast<const T *>(a.scales), static_cast<const T *>(a.biases), y, M,
-        a.N, a.K, a.group_size, kc, bv);
+    gemv_t_kernel<T, BITS, MT, RW, MODE><<<dim3((unsigned)gx, 1, nb), kThreads, smem, s>>>(
+        x, a.wq, a.scales, a.biases, y, M, a.N, a.K, a.group_size, kc, bv);
     count_launches(1);
     return cudaGetLastError();
 }
 
-template <typename T, int BITS, int MT>
+template <typename T, int BITS, int MT, int MODE>
 cudaError_t run_gemv_n(const QmmArgs &a, int M, const T *x, T *y, const BatchView &bv, int nb,
                        cudaStream_t s) {
-    constexpr int EPW = 32 / BITS;
-    const int64_t wpr = a.N / EPW;
-    const int gx = (int)((wpr + 31) / 32);
+    const int64_t cpr = a.N / Chunk<BITS>::E;
+    const int gx = (int)((cpr + 31) / 32);
     // Split K over a cluster of up to 8 CTAs so that small-N problems still
     // fill the GPU; each split is at least 64 rows of W.
     int ks = 8;
@@ -257,19 +295,19 @@ cudaError_t run_gemv_n(const QmmArgs &a, int M, const T *x, T *y, const BatchVie
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     count_launches(1);
-    return cudaLaunchKernelEx(&cfg, gemv_n_kernel<T, BITS, MT>, x, a.wq,
-                              static_cast<const T *>(a.scales), static_cast<const T *>(a.biases),
+    return cudaLaunchKernelEx(&cfg, gemv_n_kernel<T, BITS, MT, MODE>, x, a.wq, a.scales, a.biases,
                               y, M, a.N, a.K, a.group_size, k_split, bv);
 }
 
 // Largest activation tile per launch: gemv_t keeps RW*MT accumulators per
 // lane; gemv_n keeps (32/bits)*MT, capped at 32 (so MT <= bits).  Entries of
 // a batch go to gridDim.z, at most 65535 per launch.
-template <typename T, int BITS>
+template <typename T, int BITS, int MODE = QMM_MODE_AFFINE>
 cudaError_t gemv_bits(const QmmArgs &a, const BatchView &bv0, int64_t batch, cudaStream_t s) {
     const T *x = static_cast<const T *>(a.x);
     T *y = static_cast<T *>(a.y);
-    const int tile = a.transpose ? 16 : BITS;
+    // (3-/6-bit chunks hold 32 codes per lane: one activation row at a time)
+    const int tile = a.transpose ? 16 : (BITS == 3 || BITS == 6 ? 1 : BITS);
     for (int64_t b0 = 0; b0 < batch; b0 += 65535) {
         const int nb = (int)std::min<int64_t>(65535, batch - b0);
         BatchView bv = bv0;
@@ -280,17 +318,18 @@ cudaError_t gemv_bits(const QmmArgs &a, const BatchView &bv0, int64_t batch, cud
             T *ym = y + m0 * a.N;
             cudaError_t e;
             if (a.transpose) {
-                if (mt == 1) e = run_gemv_t<T, BITS, 1>(a, mt, xm, ym, bv, nb, s);
-                else if (mt == 2) e = run_gemv_t<T, BITS, 2>(a, mt, xm, ym, bv, nb, s);
-                else if (mt <= 4) e = run_gemv_t<T, BITS, 4>(a, mt, xm, ym, bv, nb, s);
-                else if (mt <= 8) e = run_gemv_t<T, BITS, 8>(a, mt, xm, ym, bv, nb, s);
-                else e = run_gemv_t<T, BITS, 16>(a, mt, xm, ym, bv, nb, s);
+                if (mt == 1) e = run_gemv_t<T, BITS, 1, MODE>(a, mt, xm, ym, bv, nb, s);
+                else if (mt == 2) e = run_gemv_t<T, BITS, 2, MODE>(a, mt, xm, ym, bv, nb, s);
+                else if (mt <= 4) e = run_gemv_t<T, BITS, 4, MODE>(a, mt, xm, ym, bv, nb, s);
+                else if (mt <= 8) e = run_gemv_t<T, BITS, 8, MODE>(a, mt, xm, ym, bv, nb, s);
+                else e = run_gemv_t<T, BITS, 16, MODE>(a, mt, xm, ym, bv, nb, s);
             } else {
-                if (mt == 1) e = run_gemv_n<T, BITS, 1>(a, mt, xm, ym, bv, nb, s);
-                else if (mt == 2) e = run_gemv_n<T, BITS, 2>(a, mt, xm, ym, bv, nb, s);
-                else if constexpr (BITS >= 4) {
-                    if (mt <= 4) e = run_gemv_n<T, BITS, 4>(a, mt, xm, ym, bv, nb, s);
-                    else if constexpr (BITS >= 8) e = run_gemv_n<T, BITS, 8>(a, mt, xm, ym, bv, nb, s);
+                if (mt == 1) e = run_gemv_n<T, BITS, 1, MODE>(a, mt, xm, ym, bv, nb, s);
+                else if constexpr (BITS == 3 || BITS == 6) e = cudaErrorInvalidValue;
+                else if (mt == 2) e = run_gemv_n<T, BITS, 2, MODE>(a, mt, xm, ym, bv, nb, s);
+                else if constexpr (BITS == 4 || BITS == 8) {
+                    if (mt <= 4) e = run_gemv_n<T, BITS, 4, MODE>(a, mt, xm, ym, bv, nb, s);
+                    else if constexpr (BITS >= 8) e = run_gemv_n<T, BITS, 8, MODE>(a, mt, xm, ym, bv, nb, s);
                     else e = cudaErrorInvalidValue;
                 } else {
                     e = cudaErrorInvalidValue;
@@ -304,9 +343,17 @@ cudaError_t gemv_bits(const QmmArgs &a, const BatchView &bv0, int64_t batch, cud
 
 template <typename T>
 cudaError_t gemv_t_dtype(const QmmArgs &a, const BatchView &bv, int64_t batch, cudaStream_t s) {
+    switch (a.mode) {
+    case QMM_MODE_MXFP4: return gemv_bits<T, 4, QMM_MODE_MXFP4>(a, bv, batch, s);
+    case QMM_MODE_NVFP4: return gemv_bits<T, 4, QMM_MODE_NVFP4>(a, bv, batch, s);
+    case QMM_MODE_MXFP8: return gemv_bits<T, 8, QMM_MODE_MXFP8>(a, bv, batch, s);
+    default: break;
+    }
     switch (a.bits) {
     case 2: return gemv_bits<T, 2>(a, bv, batch, s);
+    case 3: return gemv_bits<T, 3>(a, bv, batch, s);
     case 4: return gemv_bits<T, 4>(a, bv, batch, s);
+    case 6: return gemv_bits<T, 6>(a, bv, batch, s);
     default: return gemv_bits<T, 8>(a, bv, batch, s);
     }
 }
@@ -328,6 +375,8 @@ cudaError_t launch_gemv(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
     if (a.M == 0 || a.N == 0) return cudaSuccess;
     BatchView bv{};
     bv.gi = GatherIndex{nullptr, nullptr, 1, 1, 1};
+    bv.bias = a.bias;
+    bv.bias_value = a.bias_value;
     bv.err = device_error_word();
     return gemv_dispatch(dt, a, bv, 1, s);
 }
@@ -336,12 +385,11 @@ cudaError_t launch_gemv(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
 // expert 0, y at y[0] ([M, N]).
 cudaError_t launch_gemv_gather(qmm_dtype dt, const QmmArgs &a, const GatherIndex &gi, cudaStream_t s) {
     if (a.M == 0 || a.N == 0 || gi.batch == 0) return cudaSuccess;
-    const int bits = a.bits, epw = 32 / bits;
     const int64_t wrows = a.transpose ? a.N : a.K, wcols = a.transpose ? a.K : a.N;
     BatchView bv{};
     bv.gi = gi;
     bv.x_stride = a.M * a.K;
-    bv.w_stride = wrows * (wcols / epw);
+    bv.w_stride = wrows * (wcols * a.bits / 32);
     bv.sb_stride = wrows * (wcols / a.group_size);
     bv.y_stride = a.M * a.N;
     bv.err = device_error_word();

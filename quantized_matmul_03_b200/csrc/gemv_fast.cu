@@ -21,7 +21,7 @@
 // fixed point, x_int = rint(x * 2^sh) with sh chosen from the slice's largest
 // |x| so that |x_int| < 2^14: the representation error is at most 2^-15 of
 // the slice maximum, and every product and sum after it is exact.  A slice's
-// integer sum is scaled back by 2^-sh in fp32; sum(x) uses the exact x.
+// integer sum is multiplied by s * 2^-sh in fp32; sum(x) uses the exact x.
 // Per word of 4-bit codes this is 3 ALU + 4 DP2A instructions (8-bit codes:
 // 2 DP2A, no ALU), which keeps the ALU pipe, the limiter of an fp32
 // formulation, below the memory time.  Lane partials for a stage's rows are
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     const T *__restrict__ scales, const T *__restrict__ biases,
                     T *__restrict__ y, int M, int N, int K, int group_size, int rpc, int S,
-                    int TW, int *err) {
+                    int TW, const T *__restrict__ bias, float bias_value, int *err) {
     constexpr int EPW = 32 / BITS;       // codes per word
     constexpr int EPU = 4 * EPW;         // codes per 16-byte slice
     constexpr int STEPS = EPW / 2;       // code pairs per word
@@ -312,8 +312,11 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                             dot_word<BITS>(wv.y, &xp[m][u][1 * STEPS], a0, a1);
                             dot_word<BITS>(wv.z, &xp[m][u][2 * STEPS], a0, a1);
                             dot_word<BITS>(wv.w, &xp[m][u][3 * STEPS], a0, a1);
-                            const float t = (float)(a0 + a1) * fsc[m][u];
-                            const float c = __fmaf_rn(sc, t, bi * xsum[m][u]);
+                            // (s * 2^-sh) first: the integer sum times 2^-sh alone
+                            // can exceed the fp32 range for activations near the
+                            // top of bf16's range, while the product with s cannot
+                            // unless the result itself does.
+                            const float c = __fmaf_rn(sc * fsc[m][u], (float)(a0 + a1), bi * xsum[m][u]);
                             part[m * RPT + j] += use ? c : 0.f;
                         }
                     }
@@ -340,7 +343,7 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     __syncthreads();
     for (int idx = threadIdx.x; idx < M * nrows; idx += kThreads) {
         const int m = idx / nrows, r = idx - m * nrows;
-        y[(int64_t)m * N + r0 + r] = Dt<T>::from_f(ysm[m * rpc + r]);
+        y[(int64_t)m * N + r0 + r] = Dt<T>::from_f(ysm[m * rpc + r] + layer_bias<T>(bias, bias_value, r0 + r));
     }
 }
 
@@ -433,7 +436,8 @@ cudaError_t launch_stream(const QmmArgs &a, cudaStream_t s) {
     e = cudaLaunchKernelEx(&cfg, kern, static_cast<const T *>(a.x), a.wq,
                            static_cast<const T *>(a.scales), static_cast<const T *>(a.biases),
                            static_cast<T *>(a.y), (int)a.M, (int)a.N, (int)a.K, a.group_size,
-                           p.rpc, p.stages, p.tw, device_error_word());
+                           p.rpc, p.stages, p.tw, static_cast<const T *>(a.bias), a.bias_value,
+                           device_error_word());
     if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();
@@ -500,6 +504,7 @@ cudaError_t stream_bits(const QmmArgs &a, cudaStream_t s) {
 // slice (group_size >= codes per slice), rows at most 8 warps wide.
 bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a) {
     if (!a.transpose || a.M < 1 || a.M > 4) return false;
+    if (a.mode != QMM_MODE_AFFINE || (a.bits != 2 && a.bits != 4 && a.bits != 8)) return false;
     if (dt != QMM_BF16 && dt != QMM_F16) return false;
     const int epu = 128 / a.bits;
     if (a.K % epu != 0 || a.group_size < epu) return false;

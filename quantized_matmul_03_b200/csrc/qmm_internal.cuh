@@ -15,6 +15,9 @@
 
 namespace qmm {
 
+// Quantization modes (the `mode` string of the C ABI).
+enum QmmMode { QMM_MODE_AFFINE = 0, QMM_MODE_MXFP4 = 1, QMM_MODE_MXFP8 = 2, QMM_MODE_NVFP4 = 3 };
+
 // ---------------------------------------------------------------------------
 // Storage dtypes: fp32 <-> T conversions, round-to-nearest-even on the way in.
 // ---------------------------------------------------------------------------
@@ -86,8 +89,10 @@ struct QuantArgs {
     int group_size, bits;
     uint32_t *wq;
     void *scales, *biases;
+    int mode = QMM_MODE_AFFINE;  // microscaled: scales are bytes, no biases
 };
 cudaError_t launch_quantize(qmm_dtype dt, const QuantArgs &a, cudaStream_t s);
+cudaError_t launch_quantize_mx(qmm_dtype dt, const QuantArgs &a, cudaStream_t s);
 
 struct DequantArgs {
     const uint32_t *wq;
@@ -95,8 +100,10 @@ struct DequantArgs {
     int64_t rows, cols;
     int group_size, bits;
     void *out;
+    int mode = QMM_MODE_AFFINE;
 };
 cudaError_t launch_dequantize(qmm_dtype dt, const DequantArgs &a, cudaStream_t s);
+cudaError_t launch_dequantize_mx(qmm_dtype dt, const DequantArgs &a, cudaStream_t s);
 
 // One quantized product y[M, N] = x[M, K] (*) W.
 struct QmmArgs {
@@ -109,12 +116,26 @@ struct QmmArgs {
     bool transpose;
     void *ws = nullptr;  // stream-K workspace (zeroed flags first), or null
     size_t ws_bytes = 0;
+    // Layer bias added before the output is rounded (quantized_dense):
+    // y[m, n] += bias[n] (if bias) + bias_value.
+    const void *bias = nullptr;
+    float bias_value = 0.f;
+    int mode = QMM_MODE_AFFINE;  // microscaled: scales are bytes, biases null
 };
+
+// Bias term of output feature n: bias[n] (if any) plus the scalar.
+template <typename T>
+__device__ __forceinline__ float layer_bias(const void *bias, float value, int64_t n) {
+    return bias ? Dt<T>::to_f(static_cast<const T *>(bias)[n]) + value : value;
+}
 cudaError_t launch_gemv(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 bool gemv_supported(qmm_dtype dt, const QmmArgs &a);
 cudaError_t launch_gemv_fast(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a);
+cudaError_t launch_gemv_tc(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
+bool gemv_tc_supported(qmm_dtype dt, const QmmArgs &a);
 cudaError_t launch_gemm(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
+cudaError_t launch_mx_matmul(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);  // microscaled weights
 // Bytes of stream-K workspace the tensor-core path can use for these sizes
 // (0 when it would keep whole tiles).
 size_t gemm_workspace_size(qmm_dtype dt, int64_t M, int64_t K, int64_t N, bool transpose, int bits);

@@ -2,7 +2,8 @@
 //
 // Quantization runs along the last axis, one scale and one bias per
 // `group_size` consecutive elements, `bits`-bit codes packed 32/bits per
-// uint32 least-significant first (EMLX.Quantization, section quantize;
+// uint32 least-significant first (3- and 6-bit codes: back to back in the
+// row's bit stream, see quantize_chunk_kernel) (EMLX.Quantization, section quantize;
 // Emily.QuantizedWeight, section Layout; mlx-rs ops/quantization.rs,
 // quantize / dequantize).
 //
@@ -125,8 +126,103 @@ dequantize_kernel(const uint32_t *__restrict__ wq, const T *__restrict__ scales,
     store_elems<T, EPW>(out + word * EPW, o);
 }
 
+// 3- and 6-bit codes do not divide a word: element j of a row occupies bits
+// [j*bits, (j+1)*bits) of the row's bit stream, least significant first, so
+// 32 consecutive codes fill exactly `bits` words ("a chunk") and a chunk
+// never leaves its group (group_size >= 32).  One thread per chunk; the
+// group's min/max are reduced over its group_size/32 lanes.
+template <typename T, int BITS>
+__global__ void __launch_bounds__(256)
+quantize_chunk_kernel(const T *__restrict__ w, int64_t n_chunks, int tpg,
+                      uint32_t *__restrict__ wq, T *__restrict__ scales, T *__restrict__ biases) {
+    constexpr int QMAX = (1 << BITS) - 1;
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool valid = c < n_chunks;
+    float v[32];
+    if (valid) {
+        load_elems<T, 32>(w + c * 32, v);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+    }
+    float lo = v[0], hi = v[0];
+#pragma unroll
+    for (int j = 1; j < 32; ++j) {
+        lo = fminf(lo, v[j]);
+        hi = fmaxf(hi, v[j]);
+    }
+    for (int off = tpg >> 1; off > 0; off >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (!valid) return;
+    const float scale32 = __fdiv_rn(__fsub_rn(hi, lo), (float)QMAX);
+    const T s_t = Dt<T>::from_f(scale32);
+    const T b_t = Dt<T>::from_f(lo);
+    const float s = Dt<T>::to_f(s_t);
+    const float b = Dt<T>::to_f(b_t);
+    uint32_t out[BITS];
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) out[i] = 0u;
+    if (s != 0.f) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            int q = __float2int_rn(__fdiv_rn(__fsub_rn(v[j], b), s));
+            q = min(max(q, 0), QMAX);
+            const int bit = j * BITS, wi = bit >> 5, off = bit & 31;
+            out[wi] |= (uint32_t)q << off;
+            if (off + BITS > 32) out[wi + 1] |= (uint32_t)q >> (32 - off);
+        }
+    }
+    uint32_t *dst = wq + c * BITS;
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) dst[i] = out[i];
+    if ((threadIdx.x & (tpg - 1)) == 0) {
+        const int64_t g = c / tpg;
+        scales[g] = s_t;
+        biases[g] = b_t;
+    }
+}
+
+template <typename T, int BITS>
+__global__ void __launch_bounds__(256)
+dequantize_chunk_kernel(const uint32_t *__restrict__ wq, const T *__restrict__ scales,
+                        const T *__restrict__ biases, int64_t n_chunks, int tpg,
+                        T *__restrict__ out) {
+    constexpr uint32_t MASK = (1u << BITS) - 1u;
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= n_chunks) return;
+    const int64_t g = c / tpg;
+    const float s = Dt<T>::to_f(scales[g]);
+    const float b = Dt<T>::to_f(biases[g]);
+    uint32_t in[BITS];
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) in[i] = __ldg(wq + c * BITS + i);
+    T o[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const int bit = j * BITS, wi = bit >> 5, off = bit & 31;
+        uint32_t q = in[wi] >> off;
+        if (off + BITS > 32) q |= in[wi + 1] << (32 - off);
+        o[j] = Dt<T>::from_f(__fmaf_rn(s, (float)(q & MASK), b));
+    }
+    store_elems<T, 32>(out + c * 32, o);
+}
+
 template <typename T>
 cudaError_t quantize_t(const QuantArgs &a, cudaStream_t s) {
+    if (a.bits == 3 || a.bits == 6) {
+        const int64_t n_chunks = a.rows * (a.cols / 32);
+        const int tpg = a.group_size / 32;
+        const int64_t blocks = (n_chunks + 255) / 256;
+        auto w = static_cast<const T *>(a.w);
+        auto sc = static_cast<T *>(a.scales);
+        auto bi = static_cast<T *>(a.biases);
+        if (a.bits == 3) quantize_chunk_kernel<T, 3><<<blocks, 256, 0, s>>>(w, n_chunks, tpg, a.wq, sc, bi);
+        else quantize_chunk_kernel<T, 6><<<blocks, 256, 0, s>>>(w, n_chunks, tpg, a.wq, sc, bi);
+        count_launches(1);
+        return cudaGetLastError();
+    }
     const int epw = 32 / a.bits;
     const int64_t n_words = a.rows * (a.cols / epw);
     const int tpg = a.group_size / epw;
@@ -145,6 +241,18 @@ cudaError_t quantize_t(const QuantArgs &a, cudaStream_t s) {
 
 template <typename T>
 cudaError_t dequantize_t(const DequantArgs &a, cudaStream_t s) {
+    if (a.bits == 3 || a.bits == 6) {
+        const int64_t n_chunks = a.rows * (a.cols / 32);
+        const int tpg = a.group_size / 32;
+        const int64_t blocks = (n_chunks + 255) / 256;
+        auto sc = static_cast<const T *>(a.scales);
+        auto bi = static_cast<const T *>(a.biases);
+        auto out = static_cast<T *>(a.out);
+        if (a.bits == 3) dequantize_chunk_kernel<T, 3><<<blocks, 256, 0, s>>>(a.wq, sc, bi, n_chunks, tpg, out);
+        else dequantize_chunk_kernel<T, 6><<<blocks, 256, 0, s>>>(a.wq, sc, bi, n_chunks, tpg, out);
+        count_launches(1);
+        return cudaGetLastError();
+    }
     const int epw = 32 / a.bits;
     const int64_t n_words = a.rows * (a.cols / epw);
     const int tpg = a.group_size / epw;

@@ -56,10 +56,11 @@ def q(L, **kw):
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(bits=3), 2), (dict(bits=6), 2), (dict(bits=5), 1), (dict(bits=16), 1),
+    (dict(bits=5), 1), (dict(bits=16), 1),
     (dict(gs=48), 1), (dict(gs=16), 1), (dict(cols=96), 1), (dict(cols=0), 1),
-    (dict(rows=-1), 1), (dict(mode=b"nvfp4"), 2), (dict(mode=b"mxfp4"), 2),
-    (dict(mode=b"mxfp8"), 2), (dict(mode=b"bogus"), 1), (dict(dtype=7), 1),
+    (dict(rows=-1), 1), (dict(mode=b"nvfp4"), 1), (dict(mode=b"mxfp4"), 1),
+    (dict(mode=b"mxfp8", gs=32), 1), (dict(mode=b"mxfp4", gs=32), 1),
+    (dict(mode=b"bogus"), 1), (dict(dtype=7), 1),
     (dict(w=NULL), 1), (dict(wq=MISALIGNED), 1), (dict(b=NULL), 1),
 ])
 def test_quantize_rejects_before_launch(L, kw, status):
@@ -82,9 +83,12 @@ def mm(L, **kw):
 @pytest.mark.parametrize("kw,status", [
     (dict(K=96), 1), (dict(tr=0, N=96), 1), (dict(K=0), 1), (dict(M=-1), 1),
     (dict(b=NULL), 1), (dict(x=MISALIGNED), 1), (dict(y=NULL), 1),
-    (dict(mode=b"nvfp4"), 2), (dict(bits=3), 2), (dict(gs=256), 1),
+    (dict(mode=b"nvfp4"), 1), (dict(mode=b"nvfp4", gs=16), 1), (dict(bits=5), 1),
+    (dict(gs=256), 1),
 ])
 def test_matmul_rejects_before_launch(L, kw, status):
+    # (microscaled modes: a group size or bits other than the mode's, or a
+    # non-NULL biases pointer, are invalid arguments)
     assert mm(L, **kw) == status
 
 
@@ -109,7 +113,7 @@ def mmws(L, ws=NULL, ws_bytes=0, **kw):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(K=96), 1), (dict(tr=0, N=96), 1), (dict(b=NULL), 1), (dict(x=MISALIGNED), 1),
-    (dict(mode=b"nvfp4"), 2), (dict(bits=3), 2),
+    (dict(mode=b"nvfp4"), 1), (dict(bits=7), 1),
 ])
 def test_matmul_ws_rejects_like_the_plain_call(L, kw, status):
     assert mmws(L, **kw) == status
@@ -128,7 +132,7 @@ def test_matmul_workspace_size(L):
     need = ws(16, 4096, 4096)
     assert need > 4096                          # flags, then one partial slot per SM
     assert ws(64, 4096, 4096) == need and ws(1, 4096, 4096, tr=0) == need
-    assert ws(4, 4096, 4096) == 0               # decode rows go to the SIMT kernel
+    assert ws(4, 4096, 4096) == 0               # decode rows go to the SIMT decode kernel
     assert ws(128, 4096, 4096) == 0             # wide tiles keep whole tiles
     assert ws(64, 4096, 14336 * 4) == 0         # at least one full wave of tiles
     assert ws(16, 4096, 4096, dt=0) == 0        # f32 has no tensor-core path

@@ -33,10 +33,10 @@ def test_streamk_owner_wait_runs_out_then_recovers():
     wq, s, b = oracle.quantize(w, 64, 4)
     ref = oracle.quantized_matmul(x, wq, s, b, True, 64, 4)
     args = (x.cuda(), wq.cuda(), s.cuda(), b.cuda(), True, 64, 4)
+    qb.qmm_set_path("gemm")
     need = qb.qmm_quantized_matmul_workspace_size(m, k, n, True, 4, torch.bfloat16)
     assert need > 0
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
-    qb.qmm_set_path("gemm")
     qb.qmm_device_status()            # start from a clear error word
 
     qb.qmm_set_wait_limit_ns(100_000)  # 0.1 ms

@@ -199,6 +199,7 @@ def test_gemm_stream_k_workspace_options():
     x = wl.normal((16, 4096), seed=8, dtype=torch.bfloat16)
     wq, s, b = oracle.quantize(w, 64, 4)
     ref = oracle.quantized_matmul(x, wq, s, b, True, 64, 4)
+    qb.qmm_set_path("gemm")  # (the automatic path sends 16 rows of 4-bit codes to the decode kernel)
     need = qb.qmm_quantized_matmul_workspace_size(16, 4096, 1024, True, 4, torch.bfloat16)
     assert need > 0
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
