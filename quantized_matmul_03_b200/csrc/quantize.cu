@@ -7,11 +7,14 @@
 // Emily.QuantizedWeight, section Layout; mlx-rs ops/quantization.rs,
 // quantize / dequantize).
 //
-// Both kernels are HBM-bound streams: one thread per packed word, 16-byte
-// vector loads and stores, and the group min/max reduced across the
-// group_size/(32/bits) lanes that share a group with warp shuffles.  Every
-// floating-point step uses an explicitly rounded intrinsic so the result is
-// bit-identical to a sequential IEEE fp32 evaluation of the same rule.
+// Both kernels are HBM-bound streams with 16-byte vector loads and stores
+// (quantize: a thread per 16 bytes of codes; dequantize: a thread per packed
+// word), and the group min/max reduced across the lanes that share a group
+// with warp shuffles.  Every floating-point step uses an explicitly rounded
+// intrinsic so the result is bit-identical to a sequential IEEE fp32
+// evaluation of the same rule.
+#include <algorithm>
+
 #include "qmm_internal.cuh"
 
 namespace qmm {
@@ -52,32 +55,48 @@ __device__ __forceinline__ void store_elems(T *__restrict__ p, const T (&t)[N]) 
     }
 }
 
-// One thread per packed word; `tpg` = words per group (a power of two <= 32),
-// so the lanes of one group are contiguous and aligned within the warp.
-template <typename T, int BITS>
+// The code of one element: rint((v - b) / s) clamped to [0, QMAX], with the
+// quotient correctly rounded (IEEE division) as the rule states.  A product
+// with the rounded reciprocal differs from that quotient by at most a couple
+// of units in the last place, which can change rint only next to a half
+// integer; the exact division runs there (and for non-finite products), so
+// the result is the division's in every case.
+__device__ __forceinline__ int code_of(float v, float b, float s, float r, int qmax) {
+    const float t = __fsub_rn(v, b);
+    const float y = __fmul_rn(t, r);
+    const float f = y - floorf(y);
+    const float q = fabsf(f - 0.5f) > 1e-3f ? y : __fdiv_rn(t, s);
+    return min(max(__float2int_rn(q), 0), qmax);
+}
+
+// One thread per WPT packed words (16 bytes of codes when a group holds that
+// many); `tpg` = threads per group (a power of two <= 32), so the lanes of one
+// group are contiguous and aligned within the warp.
+template <typename T, int BITS, int WPT>
 __global__ void __launch_bounds__(256)
-quantize_kernel(const T *__restrict__ w, int64_t n_words, int tpg,
+quantize_kernel(const T *__restrict__ w, int64_t n_threads, int tpg,
                 uint32_t *__restrict__ wq, T *__restrict__ scales, T *__restrict__ biases) {
     constexpr int EPW = 32 / BITS;
+    constexpr int NE = EPW * WPT;  // elements per thread
     constexpr int QMAX = (1 << BITS) - 1;
-    const int64_t word = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const bool valid = word < n_words;
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool valid = tid < n_threads;
 
-    float v[EPW];
+    float v[NE];
     if (valid) {
-        load_elems<T, EPW>(w + word * EPW, v);
+        load_elems<T, NE>(w + tid * NE, v);
     } else {
 #pragma unroll
-        for (int j = 0; j < EPW; ++j) v[j] = 0.f;
+        for (int j = 0; j < NE; ++j) v[j] = 0.f;
     }
     float lo = v[0], hi = v[0];
 #pragma unroll
-    for (int j = 1; j < EPW; ++j) {
+    for (int j = 1; j < NE; ++j) {
         lo = fminf(lo, v[j]);
         hi = fmaxf(hi, v[j]);
     }
-    // Invalid lanes form whole groups (n_words is a multiple of tpg), and the
-    // xor partners of a lane stay inside its own group.
+    // Invalid lanes form whole groups (n_threads is a multiple of tpg), and
+    // the xor partners of a lane stay inside its own group.
     for (int off = tpg >> 1; off > 0; off >>= 1) {
         lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
         hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
@@ -89,19 +108,29 @@ quantize_kernel(const T *__restrict__ w, int64_t n_words, int tpg,
     const T b_t = Dt<T>::from_f(lo);
     const float s = Dt<T>::to_f(s_t);
     const float b = Dt<T>::to_f(b_t);
+    const float r = __frcp_rn(s);
 
-    uint32_t packed = 0;
+    uint32_t packed[WPT];
+#pragma unroll
+    for (int k = 0; k < WPT; ++k) packed[k] = 0u;
     if (s != 0.f) {
 #pragma unroll
-        for (int j = 0; j < EPW; ++j) {
-            int q = __float2int_rn(__fdiv_rn(__fsub_rn(v[j], b), s));
-            q = min(max(q, 0), QMAX);
-            packed |= (uint32_t)q << (j * BITS);
+        for (int k = 0; k < WPT; ++k) {
+#pragma unroll
+            for (int j = 0; j < EPW; ++j)
+                packed[k] |= (uint32_t)code_of(v[k * EPW + j], b, s, r, QMAX) << (j * BITS);
         }
     }
-    wq[word] = packed;
+    uint32_t *dst = wq + tid * WPT;
+    if constexpr (WPT == 4) {
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    } else if constexpr (WPT == 2) {
+        *reinterpret_cast<uint2 *>(dst) = make_uint2(packed[0], packed[1]);
+    } else {
+        dst[0] = packed[0];
+    }
     if ((threadIdx.x & (tpg - 1)) == 0) {
-        const int64_t g = word / tpg;
+        const int64_t g = tid / tpg;
         scales[g] = s_t;
         biases[g] = b_t;
     }
@@ -224,17 +253,24 @@ cudaError_t quantize_t(const QuantArgs &a, cudaStream_t s) {
         return cudaGetLastError();
     }
     const int epw = 32 / a.bits;
-    const int64_t n_words = a.rows * (a.cols / epw);
-    const int tpg = a.group_size / epw;
-    const int64_t blocks = (n_words + 255) / 256;
+    const int words_per_group = a.group_size / epw;
+    // 4 words (16 bytes of codes) per thread, fewer when a group is smaller
+    // (2-bit codes, group size 32: 2 words).
+    const int wpt = std::min(4, words_per_group);
+    const int64_t n_threads = a.rows * (a.cols / epw) / wpt;
+    const int tpg = words_per_group / wpt;
+    const int64_t blocks = (n_threads + 255) / 256;
     auto w = static_cast<const T *>(a.w);
     auto sc = static_cast<T *>(a.scales);
     auto bi = static_cast<T *>(a.biases);
-    switch (a.bits) {
-    case 2: quantize_kernel<T, 2><<<blocks, 256, 0, s>>>(w, n_words, tpg, a.wq, sc, bi); break;
-    case 4: quantize_kernel<T, 4><<<blocks, 256, 0, s>>>(w, n_words, tpg, a.wq, sc, bi); break;
-    default: quantize_kernel<T, 8><<<blocks, 256, 0, s>>>(w, n_words, tpg, a.wq, sc, bi); break;
-    }
+    if (a.bits == 2 && wpt == 2)
+        quantize_kernel<T, 2, 2><<<blocks, 256, 0, s>>>(w, n_threads, tpg, a.wq, sc, bi);
+    else if (a.bits == 2)
+        quantize_kernel<T, 2, 4><<<blocks, 256, 0, s>>>(w, n_threads, tpg, a.wq, sc, bi);
+    else if (a.bits == 4)
+        quantize_kernel<T, 4, 4><<<blocks, 256, 0, s>>>(w, n_threads, tpg, a.wq, sc, bi);
+    else
+        quantize_kernel<T, 8, 4><<<blocks, 256, 0, s>>>(w, n_threads, tpg, a.wq, sc, bi);
     count_launches(1);
     return cudaGetLastError();
 }

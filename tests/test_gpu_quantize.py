@@ -67,6 +67,35 @@ def test_invalid_args_raise():
     with pytest.raises(qb.QmmError) as e:
         qb.qmm_quantize(w, 64, 4)
     assert e.value.status == 1
-    with pytest.raises(qb.QmmError) as e:
+    with pytest.raises(qb.QmmError) as e:      # nvfp4 fixes group_size 16
         qb.qmm_quantize(w, 32, 4, mode="nvfp4")
-    assert e.value.status == 2
+    assert e.value.status == 1
+    with pytest.raises(qb.QmmError) as e:      # bits 5 is no format
+        qb.qmm_quantize(w, 32, 5)
+    assert e.value.status == 1
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_quantize_codes_on_and_next_to_ties(dtype, bits):
+    """Elements whose quotient (v - b) / s lies exactly on a half integer or a
+    few units in the last place from one: the code must be the rounded IEEE
+    quotient's, ties to even, in every group."""
+    qmax = (1 << bits) - 1
+    g = torch.Generator().manual_seed(bits)
+    rows = []
+    for r in range(64):
+        lo = float(torch.randn(1, generator=g)) * 10 ** (r % 7 - 3)
+        step = float(torch.rand(1, generator=g) + 0.05) * 10 ** (r % 5 - 2)
+        if r % 4 == 0:          # power-of-two step: s and b exact, so exact ties
+            step = 2.0 ** (r % 9 - 4)
+            lo = -float(r) * step
+        row = torch.empty(128, dtype=torch.float64)
+        row[0], row[1] = lo, lo + qmax * step
+        k = torch.randint(0, qmax, (126,), generator=g).double()
+        nudge = torch.tensor([0.0, 1e-7, -1e-7, 1e-6, -1e-6, 1e-4, -1e-4, 2e-3, -2e-3] * 14)
+        row[2:] = lo + (k + 0.5 + nudge) * step
+        rows.append(row)
+    w = torch.stack(rows).to(dtype)
+    check_quantize(w, 64, bits)
+    check_quantize(w, 32, bits)
