@@ -47,6 +47,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "mx.cuh"
 #include "ptx_sm100.cuh"
 #include "qmm_internal.cuh"
 #include "tcgen05.cuh"
@@ -64,6 +65,14 @@ constexpr int kThreads = 32 * (kWarpTmaS + 1);  // 512
 constexpr int kBM = 128;                        // weight rows per tile (UMMA M)
 constexpr int kBK = 64;                         // k per stage: one 128-byte swizzle row
 constexpr int kSkMaxBN = 64;                    // widest tile that stream-K splits
+// Packed tile of one k-block, [N, K] layout: 128 rows of kBK*bits/8 bytes
+// (3-bit codes: 24 bytes, which no tensor copy can start on for odd k-blocks,
+// so a 32-byte box from the 16-byte boundary below is staged instead).
+// [K, N] layout: 64 k-rows of 128*bits/8 bytes.
+constexpr int packed_pitch(int bits) { return bits == 3 ? 32 : kBK * bits / 8; }
+constexpr int packed_stage_bytes(int bits, bool kmajor) {
+    return kmajor ? kBM * packed_pitch(bits) : kBK * kBM * bits / 8;
+}
 
 // ---------------------------------------------------------------------------
 // Dequantization of a half k-block of one weight row (32 codes) into four
@@ -93,12 +102,41 @@ template <> struct Pair<__half> {
     }
 };
 
+// 3- and 6-bit codes: the 32 codes fill BITS words as one bit stream, code j
+// at bits [j*BITS, (j+1)*BITS), so a pair of codes (2i, 2i+1) is the 2*BITS
+// bits from bit 2i*BITS, which may straddle two words (one funnel shift).
+// The pair goes to the two 16-bit halves, then the magic-number conversion.
+template <typename T, int BITS>
+__device__ __forceinline__ void dequant_half_stream(const uint32_t *w, uint16_t s16, uint16_t b16,
+                                                    uint4 (&out)[4]) {
+    using P = Pair<T>;
+    using V2 = typename P::V2;
+    constexpr uint32_t M = (1u << BITS) - 1u;
+    const V2 s2 = P::splat(s16), b2 = P::splat(b16), off = P::off();
+    uint32_t vals[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int pos = 2 * i * BITS, wi = pos >> 5, sh = pos & 31;
+        const uint32_t u = sh + 2 * BITS <= 32 ? (w[wi] >> sh) : __funnelshift_r(w[wi], w[wi + 1], sh);
+        const uint32_t t = (u & M) | ((u << (16 - BITS)) & (M << 16)) | P::MAGIC;
+        vals[i] = P::ubits(__hfma2(__hsub2(P::bits(t), off), s2, b2));
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        out[c] = make_uint4(vals[4 * c], vals[4 * c + 1], vals[4 * c + 2], vals[4 * c + 3]);
+}
+
 // Magic-number path (4- and 2-bit codes; 8-bit codes with f16): OR a code
 // into the mantissa of OFF (exact), subtract OFF (exact), then s*q + b.
-// Produces 16-bit values in k order, 8 per output uint4.
+// Produces 16-bit values in k order, 8 per output uint4.  (3- and 6-bit
+// codes: dequant_half_stream.)
 template <typename T, int BITS>
 __device__ __forceinline__ void dequant_half(const uint32_t *w, uint16_t s16, uint16_t b16,
                                              uint4 (&out)[4]) {
+    if constexpr (BITS == 3 || BITS == 6) {
+        dequant_half_stream<T, BITS>(w, s16, b16, out);
+        return;
+    } else {
     using P = Pair<T>;
     using V2 = typename P::V2;
     constexpr int EPW = 32 / BITS;                 // codes per word
@@ -129,6 +167,7 @@ __device__ __forceinline__ void dequant_half(const uint32_t *w, uint16_t s16, ui
 #pragma unroll
     for (int c = 0; c < 4; ++c)
         out[c] = make_uint4(vals[4 * c], vals[4 * c + 1], vals[4 * c + 2], vals[4 * c + 3]);
+    }
 }
 
 // 8-bit codes with bf16 (no exact bf16 magic for 0..255): fp32 magic.
@@ -148,6 +187,38 @@ __device__ __forceinline__ void dequant_half<__nv_bfloat16, 8>(const uint32_t *w
         __nv_bfloat162 lo = __floats2bfloat162_rn(f[0], f[1]), hi = __floats2bfloat162_rn(f[2], f[3]);
         vals[2 * wi] = *reinterpret_cast<uint32_t *>(&lo);
         vals[2 * wi + 1] = *reinterpret_cast<uint32_t *>(&hi);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        out[c] = make_uint4(vals[4 * c], vals[4 * c + 1], vals[4 * c + 2], vals[4 * c + 3]);
+}
+
+// Microscaled weights (mxfp4/nvfp4: E2M1 codes, mxfp8: E4M3 codes): 32
+// elements of one row as 16-bit values X * element, exact (both factors are
+// exact in 16 bits and so is their product); x0 scales elements 0..15, x1
+// elements 16..31 (equal unless the group size is 16).
+template <typename T, int MODE>
+__device__ __forceinline__ void dequant_half_mx(const uint32_t *w, float x0, float x1, uint4 (&out)[4]) {
+    constexpr int NW = MODE == QMM_MODE_MXFP8 ? 8 : 4;  // words per 32 elements
+    uint32_t vals[16];
+#pragma unroll
+    for (int wi = 0; wi < NW; ++wi) {
+        float e[32 / NW];  // elements of one word
+        mxf::elements<MODE>(w[wi], e);
+        const float x = wi < NW / 2 ? x0 : x1;
+#pragma unroll
+        for (int i = 0; i < 16 / NW; ++i) {
+            const float a = __fmul_rn(x, e[2 * i]), b = __fmul_rn(x, e[2 * i + 1]);
+            uint32_t pr;
+            if constexpr (std::is_same<T, __half>::value) {
+                const __half2 h = __floats2half2_rn(a, b);
+                pr = *reinterpret_cast<const uint32_t *>(&h);
+            } else {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+                pr = *reinterpret_cast<const uint32_t *>(&h);
+            }
+            vals[wi * (16 / NW) + i] = pr;
+        }
     }
 #pragma unroll
     for (int c = 0; c < 4; ++c)
@@ -279,22 +350,28 @@ struct Work {
 // of row k and writes them as 16-byte chunks of an MN-major, 128-byte-swizzled
 // A tile (atoms of 64 features x 8 k-rows), which the MMA reads with the
 // A-major bit set.  Everything else is shared with the K-major path.
-template <typename T, int BITS, int BN, bool GROUPED, bool KMAJOR = true>
+// MODE: affine (scale and bias windows, 16-bit) or a microscaled mode
+// (scale bytes only: windows of 16 groups; [N, K] layout, not grouped).
+template <typename T, int BITS, int BN, bool GROUPED, bool KMAJOR = true, int MODE = QMM_MODE_AFFINE>
 __global__ void __launch_bounds__(kThreads, 1)
 qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_xs,
                 const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_s,
                 const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_y,
                 const GemmParams p) {
     static_assert(KMAJOR || !GROUPED, "the grouped product is built for the [N, K] layout");
+    constexpr bool MX = MODE != QMM_MODE_AFFINE;
+    static_assert(!MX || (KMAJOR && !GROUPED), "microscaled weights: [N, K] layout, not grouped");
     constexpr bool kF16 = std::is_same<T, __half>::value;
     constexpr int A_BYTES = kBM * kBK * 2;         // 16 KB dequantized tile
     constexpr int B_BYTES = BN * kBK * 2;          // activation tile
-    constexpr int P_ROW = kBK * BITS / 8;          // packed bytes per row per k-block
-    constexpr int P_BYTES = kBM * P_ROW;
+    constexpr int P_ROW = packed_pitch(BITS);      // staged packed bytes per row per k-block
+    constexpr int P_BYTES = packed_stage_bytes(BITS, KMAJOR);
     constexpr int W_WORDS = kBK * BITS / 32;       // packed words per row per k-block
     // [N, K] layout: the dequantized tile goes to tensor memory (A operand of
     // the MMA) instead of shared memory.  512 columns: accumulators (two
     // buffers, or one of 256 columns) then a ring of 32-column A slots.
+    // (Shared-memory A measured slower at every tile width, narrow tiles
+    // included: 16 activation rows, 14336 x 4096 int4: 26.8 against 24.4 us.)
     constexpr bool TS = KMAJOR && !GROUPED;
     constexpr int NACC = (TS && 2 * BN > 256) ? 1 : 2;
     constexpr uint32_t A_COL0 = NACC * BN < 32 ? 32 : NACC * BN;
@@ -396,10 +473,18 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 // Packed row kl (16*BITS bytes, unswizzled), half h.
                 const uint8_t *prow = pg + s * P_BYTES + kl * (16 * BITS) + h * (8 * BITS);
                 uint32_t w[2 * BITS];
+                if constexpr (BITS == 3) {  // 24 bytes, 8-byte aligned
 #pragma unroll
-                for (int q = 0; q < BITS / 2; ++q) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(prow + 16 * q);
-                    w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
+                    for (int q = 0; q < 3; ++q) {
+                        const uint2 u = *reinterpret_cast<const uint2 *>(prow + 8 * q);
+                        w[2 * q] = u.x; w[2 * q + 1] = u.y;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < BITS / 2; ++q) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(prow + 16 * q);
+                        w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
+                    }
                 }
                 // A stage s is free: its refill (full_p above) waited for the
                 // MMAs of k-block c - S.
@@ -479,7 +564,14 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     scale_bias(g1, s1, b1v);
                 }
                 ptx::mbar_wait(full_p + 8 * s, rp.phase, p.err);
-                if (p.sb_tma) {
+                float mx[4] = {0.f, 0.f, 0.f, 0.f};  // microscaled: scales of elements 16i..16i+15
+                if constexpr (MX) {
+                    // Row r's window of 16 scale bytes starts at group (g & ~15).
+                    const uint8_t *sw = gbase + (sb0 - base) + s * SB_BYTES + r * 16;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        mx[i] = mxf::scale_value<MODE>(sw[((kb * kBK + 16 * i) >> gs_log) & 15]);
+                } else if (p.sb_tma) {
                     // Row r's window of 8 groups starts at group (g0 & ~7).
                     const uint8_t *sw = gbase + (sb0 - base) + s * SB_BYTES + r * 16;
                     const int o0 = (g0 & 7) * 2, o1 = (g1 - (g0 & ~7)) * 2;
@@ -491,12 +583,31 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                 // The packed tile was staged with the swizzle matching its row
                 // width (none / 32B / 64B): 16-byte chunk q of row r sits at
                 // chunk q ^ ((r >> 2) & 1) (32-byte rows) or q ^ ((r >> 1) & 3)
-                // (64-byte rows).
+                // (64-byte rows); 48-byte rows (6-bit codes) are unswizzled.
                 const uint8_t *prow = pg + s * P_BYTES + r * P_ROW;
                 uint32_t w[2 * BITS];  // 64 codes
                 if constexpr (BITS == 2) {
                     const uint4 u = *reinterpret_cast<const uint4 *>(prow);
                     w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+                } else if constexpr (BITS == 3) {
+                    // 32-byte row staged from word (6 kb) & ~3: the k-block's six
+                    // words start at word 0 (even kb) or 2 (odd kb).
+                    const int x = (r >> 2) & 1;
+                    uint32_t a8[8];
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(prow + ((q ^ x) << 4));
+                        a8[4 * q] = u.x; a8[4 * q + 1] = u.y; a8[4 * q + 2] = u.z; a8[4 * q + 3] = u.w;
+                    }
+                    const bool odd = (kb & 1) != 0;
+#pragma unroll
+                    for (int i = 0; i < 6; ++i) w[i] = odd ? a8[i + 2] : a8[i];
+                } else if constexpr (BITS == 6) {
+#pragma unroll
+                    for (int q = 0; q < 3; ++q) {
+                        const uint4 u = *reinterpret_cast<const uint4 *>(prow + 16 * q);
+                        w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
+                    }
                 } else if constexpr (BITS == 4) {
                     const int x = (r >> 2) & 1;
 #pragma unroll
@@ -517,7 +628,8 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         uint4 out[4];
-                        dequant_half<T, BITS>(w + hh * BITS, hh ? s1 : s0, hh ? b1v : b0v, out);
+                        if constexpr (MX) dequant_half_mx<T, MODE>(w + hh * BITS, mx[2 * hh], mx[2 * hh + 1], out);
+                        else dequant_half<T, BITS>(w + hh * BITS, hh ? s1 : s0, hh ? b1v : b0v, out);
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             v[16 * hh + 4 * j] = out[j].x;
@@ -745,13 +857,20 @@ qgemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     if (role == 0) {
                         ptx::mbar_arrive_expect_tx(fb, P_BYTES);
                         if constexpr (KMAJOR)
-                            tma_load_2d(p0 + s * P_BYTES, &tmap_w, kb * W_WORDS, t.wrow0, fb);
+                            tma_load_2d(p0 + s * P_BYTES, &tmap_w, BITS == 3 ? (kb * W_WORDS) & ~3 : kb * W_WORDS,
+                                        t.wrow0, fb);
                         else  // 64 k-rows x 128 features of the [K, N] packed weight
                             tma_load_2d(p0 + s * P_BYTES, &tmap_w, t.n0 * BITS / 32, kb * kBK, fb);
                     } else if (role == 1) {
                         ptx::mbar_arrive_expect_tx(fb, bbytes);
                         for (int j = 0; j < nbox; ++j)
                             tma_load_2d(b0 + s * B_BYTES + j * 64 * kBK * 2, xmap, kb * kBK, t.m0 + 64 * j, fb);
+                    } else if constexpr (MX) {
+                        // the 16 scale bytes (8 two-byte units of the map) holding
+                        // this k-block's groups; no biases
+                        ptx::mbar_arrive_expect_tx(fb, SB_BYTES / 2);
+                        const int wx = (((kb * kBK) >> gs_log) >> 4) << 3;
+                        tma_load_2d(sb0 + s * SB_BYTES, &tmap_s, wx, t.wrow0, fb);
                     } else {
                         // the window of 8 groups holding this k-block's groups
                         ptx::mbar_arrive_expect_tx(fb, SB_BYTES);
@@ -848,9 +967,10 @@ int pick_bn(int64_t M) {
 
 // Shared-memory budget of one CTA: S stages of (A + B + P [+ scale/bias
 // windows]) plus barriers.
-template <int BITS, int BN>
+template <int BITS, int BN, bool KMAJOR = true>
 bool gemm_smem_plan(bool sb_tma, int &stages, size_t &smem, bool a_smem, size_t extra = 0) {
-    constexpr int A_BYTES = kBM * kBK * 2, B_BYTES = BN * kBK * 2, P_BYTES = kBM * kBK * BITS / 8;
+    constexpr int A_BYTES = kBM * kBK * 2, B_BYTES = BN * kBK * 2;
+    constexpr int P_BYTES = packed_stage_bytes(BITS, KMAJOR);
     const int STAGE = (a_smem ? A_BYTES : 0) + B_BYTES + P_BYTES + (sb_tma ? 2 * kBM * 16 : 0);
     constexpr size_t kSmemMax = 227 * 1024;
     const size_t fixed = 1024 /*alignment*/ + 64 /*acc bars + slot*/ + extra;
@@ -884,14 +1004,16 @@ CUtensorMapDataType act_type(bool f16) {
 }
 
 // Packed-weight map over `rows` stacked weight rows: one 128-row tile of one
-// k-block per box, swizzled to match its row width (8 / 32 / 64 bytes).
+// k-block per box (3-bit codes: 32 of the row's bytes, see packed_pitch),
+// swizzled to match its row width (16 / 32 / 64 bytes; 48 unswizzled).
 template <int BITS>
 bool make_weight_map(CUtensorMap *map, const uint32_t *wq, uint64_t rows, int64_t K) {
     const uint64_t words = (uint64_t)K * BITS / 32;
+    const CUtensorMapSwizzle sw = (BITS == 2 || BITS == 6) ? CU_TENSOR_MAP_SWIZZLE_NONE
+                                  : BITS == 8              ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                           : CU_TENSOR_MAP_SWIZZLE_32B;
     return make_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, wq, words, rows, words * 4,
-                       kBK * BITS / 32, kBM,
-                       BITS == 2 ? CU_TENSOR_MAP_SWIZZLE_NONE
-                                 : (BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B));
+                       packed_pitch(BITS) / 4, kBM, sw);
 }
 
 // Packed weight stored [K, N]: one 64 k-row x 128-feature tile per box
@@ -907,16 +1029,20 @@ bool make_weight_map_kn(CUtensorMap *map, const uint32_t *wq, int64_t K, int64_t
 // flags first, 4 per SM (a fixed place, so that calls of any shape find them
 // zero), then one fp32 partial tile slot per SM of 128 x 64 values (stream-K
 // runs only tiles of at most 64 activation rows).
-constexpr size_t kSkFlagBytes = 4096;
+constexpr size_t kSkFlagBytes = kWsFlagBytes;
 size_t sk_workspace_bytes() { return kSkFlagBytes + (size_t)num_sms() * kBM * kSkMaxBN * sizeof(float); }
 
-template <typename T, int BITS, int BN, bool KMAJOR>
+template <typename T, int BITS, int BN, bool KMAJOR, int MODE = QMM_MODE_AFFINE>
 cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
+    constexpr bool MX = MODE != QMM_MODE_AFFINE;
+    constexpr bool a_smem = !KMAJOR;  // [K, N]: MN-major A tile in shared memory
     const int64_t gpr = a.K / a.group_size;
-    // [N, K] layout: A lives in tensor memory, scale/bias windows come by
-    // TMA, and the output is staged for tensor stores when the ring keeps at
-    // least 4 stages (whole tile, else half of it per store).
-    const bool sb_tma = KMAJOR && gpr % 8 == 0;
+    // [N, K] layout: scale/bias windows come by TMA, and the output is staged
+    // for tensor stores when the ring keeps at least 4 stages (whole tile,
+    // else half of it per store).  Microscaled weights: windows of 16 scale
+    // bytes (rows of whole 16-byte units).
+    const bool sb_tma = KMAJOR && (MX ? gpr % 16 == 0 : gpr % 8 == 0);
+    if (MX && !sb_tma) return cudaErrorInvalidValue;
     int stages = 0, stg_rows = 0;
     size_t smem = 0;
     // (The [K, N] layout stages only narrow tiles, which stream-K may split;
@@ -925,11 +1051,11 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
                       (reinterpret_cast<uintptr_t>(a.y) & 15) == 0;
     if (y_ok) {
         for (int rows = BN; rows >= 16 && stg_rows == 0; rows /= 2)
-            if (gemm_smem_plan<BITS, BN>(sb_tma, stages, smem, !KMAJOR, (size_t)kEpiWarps * 64 * rows) &&
+            if (gemm_smem_plan<BITS, BN, KMAJOR>(sb_tma, stages, smem, a_smem, (size_t)kEpiWarps * 64 * rows) &&
                 stages >= 4)
                 stg_rows = rows;
     }
-    if (stg_rows == 0 && !gemm_smem_plan<BITS, BN>(sb_tma, stages, smem, !KMAJOR))
+    if (stg_rows == 0 && !gemm_smem_plan<BITS, BN, KMAJOR>(sb_tma, stages, smem, a_smem))
         return cudaErrorInvalidConfiguration;
     constexpr bool kF16 = std::is_same<T, __half>::value;
     CUtensorMap tx, tw, ts, tb, ty;
@@ -939,7 +1065,11 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
     if (KMAJOR ? !make_weight_map<BITS>(&tw, a.wq, (uint64_t)a.N, a.K)
                : !make_weight_map_kn<BITS>(&tw, a.wq, a.K, a.N))
         return cudaErrorInvalidValue;
-    if (sb_tma) {
+    if (MX) {
+        // the scale bytes read as two-byte units: [N, gpr / 2], 8 units per box
+        if (!make_sb_map(&ts, a.scales, (uint64_t)a.N, gpr / 2)) return cudaErrorInvalidValue;
+        tb = ts;  // unused
+    } else if (sb_tma) {
         if (!make_sb_map(&ts, a.scales, (uint64_t)a.N, gpr) || !make_sb_map(&tb, a.biases, (uint64_t)a.N, gpr))
             return cudaErrorInvalidValue;
     } else {
@@ -995,7 +1125,7 @@ cudaError_t run_gemm_layout(const QmmArgs &a, cudaStream_t s) {
             grid = (int)((total + len - 1) / len);
         }
     }
-    auto kern = qgemm_tc_kernel<T, BITS, BN, false, KMAJOR>;
+    auto kern = qgemm_tc_kernel<T, BITS, BN, false, KMAJOR, MODE>;
     struct Tag;
     cudaError_t e = configure_once<Tag>(smem, [&]() {
         return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1069,6 +1199,28 @@ cudaError_t run_gemm_grouped(const GroupedArgs &g, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// Microscaled weights, [N, K] layout.
+template <typename T, int MODE>
+cudaError_t gemm_mx(const QmmArgs &a, cudaStream_t s) {
+    constexpr int BITS = MODE == QMM_MODE_MXFP8 ? 8 : 4;
+    switch (pick_bn(a.M)) {
+    case 16: return run_gemm_layout<T, BITS, 16, true, MODE>(a, s);
+    case 32: return run_gemm_layout<T, BITS, 32, true, MODE>(a, s);
+    case 64: return run_gemm_layout<T, BITS, 64, true, MODE>(a, s);
+    case 128: return run_gemm_layout<T, BITS, 128, true, MODE>(a, s);
+    default: return run_gemm_layout<T, BITS, 256, true, MODE>(a, s);
+    }
+}
+
+template <typename T>
+cudaError_t gemm_mx_dtype(const QmmArgs &a, cudaStream_t s) {
+    switch (a.mode) {
+    case QMM_MODE_MXFP4: return gemm_mx<T, QMM_MODE_MXFP4>(a, s);
+    case QMM_MODE_MXFP8: return gemm_mx<T, QMM_MODE_MXFP8>(a, s);
+    default: return gemm_mx<T, QMM_MODE_NVFP4>(a, s);
+    }
+}
+
 template <typename T, int BITS>
 cudaError_t gemm_bits(const QmmArgs &a, cudaStream_t s) {
     switch (pick_bn(a.M)) {
@@ -1096,7 +1248,13 @@ cudaError_t grouped_bits(const GroupedArgs &g, cudaStream_t s) {
 // [K, N] storage), sizes in int range.
 bool gemm_supported(qmm_dtype dt, const QmmArgs &a) {
     if (dt != QMM_BF16 && dt != QMM_F16) return false;
-    if (a.mode != QMM_MODE_AFFINE || (a.bits != 2 && a.bits != 4 && a.bits != 8)) return false;
+    if (a.mode != QMM_MODE_AFFINE) {
+        // microscaled weights: [N, K] layout, scale rows of whole 16-byte units
+        if (!a.transpose || (a.K / a.group_size) % 16 != 0 || a.K % kBK != 0) return false;
+        if (a.M > INT32_MAX / 2 || a.N > INT32_MAX / 2 || a.K > INT32_MAX / 2) return false;
+        return encode_fn() != nullptr;
+    }
+    if (a.bits < 2 || a.bits > 8 || a.bits == 5 || a.bits == 7) return false;
     if (a.K % kBK != 0) return false;
     if (((a.transpose ? a.K : a.N) * a.bits / 8) % 16 != 0) return false;
     if (a.M > INT32_MAX / 2 || a.N > INT32_MAX / 2 || a.K > INT32_MAX / 2) return false;
@@ -1113,23 +1271,29 @@ size_t gemm_workspace_size(qmm_dtype dt, int64_t M, int64_t K, int64_t N, bool t
 }
 
 cudaError_t launch_gemm(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
+    if (a.mode != QMM_MODE_AFFINE)
+        return dt == QMM_BF16 ? gemm_mx_dtype<__nv_bfloat16>(a, s) : gemm_mx_dtype<__half>(a, s);
     if (dt == QMM_BF16) {
         switch (a.bits) {
         case 2: return gemm_bits<__nv_bfloat16, 2>(a, s);
+        case 3: return gemm_bits<__nv_bfloat16, 3>(a, s);
         case 4: return gemm_bits<__nv_bfloat16, 4>(a, s);
+        case 6: return gemm_bits<__nv_bfloat16, 6>(a, s);
         default: return gemm_bits<__nv_bfloat16, 8>(a, s);
         }
     }
     switch (a.bits) {
     case 2: return gemm_bits<__half, 2>(a, s);
+    case 3: return gemm_bits<__half, 3>(a, s);
     case 4: return gemm_bits<__half, 4>(a, s);
+    case 6: return gemm_bits<__half, 6>(a, s);
     default: return gemm_bits<__half, 8>(a, s);
     }
 }
 
 bool gemm_grouped_supported(qmm_dtype dt, const GroupedArgs &g) {
     if (!g.transpose) return false;
-    if (g.bits != 2 && g.bits != 4 && g.bits != 8) return false;
+    if (g.bits < 2 || g.bits > 8 || g.bits == 5 || g.bits == 7) return false;
     if (dt != QMM_BF16 && dt != QMM_F16) return false;
     if (g.K % kBK != 0) return false;
     if ((g.K * g.bits / 8) % 16 != 0) return false;
@@ -1143,13 +1307,17 @@ cudaError_t launch_gemm_grouped(qmm_dtype dt, const GroupedArgs &g, cudaStream_t
     if (dt == QMM_BF16) {
         switch (g.bits) {
         case 2: return grouped_bits<__nv_bfloat16, 2>(g, s);
+        case 3: return grouped_bits<__nv_bfloat16, 3>(g, s);
         case 4: return grouped_bits<__nv_bfloat16, 4>(g, s);
+        case 6: return grouped_bits<__nv_bfloat16, 6>(g, s);
         default: return grouped_bits<__nv_bfloat16, 8>(g, s);
         }
     }
     switch (g.bits) {
     case 2: return grouped_bits<__half, 2>(g, s);
+    case 3: return grouped_bits<__half, 3>(g, s);
     case 4: return grouped_bits<__half, 4>(g, s);
+    case 6: return grouped_bits<__half, 6>(g, s);
     default: return grouped_bits<__half, 8>(g, s);
     }
 }

@@ -20,7 +20,7 @@ namespace {
 template <int MODE> struct MxGeom;
 template <> struct MxGeom<QMM_MODE_MXFP4> { static constexpr int GS = 32, BITS = 4, EMAX = 2; };
 template <> struct MxGeom<QMM_MODE_MXFP8> { static constexpr int GS = 32, BITS = 8, EMAX = 8; };
-template <> struct MxGeom<QMM_MODE_NVFP4> { static constexpr int GS = 16, BITS = 4, EMAX = 2; };
+template <> struct MxGeom<QMM_MODE_NVFP4> { static constexpr int GS = 16, BITS = 4; };  // scale from amax / 6
 
 // floor(log2 a) of a finite a > 0 from its bits (subnormals included).
 __device__ __forceinline__ int ilog2f(float a) {

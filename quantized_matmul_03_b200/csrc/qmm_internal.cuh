@@ -54,6 +54,9 @@ __device__ __forceinline__ unsigned long long wait_limit_ns(const int *word) {
         reinterpret_cast<const char *>(word) + offsetof(DeviceState, wait_ns));
 }
 int *device_error_word();  // host: device address of the error word (current device)
+// Leading bytes of a matmul workspace that every call leaves zero (the
+// stream-K ready flags); other users of the workspace start past them.
+constexpr size_t kWsFlagBytes = 4096;
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s
 
 // Host-side test injection (qmm_inject_fault); read when a launch is built.
@@ -134,6 +137,7 @@ cudaError_t launch_gemv_fast(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a);
 cudaError_t launch_gemv_tc(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 bool gemv_tc_supported(qmm_dtype dt, const QmmArgs &a);
+size_t gemv_tc_workspace_bytes(int64_t K);
 cudaError_t launch_gemm(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 cudaError_t launch_mx_matmul(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);  // microscaled weights
 // Bytes of stream-K workspace the tensor-core path can use for these sizes

@@ -81,3 +81,71 @@ def test_gather_and_dense(bits):
                                True, 32, bits)
     qb.qmm_device_status()
     assert row_rel_err(y, ref) <= REL_TOL[torch.bfloat16]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("bits", [3, 6])
+@pytest.mark.parametrize("gs", [32, 64, 128])
+@pytest.mark.parametrize("transpose", [True, False])
+@pytest.mark.parametrize("m,n,k", [(5, 384, 512), (64, 1024, 1024), (300, 128, 512), (17, 1000, 2048)])
+def test_tensor_core_products(dtype, bits, gs, transpose, m, n, k):
+    """The tcgen05 GEMM with bit-stream codes: each 64-code k-block is BITS
+    words of a row (3-bit: staged as 32 bytes from the 16-byte boundary at or
+    below it), pairs of codes cut out with a funnel shift; both layouts."""
+    if not transpose and n % 128:
+        pytest.skip("[K, N] rows of whole 16-byte units need N % 128 == 0 for 3-bit codes")
+    rows, cols = (n, k) if transpose else (k, n)
+    w = wl.with_outliers((rows, cols), seed=m + n + bits + gs, dtype=dtype)
+    x = wl.normal((m, k), m + k + bits, 1.0, dtype)
+    wq, s, b = oracle.quantize(w, gs, bits)
+    ref = oracle.quantized_matmul(x, wq, s, b, transpose, gs, bits)
+    qb.qmm_set_path("gemm")
+    y = qb.qmm_quantized_matmul(x.cuda(), wq.cuda(), s.cuda(), b.cuda(), transpose, gs, bits)
+    qb.qmm_device_status()
+    assert row_rel_err(y, ref) <= REL_TOL[dtype]
+
+
+def test_three_bit_rows_not_in_16_byte_units():
+    """K = 576: a 3-bit row is 216 bytes, which a tensor map cannot stride, so
+    the forced tensor-core path refuses and the automatic choice takes the
+    SIMT kernel."""
+    w = wl.normal((256, 576), 80, 0.02, torch.bfloat16)
+    x = wl.normal((40, 576), 81, 1.0, torch.bfloat16)
+    wq, s, b = oracle.quantize(w, 64, 3)
+    ref = oracle.quantized_matmul(x, wq, s, b, True, 64, 3)
+    args = (x.cuda(), wq.cuda(), s.cuda(), b.cuda(), True, 64, 3)
+    qb.qmm_set_path("gemm")
+    with pytest.raises(qb.QmmError) as e:
+        qb.qmm_quantized_matmul(*args)
+    assert e.value.status == 2
+    qb.qmm_set_path("auto")
+    y = qb.qmm_quantized_matmul(*args)
+    qb.qmm_device_status()
+    assert row_rel_err(y, ref) <= REL_TOL[torch.bfloat16]
+
+
+@pytest.mark.parametrize("bits", [3, 6])
+def test_gather_on_tensor_cores(bits):
+    """gather_qmm with 256 tokens over 4 experts (grouped tcgen05 kernel)."""
+    w = wl.with_outliers((4, 512, 1024), seed=90 + bits, dtype=torch.bfloat16)
+    wq, s, b = oracle.quantize(w, 64, bits)
+    x = wl.normal((256, 1, 1024), 91 + bits, 1.0, torch.bfloat16)
+    rhs = wl.zipf_experts(256, 4, 1.2, 92 + bits)
+    ref = oracle.gather_qmm(x, wq, s, b, None, rhs, True, 64, bits)
+    y = qb.qmm_gather_qmm(x.cuda(), wq.cuda(), s.cuda(), b.cuda(), None, rhs.cuda(), True, 64, bits)
+    qb.qmm_device_status()
+    assert row_rel_err(y, ref) <= REL_TOL[torch.bfloat16]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("bits", [3, 6])
+def test_prefill_full_size_sampled(bits):
+    """x [2048, 4096] against W [14336, 4096] with 3-/6-bit codes, sampled rows
+    spread over the activation tiles."""
+    c = wl.prefill_case(4)
+    wq, s, b = oracle.quantize(c.w, 64, bits)
+    y = qb.qmm_quantized_matmul(c.x.cuda(), wq.cuda(), s.cuda(), b.cuda(), True, 64, bits)
+    torch.cuda.synchronize()
+    rows = torch.cat([torch.arange(0, 2048, 256) + o for o in (0, 1, 100, 255)])
+    ref = oracle.quantized_matmul(c.x[rows], wq, s, b, True, 64, bits)
+    assert row_rel_err(y.cpu()[rows], ref) <= REL_TOL[torch.bfloat16]

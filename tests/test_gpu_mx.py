@@ -151,3 +151,43 @@ def test_qqmm_arguments_are_checked():
     wq8, ws8, _ = qb.qmm_quantize(w, 32, 8, "mxfp8")
     args = (x.data_ptr(), 2, 64, 1, wq8.data_ptr(), ws8.data_ptr(), 16)
     assert L.qmm_qqmm(*args, 32, 8, b"mxfp8", y.data_ptr(), None, 0, None) == 6   # no workspace
+
+
+@pytest.fixture
+def _auto_path():
+    yield
+    qb.qmm_set_path("auto")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("m,n,k", [(5, 200, 512), (64, 300, 1024), (300, 128, 512), (17, 1000, 2048)])
+@pytest.mark.parametrize("path", ["gemm", "gemv"])
+def test_products_on_each_path(dtype, mode, m, n, k, path, _auto_path):
+    """Microscaled weights on the tensor-core GEMM (each 64-element k-block
+    dequantized exactly into tensor memory from E2M1/E4M3 codes and the
+    group scale bytes) and on the SIMT kernels."""
+    gs, bits = gb(mode)
+    w = wl.with_outliers((n, k), seed=m + n + bits, std=0.5, dtype=dtype)
+    x = wl.normal((m, k), m + k, 1.0, dtype)
+    wq, s, _ = oracle.quantize(w, gs, bits, mode)
+    ref = oracle.quantized_matmul(x, wq, s, None, True, gs, bits, mode)
+    qb.qmm_set_path(path)
+    y = qb.qmm_quantized_matmul(x.cuda(), wq.cuda(), s.cuda(), None, True, gs, bits, mode)
+    qb.qmm_device_status()
+    assert row_rel_err(y, ref) <= REL_TOL[dtype]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("mode", MODES)
+def test_prefill_full_size_sampled(mode):
+    """x [2048, 4096] against W [14336, 4096] in a microscaled mode, checked on
+    sampled rows spread over the activation tiles."""
+    gs, bits = gb(mode)
+    c = wl.prefill_case(4)
+    wq, s, _ = oracle.quantize(c.w, gs, bits, mode)
+    y = qb.qmm_quantized_matmul(c.x.cuda(), wq.cuda(), s.cuda(), None, True, gs, bits, mode)
+    torch.cuda.synchronize()
+    rows = torch.cat([torch.arange(0, 2048, 256) + o for o in (0, 1, 100, 255)])
+    ref = oracle.quantized_matmul(c.x[rows], wq, s, None, True, gs, bits, mode)
+    assert row_rel_err(y.cpu()[rows], ref) <= REL_TOL[torch.bfloat16]
