@@ -55,18 +55,63 @@ __device__ __forceinline__ void store_elems(T *__restrict__ p, const T (&t)[N]) 
     }
 }
 
-// The code of one element: rint((v - b) / s) clamped to [0, QMAX], with the
-// quotient correctly rounded (IEEE division) as the rule states.  A product
-// with the rounded reciprocal differs from that quotient by at most a couple
-// of units in the last place, which can change rint only next to a half
-// integer; the exact division runs there (and for non-finite products), so
-// the result is the division's in every case.
-__device__ __forceinline__ int code_of(float v, float b, float s, float r, int qmax) {
-    const float t = __fsub_rn(v, b);
-    const float y = __fmul_rn(t, r);
-    const float f = y - floorf(y);
-    const float q = fabsf(f - 0.5f) > 1e-3f ? y : __fdiv_rn(t, s);
-    return min(max(__float2int_rn(q), 0), qmax);
+// Two fp32 values in one 64-bit register, and the packed two-lane fp32
+// operations of sm_100 (each lane one IEEE operation, round to nearest even).
+__device__ __forceinline__ unsigned long long f2pack(float a, float b) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(unsigned long long v, float &a, float &b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long f2sub(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ unsigned long long f2mul(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ unsigned long long f2add(unsigned long long a, unsigned long long b) {
+    unsigned long long r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// The codes of two elements: rint((v - b) / s) clamped to [0, QMAX], with
+// the quotient correctly rounded (IEEE division) as the rule states.  A
+// product with the rounded reciprocal differs from that quotient by at most a
+// couple of units in the last place, which can change rint only next to a
+// half integer; the exact division runs there, so the result is the
+// division's in every case.  Clamping before rounding gives the same code
+// (outside [0, QMAX] both quotients end on the boundary code) and keeps the
+// value in the range where adding and subtracting 1.5 * 2^23 rounds it to an
+// integer (ties to even) and the sum's low bits hold that integer: full-rate
+// arithmetic, no conversion instructions, and the subtractions, products and
+// adds two lanes per instruction.  A NaN quotient gives code 0.
+__device__ __forceinline__ void code_pair(float v0, float v1, float b, float s, float r, float qmax,
+                                          uint32_t &c0, uint32_t &c1) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    const unsigned long long mm = f2pack(kMagic, kMagic);
+    const unsigned long long t = f2sub(f2pack(v0, v1), f2pack(b, b));
+    float y0, y1;
+    f2unpack(f2mul(t, f2pack(r, r)), y0, y1);
+    const unsigned long long y = f2pack(fminf(fmaxf(y0, 0.f), qmax), fminf(fmaxf(y1, 0.f), qmax));
+    const unsigned long long a = f2add(y, mm);
+    float d0, d1, a0, a1;
+    f2unpack(f2sub(y, f2sub(a, mm)), d0, d1);
+    f2unpack(a, a0, a1);
+    if (fabsf(d0) > 0.499f || fabsf(d1) > 0.499f) {  // next to a half integer: divide
+        float t0, t1;
+        f2unpack(t, t0, t1);
+        if (fabsf(d0) > 0.499f) a0 = __fadd_rn(fminf(fmaxf(__fdiv_rn(t0, s), 0.f), qmax), kMagic);
+        if (fabsf(d1) > 0.499f) a1 = __fadd_rn(fminf(fmaxf(__fdiv_rn(t1, s), 0.f), qmax), kMagic);
+    }
+    c0 = __float_as_uint(a0) - 0x4B400000u;
+    c1 = __float_as_uint(a1) - 0x4B400000u;
 }
 
 // One thread per WPT packed words (16 bytes of codes when a group holds that
@@ -117,8 +162,11 @@ quantize_kernel(const T *__restrict__ w, int64_t n_threads, int tpg,
 #pragma unroll
         for (int k = 0; k < WPT; ++k) {
 #pragma unroll
-            for (int j = 0; j < EPW; ++j)
-                packed[k] |= (uint32_t)code_of(v[k * EPW + j], b, s, r, QMAX) << (j * BITS);
+            for (int j = 0; j < EPW; j += 2) {
+                uint32_t c0, c1;
+                code_pair(v[k * EPW + j], v[k * EPW + j + 1], b, s, r, (float)QMAX, c0, c1);
+                packed[k] |= (c0 << (j * BITS)) | (c1 << ((j + 1) * BITS));
+            }
         }
     }
     uint32_t *dst = wq + tid * WPT;
