@@ -283,21 +283,18 @@ def bench_decode(m, steps, warmup, world, device, bits=4, packs=None):
 
 
 def bench_decode_e2e(d, steps, warmup, world, device):
-    """Same decode step through the public API with host buffers: pinned x is
-    copied in and y copied out inside the timed region."""
+    """Same decode step through the C-ABI call with host buffers
+    (qmm_quantized_matmul_host, one prepared call per weight copy): each step
+    copies pinned x in, runs the product and copies y out, all inside the
+    timed region."""
     from quantized_matmul_03_b200 import binding as qb
     c = d["case"]
     x_host = c.x.clone().pin_memory()
     y_host = torch.empty(tuple(d["y"].shape), dtype=torch.bfloat16).pin_memory()
     x_dev, y_dev = d["x"], d["y"]
     packs = d["packs"]
-
-    def step(p):
-        x_dev.copy_(x_host, non_blocking=True)
-        qb.qmm_quantized_matmul(x_dev, *p, True, c.group_size, c.bits, out=y_dev)
-        y_host.copy_(y_dev, non_blocking=True)
-
-    fns = [lambda p=p: step(p) for p in packs]
+    fns = [qb.HostMatmul(x_host, x_dev, *p, y_dev, y_host, True, c.group_size, c.bits)
+           for p in packs]
     total_ms = timed_eager(fns, steps, warmup, world)
     total_ms = max_over_ranks(world, total_ms)
     gbs = world * steps * d["bytes"] / (total_ms * 1e-3) / 1e9
@@ -346,6 +343,79 @@ def bench_moe(steps, warmup, world, device):
     nbytes = wq.shape[0] * weight_bytes(N_OUT, K_IN, c.bits, c.group_size)
     return dict(total_ms=total_ms, per_ms=per_ms, launches=launches, bytes=nbytes,
                 flops=2 * batch * N_OUT * K_IN)
+
+
+def bench_next_rows(steps, warmup, world, device, pk):
+    """The rows beyond the headline, each timed on the decode weight's shape
+    (W [14336, 4096]): dense with a bias, the microscaled modes, 3-/6-bit codes
+    and qqmm at M = 1 (weights rotating through copies larger than L2) and
+    M = 2048, plus the quantize kernel.  Returns {name: result}."""
+    from quantized_matmul_03_b200 import binding as qb
+    out = {}
+    c = wl.decode_case(1)
+    w = c.w.to(device)
+    x1 = c.x.to(device)
+    x2048 = wl.prefill_case(4).x.to(device)
+
+    def wbytes(bits, gs, sb_bytes):
+        return N_OUT * K_IN * bits // 8 + N_OUT * (K_IN // gs) * sb_bytes
+
+    def record(name, per_ms, nbytes, m):
+        flops = 2 * m * N_OUT * K_IN
+        f, bound = roofline_frac(per_ms, nbytes, flops, pk)
+        out[name] = {"us": per_ms * 1e3, "frac": f, "bound": bound,
+                     "GB/s": nbytes / (per_ms * 1e-3) / 1e9,
+                     "TFLOP/s": flops / (per_ms * 1e-3) / 1e12}
+
+    def copies(packed, n):
+        return [packed] + [tuple(t.clone() if t is not None else None for t in packed)
+                           for _ in range(n - 1)]
+
+    # quantize (row a1): bf16 weight in, codes + scales + biases out
+    wq4 = qb.qmm_quantize(w, 64, 4)
+    _, q_ms, _ = timed_launches([lambda: qb.qmm_quantize(w, 64, 4, out=wq4)], steps, warmup, world)
+    qbytes = N_OUT * K_IN * 2 + wbytes(4, 64, 4)
+    out["quantize_int4_gs64"] = {"us": q_ms * 1e3, "GB/s": qbytes / (q_ms * 1e-3) / 1e9,
+                                 "frac": qbytes / (q_ms * 1e-3) / 1e9 / pk["hbm_gbs"], "bound": "hbm"}
+    # quantized_dense: the affine product plus a bias vector in the epilogue
+    bias = torch.randn(N_OUT, device=device).to(torch.bfloat16)
+    packs = copies(wq4, L2_ROTATE)
+    y1 = torch.empty((1, N_OUT), dtype=torch.bfloat16, device=device)
+    _, ms, _ = timed_launches([lambda p=p: qb.qmm_quantized_dense(x1, *p, bias, True, 64, 4, out=y1)
+                               for p in packs], steps, warmup, world)
+    record("dense_bias_m1_int4", ms, wbytes(4, 64, 4), 1)
+    y2048 = torch.empty((2048, N_OUT), dtype=torch.bfloat16, device=device)
+    _, ms, _ = timed_launches([lambda: qb.qmm_quantized_dense(x2048, *wq4, bias, True, 64, 4, out=y2048)],
+                              max(3, steps // 4), warmup, world)
+    record("dense_bias_m2048_int4", ms, wbytes(4, 64, 4), 2048)
+    del packs
+    # microscaled modes and affine 3-/6-bit codes
+    specs = [("mxfp4", 32, 4, 1), ("mxfp8", 32, 8, 1), ("nvfp4", 16, 4, 1),
+             ("affine", 64, 3, 4), ("affine", 64, 6, 4)]
+    for mode, gs, bits, sbb in specs:
+        name = mode if mode != "affine" else f"affine_int{bits}"
+        packed = qb.qmm_quantize(w, gs, bits, mode)
+        nb = wbytes(bits, gs, sbb)
+        packs = copies(packed, max(2, -(-256_000_000 // nb)))
+        _, ms, _ = timed_launches([lambda p=p: qb.qmm_quantized_matmul(x1, *p, True, gs, bits, mode, out=y1)
+                                   for p in packs], steps, warmup, world)
+        record(f"{name}_m1", ms, nb, 1)
+        _, ms, _ = timed_launches([lambda: qb.qmm_quantized_matmul(x2048, *packed, True, gs, bits, mode,
+                                                                   out=y2048)],
+                                  max(3, steps // 4), warmup, world)
+        record(f"{name}_m2048", ms, nb, 2048)
+        if mode in ("nvfp4", "mxfp8"):
+            for m, x, y in ((1, x1, y1), (2048, x2048, y2048)):
+                wsz = int(qb.lib().qmm_qqmm_workspace_size(m, K_IN, gs, bits, 1))
+                ws = torch.empty(wsz, dtype=torch.uint8, device=device)
+                _, ms, _ = timed_launches(
+                    [lambda p=p, x=x, y=y, ws=ws: qb.qmm_qqmm(x, p[0], p[1], gs, bits, mode, out=y, workspace=ws)
+                     for p in (packs if m == 1 else [packed])], steps if m == 1 else max(3, steps // 4),
+                    warmup, world)
+                record(f"qqmm_{mode}_m{m}", ms, nb, m)
+        del packs, packed
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_suite(args, world, device, pk):
@@ -464,6 +534,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-moe", action="store_true")
+    ap.add_argument("--no-next", action="store_true",
+                    help="skip the rows beyond the headline (dense, microscaled, 3/6-bit, qqmm)")
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the prefill GEMM (for profiling); prints its own line")
     ap.add_argument("--prefill-bits", type=int, default=4)
@@ -514,6 +586,9 @@ def main():
             pre = bench_prefill(4, psteps, max(3, args.warmup // 4), world, device)
         if not args.no_moe:
             moe = bench_moe(max(3, min(args.steps, 20)), max(3, args.warmup // 4), world, device)
+        nxt = None
+        if not args.no_next:
+            nxt = bench_next_rows(max(3, min(args.steps, 20)), max(3, args.warmup // 4), world, device, pk)
     clocks = clk.summary()
 
     total_ms = max_over_ranks(world, d["total_ms"])
@@ -568,6 +643,9 @@ def main():
                          "definition": "max(weight bytes / HBM peak, flops / bf16 peak) / time",
                          "peak_src": pk["src"]}}
         line["gpu_launches"] += moe["launches"]
+    if nxt is not None:
+        line["next_rows"] = {k: {kk: round(vv, 4) if isinstance(vv, float) else vv for kk, vv in v.items()}
+                             for k, v in nxt.items()}
     if clocks:
         line["clocks"] = clocks
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

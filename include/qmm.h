@@ -149,7 +149,9 @@ qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K,
  *     QMM_OK leaves it zeroed again (after a QMM_ERR_TIMEOUT from
  *     qmm_device_status, zero it again).  Calls in flight at once must not
  *     share a workspace.  A workspace smaller than needed for a call's split
- *     is not used (whole tiles).  Misaligned: QMM_ERR_WORKSPACE.
+ *     is not used (whole tiles).  Misaligned: QMM_ERR_WORKSPACE.  (The
+ *     decode tensor-core path, QMM_PATH_DECODE_TC, writes its prepared
+ *     activations past the first 4096 bytes and leaves those bytes zero.)
  * Results: the parts of a split tile are added in a fixed order, so repeated
  *   calls return identical bits; they can differ from the whole-tile result
  *   in fp32 rounding.
@@ -164,6 +166,34 @@ qmm_status qmm_quantized_matmul_ws(const void *x, int64_t M, int64_t K,
                                    int group_size, int bits, const char *mode,
                                    void *y, void *workspace, size_t workspace_bytes,
                                    void *stream);
+
+/*
+ * qmm_quantized_matmul_host -- qmm_quantized_matmul_ws for activations and a
+ * result that live in host memory.  Nothing in the documents this library
+ * follows has a counterpart (their arrays live wherever the framework keeps
+ * them); it is the one call a host program makes per product.  On `stream`
+ * it enqueues, in order: the copy of M*K elements from x_host into x_dev,
+ * the product of x_dev into y_dev (exactly qmm_quantized_matmul_ws), and the
+ * copy of M*N elements from y_dev into y_host.
+ *   x_host, y_host: host memory; page-locked memory makes both copies
+ *     asynchronous (with pageable memory they behave as cudaMemcpyAsync
+ *     does).  y_host holds the result once the stream has completed the
+ *     call's work (cudaStreamSynchronize, or an event recorded after it).
+ *   x_dev, y_dev: caller-owned device buffers of M*K and M*N elements of the
+ *     activation dtype (x_dev as x of qmm_quantized_matmul_ws).
+ *   Element size: 4 bytes for QMM_F32, 2 for QMM_BF16/QMM_F16 (the microscaled
+ *     modes: the activation dtype given as `dtype`).
+ * Errors: those of qmm_quantized_matmul_ws (argument errors are found
+ * before anything is enqueued; when a call returns an error, the copy into
+ * y_host has not been enqueued); a NULL host buffer with a nonzero size:
+ * QMM_ERR_INVALID_ARG; a failed copy: QMM_ERR_CUDA.
+ */
+qmm_status qmm_quantized_matmul_host(const void *x_host, void *x_dev, int64_t M, int64_t K,
+                                     const uint32_t *wq, const void *scales, const void *biases,
+                                     qmm_dtype dtype, int64_t N, int transpose,
+                                     int group_size, int bits, const char *mode,
+                                     void *y_dev, void *y_host, void *workspace,
+                                     size_t workspace_bytes, void *stream);
 
 /*
  * qmm_quantized_dense -- Emily.Quantization.Layers, quantized_dense: the
@@ -332,9 +362,13 @@ qmm_status qmm_inject_fault(qmm_fault fault);
  * is QMM_PATH_AUTO).  QMM_PATH_GEMV forces the SIMT decode kernels (M <= 16
  * rows at a time), QMM_PATH_GEMM the tensor-core (tcgen05) GEMM, and
  * QMM_PATH_DECODE_TC the decode tensor-core kernel (bf16/f16, transpose,
- * 1..16 rows, 2- or 4-bit codes, K % 512 == 0, (K / group_size) % 8 == 0;
- * only when forced: AUTO keeps the faster SIMT decode kernel and GEMM).  A
- * forced path that cannot run a given call returns QMM_ERR_UNSUPPORTED.
+ * 1..16 rows, 2- or 4-bit codes, group size 32..128, K % 512 == 0; two
+ * launches per call: a prep kernel turns x into per-group block fixed point
+ * (16-bit integers split into a signed and an unsigned byte, error below
+ * 2^-15 of the group's largest |x|) in the workspace, then an integer MMA
+ * product; it needs the workspace that qmm_quantized_matmul_workspace_size
+ * reports under this path, else QMM_ERR_WORKSPACE).  A forced path that
+ * cannot run a given call returns QMM_ERR_UNSUPPORTED.
  */
 typedef enum {
     QMM_PATH_AUTO = 0,

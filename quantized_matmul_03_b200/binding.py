@@ -50,6 +50,8 @@ def lib() -> ctypes.CDLL:
                                      vp, vp],
             "qmm_quantized_matmul_ws": [vp, i64, i64, vp, vp, vp, i32, i64, i32, i32, i32, cp,
                                         vp, vp, sz, vp],
+            "qmm_quantized_matmul_host": [vp, vp, i64, i64, vp, vp, vp, i32, i64, i32, i32, i32,
+                                          cp, vp, vp, vp, sz, vp],
             "qmm_quantized_dense": [vp, i64, i64, vp, vp, vp, i32, i64, i32, i32, i32, cp,
                                     vp, ctypes.c_double, vp, vp, sz, vp],
             "qmm_qqmm": [vp, i64, i64, i32, vp, vp, i64, i32, i32, cp, vp, vp, sz, vp],
@@ -223,6 +225,64 @@ def qmm_quantized_matmul(x, wq, scales, biases, transpose: bool = True, group_si
                                          ws.numel() * ws.element_size() if ws is not None else 0,
                                          _stream(x.device)))
     return out
+
+
+class HostMatmul:
+    """One prepared ``qmm_quantized_matmul_host`` call: x from host memory,
+    the product, y back to host memory, enqueued on the current stream of
+    x_dev's device by a single C call each time the object is called.
+
+    x_host / y_host: CPU tensors (pin_memory() for asynchronous copies) of the
+    shapes of x_dev / y_dev; x_dev / y_dev: CUDA tensors.  The pointers,
+    sizes, workspace and stream are fixed when the object is made, so a call
+    costs one foreign-function call; y_host holds the result once the stream
+    has run it (torch.cuda.synchronize() or an event)."""
+
+    def __init__(self, x_host, x_dev, wq, scales, biases, y_dev, y_host, transpose: bool = True,
+                 group_size: int = 64, bits: int = 4, mode: str = "affine", workspace="auto"):
+        _cuda(x_dev, wq, scales, biases, y_dev)
+        for h, d in ((x_host, x_dev), (y_host, y_dev)):
+            if h.is_cuda or not h.is_contiguous() or h.shape != d.shape or h.dtype != d.dtype:
+                raise ValueError("host buffers must be contiguous CPU tensors shaped like the device ones")
+        K = x_dev.shape[-1]
+        M = x_dev.numel() // K if K else 0
+        N = wq.shape[-2] if transpose else wq.shape[-1] * 32 // bits
+        if y_dev.shape[-1] != N or y_dev.numel() != M * N:
+            raise ValueError(f"y must hold {M} x {N} values")
+        ws = None
+        if isinstance(workspace, str):
+            if workspace != "auto":
+                raise ValueError("workspace must be 'auto', None or a tensor")
+            if y_dev.dtype in DTYPES and mode not in MX_MODES:
+                need = qmm_quantized_matmul_workspace_size(M, K, N, transpose, bits, y_dev.dtype)
+                if need > 0:
+                    ws = _matmul_workspace(x_dev.device, need)
+        elif workspace is not None:
+            _cuda(workspace)
+            ws = workspace
+        # keep the tensors alive as long as the call may run
+        self._keep = (x_host, x_dev, wq, scales, biases, y_dev, y_host, ws)
+        self._fn = lib().qmm_quantized_matmul_host
+        self._args = (_p(x_host), _p(x_dev), M, K, _p(wq), _p(scales), _p(biases),
+                      _dtype(y_dev), N, int(bool(transpose)), group_size, bits, _mode(mode),
+                      _p(y_dev), _p(y_host), _p(ws),
+                      ws.numel() * ws.element_size() if ws is not None else 0,
+                      _stream(x_dev.device))
+
+    def __call__(self):
+        st = self._fn(*self._args)
+        if st != 0:
+            _check(st)
+
+
+def qmm_quantized_matmul_host(x_host, x_dev, wq, scales, biases, y_dev, y_host,
+                              transpose: bool = True, group_size: int = 64, bits: int = 4,
+                              mode: str = "affine", workspace="auto"):
+    """x_host -> x_dev, ``x_dev @ W`` -> y_dev, y_dev -> y_host, enqueued on the
+    current stream (one C call; see HostMatmul for the repeated form)."""
+    HostMatmul(x_host, x_dev, wq, scales, biases, y_dev, y_host, transpose, group_size, bits,
+               mode, workspace)()
+    return y_host
 
 
 def qmm_quantized_dense(x, wq, scales, biases, bias=0, transpose: bool = True,

@@ -132,9 +132,12 @@ qmm_status finish_launch(cudaError_t e, const char *what) {
 
 }  // namespace
 
-// Products with microscaled weights: the SIMT kernels (any shape, either
+// Products with microscaled weights: the tensor-core GEMM for more than a few
+// activation rows ([N, K] layout), else the SIMT kernels (any shape, either
 // layout; the gather entry takes affine weights only).
 cudaError_t launch_mx_matmul(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
+    // more than a few activation rows: the tensor-core GEMM where it applies
+    if (a.M > kGemvMaxRows && gemm_supported(dt, a)) return launch_gemm(dt, a, s);
     return launch_gemv(dt, a, s);
 }
 
@@ -249,10 +252,16 @@ namespace {
 
 // quantized_matmul with an optional layer bias (quantized_dense) and an
 // optional stream-K workspace: the implementation of the three entry points.
+qmm_status route_matmul(qmm_dtype dtype, const QmmArgs &a, cudaStream_t s);
+
+// x_host / y_host (qmm_quantized_matmul_host): when given, the copy of x_host
+// into x is enqueued once every argument has been checked, and the copy of y
+// into y_host once the product has been launched.
 qmm_status matmul_impl(const void *x, int64_t M, int64_t K, const uint32_t *wq, const void *scales,
                        const void *biases, qmm_dtype dtype, int64_t N, int transpose, int group_size,
                        int bits, const char *mode, const void *bias, double bias_value, void *y,
-                       void *workspace, size_t workspace_bytes, void *stream) {
+                       void *workspace, size_t workspace_bytes, void *stream,
+                       const void *x_host = nullptr, void *y_host = nullptr) {
     try {
         int md = QMM_MODE_AFFINE;
         qmm_status st = check_common(dtype, group_size, bits, mode, &md);
@@ -273,9 +282,37 @@ qmm_status matmul_impl(const void *x, int64_t M, int64_t K, const uint32_t *wq, 
         a.ws = workspace;
         a.ws_bytes = workspace ? workspace_bytes : 0;
         cudaStream_t s = (cudaStream_t)stream;
+        const size_t es = dtype == QMM_F32 ? 4 : 2;
+        if (x_host != nullptr) {
+            cudaError_t e = cudaMemcpyAsync(const_cast<void *>(x), x_host, (size_t)(M * K) * es,
+                                            cudaMemcpyHostToDevice, s);
+            if (e != cudaSuccess) return cuda_fail(e, "copy of x_host");
+        }
+        const qmm_status launched = route_matmul(dtype, a, s);
+        if (launched != QMM_OK || y_host == nullptr) return launched;
+        cudaError_t e = cudaMemcpyAsync(y_host, y, (size_t)(M * N) * es, cudaMemcpyDeviceToHost, s);
+        if (e != cudaSuccess) return cuda_fail(e, "copy into y_host");
+        return QMM_OK;
+    } catch (...) {
+        return fail(QMM_ERR_CUDA, "unexpected exception in qmm_quantized_matmul");
+    }
+}
+
+// Kernel choice and launch of one checked product (see qmm_set_path).
+qmm_status route_matmul(qmm_dtype dtype, const QmmArgs &a, cudaStream_t s) {
+    try {
+        const int md = a.mode;
         if (md != QMM_MODE_AFFINE) {
-            if (g_path == QMM_PATH_GEMM || g_path == QMM_PATH_DECODE_TC)
-                return fail(QMM_ERR_UNSUPPORTED, "the forced path does not take microscaled weights");
+            if (g_path == QMM_PATH_DECODE_TC)
+                return fail(QMM_ERR_UNSUPPORTED, "the decode tensor-core path takes affine weights");
+            if (g_path == QMM_PATH_GEMM) {
+                if (!gemm_supported(dtype, a))
+                    return fail(QMM_ERR_UNSUPPORTED,
+                                "the tensor-core path takes microscaled weights as bf16/f16, "
+                                "transpose, (K / group_size) %% 16 == 0");
+                return finish_launch(launch_gemm(dtype, a, s), "tensor-core gemm launch");
+            }
+            if (g_path == QMM_PATH_GEMV) return finish_launch(launch_gemv(dtype, a, s), "gemv launch");
             return finish_launch(launch_mx_matmul(dtype, a, s), "microscaled matmul launch");
         }
         const bool tc_ok = gemm_supported(dtype, a);
@@ -289,13 +326,16 @@ qmm_status matmul_impl(const void *x, int64_t M, int64_t K, const uint32_t *wq, 
         // Decode shapes of the [N, K] layout (1..4 rows) stream the weight
         // through the SIMT decode kernel; larger activation counts, and the
         // [K, N] layout at any count, use the tensor-core GEMM.  The decode
-        // tensor-core kernel runs only when forced (measured slower: its
-        // per-k-block tensor-memory stores set its pace).
+        // tensor-core kernel runs only when forced.
         if (g_path == QMM_PATH_DECODE_TC) {
             if (!gemv_tc_supported(dtype, a))
                 return fail(QMM_ERR_UNSUPPORTED,
                             "the decode tensor-core path needs bf16/f16, transpose, 1..16 rows, 2- or "
-                            "4-bit codes, K %% 512 == 0 and (K / group_size) %% 8 == 0");
+                            "4-bit codes, group size 32..128, K %% 512 == 0, 16-byte aligned operands");
+            if (a.ws == nullptr || a.ws_bytes < gemv_tc_workspace_bytes(a.K))
+                return fail(QMM_ERR_WORKSPACE,
+                            "the decode tensor-core path needs a workspace of "
+                            "qmm_quantized_matmul_workspace_size bytes");
             return finish_launch(launch_gemv_tc(dtype, a, s), "decode tensor-core launch");
         }
         const bool few_rows = a.M <= kGemvMaxRows && a.transpose;
@@ -323,6 +363,18 @@ qmm_status qmm_quantized_matmul_ws(const void *x, int64_t M, int64_t K, const ui
                        nullptr, 0.0, y, workspace, workspace_bytes, stream);
 }
 
+qmm_status qmm_quantized_matmul_host(const void *x_host, void *x_dev, int64_t M, int64_t K,
+                                     const uint32_t *wq, const void *scales, const void *biases,
+                                     qmm_dtype dtype, int64_t N, int transpose, int group_size,
+                                     int bits, const char *mode, void *y_dev, void *y_host,
+                                     void *workspace, size_t workspace_bytes, void *stream) {
+    if ((x_host == nullptr && M > 0 && K > 0) || (y_host == nullptr && M > 0 && N > 0))
+        return fail(QMM_ERR_INVALID_ARG, "x_host and y_host must not be NULL");
+    return matmul_impl(x_dev, M, K, wq, scales, biases, dtype, N, transpose, group_size, bits, mode,
+                       nullptr, 0.0, y_dev, workspace, workspace_bytes, stream,
+                       M > 0 && K > 0 ? x_host : nullptr, M > 0 && N > 0 ? y_host : nullptr);
+}
+
 qmm_status qmm_quantized_dense(const void *x, int64_t M, int64_t K, const uint32_t *wq,
                                const void *scales, const void *biases, qmm_dtype dtype, int64_t N,
                                int transpose, int group_size, int bits, const char *mode,
@@ -343,10 +395,16 @@ qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K, const uint3
 size_t qmm_quantized_matmul_workspace_size(int64_t M, int64_t K, int64_t N, int transpose,
                                            int bits, qmm_dtype dtype) {
     try {
-        // Decode shapes go to the SIMT decode kernel under the automatic path,
-        // and the forced decode tensor-core kernel takes no workspace.
+        // The forced decode tensor-core kernel keeps its prepared activations
+        // in the workspace; under the automatic path decode shapes go to the
+        // SIMT decode kernel, which takes none.
+        if (g_path == QMM_PATH_DECODE_TC) {
+            if (M < 1 || M > 16 || !transpose || (bits != 2 && bits != 4) ||
+                (dtype != QMM_BF16 && dtype != QMM_F16) || K <= 0)
+                return 0;
+            return gemv_tc_workspace_bytes(K);
+        }
         if (g_path != QMM_PATH_GEMM && M <= kGemvMaxRows && transpose) return 0;
-        if (g_path == QMM_PATH_DECODE_TC) return 0;
         return gemm_workspace_size(dtype, M, K, N, transpose != 0, bits);
     } catch (...) {
         return 0;

@@ -1,50 +1,49 @@
-// gemv_tc.cu -- decode-shaped quantized matmul on the tensor cores for 1..16
-// activation rows, W stored [N, K] (transpose), 2- and 4-bit codes, bf16/f16:
-//     y[m, n] = sum_k x[m, k] * (s[n,g] q[n,k] + b[n,g])
+// gemv_tc.cu -- decode-shaped quantized matmul on the integer tensor cores
+// for 1..16 activation rows, W stored [N, K] (transpose), 2- and 4-bit codes,
+// bf16/f16 activations:
+//     y[m, n] = sum_g s[n,g] sum_{k in g} q[n,k] x[m,k] + b[n,g] sum_{k in g} x[m,k]
 // (mlx-rs ops/quantization.rs, quantized_matmul; Emily.Quantization.Layers,
-// quantized_dense: the packed weight is streamed once per call, never
+// quantized_dense: the packed weight is streamed once per call and never
 // expanded into a dense weight in memory).
 //
-// The product is bound by reading the packed weight, but the work of turning
-// codes into something a multiplier can use is not: done on the CUDA cores
-// it sets the pace (and grows with the number of activation rows).  Here the
-// CUDA cores only place codes into 16-bit operands and the tensor cores do
-// every multiply-add, so one kernel serves 1..16 rows at the same cost, and
-// the code placement -- which does not depend on x -- runs while the previous
-// kernel of the stream is still finishing (programmatic dependent launch).
+// Formulation.  The codes enter the MMA as exact unsigned bytes and the
+// activations as exact block fixed point, so every multiply-add of a group is
+// an exact int32 sum on the tensor cores (tcgen05.mma kind::i8):
+//   activations: per row m and group g, x ~ x_int 2^-e with e chosen from the
+//     group's largest |x| so that x_int is a 16-bit integer (representation
+//     error below 2^-15 of that largest |x|; 2^-14 for a value that rounds
+//     up to 2^15 and is held at 2^15 - 1), split as x_int = 256 h + l with
+//     h in [-128, 127] (s8) and l in [0, 255] (u8);  X_g[m] = sum of x (fp32);
+//   codes: a 4-bit word w gives the bytes (w & 0x0F0F0F0F) = codes 0,2,4,6
+//     and ((w >> 4) & 0x0F0F0F0F) = codes 1,3,5,7 (2-bit: four planes, codes
+//     p, 4+p, 8+p, 12+p), so the A operand holds each word's codes in that
+//     order, and h and l are stored in the same order;
+//   per group: D_h = sum q h and D_l = sum q l (two MMAs, s8 and u8 B; both
+//     below 2^22 in magnitude for codes of at most 4 bits and groups of at
+//     most 128), then  y[m, n] += s 2^-e (256 D_h + D_l) + b X_g[m]  in fp32.
+// A prep kernel writes h, l, 2^-e and X_g once per call into the workspace;
+// the product kernel reads them with tensor copies.
 //
-// Formulation.  A code q enters the MMA as the exact 16-bit value
-// a = 1 + q/QS (the code ORed into the mantissa of 1.0 at the highest field
-// position a byte move reaches; QS = 16 for 4-bit and 4 for 2-bit codes with
-// bf16, 64 and 16 with f16).  Per group g of group_size elements the MMA
-// leaves, in fp32 tensor memory,
-//     D_g[n, m] = sum_{k in g} a[n,k] x[m,k] = X_g[m] + (1/QS) sum_{k in g} q[n,k] x[m,k]
-// with X_g[m] = sum_{k in g} x[m,k], so
-//     y[m, n] = sum_g (QS s[n,g]) (D_g[n, m] - X_g[m]) + b[n,g] X_g[m].
-// X_g comes from the MMA as well: lane 31 of every 32-lane quadrant of the A
-// operand holds code 0 everywhere (a = 1), so D_g[lane 31] = X_g.
-//
-// Orientation: UMMA M = 128 tensor-memory lanes over weight rows (each CTA
-// owns R <= 124 contiguous rows, RQ = ceil(R/4) per lane quadrant), UMMA N =
-// 16 over activation rows, K = 16 per instruction, one accumulator of 16
-// columns per group (a ring of 8).
+// Orientation: UMMA M = 128 over weight rows (each CTA owns R <= 128
+// contiguous rows; A rows past R are never read back), UMMA N = 16 over
+// activation rows (h rows and l rows), K = 32 per instruction; per group one
+// accumulator of 32 columns (16 for D_h, 16 for D_l), a ring of 16.
 //
 // Roles (512 threads, two CTAs per SM: the next call's CTA fits beside this
-// one and fills its own ring while this one finishes):
-//   warps 0, 1   TMA loads of the packed codes, 128 bytes of every owned row
-//                per stage (alternate stages), into a ring of shared-memory
-//                stages (128-byte swizzle: conflict-free row reads);
-//   warp 2       waits for the preceding grids (griddepcontrol.wait), then
-//                copies the activation rows into shared memory in the
-//                canonical 128-byte-swizzled K-major layout of the B operand;
+// one and streams its first codes while this one finishes):
+//   warps 0, 1   tensor copies of the packed codes, 128 bytes of every owned
+//                row per stage (alternate stages), 128-byte swizzled;
+//   warp 2       waits for the prep kernel (griddepcontrol.wait), then copies
+//                per four A slots their h/l tiles (one 3-D tensor copy of 4 x
+//                32 rows x 128 bytes: a tensor copy costs its issuing thread
+//                several hundred cycles, whatever its size) and the groups'
+//                (2^-e, X) table;
 //   warp 3       tensor-memory owner and MMA issuer (one elected lane);
-//   warps 4-11   code placement: two groups of four warps take alternate
-//                k-blocks of 64; thread l of quadrant q places row q*RQ + l
-//                (32 columns of bf16x2 / f16x2 per k-block) with one
-//                tcgen05.st;
-//   warps 12-15  epilogue: per group, tcgen05.ld of its quadrant's
-//                accumulator, the scale/bias step above in fp32 registers,
-//                and at the end one store of y per row.
+//   warps 4-11   code expansion: two groups of four warps take alternate A
+//                slots (128 codes of every row, 128-byte swizzled K-major u8);
+//   warps 12-15  epilogue: per group, tcgen05.ld of the quadrant's D_h and
+//                D_l, the step above in fp32 registers, and one store of y
+//                per row at the end.
 // Every wait is bounded (device error word on timeout); before exiting or
 // freeing tensor memory a CTA waits, with the fixed limit, for its own copies
 // and MMAs.  No cluster multicast is used.
@@ -59,20 +58,16 @@ namespace qmm {
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kWarpX = 2, kWarpMma = 3, kWarpUnp = 4, kWarpEpi = 12;
-// Tensor memory: all 512 columns.  A k-block's A operand goes from code
-// placement through the MMA and back to an empty slot in a round trip of a
-// few thousand cycles, so the ring must hold many k-blocks to keep both
-// sides busy.  (The next call's CTA, beside this one, streams codes into its
-// shared-memory ring while its tcgen05.alloc waits for these columns.)
-constexpr int kASlots = 12;         // A operand slots (32 columns each)
-constexpr int kDSlots = 8;          // group accumulators (16 columns each)
-constexpr int kPlaceBatch = 3;      // k-blocks a placement warp stores per wait
-constexpr int kBStageKb = 8;        // k-blocks per activation stage
+constexpr int kWarpB = 2, kWarpMma = 3, kWarpUnp = 4, kWarpEpi = 12;
+constexpr int kASlots = 2;          // A slots: 128 codes x R rows, u8
+constexpr int kSlotsPerB = 4;       // A slots per activation stage
+constexpr int kBStages = 2;         // activation ring
+constexpr int kBTile = 4096;        // h/l tile of one A slot: 32 rows x 128 bytes
+constexpr int kBStage = kSlotsPerB * kBTile + 2048;  // + the stage's table (<= 16 groups)
+constexpr int kDSlots = 16;         // group accumulators, 32 columns each
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kDCol0 = kASlots * 32;
 constexpr int kTmemThreads = 32 * (16 - kWarpMma);  // warps that use tensor memory
-constexpr int kMaxRows = 124;       // rows per CTA: 31 per quadrant + lane 31
+constexpr int kMaxRows = 128;
 constexpr size_t kSmemBudget = 110 * 1024;
 
 // Per-SM hand-off between consecutive CTAs of this kernel (see the decode
@@ -84,83 +79,132 @@ constexpr uint64_t kHandoffWaitNs = 20000;
 __device__ unsigned long long g_tc_ticket[kMaxSm];
 __device__ unsigned long long g_tc_issued[kMaxSm];
 
-struct DecParams {
-    const void *x;
-    void *y;
+// Instruction descriptors of kind::i8: s32 accumulator, A u8 (codes), B s8
+// (h) or u8 (l), both K-major, M = 128, N = 16.
+constexpr uint32_t idesc_i8(bool b_signed) {
+    return (2u << 4) | (0u << 7) | ((b_signed ? 1u : 0u) << 10) | ((uint32_t)(16 >> 3) << 17) |
+           ((uint32_t)(128 >> 4) << 24);
+}
+__device__ __forceinline__ void tc_mma_i8(uint32_t tmem_d, uint64_t desc_a, uint64_t desc_b,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(desc_a), "l"(desc_b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Byte order of the A operand (and of h and l) within a packed word: output
+// position j of a 16-element chunk holds element perm(j) of the chunk.
+template <int BITS> __host__ __device__ constexpr int perm_elem(int j) {
+    if constexpr (BITS == 4) {
+        // two words of 8 codes: 0,2,4,6,1,3,5,7 each
+        const int w = j >> 3, t = j & 7;
+        return 8 * w + (t < 4 ? 2 * t : 2 * (t - 4) + 1);
+    } else {
+        // one word of 16 codes: plane p = j / 4 holds codes p, 4+p, 8+p, 12+p
+        return 4 * (j & 3) + (j >> 2);
+    }
+}
+
+struct I8Params {
     const uint16_t *scales, *biases;
-    int M, N, K, gpr, gs_log;
-    int R, RQ;        // rows of this CTA (at most), rows per lane quadrant
-    int S;            // code-ring stages
-    int stage_bytes;  // per code stage (1024-aligned)
-    int KB;           // k-blocks of 64
-    const void *bias; // layer bias [N] or null, plus bias_value, added before rounding
+    void *y;
+    const void *bias;  // layer bias [N] or null, plus bias_value, added before rounding
     float bias_value;
+    int M, N, K, gpr, gs_log;
+    int R;             // rows per CTA (at most)
+    int S;             // code-ring stages
+    int stage_bytes;   // per code stage (1024-aligned)
+    int a_bytes;       // per A slot: whole 8-row atoms of R rows
     int *err;
 };
 
-// The code field sits at mantissa bit P of each 16-bit half of 1.0 (the
-// highest position a byte move can reach), so a = 1 + q/QS with QS =
-// 2^(mantissa bits - P): the offset 1 is at most QS times the code step,
-// which keeps the accumulator's rounding small next to the code term.
-template <typename T, int BITS> struct Field;
-template <> struct Field<__nv_bfloat16, 4> { static constexpr int P = 3; };  // QS = 16
-template <> struct Field<__nv_bfloat16, 2> { static constexpr int P = 5; };  // QS = 4
-template <> struct Field<__half, 4> { static constexpr int P = 4; };         // QS = 64
-template <> struct Field<__half, 2> { static constexpr int P = 6; };         // QS = 16
-template <typename T> struct One2;
-template <> struct One2<__nv_bfloat16> {
-    static constexpr uint32_t V = 0x3F803F80u;  // bf16 1.0 | 1.0 (7 mantissa bits)
-    static constexpr int MB = 7;
-};
-template <> struct One2<__half> {
-    static constexpr uint32_t V = 0x3C003C00u;  // f16 1.0 | 1.0 (10 mantissa bits)
-    static constexpr int MB = 10;
-};
-template <typename T, int BITS> struct Magic {
-    static constexpr int P = Field<T, BITS>::P;
-    static constexpr uint32_t ONE2 = One2<T>::V;
-    static constexpr uint32_t MASK = (((1u << BITS) - 1u) << P) * 0x00010001u;
-    static constexpr float QS = (float)(1 << (One2<T>::MB - P));
-};
-
-// Word w shifted so that the code at bit `from` lands at bit `to`.
-template <int FROM, int TO>
-__device__ __forceinline__ uint32_t align_field(uint32_t w) {
-    if constexpr (TO >= FROM) return w << (TO - FROM);
-    else return w >> (FROM - TO);
-}
-
-// Codes of one k-block of one row (64 codes) -> 32 columns of 16-bit pairs
-// (element 2i in the low half of column i), a = 1 + q/QS, in k order.
-// Byte i of a word holds codes 2i, 2i+1 (4-bit) or 4i..4i+3 (2-bit); PRMT
-// puts byte i of one shifted copy of the word in the low half and byte i of
-// another in the high half, so one AND/OR (LOP3) leaves the two codes of a
-// pair at bit P of the two mantissas.
+// ---------------------------------------------------------------------------
+// Prep: activations -> h, l (permuted byte order), (2^-e, X) per (group, row).
+// Workspace: [32][K] bytes (rows 0..15 h, 16..31 l; rows past M unused) then
+// [K / group_size][16] float2.  One thread per (row, 16-element chunk); the
+// gs/16 threads of a group are adjacent lanes.
+// ---------------------------------------------------------------------------
 template <typename T, int BITS>
-__device__ __forceinline__ void place_codes(const uint32_t (&w)[BITS * 2], uint32_t (&v)[32]) {
-    using MG = Magic<T, BITS>;
-    constexpr int P = MG::P;
-    if constexpr (BITS == 4) {
+__global__ void __launch_bounds__(256)
+qdecode_prep_kernel(const T *__restrict__ x, int M, int K, int gs_log, uint8_t *__restrict__ ws) {
+    // The next grid (the product) may start its weight stream now.
+    ptx::grid_launch_dependents();
+    // x may be the output of the preceding kernel, and the workspace may
+    // still be read by the product kernel of the previous call: wait for
+    // both (every earlier grid) to complete.
+    ptx::grid_dependency_wait();
+    const int cpr = K >> 4;  // chunks per row
+    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+    const bool ok = idx < M * cpr;
+    const int m = ok ? idx / cpr : 0, c = ok ? idx - m * cpr : 0;
+    float v[16];
+    if (ok) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)m * K + 16 * c);
 #pragma unroll
-        for (int wi = 0; wi < 8; ++wi) {
-            const uint32_t lo = align_field<0, P>(w[wi]), hi = align_field<4, P>(w[wi]);
+        for (int h = 0; h < 2; ++h) {
+            const uint4 u = __ldcg(src + h);
+            const T *t = reinterpret_cast<const T *>(&u);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t t = __byte_perm(lo, hi, (uint32_t)(i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12)));
-                v[4 * wi + i] = (t & MG::MASK) | MG::ONE2;
-            }
+            for (int i = 0; i < 8; ++i) v[8 * h + i] = Dt<T>::to_f(t[i]);
         }
     } else {
 #pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
-            const uint32_t a0 = align_field<0, P>(w[wi]), a1 = align_field<2, P>(w[wi]);
-            const uint32_t a2 = align_field<4, P>(w[wi]), a3 = align_field<6, P>(w[wi]);
+        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+    }
+    float amax = 0.f, sum = 0.f;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t sel = (uint32_t)(i | (i << 4) | ((4 + i) << 8) | ((4 + i) << 12));
-                v[8 * wi + 2 * i] = (__byte_perm(a0, a1, sel) & MG::MASK) | MG::ONE2;
-                v[8 * wi + 2 * i + 1] = (__byte_perm(a2, a3, sel) & MG::MASK) | MG::ONE2;
-            }
+    for (int i = 0; i < 16; ++i) {
+        amax = fmaxf(amax, fabsf(v[i]));
+        sum += v[i];
+    }
+    // Group of gs/16 adjacent lanes (2, 4 or 8): out-of-range threads form
+    // whole groups (M * cpr is a multiple of gs/16).
+    const int tpg = 1 << (gs_log - 4);
+    for (int o = 1; o < tpg; o <<= 1) {
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    }
+    if (!ok) return;
+    // amax < 2^ex; e = 15 - ex puts every |x 2^e| below 2^15, clamped so that
+    // 2^e and 2^-e are normal floats.
+    const int ex = (int)((__float_as_uint(amax) >> 23) & 0xffu) - 126;
+    const int e = min(126, max(-126, 15 - ex));
+    const float up = __uint_as_float((uint32_t)(127 + e) << 23);
+    uint32_t hw[4] = {0, 0, 0, 0}, lw[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const int xi = min(32767, __float2int_rn(v[perm_elem<BITS>(j)] * up));
+        const uint32_t hb = (uint32_t)(xi >> 8) & 0xffu, lb = (uint32_t)xi & 0xffu;
+        hw[j >> 2] |= hb << (8 * (j & 3));
+        lw[j >> 2] |= lb << (8 * (j & 3));
+    }
+    uint8_t *row_h = ws + (int64_t)m * K + 16 * c;
+    *reinterpret_cast<uint4 *>(row_h) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4 *>(row_h + (int64_t)16 * K) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    if ((c & (tpg - 1)) == 0) {
+        float2 *tab = reinterpret_cast<float2 *>(ws + (int64_t)32 * K);
+        tab[(int64_t)(c >> (gs_log - 4)) * 16 + m] = make_float2(__uint_as_float((uint32_t)(127 - e) << 23), sum);
+    }
+}
+
+// Codes of one row for one A slot (128 codes) -> 8 chunks of 16 u8 bytes in
+// the permuted order; w holds BITS * 4 words.
+template <int BITS>
+__device__ __forceinline__ void expand_codes(const uint32_t (&w)[BITS * 4], uint32_t (&o)[32]) {
+    if constexpr (BITS == 4) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            o[2 * i] = w[i] & 0x0F0F0F0Fu;
+            o[2 * i + 1] = (w[i] >> 4) & 0x0F0F0F0Fu;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) o[4 * i + p] = (w[i] >> (2 * p)) & 0x03030303u;
         }
     }
 }
@@ -194,56 +238,60 @@ template <> __device__ __forceinline__ void tmem_ld_cols<16>(uint32_t taddr, uin
         : "memory");
 }
 
+// An int32 of magnitude below 2^22 as a float, exactly, with two full-rate
+// operations (integer add into the mantissa of 1.5 * 2^23, then subtract it).
+__device__ __forceinline__ float small_int_to_f(uint32_t v) {
+    return __uint_as_float(v + 0x4B400000u) - 12582912.0f;
+}
+
 // MR: activation rows the kernel is built for (1, 2, 4, 8, 16; the call has
-// M <= MR).  The B operand holds NB = 8 (MR <= 8) or 16 rows; the MMA is
-// always N = 16 (with NB = 8 its rows 8..15 are other shared-memory bytes,
-// and their accumulator columns are never read).
+// M <= MR).  The MMAs always use N = 16 (h and l tiles of 16 rows each).
 template <typename T, int BITS, int MR>
 __global__ void __launch_bounds__(kThreads, 2)
-qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const DecParams p) {
+qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_b,
+                const float2 *__restrict__ tab, const I8Params p) {
     constexpr bool kF16 = std::is_same<T, __half>::value;
-    constexpr int NB = MR <= 8 ? 8 : 16;
-    constexpr int B_KB = NB * 128;                 // bytes of one k-block of B
-    constexpr int B_STAGE = kBStageKb * B_KB;
-    constexpr int KBS = BITS == 4 ? 4 : 8;         // k-blocks per 128-byte code chunk
-    constexpr uint32_t IDESC = make_idesc(kF16, 128, 16);
-    constexpr float QS = Magic<T, BITS>::QS;
+    constexpr int SPC = 512 / (BITS * 64);         // A slots per 128-byte code chunk (4-bit 2, 2-bit 4)
+    constexpr uint32_t ID_H = idesc_i8(true), ID_L = idesc_i8(false);
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = ptx::smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *gbase = smem_raw + (base - raw);
     const int S = p.S;
-    const uint32_t c0 = base;                                   // code ring
-    const uint32_t b0 = c0 + (uint32_t)S * (uint32_t)p.stage_bytes;  // activation ring
-    // (NB = 8: the MMA's rows 8..15 of the last k-block read up to 1 KB past
-    // the ring; that padding keeps them inside the allocation.)
-    const uint32_t bar0 = b0 + 2 * B_STAGE + (NB == 8 ? 1024 : 0);
+    const uint32_t c0 = base;                                          // code ring
+    const uint32_t a0 = c0 + (uint32_t)S * (uint32_t)p.stage_bytes;    // A ring
+    // (the MMA reads 128 rows of an A slot; rows past R of the last slot fall
+    // into the B ring that follows, inside the allocation)
+    const uint32_t b0 = a0 + (uint32_t)kASlots * (uint32_t)p.a_bytes;  // B ring
+    const uint32_t bar0 = b0 + kBStages * kBStage;
     const uint32_t fullC = bar0, emptyC = fullC + 8 * S;
     const uint32_t fullA = emptyC + 8 * S, emptyA = fullA + 8 * kASlots;
-    const uint32_t fullB = emptyA + 8 * kASlots, emptyB = fullB + 16;
-    const uint32_t fullD = emptyB + 16, emptyD = fullD + 8 * kDSlots;
+    const uint32_t fullB = emptyA + 8 * kASlots, emptyB = fullB + 8 * kBStages;
+    const uint32_t fullD = emptyB + 8 * kBStages, emptyD = fullD + 8 * kDSlots;
     const uint32_t done = emptyD + 8 * kDSlots, go = done + 8;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + (go + 8 - base));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r0 = blockIdx.x * p.R;
     const int R = max(0, min(p.R, p.N - r0));
-    const int KB = p.KB;
-    const int NST = KB / KBS;                      // code stages
+    const int NA = p.K >> 7;                       // A slots (128 codes each)
+    const int NST = NA / SPC;                      // code stages
     const int G = p.K >> p.gs_log;                 // groups per row
+    const int gpa = 128 >> p.gs_log;               // groups per A slot
+    const int gpb = gpa * kSlotsPerB;              // groups per activation stage
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             ptx::mbar_init(fullC + 8 * s, 1);
-            ptx::mbar_init(emptyC + 8 * s, 8);     // every placement warp, once per stage
+            ptx::mbar_init(emptyC + 8 * s, 8);     // every expansion warp, once per stage
         }
         for (int a = 0; a < kASlots; ++a) {
-            ptx::mbar_init(fullA + 8 * a, 4);      // the four warps of one placement group
+            ptx::mbar_init(fullA + 8 * a, 4);      // the four warps of one expansion group
             ptx::mbar_init(emptyA + 8 * a, 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kBStages; ++b) {
             ptx::mbar_init(fullB + 8 * b, 1);
-            ptx::mbar_init(emptyB + 8 * b, 1);
+            ptx::mbar_init(emptyB + 8 * b, 5);     // the MMAs' commit + the four epilogue warps
         }
         for (int d = 0; d < kDSlots; ++d) {
             ptx::mbar_init(fullD + 8 * d, 1);
@@ -254,9 +302,10 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const DecParams p) {
         ptx::fence_mbar_init();
     }
     __syncthreads();  // barriers initialised
-    // Let the next call in the stream start its prologue and its own code
-    // stream now.  Before griddepcontrol.wait this grid reads only the packed
-    // weight, its scales and biases (the rule for their writers is in qmm.h).
+    // Let the next kernel of the stream launch (the next call's prep kernel,
+    // which waits for this grid before it writes the workspace).  Before
+    // griddepcontrol.wait this grid reads only the packed weight, its scales
+    // and biases (the rule for their writers is in qmm.h).
     ptx::grid_launch_dependents();
     // The producers start at once; the warps that use tensor memory wait for
     // the allocation (which waits for the CTA of the previous call on this SM
@@ -273,7 +322,7 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const DecParams p) {
         tmem = *tmem_slot;
     }
 
-    if (warp < kWarpX) {
+    if (warp < kWarpB) {
         // ---------------- packed-code producers ----------------
         if (lane == 0) {
             uint32_t smid;
@@ -307,64 +356,54 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const DecParams p) {
             for (int st = max(0, NST - S); st < NST; ++st)
                 if ((st & 1) == warp) ptx::mbar_drain(fullC + 8 * (st % S), (st / S) & 1, p.err);
         }
-    } else if (warp == kWarpX) {
-        // ---------------- activations (B operand) ----------------
-        // x may be the output of the preceding kernel: wait for it.  The rows
-        // are read through L2 only (ld.global.cg), never from a stale L1 line.
-        ptx::grid_dependency_wait();
-        const T *x = static_cast<const T *>(p.x);
-        const int units = p.M * 64;  // (row, k-block of the stage, 16-byte chunk)
-        for (int bs = 0; bs < KB / kBStageKb; ++bs) {
-            const int slot = bs & 1;
-            if (bs >= 2) ptx::mbar_wait(emptyB + 8 * slot, ((bs >> 1) - 1) & 1, p.err);
-            uint8_t *dst = gbase + (b0 - base) + slot * B_STAGE;
-            for (int u0 = 0; u0 < units; u0 += 32 * 4) {
-                uint4 v[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int u = u0 + 32 * i + lane;
-                    if (u < units) {
-                        const int r = u >> 6, b = (u >> 3) & 7, c = u & 7;
-                        v[i] = __ldcg(reinterpret_cast<const uint4 *>(x + (int64_t)r * p.K +
-                                                                      (bs * kBStageKb + b) * 64 + c * 8));
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int u = u0 + 32 * i + lane;
-                    if (u < units) {
-                        const int r = u >> 6, b = (u >> 3) & 7, c = u & 7;
-                        *reinterpret_cast<uint4 *>(dst + b * B_KB + r * 128 + ((c ^ (r & 7)) << 4)) = v[i];
-                    }
-                }
+    } else if (warp == kWarpB) {
+        // ---------------- h/l tiles and tables ----------------
+        if (lane == 0) {
+            // The workspace is written by this call's prep kernel: wait for it.
+            ptx::grid_dependency_wait();
+            const uint32_t tbytes = (uint32_t)gpb * 16u * 8u;
+            const int NB = NA / kSlotsPerB;
+            for (int bt = 0; bt < NB; ++bt) {
+                const int bs = bt % kBStages;
+                if (bt >= kBStages) ptx::mbar_wait(emptyB + 8 * bs, ((bt / kBStages) - 1) & 1, p.err);
+                const uint32_t dst = b0 + (uint32_t)bs * kBStage;
+                ptx::mbar_arrive_expect_tx(fullB + 8 * bs, (uint32_t)(kSlotsPerB * kBTile) + tbytes);
+                tma_load_3d(dst, &tmap_b, 0, 0, bt * kSlotsPerB, fullB + 8 * bs);
+                ptx::bulk_g2s(dst + kSlotsPerB * kBTile, tab + (int64_t)bt * gpb * 16, tbytes, fullB + 8 * bs);
             }
-            ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(fullB + 8 * slot);
+            for (int bt = max(0, NB - kBStages); bt < NB; ++bt)
+                ptx::mbar_drain(fullB + 8 * (bt % kBStages), (bt / kBStages) & 1, p.err);
         }
     } else if (warp == kWarpMma) {
         // ---------------- MMA issuer ----------------
         const bool leader = elect_one();
         const int gs_mask = (1 << p.gs_log) - 1;
-        for (int kb = 0; kb < KB; ++kb) {
-            const int a = kb % kASlots;
-            const int bslot = (kb / kBStageKb) & 1;
+        for (int a = 0; a < NA; ++a) {
+            const int as = a % kASlots, bt = a / kSlotsPerB, bs = bt % kBStages, sub = a - bt * kSlotsPerB;
             if (leader) {
-                ptx::mbar_wait<false>(fullA + 8 * a, (kb / kASlots) & 1, p.err);
-                if (kb % kBStageKb == 0) ptx::mbar_wait<false>(fullB + 8 * bslot, (kb / (2 * kBStageKb)) & 1, p.err);
-                const uint64_t db = sw128_desc(b0 + bslot * B_STAGE + (kb % kBStageKb) * B_KB);
+                ptx::mbar_wait<false>(fullA + 8 * as, (a / kASlots) & 1, p.err);
+                if (sub == 0) ptx::mbar_wait<false>(fullB + 8 * bs, (bt / kBStages) & 1, p.err);
+                tc_fence_after();
+                const uint32_t btile = b0 + (uint32_t)bs * kBStage + (uint32_t)sub * kBTile;
+                const uint64_t da = sw128_desc(a0 + (uint32_t)as * (uint32_t)p.a_bytes);
+                const uint64_t dh = sw128_desc(btile);
+                const uint64_t dl = sw128_desc(btile + 2048u);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const int e0 = kb * 64 + 16 * j;
+                    const int e0 = a * 128 + 32 * j;
                     const int g = e0 >> p.gs_log, d = g & (kDSlots - 1);
-                    const bool first = (e0 & gs_mask) == 0, last = ((e0 + 16) & gs_mask) == 0;
-                    if (first && g >= kDSlots) ptx::mbar_wait<false>(emptyD + 8 * d, ((g / kDSlots) - 1) & 1, p.err);
-                    tc_fence_after();
-                    tc_mma_ts(tmem + kDCol0 + 16u * d, tmem + 32u * a + 8u * j, db + 2u * j, IDESC, first ? 0u : 1u);
+                    const bool first = (e0 & gs_mask) == 0, last = ((e0 + 32) & gs_mask) == 0;
+                    if (first && g >= kDSlots) {
+                        ptx::mbar_wait<false>(emptyD + 8 * d, ((g / kDSlots) - 1) & 1, p.err);
+                        tc_fence_after();
+                    }
+                    // K = 32 bytes per instruction: 2 units of 16 bytes along the rows.
+                    tc_mma_i8(tmem + 32u * d, da + 2u * j, dh + 2u * j, ID_H, first ? 0u : 1u);
+                    tc_mma_i8(tmem + 32u * d + 16u, da + 2u * j, dl + 2u * j, ID_L, first ? 0u : 1u);
                     if (last) tc_commit(fullD + 8 * d);
                 }
-                tc_commit(emptyA + 8 * a);
-                if (kb % kBStageKb == kBStageKb - 1 || kb == KB - 1) tc_commit(emptyB + 8 * bslot);
+                tc_commit(emptyA + 8 * as);
+                if (sub == kSlotsPerB - 1) tc_commit(emptyB + 8 * bs);
             }
             __syncwarp();
         }
@@ -376,113 +415,87 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const DecParams p) {
         }
         __syncwarp();
     } else if (warp < kWarpEpi) {
-        // ---------------- code placement ----------------
+        // ---------------- code expansion ----------------
         const int h = (warp - kWarpUnp) >> 2, q = warp & 3;
-        const int j = q * p.RQ + lane;                 // row of this lane within the CTA
-        const bool valid = lane < p.RQ && j < R;       // (lane 31 never holds a row)
-        // Batches of kPlaceBatch own k-blocks: each is stored as soon as it is
-        // placed, and one tcgen05.wait::st covers the batch before its A
-        // slots are published.
-        for (int kb0 = h; kb0 < KB; kb0 += 2 * kPlaceBatch) {
+        const int j = 32 * q + lane;                  // row of this lane within the CTA
+        const bool valid = j < R;
+        const uint32_t arow = (uint32_t)(j >> 3) * 1024u + (uint32_t)(j & 7) * 128u;
+        for (int a = h; a < NA; a += 2) {
+            const int st = a / SPC, sp = a - st * SPC;
+            const int slot = st % S;
+            if (sp < 2) ptx::mbar_wait(fullC + 8 * slot, (st / S) & 1, p.err);
+            const int as = a % kASlots;
+            if (a >= kASlots) ptx::mbar_wait<false>(emptyA + 8 * as, ((a / kASlots) - 1) & 1, p.err);
+            uint32_t w[BITS * 4];
+            if (valid) {
+                const uint8_t *row = gbase + (c0 - base) + slot * p.stage_bytes + j * 128;
 #pragma unroll
-            for (int t = 0; t < kPlaceBatch; ++t) {
-                const int kb = kb0 + 2 * t;
-                if (kb >= KB) break;
-                const int st = kb / KBS, kbs = kb % KBS;
-                const int slot = st % S;
-                if (kbs < 2) ptx::mbar_wait(fullC + 8 * slot, (st / S) & 1, p.err);
-                const int a = kb % kASlots;
-                if (kb >= kASlots) ptx::mbar_wait<false>(emptyA + 8 * a, ((kb / kASlots) - 1) & 1, p.err);
-                uint32_t w[BITS * 2];
-#pragma unroll
-                for (int i = 0; i < BITS * 2; ++i) w[i] = 0;  // code 0 (a = 1) for lanes without a row
-                if (valid) {
-                    const uint8_t *row = gbase + (c0 - base) + slot * p.stage_bytes + j * 128;
-#pragma unroll
-                    for (int c = 0; c < BITS / 2; ++c) {
-                        const int chunk = (kbs * (BITS / 2) + c) ^ (j & 7);
-                        const uint4 u = *reinterpret_cast<const uint4 *>(row + (chunk << 4));
-                        w[4 * c] = u.x;
-                        w[4 * c + 1] = u.y;
-                        w[4 * c + 2] = u.z;
-                        w[4 * c + 3] = u.w;
-                    }
+                for (int c = 0; c < BITS; ++c) {     // BITS chunks of 16 bytes = 128 codes
+                    const int chunk = (sp * BITS + c) ^ (j & 7);
+                    const uint4 u = *reinterpret_cast<const uint4 *>(row + (chunk << 4));
+                    w[4 * c] = u.x;
+                    w[4 * c + 1] = u.y;
+                    w[4 * c + 2] = u.z;
+                    w[4 * c + 3] = u.w;
                 }
-                __syncwarp();
-                // This group's reads of the stage are done after its last k-block there.
-                if (lane == 0 && kbs >= KBS - 2) ptx::mbar_arrive(emptyC + 8 * slot);
-                uint32_t v[32];
-                place_codes<T, BITS>(w, v);
-                tc_fence_after();
-                tmem_st32(tmem + ((uint32_t)(32 * q) << 16) + 32u * a, v);
             }
-            tmem_st_wait();
-            tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
+            // This group's reads of the stage are done after its last slot there.
+            if (lane == 0 && sp >= SPC - 2) ptx::mbar_arrive(emptyC + 8 * slot);
+            if (valid) {
+                uint32_t o[32];
+                expand_codes<BITS>(w, o);
+                uint8_t *dst = gbase + (a0 - base) + as * p.a_bytes + arow;
 #pragma unroll
-                for (int t = 0; t < kPlaceBatch; ++t) {
-                    const int kb = kb0 + 2 * t;
-                    if (kb < KB) ptx::mbar_arrive(fullA + 8 * (kb % kASlots));
-                }
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(dst + ((c ^ (j & 7)) << 4)) =
+                        make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
             }
+            ptx::fence_proxy_async_smem();  // generic writes -> tensor-core reads
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(fullA + 8 * as);
         }
     } else {
         // ---------------- epilogue ----------------
         const int q = warp & 3;
-        const int j = q * p.RQ + lane;
-        const bool valid = lane < p.RQ && j < R;
+        const int j = 32 * q + lane;
         const int64_t rowg = (int64_t)r0 + j;
+        const bool valid = j < R;
         const uint16_t *srow = p.scales + (valid ? rowg : 0) * p.gpr;
         const uint16_t *brow = p.biases + (valid ? rowg : 0) * p.gpr;
-        // Scale/bias windows of 8 groups (16 bytes), one window ahead.
-        uint4 s_cur = make_uint4(0, 0, 0, 0), b_cur = s_cur, s_nxt = s_cur, b_nxt = s_cur;
-        if (valid) {
-            s_cur = __ldg(reinterpret_cast<const uint4 *>(srow));
-            b_cur = __ldg(reinterpret_cast<const uint4 *>(brow));
-            if (G > 8) {
-                s_nxt = __ldg(reinterpret_cast<const uint4 *>(srow + 8));
-                b_nxt = __ldg(reinterpret_cast<const uint4 *>(brow + 8));
-            }
-        }
         float acc[MR];
 #pragma unroll
         for (int m = 0; m < MR; ++m) acc[m] = 0.f;
-        int wbase = 0;
         for (int g = 0; g < G; ++g) {
             const int d = g & (kDSlots - 1);
-            if (g >= wbase + 8) {
-                s_cur = s_nxt;
-                b_cur = b_nxt;
-                wbase += 8;
-                if (valid && wbase + 8 < G) {
-                    s_nxt = __ldg(reinterpret_cast<const uint4 *>(srow + wbase + 8));
-                    b_nxt = __ldg(reinterpret_cast<const uint4 *>(brow + wbase + 8));
-                }
-            }
+            const int bt = g / gpb, bs = bt % kBStages, gl = g - bt * gpb;
+            // The table of this activation stage came with its h/l tiles.
+            if (gl == 0) ptx::mbar_wait<false>(fullB + 8 * bs, (bt / kBStages) & 1, p.err);
+            const uint16_t s16 = valid ? __ldg(srow + g) : (uint16_t)0;
+            const uint16_t b16 = valid ? __ldg(brow + g) : (uint16_t)0;
+            const float s = kF16 ? __half2float(__ushort_as_half(s16)) : __uint_as_float((uint32_t)s16 << 16);
+            const float bv = kF16 ? __half2float(__ushort_as_half(b16)) : __uint_as_float((uint32_t)b16 << 16);
+            const float2 *tb =
+                reinterpret_cast<const float2 *>(gbase + (b0 - base) + bs * kBStage + kSlotsPerB * kBTile) + gl * 16;
             ptx::mbar_wait<false>(fullD + 8 * d, (g / kDSlots) & 1, p.err);
             tc_fence_after();
-            uint32_t v[MR];
-            tmem_ld_cols<MR>(tmem + ((uint32_t)(32 * q) << 16) + kDCol0 + 16u * d, v);
+            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + 32u * d;
+            uint32_t vh[MR], vl[MR];
+            tmem_ld_cols<MR>(taddr, vh);
+            tmem_ld_cols<MR>(taddr + 16u, vl);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(emptyD + 8 * d);
-            const int o = g - wbase;
-            const uint32_t sw = pick_word(s_cur, o >> 1), bw = pick_word(b_cur, o >> 1);
-            const uint16_t s16 = (uint16_t)((o & 1) ? (sw >> 16) : (sw & 0xffffu));
-            const uint16_t b16 = (uint16_t)((o & 1) ? (bw >> 16) : (bw & 0xffffu));
-            const float s = kF16 ? __half2float(__ushort_as_half(s16)) : __uint_as_float((uint32_t)s16 << 16);
-            const float bv = kF16 ? __half2float(__ushort_as_half(b16)) : __uint_as_float((uint32_t)b16 << 16);
-            const float sp = s * QS;                   // exact
 #pragma unroll
             for (int m = 0; m < MR; ++m) {
-                const float dm = __uint_as_float(v[m]);
-                const float xs = __shfl_sync(0xffffffffu, dm, 31);  // X_g[m] from the all-ones lane
-                // (QS s)(D - X) + b X: the difference first, so that no term is
-                // larger than the result's own scale.
-                acc[m] = __fmaf_rn(sp, dm - xs, __fmaf_rn(bv, xs, acc[m]));
+                const float2 px = tb[m];                  // (2^-e, X_g[m])
+                const float v = __fmaf_rn(256.f, small_int_to_f(vh[m]), small_int_to_f(vl[m]));
+                acc[m] = __fmaf_rn(s * px.x, v, __fmaf_rn(bv, px.y, acc[m]));
             }
+            // The stage's table has been read by this warp after its last group.
+            __syncwarp();
+            if (lane == 0 && gl == gpb - 1) ptx::mbar_arrive(emptyB + 8 * bs);
         }
         if (valid) {
             T *y = static_cast<T *>(p.y);
@@ -501,23 +514,22 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const DecParams p) {
 }
 
 struct TcPlan {
-    int grid, R, RQ, S, stage_bytes;
+    int grid, R, S, stage_bytes, a_bytes;
     size_t smem;
 };
 
-bool plan_tc(const QmmArgs &a, int mr, TcPlan &p) {
+bool plan_tc(const QmmArgs &a, TcPlan &p) {
     const int64_t sms = num_sms();
     int64_t G = std::min<int64_t>(sms, (a.N + 7) / 8);
     int64_t R = std::min<int64_t>((a.N + G - 1) / G, kMaxRows);
     G = (a.N + R - 1) / R;  // every CTA owns at least one row
     p.grid = (int)G;
     p.R = (int)R;
-    p.RQ = (int)((R + 3) / 4);
     p.stage_bytes = (int)(((R * 128) + 1023) / 1024 * 1024);
-    const int nb = mr <= 8 ? 8 : 16;
-    const size_t bring = (size_t)2 * kBStageKb * nb * 128 + (nb == 8 ? 1024 : 0);
+    p.a_bytes = (int)(((R + 7) / 8) * 1024);
+    const size_t ring_b = (size_t)kBStages * kBStage;
     const size_t bars = 512;
-    const size_t fixed = 1024 /*alignment*/ + bring + bars;
+    const size_t fixed = 1024 /*alignment*/ + (size_t)kASlots * p.a_bytes + ring_b + bars;
     if (fixed + 2 * (size_t)p.stage_bytes > kSmemBudget) return false;
     p.S = (int)std::min<size_t>(8, (kSmemBudget - fixed) / p.stage_bytes);
     p.smem = fixed + (size_t)p.S * p.stage_bytes;
@@ -528,7 +540,7 @@ template <typename T, int BITS, int MR>
 cudaError_t launch_tc(const QmmArgs &a, cudaStream_t s) {
     auto kern = qgemv_tc_kernel<T, BITS, MR>;
     TcPlan p{};
-    if (!plan_tc(a, MR, p)) return cudaErrorInvalidValue;
+    if (!plan_tc(a, p)) return cudaErrorInvalidValue;
     struct Tag;
     cudaError_t e = configure_once<Tag>(p.smem, [&]() {
         cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
@@ -537,15 +549,41 @@ cudaError_t launch_tc(const QmmArgs &a, cudaStream_t s) {
                                     cudaSharedmemCarveoutMaxShared);
     });
     if (e != cudaSuccess) return e;
+    uint8_t *ws = static_cast<uint8_t *>(a.ws) + kWsFlagBytes;
+    const int gs_log = __builtin_ctz((unsigned)a.group_size);
     // Packed codes as [N rows, K*BITS/32 words]: a box is 32 words (128 bytes)
-    // of R rows, 128-byte swizzled; rows past N read as zero.
-    CUtensorMap tw;
+    // of R rows, 128-byte swizzled; rows past N read as zero.  h/l, [32, K]
+    // bytes, viewed as [K/128 slots][32 rows][128 bytes]: a box is the 32 x 128
+    // tiles of kSlotsPerB consecutive slots, 128-byte swizzled, tile after tile.
+    CUtensorMap tw, tb;
     const uint64_t words = (uint64_t)a.K * BITS / 32;
     if (!make_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.wq, words, (uint64_t)a.N, words * 4, 32,
                      (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    DecParams dp{};
-    dp.x = a.x;
+    {
+        const uint64_t dims[3] = {128, 32, (uint64_t)a.K / 128};
+        const uint64_t strides[2] = {(uint64_t)a.K, 128};
+        const uint32_t box[3] = {128, 32, (uint32_t)kSlotsPerB};
+        if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, ws, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    {
+        const int64_t threads = a.M * (a.K / 16);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)((threads + 255) / 256), 1, 1);
+        cfg.blockDim = dim3(256, 1, 1);
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, qdecode_prep_kernel<T, BITS>, static_cast<const T *>(a.x), (int)a.M,
+                               (int)a.K, gs_log, ws);
+        if (e != cudaSuccess) return e;
+        count_launches(1);
+    }
+    I8Params dp{};
     dp.y = a.y;
     dp.scales = static_cast<const uint16_t *>(a.scales);
     dp.biases = static_cast<const uint16_t *>(a.biases);
@@ -553,26 +591,23 @@ cudaError_t launch_tc(const QmmArgs &a, cudaStream_t s) {
     dp.N = (int)a.N;
     dp.K = (int)a.K;
     dp.gpr = (int)(a.K / a.group_size);
-    dp.gs_log = __builtin_ctz((unsigned)a.group_size);
+    dp.gs_log = gs_log;
     dp.R = p.R;
-    dp.RQ = p.RQ;
     dp.S = p.S;
     dp.stage_bytes = p.stage_bytes;
-    dp.KB = (int)(a.K / 64);
+    dp.a_bytes = p.a_bytes;
     dp.bias = a.bias;
     dp.bias_value = a.bias_value;
     dp.err = device_error_word();
+    const float2 *tab = reinterpret_cast<const float2 *>(ws + (size_t)32 * a.K);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, tw, dp);
+    e = cudaLaunchKernelEx(&cfg, kern, tw, tb, tab, dp);
     if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();
@@ -589,21 +624,30 @@ cudaError_t tc_rows(const QmmArgs &a, cudaStream_t s) {
 
 }  // namespace
 
+// Workspace of the decode tensor-core path: past the leading flag bytes
+// (left untouched), h/l as [32, K] bytes and the (2^-e, X) table,
+// K / group_size x 16 float2, at most K / 32 groups.
+size_t gemv_tc_workspace_bytes(int64_t K) {
+    return kWsFlagBytes + (size_t)32 * (size_t)K + (size_t)(K / 32) * 16 * sizeof(float2);
+}
+
 // bf16/f16, transpose, 1..16 rows, 2- or 4-bit codes, K a multiple of 512
-// (whole activation stages and code chunks), groups per row a multiple of 8
-// (16-byte scale/bias windows), 16-byte aligned operands.
+// (whole code chunks), group size 32/64/128, 16-byte aligned operands.  (The
+// call also needs a workspace of gemv_tc_workspace_bytes(K), checked apart.)
 bool gemv_tc_supported(qmm_dtype dt, const QmmArgs &a) {
     if (!a.transpose || a.M < 1 || a.M > 16) return false;
     if (dt != QMM_BF16 && dt != QMM_F16) return false;
     if (a.mode != QMM_MODE_AFFINE) return false;
     if (a.bits != 2 && a.bits != 4) return false;
-    if (a.K % 512 != 0 || (a.K / a.group_size) % 8 != 0) return false;
+    if (a.group_size < 32 || a.group_size > 128) return false;
+    if (a.K % 512 != 0) return false;
     if (a.N < 1 || a.N > (1 << 30) || a.K > (1 << 20)) return false;
     if ((reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.wq) |
-         reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases)) & 15)
+         reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases) |
+         reinterpret_cast<uintptr_t>(a.ws)) & 15)
         return false;
     TcPlan p{};
-    if (!plan_tc(a, a.M <= 8 ? 8 : 16, p)) return false;
+    if (!plan_tc(a, p)) return false;
     return encode_fn() != nullptr;
 }
 

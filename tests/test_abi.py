@@ -142,3 +142,26 @@ def test_matmul_workspace_size(L):
 def test_fault_injection_rejects_unknown_values(L):
     assert L.qmm_inject_fault(99) == 1
     assert L.qmm_inject_fault(0) == 0
+
+
+def mmhost(L, xh=FAKE, yh=FAKE, **kw):
+    a = dict(x=FAKE, M=2, K=128, wq=FAKE, s=FAKE, b=FAKE, dtype=1, N=64, tr=1, gs=64,
+             bits=4, mode=None, y=FAKE)
+    a.update(kw)
+    return L.qmm_quantized_matmul_host(xh, a["x"], a["M"], a["K"], a["wq"], a["s"], a["b"],
+                                       a["dtype"], a["N"], a["tr"], a["gs"], a["bits"], a["mode"],
+                                       a["y"], yh, NULL, 0, NULL)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(xh=NULL), 1), (dict(yh=NULL), 1), (dict(K=96), 1), (dict(b=NULL), 1),
+    (dict(x=MISALIGNED), 1), (dict(bits=7), 1), (dict(mode=b"nvfp4"), 1),
+])
+def test_matmul_host_rejects_before_any_copy(L, kw, status):
+    """The host-buffer entry checks every argument (and that the host buffers
+    are given) before it enqueues a copy: these calls touch no device."""
+    assert mmhost(L, **kw) == status
+
+
+def test_matmul_host_empty_is_a_noop(L):
+    assert mmhost(L, M=0, x=NULL, y=NULL, xh=NULL, yh=NULL) == 0
