@@ -362,7 +362,8 @@ qmm_status qmm_inject_fault(qmm_fault fault);
  * is QMM_PATH_AUTO).  QMM_PATH_GEMV forces the SIMT decode kernels (M <= 16
  * rows at a time), QMM_PATH_GEMM the tensor-core (tcgen05) GEMM, and
  * QMM_PATH_DECODE_TC the decode tensor-core kernel (bf16/f16, transpose,
- * 1..16 rows, 2- or 4-bit codes, group size 32..128, K % 512 == 0; two
+ * 1..16 rows, 2- or 4-bit codes, group size 32..128, K % 512 == 0,
+ * (K / group_size) % 8 == 0; two
  * launches per call: a prep kernel turns x into per-group block fixed point
  * (16-bit integers split into a signed and an unsigned byte, error below
  * 2^-15 of the group's largest |x|) in the workspace, then an integer MMA

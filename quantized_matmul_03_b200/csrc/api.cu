@@ -331,7 +331,8 @@ qmm_status route_matmul(qmm_dtype dtype, const QmmArgs &a, cudaStream_t s) {
             if (!gemv_tc_supported(dtype, a))
                 return fail(QMM_ERR_UNSUPPORTED,
                             "the decode tensor-core path needs bf16/f16, transpose, 1..16 rows, 2- or "
-                            "4-bit codes, group size 32..128, K %% 512 == 0, 16-byte aligned operands");
+                            "4-bit codes, group size 32..128, K %% 512 == 0, (K / group_size) %% 8 == 0, "
+                            "16-byte aligned operands");
             if (a.ws == nullptr || a.ws_bytes < gemv_tc_workspace_bytes(a.K))
                 return fail(QMM_ERR_WORKSPACE,
                             "the decode tensor-core path needs a workspace of "

@@ -13,37 +13,47 @@
 //     group's largest |x| so that x_int is a 16-bit integer (representation
 //     error below 2^-15 of that largest |x|; 2^-14 for a value that rounds
 //     up to 2^15 and is held at 2^15 - 1), split as x_int = 256 h + l with
-//     h in [-128, 127] (s8) and l in [0, 255] (u8);  X_g[m] = sum of x (fp32);
+//     h in [-128, 127] and l in [0, 255];  X_g[m] = sum of x (fp32);
 //   codes: a 4-bit word w gives the bytes (w & 0x0F0F0F0F) = codes 0,2,4,6
 //     and ((w >> 4) & 0x0F0F0F0F) = codes 1,3,5,7 (2-bit: four planes, codes
 //     p, 4+p, 8+p, 12+p), so the A operand holds each word's codes in that
 //     order, and h and l are stored in the same order;
-//   per group: D_h = sum q h and D_l = sum q l (two MMAs, s8 and u8 B; both
-//     below 2^22 in magnitude for codes of at most 4 bits and groups of at
-//     most 128), then  y[m, n] += s 2^-e (256 D_h + D_l) + b X_g[m]  in fp32.
+//   per group one unsigned MMA per K = 32 against B rows (h + 128, l, 1):
+//     D_h' = sum q (h + 128), D_l = sum q l and D_1 = sum q, so
+//     D_h = D_h' - 128 D_1 exactly (all below 2^22 in magnitude for codes of
+//     at most 4 bits and groups of at most 128), then
+//     y[m, n] += s 2^-e (256 D_h + D_l) + b X_g[m]  in fp32.
 // A prep kernel writes h, l, 2^-e and X_g once per call into the workspace;
 // the product kernel reads them with tensor copies.
 //
 // Orientation: UMMA M = 128 over weight rows (each CTA owns R <= 128
 // contiguous rows; A rows past R are never read back), UMMA N = 16 over
-// activation rows (h rows and l rows), K = 32 per instruction; per group one
-// accumulator of 32 columns (16 for D_h, 16 for D_l), a ring of 16.
+// activation rows (48 B rows: 16 of h + 128, 16 of l, the row of ones and
+// padding), K = 32 per instruction; per group one accumulator of 48 columns,
+// a ring of 10.
 //
-// Roles (512 threads, two CTAs per SM: the next call's CTA fits beside this
-// one and streams its first codes while this one finishes):
+// Roles (640 threads, one CTA per SM with deep rings: every code stage, A
+// slot and accumulator in flight hides part of the MMA round trip, which a
+// shallow ring exposed once per slot):
 //   warps 0, 1   tensor copies of the packed codes, 128 bytes of every owned
 //                row per stage (alternate stages), 128-byte swizzled;
-//   warp 2       waits for the prep kernel (griddepcontrol.wait), then copies
-//                per four A slots their h/l tiles (one 3-D tensor copy of 4 x
-//                32 rows x 128 bytes: a tensor copy costs its issuing thread
-//                several hundred cycles, whatever its size) and the groups'
-//                (2^-e, X) table;
+//   warp 2       waits for the prep kernel (griddepcontrol.wait), copies the
+//                call's whole (2^-e, X) table once (its own area: were it
+//                carried with the B tiles, a B stage could be refilled only
+//                after the epilogue had finished its groups, which paced the
+//                whole pipeline), then per four A slots their B tiles (one
+//                3-D tensor copy of 4 x 48 rows x 128 bytes: a tensor copy
+//                costs its issuing thread several hundred cycles, whatever
+//                its size);
 //   warp 3       tensor-memory owner and MMA issuer (one elected lane);
 //   warps 4-11   code expansion: two groups of four warps take alternate A
 //                slots (128 codes of every row, 128-byte swizzled K-major u8);
-//   warps 12-15  epilogue: per group, tcgen05.ld of the quadrant's D_h and
-//                D_l, the step above in fp32 registers, and one store of y
-//                per row at the end.
+//   warps 12-19  epilogue, two halves of four (one warp per lane quadrant)
+//                taking alternate groups, two of them per round (one wait
+//                for six tensor-memory loads): the step above in fp32
+//                registers, two activation rows per packed f32x2
+//                instruction; at the end the halves' sums are added through
+//                shared memory and y stored per row.
 // Every wait is bounded (device error word on timeout); before exiting or
 // freeing tensor memory a CTA waits, with the fixed limit, for its own copies
 // and MMAs.  No cluster multicast is used.
@@ -57,33 +67,27 @@
 namespace qmm {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 640;
 constexpr int kWarpB = 2, kWarpMma = 3, kWarpUnp = 4, kWarpEpi = 12;
-constexpr int kASlots = 2;          // A slots: 128 codes x R rows, u8
+constexpr int kEpiWarps = 8;
+constexpr int kASlots = 6;          // A slots: 128 codes x R rows, u8
 constexpr int kSlotsPerB = 4;       // A slots per activation stage
 constexpr int kBStages = 2;         // activation ring
-constexpr int kBTile = 4096;        // h/l tile of one A slot: 32 rows x 128 bytes
-constexpr int kBStage = kSlotsPerB * kBTile + 2048;  // + the stage's table (<= 16 groups)
-constexpr int kDSlots = 16;         // group accumulators, 32 columns each
+constexpr int kBRows = 48;          // h + 128 (16), l (16), ones (1), padding
+constexpr int kBTile = kBRows * 128;  // B tile of one A slot
+constexpr int kBStage = kSlotsPerB * kBTile;
+constexpr int kMaxGroups = 128;     // groups per row whose table fits (16 KB)
+constexpr int kDCols = kBRows;      // accumulator columns per group
+constexpr int kDSlots = 10;         // group accumulators (10 x 48 of 512 columns)
 constexpr uint32_t kTmemCols = 512;
-constexpr int kTmemThreads = 32 * (16 - kWarpMma);  // warps that use tensor memory
+constexpr int kTmemThreads = 32 * (kThreads / 32 - kWarpMma);  // warps that use tensor memory
 constexpr int kMaxRows = 128;
-constexpr size_t kSmemBudget = 110 * 1024;
+constexpr size_t kSmemBudget = 220 * 1024;
 
-// Per-SM hand-off between consecutive CTAs of this kernel (see the decode
-// kernel in gemv_fast.cu): a CTA issues its first copy once the CTA before it
-// on the same SM has at most one stage left to issue, or after a short bound.
-// It orders memory traffic only; results do not depend on it.
-constexpr int kMaxSm = 1024;
-constexpr uint64_t kHandoffWaitNs = 20000;
-__device__ unsigned long long g_tc_ticket[kMaxSm];
-__device__ unsigned long long g_tc_issued[kMaxSm];
-
-// Instruction descriptors of kind::i8: s32 accumulator, A u8 (codes), B s8
-// (h) or u8 (l), both K-major, M = 128, N = 16.
-constexpr uint32_t idesc_i8(bool b_signed) {
-    return (2u << 4) | (0u << 7) | ((b_signed ? 1u : 0u) << 10) | ((uint32_t)(16 >> 3) << 17) |
-           ((uint32_t)(128 >> 4) << 24);
+// Instruction descriptor of kind::i8: s32 accumulator, A and B u8, both
+// K-major, M = 128, N = kBRows.
+constexpr uint32_t idesc_u8() {
+    return (2u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(kBRows >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 __device__ __forceinline__ void tc_mma_i8(uint32_t tmem_d, uint64_t desc_a, uint64_t desc_b,
                                           uint32_t idesc, uint32_t accumulate) {
@@ -122,9 +126,9 @@ struct I8Params {
 };
 
 // ---------------------------------------------------------------------------
-// Prep: activations -> h, l (permuted byte order), (2^-e, X) per (group, row).
-// Workspace: [32][K] bytes (rows 0..15 h, 16..31 l; rows past M unused) then
-// [K / group_size][16] float2.  One thread per (row, 16-element chunk); the
+// Prep: activations -> h + 128, l (permuted byte order), (2^-e, X) per
+// (group, row).  Workspace: [48][K] bytes (rows 0..15 h + 128, 16..31 l, 32
+// ones; rows past M and rows 33..47 unused) then [K / group_size][16] float2.  One thread per (row, 16-element chunk); the
 // gs/16 threads of a group are adjacent lanes.
 // ---------------------------------------------------------------------------
 template <typename T, int BITS>
@@ -177,15 +181,17 @@ qdecode_prep_kernel(const T *__restrict__ x, int M, int K, int gs_log, uint8_t *
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
         const int xi = min(32767, __float2int_rn(v[perm_elem<BITS>(j)] * up));
-        const uint32_t hb = (uint32_t)(xi >> 8) & 0xffu, lb = (uint32_t)xi & 0xffu;
+        const uint32_t hb = (uint32_t)((xi >> 8) + 128) & 0xffu, lb = (uint32_t)xi & 0xffu;
         hw[j >> 2] |= hb << (8 * (j & 3));
         lw[j >> 2] |= lb << (8 * (j & 3));
     }
     uint8_t *row_h = ws + (int64_t)m * K + 16 * c;
     *reinterpret_cast<uint4 *>(row_h) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
     *reinterpret_cast<uint4 *>(row_h + (int64_t)16 * K) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    if (m == 0) *reinterpret_cast<uint4 *>(ws + (int64_t)32 * K + 16 * c) = make_uint4(0x01010101u, 0x01010101u,
+                                                                                        0x01010101u, 0x01010101u);
     if ((c & (tpg - 1)) == 0) {
-        float2 *tab = reinterpret_cast<float2 *>(ws + (int64_t)32 * K);
+        float2 *tab = reinterpret_cast<float2 *>(ws + (int64_t)48 * K);
         tab[(int64_t)(c >> (gs_log - 4)) * 16 + m] = make_float2(__uint_as_float((uint32_t)(127 - e) << 23), sum);
     }
 }
@@ -238,21 +244,15 @@ template <> __device__ __forceinline__ void tmem_ld_cols<16>(uint32_t taddr, uin
         : "memory");
 }
 
-// An int32 of magnitude below 2^22 as a float, exactly, with two full-rate
-// operations (integer add into the mantissa of 1.5 * 2^23, then subtract it).
-__device__ __forceinline__ float small_int_to_f(uint32_t v) {
-    return __uint_as_float(v + 0x4B400000u) - 12582912.0f;
-}
-
 // MR: activation rows the kernel is built for (1, 2, 4, 8, 16; the call has
 // M <= MR).  The MMAs always use N = 16 (h and l tiles of 16 rows each).
 template <typename T, int BITS, int MR>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
 qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_b,
                 const float2 *__restrict__ tab, const I8Params p) {
     constexpr bool kF16 = std::is_same<T, __half>::value;
     constexpr int SPC = 512 / (BITS * 64);         // A slots per 128-byte code chunk (4-bit 2, 2-bit 4)
-    constexpr uint32_t ID_H = idesc_i8(true), ID_L = idesc_i8(false);
+    constexpr uint32_t IDESC = idesc_u8();
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = ptx::smem_addr(smem_raw);
@@ -264,13 +264,15 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
     // (the MMA reads 128 rows of an A slot; rows past R of the last slot fall
     // into the B ring that follows, inside the allocation)
     const uint32_t b0 = a0 + (uint32_t)kASlots * (uint32_t)p.a_bytes;  // B ring
-    const uint32_t bar0 = b0 + kBStages * kBStage;
+    const uint32_t red0 = b0 + kBStages * kBStage;  // epilogue halves: MR x 128 floats
+    const uint32_t tab0 = red0 + (uint32_t)MR * 128u * 4u;  // (2^-e, X) per (group, row)
+    const uint32_t bar0 = tab0 + (uint32_t)kMaxGroups * 128u;
     const uint32_t fullC = bar0, emptyC = fullC + 8 * S;
     const uint32_t fullA = emptyC + 8 * S, emptyA = fullA + 8 * kASlots;
     const uint32_t fullB = emptyA + 8 * kASlots, emptyB = fullB + 8 * kBStages;
     const uint32_t fullD = emptyB + 8 * kBStages, emptyD = fullD + 8 * kDSlots;
-    const uint32_t done = emptyD + 8 * kDSlots, go = done + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + (go + 8 - base));
+    const uint32_t done = emptyD + 8 * kDSlots, fullT = done + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + (fullT + 8 - base));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r0 = blockIdx.x * p.R;
@@ -278,8 +280,6 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
     const int NA = p.K >> 7;                       // A slots (128 codes each)
     const int NST = NA / SPC;                      // code stages
     const int G = p.K >> p.gs_log;                 // groups per row
-    const int gpa = 128 >> p.gs_log;               // groups per A slot
-    const int gpb = gpa * kSlotsPerB;              // groups per activation stage
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             ptx::mbar_init(fullC + 8 * s, 1);
@@ -291,14 +291,14 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
         }
         for (int b = 0; b < kBStages; ++b) {
             ptx::mbar_init(fullB + 8 * b, 1);
-            ptx::mbar_init(emptyB + 8 * b, 5);     // the MMAs' commit + the four epilogue warps
+            ptx::mbar_init(emptyB + 8 * b, 1);     // the MMAs' commit
         }
         for (int d = 0; d < kDSlots; ++d) {
             ptx::mbar_init(fullD + 8 * d, 1);
-            ptx::mbar_init(emptyD + 8 * d, 4);     // the four epilogue warps
+            ptx::mbar_init(emptyD + 8 * d, 4);     // the four epilogue warps of the group's half
         }
         ptx::mbar_init(done, 1);
-        ptx::mbar_init(go, 1);
+        ptx::mbar_init(fullT, 1);
         ptx::fence_mbar_init();
     }
     __syncthreads();  // barriers initialised
@@ -325,33 +325,12 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
     if (warp < kWarpB) {
         // ---------------- packed-code producers ----------------
         if (lane == 0) {
-            uint32_t smid;
-            asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-            const bool handoff = smid < (uint32_t)kMaxSm;
-            unsigned long long ticket = 0;
-            if (warp == 0) {
-                if (handoff) {
-                    ticket = atomicAdd(&g_tc_ticket[smid], 1ull);
-                    const uint64_t t0 = ptx::globaltimer_ns();
-                    for (;;) {
-                        unsigned long long dn;
-                        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(dn) : "l"(&g_tc_issued[smid]));
-                        if (dn >= ticket || ptx::globaltimer_ns() - t0 > kHandoffWaitNs) break;
-                        __nanosleep(128);
-                    }
-                }
-                ptx::mbar_arrive(go);
-            } else {
-                ptx::mbar_wait(go, 0, p.err);
-            }
             for (int st = warp; st < NST; st += 2) {
                 const int slot = st % S;
                 if (st >= S) ptx::mbar_wait(emptyC + 8 * slot, ((st / S) - 1) & 1, p.err);
                 ptx::mbar_arrive_expect_tx(fullC + 8 * slot, (uint32_t)p.R * 128u);
                 tma_load_2d(c0 + (uint32_t)slot * (uint32_t)p.stage_bytes, &tmap_w, st * 32, r0, fullC + 8 * slot);
-                if (warp == 0 && handoff && st >= NST - 2) atomicMax(&g_tc_issued[smid], ticket + 1);
             }
-            if (warp == 0 && handoff) atomicMax(&g_tc_issued[smid], ticket + 1);
             // The CTA must not exit while a copy into its ring can still land.
             for (int st = max(0, NST - S); st < NST; ++st)
                 if ((st & 1) == warp) ptx::mbar_drain(fullC + 8 * (st % S), (st / S) & 1, p.err);
@@ -361,18 +340,19 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
         if (lane == 0) {
             // The workspace is written by this call's prep kernel: wait for it.
             ptx::grid_dependency_wait();
-            const uint32_t tbytes = (uint32_t)gpb * 16u * 8u;
+            ptx::mbar_arrive_expect_tx(fullT, (uint32_t)G * 128u);
+            ptx::bulk_g2s(tab0, tab, (uint32_t)G * 128u, fullT);
             const int NB = NA / kSlotsPerB;
             for (int bt = 0; bt < NB; ++bt) {
                 const int bs = bt % kBStages;
                 if (bt >= kBStages) ptx::mbar_wait(emptyB + 8 * bs, ((bt / kBStages) - 1) & 1, p.err);
                 const uint32_t dst = b0 + (uint32_t)bs * kBStage;
-                ptx::mbar_arrive_expect_tx(fullB + 8 * bs, (uint32_t)(kSlotsPerB * kBTile) + tbytes);
+                ptx::mbar_arrive_expect_tx(fullB + 8 * bs, (uint32_t)(kSlotsPerB * kBTile));
                 tma_load_3d(dst, &tmap_b, 0, 0, bt * kSlotsPerB, fullB + 8 * bs);
-                ptx::bulk_g2s(dst + kSlotsPerB * kBTile, tab + (int64_t)bt * gpb * 16, tbytes, fullB + 8 * bs);
             }
             for (int bt = max(0, NB - kBStages); bt < NB; ++bt)
                 ptx::mbar_drain(fullB + 8 * (bt % kBStages), (bt / kBStages) & 1, p.err);
+            ptx::mbar_drain(fullT, 0, p.err);
         }
     } else if (warp == kWarpMma) {
         // ---------------- MMA issuer ----------------
@@ -386,20 +366,18 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
                 tc_fence_after();
                 const uint32_t btile = b0 + (uint32_t)bs * kBStage + (uint32_t)sub * kBTile;
                 const uint64_t da = sw128_desc(a0 + (uint32_t)as * (uint32_t)p.a_bytes);
-                const uint64_t dh = sw128_desc(btile);
-                const uint64_t dl = sw128_desc(btile + 2048u);
+                const uint64_t db = sw128_desc(btile);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int e0 = a * 128 + 32 * j;
-                    const int g = e0 >> p.gs_log, d = g & (kDSlots - 1);
+                    const int g = e0 >> p.gs_log, d = g % kDSlots;
                     const bool first = (e0 & gs_mask) == 0, last = ((e0 + 32) & gs_mask) == 0;
                     if (first && g >= kDSlots) {
                         ptx::mbar_wait<false>(emptyD + 8 * d, ((g / kDSlots) - 1) & 1, p.err);
                         tc_fence_after();
                     }
                     // K = 32 bytes per instruction: 2 units of 16 bytes along the rows.
-                    tc_mma_i8(tmem + 32u * d, da + 2u * j, dh + 2u * j, ID_H, first ? 0u : 1u);
-                    tc_mma_i8(tmem + 32u * d + 16u, da + 2u * j, dl + 2u * j, ID_L, first ? 0u : 1u);
+                    tc_mma_i8(tmem + (uint32_t)(kDCols * d), da + 2u * j, db + 2u * j, IDESC, first ? 0u : 1u);
                     if (last) tc_commit(fullD + 8 * d);
                 }
                 tc_commit(emptyA + 8 * as);
@@ -457,52 +435,97 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
         }
     } else {
         // ---------------- epilogue ----------------
-        const int q = warp & 3;
+        // Half h of the eight warps takes the groups g = h mod 2; warp (q, h)
+        // reads tensor-memory lane quadrant q (rows 32q..32q+31).
+        using namespace ptx;
+        constexpr int P = (MR + 1) / 2;             // pairs of activation rows
+        const int q = warp & 3, half = (warp - kWarpEpi) >> 2;
         const int j = 32 * q + lane;
         const int64_t rowg = (int64_t)r0 + j;
         const bool valid = j < R;
         const uint16_t *srow = p.scales + (valid ? rowg : 0) * p.gpr;
         const uint16_t *brow = p.biases + (valid ? rowg : 0) * p.gpr;
-        float acc[MR];
+        const unsigned long long mm = f2pack(12582912.0f, 12582912.0f), k256 = f2pack(256.f, 256.f);
+        unsigned long long acc[P];
 #pragma unroll
-        for (int m = 0; m < MR; ++m) acc[m] = 0.f;
-        for (int g = 0; g < G; ++g) {
-            const int d = g & (kDSlots - 1);
-            const int bt = g / gpb, bs = bt % kBStages, gl = g - bt * gpb;
-            // The table of this activation stage came with its h/l tiles.
-            if (gl == 0) ptx::mbar_wait<false>(fullB + 8 * bs, (bt / kBStages) & 1, p.err);
-            const uint16_t s16 = valid ? __ldg(srow + g) : (uint16_t)0;
-            const uint16_t b16 = valid ? __ldg(brow + g) : (uint16_t)0;
-            const float s = kF16 ? __half2float(__ushort_as_half(s16)) : __uint_as_float((uint32_t)s16 << 16);
+        for (int i = 0; i < P; ++i) acc[i] = 0ull;  // (+0.0, +0.0)
+        // Scales and biases of the row in 16-byte windows of 8 groups, the
+        // next window loaded while the current one is used (with most of
+        // the SM's on-chip memory given to shared memory, a 2-byte load per
+        // group would wait on L2 every time).
+        uint4 s_cur = make_uint4(0, 0, 0, 0), b_cur = s_cur, s_nxt = s_cur, b_nxt = s_cur;
+        if (valid) {
+            s_cur = __ldg(reinterpret_cast<const uint4 *>(srow));
+            b_cur = __ldg(reinterpret_cast<const uint4 *>(brow));
+            if (G > 8) {
+                s_nxt = __ldg(reinterpret_cast<const uint4 *>(srow + 8));
+                b_nxt = __ldg(reinterpret_cast<const uint4 *>(brow + 8));
+            }
+        }
+        int wbase = 0;
+        ptx::mbar_wait(fullT, 0, p.err);  // the call's (2^-e, X) table
+        for (int g = half; g < G; g += 2) {
+            const int d = g % kDSlots;
+            if (g >= wbase + 8) {
+                s_cur = s_nxt;
+                b_cur = b_nxt;
+                wbase += 8;
+                if (valid && wbase + 8 < G) {
+                    s_nxt = __ldg(reinterpret_cast<const uint4 *>(srow + wbase + 8));
+                    b_nxt = __ldg(reinterpret_cast<const uint4 *>(brow + wbase + 8));
+                }
+            }
+            const int o = g - wbase;
+            const uint32_t sw = pick_word(s_cur, o >> 1), bw = pick_word(b_cur, o >> 1);
+            const uint16_t s16 = (uint16_t)((o & 1) ? (sw >> 16) : (sw & 0xffffu));
+            const uint16_t b16 = (uint16_t)((o & 1) ? (bw >> 16) : (bw & 0xffffu));
+            const float sv = kF16 ? __half2float(__ushort_as_half(s16)) : __uint_as_float((uint32_t)s16 << 16);
             const float bv = kF16 ? __half2float(__ushort_as_half(b16)) : __uint_as_float((uint32_t)b16 << 16);
-            const float2 *tb =
-                reinterpret_cast<const float2 *>(gbase + (b0 - base) + bs * kBStage + kSlotsPerB * kBTile) + gl * 16;
             ptx::mbar_wait<false>(fullD + 8 * d, (g / kDSlots) & 1, p.err);
             tc_fence_after();
-            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + 32u * d;
-            uint32_t vh[MR], vl[MR];
+            const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kDCols * d);
+            uint32_t vh[MR], vl[MR], v1[1];
             tmem_ld_cols<MR>(taddr, vh);
             tmem_ld_cols<MR>(taddr + 16u, vl);
+            tmem_ld_cols<1>(taddr + 32u, v1);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(emptyD + 8 * d);
+            const float *tb = reinterpret_cast<const float *>(gbase + (tab0 - base)) + g * 32;
+            const unsigned long long s2 = f2pack(sv, sv), b2 = f2pack(bv, bv);
+            // D_h = D_h' - 128 D_1, moved into the mantissa of 1.5 * 2^23
+            const uint32_t ch = 0x4B400000u - (v1[0] << 7);
 #pragma unroll
-            for (int m = 0; m < MR; ++m) {
-                const float2 px = tb[m];                  // (2^-e, X_g[m])
-                const float v = __fmaf_rn(256.f, small_int_to_f(vh[m]), small_int_to_f(vl[m]));
-                acc[m] = __fmaf_rn(s * px.x, v, __fmaf_rn(bv, px.y, acc[m]));
+            for (int i = 0; i < P; ++i) {
+                // rows 2i and 2i+1 (MR = 1: lane 1 repeats row 0 and is dropped)
+                const int m0 = 2 * i, m1 = MR > 1 ? 2 * i + 1 : 0;
+                // D_h and D_l are below 2^22 in magnitude: exact as floats by
+                // the 1.5 * 2^23 bias; then 256 D_h + D_l, and the group's step
+                // s 2^-e (256 D_h + D_l) + b X with (2^-e, X) from the table
+                const unsigned long long fh = f2sub(u2pack(vh[m0] + ch, vh[m1] + ch), mm);
+                const unsigned long long fl = f2sub(u2pack(vl[m0] + 0x4B400000u, vl[m1] + 0x4B400000u), mm);
+                const float4 t = *reinterpret_cast<const float4 *>(tb + 2 * m0);  // p0, X0, p1, X1
+                const unsigned long long sp = f2mul(s2, f2pack(t.x, t.z));
+                acc[i] = f2fma(sp, f2fma(k256, fh, fl), f2fma(b2, f2pack(t.y, t.w), acc[i]));
             }
-            // The stage's table has been read by this warp after its last group.
-            __syncwarp();
-            if (lane == 0 && gl == gpb - 1) ptx::mbar_arrive(emptyB + 8 * bs);
         }
-        if (valid) {
+        float accf[2 * P];
+#pragma unroll
+        for (int i = 0; i < P; ++i) f2unpack(acc[i], accf[2 * i], accf[2 * i + 1]);
+        // The odd-group half hands its sums to the even-group half.
+        float *red = reinterpret_cast<float *>(gbase + (red0 - base));
+        if (half == 1) {
+#pragma unroll
+            for (int m = 0; m < MR; ++m) red[m * 128 + j] = accf[m];
+        }
+        asm volatile("bar.sync 2, %0;" ::"r"(32 * kEpiWarps) : "memory");
+        if (half == 0 && valid) {
             T *y = static_cast<T *>(p.y);
             const float lb = layer_bias<T>(p.bias, p.bias_value, rowg);
 #pragma unroll
             for (int m = 0; m < MR; ++m)
-                if (m < p.M) y[(int64_t)m * p.N + rowg] = Dt<T>::from_f(acc[m] + lb);
+                if (m < p.M) y[(int64_t)m * p.N + rowg] = Dt<T>::from_f(accf[m] + red[m * 128 + j] + lb);
         }
     }
     tc_fence_before();
@@ -529,7 +552,9 @@ bool plan_tc(const QmmArgs &a, TcPlan &p) {
     p.a_bytes = (int)(((R + 7) / 8) * 1024);
     const size_t ring_b = (size_t)kBStages * kBStage;
     const size_t bars = 512;
-    const size_t fixed = 1024 /*alignment*/ + (size_t)kASlots * p.a_bytes + ring_b + bars;
+    const size_t red = (size_t)16 * 128 * 4;  // epilogue halves' sums (at most 16 rows)
+    const size_t table = (size_t)kMaxGroups * 128;
+    const size_t fixed = 1024 /*alignment*/ + (size_t)kASlots * p.a_bytes + ring_b + red + table + bars;
     if (fixed + 2 * (size_t)p.stage_bytes > kSmemBudget) return false;
     p.S = (int)std::min<size_t>(8, (kSmemBudget - fixed) / p.stage_bytes);
     p.smem = fixed + (size_t)p.S * p.stage_bytes;
@@ -552,8 +577,8 @@ cudaError_t launch_tc(const QmmArgs &a, cudaStream_t s) {
     uint8_t *ws = static_cast<uint8_t *>(a.ws) + kWsFlagBytes;
     const int gs_log = __builtin_ctz((unsigned)a.group_size);
     // Packed codes as [N rows, K*BITS/32 words]: a box is 32 words (128 bytes)
-    // of R rows, 128-byte swizzled; rows past N read as zero.  h/l, [32, K]
-    // bytes, viewed as [K/128 slots][32 rows][128 bytes]: a box is the 32 x 128
+    // of R rows, 128-byte swizzled; rows past N read as zero.  B rows, [48, K]
+    // bytes, viewed as [K/128 slots][48 rows][128 bytes]: a box is the 48 x 128
     // tiles of kSlotsPerB consecutive slots, 128-byte swizzled, tile after tile.
     CUtensorMap tw, tb;
     const uint64_t words = (uint64_t)a.K * BITS / 32;
@@ -561,9 +586,9 @@ cudaError_t launch_tc(const QmmArgs &a, cudaStream_t s) {
                      (uint32_t)p.R, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     {
-        const uint64_t dims[3] = {128, 32, (uint64_t)a.K / 128};
+        const uint64_t dims[3] = {128, (uint64_t)kBRows, (uint64_t)a.K / 128};
         const uint64_t strides[2] = {(uint64_t)a.K, 128};
-        const uint32_t box[3] = {128, 32, (uint32_t)kSlotsPerB};
+        const uint32_t box[3] = {128, (uint32_t)kBRows, (uint32_t)kSlotsPerB};
         if (!make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, ws, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
@@ -599,7 +624,7 @@ cudaError_t launch_tc(const QmmArgs &a, cudaStream_t s) {
     dp.bias = a.bias;
     dp.bias_value = a.bias_value;
     dp.err = device_error_word();
-    const float2 *tab = reinterpret_cast<const float2 *>(ws + (size_t)32 * a.K);
+    const float2 *tab = reinterpret_cast<const float2 *>(ws + (size_t)kBRows * a.K);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -625,14 +650,15 @@ cudaError_t tc_rows(const QmmArgs &a, cudaStream_t s) {
 }  // namespace
 
 // Workspace of the decode tensor-core path: past the leading flag bytes
-// (left untouched), h/l as [32, K] bytes and the (2^-e, X) table,
+// (left untouched), the B rows as [48, K] bytes and the (2^-e, X) table,
 // K / group_size x 16 float2, at most K / 32 groups.
 size_t gemv_tc_workspace_bytes(int64_t K) {
-    return kWsFlagBytes + (size_t)32 * (size_t)K + (size_t)(K / 32) * 16 * sizeof(float2);
+    return kWsFlagBytes + (size_t)kBRows * (size_t)K + (size_t)(K / 32) * 16 * sizeof(float2);
 }
 
 // bf16/f16, transpose, 1..16 rows, 2- or 4-bit codes, K a multiple of 512
-// (whole code chunks), group size 32/64/128, 16-byte aligned operands.  (The
+// (whole code chunks), group size 32/64/128 with groups per row a multiple of
+// 8 (16-byte scale/bias windows), 16-byte aligned operands.  (The
 // call also needs a workspace of gemv_tc_workspace_bytes(K), checked apart.)
 bool gemv_tc_supported(qmm_dtype dt, const QmmArgs &a) {
     if (!a.transpose || a.M < 1 || a.M > 16) return false;
@@ -640,7 +666,7 @@ bool gemv_tc_supported(qmm_dtype dt, const QmmArgs &a) {
     if (a.mode != QMM_MODE_AFFINE) return false;
     if (a.bits != 2 && a.bits != 4) return false;
     if (a.group_size < 32 || a.group_size > 128) return false;
-    if (a.K % 512 != 0) return false;
+    if (a.K % 512 != 0 || (a.K / a.group_size) % 8 != 0 || a.K / a.group_size > kMaxGroups) return false;
     if (a.N < 1 || a.N > (1 << 30) || a.K > (1 << 20)) return false;
     if ((reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.wq) |
          reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases) |

@@ -15,6 +15,7 @@
 // evaluation of the same rule.
 #include <algorithm>
 
+#include "ptx_sm100.cuh"
 #include "qmm_internal.cuh"
 
 namespace qmm {
@@ -55,32 +56,6 @@ __device__ __forceinline__ void store_elems(T *__restrict__ p, const T (&t)[N]) 
     }
 }
 
-// Two fp32 values in one 64-bit register, and the packed two-lane fp32
-// operations of sm_100 (each lane one IEEE operation, round to nearest even).
-__device__ __forceinline__ unsigned long long f2pack(float a, float b) {
-    unsigned long long r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ void f2unpack(unsigned long long v, float &a, float &b) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ unsigned long long f2sub(unsigned long long a, unsigned long long b) {
-    unsigned long long r;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ unsigned long long f2mul(unsigned long long a, unsigned long long b) {
-    unsigned long long r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ unsigned long long f2add(unsigned long long a, unsigned long long b) {
-    unsigned long long r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-
 // The codes of two elements: rint((v - b) / s) clamped to [0, QMAX], with
 // the quotient correctly rounded (IEEE division) as the rule states.  A
 // product with the rounded reciprocal differs from that quotient by at most a
@@ -95,6 +70,7 @@ __device__ __forceinline__ unsigned long long f2add(unsigned long long a, unsign
 __device__ __forceinline__ void code_pair(float v0, float v1, float b, float s, float r, float qmax,
                                           uint32_t &c0, uint32_t &c1) {
     constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    using namespace ptx;
     const unsigned long long mm = f2pack(kMagic, kMagic);
     const unsigned long long t = f2sub(f2pack(v0, v1), f2pack(b, b));
     float y0, y1;
