@@ -523,6 +523,47 @@ def run_reference(args, world, rank):
     return 0
 
 
+PROFILE_CASES = ("decode_m1", "decode_m16", "decode_tc_m16", "prefill", "moe", "quantize", "kn_m256")
+
+
+def profile_case(name, steps, warmup, device):
+    """Run one workload's call `warmup + steps` times and nothing else (for a
+    profiler's launch filter): the decode weight (14336 x 4096 bf16, int4
+    gs64) at M = 1, at M = 16 on the automatic path and on the forced decode
+    tensor-core path; the prefill product (M = 2048); the MoE gather; the
+    quantize of the decode weight; the 4096^2 sweep weight stored [K, N] at
+    M = 256."""
+    from quantized_matmul_03_b200 import binding as qb
+    if name == "moe":
+        c = wl.moe_case()
+        wq, s, b = make_packed(c.w, c.group_size, c.bits, 1, device)[0]
+        x, rhs = c.x.to(device), c.rhs_indices.to(device)
+        fn = lambda: qb.qmm_gather_qmm(x, wq, s, b, None, rhs, True, c.group_size, c.bits)
+    elif name == "kn_m256":
+        w = wl.with_outliers((K_IN, K_IN), seed=3, dtype=torch.bfloat16)
+        wq, s, b = make_packed(w, 64, 4, 1, device)[0]
+        x = wl.normal((256, K_IN), 4, 1.0, torch.bfloat16).to(device)
+        fn = lambda: qb.qmm_quantized_matmul(x, wq, s, b, False, 64, 4)
+    else:
+        c = wl.decode_case(1) if name != "prefill" else wl.prefill_case(4)
+        if name == "quantize":
+            w = c.w.to(device)
+            fn = lambda: qb.qmm_quantize(w, c.group_size, c.bits)
+        else:
+            wq, s, b = make_packed(c.w, c.group_size, c.bits, 1, device)[0]
+            m = {"decode_m1": 1, "decode_m16": 16, "decode_tc_m16": 16}.get(name, 2048)
+            x = (c.x if name == "prefill" else wl.decode_case(m).x).to(device)
+            if name == "decode_tc_m16":
+                qb.qmm_set_path("decode_tc")
+            fn = lambda: qb.qmm_quantized_matmul(x, wq, s, b, True, c.group_size, c.bits)
+    for _ in range(warmup + steps):
+        fn()
+    torch.cuda.synchronize()
+    qb.qmm_device_status()
+    qb.qmm_set_path("auto")
+    print(json.dumps({"case": name, "calls": warmup + steps}), flush=True)
+
+
 METRIC = "int4 qmm weight GB/s at M=1 and TFLOP/s at M=2048, % of roofline"
 
 
@@ -543,6 +584,9 @@ def main():
                     help="time every configuration (decode M 1/4/8/16, prefill int4/int8, "
                          "the 54-point sweep, MoE) and print one JSON line of results")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=PROFILE_CASES,
+                    help="run one workload's call warmup + steps times and print nothing else "
+                         "(for a profiler); no timing")
     ap.add_argument("--cpu-budget-s", type=float, default=10.0)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -559,6 +603,10 @@ def main():
     qb.lib()  # fails loudly if the library was not built
     device = torch.device("cuda", local)
     pk = peaks()
+
+    if args.case:
+        profile_case(args.case, args.steps, args.warmup, device)
+        return 0
 
     if args.suite:
         with ClockSampler(local) as clk:

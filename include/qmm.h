@@ -368,8 +368,10 @@ qmm_status qmm_inject_fault(qmm_fault fault);
  * (16-bit integers split into a signed and an unsigned byte, error below
  * 2^-15 of the group's largest |x|) in the workspace, then an integer MMA
  * product; it needs the workspace that qmm_quantized_matmul_workspace_size
- * reports under this path, else QMM_ERR_WORKSPACE).  A forced path that
- * cannot run a given call returns QMM_ERR_UNSUPPORTED.
+ * reports under this path, else QMM_ERR_WORKSPACE; QMM_PATH_AUTO takes it
+ * for 2-bit codes with 3..8 rows when the workspace is given, where it is
+ * the fastest kernel).  A forced path that cannot run a given call returns
+ * QMM_ERR_UNSUPPORTED.
  */
 typedef enum {
     QMM_PATH_AUTO = 0,

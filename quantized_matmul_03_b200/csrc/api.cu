@@ -339,6 +339,13 @@ qmm_status route_matmul(qmm_dtype dtype, const QmmArgs &a, cudaStream_t s) {
                             "qmm_quantized_matmul_workspace_size bytes");
             return finish_launch(launch_gemv_tc(dtype, a, s), "decode tensor-core launch");
         }
+        // 2-bit codes, 3..8 rows: the decode tensor-core kernel when the
+        // caller gave its workspace (14336 x 4096, 4 rows: 18.0 against
+        // 30.9 us on the SIMT decode kernel; 8 rows: 21.6 against 23.6 us on
+        // the GEMM).  Elsewhere it is not faster.
+        if (g_path == QMM_PATH_AUTO && a.bits == 2 && a.M >= 3 && a.M <= 8 && gemv_tc_supported(dtype, a) &&
+            a.ws != nullptr && a.ws_bytes >= gemv_tc_workspace_bytes(a.K))
+            return finish_launch(launch_gemv_tc(dtype, a, s), "decode tensor-core launch");
         const bool few_rows = a.M <= kGemvMaxRows && a.transpose;
         if (g_path == QMM_PATH_GEMV || few_rows || !tc_ok) {
             if (gemv_fast_supported(dtype, a))
@@ -405,6 +412,9 @@ size_t qmm_quantized_matmul_workspace_size(int64_t M, int64_t K, int64_t N, int 
                 return 0;
             return gemv_tc_workspace_bytes(K);
         }
+        if (g_path == QMM_PATH_AUTO && bits == 2 && M >= 3 && M <= 8 && transpose &&
+            (dtype == QMM_BF16 || dtype == QMM_F16) && K > 0 && K % 512 == 0)
+            return std::max(gemv_tc_workspace_bytes(K), gemm_workspace_size(dtype, M, K, N, true, bits));
         if (g_path != QMM_PATH_GEMM && M <= kGemvMaxRows && transpose) return 0;
         return gemm_workspace_size(dtype, M, K, N, transpose != 0, bits);
     } catch (...) {

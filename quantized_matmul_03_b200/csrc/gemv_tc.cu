@@ -45,7 +45,11 @@
 //                3-D tensor copy of 4 x 48 rows x 128 bytes: a tensor copy
 //                costs its issuing thread several hundred cycles, whatever
 //                its size);
-//   warp 3       tensor-memory owner and MMA issuer (one elected lane);
+//   warps 3, 20  MMA issuers (one elected lane each) for the even and the
+//                odd A slots: a tcgen05 instruction occupies its issuing
+//                thread for ~100+ cycles, so one thread issuing 4 MMAs and
+//                3 commits per slot set the pace; warp 3 also owns tensor
+//                memory;
 //   warps 4-11   code expansion: two groups of four warps take alternate A
 //                slots (128 codes of every row, 128-byte swizzled K-major u8);
 //   warps 12-19  epilogue, two halves of four (one warp per lane quadrant)
@@ -67,9 +71,10 @@
 namespace qmm {
 namespace {
 
-constexpr int kThreads = 640;
+constexpr int kThreads = 672;
 constexpr int kWarpB = 2, kWarpMma = 3, kWarpUnp = 4, kWarpEpi = 12;
 constexpr int kEpiWarps = 8;
+constexpr int kWarpMma2 = kWarpEpi + kEpiWarps;  // 20: the second MMA issuer
 constexpr int kASlots = 6;          // A slots: 128 codes x R rows, u8
 constexpr int kSlotsPerB = 4;       // A slots per activation stage
 constexpr int kBStages = 2;         // activation ring
@@ -79,6 +84,19 @@ constexpr int kBStage = kSlotsPerB * kBTile;
 constexpr int kMaxGroups = 128;     // groups per row whose table fits (16 KB)
 constexpr int kDCols = kBRows;      // accumulator columns per group
 constexpr int kDSlots = 10;         // group accumulators (10 x 48 of 512 columns)
+constexpr int kDPerIssuer = kDSlots / 2;  // each MMA issuer has its own five
+
+// Accumulator slot and use of group g: the issuer of its A slot (128 codes,
+// gpa groups) takes the slots par*5 .. par*5+4 in turn, so each slot's uses
+// come from one thread in order (two issuers sharing slots could get two
+// phases ahead of a slot's barrier, where a parity wait cannot tell them
+// apart).
+__device__ __forceinline__ void group_slot(int g, int gpa, int &d, int &use) {
+    const int a = g / gpa, par = a & 1;
+    const int k = (a >> 1) * gpa + (g - a * gpa);  // ordinal among the issuer's groups
+    d = par * kDPerIssuer + k % kDPerIssuer;
+    use = k / kDPerIssuer;
+}
 constexpr uint32_t kTmemCols = 512;
 constexpr int kTmemThreads = 32 * (kThreads / 32 - kWarpMma);  // warps that use tensor memory
 constexpr int kMaxRows = 128;
@@ -280,6 +298,7 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
     const int NA = p.K >> 7;                       // A slots (128 codes each)
     const int NST = NA / SPC;                      // code stages
     const int G = p.K >> p.gs_log;                 // groups per row
+    const int gpa = 128 >> p.gs_log;               // groups per A slot
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             ptx::mbar_init(fullC + 8 * s, 1);
@@ -291,13 +310,13 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
         }
         for (int b = 0; b < kBStages; ++b) {
             ptx::mbar_init(fullB + 8 * b, 1);
-            ptx::mbar_init(emptyB + 8 * b, 1);     // the MMAs' commit
+            ptx::mbar_init(emptyB + 8 * b, 2);     // one commit from each MMA issuer
         }
         for (int d = 0; d < kDSlots; ++d) {
             ptx::mbar_init(fullD + 8 * d, 1);
             ptx::mbar_init(emptyD + 8 * d, 4);     // the four epilogue warps of the group's half
         }
-        ptx::mbar_init(done, 1);
+        ptx::mbar_init(done, 2);               // both MMA issuers
         ptx::mbar_init(fullT, 1);
         ptx::fence_mbar_init();
     }
@@ -354,15 +373,20 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
                 ptx::mbar_drain(fullB + 8 * (bt % kBStages), (bt / kBStages) & 1, p.err);
             ptx::mbar_drain(fullT, 0, p.err);
         }
-    } else if (warp == kWarpMma) {
-        // ---------------- MMA issuer ----------------
+    } else if (warp == kWarpMma || warp == kWarpMma2) {
+        // ---------------- MMA issuers ----------------
+        // Issuer par takes the A slots a = par mod 2.  A group lies inside one
+        // slot, so each accumulator is written by one issuer per use; an A
+        // slot index recurs kASlots (even) slots later, with the same issuer;
+        // each activation stage is released by one commit from each.
+        const int par = warp == kWarpMma2 ? 1 : 0;
         const bool leader = elect_one();
         const int gs_mask = (1 << p.gs_log) - 1;
-        for (int a = 0; a < NA; ++a) {
+        for (int a = par; a < NA; a += 2) {
             const int as = a % kASlots, bt = a / kSlotsPerB, bs = bt % kBStages, sub = a - bt * kSlotsPerB;
             if (leader) {
                 ptx::mbar_wait<false>(fullA + 8 * as, (a / kASlots) & 1, p.err);
-                if (sub == 0) ptx::mbar_wait<false>(fullB + 8 * bs, (bt / kBStages) & 1, p.err);
+                if (sub == par) ptx::mbar_wait<false>(fullB + 8 * bs, (bt / kBStages) & 1, p.err);
                 tc_fence_after();
                 const uint32_t btile = b0 + (uint32_t)bs * kBStage + (uint32_t)sub * kBTile;
                 const uint64_t da = sw128_desc(a0 + (uint32_t)as * (uint32_t)p.a_bytes);
@@ -370,10 +394,12 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int e0 = a * 128 + 32 * j;
-                    const int g = e0 >> p.gs_log, d = g % kDSlots;
+                    const int g = e0 >> p.gs_log;
+                    int d, use;
+                    group_slot(g, gpa, d, use);
                     const bool first = (e0 & gs_mask) == 0, last = ((e0 + 32) & gs_mask) == 0;
-                    if (first && g >= kDSlots) {
-                        ptx::mbar_wait<false>(emptyD + 8 * d, ((g / kDSlots) - 1) & 1, p.err);
+                    if (first && use > 0) {
+                        ptx::mbar_wait<false>(emptyD + 8 * d, (use - 1) & 1, p.err);
                         tc_fence_after();
                     }
                     // K = 32 bytes per instruction: 2 units of 16 bytes along the rows.
@@ -381,7 +407,7 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
                     if (last) tc_commit(fullD + 8 * d);
                 }
                 tc_commit(emptyA + 8 * as);
-                if (sub == kSlotsPerB - 1) tc_commit(emptyB + 8 * bs);
+                if (sub >= kSlotsPerB - 2) tc_commit(emptyB + 8 * bs);
             }
             __syncwarp();
         }
@@ -465,7 +491,8 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
         int wbase = 0;
         ptx::mbar_wait(fullT, 0, p.err);  // the call's (2^-e, X) table
         for (int g = half; g < G; g += 2) {
-            const int d = g % kDSlots;
+            int d, use;
+            group_slot(g, gpa, d, use);
             if (g >= wbase + 8) {
                 s_cur = s_nxt;
                 b_cur = b_nxt;
@@ -481,7 +508,7 @@ qgemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
             const uint16_t b16 = (uint16_t)((o & 1) ? (bw >> 16) : (bw & 0xffffu));
             const float sv = kF16 ? __half2float(__ushort_as_half(s16)) : __uint_as_float((uint32_t)s16 << 16);
             const float bv = kF16 ? __half2float(__ushort_as_half(b16)) : __uint_as_float((uint32_t)b16 << 16);
-            ptx::mbar_wait<false>(fullD + 8 * d, (g / kDSlots) & 1, p.err);
+            ptx::mbar_wait<false>(fullD + 8 * d, use & 1, p.err);
             tc_fence_after();
             const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kDCols * d);
             uint32_t vh[MR], vl[MR], v1[1];

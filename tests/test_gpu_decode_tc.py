@@ -169,3 +169,20 @@ def test_repeated_calls_agree_bit_for_bit():
     torch.cuda.synchronize()
     for i, y in enumerate(ys):
         assert torch.equal(y, y0[i % 3])
+
+
+@pytest.mark.parametrize("m", [3, 4, 8])
+def test_automatic_path_takes_it_for_two_bit_rows(m):
+    """Under the automatic path, 2-bit codes with 3..8 activation rows and a
+    workspace run on this kernel (two launches), within the tolerance."""
+    w = wl.with_outliers((4096, 4096), seed=80 + m, dtype=torch.bfloat16)
+    x = wl.normal((m, 4096), 81 + m, 1.0, torch.bfloat16)
+    wq, s, b = oracle.quantize(w, 64, 2)
+    ref = oracle.quantized_matmul(x, wq, s, b, True, 64, 2)
+    args = (x.cuda(), wq.cuda(), s.cuda(), b.cuda(), True, 64, 2)
+    qb.qmm_set_path("auto")
+    n0 = qb.qmm_launch_count()
+    y = qb.qmm_quantized_matmul(*args)
+    qb.qmm_device_status()
+    assert qb.qmm_launch_count() - n0 == 2
+    assert row_rel_err(y, ref) <= REL_TOL[torch.bfloat16]
