@@ -14,6 +14,7 @@
 // intrinsic so the result is bit-identical to a sequential IEEE fp32
 // evaluation of the same rule.
 #include <algorithm>
+#include <type_traits>
 
 #include "ptx_sm100.cuh"
 #include "qmm_internal.cuh"
@@ -93,8 +94,9 @@ __device__ __forceinline__ void code_pair(float v0, float v1, float b, float s, 
 // One thread per WPT packed words (16 bytes of codes when a group holds that
 // many); `tpg` = threads per group (a power of two <= 32), so the lanes of one
 // group are contiguous and aligned within the warp.
+// 16-bit elements with 4- or 8-bit codes fit 40 registers: six CTAs per SM.
 template <typename T, int BITS, int WPT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, (sizeof(T) == 2 && BITS >= 4) ? 6 : 1)
 quantize_kernel(const T *__restrict__ w, int64_t n_threads, int tpg,
                 uint32_t *__restrict__ wq, T *__restrict__ scales, T *__restrict__ biases) {
     constexpr int EPW = 32 / BITS;
@@ -103,18 +105,46 @@ quantize_kernel(const T *__restrict__ w, int64_t n_threads, int tpg,
     const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const bool valid = tid < n_threads;
 
-    float v[NE];
-    if (valid) {
-        load_elems<T, NE>(w + tid * NE, v);
+    // 16-bit elements stay packed two per register (half the registers of
+    // fp32 copies: more threads per SM) and the group's min and max are taken
+    // on the pairs with packed 16-bit min/max (exact selections, NaN-ignoring
+    // like fminf/fmaxf); each pair is widened to fp32 only to form its codes.
+    constexpr bool kPacked = sizeof(T) == 2;
+    constexpr int NV = kPacked ? 1 : NE;
+    constexpr int NR = kPacked ? NE / 2 : 1;
+    float v[NV];
+    uint32_t raw[NR];
+    float lo, hi;
+    if constexpr (kPacked) {
+        using V2 = typename std::conditional<std::is_same<T, __half>::value, __half2, __nv_bfloat162>::type;
+#pragma unroll
+        for (int i = 0; i < NR; i += 4) {
+            const uint4 u = valid ? __ldg(reinterpret_cast<const uint4 *>(w + tid * NE) + i / 4) : make_uint4(0, 0, 0, 0);
+            raw[i] = u.x; raw[i + 1] = u.y; raw[i + 2] = u.z; raw[i + 3] = u.w;
+        }
+        V2 mn = *reinterpret_cast<const V2 *>(&raw[0]), mx = mn;
+#pragma unroll
+        for (int i = 1; i < NR; ++i) {
+            const V2 t = *reinterpret_cast<const V2 *>(&raw[i]);
+            mn = __hmin2(mn, t);
+            mx = __hmax2(mx, t);
+        }
+        lo = fminf(Dt<T>::to_f(mn.x), Dt<T>::to_f(mn.y));
+        hi = fmaxf(Dt<T>::to_f(mx.x), Dt<T>::to_f(mx.y));
     } else {
+        if (valid) {
+            load_elems<T, NE>(w + tid * NE, v);
+        } else {
 #pragma unroll
-        for (int j = 0; j < NE; ++j) v[j] = 0.f;
-    }
-    float lo = v[0], hi = v[0];
+            for (int j = 0; j < NV; ++j) v[j] = 0.f;
+        }
+        lo = v[0];
+        hi = v[0];
 #pragma unroll
-    for (int j = 1; j < NE; ++j) {
-        lo = fminf(lo, v[j]);
-        hi = fmaxf(hi, v[j]);
+        for (int j = 1; j < NV; ++j) {
+            lo = fminf(lo, v[j]);
+            hi = fmaxf(hi, v[j]);
+        }
     }
     // Invalid lanes form whole groups (n_threads is a multiple of tpg), and
     // the xor partners of a lane stay inside its own group.
@@ -139,8 +169,17 @@ quantize_kernel(const T *__restrict__ w, int64_t n_threads, int tpg,
         for (int k = 0; k < WPT; ++k) {
 #pragma unroll
             for (int j = 0; j < EPW; j += 2) {
+                float v0, v1;
+                if constexpr (kPacked) {
+                    const uint32_t pr = raw[(k * EPW + j) / 2];
+                    v0 = Dt<T>::to_f(*reinterpret_cast<const T *>(&pr));
+                    v1 = Dt<T>::to_f(*(reinterpret_cast<const T *>(&pr) + 1));
+                } else {
+                    v0 = v[k * EPW + j];
+                    v1 = v[k * EPW + j + 1];
+                }
                 uint32_t c0, c1;
-                code_pair(v[k * EPW + j], v[k * EPW + j + 1], b, s, r, (float)QMAX, c0, c1);
+                code_pair(v0, v1, b, s, r, (float)QMAX, c0, c1);
                 packed[k] |= (c0 << (j * BITS)) | (c1 << ((j + 1) * BITS));
             }
         }
