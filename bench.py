@@ -523,7 +523,8 @@ def run_reference(args, world, rank):
     return 0
 
 
-PROFILE_CASES = ("decode_m1", "decode_m16", "decode_tc_m16", "prefill", "moe", "quantize", "kn_m256")
+PROFILE_CASES = ("decode_m1", "decode_m16", "decode_tc_m16", "prefill", "moe", "quantize", "kn_m256",
+                 "decode_m1_mxfp4", "decode_m1_nvfp4")
 
 
 def profile_case(name, steps, warmup, device):
@@ -532,13 +533,20 @@ def profile_case(name, steps, warmup, device):
     gs64) at M = 1, at M = 16 on the automatic path and on the forced decode
     tensor-core path; the prefill product (M = 2048); the MoE gather; the
     quantize of the decode weight; the 4096^2 sweep weight stored [K, N] at
-    M = 256."""
+    M = 256; the decode weight in mxfp4 / nvfp4 at M = 1."""
     from quantized_matmul_03_b200 import binding as qb
     if name == "moe":
         c = wl.moe_case()
         wq, s, b = make_packed(c.w, c.group_size, c.bits, 1, device)[0]
         x, rhs = c.x.to(device), c.rhs_indices.to(device)
         fn = lambda: qb.qmm_gather_qmm(x, wq, s, b, None, rhs, True, c.group_size, c.bits)
+    elif name in ("decode_m1_mxfp4", "decode_m1_nvfp4"):
+        mode = name.rsplit("_", 1)[1]
+        c = wl.decode_case(1)
+        gs = 32 if mode == "mxfp4" else 16
+        wq, s, _ = qb.qmm_quantize(c.w.to(device), gs, 4, mode)
+        x = c.x.to(device)
+        fn = lambda: qb.qmm_quantized_matmul(x, wq, s, None, True, gs, 4, mode)
     elif name == "kn_m256":
         w = wl.with_outliers((K_IN, K_IN), seed=3, dtype=torch.bfloat16)
         wq, s, b = make_packed(w, 64, 4, 1, device)[0]

@@ -174,7 +174,11 @@ qmm_status qmm_quantized_matmul_ws(const void *x, int64_t M, int64_t K,
  * them); it is the one call a host program makes per product.  On `stream`
  * it enqueues, in order: the copy of M*K elements from x_host into x_dev,
  * the product of x_dev into y_dev (exactly qmm_quantized_matmul_ws), and the
- * copy of M*N elements from y_dev into y_host.
+ * copy of M*N elements from y_dev into y_host.  Page-locked host buffers are
+ * copied by kernels that read or write their device mapping (each waits for
+ * the preceding kernel of the stream, and lets the next one start early), so
+ * consecutive calls overlap like device-only calls; other host memory goes
+ * through the copy engines.
  *   x_host, y_host: host memory; page-locked memory makes both copies
  *     asynchronous (with pageable memory they behave as cudaMemcpyAsync
  *     does).  y_host holds the result once the stream has completed the

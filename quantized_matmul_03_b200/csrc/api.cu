@@ -136,8 +136,10 @@ qmm_status finish_launch(cudaError_t e, const char *what) {
 // activation rows ([N, K] layout), else the SIMT kernels (any shape, either
 // layout; the gather entry takes affine weights only).
 cudaError_t launch_mx_matmul(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
-    // more than a few activation rows: the tensor-core GEMM where it applies
+    // more than a few activation rows: the tensor-core GEMM where it applies;
+    // a few rows of E2M1 codes: the streaming decode kernel
     if (a.M > kGemvMaxRows && gemm_supported(dt, a)) return launch_gemm(dt, a, s);
+    if (gemv_fast_supported(dt, a)) return launch_gemv_fast(dt, a, s);
     return launch_gemv(dt, a, s);
 }
 
@@ -283,14 +285,22 @@ qmm_status matmul_impl(const void *x, int64_t M, int64_t K, const uint32_t *wq, 
         a.ws_bytes = workspace ? workspace_bytes : 0;
         cudaStream_t s = (cudaStream_t)stream;
         const size_t es = dtype == QMM_F32 ? 4 : 2;
+        // Page-locked host buffers are copied by kernels that read or write
+        // their device mapping (chained with the product by programmatic
+        // dependent launch); other host memory by the copy engines.
         if (x_host != nullptr) {
-            cudaError_t e = cudaMemcpyAsync(const_cast<void *>(x), x_host, (size_t)(M * K) * es,
-                                            cudaMemcpyHostToDevice, s);
+            const size_t bytes = (size_t)(M * K) * es;
+            const void *xm = mapped_host_pointer(x_host);
+            cudaError_t e = xm ? launch_mapped_copy(xm, const_cast<void *>(x), bytes, s)
+                               : cudaMemcpyAsync(const_cast<void *>(x), x_host, bytes, cudaMemcpyHostToDevice, s);
             if (e != cudaSuccess) return cuda_fail(e, "copy of x_host");
         }
         const qmm_status launched = route_matmul(dtype, a, s);
         if (launched != QMM_OK || y_host == nullptr) return launched;
-        cudaError_t e = cudaMemcpyAsync(y_host, y, (size_t)(M * N) * es, cudaMemcpyDeviceToHost, s);
+        const size_t bytes = (size_t)(M * N) * es;
+        void *ym = const_cast<void *>(mapped_host_pointer(y_host));
+        cudaError_t e = ym ? launch_mapped_copy(y, ym, bytes, s)
+                           : cudaMemcpyAsync(y_host, y, bytes, cudaMemcpyDeviceToHost, s);
         if (e != cudaSuccess) return cuda_fail(e, "copy into y_host");
         return QMM_OK;
     } catch (...) {
@@ -312,7 +322,10 @@ qmm_status route_matmul(qmm_dtype dtype, const QmmArgs &a, cudaStream_t s) {
                                 "transpose, (K / group_size) %% 16 == 0");
                 return finish_launch(launch_gemm(dtype, a, s), "tensor-core gemm launch");
             }
-            if (g_path == QMM_PATH_GEMV) return finish_launch(launch_gemv(dtype, a, s), "gemv launch");
+            if (g_path == QMM_PATH_GEMV)
+                return finish_launch(gemv_fast_supported(dtype, a) ? launch_gemv_fast(dtype, a, s)
+                                                                    : launch_gemv(dtype, a, s),
+                                     "gemv launch");
             return finish_launch(launch_mx_matmul(dtype, a, s), "microscaled matmul launch");
         }
         const bool tc_ok = gemm_supported(dtype, a);

@@ -25,12 +25,22 @@
 // Per word of 4-bit codes this is 3 ALU + 4 DP2A instructions (8-bit codes:
 // 2 DP2A, no ALU), which keeps the ALU pipe, the limiter of an fp32
 // formulation, below the memory time.  Lane partials for a stage's rows are
-// combined by a butterfly reduce-scatter and shared-memory atomics; results
-// leave as one coalesced store per CTA.
+// combined by a butterfly reduce-scatter into one shared-memory slot per
+// warp, summed in a fixed warp order at the end (results repeat bit for bit);
+// they leave as one coalesced store per CTA.
+//
+// Microscaled E2M1 weights (mxfp4, nvfp4; Emily.QuantizedWeight, Microscaled
+// modes): twice an E2M1 value is an integer in [-12, 12].  Four codes become
+// the bytes 128 + 2e with two PRMT table lookups and one IADD3 (see
+// e2m1_word_to_u8), and DP2A takes them as it takes affine codes; the 128
+// offset is taken out by starting each group's accumulator at -128 sum(x_int).
+// Per group the integer sum is scaled by X/2 (X the group's scale value),
+// with no bias term.  The stages then carry the codes and the scale bytes.
 #include <algorithm>
 #include <cstdlib>
 #include <type_traits>
 
+#include "mx.cuh"
 #include "ptx_sm100.cuh"
 #include "qmm_internal.cuh"
 
@@ -115,7 +125,33 @@ __device__ __forceinline__ float h16_to_f(uint16_t h, bool is_bf16) {
     return is_bf16 ? __uint_as_float((uint32_t)h << 16) : __half2float(__ushort_as_half(h));
 }
 
-template <typename T, int BITS, int MR, int UPL, int RPT>
+// 2 * E2M1 magnitude of codes 0..7, as a PRMT table of 8 bytes.
+constexpr uint32_t kE2m1Lo = 0x03020100u, kE2m1Hi = 0x0C080604u;
+
+// PRMT in its generic form: byte n of the result is byte (c >> 4n) & 7 of
+// {b:a}, or, when bit 3 of that nibble is set, that byte's sign replicated.
+// (__byte_perm is defined on the three low selector bits only, so the sign
+// form is written out.)
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// The eight E2M1 codes of w (code j at bits 4j..4j+3, its sign in bit 3 of
+// the nibble) as unsigned bytes 128 + 2 e_j: v[0] holds codes 0..3, v[1]
+// codes 4..7.  A PRMT on the raw nibbles gives the table magnitude of every
+// non-negative code and 0 for a negative one (the code's sign bit asks for
+// the sign of a table byte, and every table byte is positive); on the
+// nibbles with their sign bits flipped it gives the converse.  Per byte the
+// sum 128 + pos - neg lies in [116, 140], so no byte borrows from another.
+__device__ __forceinline__ void e2m1_word_to_u8(uint32_t w, uint32_t *v) {
+    const uint32_t wn = w ^ 0x88888888u;
+    v[0] = prmt(kE2m1Lo, kE2m1Hi, w) + 0x80808080u - prmt(kE2m1Lo, kE2m1Hi, wn);
+    v[1] = prmt(kE2m1Lo, kE2m1Hi, w >> 16) + 0x80808080u - prmt(kE2m1Lo, kE2m1Hi, wn >> 16);
+}
+
+template <typename T, int BITS, int MR, int UPL, int RPT, int MODE = QMM_MODE_AFFINE>
 __global__ void __launch_bounds__(kThreads, 1)
 qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     const T *__restrict__ scales, const T *__restrict__ biases,
@@ -126,6 +162,9 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     constexpr int STEPS = EPW / 2;       // code pairs per word
     constexpr int V = MR * RPT;          // partials per lane per stage
     constexpr bool kBF16 = std::is_same<T, __nv_bfloat16>::value;
+    constexpr bool MX = MODE != QMM_MODE_AFFINE;   // E2M1 elements, scale bytes, no biases
+    constexpr bool NV = MODE == QMM_MODE_NVFP4;    // two groups of 16 per 32-code slice
+    static_assert(!MX || BITS == 4, "microscaled codes here are E2M1");
     static_assert((V & (V - 1)) == 0 && V <= 32, "V must be a power of two <= 32");
 
     extern __shared__ __align__(128) uint8_t smem[];
@@ -133,8 +172,9 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     const int SR = NT * RPT;                 // rows per stage
     const int row_bytes = K / 8 * BITS;
     const int gpr = K / group_size;
-    const int sb_bytes = gpr * 2;
-    const int stage_bytes = SR * (row_bytes + 2 * sb_bytes);
+    constexpr int NSB = MX ? 1 : 2;          // per-group arrays per row: scales (+ biases)
+    const int sb_bytes = MX ? gpr : gpr * 2;  // bytes of one array per row
+    const int stage_bytes = SR * (row_bytes + NSB * sb_bytes);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)S * stage_bytes);
     float *ysm = reinterpret_cast<float *>(bars + 2 * S);
     const int r0 = blockIdx.x * rpc;
@@ -143,7 +183,7 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t full0 = ptx::smem_addr(bars), empty0 = ptx::smem_addr(bars + S);
 
-    for (int i = threadIdx.x; i < MR * rpc; i += kThreads) ysm[i] = 0.f;
+    for (int i = threadIdx.x; i < TW * MR * rpc; i += kThreads) ysm[i] = 0.f;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             ptx::mbar_init(full0 + 8 * s, 1);
@@ -189,11 +229,12 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                 const uint32_t wb = (uint32_t)(nr * row_bytes), sb = (uint32_t)(nr * sb_bytes);
                 const uint32_t st = ptx::smem_addr(smem + (size_t)s * stage_bytes);
                 const uint32_t bar = full0 + 8 * s;
-                ptx::mbar_arrive_expect_tx(bar, wb + 2 * sb);
+                ptx::mbar_arrive_expect_tx(bar, wb + NSB * sb);
                 const int64_t roff = (int64_t)i * SR;
                 ptx::bulk_g2s(st, wsrc + roff * row_bytes, wb, bar);
                 ptx::bulk_g2s(st + SR * row_bytes, ssrc + roff * sb_bytes, sb, bar);
-                ptx::bulk_g2s(st + SR * row_bytes + SR * sb_bytes, bsrc + roff * sb_bytes, sb, bar);
+                if constexpr (!MX)
+                    ptx::bulk_g2s(st + SR * row_bytes + SR * sb_bytes, bsrc + roff * sb_bytes, sb, bar);
                 if (handoff && i == max(0, nst - 2)) atomicMax(&g_sm_issued[smid], ticket + 1);
                 if (++s == S) {
                     s = 0;
@@ -225,7 +266,8 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
         }
 
         // The activations may be the output of the preceding kernel in the
-        // stream: wait for it (and for every earlier grid) to complete.
+        // stream: wait for it (and for every earlier grid) to complete and
+        // its writes to become visible to this grid.
         ptx::grid_dependency_wait();
         // Activations in 16-bit block fixed point per slice (see the header):
         // packed (lo, hi) int16 pairs in DP2A order, the slice's scale-back
@@ -233,6 +275,9 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
         int xp[MR][UPL][4 * STEPS];
         float fsc[MR][UPL];
         float xsum[MR][UPL];
+        // E2M1: -128 times the sum of x_int over each group of the slice (the
+        // codes enter DP2A as 128 + 2e); nvfp4 has two groups per slice
+        int xoff[MR][UPL][2];
 #pragma unroll
         for (int m = 0; m < MR; ++m) {
 #pragma unroll
@@ -262,13 +307,18 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                 const float up = __uint_as_float((uint32_t)(127 + sh) << 23);
                 fsc[m][u] = __uint_as_float((uint32_t)(127 - sh) << 23);
                 xsum[m][u] = sum;
+                xoff[m][u][0] = xoff[m][u][1] = 0;
 #pragma unroll
                 for (int wd = 0; wd < 4; ++wd) {
 #pragma unroll
                     for (int k = 0; k < STEPS; ++k) {
-                        const int lo = __float2int_rn(xv[wd * EPW + Planes<BITS>::elem(k, 0)] * up);
-                        const int hi = __float2int_rn(xv[wd * EPW + Planes<BITS>::elem(k, 1)] * up);
+                        // affine: plane order; E2M1: consecutive pairs
+                        const int e0 = MX ? 2 * k : Planes<BITS>::elem(k, 0);
+                        const int e1 = MX ? 2 * k + 1 : Planes<BITS>::elem(k, 1);
+                        const int lo = __float2int_rn(xv[wd * EPW + e0] * up);
+                        const int hi = __float2int_rn(xv[wd * EPW + e1] * up);
                         xp[m][u][wd * STEPS + k] = (lo & 0xffff) | (hi << 16);
+                        if constexpr (MX) xoff[m][u][NV && wd >= 2] -= 128 * (lo + hi);
                     }
                 }
             }
@@ -301,10 +351,39 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
 #pragma unroll
                     for (int u = 0; u < UPL; ++u) {
                         const uint4 wv = *reinterpret_cast<const uint4 *>(wrow + soff[u]);
+                        const bool use = rv && sv[u];
+                        if constexpr (MX) {
+                            // X/2 of the slice's group (groups 2 slice and 2 slice + 1
+                            // for nvfp4), exact in fp32
+                            const float x0 = 0.5f * mxf::scale_value<MODE>(srow[gi[u]]);
+                            const float x1 = NV ? 0.5f * mxf::scale_value<MODE>(srow[gi[u] + 1]) : 0.f;
+                            uint32_t v[8];
+                            e2m1_word_to_u8(wv.x, v + 0);
+                            e2m1_word_to_u8(wv.y, v + 2);
+                            e2m1_word_to_u8(wv.z, v + 4);
+                            e2m1_word_to_u8(wv.w, v + 6);
+#pragma unroll
+                            for (int m = 0; m < MR; ++m) {
+                                // a: codes 0..15 (nvfp4: the first group), b: codes 16..31
+                                int a0 = xoff[m][u][0], a1 = 0, b0 = xoff[m][u][1], b1 = 0;
+#pragma unroll
+                                for (int q = 0; q < 8; ++q) {
+                                    int &c0 = (NV && q >= 4) ? b0 : a0;
+                                    int &c1 = (NV && q >= 4) ? b1 : a1;
+                                    // word q / 2, codes 4 (q % 2) .. +3: pairs (0,1) and (2,3)
+                                    c0 = dp2a_lo(xp[m][u][(q >> 1) * STEPS + 2 * (q & 1)], v[q], c0);
+                                    c1 = dp2a_hi(xp[m][u][(q >> 1) * STEPS + 2 * (q & 1) + 1], v[q], c1);
+                                }
+                                // (X/2 * 2^-sh) first, as for the affine scale below
+                                float c = (x0 * fsc[m][u]) * (float)(a0 + a1);
+                                if constexpr (NV) c = __fmaf_rn(x1 * fsc[m][u], (float)(b0 + b1), c);
+                                part[m * RPT + j] += use ? c : 0.f;
+                            }
+                            continue;
+                        }
                         const float sc = h16_to_f(*reinterpret_cast<const uint16_t *>(srow + gi[u] * 2), kBF16);
                         const float bi = h16_to_f(
                             *reinterpret_cast<const uint16_t *>(srow + SR * sb_bytes + gi[u] * 2), kBF16);
-                        const bool use = rv && sv[u];
 #pragma unroll
                         for (int m = 0; m < MR; ++m) {
                             int a0 = 0, a1 = 0;
@@ -332,7 +411,7 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
             if (active && lane < V) {
                 const int m = lane / RPT, j = lane - m * RPT;
                 const int r = i * SR + team + j * NT;
-                if (m < M && r < nrows) atomicAdd(&ysm[m * rpc + r], v);
+                if (m < M && r < nrows) ysm[(wt * MR + m) * rpc + r] = v;
             }
             if (++s == S) {
                 s = 0;
@@ -341,9 +420,12 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
         }
     }
     __syncthreads();
+    // A row's team warps in a fixed order, so that results repeat bit for bit.
     for (int idx = threadIdx.x; idx < M * nrows; idx += kThreads) {
         const int m = idx / nrows, r = idx - m * nrows;
-        y[(int64_t)m * N + r0 + r] = Dt<T>::from_f(ysm[m * rpc + r] + layer_bias<T>(bias, bias_value, r0 + r));
+        float acc = 0.f;
+        for (int t = 0; t < TW; ++t) acc += ysm[(t * MR + m) * rpc + r];
+        y[(int64_t)m * N + r0 + r] = Dt<T>::from_f(acc + layer_bias<T>(bias, bias_value, r0 + r));
     }
 }
 
@@ -370,19 +452,24 @@ bool plan_stream(const QmmArgs &a, int mr, int ctas_per_sm, StreamPlan &p) {
     p.rpt = rows_per_team_stage(mr);
     p.sr = nt * p.rpt;
     const int64_t row_bytes = a.K / 8 * bits;
-    const int64_t sb_bytes = a.K / a.group_size * 2;
-    const int64_t stage = (int64_t)p.sr * (row_bytes + 2 * sb_bytes);
+    // per row: scales and biases (affine, 16-bit) or scale bytes (E2M1)
+    const bool mx = a.mode != QMM_MODE_AFFINE;
+    const int64_t sb_bytes = a.K / a.group_size * (mx ? 1 : 2);
+    const int64_t stage = (int64_t)p.sr * (row_bytes + (mx ? 1 : 2) * sb_bytes);
     const int64_t ctas = (int64_t)num_sms() * ctas_per_sm;
     int64_t rpc = (a.N + ctas - 1) / ctas;
-    rpc = std::min<int64_t>(rpc, 2048 / mr);
+    // rows per CTA: at most 2048 / mr, and partial slots (one per team warp,
+    // activation row and row) of at most 24 KB
+    rpc = std::min<int64_t>(rpc, std::min<int64_t>(2048 / mr, 6144 / (p.tw * mr)));
     rpc = std::max<int64_t>(rpc, 1);
     p.rpc = (int)rpc;
     p.grid = (int)((a.N + rpc - 1) / rpc);
     const size_t budget = kSmemPerSm / ctas_per_sm;
-    const size_t fixed = 16 * 8 + (size_t)mr * p.rpc * 4 + 128;
+    const size_t slots = (size_t)p.tw * mr * p.rpc * 4;
+    const size_t fixed = 16 * 8 + slots + 128;
     if ((size_t)stage * 2 + fixed > budget) return false;
     p.stages = (int)std::min<int64_t>(8, (int64_t)((budget - fixed) / stage));
-    p.smem = (size_t)p.stages * stage + (size_t)2 * p.stages * 8 + (size_t)mr * p.rpc * 4;
+    p.smem = (size_t)p.stages * stage + (size_t)2 * p.stages * 8 + slots;
     return p.stages >= 2;
 }
 
@@ -399,10 +486,10 @@ bool stream_variant_fits(int bits, int mr, int upl) {
     return false;
 }
 
-template <typename T, int BITS, int MR, int UPL>
+template <typename T, int BITS, int MR, int UPL, int MODE>
 cudaError_t launch_stream(const QmmArgs &a, cudaStream_t s) {
     constexpr int RPT = MR == 4 ? 2 : 4;
-    auto kern = qgemv_stream_kernel<T, BITS, MR, UPL, RPT>;
+    auto kern = qgemv_stream_kernel<T, BITS, MR, UPL, RPT, MODE>;
     // One CTA per SM (the next call's CTAs take the other half of the SM).
     StreamPlan p{};
     if (!plan_stream(a, MR, 1, p)) return cudaErrorInvalidValue;
@@ -444,22 +531,22 @@ cudaError_t launch_stream(const QmmArgs &a, cudaStream_t s) {
 }
 
 // One launch for rows [0, mr) of a (mr in {1, 2, 4}, a variant that fits).
-template <typename T, int BITS>
+template <typename T, int BITS, int MODE>
 cudaError_t stream_rows(const QmmArgs &a, int mr, cudaStream_t s) {
     StreamPlan p{};
     if (!plan_stream(a, mr, 1, p)) return cudaErrorInvalidValue;
     if (mr == 1) {
-        if (p.upl == 1) return launch_stream<T, BITS, 1, 1>(a, s);
-        if constexpr (BITS != 2) return launch_stream<T, BITS, 1, 2>(a, s);
+        if (p.upl == 1) return launch_stream<T, BITS, 1, 1, MODE>(a, s);
+        if constexpr (BITS != 2) return launch_stream<T, BITS, 1, 2, MODE>(a, s);
     }
     if constexpr (BITS != 2) {
-        if (mr == 2 && p.upl == 1) return launch_stream<T, BITS, 2, 1>(a, s);
+        if (mr == 2 && p.upl == 1) return launch_stream<T, BITS, 2, 1, MODE>(a, s);
     }
     if constexpr (BITS == 8) {
-        if (mr == 2) return launch_stream<T, BITS, 2, 2>(a, s);
+        if (mr == 2) return launch_stream<T, BITS, 2, 2, MODE>(a, s);
     }
     if constexpr (BITS != 2) {
-        if (mr == 4 && p.upl == 1) return launch_stream<T, BITS, 4, 1>(a, s);
+        if (mr == 4 && p.upl == 1) return launch_stream<T, BITS, 4, 1, MODE>(a, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -481,7 +568,7 @@ int pick_rows(const QmmArgs &a, int64_t rows) {
 // Rows go through the widest variant that fits, a launch per row block (for
 // example 4-bit codes: 3 or 4 rows in one 4-row launch; 2-bit codes: 3 rows =
 // 2 + 1).
-template <typename T, int BITS>
+template <typename T, int BITS, int MODE = QMM_MODE_AFFINE>
 cudaError_t stream_bits(const QmmArgs &a, cudaStream_t s) {
     for (int64_t m0 = 0; m0 < a.M;) {
         const int mr = pick_rows(a, a.M - m0);
@@ -490,7 +577,7 @@ cudaError_t stream_bits(const QmmArgs &a, cudaStream_t s) {
         t.M = std::min<int64_t>(mr, a.M - m0);
         t.x = static_cast<const T *>(a.x) + m0 * a.K;
         t.y = static_cast<T *>(a.y) + m0 * a.N;
-        const cudaError_t e = stream_rows<T, BITS>(t, mr, s);
+        const cudaError_t e = stream_rows<T, BITS, MODE>(t, mr, s);
         if (e != cudaSuccess) return e;
         m0 += t.M;
     }
@@ -501,14 +588,21 @@ cudaError_t stream_bits(const QmmArgs &a, cudaStream_t s) {
 
 // Fast path: bf16/f16, transpose layout, 1..4 rows, whole 16-byte slices per
 // row, scales/biases rows of whole 16-byte units, no group boundary inside a
-// slice (group_size >= codes per slice), rows at most 8 warps wide.
+// slice (group_size >= codes per slice; nvfp4: exactly two groups per slice),
+// rows at most 12 warps wide.  Affine 2-, 4- and 8-bit codes, mxfp4, nvfp4.
 bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a) {
     if (!a.transpose || a.M < 1 || a.M > 4) return false;
-    if (a.mode != QMM_MODE_AFFINE || (a.bits != 2 && a.bits != 4 && a.bits != 8)) return false;
     if (dt != QMM_BF16 && dt != QMM_F16) return false;
     const int epu = 128 / a.bits;
-    if (a.K % epu != 0 || a.group_size < epu) return false;
-    if ((a.K / a.group_size) % 8 != 0) return false;
+    if (a.mode == QMM_MODE_AFFINE) {
+        if (a.bits != 2 && a.bits != 4 && a.bits != 8) return false;
+        if (a.K % epu != 0 || a.group_size < epu) return false;
+        if ((a.K / a.group_size) % 8 != 0) return false;
+    } else {
+        if (a.mode != QMM_MODE_MXFP4 && a.mode != QMM_MODE_NVFP4) return false;
+        if (a.bits != 4 || a.K % epu != 0) return false;
+        if ((a.K / a.group_size) % 16 != 0) return false;  // scale rows of whole 16-byte units
+    }
     if (a.N > (1 << 30) || a.K > (1 << 24)) return false;
     if ((reinterpret_cast<uintptr_t>(a.scales) | reinterpret_cast<uintptr_t>(a.biases) |
          reinterpret_cast<uintptr_t>(a.wq)) & 15)
@@ -519,6 +613,12 @@ bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a) {
 }
 
 cudaError_t launch_gemv_fast(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
+    if (a.mode == QMM_MODE_MXFP4)
+        return dt == QMM_BF16 ? stream_bits<__nv_bfloat16, 4, QMM_MODE_MXFP4>(a, s)
+                              : stream_bits<__half, 4, QMM_MODE_MXFP4>(a, s);
+    if (a.mode == QMM_MODE_NVFP4)
+        return dt == QMM_BF16 ? stream_bits<__nv_bfloat16, 4, QMM_MODE_NVFP4>(a, s)
+                              : stream_bits<__half, 4, QMM_MODE_NVFP4>(a, s);
     if (dt == QMM_BF16) {
         switch (a.bits) {
         case 2: return stream_bits<__nv_bfloat16, 2>(a, s);

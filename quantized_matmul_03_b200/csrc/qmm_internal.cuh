@@ -138,6 +138,11 @@ bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a);
 cudaError_t launch_gemv_tc(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 bool gemv_tc_supported(qmm_dtype dt, const QmmArgs &a);
 size_t gemv_tc_workspace_bytes(int64_t K);
+// Copies for qmm_quantized_matmul_host (copy.cu): the device address of a
+// page-locked host pointer (nullptr if it is not page-locked), and a copy
+// kernel chained by programmatic dependent launch.
+const void *mapped_host_pointer(const void *p);
+cudaError_t launch_mapped_copy(const void *src, void *dst, size_t bytes, cudaStream_t s);
 cudaError_t launch_gemm(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);
 cudaError_t launch_mx_matmul(qmm_dtype dt, const QmmArgs &a, cudaStream_t s);  // microscaled weights
 // Bytes of stream-K workspace the tensor-core path can use for these sizes
