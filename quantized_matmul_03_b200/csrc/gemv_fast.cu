@@ -21,7 +21,9 @@
 // fixed point, x_int = rint(x * 2^sh) with sh chosen from the slice's largest
 // |x| so that |x_int| < 2^14: the representation error is at most 2^-15 of
 // the slice maximum, and every product and sum after it is exact.  A slice's
-// integer sum is multiplied by s * 2^-sh in fp32; sum(x) uses the exact x.
+// integer sum is multiplied by s * 2^-sh in fp32, and sum(x) is the sum of the
+// same fixed-point values, so the result is the exact product of the
+// dequantized weight with the rounded activations, rounded once per slice.
 // Per word of 4-bit codes this is 3 ALU + 4 DP2A instructions (8-bit codes:
 // 2 DP2A, no ALU), which keeps the ALU pipe, the limiter of an fp32
 // formulation, below the memory time.  Lane partials for a stage's rows are
@@ -125,6 +127,14 @@ __device__ __forceinline__ float h16_to_f(uint16_t h, bool is_bf16) {
     return is_bf16 ? __uint_as_float((uint32_t)h << 16) : __half2float(__ushort_as_half(h));
 }
 
+// Element e of 16-bit elements packed two per word (element 2k in the low half).
+template <bool BF16, int N>
+__device__ __forceinline__ float elem_to_f(const uint32_t (&w)[N], int e) {
+    const uint32_t v = w[e >> 1];
+    if constexpr (BF16) return __uint_as_float((e & 1) ? (v & 0xFFFF0000u) : (v << 16));
+    return __half2float(__ushort_as_half((unsigned short)((e & 1) ? (v >> 16) : (v & 0xFFFFu))));
+}
+
 // 2 * E2M1 magnitude of codes 0..7, as a PRMT table of 8 bytes.
 constexpr uint32_t kE2m1Lo = 0x03020100u, kE2m1Hi = 0x0C080604u;
 
@@ -151,12 +161,19 @@ __device__ __forceinline__ void e2m1_word_to_u8(uint32_t w, uint32_t *v) {
     v[1] = prmt(kE2m1Lo, kE2m1Hi, w >> 16) + 0x80808080u - prmt(kE2m1Lo, kE2m1Hi, wn >> 16);
 }
 
+// One-row variants with one slice per lane are held to 72 registers, so that
+// two CTAs (this call's and the next one's) fit the SM's register file (416
+// threads x 72 x 2 <= 65536).  A minimum-blocks launch bound gave 64 registers
+// and a slower loop.
+template <int BITS, int MR, int UPL>
+constexpr int stream_max_regs() { return (MR == 1 && UPL == 1 && BITS != 2) ? 72 : 168; }
+
 template <typename T, int BITS, int MR, int UPL, int RPT, int MODE = QMM_MODE_AFFINE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1) __maxnreg__((stream_max_regs<BITS, MR, UPL>()))
 qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     const T *__restrict__ scales, const T *__restrict__ biases,
-                    T *__restrict__ y, int M, int N, int K, int group_size, int rpc, int S,
-                    int TW, const T *__restrict__ bias, float bias_value, int *err) {
+                    T *__restrict__ y, int M, int N, int K, int group_size, int rpc, int R,
+                    int q, int S, int TW, const T *__restrict__ bias, float bias_value, int *err) {
     constexpr int EPW = 32 / BITS;       // codes per word
     constexpr int EPU = 4 * EPW;         // codes per 16-byte slice
     constexpr int STEPS = EPW / 2;       // code pairs per word
@@ -177,9 +194,16 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     const int stage_bytes = SR * (row_bytes + NSB * sb_bytes);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (size_t)S * stage_bytes);
     float *ysm = reinterpret_cast<float *>(bars + 2 * S);
-    const int r0 = blockIdx.x * rpc;
-    const int nrows = max(0, min(rpc, N - r0));
-    const int nst = (nrows + SR - 1) / SR;
+    // Rows: R rounds of SR-row stages dealt across the grid (stage i of CTA b
+    // holds rows (i * grid + b) * SR ...), so that the copies in flight at
+    // any moment cover one contiguous stretch of the weight; then one final
+    // stage of at most q rows per CTA.  Local row r of stage i = r / SR.
+    const int grid = (int)gridDim.x, b = (int)blockIdx.x;
+    const int tr0 = R * grid * SR + b * q;           // first row of the final stage
+    const int nq = max(0, min(q, N - tr0));
+    const int nrows = R * SR + nq;                   // rows of this CTA (<= rpc)
+    const int nst = R + (nq > 0 ? 1 : 0);
+    auto stage_row0 = [&](int i) { return i < R ? (i * grid + b) * SR : tr0; };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t full0 = ptx::smem_addr(bars), empty0 = ptx::smem_addr(bars + S);
 
@@ -205,9 +229,9 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     if (warp == 0) {
         // ---------------- producer ----------------
         if (lane == 0) {
-            const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(wq) + (int64_t)r0 * row_bytes;
-            const uint8_t *ssrc = reinterpret_cast<const uint8_t *>(scales) + (int64_t)r0 * sb_bytes;
-            const uint8_t *bsrc = reinterpret_cast<const uint8_t *>(biases) + (int64_t)r0 * sb_bytes;
+            const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(wq);
+            const uint8_t *ssrc = reinterpret_cast<const uint8_t *>(scales);
+            const uint8_t *bsrc = reinterpret_cast<const uint8_t *>(biases);
             uint32_t smid;
             asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
             const bool handoff = smid < (uint32_t)kMaxSm;
@@ -230,7 +254,7 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                 const uint32_t st = ptx::smem_addr(smem + (size_t)s * stage_bytes);
                 const uint32_t bar = full0 + 8 * s;
                 ptx::mbar_arrive_expect_tx(bar, wb + NSB * sb);
-                const int64_t roff = (int64_t)i * SR;
+                const int64_t roff = stage_row0(i);
                 ptx::bulk_g2s(st, wsrc + roff * row_bytes, wb, bar);
                 ptx::bulk_g2s(st + SR * row_bytes, ssrc + roff * sb_bytes, sb, bar);
                 if constexpr (!MX)
@@ -271,7 +295,7 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
         ptx::grid_dependency_wait();
         // Activations in 16-bit block fixed point per slice (see the header):
         // packed (lo, hi) int16 pairs in DP2A order, the slice's scale-back
-        // 2^-sh, and the exact slice sum of x for the bias term.
+        // 2^-sh, and the slice sum of the fixed-point values for the bias term.
         int xp[MR][UPL][4 * STEPS];
         float fsc[MR][UPL];
         float xsum[MR][UPL];
@@ -283,21 +307,26 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
 #pragma unroll
             for (int u = 0; u < UPL; ++u) {
                 const bool ok = sv[u] && m < M;
-                float xv[EPU];
-                float amax = 0.f, sum = 0.f;
+                uint32_t raw[EPU / 2];  // the slice's 16-bit elements, two per word
 #pragma unroll
                 for (int c = 0; c < EPU / 8; ++c) {
-                    uint4 raw = ok ? *reinterpret_cast<const uint4 *>(
-                                         x + (int64_t)m * K + (int64_t)sl[u] * EPU + 8 * c)
-                                   : make_uint4(0, 0, 0, 0);
-                    const uint16_t *h = reinterpret_cast<const uint16_t *>(&raw);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        xv[8 * c + q] = h16_to_f(h[q], kBF16);
-                        amax = fmaxf(amax, fabsf(xv[8 * c + q]));
-                        sum += xv[8 * c + q];
-                    }
+                    const uint4 r = ok ? *reinterpret_cast<const uint4 *>(
+                                             x + (int64_t)m * K + (int64_t)sl[u] * EPU + 8 * c)
+                                       : make_uint4(0, 0, 0, 0);
+                    raw[4 * c] = r.x;
+                    raw[4 * c + 1] = r.y;
+                    raw[4 * c + 2] = r.z;
+                    raw[4 * c + 3] = r.w;
                 }
+                // Largest |x|: the bit patterns of non-negative IEEE values
+                // order as the values, so a packed unsigned 16-bit max of the
+                // words with their sign bits cleared finds it.
+                uint32_t mx2 = 0;
+#pragma unroll
+                for (int q = 0; q < EPU / 2; ++q) mx2 = ptx::max_u16x2(mx2, raw[q] & 0x7FFF7FFFu);
+                const uint32_t mbits = max(mx2 & 0xFFFFu, mx2 >> 16);
+                const float amax = kBF16 ? __uint_as_float(mbits << 16)
+                                         : __half2float(__ushort_as_half((unsigned short)mbits));
                 // amax < 2^ex (ex = biased exponent - 126); x * 2^sh < 2^14 with
                 // sh = 14 - ex, clamped so that 2^sh and 2^-sh are normal floats
                 // (the lower clamp is reached by no finite 16-bit value: bf16
@@ -306,8 +335,12 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                 const int sh = min(126, max(-126, 14 - ex));
                 const float up = __uint_as_float((uint32_t)(127 + sh) << 23);
                 fsc[m][u] = __uint_as_float((uint32_t)(127 - sh) << 23);
-                xsum[m][u] = sum;
-                xoff[m][u][0] = xoff[m][u][1] = 0;
+                // x_int = rint(x 2^sh) by adding 1.5 * 2^23: x 2^sh is exact and
+                // |x 2^sh| < 2^14, so the sum rounds (to nearest, ties to even)
+                // at the units place and its low 16 bits are x_int's two's
+                // complement; the sum of the words, less the offsets, is the
+                // exact sum of the x_int.
+                uint32_t isum[2] = {0u, 0u};
 #pragma unroll
                 for (int wd = 0; wd < 4; ++wd) {
 #pragma unroll
@@ -315,11 +348,24 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                         // affine: plane order; E2M1: consecutive pairs
                         const int e0 = MX ? 2 * k : Planes<BITS>::elem(k, 0);
                         const int e1 = MX ? 2 * k + 1 : Planes<BITS>::elem(k, 1);
-                        const int lo = __float2int_rn(xv[wd * EPW + e0] * up);
-                        const int hi = __float2int_rn(xv[wd * EPW + e1] * up);
-                        xp[m][u][wd * STEPS + k] = (lo & 0xffff) | (hi << 16);
-                        if constexpr (MX) xoff[m][u][NV && wd >= 2] -= 128 * (lo + hi);
+                        const uint32_t lo = __float_as_uint(
+                            __fmaf_rn(elem_to_f<kBF16>(raw, wd * EPW + e0), up, 12582912.0f));
+                        const uint32_t hi = __float_as_uint(
+                            __fmaf_rn(elem_to_f<kBF16>(raw, wd * EPW + e1), up, 12582912.0f));
+                        xp[m][u][wd * STEPS + k] = (int)__byte_perm(lo, hi, 0x5410);
+                        isum[NV && wd >= 2] += lo + hi;
                     }
+                }
+                constexpr uint32_t kOff = 0x4B400000u;  // the bits of 1.5 * 2^23
+                if constexpr (MX) {
+                    const int g0 = (int)(isum[0] - (NV ? EPU / 2 : EPU) * kOff);
+                    const int g1 = NV ? (int)(isum[1] - (EPU / 2) * kOff) : 0;
+                    xoff[m][u][0] = -128 * g0;
+                    xoff[m][u][1] = -128 * g1;
+                    xsum[m][u] = 0.f;
+                } else {
+                    xsum[m][u] = fsc[m][u] * (float)(int)(isum[0] - EPU * kOff);
+                    xoff[m][u][0] = xoff[m][u][1] = 0;
                 }
             }
         }
@@ -356,7 +402,8 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                             // X/2 of the slice's group (groups 2 slice and 2 slice + 1
                             // for nvfp4), exact in fp32
                             const float x0 = 0.5f * mxf::scale_value<MODE>(srow[gi[u]]);
-                            const float x1 = NV ? 0.5f * mxf::scale_value<MODE>(srow[gi[u] + 1]) : 0.f;
+                            [[maybe_unused]] const float x1 =
+                                NV ? 0.5f * mxf::scale_value<MODE>(srow[gi[u] + 1]) : 0.f;
                             uint32_t v[8];
                             e2m1_word_to_u8(wv.x, v + 0);
                             e2m1_word_to_u8(wv.y, v + 2);
@@ -425,12 +472,14 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
         const int m = idx / nrows, r = idx - m * nrows;
         float acc = 0.f;
         for (int t = 0; t < TW; ++t) acc += ysm[(t * MR + m) * rpc + r];
-        y[(int64_t)m * N + r0 + r] = Dt<T>::from_f(acc + layer_bias<T>(bias, bias_value, r0 + r));
+        const int i = min(r / SR, R);
+        const int gr = stage_row0(i) + (r - i * SR);
+        y[(int64_t)m * N + gr] = Dt<T>::from_f(acc + layer_bias<T>(bias, bias_value, gr));
     }
 }
 
 struct StreamPlan {
-    int upl, tw, rpt, sr, stages, rpc, grid;
+    int upl, tw, rpt, sr, stages, rpc, rounds, q, grid;
     size_t smem;
 };
 
@@ -456,14 +505,20 @@ bool plan_stream(const QmmArgs &a, int mr, int ctas_per_sm, StreamPlan &p) {
     const bool mx = a.mode != QMM_MODE_AFFINE;
     const int64_t sb_bytes = a.K / a.group_size * (mx ? 1 : 2);
     const int64_t stage = (int64_t)p.sr * (row_bytes + (mx ? 1 : 2) * sb_bytes);
+    // One CTA per SM (more, in waves, when a CTA's rows would pass 2048 / mr
+    // or its partial slots -- one per team warp, activation row and row --
+    // 24 KB); fewer for small N.
     const int64_t ctas = (int64_t)num_sms() * ctas_per_sm;
-    int64_t rpc = (a.N + ctas - 1) / ctas;
-    // rows per CTA: at most 2048 / mr, and partial slots (one per team warp,
-    // activation row and row) of at most 24 KB
-    rpc = std::min<int64_t>(rpc, std::min<int64_t>(2048 / mr, 6144 / (p.tw * mr)));
-    rpc = std::max<int64_t>(rpc, 1);
-    p.rpc = (int)rpc;
-    p.grid = (int)((a.N + rpc - 1) / rpc);
+    const int64_t cap = std::max<int64_t>(1, std::min<int64_t>(2048 / mr, 6144 / (p.tw * mr)));
+    int64_t grid = std::min<int64_t>(ctas, a.N);
+    if ((a.N + grid - 1) / grid > cap) grid = (a.N + cap - 1) / cap;
+    if (grid > (1 << 30) / p.sr) return false;
+    // R full rounds of sr-row stages over the grid, then q rows per CTA
+    p.rounds = (int)(a.N / (grid * p.sr));
+    const int64_t rem = a.N - (int64_t)p.rounds * grid * p.sr;
+    p.q = (int)((rem + grid - 1) / grid);
+    p.rpc = p.rounds * p.sr + p.q;
+    p.grid = (int)grid;
     const size_t budget = kSmemPerSm / ctas_per_sm;
     const size_t slots = (size_t)p.tw * mr * p.rpc * 4;
     const size_t fixed = 16 * 8 + slots + 128;
@@ -523,7 +578,7 @@ cudaError_t launch_stream(const QmmArgs &a, cudaStream_t s) {
     e = cudaLaunchKernelEx(&cfg, kern, static_cast<const T *>(a.x), a.wq,
                            static_cast<const T *>(a.scales), static_cast<const T *>(a.biases),
                            static_cast<T *>(a.y), (int)a.M, (int)a.N, (int)a.K, a.group_size,
-                           p.rpc, p.stages, p.tw, static_cast<const T *>(a.bias), a.bias_value,
+                           p.rpc, p.rounds, p.q, p.stages, p.tw, static_cast<const T *>(a.bias), a.bias_value,
                            device_error_word());
     if (e != cudaSuccess) return e;
     count_launches(1);

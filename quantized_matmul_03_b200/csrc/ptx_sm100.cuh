@@ -129,6 +129,13 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         : "memory");
 }
 
+// Per 16-bit half, the unsigned maximum of a and b (sm_90 and later).
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 // Two fp32 values in one 64-bit register (x in the low half), and the packed
 // two-lane fp32 operations of sm_100 (each lane one IEEE operation, round to
 // nearest even).
