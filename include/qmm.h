@@ -177,8 +177,10 @@ qmm_status qmm_quantized_matmul_ws(const void *x, int64_t M, int64_t K,
  * copy of M*N elements from y_dev into y_host.  Page-locked host buffers are
  * copied by kernels that read or write their device mapping (each waits for
  * the preceding kernel of the stream, and lets the next one start early), so
- * consecutive calls overlap like device-only calls; other host memory goes
- * through the copy engines.
+ * consecutive calls overlap like device-only calls; when the product runs on
+ * the streaming decode kernel (W [N, K], 1..4 rows), that kernel also writes
+ * the result into a page-locked y_host itself and no copy follows.  Other
+ * host memory goes through the copy engines.
  *   x_host, y_host: host memory; page-locked memory makes both copies
  *     asynchronous (with pageable memory they behave as cudaMemcpyAsync
  *     does).  y_host holds the result once the stream has completed the
@@ -198,6 +200,31 @@ qmm_status qmm_quantized_matmul_host(const void *x_host, void *x_dev, int64_t M,
                                      int group_size, int bits, const char *mode,
                                      void *y_dev, void *y_host, void *workspace,
                                      size_t workspace_bytes, void *stream);
+
+/*
+ * qmm_mapped_pointer -- the address through which kernels on the current
+ * device reach the page-locked host memory at `host` (cudaHostAlloc, or
+ * cudaHostRegister'ed with mapping), or NULL when `host` is NULL, not
+ * page-locked or not mapped.  One runtime query per call.
+ *
+ * qmm_quantized_matmul_mapped -- qmm_quantized_matmul_host for page-locked
+ * buffers whose mappings the caller looked up once with qmm_mapped_pointer,
+ * for the repeated per-step call of a serving loop: nothing is queried per
+ * call, x is copied in by a kernel and the result reaches y_map as in
+ * qmm_quantized_matmul_host.
+ *   x_map, y_map: mappings returned by qmm_mapped_pointer for host buffers of
+ *     M*K and M*N elements; the memory must stay page-locked (and mapped)
+ *     while calls that use it are in flight.  NULL with a nonzero size:
+ *     QMM_ERR_INVALID_ARG.
+ *   Every other argument, the results and the errors: as
+ *     qmm_quantized_matmul_host.
+ */
+void *qmm_mapped_pointer(const void *host);
+qmm_status qmm_quantized_matmul_mapped(const void *x_map, void *x_dev, int64_t M, int64_t K,
+                                       const uint32_t *wq, const void *scales, const void *biases,
+                                       qmm_dtype dtype, int64_t N, int transpose, int group_size,
+                                       int bits, const char *mode, void *y_dev, void *y_map,
+                                       void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * qmm_quantized_dense -- Emily.Quantization.Layers, quantized_dense: the

@@ -52,6 +52,8 @@ def lib() -> ctypes.CDLL:
                                         vp, vp, sz, vp],
             "qmm_quantized_matmul_host": [vp, vp, i64, i64, vp, vp, vp, i32, i64, i32, i32, i32,
                                           cp, vp, vp, vp, sz, vp],
+            "qmm_quantized_matmul_mapped": [vp, vp, i64, i64, vp, vp, vp, i32, i64, i32, i32,
+                                            i32, cp, vp, vp, vp, sz, vp],
             "qmm_quantized_dense": [vp, i64, i64, vp, vp, vp, i32, i64, i32, i32, i32, cp,
                                     vp, ctypes.c_double, vp, vp, sz, vp],
             "qmm_qqmm": [vp, i64, i64, i32, vp, vp, i64, i32, i32, cp, vp, vp, sz, vp],
@@ -82,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.qmm_launch_count.restype = ctypes.c_uint64
         L.qmm_version.argtypes = []
         L.qmm_version.restype = i32
+        L.qmm_mapped_pointer.argtypes = [vp]
+        L.qmm_mapped_pointer.restype = vp
         _lib = L
     return _lib
 
@@ -235,8 +239,10 @@ class HostMatmul:
     x_host / y_host: CPU tensors (pin_memory() for asynchronous copies) of the
     shapes of x_dev / y_dev; x_dev / y_dev: CUDA tensors.  The pointers,
     sizes, workspace and stream are fixed when the object is made, so a call
-    costs one foreign-function call; y_host holds the result once the stream
-    has run it (torch.cuda.synchronize() or an event)."""
+    costs one foreign-function call; when both host tensors are page-locked,
+    their device mappings are looked up here once and each call goes through
+    qmm_quantized_matmul_mapped.  y_host holds the result once the stream has
+    run it (torch.cuda.synchronize() or an event)."""
 
     def __init__(self, x_host, x_dev, wq, scales, biases, y_dev, y_host, transpose: bool = True,
                  group_size: int = 64, bits: int = 4, mode: str = "affine", workspace="auto"):
@@ -262,10 +268,17 @@ class HostMatmul:
             ws = workspace
         # keep the tensors alive as long as the call may run
         self._keep = (x_host, x_dev, wq, scales, biases, y_dev, y_host, ws)
+        xh, yh = _p(x_host), _p(y_host)
         self._fn = lib().qmm_quantized_matmul_host
-        self._args = (_p(x_host), _p(x_dev), M, K, _p(wq), _p(scales), _p(biases),
+        if x_host.is_pinned() and y_host.is_pinned():
+            with torch.cuda.device(x_dev.device):
+                xm, ym = lib().qmm_mapped_pointer(xh), lib().qmm_mapped_pointer(yh)
+            if xm and ym:
+                xh, yh = xm, ym
+                self._fn = lib().qmm_quantized_matmul_mapped
+        self._args = (xh, _p(x_dev), M, K, _p(wq), _p(scales), _p(biases),
                       _dtype(y_dev), N, int(bool(transpose)), group_size, bits, _mode(mode),
-                      _p(y_dev), _p(y_host), _p(ws),
+                      _p(y_dev), yh, _p(ws),
                       ws.numel() * ws.element_size() if ws is not None else 0,
                       _stream(x_dev.device))
 

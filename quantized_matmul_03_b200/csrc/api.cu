@@ -258,12 +258,14 @@ qmm_status route_matmul(qmm_dtype dtype, const QmmArgs &a, cudaStream_t s);
 
 // x_host / y_host (qmm_quantized_matmul_host): when given, the copy of x_host
 // into x is enqueued once every argument has been checked, and the copy of y
-// into y_host once the product has been launched.
+// into y_host once the product has been launched (unless the product kernel
+// wrote y_host itself).  mapped: x_host / y_host are already the device
+// mappings of page-locked host memory (qmm_quantized_matmul_mapped).
 qmm_status matmul_impl(const void *x, int64_t M, int64_t K, const uint32_t *wq, const void *scales,
                        const void *biases, qmm_dtype dtype, int64_t N, int transpose, int group_size,
                        int bits, const char *mode, const void *bias, double bias_value, void *y,
                        void *workspace, size_t workspace_bytes, void *stream,
-                       const void *x_host = nullptr, void *y_host = nullptr) {
+                       const void *x_host = nullptr, void *y_host = nullptr, bool mapped = false) {
     try {
         int md = QMM_MODE_AFFINE;
         qmm_status st = check_common(dtype, group_size, bits, mode, &md);
@@ -287,18 +289,21 @@ qmm_status matmul_impl(const void *x, int64_t M, int64_t K, const uint32_t *wq, 
         const size_t es = dtype == QMM_F32 ? 4 : 2;
         // Page-locked host buffers are copied by kernels that read or write
         // their device mapping (chained with the product by programmatic
-        // dependent launch); other host memory by the copy engines.
+        // dependent launch), or written by the product kernel itself; other
+        // host memory goes through the copy engines.
         if (x_host != nullptr) {
             const size_t bytes = (size_t)(M * K) * es;
-            const void *xm = mapped_host_pointer(x_host);
+            const void *xm = mapped ? x_host : mapped_host_pointer(x_host);
             cudaError_t e = xm ? launch_mapped_copy(xm, const_cast<void *>(x), bytes, s)
                                : cudaMemcpyAsync(const_cast<void *>(x), x_host, bytes, cudaMemcpyHostToDevice, s);
             if (e != cudaSuccess) return cuda_fail(e, "copy of x_host");
         }
+        void *ym = nullptr;
+        if (y_host != nullptr) ym = mapped ? y_host : const_cast<void *>(mapped_host_pointer(y_host));
+        a.y2 = ym;
         const qmm_status launched = route_matmul(dtype, a, s);
-        if (launched != QMM_OK || y_host == nullptr) return launched;
+        if (launched != QMM_OK || y_host == nullptr || a.y2_written) return launched;
         const size_t bytes = (size_t)(M * N) * es;
-        void *ym = const_cast<void *>(mapped_host_pointer(y_host));
         cudaError_t e = ym ? launch_mapped_copy(y, ym, bytes, s)
                            : cudaMemcpyAsync(y_host, y, bytes, cudaMemcpyDeviceToHost, s);
         if (e != cudaSuccess) return cuda_fail(e, "copy into y_host");
@@ -394,6 +399,27 @@ qmm_status qmm_quantized_matmul_host(const void *x_host, void *x_dev, int64_t M,
     return matmul_impl(x_dev, M, K, wq, scales, biases, dtype, N, transpose, group_size, bits, mode,
                        nullptr, 0.0, y_dev, workspace, workspace_bytes, stream,
                        M > 0 && K > 0 ? x_host : nullptr, M > 0 && N > 0 ? y_host : nullptr);
+}
+
+qmm_status qmm_quantized_matmul_mapped(const void *x_map, void *x_dev, int64_t M, int64_t K,
+                                       const uint32_t *wq, const void *scales, const void *biases,
+                                       qmm_dtype dtype, int64_t N, int transpose, int group_size,
+                                       int bits, const char *mode, void *y_dev, void *y_map,
+                                       void *workspace, size_t workspace_bytes, void *stream) {
+    if ((x_map == nullptr && M > 0 && K > 0) || (y_map == nullptr && M > 0 && N > 0))
+        return fail(QMM_ERR_INVALID_ARG, "x_map and y_map must not be NULL");
+    return matmul_impl(x_dev, M, K, wq, scales, biases, dtype, N, transpose, group_size, bits, mode,
+                       nullptr, 0.0, y_dev, workspace, workspace_bytes, stream,
+                       M > 0 && K > 0 ? x_map : nullptr, M > 0 && N > 0 ? y_map : nullptr, true);
+}
+
+void *qmm_mapped_pointer(const void *host) {
+    if (host == nullptr) return nullptr;
+    try {
+        return const_cast<void *>(mapped_host_pointer(host));
+    } catch (...) {
+        return nullptr;
+    }
 }
 
 qmm_status qmm_quantized_dense(const void *x, int64_t M, int64_t K, const uint32_t *wq,

@@ -15,7 +15,14 @@
 namespace qmm {
 namespace {
 
-__global__ void __launch_bounds__(256)
+// Small CTAs: a copy kernel launched early sits in griddepcontrol.wait beside
+// the two decode-kernel CTAs of an SM (this call's and the next one's), which
+// leave it only ~5,600 registers; a larger CTA there would keep the next
+// call's CTA from starting early on that SM.
+constexpr int kCopyThreads = 64;
+constexpr int kCopyUnroll = 8;  // 16-byte loads in flight per thread
+
+__global__ void __launch_bounds__(kCopyThreads)
 mapped_copy_kernel(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst, int64_t bytes, int vec16) {
     // Let the next kernel of the stream (the product, or the next step's
     // copy) launch now; it waits for this grid where it depends on it.
@@ -24,9 +31,24 @@ mapped_copy_kernel(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst, i
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (vec16) {
+        // all of a thread's loads first (one round trip over the bus), then
+        // the stores
         const uint4 *s = reinterpret_cast<const uint4 *>(src);
         uint4 *d = reinterpret_cast<uint4 *>(dst);
-        for (int64_t i = t0; i < bytes / 16; i += stride) d[i] = __ldcg(s + i);
+        const int64_t n = bytes / 16;
+        for (int64_t i0 = t0; i0 < n; i0 += stride * kCopyUnroll) {
+            uint4 v[kCopyUnroll];
+#pragma unroll
+            for (int u = 0; u < kCopyUnroll; ++u) {
+                const int64_t i = i0 + u * stride;
+                if (i < n) v[u] = __ldcg(s + i);
+            }
+#pragma unroll
+            for (int u = 0; u < kCopyUnroll; ++u) {
+                const int64_t i = i0 + u * stride;
+                if (i < n) d[i] = v[u];
+            }
+        }
     } else {
         for (int64_t i = t0; i < bytes; i += stride) dst[i] = __ldcg(src + i);
     }
@@ -52,10 +74,11 @@ cudaError_t launch_mapped_copy(const void *src, void *dst, size_t bytes, cudaStr
     const bool vec16 = bytes % 16 == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0 &&
                        (reinterpret_cast<uintptr_t>(dst) & 15) == 0;
     const int64_t units = vec16 ? (int64_t)(bytes / 16) : (int64_t)bytes;
-    const unsigned grid = (unsigned)std::min<int64_t>((units + 255) / 256, 4 * (int64_t)num_sms());
+    const int64_t per_cta = (int64_t)kCopyThreads * (vec16 ? kCopyUnroll : 1);
+    const unsigned grid = (unsigned)std::min<int64_t>((units + per_cta - 1) / per_cta, 4 * (int64_t)num_sms());
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
-    cfg.blockDim = dim3(256, 1, 1);
+    cfg.blockDim = dim3(kCopyThreads, 1, 1);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -62,9 +62,10 @@ constexpr int kThreads = 32 * (kCW + 1);  // plus one producer warp
 // for two or three stages left, was measured slower).  This orders memory
 // traffic only: results do not depend on it.
 constexpr int kMaxSm = 1024;
-constexpr uint64_t kHandoffWaitNs = 20000;
+constexpr uint64_t kHandoffWaitNs = 8000;
 __device__ unsigned long long g_sm_ticket[kMaxSm];  // CTAs that entered, per SM
 __device__ unsigned long long g_sm_issued[kMaxSm];  // highest ticket + 1 with <= 1 stage to issue
+__device__ unsigned long long g_sm_grid[kMaxSm];    // %gridid of the latest ticket's CTA
 
 // Code planes of a packed word: plane p = (w >> p*BITS) & byte-mask, whose
 // byte j is code j*NP + p (NP = 8/BITS planes).  DP2A.lo takes bytes 0,1 and
@@ -173,7 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1) __maxnreg__((stream_max_regs<BITS
 qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
                     const T *__restrict__ scales, const T *__restrict__ biases,
                     T *__restrict__ y, int M, int N, int K, int group_size, int rpc, int R,
-                    int q, int S, int TW, const T *__restrict__ bias, float bias_value, int *err) {
+                    int q, int S, int TW, const T *__restrict__ bias, float bias_value, int *err,
+                    T *__restrict__ y2) {
     constexpr int EPW = 32 / BITS;       // codes per word
     constexpr int EPU = 4 * EPW;         // codes per 16-byte slice
     constexpr int STEPS = EPW / 2;       // code pairs per word
@@ -208,12 +210,29 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     const uint32_t full0 = ptx::smem_addr(bars), empty0 = ptx::smem_addr(bars + S);
 
     for (int i = threadIdx.x; i < TW * MR * rpc; i += kThreads) ysm[i] = 0.f;
+    // Thread 0 is the producer (warp 0, lane 0); it takes the SM's hand-off
+    // ticket before this grid lets the next one launch, so that on every SM
+    // the tickets follow the order of the calls (a CTA of a later call that
+    // took an earlier ticket would hold this one back until the hand-off's
+    // time bound).
+    // A CTA that finds a CTA of its own grid ahead of it on the SM (the grid
+    // did not fit one CTA per SM beside the previous call) does not wait.
+    uint32_t smid = 0;
+    unsigned long long ticket = 0;
+    bool same_grid = false;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             ptx::mbar_init(full0 + 8 * s, 1);
             ptx::mbar_init(empty0 + 8 * s, kCW);
         }
         ptx::fence_mbar_init();
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        if (smid < (uint32_t)kMaxSm) {
+            unsigned long long gid;
+            asm volatile("mov.u64 %0, %%gridid;" : "=l"(gid));
+            ticket = atomicAdd(&g_sm_ticket[smid], 1ull);
+            same_grid = atomicExch(&g_sm_grid[smid], gid) == gid;
+        }
     }
     __syncthreads();
     // Let the next launch in the stream begin its own prologue (barrier set-up
@@ -221,7 +240,8 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
     // reads before grid_dependency_wait() is the packed weight, its scales and
     // biases.  Only a preceding kernel that itself allows an early start
     // (griddepcontrol.launch_dependents) can still be running then: in this
-    // library that is this kernel, which writes none of them; qmm_quantize,
+    // library that is this kernel or a copy kernel of the host-buffer calls,
+    // which write none of them; qmm_quantize,
     // which does write them, never allows it, so a call after it starts only
     // once it has completed.  The header states the rule for other writers.
     ptx::grid_launch_dependents();
@@ -232,12 +252,8 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
             const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(wq);
             const uint8_t *ssrc = reinterpret_cast<const uint8_t *>(scales);
             const uint8_t *bsrc = reinterpret_cast<const uint8_t *>(biases);
-            uint32_t smid;
-            asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
             const bool handoff = smid < (uint32_t)kMaxSm;
-            unsigned long long ticket = 0;
-            if (handoff) {
-                ticket = atomicAdd(&g_sm_ticket[smid], 1ull);
+            if (handoff && !same_grid) {
                 const uint64_t t0 = ptx::globaltimer_ns();
                 for (;;) {
                     unsigned long long done;
@@ -474,7 +490,9 @@ qgemv_stream_kernel(const T *__restrict__ x, const uint32_t *__restrict__ wq,
         for (int t = 0; t < TW; ++t) acc += ysm[(t * MR + m) * rpc + r];
         const int i = min(r / SR, R);
         const int gr = stage_row0(i) + (r - i * SR);
-        y[(int64_t)m * N + gr] = Dt<T>::from_f(acc + layer_bias<T>(bias, bias_value, gr));
+        const T v = Dt<T>::from_f(acc + layer_bias<T>(bias, bias_value, gr));
+        y[(int64_t)m * N + gr] = v;
+        if (y2) y2[(int64_t)m * N + gr] = v;  // (host memory through its mapping)
     }
 }
 
@@ -579,7 +597,7 @@ cudaError_t launch_stream(const QmmArgs &a, cudaStream_t s) {
                            static_cast<const T *>(a.scales), static_cast<const T *>(a.biases),
                            static_cast<T *>(a.y), (int)a.M, (int)a.N, (int)a.K, a.group_size,
                            p.rpc, p.rounds, p.q, p.stages, p.tw, static_cast<const T *>(a.bias), a.bias_value,
-                           device_error_word());
+                           device_error_word(), static_cast<T *>(a.y2));
     if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();
@@ -632,6 +650,7 @@ cudaError_t stream_bits(const QmmArgs &a, cudaStream_t s) {
         t.M = std::min<int64_t>(mr, a.M - m0);
         t.x = static_cast<const T *>(a.x) + m0 * a.K;
         t.y = static_cast<T *>(a.y) + m0 * a.N;
+        if (a.y2) t.y2 = static_cast<T *>(a.y2) + m0 * a.N;
         const cudaError_t e = stream_rows<T, BITS, MODE>(t, mr, s);
         if (e != cudaSuccess) return e;
         m0 += t.M;
@@ -668,6 +687,7 @@ bool gemv_fast_supported(qmm_dtype dt, const QmmArgs &a) {
 }
 
 cudaError_t launch_gemv_fast(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
+    a.y2_written = a.y2 != nullptr;
     if (a.mode == QMM_MODE_MXFP4)
         return dt == QMM_BF16 ? stream_bits<__nv_bfloat16, 4, QMM_MODE_MXFP4>(a, s)
                               : stream_bits<__half, 4, QMM_MODE_MXFP4>(a, s);

@@ -124,6 +124,11 @@ struct QmmArgs {
     const void *bias = nullptr;
     float bias_value = 0.f;
     int mode = QMM_MODE_AFFINE;  // microscaled: scales are bytes, biases null
+    // A second destination for the result (the device mapping of page-locked
+    // host memory, [*, N]), or null.  Kernels that can write it in their
+    // epilogue set y2_written; otherwise the caller copies y there.
+    void *y2 = nullptr;
+    mutable bool y2_written = false;
 };
 
 // Bias term of output feature n: bias[n] (if any) plus the scalar.

@@ -166,3 +166,33 @@ def test_matmul_host_rejects_before_any_copy(L, kw, status):
 
 def test_matmul_host_empty_is_a_noop(L):
     assert mmhost(L, M=0, x=NULL, y=NULL, xh=NULL, yh=NULL) == 0
+
+
+def mmmapped(L, xm=FAKE, ym=FAKE, **kw):
+    a = dict(x=FAKE, M=2, K=128, wq=FAKE, s=FAKE, b=FAKE, dtype=1, N=64, tr=1, gs=64,
+             bits=4, mode=None, y=FAKE)
+    a.update(kw)
+    return L.qmm_quantized_matmul_mapped(xm, a["x"], a["M"], a["K"], a["wq"], a["s"], a["b"],
+                                         a["dtype"], a["N"], a["tr"], a["gs"], a["bits"],
+                                         a["mode"], a["y"], ym, NULL, 0, NULL)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(xm=NULL), 1), (dict(ym=NULL), 1), (dict(K=96), 1), (dict(b=NULL), 1),
+    (dict(x=MISALIGNED), 1), (dict(bits=7), 1),
+])
+def test_matmul_mapped_rejects_before_any_copy(L, kw, status):
+    """The mapped entry checks its mappings and every argument before it
+    enqueues anything."""
+    assert mmmapped(L, **kw) == status
+
+
+def test_matmul_mapped_empty_is_a_noop(L):
+    assert mmmapped(L, M=0, x=NULL, y=NULL, xm=NULL, ym=NULL) == 0
+
+
+def test_mapped_pointer_of_ordinary_memory_is_null(L):
+    """Pageable host memory (and NULL) has no device mapping."""
+    buf = ctypes.create_string_buffer(256)
+    assert L.qmm_mapped_pointer(ctypes.addressof(buf)) is None
+    assert L.qmm_mapped_pointer(None) is None

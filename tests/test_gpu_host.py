@@ -67,3 +67,50 @@ def test_f32_and_odd_sizes():
     torch.cuda.synchronize()
     ref = oracle.quantized_matmul(x, wq.cpu(), s.cpu(), b.cpu(), True, 64, 4)
     assert row_rel_err(y_host, ref) <= REL_TOL[torch.float32]
+
+
+@pytest.mark.parametrize("m,launches", [(1, 2), (4, 2), (40, 3)])
+def test_prepared_mapped_call(m, launches):
+    """Page-locked buffers: the prepared call looks their mappings up once and
+    goes through qmm_quantized_matmul_mapped.  With 1..4 rows the decode
+    kernel writes y_host itself (copy in + product: two launches); with 40
+    rows the GEMM result is copied out by a kernel (three launches).  y_dev
+    holds the result too."""
+    w = wl.with_outliers((2000, 4096), seed=96 + m, dtype=torch.bfloat16)
+    wq, s, b = (t.cuda() for t in oracle.quantize(w, 64, 4))
+    x = wl.normal((m, 4096), 97 + m, 1.0, torch.bfloat16)
+    x_host, y_host = x.pin_memory(), torch.zeros((m, 2000), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x, device="cuda")
+    y_dev = torch.zeros((m, 2000), dtype=torch.bfloat16, device="cuda")
+    call = qb.HostMatmul(x_host, x_dev, wq, s, b, y_dev, y_host, True, 64, 4)
+    assert call._fn is qb.lib().qmm_quantized_matmul_mapped
+    n0 = qb.qmm_launch_count()
+    call()
+    torch.cuda.synchronize()
+    qb.qmm_device_status()
+    assert qb.qmm_launch_count() - n0 == launches
+    y_ref = qb.qmm_quantized_matmul(x.cuda(), wq, s, b, True, 64, 4)
+    torch.cuda.synchronize()
+    assert torch.equal(y_host, y_ref.cpu()) and torch.equal(y_dev, y_ref)
+
+
+def test_prepared_calls_back_to_back():
+    """Three prepared calls (three weights, shared x_dev / y_dev, own host
+    outputs) enqueued twice over without synchronization."""
+    ws = [wl.with_outliers((3000, 2048), seed=98 + i, dtype=torch.bfloat16) for i in range(3)]
+    packs = [tuple(t.cuda() for t in oracle.quantize(w, 64, 4)) for w in ws]
+    xs = [wl.normal((1, 2048), 99 + i, 1.0, torch.bfloat16).pin_memory() for i in range(3)]
+    ys = [torch.empty((1, 3000), dtype=torch.bfloat16).pin_memory() for _ in range(6)]
+    x_dev = torch.empty((1, 2048), dtype=torch.bfloat16, device="cuda")
+    y_dev = torch.empty((1, 3000), dtype=torch.bfloat16, device="cuda")
+    calls = [qb.HostMatmul(xs[i % 3], x_dev, *packs[i % 3], y_dev, ys[i], True, 64, 4)
+             for i in range(6)]
+    torch.cuda.synchronize()
+    for c in calls:
+        c()
+    torch.cuda.synchronize()
+    qb.qmm_device_status()
+    for i in range(6):
+        ref = qb.qmm_quantized_matmul(xs[i % 3].cuda(), *packs[i % 3], True, 64, 4)
+        torch.cuda.synchronize()
+        assert torch.equal(ys[i], ref.cpu()), f"step {i}"
