@@ -390,7 +390,10 @@ qmm_status qmm_inject_fault(qmm_fault fault);
 
 /*
  * Kernel-path selection for qmm_quantized_matmul (process-wide; the default
- * is QMM_PATH_AUTO).  QMM_PATH_GEMV forces the SIMT decode kernels (M <= 16
+ * is QMM_PATH_AUTO: 1..4 rows of a W [N, K] product run on the streaming
+ * decode kernel when it takes the codes -- affine 2/4/8 bits, mxfp4, nvfp4 --
+ * and on the tensor-core GEMM otherwise (bf16/f16); more rows, and W [K, N],
+ * on the GEMM).  QMM_PATH_GEMV forces the SIMT decode kernels (M <= 16
  * rows at a time), QMM_PATH_GEMM the tensor-core (tcgen05) GEMM, and
  * QMM_PATH_DECODE_TC the decode tensor-core kernel (bf16/f16, transpose,
  * 1..16 rows, 2- or 4-bit codes, group size 32..128, K % 512 == 0,

@@ -137,9 +137,11 @@ qmm_status finish_launch(cudaError_t e, const char *what) {
 // layout; the gather entry takes affine weights only).
 cudaError_t launch_mx_matmul(qmm_dtype dt, const QmmArgs &a, cudaStream_t s) {
     // more than a few activation rows: the tensor-core GEMM where it applies;
-    // a few rows of E2M1 codes: the streaming decode kernel
+    // a few rows of E2M1 codes: the streaming decode kernel; a few rows of
+    // E4M3 codes: the GEMM too (the SIMT kernel is ~3x slower there)
     if (a.M > kGemvMaxRows && gemm_supported(dt, a)) return launch_gemm(dt, a, s);
     if (gemv_fast_supported(dt, a)) return launch_gemv_fast(dt, a, s);
+    if (gemm_supported(dt, a)) return launch_gemm(dt, a, s);
     return launch_gemv(dt, a, s);
 }
 
@@ -342,9 +344,11 @@ qmm_status route_matmul(qmm_dtype dtype, const QmmArgs &a, cudaStream_t s) {
             return finish_launch(launch_gemm(dtype, a, s), "tensor-core gemm launch");
         }
         // Decode shapes of the [N, K] layout (1..4 rows) stream the weight
-        // through the SIMT decode kernel; larger activation counts, and the
-        // [K, N] layout at any count, use the tensor-core GEMM.  The decode
-        // tensor-core kernel runs only when forced.
+        // through the SIMT decode kernel where it takes the codes (2/4/8
+        // bits), else through the tensor-core GEMM (3/6 bits: ~3x faster than
+        // the general SIMT kernel); larger activation counts, and the [K, N]
+        // layout at any count, use the GEMM.  The decode tensor-core kernel
+        // runs when forced, and for the 2-bit case below.
         if (g_path == QMM_PATH_DECODE_TC) {
             if (!gemv_tc_supported(dtype, a))
                 return fail(QMM_ERR_UNSUPPORTED,
@@ -368,7 +372,8 @@ qmm_status route_matmul(qmm_dtype dtype, const QmmArgs &a, cudaStream_t s) {
         if (g_path == QMM_PATH_GEMV || few_rows || !tc_ok) {
             if (gemv_fast_supported(dtype, a))
                 return finish_launch(launch_gemv_fast(dtype, a, s), "gemv launch");
-            return finish_launch(launch_gemv(dtype, a, s), "gemv launch");
+            if (g_path == QMM_PATH_GEMV || !tc_ok)
+                return finish_launch(launch_gemv(dtype, a, s), "gemv launch");
         }
         return finish_launch(launch_gemm(dtype, a, s), "tensor-core gemm launch");
     } catch (...) {
@@ -454,7 +459,10 @@ size_t qmm_quantized_matmul_workspace_size(int64_t M, int64_t K, int64_t N, int 
         if (g_path == QMM_PATH_AUTO && bits == 2 && M >= 3 && M <= 8 && transpose &&
             (dtype == QMM_BF16 || dtype == QMM_F16) && K > 0 && K % 512 == 0)
             return std::max(gemv_tc_workspace_bytes(K), gemm_workspace_size(dtype, M, K, N, true, bits));
-        if (g_path != QMM_PATH_GEMM && M <= kGemvMaxRows && transpose) return 0;
+        // 1..4 rows of [N, K]: the streaming decode kernel (no workspace)
+        // takes 2-, 4- and 8-bit codes; 3- and 6-bit codes go to the GEMM.
+        if (g_path != QMM_PATH_GEMM && M <= kGemvMaxRows && transpose && bits != 3 && bits != 6)
+            return 0;
         return gemm_workspace_size(dtype, M, K, N, transpose != 0, bits);
     } catch (...) {
         return 0;
