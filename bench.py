@@ -22,6 +22,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -229,12 +230,21 @@ def peaks():
             "src": "fallback"}
 
 
+def strip_comments(text: str) -> str:
+    """C/C++ source without its comments and blank lines (the kernel sources
+    hold no string literal with comment markers)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash(files) -> str:
     """Hash of the CUDA sources a kernel is built from (its .cu and the
-    device headers it includes)."""
+    device headers it includes), comments removed: an edit to a comment does
+    not change the kernel, an edit to the code does."""
     h = hashlib.sha256()
     for name in sorted(files):
-        h.update((ROOT / "quantized_matmul_03_b200" / "csrc" / name).read_bytes())
+        h.update(strip_comments((ROOT / "quantized_matmul_03_b200" / "csrc" / name).read_text()).encode())
     return h.hexdigest()[:16]
 
 

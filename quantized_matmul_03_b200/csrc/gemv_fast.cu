@@ -3,11 +3,13 @@
 // with W stored [N, K] (mlx-rs ops/quantization.rs, quantized_matmul;
 // Emily.Quantization.Layers, quantized_dense with transpose: true).
 //
-// Memory side.  Each CTA owns a contiguous block of weight rows, which is one
-// contiguous byte range of the packed weight (and of the scales and biases).
-// A producer warp streams it through a ring of shared-memory stages with 1-D
-// bulk copies (cp.async.bulk) completing on mbarriers, so ~100 KB per SM are in
-// flight regardless of register pressure.  The weight is read exactly once.
+// Memory side.  The weight's rows are cut into stages of SR rows, each one
+// contiguous byte range of the packed weight (and of the scales and biases),
+// dealt round-robin over the CTAs so that the copies in flight at any moment
+// cover one contiguous stretch of memory.  A producer warp streams a CTA's
+// stages through a ring of shared-memory slots with 1-D bulk copies
+// (cp.async.bulk) completing on mbarriers, so ~100 KB per SM are in flight
+// regardless of register pressure.  The weight is read exactly once.
 //
 // Arithmetic side.  A team of TW consumer warps covers one weight row; lane l
 // owns the same 16-byte slice(s) of every row, so its activations live in
@@ -28,8 +30,8 @@
 // 2 DP2A, no ALU), which keeps the ALU pipe, the limiter of an fp32
 // formulation, below the memory time.  Lane partials for a stage's rows are
 // combined by a butterfly reduce-scatter into one shared-memory slot per
-// warp, summed in a fixed warp order at the end (results repeat bit for bit);
-// they leave as one coalesced store per CTA.
+// warp, summed in a fixed warp order at the end (results repeat bit for bit)
+// and written out in one pass per CTA.
 //
 // Microscaled E2M1 weights (mxfp4, nvfp4; Emily.QuantizedWeight, Microscaled
 // modes): twice an E2M1 value is an integer in [-12, 12].  Four codes become
