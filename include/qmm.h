@@ -176,8 +176,8 @@ qmm_status qmm_quantized_matmul_ws(const void *x, int64_t M, int64_t K,
  * the product of x_dev into y_dev (exactly qmm_quantized_matmul_ws), and the
  * copy of M*N elements from y_dev into y_host.  Page-locked host buffers are
  * copied by kernels that read or write their device mapping (each waits for
- * the preceding kernel of the stream, and lets the next one start early), so
- * consecutive calls overlap like device-only calls; when the product runs on
+ * the preceding kernel of the stream, then lets the next one start, so the
+ * product fills its weight ring while x is copied); when the product runs on
  * the streaming decode kernel (W [N, K], 1..4 rows), that kernel also writes
  * the result into a page-locked y_host itself and no copy follows.  Other
  * host memory goes through the copy engines.

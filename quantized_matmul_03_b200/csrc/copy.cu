@@ -24,10 +24,11 @@ constexpr int kCopyUnroll = 8;  // 16-byte loads in flight per thread
 
 __global__ void __launch_bounds__(kCopyThreads)
 mapped_copy_kernel(const uint8_t *__restrict__ src, uint8_t *__restrict__ dst, int64_t bytes, int vec16) {
-    // Let the next kernel of the stream (the product, or the next step's
-    // copy) launch now; it waits for this grid where it depends on it.
-    ptx::grid_launch_dependents();
+    // Wait for the preceding grid (the previous product), then let the next
+    // kernel of the stream launch: it is placed once the previous call's CTAs
+    // have left the SMs (one per SM), and fills its ring while this copy runs.
     ptx::grid_dependency_wait();
+    ptx::grid_launch_dependents();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (vec16) {
