@@ -141,8 +141,9 @@ qmm_status qmm_quantized_matmul(const void *x, int64_t M, int64_t K,
  * workspace only lets the tensor-core path split the k-blocks of each output
  * tile over several CTAs ("stream-K") when a problem has fewer 128-feature
  * weight tiles than the GPU has SMs and at most 64 activation rows per tile
- * (decode batches of 5..64 rows with W [N, K], 1..64 rows with W [K, N], small
- * weights), so that every SM works.
+ * (decode batches of 5..64 rows with W [N, K] -- 1..64 rows for 3- and 6-bit
+ * codes, which the streaming decode kernel does not take -- 1..64 rows with
+ * W [K, N], small weights), so that every SM works.
  *   workspace: NULL (whole tiles, exactly qmm_quantized_matmul), or device
  *     memory of at least qmm_quantized_matmul_workspace_size(...) bytes,
  *     256-byte aligned, ZEROED before its first use; every call that returns
