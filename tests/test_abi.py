@@ -133,6 +133,9 @@ def test_matmul_workspace_size(L):
     assert need > 4096                          # flags, then one partial slot per SM
     assert ws(64, 4096, 4096) == need and ws(1, 4096, 4096, tr=0) == need
     assert ws(4, 4096, 4096) == 0               # decode rows go to the SIMT decode kernel
+    assert ws(1, 4096, 4096, bits=8) == 0       # (8-bit codes too)
+    assert ws(1, 4096, 4096, bits=3) > 4096     # 3/6-bit rows: the tensor-core GEMM, split
+    assert ws(4, 4096, 14336, bits=6) > 4096
     assert ws(4, 4096, 4096, bits=2) >= 4096 + 48 * 4096   # 2-bit rows: the decode tensor-core kernel
     assert ws(128, 4096, 4096) == 0             # wide tiles keep whole tiles
     assert ws(64, 4096, 14336 * 4) == 0         # at least one full wave of tiles
