@@ -105,3 +105,41 @@ def test_affine_planes_hold_the_codes_the_kernel_pairs(bits):
         plane = (words >> (p * bits)) & mask
         for j in range(4):
             assert np.array_equal((plane >> (8 * j)) & 0xFF, codes[:, j * npl + p])
+
+
+def block_shift(amax):
+    """sh with |x 2^sh| < 2^14 for |x| <= amax (the kernel's choice)."""
+    ex = ((amax.view(np.uint32) >> 23) & 0xFF).astype(np.int64) - 126
+    return np.clip(14 - ex, -126, 126)
+
+
+@pytest.mark.parametrize("amax_factor", [1.0, 3.0, 1000.0])
+def test_magic_rounding_gives_rint_of_the_scaled_activation(amax_factor):
+    """x 2^sh + 1.5 * 2^23 in fp32 (exact product, one rounding) has
+    rint(x 2^sh) (ties to even) in its low 16 bits, and |x_int| < 2^14, for
+    every finite bf16 x and slice maxima at or above |x|."""
+    bits = np.arange(0, 1 << 16, dtype=np.uint32)
+    x = (bits << 16).view(np.float32)
+    x = x[np.isfinite(x)]
+    with np.errstate(over="ignore"):        # maxima past fp32's range are dropped
+        amax = (np.abs(x) * np.float32(amax_factor)).astype(np.float32)
+    keep = np.isfinite(amax)
+    x, amax = x[keep], amax[keep]
+    sh = block_shift(amax)
+    up = np.ldexp(np.float32(1.0), sh).astype(np.float32)
+    scaled = (x * up).astype(np.float32)               # exact: a power-of-two scale
+    t = (scaled + np.float32(12582912.0)).astype(np.float32)
+    low = (t.view(np.uint32) & 0xFFFF).astype(np.uint16).view(np.int16).astype(np.int64)
+    want = np.rint(scaled.astype(np.float64)).astype(np.int64)
+    assert np.array_equal(low, want)
+    assert np.abs(want).max() < (1 << 14)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_packed_max_of_magnitude_bits_is_the_largest_magnitude(dtype):
+    g = torch.Generator().manual_seed(5)
+    x = (torch.randn(4096, 32, generator=g) * torch.logspace(-6, 4, 32)).to(dtype)
+    raw = x.view(torch.int16).numpy().astype(np.uint16) & 0x7FFF
+    got = raw.max(axis=1).astype(np.uint16).view(np.int16)
+    want = x.abs().max(dim=1).values.view(torch.int16).numpy()
+    assert np.array_equal(got, want)
